@@ -1,0 +1,237 @@
+"""CPU oracle for the fused KV-cache rotate-and-quantize path.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package's ``smoke()`` check
+and the benchmark's CPU-baseline / reference legs may import this module.  The
+product path (the CUDA library and its binding) never imports, loads or
+calls it, and it shares no code with that path.
+
+The arithmetic lives in ``kvq_oracle.c`` (plain C99, compiled with
+``-O2 -ffp-contract=off``, no fast-math).  This module only compiles it,
+loads it with ctypes and marshals numpy arrays.  ctypes releases the GIL
+during each foreign call, so callers may run row slices in Python threads.
+
+Functions pinned by the ``-m "not gpu"`` tests: every public function here.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "kvq_oracle.c")
+LIBRARY = os.path.join(_HERE, "libkvq_oracle.so")
+
+CFLAGS = ["-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math",
+          "-fPIC", "-shared", "-Wall", "-Wextra"]
+
+_lock = threading.Lock()
+
+
+def build(source: str = SOURCE, output: str = LIBRARY) -> str:
+    """Compile the C oracle into a shared library (gcc).  Returns its path."""
+    cmd = ["gcc", *CFLAGS, source, "-o", output, "-lm"]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    return output
+
+
+def _needs_build(output: str, source: str) -> bool:
+    return (not os.path.exists(output)
+            or os.path.getmtime(output) < os.path.getmtime(source))
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+class Oracle:
+    """ctypes handle on one compiled copy of the C oracle."""
+
+    def __init__(self, library: str | None = None):
+        if library is None:
+            with _lock:
+                if _needs_build(LIBRARY, SOURCE):
+                    build()
+            library = LIBRARY
+        self.path = library
+        lib = ctypes.CDLL(library)
+        sig = {
+            "kvqo_f32_to_f16": (ctypes.c_uint16, [ctypes.c_float]),
+            "kvqo_f16_to_f32": (ctypes.c_float, [ctypes.c_uint16]),
+            "kvqo_norm_const": (ctypes.c_float, [_I]),
+            "kvqo_fwht_f64": (None, [_P, _I]),
+            "kvqo_fwht_f32": (None, [_P, _I]),
+            "kvqo_rotate_f64": (None, [_P, _P, _P, _I, _P]),
+            "kvqo_unrotate_f64": (None, [_P, _P, _P, _I, _P]),
+            "kvqo_rotate_f32": (_I, [_P, _P, _P, _I64, _I, _P]),
+            "kvqo_unrotate_f32": (_I, [_P, _P, _P, _I64, _I, _P]),
+            "kvqo_quantize_codes": (_I, [_P, _P, _P, _I64, _I, _I, _P, _P]),
+            "kvqo_quantize_codes_divform": (_I, [_P, _P, _P, _I64, _I, _I, _P]),
+            "kvqo_quantize": (_I, [_P, _P, _P, _I64, _I, _I, _P, _P]),
+            "kvqo_dequantize": (_I, [_P, _P, _P, _P, _I64, _I, _I, _P]),
+            "kvqo_dequantize_f32": (_I, [_P, _P, _P, _P, _I64, _I, _I, _P]),
+            "kvqo_pack": (None, [_P, _I64, _P]),
+            "kvqo_unpack": (None, [_P, _I64, _P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        self._lib = lib
+
+    # ---- scalar helpers -------------------------------------------------
+    def f32_to_f16_bits(self, f: float) -> int:
+        return int(self._lib.kvqo_f32_to_f16(float(f)))
+
+    def f16_bits_to_f32(self, bits: int) -> float:
+        return float(self._lib.kvqo_f16_to_f32(int(bits)))
+
+    def norm_const(self, D: int) -> float:
+        return float(self._lib.kvqo_norm_const(int(D)))
+
+    # ---- transforms -----------------------------------------------------
+    def fwht_f64(self, v: np.ndarray) -> np.ndarray:
+        out = np.ascontiguousarray(v, dtype=np.float64).copy()
+        self._lib.kvqo_fwht_f64(_ptr(out), out.shape[-1])
+        return out
+
+    def fwht_f32(self, v: np.ndarray) -> np.ndarray:
+        out = np.ascontiguousarray(v, dtype=np.float32).copy()
+        self._lib.kvqo_fwht_f32(_ptr(out), out.shape[-1])
+        return out
+
+    def rotate_f64(self, x, lam, signs) -> np.ndarray:
+        x = np.ascontiguousarray(x, dtype=np.float64)
+        lam = np.ascontiguousarray(lam, dtype=np.float64)
+        s = np.ascontiguousarray(signs, dtype=np.int8)
+        y = np.empty_like(x)
+        self._lib.kvqo_rotate_f64(_ptr(x), _ptr(lam), _ptr(s), x.shape[-1], _ptr(y))
+        return y
+
+    def unrotate_f64(self, y, lam, signs) -> np.ndarray:
+        y = np.ascontiguousarray(y, dtype=np.float64)
+        lam = np.ascontiguousarray(lam, dtype=np.float64)
+        s = np.ascontiguousarray(signs, dtype=np.int8)
+        x = np.empty_like(y)
+        self._lib.kvqo_unrotate_f64(_ptr(y), _ptr(lam), _ptr(s), y.shape[-1], _ptr(x))
+        return x
+
+    def rotate_f32(self, x_f16, lam, signs) -> np.ndarray:
+        x = _rows_f16(x_f16)
+        lam, s = _params(lam, signs)
+        y = np.empty(x.shape, dtype=np.float32)
+        _check(self._lib.kvqo_rotate_f32(_ptr(x), _ptr(lam), _ptr(s),
+                                         x.shape[0], x.shape[1], _ptr(y)))
+        return y
+
+    def unrotate_f32(self, y, lam, signs) -> np.ndarray:
+        y = np.ascontiguousarray(np.atleast_2d(y), dtype=np.float32)
+        lam, s = _params(lam, signs)
+        x = np.empty_like(y)
+        _check(self._lib.kvqo_unrotate_f32(_ptr(y), _ptr(lam), _ptr(s),
+                                           y.shape[0], y.shape[1], _ptr(x)))
+        return x
+
+    # ---- the quantiser ----------------------------------------------------
+    def quantize_codes(self, x_f16, lam, signs, group: int):
+        """Unpacked codes int8[n, D] and fp16 scales [n, D/group]."""
+        x = _rows_f16(x_f16)
+        lam, s = _params(lam, signs)
+        n, D = x.shape
+        codes = np.empty((n, D), dtype=np.int8)
+        scales = np.empty((n, D // group), dtype=np.uint16)
+        _check(self._lib.kvqo_quantize_codes(_ptr(x), _ptr(lam), _ptr(s), n, D,
+                                             group, _ptr(codes), _ptr(scales)))
+        return codes, scales.view(np.float16)
+
+    def quantize_codes_divform(self, x_f16, lam, signs, group: int):
+        x = _rows_f16(x_f16)
+        lam, s = _params(lam, signs)
+        n, D = x.shape
+        codes = np.empty((n, D), dtype=np.int8)
+        _check(self._lib.kvqo_quantize_codes_divform(_ptr(x), _ptr(lam), _ptr(s),
+                                                     n, D, group, _ptr(codes)))
+        return codes
+
+    def quantize(self, x_f16, lam, signs, group: int):
+        """Packed codes uint8[n, D/2] and fp16 scales [n, D/group]."""
+        x = _rows_f16(x_f16)
+        lam, s = _params(lam, signs)
+        n, D = x.shape
+        packed = np.empty((n, D // 2), dtype=np.uint8)
+        scales = np.empty((n, D // group), dtype=np.uint16)
+        _check(self._lib.kvqo_quantize(_ptr(x), _ptr(lam), _ptr(s), n, D, group,
+                                       _ptr(packed), _ptr(scales)))
+        return packed, scales.view(np.float16)
+
+    def dequantize(self, packed, scales, lam, signs, group: int) -> np.ndarray:
+        """fp16 [n, D] from packed codes and fp16 scales."""
+        packed = np.ascontiguousarray(np.atleast_2d(packed), dtype=np.uint8)
+        sc = np.ascontiguousarray(np.atleast_2d(scales)).view(np.uint16)
+        lam, s = _params(lam, signs)
+        n, D = packed.shape[0], packed.shape[1] * 2
+        out = np.empty((n, D), dtype=np.uint16)
+        _check(self._lib.kvqo_dequantize(_ptr(packed), _ptr(sc), _ptr(lam), _ptr(s),
+                                         n, D, group, _ptr(out)))
+        return out.view(np.float16)
+
+    def dequantize_f32(self, codes, scales, lam, signs, group: int) -> np.ndarray:
+        """fp32 [n, D] (no final fp16 rounding) from unpacked codes."""
+        codes = np.ascontiguousarray(np.atleast_2d(codes), dtype=np.int8)
+        sc = np.ascontiguousarray(np.atleast_2d(scales)).view(np.uint16)
+        lam, s = _params(lam, signs)
+        n, D = codes.shape
+        out = np.empty((n, D), dtype=np.float32)
+        _check(self._lib.kvqo_dequantize_f32(_ptr(codes), _ptr(sc), _ptr(lam), _ptr(s),
+                                             n, D, group, _ptr(out)))
+        return out
+
+    def pack(self, codes) -> np.ndarray:
+        codes = np.ascontiguousarray(codes, dtype=np.int8)
+        out = np.empty(codes.shape[:-1] + (codes.shape[-1] // 2,), dtype=np.uint8)
+        self._lib.kvqo_pack(_ptr(codes), codes.size, _ptr(out))
+        return out
+
+    def unpack(self, packed) -> np.ndarray:
+        packed = np.ascontiguousarray(packed, dtype=np.uint8)
+        out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), dtype=np.int8)
+        self._lib.kvqo_unpack(_ptr(packed), packed.size * 2, _ptr(out))
+        return out
+
+
+def _rows_f16(x) -> np.ndarray:
+    x = np.atleast_2d(np.asarray(x))
+    if x.dtype != np.float16:
+        raise TypeError("oracle input rows must be float16")
+    return np.ascontiguousarray(x).view(np.uint16)
+
+
+def _params(lam, signs):
+    lam = np.ascontiguousarray(lam, dtype=np.float32)
+    s = np.ascontiguousarray(signs, dtype=np.int8)
+    return lam, s
+
+
+def _check(rc: int) -> None:
+    if rc != 0:
+        raise ValueError(f"oracle rejected the shape (status {rc})")
+
+
+_default: Oracle | None = None
+
+
+def get() -> Oracle:
+    """The oracle compiled from this directory's source (built on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default

@@ -1,0 +1,374 @@
+/*
+ * kvq_oracle.c -- plain, slow CPU oracle for the fused KV-cache
+ * rotate-and-quantize path (lambda smooth scale -> random signs ->
+ * normalised Walsh-Hadamard transform -> per-group abs-max int4 with fp16
+ * group scales -> nibble packing) and its inverse.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
+ * calls this file.  It is used by the tests, by the package's smoke check and
+ * by the benchmark's CPU-baseline leg, and by nothing else.  It shares no
+ * code, header, table or constant with the CUDA path.
+ *
+ * Sources (the method is described on these pages; no code is printed there):
+ *   [P3]  "When Quantization Is Free: An int4 KV Cache That Outruns fp16 on
+ *         Apple Silicon" (arXiv 2605.05699), Abstract: one fused kernel does
+ *         sign-randomised transform + per-channel lambda + per-group abs-max +
+ *         int4 nibble pack; SRFT and SRHT give indistinguishable quality.
+ *   [P5]  Same title, technical summary ("Technische Samenvatting"),
+ *         Methodologie 1 (fixed random sign vector s, transform of diag(s) x),
+ *         Methodologie 2 (kernel steps: load & sign-multiply, transform,
+ *         per-channel lambda rescale, per-group absolute-max reduction, round
+ *         to signed int4, pack two int4 values per byte),
+ *         Methodologie 3 (per-channel + per-group scaling, groups of 16).
+ *   [P1]  "The Kernel That Finally Did Something -- And Didn't Quite Agree
+ *         With Itself" (VeloxQuant-MLX blog), "What VecInfer does" and "The
+ *         kernel toggle": smooth scale is applied before the Hadamard
+ *         transform, and the inverse runs dequantize -> inverse transform ->
+ *         unscale.
+ *
+ * Readings taken where the pages are silent (each is also listed in the
+ * design notes):
+ *   - lambda multiplies x BEFORE the rotation; the inverse divides by lambda
+ *     last (order of [P1]; [P5] puts lambda after the transform).
+ *   - rotation = SRHT: y = H_D diag(s) (lambda . x) / sqrt(D), H_D the
+ *     Sylvester Hadamard matrix H_ij = (-1)^popcount(i & j), s in {+1,-1}^D
+ *     ([P3] reports SRHT indistinguishable from the paper's SRFT).
+ *   - the unnormalised transform runs radix-2 butterflies with ascending
+ *     half-width h = 1, 2, ..., D/2; 1/sqrt(D) is one fp32 multiply after it.
+ *   - quantiser: symmetric, scale S = fp16_rne(max|y| / 7), codes
+ *     q = clamp(rint(y * (1/S)), -8, 7), rint = round half to even; S = 0
+ *     (all codes 0) when the fp16 scale is zero; a scale above the largest
+ *     finite fp16 saturates to 65504.
+ *   - nibble order: element 2b in the low nibble of byte b, element 2b+1 in
+ *     the high nibble, 4-bit two's complement.
+ *   - precision: the quantiser's decisions (codes, fp16 scale) are taken in
+ *     fp32 with the fixed operation order below, the precision the GPU kernel
+ *     uses; the double-precision functions exist to pin the fp32 ones.
+ *
+ * Compile with -O2 -ffp-contract=off and without -ffast-math: every line
+ * below is one IEEE operation with one rounding, in the order written.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define KVQO_DMAX 4096
+
+/* ------------------------------------------------------------------ */
+/* IEEE binary16 <-> binary32 conversion (round to nearest even).       */
+/* ------------------------------------------------------------------ */
+
+uint16_t kvqo_f32_to_f16(float f)
+{
+    _Float16 h = (_Float16)f;
+    uint16_t bits;
+    memcpy(&bits, &h, sizeof bits);
+    return bits;
+}
+
+float kvqo_f16_to_f32(uint16_t bits)
+{
+    _Float16 h;
+    memcpy(&h, &bits, sizeof h);
+    return (float)h;
+}
+
+/* The normalisation constant: the fp32 value nearest 1/sqrt(D). */
+float kvqo_norm_const(int D)
+{
+    return (float)(1.0 / sqrt((double)D));
+}
+
+static int is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+
+/* Shapes the oracle accepts: D a power of two in [2, KVQO_DMAX],
+ * G a power of two with 2 <= G <= D.  Returns 0 if valid. */
+static int check_shape(int D, int G)
+{
+    if (!is_pow2(D) || D < 2 || D > KVQO_DMAX) return -3;
+    if (!is_pow2(G) || G < 2 || G > D) return -4;
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Unnormalised fast Walsh-Hadamard transform, Sylvester (natural)     */
+/* order, radix-2 butterflies with ascending half-width h.             */
+/* [P3] Abstract (SRHT); [P5] Methodologie 1.                          */
+/* ------------------------------------------------------------------ */
+
+void kvqo_fwht_f64(double *v, int D)
+{
+    for (int h = 1; h < D; h <<= 1)
+        for (int i = 0; i < D; i += 2 * h)
+            for (int k = i; k < i + h; ++k) {
+                double a = v[k];
+                double b = v[k + h];
+                v[k] = a + b;
+                v[k + h] = a - b;
+            }
+}
+
+void kvqo_fwht_f32(float *v, int D)
+{
+    for (int h = 1; h < D; h <<= 1)
+        for (int i = 0; i < D; i += 2 * h)
+            for (int k = i; k < i + h; ++k) {
+                float a = v[k];
+                float b = v[k + h];
+                v[k] = a + b;
+                v[k + h] = a - b;
+            }
+}
+
+/* ------------------------------------------------------------------ */
+/* Double-precision rotation and its inverse, the definitions that pin */
+/* the fp32 path:  y = H diag(s) (lambda . x) / sqrt(D)                 */
+/*                 x = (diag(s) H y / sqrt(D)) / lambda                */
+/* ------------------------------------------------------------------ */
+
+void kvqo_rotate_f64(const double *x, const double *lam, const int8_t *s,
+                     int D, double *y)
+{
+    double inv = 1.0 / sqrt((double)D);
+    for (int i = 0; i < D; ++i) y[i] = x[i] * lam[i] * (double)s[i];
+    kvqo_fwht_f64(y, D);
+    for (int i = 0; i < D; ++i) y[i] *= inv;
+}
+
+void kvqo_unrotate_f64(const double *y, const double *lam, const int8_t *s,
+                       int D, double *x)
+{
+    double inv = 1.0 / sqrt((double)D);
+    for (int i = 0; i < D; ++i) x[i] = y[i];
+    kvqo_fwht_f64(x, D);
+    for (int i = 0; i < D; ++i) x[i] = x[i] * inv * (double)s[i] / lam[i];
+}
+
+/* ------------------------------------------------------------------ */
+/* fp32 forward rotation of one fp16 row (steps: load, lambda & sign,  */
+/* transform, normalise).  [P5] Methodologie 2, first two steps;       */
+/* lambda before the transform per [P1].                                */
+/* ------------------------------------------------------------------ */
+
+static void rotate_row_f32(const uint16_t *x, const float *lam,
+                           const int8_t *s, int D, float c, float *y)
+{
+    for (int i = 0; i < D; ++i) {
+        float t = kvqo_f16_to_f32(x[i]) * lam[i];   /* one rounding  */
+        y[i] = (s[i] < 0) ? -t : t;                 /* exact         */
+    }
+    kvqo_fwht_f32(y, D);
+    for (int i = 0; i < D; ++i) y[i] = y[i] * c;
+}
+
+int kvqo_rotate_f32(const uint16_t *x, const float *lam, const int8_t *s,
+                    int64_t n, int D, float *y)
+{
+    if (!is_pow2(D) || D < 2 || D > KVQO_DMAX || n < 0) return -3;
+    float c = kvqo_norm_const(D);
+    for (int64_t r = 0; r < n; ++r)
+        rotate_row_f32(x + r * D, lam, s, D, c, y + r * D);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Per-group abs-max int4 quantisation of one rotated row.              */
+/* [P5] Methodologie 2 ("per-group absolute-max reduction, round to    */
+/* signed int4"), Methodologie 3 (per-group scaling).                  */
+/* ------------------------------------------------------------------ */
+
+static void quantize_rotated_row(const float *y, int D, int G,
+                                 int8_t *q, uint16_t *scales)
+{
+    for (int j = 0; j < D / G; ++j) {
+        const float *yg = y + j * G;
+        float a = 0.0f;
+        for (int i = 0; i < G; ++i) {
+            float m = fabsf(yg[i]);
+            if (m > a) a = m;
+        }
+        uint16_t sb = kvqo_f32_to_f16(a / 7.0f);
+        if (sb == 0x7C00u) sb = 0x7BFFu;            /* saturate to 65504 */
+        scales[j] = sb;
+        float sf = kvqo_f16_to_f32(sb);
+        if (sf == 0.0f) {
+            for (int i = 0; i < G; ++i) q[j * G + i] = 0;
+            continue;
+        }
+        float r = 1.0f / sf;
+        for (int i = 0; i < G; ++i) {
+            float t = rintf(yg[i] * r);              /* half to even  */
+            if (t > 7.0f) t = 7.0f;
+            if (t < -8.0f) t = -8.0f;
+            q[j * G + i] = (int8_t)t;
+        }
+    }
+}
+
+/* Codes unpacked, one int8 per element: codes[n][D], scales[n][D/G]
+ * (fp16 bit patterns). */
+int kvqo_quantize_codes(const uint16_t *x, const float *lam, const int8_t *s,
+                        int64_t n, int D, int G, int8_t *codes,
+                        uint16_t *scales)
+{
+    int rc = check_shape(D, G);
+    if (rc) return rc;
+    if (n < 0) return -5;
+    float c = kvqo_norm_const(D);
+    float y[KVQO_DMAX];
+    for (int64_t r = 0; r < n; ++r) {
+        rotate_row_f32(x + r * D, lam, s, D, c, y);
+        quantize_rotated_row(y, D, G, codes + r * D, scales + r * (D / G));
+    }
+    return 0;
+}
+
+/* Two int4 codes per byte: element 2b in the low nibble, 2b+1 in the high
+ * nibble ([P5] Methodologie 2, last step). */
+void kvqo_pack(const int8_t *codes, int64_t count, uint8_t *packed)
+{
+    for (int64_t b = 0; b < count / 2; ++b) {
+        unsigned lo = (unsigned)codes[2 * b] & 0xFu;
+        unsigned hi = (unsigned)codes[2 * b + 1] & 0xFu;
+        packed[b] = (uint8_t)(lo | (hi << 4));
+    }
+}
+
+void kvqo_unpack(const uint8_t *packed, int64_t count, int8_t *codes)
+{
+    for (int64_t b = 0; b < count / 2; ++b) {
+        int lo = packed[b] & 0xF;
+        int hi = (packed[b] >> 4) & 0xF;
+        codes[2 * b] = (int8_t)(lo >= 8 ? lo - 16 : lo);
+        codes[2 * b + 1] = (int8_t)(hi >= 8 ? hi - 16 : hi);
+    }
+}
+
+/* The whole forward path: packed[n][D/2] bytes, scales[n][D/G] fp16 bits. */
+int kvqo_quantize(const uint16_t *x, const float *lam, const int8_t *s,
+                  int64_t n, int D, int G, uint8_t *packed, uint16_t *scales)
+{
+    int rc = check_shape(D, G);
+    if (rc) return rc;
+    if (n < 0) return -5;
+    float c = kvqo_norm_const(D);
+    float y[KVQO_DMAX];
+    int8_t q[KVQO_DMAX];
+    for (int64_t r = 0; r < n; ++r) {
+        rotate_row_f32(x + r * D, lam, s, D, c, y);
+        quantize_rotated_row(y, D, G, q, scales + r * (D / G));
+        kvqo_pack(q, D, packed + r * (D / 2));
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Inverse path: unpack -> times scale -> inverse rotation -> / lambda. */
+/* H/sqrt(D) is symmetric and orthogonal, so it is its own inverse, and */
+/* diag(s) is its own inverse.  Order per [P1] ("dequantize, inverse    */
+/* transform, unscale").  Division by lambda is a multiply by the fp32  */
+/* reciprocal 1/lambda.                                                 */
+/* ------------------------------------------------------------------ */
+
+static void dequantize_row(const int8_t *q, const uint16_t *scales,
+                           const float *lam, const int8_t *s, int D, int G,
+                           float c, float *w)
+{
+    for (int i = 0; i < D; ++i)
+        w[i] = (float)q[i] * kvqo_f16_to_f32(scales[i / G]);   /* exact */
+    kvqo_fwht_f32(w, D);
+    for (int i = 0; i < D; ++i) {
+        float z = w[i] * c;
+        float zs = (s[i] < 0) ? -z : z;                         /* exact */
+        float il = 1.0f / lam[i];
+        w[i] = zs * il;
+    }
+}
+
+int kvqo_dequantize(const uint8_t *packed, const uint16_t *scales,
+                    const float *lam, const int8_t *s, int64_t n, int D,
+                    int G, uint16_t *out)
+{
+    int rc = check_shape(D, G);
+    if (rc) return rc;
+    if (n < 0) return -5;
+    float c = kvqo_norm_const(D);
+    int8_t q[KVQO_DMAX];
+    float w[KVQO_DMAX];
+    for (int64_t r = 0; r < n; ++r) {
+        kvqo_unpack(packed + r * (D / 2), D, q);
+        dequantize_row(q, scales + r * (D / G), lam, s, D, G, c, w);
+        for (int i = 0; i < D; ++i) out[r * D + i] = kvqo_f32_to_f16(w[i]);
+    }
+    return 0;
+}
+
+/* The inverse without the final fp16 rounding (fp32 output), from codes. */
+int kvqo_dequantize_f32(const int8_t *codes, const uint16_t *scales,
+                        const float *lam, const int8_t *s, int64_t n, int D,
+                        int G, float *out)
+{
+    int rc = check_shape(D, G);
+    if (rc) return rc;
+    if (n < 0) return -5;
+    float c = kvqo_norm_const(D);
+    for (int64_t r = 0; r < n; ++r)
+        dequantize_row(codes + r * D, scales + r * (D / G), lam, s, D, G, c,
+                       out + r * D);
+    return 0;
+}
+
+/* fp32 inverse rotation of rotated rows (no quantisation): y -> x. */
+int kvqo_unrotate_f32(const float *y, const float *lam, const int8_t *s,
+                      int64_t n, int D, float *x)
+{
+    if (!is_pow2(D) || D < 2 || D > KVQO_DMAX || n < 0) return -3;
+    float c = kvqo_norm_const(D);
+    for (int64_t r = 0; r < n; ++r) {
+        float *w = x + r * D;
+        for (int i = 0; i < D; ++i) w[i] = y[r * D + i];
+        kvqo_fwht_f32(w, D);
+        for (int i = 0; i < D; ++i) {
+            float z = w[i] * c;
+            float zs = (s[i] < 0) ? -z : z;
+            w[i] = zs * (1.0f / lam[i]);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Textbook cross-check form of the quantiser: codes = rint(y / S) with */
+/* an IEEE division per element instead of a multiply by 1/S.  Used    */
+/* only to show that the two forms disagree at near-ties alone.        */
+/* ------------------------------------------------------------------ */
+
+int kvqo_quantize_codes_divform(const uint16_t *x, const float *lam,
+                                const int8_t *s, int64_t n, int D, int G,
+                                int8_t *codes)
+{
+    int rc = check_shape(D, G);
+    if (rc) return rc;
+    float c = kvqo_norm_const(D);
+    float y[KVQO_DMAX];
+    for (int64_t r = 0; r < n; ++r) {
+        rotate_row_f32(x + r * D, lam, s, D, c, y);
+        for (int j = 0; j < D / G; ++j) {
+            float a = 0.0f;
+            for (int i = 0; i < G; ++i) {
+                float m = fabsf(y[j * G + i]);
+                if (m > a) a = m;
+            }
+            uint16_t sb = kvqo_f32_to_f16(a / 7.0f);
+            if (sb == 0x7C00u) sb = 0x7BFFu;
+            float sf = kvqo_f16_to_f32(sb);
+            for (int i = 0; i < G; ++i) {
+                float t = (sf == 0.0f) ? 0.0f : rintf(y[j * G + i] / sf);
+                if (t > 7.0f) t = 7.0f;
+                if (t < -8.0f) t = -8.0f;
+                codes[r * D + j * G + i] = (int8_t)t;
+            }
+        }
+    }
+    return 0;
+}

@@ -1,0 +1,371 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each pin takes an ``oracle.Oracle`` and raises AssertionError on failure.  They
+check the oracle against what the pages and the mathematics fix:
+
+* brute force: the transform against the dense Sylvester matrix built two
+  independent ways (Kronecker powers and the popcount formula);
+* the rotation's orthogonality (norm preservation, exact inverse);
+* closed forms: zero rows, an impulse (every code +-7 with the Hadamard sign
+  pattern), constant rows, a saturating row;
+* the quantiser's error bound |y - q S| <= S/2 and the codes' range;
+* library routines: fp16 conversion against numpy's IEEE cast;
+* hand-worked examples (tests/golden/worked_examples.json) and the pages'
+  printed compression figure (tests/golden/accounting.json).
+
+``tests/test_oracle.py`` runs every pin on the oracle; ``tests/
+test_oracle_mutants.py`` plants plausible mistakes in copies of the oracle's
+C source and checks that at least one pin fails for each.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+from kv_cache_quantization_02_b200 import workloads
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+U32 = 2.0 ** -24          # unit roundoff of fp32
+
+
+def sylvester_kron(D: int) -> np.ndarray:
+    H = np.array([[1.0]])
+    while H.shape[0] < D:
+        H = np.kron(H, np.array([[1.0, 1.0], [1.0, -1.0]]))
+    return H
+
+
+def sylvester_popcount(D: int) -> np.ndarray:
+    i = np.arange(D)[:, None]
+    j = np.arange(D)[None, :]
+    bits = np.vectorize(lambda v: bin(int(v)).count("1"))(i & j)
+    return np.where(bits % 2 == 0, 1.0, -1.0)
+
+
+def _rand_params(rng, D):
+    lam = rng.uniform(0.5, 2.0, D).astype(np.float32)
+    s = np.where(rng.random(D) < 0.5, -1, 1).astype(np.int8)
+    return lam, s
+
+
+def _rows(rng, n, D, outliers=4, gain=20.0):
+    x = rng.standard_normal((n, D))
+    if outliers:
+        x[:, rng.permutation(D)[:outliers]] *= gain
+    return x.astype(np.float16)
+
+
+# --------------------------------------------------------------------------
+def pin_f16_conversion(o):
+    """fp32 -> fp16 (RNE) and fp16 -> fp32 against numpy's IEEE casts."""
+    all_bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ref = all_bits.view(np.float16).astype(np.float32)
+    finite = np.isfinite(ref)
+    got = np.array([o.f16_bits_to_f32(int(b)) for b in all_bits[finite]],
+                   dtype=np.float32)
+    assert np.array_equal(got, ref[finite]), "fp16 -> fp32 differs from numpy"
+    # midpoints between neighbouring fp16 values are ties: RNE picks the even one
+    pos = ref[finite & (ref >= 0)]
+    pos = np.unique(pos)
+    mids = ((pos[:-1].astype(np.float64) + pos[1:].astype(np.float64)) / 2)
+    mids = mids[np.abs(mids) < 65504].astype(np.float32)
+    rng = np.random.default_rng(7)
+    vals = np.concatenate([
+        mids[::37], -mids[::41], rng.standard_normal(2000).astype(np.float32) * 100,
+        np.array([0.0, -0.0, 65504.0, 65519.0, 65520.0, 1e6, -1e6, 2.0 ** -24,
+                  2.0 ** -25, 2.0 ** -25 * 1.0000001, 3 * 2.0 ** -26, 2.0 ** -14,
+                  6.1e-5, 1.0 / 7.0], dtype=np.float32)])
+    for v in vals:
+        with np.errstate(over="ignore"):
+            want = int(np.float32(v).astype(np.float16).view(np.uint16))
+        got = o.f32_to_f16_bits(float(v))
+        assert got == want, f"fp32 {v!r} -> fp16 bits {got:#06x}, numpy {want:#06x}"
+
+
+def pin_norm_const(o):
+    """c is the fp32 value nearest 1/sqrt(D) (exact rational check)."""
+    assert o.norm_const(64) == 0.125 and o.norm_const(256) == 0.0625
+    assert np.float32(o.norm_const(128)).view(np.uint32) == 0x3DB504F3
+    for k in range(1, 13):
+        D = 1 << k
+        c = Fraction(o.norm_const(D))
+        ulp = Fraction(float(np.spacing(np.float32(float(c)))))
+        lo, hi = c - ulp / 2, c + ulp / 2
+        assert lo * lo * D < 1 < hi * hi * D, f"c for D={D} is not the nearest fp32"
+
+
+def pin_fwht_dense(o):
+    """Unnormalised transform == dense Sylvester matrix (two constructions)."""
+    rng = np.random.default_rng(1)
+    for k in range(1, 9):
+        D = 1 << k
+        H = sylvester_kron(D)
+        assert np.array_equal(H, sylvester_popcount(D))
+        v = rng.standard_normal((3, D))
+        for row in v:
+            got = o.fwht_f64(row)
+            np.testing.assert_allclose(got, H @ row, rtol=0, atol=1e-12 * D)
+        iv = rng.integers(-50, 50, size=D).astype(np.float64)
+        assert np.array_equal(o.fwht_f64(iv), H @ iv)
+        assert np.array_equal(o.fwht_f32(iv.astype(np.float32)),
+                              (H @ iv).astype(np.float32))
+
+
+def pin_rotation_dense(o):
+    """rotate_f64 == H diag(s) (lambda . x) / sqrt(D); unrotate is its inverse."""
+    rng = np.random.default_rng(2)
+    for D in (2, 4, 8, 16, 32, 64, 128, 256):
+        H = sylvester_kron(D)
+        lam, s = _rand_params(rng, D)
+        M = H @ np.diag(s.astype(np.float64)) / math.sqrt(D)
+        np.testing.assert_allclose(M.T @ M, np.eye(D), atol=1e-12)
+        x = rng.standard_normal(D) * 3
+        y = o.rotate_f64(x, lam, s)
+        np.testing.assert_allclose(y, M @ (lam.astype(np.float64) * x), atol=1e-12)
+        xb = o.unrotate_f64(y, lam, s)
+        np.testing.assert_allclose(xb, (M.T @ y) / lam.astype(np.float64), atol=1e-12)
+        np.testing.assert_allclose(xb, x, atol=1e-12)
+
+
+def _fwht_err_bound(x64, lam, D):
+    """Forward-error bound of the fp32 path against exact arithmetic: one
+    rounding at x*lambda, log2(D) roundings per butterfly path, one at *c,
+    and the error of c itself."""
+    terms = np.abs(x64 * lam.astype(np.float64))
+    l1 = terms.sum(axis=-1, keepdims=True)
+    return (math.log2(D) + 3) * U32 * l1 / math.sqrt(D) * 1.01
+
+
+def pin_rotate_f32(o):
+    """fp32 forward rotation within its rounding bound of the f64 definition."""
+    rng = np.random.default_rng(3)
+    for D in (4, 16, 64, 128, 256):
+        lam, s = _rand_params(rng, D)
+        x = _rows(rng, 16, D)
+        y32 = o.rotate_f32(x, lam, s).astype(np.float64)
+        x64 = x.astype(np.float64)
+        y64 = np.stack([o.rotate_f64(r, lam, s) for r in x64])
+        bound = _fwht_err_bound(x64, lam, D)
+        assert np.all(np.abs(y32 - y64) <= bound), f"fp32 rotation off at D={D}"
+
+
+def pin_norm_preservation(o):
+    rng = np.random.default_rng(4)
+    for D in (8, 64, 128, 256):
+        lam, s = _rand_params(rng, D)
+        x = _rows(rng, 8, D)
+        x64 = x.astype(np.float64)
+        ref = np.linalg.norm(x64 * lam.astype(np.float64), axis=1)
+        y64 = np.stack([o.rotate_f64(r, lam, s) for r in x64])
+        np.testing.assert_allclose(np.linalg.norm(y64, axis=1), ref, rtol=1e-12)
+        y32 = o.rotate_f32(x, lam, s).astype(np.float64)
+        np.testing.assert_allclose(np.linalg.norm(y32, axis=1), ref, rtol=1e-6)
+
+
+def pin_roundtrip_unquantized(o):
+    """rotate -> inverse recovers x (f64: to 1e-5 absolute and far below;
+    fp32: to 1e-5 of the row's largest magnitude)."""
+    rng = np.random.default_rng(5)
+    for D in (16, 64, 128, 256):
+        lam, s = _rand_params(rng, D)
+        x = _rows(rng, 8, D)
+        x64 = x.astype(np.float64)
+        back = np.stack([o.unrotate_f64(o.rotate_f64(r, lam, s), lam, s) for r in x64])
+        assert np.max(np.abs(back - x64)) <= 1e-5
+        np.testing.assert_allclose(back, x64, atol=1e-12 * np.abs(x64).max())
+        b32 = o.unrotate_f32(o.rotate_f32(x, lam, s), lam, s).astype(np.float64)
+        scale = np.abs(x64).max(axis=1, keepdims=True)
+        assert np.all(np.abs(b32 - x64) <= 1e-5 * scale)
+
+
+def _scales_f32(scales):
+    return np.asarray(scales).astype(np.float32)
+
+
+def pin_code_invariants(o):
+    """Codes lie in [-8, 7]; every group with a normal scale has max|q| = 7;
+    the scale is the fp16 rounding of max|y|/7."""
+    rng = np.random.default_rng(6)
+    cases = []
+    for D, G in ((64, 16), (64, 64), (128, 32), (128, 16), (256, 32), (256, 64), (256, 256)):
+        lam, s = _rand_params(rng, D)
+        cases.append((_rows(rng, 24, D), lam, s, G))
+    w = workloads.WORKLOADS["qwen2.5-1.5b"]
+    lam, s = workloads.params(w.D, w.seed)
+    cases.append((workloads.host_rows(w, 64), lam, s, 32))
+    for x, lam, s, G in cases:
+        D = x.shape[1]
+        q, S = o.quantize_codes(x, lam, s, G)
+        assert q.min() >= -8 and q.max() <= 7
+        Sf = _scales_f32(S)
+        y = o.rotate_f32(x, lam, s)
+        a = np.abs(y).reshape(len(x), D // G, G).max(axis=2)
+        want = (a / np.float32(7.0)).astype(np.float32).astype(np.float16).astype(np.float32)
+        assert np.array_equal(Sf, want), "scale is not fp16(max|y|/7)"
+        qm = np.abs(q.astype(np.int32)).reshape(len(x), D // G, G).max(axis=2)
+        normal = Sf >= 2.0 ** -14
+        assert np.all(qm[normal] == 7), "a group with a normal scale lacks |q| = 7"
+        assert not np.any(q.reshape(len(x), D // G, G)[normal] == -8)
+
+
+def pin_error_bound(o):
+    """|y_i - q_i S_j| <= S_j / 2 for every element of a normal-scale group,
+    and the reconstruction error obeys the same bound after the inverse:
+    ||lambda.(x - x_hat)||_2 <= sqrt(sum_j G S_j^2) / 2 (+ fp32 slack)."""
+    rng = np.random.default_rng(8)
+    for D, G in ((64, 32), (128, 32), (128, 16), (256, 64)):
+        lam, s = _rand_params(rng, D)
+        x = _rows(rng, 32, D)
+        q, S = o.quantize_codes(x, lam, s, G)
+        Sf = _scales_f32(S).astype(np.float64)
+        y = o.rotate_f32(x, lam, s).astype(np.float64)
+        Se = np.repeat(Sf, G, axis=1)
+        err = np.abs(y - q * Se)
+        ok = Se >= 2.0 ** -14
+        assert np.all(err[ok] <= Se[ok] / 2 * (1 + 1e-6)), "quantiser error above S/2"
+        xh = o.dequantize_f32(q, S, lam, s, G).astype(np.float64)
+        lhs = np.linalg.norm(lam.astype(np.float64) * (x.astype(np.float64) - xh), axis=1)
+        rhs = 0.5 * np.sqrt(G * (Sf ** 2).sum(axis=1))
+        slack = (math.log2(D) + 4) * U32 * np.abs(y).sum(axis=1) * 2
+        assert np.all(lhs <= rhs + slack), "round trip exceeds the quantiser bound"
+
+
+def pin_dequant_vs_f64(o):
+    """fp32 inverse path within rounding of the f64 inverse rotation of q*S,
+    and the fp16 output is the RNE cast of the fp32 output."""
+    rng = np.random.default_rng(9)
+    for D, G in ((16, 16), (64, 16), (128, 32), (256, 64)):
+        lam, s = _rand_params(rng, D)
+        q = rng.integers(-8, 8, size=(12, D)).astype(np.int8)
+        S = (rng.uniform(0.01, 3.0, size=(12, D // G))).astype(np.float16)
+        got = o.dequantize_f32(q, S, lam, s, G).astype(np.float64)
+        u = q * np.repeat(S.astype(np.float64), G, axis=1)
+        ref = np.stack([o.unrotate_f64(r, lam, s) for r in u])
+        bound = (math.log2(D) + 4) * U32 * np.abs(u).sum(axis=1, keepdims=True) \
+            / math.sqrt(D) / lam.astype(np.float64).min() * 1.01
+        assert np.all(np.abs(got - ref) <= bound), f"inverse path off at D={D}"
+        # and against the dense matrix directly
+        H = sylvester_kron(D)
+        dense = (u @ H.T) / math.sqrt(D) * s.astype(np.float64) / lam.astype(np.float64)
+        assert np.all(np.abs(got - dense) <= bound)
+        packed = o.pack(q)
+        out16 = o.dequantize(packed, S, lam, s, G)
+        assert np.array_equal(out16.view(np.uint16),
+                              got.astype(np.float32).astype(np.float16).view(np.uint16))
+
+
+def pin_special_cases(o):
+    rng = np.random.default_rng(10)
+    for D, G in ((64, 16), (128, 32), (256, 64)):
+        lam, s = _rand_params(rng, D)
+        # zero rows
+        z = np.zeros((2, D), dtype=np.float16)
+        q, S = o.quantize_codes(z, lam, s, G)
+        assert not q.any() and not S.astype(np.float32).any()
+        assert not o.dequantize(o.pack(q), S, lam, s, G).astype(np.float32).any()
+        # impulse alpha e_k with lambda = 1: |y_i| = |alpha|/sqrt(D) for all i,
+        # every code +-7 with sign = sign(alpha) s_k H[k, i]
+        ones = np.ones(D, dtype=np.float32)
+        H = sylvester_popcount(D)
+        for k, alpha in ((0, 3.0), (D // 3, -1.5), (D - 1, 250.0)):
+            x = np.zeros((1, D), dtype=np.float16)
+            x[0, k] = alpha
+            q, S = o.quantize_codes(x, ones, s, G)
+            want = (7 * np.sign(alpha) * s[k] * H[k]).astype(np.int8)
+            assert np.array_equal(q[0], want), "impulse codes wrong"
+            y = np.float32(alpha) * np.float32(o.norm_const(D))
+            sw = (np.abs(y) / np.float32(7)).astype(np.float16)
+            assert np.all(S[0] == sw)
+        # constant row, lambda = 1, signs = +1: all energy in coefficient 0
+        pos = np.ones(D, dtype=np.int8)
+        x = np.full((1, D), 0.75, dtype=np.float16)
+        q, S = o.quantize_codes(x, ones, pos, G)
+        assert q[0, 0] == 7 and not q[0, 1:].any()
+        assert np.all(S[0, 1:].astype(np.float32) == 0) and S[0, 0] > 0
+        out = o.dequantize(o.pack(q), S, ones, pos, G).astype(np.float32)
+        assert np.all(out == out[0, 0]) and abs(out[0, 0] - 0.75) < 0.75 / 7
+    # saturating scale: D=256 rows of 65504 with lambda = 2
+    D, G = 256, 64
+    x = np.full((1, D), 65504.0, dtype=np.float16)
+    q, S = o.quantize_codes(x, np.full(D, 2.0, np.float32), np.ones(D, np.int8), G)
+    assert S.view(np.uint16)[0, 0] == 0x7BFF and q[0, 0] == 7
+
+
+def pin_worked_examples(o):
+    with open(os.path.join(GOLDEN, "worked_examples.json")) as f:
+        ex = json.load(f)
+    for e in ex["examples"]:
+        x = np.array([e["x"]], dtype=np.float16)
+        assert np.array_equal(x.astype(np.float64)[0], np.array(e["x"])), "fixture x not fp16"
+        lam = np.array(e["lambda"], dtype=np.float32)
+        s = np.array(e["signs"], dtype=np.int8)
+        G = e["G"]
+        y = o.rotate_f32(x, lam, s)
+        assert np.array_equal(y[0].astype(np.float64), np.array(e["y"])), e["name"]
+        q, S = o.quantize_codes(x, lam, s, G)
+        assert q[0].tolist() == e["codes"], e["name"]
+        assert S.view(np.uint16)[0].tolist() == e["scale_bits"], e["name"]
+        packed, S2 = o.quantize(x, lam, s, G)
+        assert packed[0].tolist() == e["packed"], e["name"]
+        out = o.dequantize(packed, S2, lam, s, G)
+        assert out[0].astype(np.float64).tolist() == e["dequant"], e["name"]
+
+
+def pin_divform_near_ties(o):
+    """Multiplying by 1/S and dividing by S pick different codes only within
+    a few ulp of a rounding tie, and then differ by one."""
+    rng = np.random.default_rng(11)
+    D, G = 128, 32
+    lam, s = _rand_params(rng, D)
+    x = _rows(rng, 512, D)
+    q, S = o.quantize_codes(x, lam, s, G)
+    qd = o.quantize_codes_divform(x, lam, s, G)
+    diff = q != qd
+    if diff.any():
+        assert np.abs(q.astype(int) - qd.astype(int)).max() == 1
+        y = o.rotate_f32(x, lam, s).astype(np.float64)
+        t = y / np.repeat(S.astype(np.float64), G, axis=1)
+        frac = np.abs(np.abs(t - np.floor(t)) - 0.5)
+        assert np.all(frac[diff] < 1e-5)
+    assert diff.mean() <= 1e-3
+
+
+def pin_pack_layout(o):
+    """Low nibble = even element, two's complement; pack/unpack are inverse."""
+    assert o.pack(np.array([1, 2], dtype=np.int8)).tolist() == [0x21]
+    assert o.pack(np.array([-1, -8], dtype=np.int8)).tolist() == [0x8F]
+    assert o.pack(np.array([7, -7], dtype=np.int8)).tolist() == [0x97]
+    allc = np.array([(a, b) for a in range(-8, 8) for b in range(-8, 8)],
+                    dtype=np.int8).reshape(-1)
+    assert np.array_equal(o.unpack(o.pack(allc)), allc)
+
+
+def pin_accounting(o):
+    """Storage per vector and the pages' printed compression ratio."""
+    with open(os.path.join(GOLDEN, "accounting.json")) as f:
+        acc = json.load(f)
+    G = acc["compression_upper_group"]
+    ratio = 16.0 / (4.0 + 16.0 / G)
+    assert round(ratio, 2) == acc["compression_upper_printed"]
+    assert 16.0 / (4.0 + 16.0 / acc["group_size_in_methodology"]) >= acc["compression_lower_printed"]
+    rng = np.random.default_rng(12)
+    for D, G in ((64, 16), (128, 32), (256, 64)):
+        lam, s = _rand_params(rng, D)
+        packed, S = o.quantize(_rows(rng, 3, D), lam, s, G)
+        fp16_bytes = 2 * D
+        stored = packed.shape[1] + 2 * S.shape[1]
+        assert stored == D // 2 + 2 * D // G
+        assert abs(fp16_bytes / stored - 16.0 / (4.0 + 16.0 / G)) < 1e-12
+
+
+ALL_PINS = [
+    pin_f16_conversion, pin_norm_const, pin_fwht_dense, pin_rotation_dense,
+    pin_rotate_f32, pin_norm_preservation, pin_roundtrip_unquantized,
+    pin_code_invariants, pin_error_bound, pin_dequant_vs_f64,
+    pin_special_cases, pin_worked_examples, pin_divform_near_ties,
+    pin_pack_layout, pin_accounting,
+]

@@ -1,0 +1,74 @@
+"""Plant plausible mistakes in copies of the oracle's C source (on the CPU)
+and check that the pins catch every one.  This is what makes the pins
+trustworthy: a dropped term, a wrong sign, a wrong constant, a swapped index
+or a wrong rounding mode anywhere in the oracle fails at least one of them."""
+import os
+import tempfile
+
+import pytest
+
+import oracle
+import oracle_pins
+
+# (name, text to replace, replacement, which occurrence (0-based))
+MUTANTS = [
+    ("fwht_f64_sign", "v[k + h] = a - b;", "v[k + h] = b - a;", 0),
+    ("fwht_f32_sign", "v[k + h] = a - b;", "v[k + h] = b - a;", 1),
+    ("fwht_f32_drop_term", "v[k] = a + b;", "v[k] = a;", 1),
+    ("fwht_f32_index", "float b = v[k + h];", "float b = v[k + h - (h > 1)];", 0),
+    ("fwht_stage_skipped", "for (int h = 1; h < D; h <<= 1)", "for (int h = 2; h < D; h <<= 1)", 1),
+    ("lambda_divides", "* lam[i];   /* one rounding  */", "/ lam[i];   /* one rounding  */", 0),
+    ("lambda_dropped", "* lam[i];   /* one rounding  */", ";   /* one rounding  */", 0),
+    ("sign_dropped", "y[i] = (s[i] < 0) ? -t : t;", "y[i] = t;", 0),
+    ("norm_const", "(float)(1.0 / sqrt((double)D))", "(float)(1.0 / (double)D)", 0),
+    ("normalise_skipped", "for (int i = 0; i < D; ++i) y[i] = y[i] * c;", "(void)c;", 0),
+    ("scale_div8", "kvqo_f32_to_f16(a / 7.0f);", "kvqo_f32_to_f16(a / 8.0f);", 0),
+    ("absmax_min", "if (m > a) a = m;", "if (m < a) a = m;", 0),
+    ("no_saturation", "if (sb == 0x7C00u) sb = 0x7BFFu;            /* saturate to 65504 */", "", 0),
+    ("round_half_away", "rintf(yg[i] * r)", "roundf(yg[i] * r)", 0),
+    ("truncate", "rintf(yg[i] * r)", "truncf(yg[i] * r)", 0),
+    ("clamp_low_7", "if (t < -8.0f) t = -8.0f;", "if (t < -7.0f) t = -7.0f;", 0),
+    ("nibble_order", "packed[b] = (uint8_t)(lo | (hi << 4));", "packed[b] = (uint8_t)(hi | (lo << 4));", 0),
+    ("unpack_no_sign_ext", "codes[2 * b] = (int8_t)(lo >= 8 ? lo - 16 : lo);", "codes[2 * b] = (int8_t)lo;", 0),
+    ("deq_scale_index", "kvqo_f16_to_f32(scales[i / G]);", "kvqo_f16_to_f32(scales[0]);", 0),
+    ("deq_no_norm", "float z = w[i] * c;", "float z = w[i];", 0),
+    ("deq_no_sign", "float zs = (s[i] < 0) ? -z : z;                         /* exact */", "float zs = z;", 0),
+    ("deq_lambda_mult", "float il = 1.0f / lam[i];", "float il = lam[i];", 0),
+    ("unrotate_f64_lambda", "(double)s[i] / lam[i];", "(double)s[i] * lam[i];", 0),
+    ("f16_round_trunc", "_Float16 h = (_Float16)f;", "_Float16 h = (_Float16)(f - f * 0x1p-12f);", 0),
+]
+
+
+def _mutate(src: str, old: str, new: str, occ: int) -> str:
+    idx = -1
+    for _ in range(occ + 1):
+        idx = src.index(old, idx + 1)
+    return src[:idx] + new + src[idx + len(old):]
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(oracle.SOURCE) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name,old,new,occ", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(source, name, old, new, occ):
+    mutated = _mutate(source, old, new, occ)
+    assert mutated != source
+    with tempfile.TemporaryDirectory() as td:
+        src = os.path.join(td, "mutant.c")
+        lib = os.path.join(td, "libmutant.so")
+        with open(src, "w") as f:
+            f.write(mutated)
+        oracle.build(src, lib)
+        o = oracle.Oracle(lib)
+        failed = []
+        for pin in oracle_pins.ALL_PINS:
+            try:
+                pin(o)
+            except AssertionError:
+                failed.append(pin.__name__)
+            except (ValueError, FloatingPointError):
+                failed.append(pin.__name__)
+        assert failed, f"no pin caught mutant {name}"
