@@ -1,0 +1,474 @@
+#!/usr/bin/env python
+"""Benchmark of the fused KV-cache rotate-and-quantize path on B200.
+
+One step = one pass of the whole path over one batch: kvq_quantize of the
+batch (fp16 -> int4 codes + fp16 group scales) followed by kvq_dequantize of
+the result (-> fp16).  The default batch is a Qwen3-8B-shaped prefill cache:
+36 layers x 8 KV heads x 32768 tokens x (K, V) = 18,874,368 vectors of D=128,
+group 32, synthetic Student-t(3) values with 4 outlier channels x20.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs under torchrun, one process per GPU; every rank quantises its own
+cache shard of the same shape (weak scaling, no collective on the data path);
+the time is the maximum over ranks.  Rank 0 prints one JSON line.
+
+`value` (Gvec/s, higher is better) = vectors of all ranks / device time of
+the K timed steps, inputs resident in HBM.  `e2e` is the same metric through
+the public API with the inputs in pinned host memory: each step copies the
+fp16 batch host->device, quantises, dequantises and copies the fp16 result
+back, chunked over three streams so that the copies overlap.  `roofline`
+reports the slower kernel's algorithmic HBM bytes per launch over its
+CUDA-event duration against the measured copy bandwidth.  `cpu_baseline` is
+the CPU oracle timed on the host's cores over a bounded sample of the same
+workload.  `--impl reference` times that oracle alone as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from kv_cache_quantization_02_b200 import workloads  # noqa: E402
+
+METRIC = "Gvec/s quantize+pack and dequant at D=128; achieved HBM GB/s vs B200 peak"
+UNIT = "Gvec/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCE = os.path.join(ROOT, "kv_cache_quantization_02_b200", "csrc", "kvq.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "kvq_traffic_qwen3_8b.json")
+
+
+def bytes_per_vector(D: int, G: int) -> int:
+    """Algorithmic HBM bytes per vector, the same for quantize and dequant:
+    2D (fp16 row) + D/2 (codes) + 2D/G (fp16 scales)."""
+    return 2 * D + D // 2 + 2 * (D // G)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (host logic, covered by the gloo tests)
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Maximum of a float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def shard_seed_offset(rank: int) -> int:
+    """Each rank draws a different cache shard of the same shape."""
+    return 1000 + rank
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML polling thread; read-only)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.error = None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001 - report, do not fail the bench
+            self._nv = None
+            self.error = repr(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception as e:  # noqa: BLE001
+                self.error = repr(e)
+                return
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nv is not None:
+            self._t.join()
+
+    def summary(self):
+        names = [k for k, bit in self.REASONS.items() if self.reasons & bit]
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": names,
+               "samples": len(self.samples), "source": "NVML, polled during the timed region"}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+
+# ---------------------------------------------------------------------------
+# peaks and the committed ncu traffic summary
+# ---------------------------------------------------------------------------
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_sha() -> str:
+    with open(KERNEL_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def traffic_per_launch(kernel: str, n_vec: int):
+    """DRAM bytes per launch from the committed ncu summary, scaled by vectors,
+    or None when the kernel source changed since those counters were taken."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except Exception:  # noqa: BLE001
+        return None
+    if t.get("kernel_source_sha256") != kernel_source_sha():
+        return None
+    k = t.get("kernels", {}).get(kernel)
+    if not k:
+        return None
+    return k["dram_bytes_per_vector"] * n_vec
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample, all host cores via threads; ctypes
+# releases the GIL during each call)
+# ---------------------------------------------------------------------------
+
+class OracleTimer:
+    """Times the CPU oracle (quantize + dequantize) over a bounded sample of a
+    workload, split across host threads.  The sample is drawn once (a pool of
+    at most 2^18 rows, tiled to the sample size: the oracle's work per row
+    does not depend on the values)."""
+
+    def __init__(self, w: workloads.Workload, G: int, target_s: float,
+                 threads: int | None = None):
+        import numpy as np
+        import oracle
+
+        self.o = oracle.get()
+        self.G = G
+        self.lam, self.s = workloads.params(w.D, w.seed)
+        self.threads = threads or len(os.sched_getaffinity(0))
+        probe = workloads.host_rows(w, 2048, seed_offset=77)
+        t0 = time.perf_counter()
+        self._one(probe)
+        per_row = (time.perf_counter() - t0) / len(probe)
+        rows = int(target_s * self.threads / max(per_row, 1e-9))
+        self.rows = max(self.threads * 256, min(rows, 1 << 22))
+        pool = workloads.host_rows(w, min(self.rows, 1 << 18), seed_offset=78)
+        reps = -(-self.rows // len(pool))
+        x16 = np.concatenate([pool] * reps)[: self.rows]
+        self.parts = [np.ascontiguousarray(p) for p in np.array_split(x16, self.threads)]
+
+    def _one(self, x16):
+        packed, scales = self.o.quantize(x16, self.lam, self.s, self.G)
+        self.o.dequantize(packed, scales, self.lam, self.s, self.G)
+
+    def run(self) -> float:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(self.threads) as ex:
+            t0 = time.perf_counter()
+            list(ex.map(self._one, self.parts))
+            return time.perf_counter() - t0
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args):
+    import torch
+    from kv_cache_quantization_02_b200 import kvq
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    w = workloads.WORKLOADS[args.workload]
+    G = args.group or w.groups[0]
+    n = args.n_vec or w.n_vec
+    D = w.D
+    lam, s = workloads.params(D, w.seed)
+    lam_t = torch.from_numpy(lam).to(dev)
+    s_t = torch.from_numpy(s).to(dev)
+
+    x = workloads.device_rows(w, n, dev, seed_offset=shard_seed_offset(rank))
+    packed = torch.empty((n, D // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((n, D // G), dtype=torch.float16, device=dev)
+    out = torch.empty((n, D), dtype=torch.float16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kvq.quantize(x, lam_t, s_t, G, packed=packed, scales=scales, stream=stream)
+        kvq.dequantize(packed, scales, lam_t, s_t, G, out=out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clocks:
+        start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            kvq.quantize(x, lam_t, s_t, G, packed=packed, scales=scales, stream=stream)
+            ev[i][1].record(stream)
+            kvq.dequantize(packed, scales, lam_t, s_t, G, out=out, stream=stream)
+            ev[i][2].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    elapsed_ms = start.elapsed_time(end)
+    q_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    d_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
+    q_ms = max_over_ranks(q_ms, world, dev)
+    d_ms = max_over_ranks(d_ms, world, dev)
+
+    bpv = bytes_per_vector(D, G)
+    total_vec = n * world
+    value = total_vec * K / (elapsed_ms / 1e3) / 1e9
+    peak, peak_kind = hbm_peak()
+    kern = {"kvq_quantize": q_ms, "kvq_dequantize": d_ms}
+    top = max(kern, key=kern.get)
+    achieved = bpv * n / (kern[top] / 1e3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, torch, kvq, dev, x, lam_t, s_t, G, world)
+    del x, out, packed, scales
+    torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        ot = OracleTimer(w, G, args.cpu_seconds)
+        dt = ot.run()
+        cpu = {"value": ot.rows / dt / 1e9, "unit": UNIT, "cores": ot.threads,
+               "kind": "oracle",
+               "sample": f"{ot.rows} vectors of the {w.name} distribution (host-drawn), "
+                         f"quantize+dequantize, {dt:.1f} s on {ot.threads} threads"}
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(elapsed_ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {
+            "workload": w.name, "n_vec_per_gpu": n, "D": D, "group": G, "shape": w.shape,
+            "values": w.note, "l2": "inputs larger than L2 (no flush)",
+            "parallelism": f"weak: {world} independent cache shard(s), no collective",
+            "global_batch": total_vec,
+        },
+        "detail": {
+            "quantize_ms": round(q_ms, 5), "dequantize_ms": round(d_ms, 5),
+            "quantize_gvec_s": round(n * world / (q_ms / 1e3) / 1e9, 4),
+            "dequantize_gvec_s": round(n * world / (d_ms / 1e3) / 1e9, 4),
+            "quantize_gbs": round(bpv * n / (q_ms / 1e3) / 1e9, 1),
+            "dequantize_gbs": round(bpv * n / (d_ms / 1e3) / 1e9, 1),
+            "bytes_per_vector": bpv,
+            "frac_of_8tbs": {"kvq_quantize": round(bpv * n / (q_ms / 1e3) / 1e9 / 8000, 4),
+                             "kvq_dequantize": round(bpv * n / (d_ms / 1e3) / 1e9 / 8000, 4)},
+        },
+        "roofline": {
+            "kernel": top, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+            "peak_kind": peak_kind, "unit": "GB/s", "frac": round(achieved / peak, 4),
+            "traffic": traffic_per_launch(top, n),
+            "algorithmic_bytes_per_launch": bpv * n,
+        },
+        "gpu_launches": 2 * K * world,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    return line
+
+
+def run_e2e(args, torch, kvq, dev, x_dev, lam_t, s_t, G, world):
+    """Host fp16 batch -> device -> quantize -> dequantize -> host fp16, per step,
+    chunked over three streams so that H2D, compute and D2H of different chunks
+    overlap.  Device-timed (events on the copy streams) and max over ranks."""
+    n, D = x_dev.shape
+    chunks = args.e2e_chunks
+    bounds = [(n * i) // chunks for i in range(chunks + 1)]
+    host_in = torch.empty((n, D), dtype=torch.float16, pin_memory=True)
+    host_in.copy_(x_dev, non_blocking=False)
+    host_out = torch.empty((n, D), dtype=torch.float16, pin_memory=True)
+    d_in = torch.empty_like(x_dev)
+    d_out = torch.empty_like(x_dev)
+    d_packed = torch.empty((n, D // 2), dtype=torch.uint8, device=dev)
+    d_scales = torch.empty((n, D // G), dtype=torch.float16, device=dev)
+    s_h2d, s_comp, s_d2h = (torch.cuda.Stream(dev) for _ in range(3))
+
+    def one_step():
+        for i in range(chunks):
+            a, b = bounds[i], bounds[i + 1]
+            e_in = torch.cuda.Event()
+            with torch.cuda.stream(s_h2d):
+                d_in[a:b].copy_(host_in[a:b], non_blocking=True)
+                e_in.record(s_h2d)
+            s_comp.wait_event(e_in)
+            kvq.quantize(d_in[a:b], lam_t, s_t, G, packed=d_packed[a:b],
+                         scales=d_scales[a:b], stream=s_comp)
+            kvq.dequantize(d_packed[a:b], d_scales[a:b], lam_t, s_t, G,
+                           out=d_out[a:b], stream=s_comp)
+            e_c = torch.cuda.Event()
+            e_c.record(s_comp)
+            s_d2h.wait_event(e_c)
+            with torch.cuda.stream(s_d2h):
+                host_out[a:b].copy_(d_out[a:b], non_blocking=True)
+
+    one_step()
+    torch.cuda.synchronize(dev)
+    K = max(1, min(args.steps, args.e2e_steps))
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    start.record(s_h2d)
+    s_comp.wait_event(start)
+    s_d2h.wait_event(start)
+    for _ in range(K):
+        one_step()
+    s_d2h.wait_stream(s_h2d)
+    s_d2h.wait_stream(s_comp)
+    end.record(s_d2h)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    ok = bool(torch.equal(host_out[:4096].to(dev), d_out[:4096]))
+    return {"value": round(n * world * K / (ms / 1e3) / 1e9, 4), "unit": UNIT,
+            "h2d_bytes_per_step": n * D * 2, "d2h_bytes_per_step": n * D * 2,
+            "steps": K, "ms_per_step": round(ms / K, 3), "chunks": chunks,
+            "result_copied_back": ok}
+
+
+# ---------------------------------------------------------------------------
+# the reference arm: the CPU oracle, as it stands, on the host's cores
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    w = workloads.WORKLOADS[args.workload]
+    G = args.group or w.groups[0]
+    ot = OracleTimer(w, G, args.ref_step_seconds)
+    times = [ot.run() for _ in range(args.warmup + args.steps)][args.warmup:]
+    tot_s = sum(times)
+    value = ot.rows * len(times) / tot_s / 1e9
+    rows, threads = ot.rows, ot.threads
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tot_s / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "n_vec_per_gpu": w.n_vec, "D": w.D, "group": G,
+                   "shape": w.shape, "values": w.note,
+                   "sample_per_step": f"{rows} vectors (bounded sample of the workload)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} vectors per step, quantize+dequantize"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def parse(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default="qwen3-8b-prefill", choices=sorted(workloads.WORKLOADS))
+    p.add_argument("--group", type=int, default=None)
+    p.add_argument("--n-vec", type=int, default=None, help="override vectors per GPU (profiling)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-chunks", type=int, default=16)
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--ref-step-seconds", type=float, default=2.0)
+    args = p.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours" and args.n_vec is None:
+        p.error("--warmup must be >= 3")
+    return args
+
+
+def main(argv=None):
+    args = parse(argv)
+    line = run_reference(args) if args.impl == "reference" else run_gpu(args)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,122 @@
+/*
+ * kvq.h -- C ABI of the B200 (sm_100a) fused KV-cache rotate-and-quantize
+ * library (libkvq.so).
+ *
+ * The operation, per KV vector x of length D (one layer / K-or-V / kv-head /
+ * token row of an fp16 cache):
+ *
+ *   y = H_D diag(s) (lambda . x) / sqrt(D)          (smooth scale + SRHT)
+ *   S_j = fp16(max_{i in group j} |y_i| / 7)         (per-group abs-max)
+ *   q_i = clamp(rint(y_i * (1/S_j)), -8, 7)          (signed int4)
+ *   two codes per byte, even element in the low nibble
+ *
+ * and the inverse  x_hat = (diag(s) H_D (q . S) / sqrt(D)) / lambda.
+ *
+ * Sources: "When Quantization Is Free: An int4 KV Cache That Outruns fp16 on
+ * Apple Silicon" (arXiv 2605.05699) -- Abstract (one fused kernel: sign-
+ * randomised transform + per-channel lambda + per-group abs-max + int4
+ * nibble pack; SRFT and SRHT equivalent in quality) and the technical
+ * summary on gist.science, Methodologie 1-3 (fixed random sign vector;
+ * kernel steps load & sign-multiply, transform, lambda rescale, per-group
+ * absolute-max reduction, round to signed int4, pack two int4 per byte;
+ * groups of 16).  The order "smooth scale, Hadamard transform, quantize /
+ * dequantize, inverse transform, unscale" follows "The Kernel That Finally
+ * Did Something" (VeloxQuant-MLX blog), section "The kernel toggle".
+ *
+ * Exact arithmetic contract (what makes results reproducible bit for bit):
+ *   - x_i * lambda_i is rounded to fp32 before any addition (no FMA);
+ *   - the unnormalised transform runs radix-2 butterflies with ascending
+ *     half-width h = 1, 2, ..., D/2, each output one fp32 a+b or a-b;
+ *   - y_i = v_i * c with c the fp32 value nearest 1/sqrt(D);
+ *   - S_j = fp16 round-to-nearest-even of the fp32 IEEE quotient max|y|/7,
+ *     saturated to 65504; a zero S_j gives zero codes;
+ *   - q_i = rint(y_i * r_j), r_j = fp32 IEEE reciprocal of S_j, round half
+ *     to even, saturated to [-8, 7];
+ *   - inverse: u_i = q_i * S_j (exact), the same transform, z_i = u_i * c,
+ *     out_i = fp16_rne((s_i z_i) * (1/lambda_i)), 1/lambda_i an fp32 IEEE
+ *     reciprocal.
+ *
+ * Memory: every pointer is DEVICE memory owned by the caller.  The library
+ * allocates nothing, keeps no state between calls except a per-device cache
+ * of launch limits, and never synchronises.  Calls are asynchronous on
+ * `stream` (a cudaStream_t; NULL means the legacy default stream).
+ *
+ * Errors: a failed precondition returns a negative kvq_status before any
+ * launch, and nothing is written.  A launch failure returns
+ * KVQ_ERR_LAUNCH.  Faults during execution surface, as usual in CUDA, at
+ * the caller's next synchronising runtime call.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KVQ_OK = 0,
+    KVQ_ERR_NULL = -1,    /* a required pointer is NULL                    */
+    KVQ_ERR_ALIGN = -2,   /* a pointer violates its alignment requirement  */
+    KVQ_ERR_DIM = -3,     /* D is not 64, 128 or 256                        */
+    KVQ_ERR_GROUP = -4,   /* group is not a power of two in [16, D]         */
+    KVQ_ERR_COUNT = -5,   /* n_vec < 0                                      */
+    KVQ_ERR_LAUNCH = -6   /* the kernel launch failed (see kvq_last_cuda_error) */
+} kvq_status;
+
+/*
+ * kvq_quantize -- rotate, quantise and pack n_vec vectors.
+ *
+ *   x       [in]  fp16 (IEEE binary16 bits) [n_vec][D], row-major, contiguous.
+ *                 32-byte aligned.  Finite values (NaN/Inf are not supported).
+ *   lambda  [in]  float32 [D]  per-channel smooth scale; 4-byte aligned;
+ *                 finite and non-zero.
+ *   signs   [in]  int8 [D]  the random sign vector; each entry +1 or -1 (any
+ *                 negative value is read as -1, anything else as +1).
+ *   n_vec         number of vectors (rows); 0 is a no-op returning KVQ_OK.
+ *   D             head dimension: 64, 128 or 256.
+ *   group         group size G: a power of two with 16 <= G <= D.
+ *   packed  [out] uint8 [n_vec][D/2]: code 2b in the low nibble of byte b,
+ *                 code 2b+1 in the high nibble, 4-bit two's complement.
+ *                 16-byte aligned.
+ *   scales  [out] fp16 bits [n_vec][D/G]; 2-byte aligned.
+ *   stream        cudaStream_t to launch on.
+ *
+ * `x` must not overlap `packed` or `scales`.
+ */
+int kvq_quantize(const uint16_t *x, const float *lambda, const int8_t *signs,
+                 int64_t n_vec, int D, int group,
+                 uint8_t *packed, uint16_t *scales, void *stream);
+
+/*
+ * kvq_dequantize -- unpack, rescale, inverse-rotate and un-scale n_vec
+ * vectors.  Same layouts and conventions as kvq_quantize.
+ *
+ *   packed  [in]  uint8 [n_vec][D/2]; 16-byte aligned.
+ *   scales  [in]  fp16 bits [n_vec][D/G]; 2-byte aligned.
+ *   lambda, signs, n_vec, D, group: as for kvq_quantize (same values that
+ *                 produced the codes).
+ *   x_out   [out] fp16 bits [n_vec][D]; 32-byte aligned; must not overlap
+ *                 the inputs.
+ */
+int kvq_dequantize(const uint8_t *packed, const uint16_t *scales,
+                   const float *lambda, const int8_t *signs,
+                   int64_t n_vec, int D, int group,
+                   uint16_t *x_out, void *stream);
+
+/* Human-readable name of a kvq_status value (static storage). */
+const char *kvq_status_string(int status);
+
+/* The cudaError_t value behind the calling thread's last KVQ_ERR_LAUNCH
+ * (0 if none). */
+int kvq_last_cuda_error(void);
+
+/* Library ABI version: (major << 16) | minor. */
+int kvq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

@@ -1,0 +1,148 @@
+"""Thin Python binding of libkvq.so (include/kvq.h), argument marshalling only.
+
+The raw entry points keep the C names and take integer device addresses:
+
+    kvq_quantize(x, lam, signs, n_vec, D, group, packed, scales, stream) -> status
+    kvq_dequantize(packed, scales, lam, signs, n_vec, D, group, x_out, stream) -> status
+
+``quantize`` / ``dequantize`` accept torch CUDA tensors, allocate outputs
+with torch when none are given, call the C entry point on the current (or
+given) stream and raise ``KvqError`` on a non-zero status.  Every step of the
+computation runs in the library's CUDA kernels; there is no fallback.  If the
+library is missing, importing this module raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch  # loads libcudart first, so the library shares torch's runtime
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_PKG, "libkvq.so")
+
+if not os.path.exists(LIBRARY):
+    raise ImportError(
+        f"{LIBRARY} is not built; run `python -m kv_cache_quantization_02_b200.build`")
+
+_lib = ctypes.CDLL(LIBRARY)
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I = ctypes.c_int
+
+_lib.kvq_quantize.restype = _I
+_lib.kvq_quantize.argtypes = [_P, _P, _P, _I64, _I, _I, _P, _P, _P]
+_lib.kvq_dequantize.restype = _I
+_lib.kvq_dequantize.argtypes = [_P, _P, _P, _P, _I64, _I, _I, _P, _P]
+_lib.kvq_status_string.restype = ctypes.c_char_p
+_lib.kvq_status_string.argtypes = [_I]
+_lib.kvq_last_cuda_error.restype = _I
+_lib.kvq_last_cuda_error.argtypes = []
+_lib.kvq_version.restype = _I
+_lib.kvq_version.argtypes = []
+
+KVQ_OK = 0
+KVQ_ERR_NULL = -1
+KVQ_ERR_ALIGN = -2
+KVQ_ERR_DIM = -3
+KVQ_ERR_GROUP = -4
+KVQ_ERR_COUNT = -5
+KVQ_ERR_LAUNCH = -6
+
+
+class KvqError(RuntimeError):
+    def __init__(self, status: int):
+        msg = kvq_status_string(status)
+        if status == KVQ_ERR_LAUNCH:
+            msg += f" (cudaError {kvq_last_cuda_error()})"
+        super().__init__(msg)
+        self.status = status
+
+
+# ---- raw C entry points -------------------------------------------------
+
+def kvq_quantize(x: int, lam: int, signs: int, n_vec: int, D: int, group: int,
+                 packed: int, scales: int, stream: int = 0) -> int:
+    return _lib.kvq_quantize(x, lam, signs, n_vec, D, group, packed, scales, stream)
+
+
+def kvq_dequantize(packed: int, scales: int, lam: int, signs: int, n_vec: int,
+                   D: int, group: int, x_out: int, stream: int = 0) -> int:
+    return _lib.kvq_dequantize(packed, scales, lam, signs, n_vec, D, group, x_out, stream)
+
+
+def kvq_status_string(status: int) -> str:
+    return _lib.kvq_status_string(status).decode()
+
+
+def kvq_last_cuda_error() -> int:
+    return _lib.kvq_last_cuda_error()
+
+
+def kvq_version() -> int:
+    return _lib.kvq_version()
+
+
+# ---- torch-tensor convenience --------------------------------------------
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _need(t: torch.Tensor, dtype, shape, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def quantize(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: int,
+             packed: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+             stream=None):
+    """x: fp16 [n, D] -> (packed uint8 [n, D/2], scales fp16 [n, D/group])."""
+    if x.dim() != 2:
+        raise ValueError("x must be [n_vec, D]")
+    n, D = x.shape
+    _need(x, torch.float16, (n, D), "x")
+    _need(lam, torch.float32, (D,), "lambda")
+    _need(signs, torch.int8, (D,), "signs")
+    if packed is None:
+        packed = torch.empty((n, D // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((n, max(D // group, 1)), dtype=torch.float16, device=x.device)
+    _need(packed, torch.uint8, (n, D // 2), "packed")
+    _need(scales, torch.float16, (n, max(D // group, 1)), "scales")
+    rc = kvq_quantize(x.data_ptr(), lam.data_ptr(), signs.data_ptr(), n, D, group,
+                      packed.data_ptr(), scales.data_ptr(), _stream_handle(stream))
+    if rc != KVQ_OK:
+        raise KvqError(rc)
+    return packed, scales
+
+
+def dequantize(packed: torch.Tensor, scales: torch.Tensor, lam: torch.Tensor,
+               signs: torch.Tensor, group: int, out: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """(packed uint8 [n, D/2], scales fp16 [n, D/group]) -> fp16 [n, D]."""
+    if packed.dim() != 2:
+        raise ValueError("packed must be [n_vec, D/2]")
+    n, D = packed.shape[0], packed.shape[1] * 2
+    _need(packed, torch.uint8, (n, D // 2), "packed")
+    _need(scales, torch.float16, (n, max(D // group, 1)), "scales")
+    _need(lam, torch.float32, (D,), "lambda")
+    _need(signs, torch.int8, (D,), "signs")
+    if out is None:
+        out = torch.empty((n, D), dtype=torch.float16, device=packed.device)
+    _need(out, torch.float16, (n, D), "out")
+    rc = kvq_dequantize(packed.data_ptr(), scales.data_ptr(), lam.data_ptr(),
+                        signs.data_ptr(), n, D, group, out.data_ptr(),
+                        _stream_handle(stream))
+    if rc != KVQ_OK:
+        raise KvqError(rc)
+    return out

@@ -1,0 +1,105 @@
+"""The C-ABI library loads, exports every symbol include/kvq.h declares, and
+rejects bad arguments with a status before touching the GPU (no GPU needed:
+every call here returns before any CUDA runtime call)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kvq.h")
+
+
+def _declared():
+    with open(HEADER) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kvq_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    from kv_cache_quantization_02_b200 import kvq
+    return kvq
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for want in ("kvq_quantize", "kvq_dequantize", "kvq_status_string"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(kvq):
+    lib = ctypes.CDLL(kvq.LIBRARY)
+    for name in _declared():
+        assert hasattr(lib, name), f"{name} declared in kvq.h but not exported"
+    out = subprocess.run(["nm", "-D", "--defined-only", kvq.LIBRARY],
+                         capture_output=True, text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (kvq_[a-z0-9_]+)\b", out))
+    assert exported == set(_declared()), f"exports {exported} != header {_declared()}"
+
+
+def test_version_and_status_strings(kvq):
+    assert kvq.kvq_version() >> 16 == 1
+    for st in range(-6, 1):
+        s = kvq.kvq_status_string(st)
+        assert s.startswith("KVQ_")
+    assert "unknown" in kvq.kvq_status_string(-99)
+    assert kvq.kvq_last_cuda_error() == 0
+
+
+# Fake, never-dereferenced device addresses: every case below fails a
+# precondition, so the library returns before any CUDA call.
+A = 0x7F0000000000          # 256-byte aligned
+
+
+@pytest.mark.parametrize("D,G,n,want", [
+    (96, 32, 10, -3), (32, 32, 10, -3), (512, 32, 10, -3),
+    (128, 8, 10, -4), (128, 24, 10, -4), (128, 256, 10, -4), (64, 128, 10, -4),
+    (128, 32, -1, -5),
+])
+def test_shape_errors(kvq, D, G, n, want):
+    assert kvq.kvq_quantize(A, A, A, n, D, G, A, A, 0) == want
+    assert kvq.kvq_dequantize(A, A, A, A, n, D, G, A, 0) == want
+
+
+def test_zero_vectors_is_a_noop(kvq):
+    assert kvq.kvq_quantize(0, 0, 0, 0, 128, 32, 0, 0, 0) == 0
+    assert kvq.kvq_dequantize(0, 0, 0, 0, 0, 128, 32, 0, 0) == 0
+
+
+@pytest.mark.parametrize("which", range(5))
+def test_null_pointers(kvq, which):
+    q = [A, A, A, A, A]
+    q[which] = 0
+    x, lam, s, packed, scales = q
+    assert kvq.kvq_quantize(x, lam, s, 4, 128, 32, packed, scales, 0) == -1
+    packed, scales, lam, s, out = q
+    assert kvq.kvq_dequantize(packed, scales, lam, s, 4, 128, 32, out, 0) == -1
+
+
+def test_alignment(kvq):
+    assert kvq.kvq_quantize(A + 16, A, A, 4, 128, 32, A, A, 0) == -2      # x needs 32
+    assert kvq.kvq_quantize(A, A + 2, A, 4, 128, 32, A, A, 0) == -2       # lambda needs 4
+    assert kvq.kvq_quantize(A, A, A, 4, 128, 32, A + 8, A, 0) == -2       # packed needs 16
+    assert kvq.kvq_quantize(A, A, A, 4, 128, 32, A, A + 1, 0) == -2       # scales need 2
+    assert kvq.kvq_dequantize(A + 8, A, A, A, 4, 128, 32, A, 0) == -2
+    assert kvq.kvq_dequantize(A, A + 1, A, A, 4, 128, 32, A, 0) == -2
+    assert kvq.kvq_dequantize(A, A, A + 1, A, 4, 128, 32, A, 0) == -2
+    assert kvq.kvq_dequantize(A, A, A, A, 4, 128, 32, A + 16, 0) == -2    # x_out needs 32
+
+
+def test_binding_fails_loudly_without_the_library(tmp_path):
+    """The product path has no fallback: a missing library is an ImportError."""
+    import importlib.util
+    import shutil
+    pkg = tmp_path / "kv_cache_quantization_02_b200"
+    pkg.mkdir()
+    src = os.path.join(ROOT, "kv_cache_quantization_02_b200", "kvq.py")
+    shutil.copy(src, pkg / "kvq.py")
+    spec = importlib.util.spec_from_file_location("kvq_nolib", pkg / "kvq.py")
+    mod = importlib.util.module_from_spec(spec)
+    with pytest.raises(ImportError):
+        spec.loader.exec_module(mod)
