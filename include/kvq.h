@@ -38,13 +38,18 @@
  *
  * Memory: every pointer is DEVICE memory owned by the caller.  The library
  * allocates nothing, keeps no state between calls except a per-device cache
- * of launch limits, and never synchronises.  Calls are asynchronous on
- * `stream` (a cudaStream_t; NULL means the legacy default stream).
+ * of launch limits and one per-device fault word (below), and never
+ * synchronises.  Calls are asynchronous on `stream` (a cudaStream_t; NULL
+ * means the legacy default stream) and launch on the calling thread's
+ * current device, which must own the buffers and the stream.
  *
  * Errors: a failed precondition returns a negative kvq_status before any
  * launch, and nothing is written.  A launch failure returns
  * KVQ_ERR_LAUNCH.  Faults during execution surface, as usual in CUDA, at
- * the caller's next synchronising runtime call.
+ * the caller's next synchronising runtime call.  The kernels stage data with
+ * asynchronous bulk copies and wait for them on shared-memory barriers; every
+ * such wait is bounded, and a block that gives up sets the device's fault
+ * word and returns with its outputs incomplete (kvq_fault_status).
  */
 #ifndef KVQ_H
 #define KVQ_H
@@ -69,7 +74,7 @@ typedef enum {
  * kvq_quantize -- rotate, quantise and pack n_vec vectors.
  *
  *   x       [in]  fp16 (IEEE binary16 bits) [n_vec][D], row-major, contiguous.
- *                 32-byte aligned.  Finite values (NaN/Inf are not supported).
+ *                 16-byte aligned.  Finite values (NaN/Inf are not supported).
  *   lambda  [in]  float32 [D]  per-channel smooth scale; 4-byte aligned;
  *                 finite and non-zero.
  *   signs   [in]  int8 [D]  the random sign vector; each entry +1 or -1 (any
@@ -97,13 +102,33 @@ int kvq_quantize(const uint16_t *x, const float *lambda, const int8_t *signs,
  *   scales  [in]  fp16 bits [n_vec][D/G]; 2-byte aligned.
  *   lambda, signs, n_vec, D, group: as for kvq_quantize (same values that
  *                 produced the codes).
- *   x_out   [out] fp16 bits [n_vec][D]; 32-byte aligned; must not overlap
+ *   x_out   [out] fp16 bits [n_vec][D]; 16-byte aligned; must not overlap
  *                 the inputs.
  */
 int kvq_dequantize(const uint8_t *packed, const uint16_t *scales,
                    const float *lambda, const int8_t *signs,
                    int64_t n_vec, int D, int group,
                    uint16_t *x_out, void *stream);
+
+/*
+ * kvq_fault_status -- the current device's fault word: 0 when every bounded
+ * wait of every kernel so far completed; bit 0 set when a quantize or
+ * dequantize block gave up waiting for its bulk copies (its outputs are then
+ * incomplete); bit 1 set by kvq_selftest_wait_timeout.  Non-zero `clear`
+ * resets the word.  Synchronous (it copies the word to the host, which waits
+ * for prior work on the device's legacy default stream).  Returns -1 if the
+ * word cannot be read.
+ */
+int kvq_fault_status(int clear);
+
+/*
+ * kvq_selftest_wait_timeout -- launches one block that waits, at most `limit`
+ * polls, on a shared-memory barrier that nothing completes, and then takes
+ * the same give-up path as the real kernels (sets bit 1 of the fault word and
+ * returns).  It exists to test that path; it touches no caller memory.
+ * Returns KVQ_OK or KVQ_ERR_LAUNCH.
+ */
+int kvq_selftest_wait_timeout(uint32_t limit, void *stream);
 
 /* Human-readable name of a kvq_status value (static storage). */
 const char *kvq_status_string(int status);

@@ -12,20 +12,26 @@
 // Kernel That Finally Did Something" (VeloxQuant-MLX blog), "The kernel
 // toggle".
 //
-// Work decomposition.  A vector of D fp16 channels is owned by a team of
-// LANES = D/32 consecutive lanes of one warp; lane `sub` of the team holds
-// channels [32*sub, 32*sub + 32) in registers as 16 packed fp32 pairs
-// p[m] = (v[m], v[m+16]), m = 0..15.  The butterfly with half-width h then
-// runs as
-//   h = 1, 2, 4, 8   : packed f32x2 adds/subs between pairs p[m], p[m+h];
-//   h = 16           : inside each pair;
-//   h = 32 .. D/2    : across the team's lanes with __shfl_xor_sync, one
-//                      fused multiply-add by +-1 per element.
-// Every butterfly output is one IEEE fp32 a+b or a-b of the same operands, in
-// the same ascending-h order as the plain sequential loop, so the result is
-// bit-identical to it.  Loads and stores are 256-bit (one full 32-byte
-// sector per lane); a warp covers 32/LANES vectors per iteration and walks a
-// grid-stride loop, so every lane executes every shuffle.
+// Work decomposition.  One lane owns EPT = min(D, 128) channels of a vector
+// (a vector is owned by LANES = D / EPT lanes: one, or two at D = 256) and
+// holds them in registers as EPT/2 packed fp32 pairs p[m] = (v[m], v[m+EPT/2]).
+// The butterfly with half-width h then runs as packed f32x2 adds/subs between
+// pair registers for h < EPT/2, inside each pair for h = EPT/2, and across
+// the two lanes with __shfl_xor_sync for h = EPT (D = 256 only).  Every
+// butterfly output is one IEEE fp32 a+b or a-b of the same operands in the
+// same ascending-h order as the plain sequential loop, so the result is
+// bit-identical to it.
+//
+// Data movement.  A persistent block of 128 lanes walks tiles of 128 / LANES
+// vectors.  Quantize: the tile's fp16 rows arrive in shared memory through
+// per-row TMA bulk copies (cp.async.bulk, no multicast) into a double-
+// buffered ring, at a row stride that makes the lanes' 16-byte reads
+// bank-conflict free; codes and scales leave with 16-byte and 2-byte stores.
+// Dequantize: the tile's packed codes arrive as one bulk copy; each lane
+// writes its fp16 row into a padded shared-memory staging row and a per-row
+// bulk store (cp.async.bulk shared->global) writes it out.  Every mbarrier
+// wait is bounded; a block that gives up sets a device fault word, drains its
+// own copies and returns (kvq_fault_status reads the word).
 //
 // This translation unit is compiled with --fmad=false and uses only _rn
 // intrinsics on the contract-sensitive steps, so no multiply is ever fused
@@ -42,137 +48,145 @@
 
 namespace {
 
-constexpr int kThreads = 256;          // threads per block (8 warps)
-constexpr int kChunk = 32;             // channels per lane
+constexpr int kThreads = 128;              // lanes per block (4 warps)
 constexpr unsigned kFullMask = 0xffffffffu;
+constexpr uint32_t kSpinLimit = 1u << 22;  // bounded mbarrier waits
 constexpr int kMaxDevices = 64;
 
 thread_local int g_last_cuda_error = 0;
 
+// Non-zero once some block gave up a bounded wait (see kvq_fault_status).
+__device__ unsigned int g_kvq_fault = 0;
+
 // ---------------------------------------------------------------------------
-// Memory access helpers (256-bit where a lane moves a whole 32-byte sector).
+// Tile geometry.  RS is the shared-memory stride of one vector's fp16 row
+// (second half at +HS when D = 256); with it the 16-byte accesses of the 8
+// lanes of a quarter-warp phase fall into 8 distinct bank groups.
+// ---------------------------------------------------------------------------
+template <int D>
+struct Tile {
+  static constexpr int EPT = D < 128 ? D : 128;    // channels per lane
+  static constexpr int LANES = D / EPT;             // lanes per vector
+  static constexpr int NP = EPT / 2;                // fp32 pairs per lane
+  static constexpr int HALF = EPT / 2;              // pair (m, m + HALF)
+  static constexpr int ROWS = kThreads / LANES;     // vectors per tile
+  static constexpr int SEG = EPT * 2;               // bytes of a lane's fp16 segment
+  static constexpr int RS = (D == 256) ? 544 : 2 * D + 16;
+  static constexpr int HS = (D == 256) ? 272 : 0;
+  static constexpr int STAGE = ROWS * RS;           // bytes of one fp16 tile
+  static constexpr int TAB = LANES * NP * 8;        // per-channel pair table
+  static constexpr int PIN = ROWS * (D / 2);        // bytes of one packed tile
+};
+
+template <int D>
+constexpr int quantize_smem_bytes() { return 2 * Tile<D>::STAGE + Tile<D>::TAB + 16; }
+template <int D>
+constexpr int dequantize_smem_bytes() { return 2 * Tile<D>::PIN + Tile<D>::STAGE + Tile<D>::TAB + 16; }
+
+// ---------------------------------------------------------------------------
+// Asynchronous copies and barriers.
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ void ld_nc_v8(const void* p, uint32_t (&r)[8]) {
-  asm("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]),
-        "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-      : "l"(p));
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-
-__device__ __forceinline__ void ld_nc_v4(const void* p, uint32_t (&r)[4]) {
-  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-      : "l"(p));
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_addr(bar)), "r"(count) : "memory");
 }
-
-__device__ __forceinline__ void st_v8(void* p, const uint32_t (&r)[8]) {
-  asm volatile("st.global.v8.u32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
-               :: "l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]),
-                  "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-               : "memory");
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+               :: "r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+// Waits for the phase with the given parity; false if `limit` polls passed.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
+  const uint32_t a = smem_addr(bar);
+  for (uint32_t it = 0; it < limit; ++it) {
+    uint32_t ok;
+    asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+                 " selp.u32 %0, 1, 0, p;\n}" : "=r"(ok) : "r"(a), "r"(parity) : "memory");
+    if (ok) return true;
+  }
+  return false;
+}
+// global -> shared bulk copy completing on an mbarrier (no multicast)
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               :: "r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
+}
+// shared -> global bulk copy, tracked per thread in bulk groups
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               :: "l"(dst), "r"(smem_addr(src)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void st_v4(void* p, const uint32_t (&r)[4]) {
   asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};"
-               :: "l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3])
-               : "memory");
+               :: "l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]) : "memory");
 }
+
+// ---------------------------------------------------------------------------
+// Arithmetic helpers.
+// ---------------------------------------------------------------------------
 
 __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t w) {
   __half2 h = *reinterpret_cast<__half2*>(&w);
   return __half22float2(h);
 }
-
 __device__ __forceinline__ uint32_t float2_to_half2_bits(float lo, float hi) {
   __half2 h = __floats2half2_rn(lo, hi);   // .x (low 16 bits) = lo
   return *reinterpret_cast<uint32_t*>(&h);
 }
-
 __device__ __forceinline__ float half_bits_to_float(uint16_t b) {
   return __half2float(__ushort_as_half(b));
 }
-
-// a - b as one rounding: fma(b, -1, a).
+// a - b with one rounding: fma(b, -1, a).
 __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
   return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
 }
-
-// ---------------------------------------------------------------------------
-// Unnormalised Walsh-Hadamard transform of one vector held by a team of
-// LANES lanes, 32 channels per lane as pairs p[m] = (v[m], v[m+16]).
-// Stages in ascending half-width h = 1 .. D/2.
-// ---------------------------------------------------------------------------
-
-template <int LANES>
-__device__ __forceinline__ void fwht_team(float2 (&p)[16], int sub) {
-#pragma unroll
-  for (int h = 1; h < 16; h <<= 1) {
-#pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      if ((m & h) == 0) {
-        const float2 a = p[m];
-        const float2 b = p[m + h];
-        p[m] = __fadd2_rn(a, b);
-        p[m + h] = fsub2(a, b);
-      }
-    }
-  }
-  // h = 16: the two halves of each pair.
-#pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    const float a = p[m].x, b = p[m].y;
-    p[m] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
-  }
-  // h = 32 .. 16*LANES: partner lane sub ^ bit.  The lower partner keeps
-  // a + b, the upper one b_partner - a_own = fma(-1, own, partner).
-#pragma unroll
-  for (int bit = 1; bit < LANES; bit <<= 1) {
-    const float sg = (sub & bit) ? -1.0f : 1.0f;
-    const float2 sg2 = make_float2(sg, sg);
-#pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      float2 o;
-      o.x = __shfl_xor_sync(kFullMask, p[m].x, bit);
-      o.y = __shfl_xor_sync(kFullMask, p[m].y, bit);
-      p[m] = __ffma2_rn(sg2, p[m], o);
-    }
-  }
+// max(a, |b|, |c|)
+__device__ __forceinline__ float amax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
+  return d;
 }
 
-// Per-channel constant table laid out so that lane `sub` reads its pairs
-// (p[2j], p[2j+1]) as one float4 at [j][sub]: conflict-free across subs.
-template <int LANES>
-__device__ __forceinline__ void fill_pair_table(float4 (*tab)[LANES],
-                                                const float* __restrict__ lam,
-                                                const int8_t* __restrict__ sg,
-                                                bool reciprocal) {
-  for (int i = threadIdx.x; i < 8 * LANES; i += blockDim.x) {
-    const int j = i / LANES, sub = i % LANES;
-    const int base = kChunk * sub + 2 * j;
-    const int ch[4] = {base, base + 16, base + 1, base + 17};
-    float v[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      float l = lam[ch[k]];
-      if (reciprocal) l = __frcp_rn(l);          // fp32 IEEE 1/lambda
-      v[k] = (sg[ch[k]] < 0) ? -l : l;           // exact sign flip
-    }
-    tab[j][sub] = make_float4(v[0], v[1], v[2], v[3]);
-  }
+// fp32 quotient a / 7, correctly rounded: q0 = a * RN(1/7), then one residual
+// correction r = a - 7 q0 (exact by fma), q = q0 + r * RN(1/7) (Markstein's
+// division by a known divisor; equal to IEEE a / 7.0f for every positive
+// finite fp32 a, checked exhaustively).
+__device__ __forceinline__ float div7_rn(float a) {
+  const float zh = 0x1.24924ap-3f;               // RN(1/7)
+  const float q0 = __fmul_rn(a, zh);
+  const float r = __fmaf_rn(-q0, 7.0f, a);
+  return __fmaf_rn(r, zh, q0);
 }
-
-// Scale of one group: S = fp16_rne(a / 7) saturated to 65504; r = 1/S
-// (r = 0 when S = 0, which makes every code of the group 0).
+// fp32 reciprocal of a positive fp16 value s, correctly rounded: approximate
+// reciprocal plus one Newton-Raphson step.  1/s lies at least 2^-35 (relative)
+// away from every rounding midpoint because s has an 11-bit significand, far
+// beyond the step's error; checked against IEEE 1/s for every positive
+// finite fp16 s.
+__device__ __forceinline__ float rcp_f16val(float s) {
+  float r0;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(s));
+  const float e = __fmaf_rn(-s, r0, 1.0f);
+  return __fmaf_rn(r0, e, r0);
+}
+// Scale of one group: S = fp16_rne(a / 7) saturated to 65504 (satfinite);
+// r = 1/S, or 0 when S = 0 (which makes every code of the group 0).
 __device__ __forceinline__ uint16_t group_scale(float a, float& r) {
-  const float q = __fdiv_rn(a, 7.0f);
-  uint16_t b = __half_as_ushort(__float2half_rn(q));
-  if (b == 0x7C00u) b = 0x7BFFu;
+  uint16_t b;
+  asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(b) : "f"(div7_rn(a)));
   const float sf = half_bits_to_float(b);
-  r = (sf == 0.0f) ? 0.0f : __frcp_rn(sf);
+  r = (sf == 0.0f) ? 0.0f : rcp_f16val(sf);
   return b;
 }
-
 // Eight codes -> one 32-bit word, code k in bits [4k, 4k+4), each saturated
 // to [-8, 7] by the packing conversion.
 __device__ __forceinline__ uint32_t pack8(const int (&q)[8]) {
@@ -183,242 +197,409 @@ __device__ __forceinline__ uint32_t pack8(const int (&q)[8]) {
   asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(q[1]), "r"(q[0]), "r"(d));
   return d;
 }
+// w * s for fp16 operands, exact in fp32 (a product of two fp16 values has at
+// most 22 significant bits); the -0.0 addend keeps the sign of a zero product.
+__device__ __forceinline__ float mul_f16_f32(__half w, uint16_t s) {
+  float d;
+  asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(__half_as_ushort(w)), "h"(s), "f"(-0.0f));
+  return d;
+}
 
-// Signed 4-bit field k of w, sign-extended.
-__device__ __forceinline__ int nibble(uint32_t w, int k) {
-  return static_cast<int>(w << (28 - 4 * k)) >> 28;
+// ---------------------------------------------------------------------------
+// Walsh-Hadamard butterflies (unnormalised, Sylvester order) on one vector
+// held as pairs p[m] = (v[m], v[m+HALF]) by LANES lanes, from half-width H0
+// upwards (stages below H0 already applied).
+// ---------------------------------------------------------------------------
+template <int EPT, int LANES, int H0 = 1>
+__device__ __forceinline__ void fwht_pairs(float2 (&p)[EPT / 2], int sub) {
+  constexpr int NP = EPT / 2;
+#pragma unroll
+  for (int h = H0; h < NP; h <<= 1) {
+#pragma unroll
+    for (int m = 0; m < NP; ++m) {
+      if ((m & h) == 0) {
+        const float2 a = p[m];
+        const float2 b = p[m + h];
+        p[m] = __fadd2_rn(a, b);
+        p[m + h] = fsub2(a, b);
+      }
+    }
+  }
+  // h = HALF: the two halves of each pair
+#pragma unroll
+  for (int m = 0; m < NP; ++m) {
+    const float a = p[m].x, b = p[m].y;
+    p[m] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
+  }
+  // h = EPT (two lanes per vector): the lower lane keeps a + b, the upper one
+  // a_partner - b_own = fma(-1, own, partner).
+#pragma unroll
+  for (int bit = 1; bit < LANES; bit <<= 1) {
+    const float sg = (sub & bit) ? -1.0f : 1.0f;
+    const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+    for (int m = 0; m < NP; ++m) {
+      float2 o;
+      o.x = __shfl_xor_sync(kFullMask, p[m].x, bit);
+      o.y = __shfl_xor_sync(kFullMask, p[m].y, bit);
+      p[m] = __ffma2_rn(sg2, p[m], o);
+    }
+  }
+}
+
+// Per-channel table: tab[sub * NP/2 + q] = (c[2q], c[2q+HALF], c[2q+1],
+// c[2q+1+HALF]) over lane `sub`'s channels, c = lambda*s (quantize) or
+// s * fp32(1/lambda) (dequantize).  Both products are exact sign flips.
+template <int D>
+__device__ __forceinline__ void fill_tab(float4* tab, const float* __restrict__ lam,
+                                         const int8_t* __restrict__ sg, bool reciprocal) {
+  using T = Tile<D>;
+  for (int i = threadIdx.x; i < T::LANES * (T::NP / 2); i += blockDim.x) {
+    const int sub = i / (T::NP / 2), q = i % (T::NP / 2);
+    const int base = T::EPT * sub + 2 * q;
+    const int ch[4] = {base, base + T::HALF, base + 1, base + 1 + T::HALF};
+    float v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float l = lam[ch[k]];
+      if (reciprocal) l = __frcp_rn(l);          // fp32 IEEE 1/lambda
+      v[k] = (sg[ch[k]] < 0) ? -l : l;
+    }
+    tab[i] = make_float4(v[0], v[1], v[2], v[3]);
+  }
 }
 
 // ---------------------------------------------------------------------------
 // Quantize: fp16 [n][D] -> packed u8 [n][D/2] + fp16 scales [n][D/G].
 // ---------------------------------------------------------------------------
-
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads)
-kvq_quantize_kernel(const uint16_t* __restrict__ x,
-                    const float* __restrict__ lam,
-                    const int8_t* __restrict__ sgn,
-                    int64_t n, float c,
-                    uint8_t* __restrict__ packed,
-                    uint16_t* __restrict__ scales) {
-  constexpr int LANES = D / kChunk;
-  constexpr int VPW = 32 / LANES;                 // vectors per warp
-  constexpr int GPL = G / kChunk;                 // lanes per group (G >= 32)
-  __shared__ float4 ls_tab[8][LANES];             // lambda * s, paired
-  fill_pair_table<LANES>(ls_tab, lam, sgn, false);
+__global__ void __launch_bounds__(kThreads, 3)
+kvq_quantize_kernel(const uint16_t* __restrict__ x, const float* __restrict__ lam,
+                    const int8_t* __restrict__ sgn, int64_t n, float c,
+                    uint8_t* __restrict__ packed, uint16_t* __restrict__ scales) {
+  using T = Tile<D>;
+  constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF, ROWS = T::ROWS;
+  constexpr int GX = (G < HALF) ? G : HALF;      // pairs spanned by one group (G <= HALF)
+  constexpr int NGH = HALF / GX;                 // groups per half-lane
+  extern __shared__ __align__(128) uint8_t smem[];
+  const float4* tab = reinterpret_cast<const float4*>(smem + 2 * T::STAGE);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 2 * T::STAGE + T::TAB);
+  const int tid = threadIdx.x;
+  const int sub = tid % LANES;
+  const int rin = tid / LANES;
+  fill_tab<D>(reinterpret_cast<float4*>(smem + 2 * T::STAGE), lam, sgn, false);
+  if (tid == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   __syncthreads();
 
-  const int lane = threadIdx.x & 31;
-  const int sub = lane % LANES;
-  const int team = lane / LANES;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+  const int64_t ntiles = (n + ROWS - 1) / ROWS;
+  // tile k of this block -> stage k & 1; every lane copies its own segment
+  auto issue = [&](int64_t k) {
+    const int64_t tile = blockIdx.x + k * gridDim.x;
+    if (tile >= ntiles) return;
+    const int64_t row0 = tile * ROWS;
+    const int valid = static_cast<int>(n - row0 < ROWS ? n - row0 : ROWS);
+    uint64_t* b = &bar[k & 1];
+    if (tid == 0) mbar_expect_tx(b, static_cast<uint32_t>(valid) * 2 * D);
+    if (rin < valid)
+      bulk_g2s(smem + (k & 1) * T::STAGE + rin * T::RS + sub * T::HS,
+               x + (row0 + rin) * D + sub * EPT, T::SEG, b);
+  };
+  issue(0);
+  issue(1);
   const float2 c2 = make_float2(c, c);
-
-  for (int64_t base = warp * VPW; base < n; base += nwarps * VPW) {
-    const int64_t row = base + team;
+  const float4* mytab = tab + sub * (NP / 2);
+  for (int64_t k = 0;; ++k) {
+    const int64_t tile = blockIdx.x + k * gridDim.x;
+    if (tile >= ntiles) break;
+    const bool ok = mbar_wait(&bar[k & 1], static_cast<uint32_t>((k >> 1) & 1), kSpinLimit);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) atomicOr(&g_kvq_fault, 1u);
+      if (blockIdx.x + (k + 1) * gridDim.x < ntiles)
+        mbar_wait(&bar[(k + 1) & 1], static_cast<uint32_t>(((k + 1) >> 1) & 1), kSpinLimit);
+      return;
+    }
+    const int64_t row = tile * ROWS + rin;
     const bool active = row < n;
-    const int64_t rrow = active ? row : n - 1;
 
-    // a1: load 32 fp16 channels, widen, multiply by lambda*s (one rounding).
-    const uint16_t* src = x + rrow * D + sub * kChunk;
-    uint32_t w[16];
-    {
-      uint32_t lo[8], hi[8];
-      ld_nc_v8(src, lo);
-      ld_nc_v8(src + 16, hi);
+    // a1: widen fp16 and multiply by lambda*s (one rounding per element).
+    const uint4* seg = reinterpret_cast<const uint4*>(smem + (k & 1) * T::STAGE + rin * T::RS + sub * T::HS);
+    float2 p[NP];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) { w[j] = lo[j]; w[8 + j] = hi[j]; }
-    }
-    float2 p[16];
+    for (int j = 0; j < NP / 8; ++j) {
+      const uint4 a = seg[j];                // channels 8j .. 8j+7
+      const uint4 b = seg[j + HALF / 8];     // channels HALF+8j .. HALF+8j+7
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float2 a = half2_bits_to_float2(w[j]);       // channels 2j, 2j+1
-      const float2 b = half2_bits_to_float2(w[8 + j]);   // channels 2j+16, 2j+17
-      const float4 t = ls_tab[j][sub];
-      p[2 * j] = __fmul2_rn(make_float2(a.x, b.x), make_float2(t.x, t.y));
-      p[2 * j + 1] = __fmul2_rn(make_float2(a.y, b.y), make_float2(t.z, t.w));
-    }
-
-    // a2: transform; a3: normalise.
-    fwht_team<LANES>(p, sub);
-#pragma unroll
-    for (int m = 0; m < 16; ++m) p[m] = __fmul2_rn(p[m], c2);
-
-    // a4: group abs-max.  .x holds channels 0..15 of the chunk, .y 16..31.
-    float ax = 0.0f, ay = 0.0f;
-#pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      ax = fmaxf(ax, fabsf(p[m].x));
-      ay = fmaxf(ay, fabsf(p[m].y));
-    }
-    float rx, ry;
-    uint16_t sbx, sby = 0;
-    if constexpr (G == 16) {
-      sbx = group_scale(ax, rx);
-      sby = group_scale(ay, ry);
-    } else {
-      float a = fmaxf(ax, ay);
-#pragma unroll
-      for (int bit = 1; bit < GPL; bit <<= 1)
-        a = fmaxf(a, __shfl_xor_sync(kFullMask, a, bit));
-      sbx = group_scale(a, rx);
-      ry = rx;
-    }
-
-    // a6: codes = rint(y * r), saturated to [-8, 7] while packing (a7).
-    const float2 r2 = make_float2(rx, ry);
-    int qx[16], qy[16];
-#pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const float2 t = __fmul2_rn(p[m], r2);
-      qx[m] = __float2int_rn(t.x);
-      qy[m] = __float2int_rn(t.y);
-    }
-    uint32_t out[4];
-    {
-      int q8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) q8[k] = qx[k];
-      out[0] = pack8(q8);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) q8[k] = qx[8 + k];
-      out[1] = pack8(q8);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) q8[k] = qy[k];
-      out[2] = pack8(q8);
-#pragma unroll
-      for (int k = 0; k < 8; ++k) q8[k] = qy[8 + k];
-      out[3] = pack8(q8);
-    }
-    if (active) {
-      st_v4(packed + row * (D / 2) + sub * 16, out);
-      uint16_t* srow = scales + row * (D / G);
-      if constexpr (G == 16) {
-        srow[2 * sub] = sbx;
-        srow[2 * sub + 1] = sby;
-      } else if constexpr (G == 32) {
-        srow[sub] = sbx;
-      } else {
-        if (sub % GPL == 0) srow[sub / GPL] = sbx;
+      for (int t = 0; t < 4; ++t) {
+        const float2 fa = half2_bits_to_float2(aw[t]);
+        const float2 fb = half2_bits_to_float2(bw[t]);
+        const float4 l = mytab[4 * j + t];
+        p[8 * j + 2 * t] = __fmul2_rn(make_float2(fa.x, fb.x), make_float2(l.x, l.y));
+        p[8 * j + 2 * t + 1] = __fmul2_rn(make_float2(fa.y, fb.y), make_float2(l.z, l.w));
       }
     }
+    // a2, a3: transform, normalise.
+    fwht_pairs<EPT, LANES>(p, sub);
+#pragma unroll
+    for (int m = 0; m < NP; ++m) p[m] = __fmul2_rn(p[m], c2);
+
+    // a4, a5: group abs-max and scales.  Pair .x holds channels [0, HALF) of
+    // the lane, .y holds [HALF, EPT).
+    float rx[NGH], ry[NGH];
+    uint16_t bx[NGH], by[NGH];
+    if constexpr (G <= HALF) {
+#pragma unroll
+      for (int j = 0; j < NGH; ++j) {
+        float ax = 0.f, ay = 0.f;
+#pragma unroll
+        for (int m = 0; m < GX; m += 2) {
+          ax = amax3(ax, p[j * GX + m].x, p[j * GX + m + 1].x);
+          ay = amax3(ay, p[j * GX + m].y, p[j * GX + m + 1].y);
+        }
+        bx[j] = group_scale(ax, rx[j]);
+        by[j] = group_scale(ay, ry[j]);
+      }
+    } else {
+      float a = 0.f;
+#pragma unroll
+      for (int m = 0; m < NP; ++m) a = amax3(a, p[m].x, p[m].y);
+#pragma unroll
+      for (int bit = 1; bit < G / EPT; bit <<= 1) a = fmaxf(a, __shfl_xor_sync(kFullMask, a, bit));
+      bx[0] = group_scale(a, rx[0]);
+      ry[0] = rx[0];
+      by[0] = bx[0];
+    }
+
+    // a6, a7: codes = rint(y * r) (half to even), saturated and packed.
+    uint32_t out[EPT / 8];
+#pragma unroll
+    for (int k8 = 0; k8 < NP / 8; ++k8) {
+      int qa[8], qb[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int m = 8 * k8 + t;
+        const float2 v = __fmul2_rn(p[m], make_float2(rx[m / GX], ry[m / GX]));
+        qa[t] = __float2int_rn(v.x);
+        qb[t] = __float2int_rn(v.y);
+      }
+      out[k8] = pack8(qa);
+      out[k8 + NP / 8] = pack8(qb);
+    }
+    if (active) {
+      uint8_t* dst = packed + row * (D / 2) + sub * (EPT / 2);
+#pragma unroll
+      for (int k4 = 0; k4 < EPT / 32; ++k4) {
+        const uint32_t t4[4] = {out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]};
+        st_v4(dst + 16 * k4, t4);
+      }
+      uint16_t* srow = scales + row * (D / G);
+      if constexpr (G <= HALF) {
+#pragma unroll
+        for (int j = 0; j < NGH; ++j) {
+          srow[sub * (EPT / G) + j] = bx[j];
+          srow[sub * (EPT / G) + NGH + j] = by[j];
+        }
+      } else {
+        if (sub % (G / EPT) == 0) srow[sub / (G / EPT)] = bx[0];
+      }
+    }
+    __syncthreads();          // everyone is done with stage k & 1
+    issue(k + 2);
   }
 }
 
 // ---------------------------------------------------------------------------
 // Dequantize: packed u8 [n][D/2] + fp16 scales [n][D/G] -> fp16 [n][D].
 // ---------------------------------------------------------------------------
-
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads)
-kvq_dequantize_kernel(const uint8_t* __restrict__ packed,
-                      const uint16_t* __restrict__ scales,
-                      const float* __restrict__ lam,
-                      const int8_t* __restrict__ sgn,
-                      int64_t n, float c,
-                      uint16_t* __restrict__ x_out) {
-  constexpr int LANES = D / kChunk;
-  constexpr int VPW = 32 / LANES;
-  constexpr int GPL = G / kChunk;
-  __shared__ float4 sil_tab[8][LANES];            // s / lambda, paired
-  fill_pair_table<LANES>(sil_tab, lam, sgn, true);
+__global__ void __launch_bounds__(kThreads, 3)
+kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
+                      const float* __restrict__ lam, const int8_t* __restrict__ sgn,
+                      int64_t n, float c, uint16_t* __restrict__ x_out) {
+  using T = Tile<D>;
+  constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF, ROWS = T::ROWS;
+  constexpr int PIN = T::PIN;
+  constexpr int GX = (G < HALF) ? G : HALF;
+  constexpr int NGH = HALF / GX;
+  constexpr int HG = (G < NP) ? G : NP;          // butterfly stages h < HG stay inside a group
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* stage_out = smem + 2 * PIN;
+  const float4* tab = reinterpret_cast<const float4*>(smem + 2 * PIN + T::STAGE);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 2 * PIN + T::STAGE + T::TAB);
+  const int tid = threadIdx.x;
+  const int sub = tid % LANES;
+  const int rin = tid / LANES;
+  fill_tab<D>(reinterpret_cast<float4*>(smem + 2 * PIN + T::STAGE), lam, sgn, true);
+  if (tid == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   __syncthreads();
 
-  const int lane = threadIdx.x & 31;
-  const int sub = lane % LANES;
-  const int team = lane / LANES;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kThreads) >> 5;
+  const int64_t ntiles = (n + ROWS - 1) / ROWS;
+  auto issue = [&](int64_t k) {
+    const int64_t tile = blockIdx.x + k * gridDim.x;
+    if (tile >= ntiles || tid != 0) return;
+    const int64_t row0 = tile * ROWS;
+    const int valid = static_cast<int>(n - row0 < ROWS ? n - row0 : ROWS);
+    uint64_t* b = &bar[k & 1];
+    mbar_expect_tx(b, static_cast<uint32_t>(valid) * (D / 2));
+    bulk_g2s(smem + (k & 1) * PIN, packed + row0 * (D / 2), static_cast<uint32_t>(valid) * (D / 2), b);
+  };
+  issue(0);
+  issue(1);
   const float2 c2 = make_float2(c, c);
-
-  for (int64_t base = warp * VPW; base < n; base += nwarps * VPW) {
-    const int64_t row = base + team;
+  const float4* mytab = tab + sub * (NP / 2);
+  const __half2 k1032 = __floats2half2_rn(1032.0f, 1032.0f);
+  const __half2 k16th = __floats2half2_rn(0.0625f, 0.0625f);
+  const __half2 km72 = __floats2half2_rn(-72.0f, -72.0f);
+  for (int64_t k = 0;; ++k) {
+    const int64_t tile = blockIdx.x + k * gridDim.x;
+    if (tile >= ntiles) break;
+    const int64_t row = tile * ROWS + rin;
     const bool active = row < n;
     const int64_t rrow = active ? row : n - 1;
-
-    // a8: 16 bytes of codes (channels 32*sub .. +31) and their scales.
-    uint32_t w[4];
-    ld_nc_v4(packed + rrow * (D / 2) + sub * 16, w);
     const uint16_t* srow = scales + rrow * (D / G);
-    float sx, sy;
-    if constexpr (G == 16) {
-      sx = half_bits_to_float(srow[2 * sub]);
-      sy = half_bits_to_float(srow[2 * sub + 1]);
+    uint16_t sx[NGH], sy[NGH];
+    if constexpr (G <= HALF) {
+#pragma unroll
+      for (int j = 0; j < NGH; ++j) {
+        sx[j] = srow[sub * (EPT / G) + j];
+        sy[j] = srow[sub * (EPT / G) + NGH + j];
+      }
     } else {
-      sx = half_bits_to_float(srow[sub / GPL]);
-      sy = sx;
+      sx[0] = srow[sub / (G / EPT)];
+      sy[0] = sx[0];
     }
-    const float2 s2 = make_float2(sx, sy);
-    float2 p[16];
+    const bool ok = mbar_wait(&bar[k & 1], static_cast<uint32_t>((k >> 1) & 1), kSpinLimit);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) atomicOr(&g_kvq_fault, 1u);
+      if (blockIdx.x + (k + 1) * gridDim.x < ntiles)
+        mbar_wait(&bar[(k + 1) & 1], static_cast<uint32_t>(((k + 1) >> 1) & 1), kSpinLimit);
+      bulk_wait0();
+      return;
+    }
+    // a8: the lane's EPT/2 bytes of codes; nibbles biased to n = q + 8.
+    const uint4* seg = reinterpret_cast<const uint4*>(smem + (k & 1) * PIN + rin * (D / 2) + sub * (EPT / 2));
+    uint32_t w[EPT / 8];
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const float qa = __int2float_rn(nibble(w[m / 8], m % 8));
-      const float qb = __int2float_rn(nibble(w[2 + m / 8], m % 8));
-      p[m] = __fmul2_rn(make_float2(qa, qb), s2);       // exact
+    for (int j = 0; j < EPT / 32; ++j) {
+      const uint4 a = seg[j];
+      w[4 * j] = a.x ^ 0x88888888u;
+      w[4 * j + 1] = a.y ^ 0x88888888u;
+      w[4 * j + 2] = a.z ^ 0x88888888u;
+      w[4 * j + 3] = a.w ^ 0x88888888u;
     }
+    // Codes as exact fp16 integers in pairs hq[m] = (q[m], q[m+HALF]):
+    // (n | 0x6400) is the fp16 value 1024 + n, (16 n | 0x6400) is 1024 + 16 n.
+    __half2 hq[NP];
+#pragma unroll
+    for (int kw = 0; kw < NP / 8; ++kw) {
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        // byte t of word kw to byte 0, byte t of word kw + HALF/8 to byte 2
+        const uint32_t xb = __byte_perm(w[kw], w[kw + HALF / 8], 0x0400u | (t << 8) | t);
+        const uint32_t lo = (xb & 0x000F000Fu) | 0x64006400u;
+        const uint32_t hi = (xb & 0x00F000F0u) | 0x64006400u;
+        hq[8 * kw + 2 * t] = __hsub2(*reinterpret_cast<const __half2*>(&lo), k1032);
+        hq[8 * kw + 2 * t + 1] = __hfma2(*reinterpret_cast<const __half2*>(&hi), k16th, km72);
+      }
+    }
+    // a9 (first part): butterfly stages inside a group act on integers of
+    // magnitude <= 8 * 2^stage <= 512, exact in fp16; u = W * S is then exact
+    // in fp32 and equal, stage for stage, to the fp32 butterfly of q * S.
+#pragma unroll
+    for (int h = 1; h < HG; h <<= 1) {
+#pragma unroll
+      for (int m = 0; m < NP; ++m) {
+        if ((m & h) == 0) {
+          const __half2 a = hq[m], b = hq[m + h];
+          hq[m] = __hadd2(a, b);
+          hq[m + h] = __hsub2(a, b);
+        }
+      }
+    }
+    float2 p[NP];
+#pragma unroll
+    for (int m = 0; m < NP; ++m)
+      p[m] = make_float2(mul_f16_f32(__low2half(hq[m]), sx[m / GX]),
+                         mul_f16_f32(__high2half(hq[m]), sy[m / GX]));
+    // a9 (rest): the stages that cross groups, in fp32.
+    fwht_pairs<EPT, LANES, HG>(p, sub);
 
-    // a9: inverse rotation (same transform), normalise; a10: s / lambda.
-    fwht_team<LANES>(p, sub);
-    uint32_t o[16];
+    // a10: normalise, s / lambda, fp16; stage the row and bulk-store it.
+    bulk_wait_read0();        // this lane's previous store has read its row
+    uint4* orow = reinterpret_cast<uint4*>(stage_out + rin * T::RS + sub * T::HS);
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 t = sil_tab[j][sub];
-      const float2 a = __fmul2_rn(__fmul2_rn(p[2 * j], c2), make_float2(t.x, t.y));
-      const float2 b = __fmul2_rn(__fmul2_rn(p[2 * j + 1], c2), make_float2(t.z, t.w));
-      o[j] = float2_to_half2_bits(a.x, b.x);         // channels 2j, 2j+1
-      o[8 + j] = float2_to_half2_bits(a.y, b.y);     // channels 2j+16, 2j+17
+    for (int j = 0; j < NP / 8; ++j) {
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float4 l = mytab[4 * j + t];
+        const float2 a = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t], c2), make_float2(l.x, l.y));
+        const float2 b = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t + 1], c2), make_float2(l.z, l.w));
+        lo[t] = float2_to_half2_bits(a.x, b.x);   // channels 8j+2t, +1
+        hi[t] = float2_to_half2_bits(a.y, b.y);   // channels HALF+8j+2t, +1
+      }
+      orow[j] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      orow[j + HALF / 8] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     }
+    fence_proxy_async();
     if (active) {
-      uint16_t* dst = x_out + row * D + sub * kChunk;
-      uint32_t lo[8], hi[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) { lo[j] = o[j]; hi[j] = o[8 + j]; }
-      st_v8(dst, lo);
-      st_v8(dst + 16, hi);
+      bulk_s2g(x_out + row * D + sub * EPT, orow, T::SEG);
+      bulk_commit();
     }
+    __syncthreads();          // everyone is done with packed stage k & 1
+    issue(k + 2);
   }
+  bulk_wait0();
+}
+
+// A barrier that nothing completes, waited on with a short limit: exercises
+// the bounded-wait give-up path (fault word) without any real copy.
+__global__ void kvq_wait_timeout_kernel(uint32_t limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) { mbar_init(&bar, 1); mbar_fence_init(); }
+  __syncthreads();
+  const bool ok = mbar_wait(&bar, 0, limit);
+  if (__syncthreads_or(!ok) && threadIdx.x == 0) atomicOr(&g_kvq_fault, 2u);
 }
 
 // ---------------------------------------------------------------------------
 // Launch plumbing.
 // ---------------------------------------------------------------------------
 
-struct DeviceInfo {
-  std::atomic<int> sms{0};
-};
-DeviceInfo g_dev[kMaxDevices];
+std::atomic<int> g_sms[kMaxDevices];
 
 int sm_count(int dev) {
   if (dev < 0 || dev >= kMaxDevices) return 0;
-  int v = g_dev[dev].sms.load(std::memory_order_relaxed);
+  int v = g_sms[dev].load(std::memory_order_relaxed);
   if (v == 0) {
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    g_dev[dev].sms.store(v, std::memory_order_relaxed);
+    g_sms[dev].store(v, std::memory_order_relaxed);
   }
   return v;
 }
 
-template <typename Kernel>
-int blocks_per_sm(Kernel k, int dev) {
+// Resident blocks per SM of one kernel instance on one device; the first call
+// also raises the instance's dynamic shared-memory limit.
+template <int KIND, int D, int G, typename Kernel>
+int blocks_per_sm(Kernel k, int dev, int smem) {
   static std::atomic<int> cache[kMaxDevices];
   if (dev < 0 || dev >= kMaxDevices) return 1;
   int v = cache[dev].load(std::memory_order_relaxed);
   if (v == 0) {
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k, kThreads, 0) != cudaSuccess || v < 1)
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k, kThreads, smem) != cudaSuccess || v < 1)
       v = 1;
     cache[dev].store(v, std::memory_order_relaxed);
   }
   return v;
 }
 
-template <typename Kernel>
-int grid_for(Kernel k, int64_t n, int D) {
+template <int KIND, int D, int G, typename Kernel>
+int grid_for(Kernel k, int64_t n, int smem) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-  const int64_t per_block = static_cast<int64_t>(kThreads / 32) * (32 / (D / kChunk));
-  const int64_t need = (n + per_block - 1) / per_block;
-  int64_t cap = static_cast<int64_t>(sm_count(dev)) * blocks_per_sm(k, dev);
+  const int64_t need = (n + Tile<D>::ROWS - 1) / Tile<D>::ROWS;
+  int64_t cap = static_cast<int64_t>(sm_count(dev)) * blocks_per_sm<KIND, D, G>(k, dev, smem);
   if (cap < 1) cap = 1;
   return static_cast<int>(need < cap ? need : cap);
 }
@@ -449,9 +630,10 @@ template <int D, int G>
 int launch_quantize(const uint16_t* x, const float* lam, const int8_t* s, int64_t n,
                     uint8_t* packed, uint16_t* scales, cudaStream_t st) {
   auto k = kvq_quantize_kernel<D, G>;
-  const int grid = grid_for(k, n, D);
+  constexpr int smem = quantize_smem_bytes<D>();
+  const int grid = grid_for<0, D, G>(k, n, smem);
   (void)cudaGetLastError();
-  k<<<grid, kThreads, 0, st>>>(x, lam, s, n, norm_const(D), packed, scales);
+  k<<<grid, kThreads, smem, st>>>(x, lam, s, n, norm_const(D), packed, scales);
   return finish_launch();
 }
 
@@ -459,9 +641,10 @@ template <int D, int G>
 int launch_dequantize(const uint8_t* packed, const uint16_t* scales, const float* lam,
                       const int8_t* s, int64_t n, uint16_t* out, cudaStream_t st) {
   auto k = kvq_dequantize_kernel<D, G>;
-  const int grid = grid_for(k, n, D);
+  constexpr int smem = dequantize_smem_bytes<D>();
+  const int grid = grid_for<1, D, G>(k, n, smem);
   (void)cudaGetLastError();
-  k<<<grid, kThreads, 0, st>>>(packed, scales, lam, s, n, norm_const(D), out);
+  k<<<grid, kThreads, smem, st>>>(packed, scales, lam, s, n, norm_const(D), out);
   return finish_launch();
 }
 
@@ -507,7 +690,7 @@ int kvq_quantize(const uint16_t* x, const float* lambda, const int8_t* signs,
   if (rc != KVQ_OK) return rc;
   if (n_vec == 0) return KVQ_OK;
   if (!x || !lambda || !signs || !packed || !scales) return KVQ_ERR_NULL;
-  if (!aligned(x, 32) || !aligned(packed, 16) || !aligned(scales, 2) || !aligned(lambda, 4))
+  if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(scales, 2) || !aligned(lambda, 4))
     return KVQ_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   KVQ_DISPATCH(launch_quantize, D, group, x, lambda, signs, n_vec, packed, scales, st);
@@ -520,10 +703,26 @@ int kvq_dequantize(const uint8_t* packed, const uint16_t* scales, const float* l
   if (rc != KVQ_OK) return rc;
   if (n_vec == 0) return KVQ_OK;
   if (!packed || !scales || !lambda || !signs || !x_out) return KVQ_ERR_NULL;
-  if (!aligned(x_out, 32) || !aligned(packed, 16) || !aligned(scales, 2) || !aligned(lambda, 4))
+  if (!aligned(x_out, 16) || !aligned(packed, 16) || !aligned(scales, 2) || !aligned(lambda, 4))
     return KVQ_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   KVQ_DISPATCH(launch_dequantize, D, group, packed, scales, lambda, signs, n_vec, x_out, st);
+}
+
+int kvq_fault_status(int clear) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_kvq_fault, sizeof v) != cudaSuccess) return -1;
+  if (clear && v) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_kvq_fault, &zero, sizeof zero) != cudaSuccess) return -1;
+  }
+  return static_cast<int>(v);
+}
+
+int kvq_selftest_wait_timeout(uint32_t limit, void* stream) {
+  (void)cudaGetLastError();
+  kvq_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit);
+  return finish_launch();
 }
 
 const char* kvq_status_string(int status) {
@@ -541,6 +740,6 @@ const char* kvq_status_string(int status) {
 
 int kvq_last_cuda_error(void) { return g_last_cuda_error; }
 
-int kvq_version(void) { return (1 << 16) | 0; }
+int kvq_version(void) { return (1 << 16) | 1; }
 
 }  // extern "C"

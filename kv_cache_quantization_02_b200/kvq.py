@@ -41,6 +41,10 @@ _lib.kvq_last_cuda_error.restype = _I
 _lib.kvq_last_cuda_error.argtypes = []
 _lib.kvq_version.restype = _I
 _lib.kvq_version.argtypes = []
+_lib.kvq_fault_status.restype = _I
+_lib.kvq_fault_status.argtypes = [_I]
+_lib.kvq_selftest_wait_timeout.restype = _I
+_lib.kvq_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _P]
 
 KVQ_OK = 0
 KVQ_ERR_NULL = -1
@@ -82,6 +86,14 @@ def kvq_last_cuda_error() -> int:
 
 def kvq_version() -> int:
     return _lib.kvq_version()
+
+
+def kvq_fault_status(clear: bool = False) -> int:
+    return _lib.kvq_fault_status(1 if clear else 0)
+
+
+def kvq_selftest_wait_timeout(limit: int, stream: int = 0) -> int:
+    return _lib.kvq_selftest_wait_timeout(limit, stream)
 
 
 # ---- torch-tensor convenience --------------------------------------------

@@ -81,14 +81,14 @@ def test_null_pointers(kvq, which):
 
 
 def test_alignment(kvq):
-    assert kvq.kvq_quantize(A + 16, A, A, 4, 128, 32, A, A, 0) == -2      # x needs 32
+    assert kvq.kvq_quantize(A + 8, A, A, 4, 128, 32, A, A, 0) == -2       # x needs 16
     assert kvq.kvq_quantize(A, A + 2, A, 4, 128, 32, A, A, 0) == -2       # lambda needs 4
     assert kvq.kvq_quantize(A, A, A, 4, 128, 32, A + 8, A, 0) == -2       # packed needs 16
     assert kvq.kvq_quantize(A, A, A, 4, 128, 32, A, A + 1, 0) == -2       # scales need 2
     assert kvq.kvq_dequantize(A + 8, A, A, A, 4, 128, 32, A, 0) == -2
     assert kvq.kvq_dequantize(A, A + 1, A, A, 4, 128, 32, A, 0) == -2
     assert kvq.kvq_dequantize(A, A, A + 1, A, 4, 128, 32, A, 0) == -2
-    assert kvq.kvq_dequantize(A, A, A, A, 4, 128, 32, A + 16, 0) == -2    # x_out needs 32
+    assert kvq.kvq_dequantize(A, A, A, A, 4, 128, 32, A + 8, 0) == -2     # x_out needs 16
 
 
 def test_binding_fails_loudly_without_the_library(tmp_path):

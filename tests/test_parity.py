@@ -136,7 +136,7 @@ def test_misaligned_input_is_rejected(env):
     D, G, n = 128, 32, 4
     dev = torch.device("cuda")
     flat = torch.zeros(n * D + 64, dtype=torch.float16, device=dev)
-    x = flat[8:8 + n * D].view(n, D)            # 16-byte offset: not 32-aligned
+    x = flat[4:4 + n * D].view(n, D)            # 8-byte offset: not 16-aligned
     lam = torch.ones(D, dtype=torch.float32, device=dev)
     s = torch.ones(D, dtype=torch.int8, device=dev)
     with pytest.raises(kvq.KvqError) as ei:
