@@ -66,7 +66,7 @@ typedef enum {
     KVQ_ERR_ALIGN = -2,   /* a pointer violates its alignment requirement  */
     KVQ_ERR_DIM = -3,     /* D is not 64, 128 or 256                        */
     KVQ_ERR_GROUP = -4,   /* group is not a power of two in [16, D]         */
-    KVQ_ERR_COUNT = -5,   /* n_vec < 0                                      */
+    KVQ_ERR_COUNT = -5,   /* n_vec < 0 or n_vec > 2^31 - 256                */
     KVQ_ERR_LAUNCH = -6   /* the kernel launch failed (see kvq_last_cuda_error) */
 } kvq_status;
 
@@ -79,7 +79,10 @@ typedef enum {
  *                 finite and non-zero.
  *   signs   [in]  int8 [D]  the random sign vector; each entry +1 or -1 (any
  *                 negative value is read as -1, anything else as +1).
- *   n_vec         number of vectors (rows); 0 is a no-op returning KVQ_OK.
+ *   n_vec         number of vectors (rows), 0 <= n_vec <= 2^31 - 256 (the copy
+ *                 engine's row coordinates are 32-bit); 0 is a no-op
+ *                 returning KVQ_OK; larger counts return KVQ_ERR_COUNT
+ *                 (split the call).
  *   D             head dimension: 64, 128 or 256.
  *   group         group size G: a power of two with 16 <= G <= D.
  *   packed  [out] uint8 [n_vec][D/2]: code 2b in the low nibble of byte b,

@@ -23,20 +23,23 @@
 // bit-identical to it.
 //
 // Data movement.  A persistent block of 128 lanes walks tiles of 128 / LANES
-// vectors.  Quantize: the tile's fp16 rows arrive in shared memory through
-// per-row TMA bulk copies (cp.async.bulk, no multicast) into a double-
-// buffered ring, at a row stride that makes the lanes' 16-byte reads
-// bank-conflict free; codes and scales leave with 16-byte and 2-byte stores.
-// Dequantize: the tile's packed codes arrive as one bulk copy; each lane
-// writes its fp16 row into a padded shared-memory staging row and a per-row
-// bulk store (cp.async.bulk shared->global) writes it out.  Every mbarrier
-// wait is bounded; a block that gives up sets a device fault word, drains its
-// own copies and returns (kvq_fault_status reads the word).
+// vectors, double-buffered in shared memory.  Each fp16 tile moves as Q = D/64
+// tensor copies (one per 64-channel quarter of the rows, 2-D maps of 64
+// channels x n rows with the 128-byte swizzle), issued by one thread; chunk c
+// of tile row t lands at chunk c ^ (t mod 8), so lanes reading consecutive
+// rows hit distinct bank groups.  Quantize: tensor loads in, 16-byte code
+// stores and 2-byte scale stores out.  Dequantize: the tile's packed codes
+// arrive as one bulk copy; the lanes write their fp16 rows into a swizzled
+// staging tile that leaves as Q tensor stores (rows past n are clipped by the
+// copy engine).  No copy uses multicast.  Every mbarrier wait is bounded; a
+// block that gives up sets a device fault word, drains its own copies and
+// returns (kvq_fault_status reads the word).
 //
 // This translation unit is compiled with --fmad=false and uses only _rn
 // intrinsics on the contract-sensitive steps, so no multiply is ever fused
 // into a following add.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
 
@@ -52,6 +55,7 @@ constexpr int kThreads = 128;              // lanes per block (4 warps)
 constexpr unsigned kFullMask = 0xffffffffu;
 constexpr uint32_t kSpinLimit = 1u << 22;  // bounded mbarrier waits
 constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxVectors = (int64_t{1} << 31) - 256;  // tensor-copy row coordinates are 32-bit
 
 thread_local int g_last_cuda_error = 0;
 
@@ -59,9 +63,8 @@ thread_local int g_last_cuda_error = 0;
 __device__ unsigned int g_kvq_fault = 0;
 
 // ---------------------------------------------------------------------------
-// Tile geometry.  RS is the shared-memory stride of one vector's fp16 row
-// (second half at +HS when D = 256); with it the 16-byte accesses of the 8
-// lanes of a quarter-warp phase fall into 8 distinct bank groups.
+// Tile geometry: ROWS vectors per tile, the fp16 rows split into Q quarters
+// of 64 channels (128 bytes), each quarter a [ROWS][128 B] swizzled block.
 // ---------------------------------------------------------------------------
 template <int D>
 struct Tile {
@@ -70,18 +73,33 @@ struct Tile {
   static constexpr int NP = EPT / 2;                // fp32 pairs per lane
   static constexpr int HALF = EPT / 2;              // pair (m, m + HALF)
   static constexpr int ROWS = kThreads / LANES;     // vectors per tile
-  static constexpr int SEG = EPT * 2;               // bytes of a lane's fp16 segment
-  static constexpr int RS = (D == 256) ? 544 : 2 * D + 16;
-  static constexpr int HS = (D == 256) ? 272 : 0;
-  static constexpr int STAGE = ROWS * RS;           // bytes of one fp16 tile
+  static constexpr int Q = D / 64;                  // 64-channel quarters of a row
+  static constexpr int QB = ROWS * 128;             // bytes of one quarter of a tile
+  static constexpr int STAGE = Q * QB;              // bytes of one fp16 tile (= ROWS * 2D)
   static constexpr int TAB = LANES * NP * 8;        // per-channel pair table
   static constexpr int PIN = ROWS * (D / 2);        // bytes of one packed tile
 };
 
+// Byte offset, inside one fp16 tile, of 16-byte chunk c (channels 8c..8c+7) of
+// quarter q of tile row t.  Each quarter is a [ROWS][128 B] block written by a
+// 128-byte-swizzled tensor copy: chunk c of row t sits at chunk c ^ (t mod 8),
+// so the 8 lanes of a quarter-warp phase, which read 8 consecutive rows,
+// touch 8 distinct bank groups.
 template <int D>
-constexpr int quantize_smem_bytes() { return 2 * Tile<D>::STAGE + Tile<D>::TAB + 16; }
+__device__ __forceinline__ int tile_off(int q, int t, int c) {
+  return q * Tile<D>::QB + t * 128 + ((c ^ (t & 7)) << 4);
+}
+
+// The kernel arguments that describe a tensor copy of the fp16 rows: one 2-D
+// map (64 channels x n rows, row stride 2D bytes) per quarter.
+struct RowMaps {
+  CUtensorMap q[4];
+};
+
 template <int D>
-constexpr int dequantize_smem_bytes() { return 2 * Tile<D>::PIN + Tile<D>::STAGE + Tile<D>::TAB + 16; }
+constexpr int quantize_smem_bytes() { return 1024 + 2 * Tile<D>::STAGE + Tile<D>::TAB + 16; }
+template <int D>
+constexpr int dequantize_smem_bytes() { return 1024 + Tile<D>::STAGE + 2 * Tile<D>::PIN + Tile<D>::TAB + 16; }
 
 // ---------------------------------------------------------------------------
 // Asynchronous copies and barriers.
@@ -116,10 +134,16 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                :: "r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
 }
-// shared -> global bulk copy, tracked per thread in bulk groups
-__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
-               :: "l"(dst), "r"(smem_addr(src)), "r"(bytes) : "memory");
+// 2-D tensor tile load (128B swizzle via the map), completing on an mbarrier
+__device__ __forceinline__ void tensor_g2s(void* dst, const CUtensorMap* map, int x0, int y0, uint64_t* bar) {
+  asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+               :: "r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x0), "r"(y0), "r"(smem_addr(bar))
+               : "memory");
+}
+// 2-D tensor tile store, tracked in bulk groups; rows outside the tensor are skipped
+__device__ __forceinline__ void tensor_s2g(const CUtensorMap* map, int x0, int y0, const void* src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
+               :: "l"(reinterpret_cast<uint64_t>(map)), "r"(x0), "r"(y0), "r"(smem_addr(src)) : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
@@ -274,60 +298,59 @@ __device__ __forceinline__ void fill_tab(float4* tab, const float* __restrict__ 
 // ---------------------------------------------------------------------------
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 3)
-kvq_quantize_kernel(const uint16_t* __restrict__ x, const float* __restrict__ lam,
+kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restrict__ lam,
                     const int8_t* __restrict__ sgn, int64_t n, float c,
                     uint8_t* __restrict__ packed, uint16_t* __restrict__ scales) {
   using T = Tile<D>;
   constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF, ROWS = T::ROWS;
   constexpr int GX = (G < HALF) ? G : HALF;      // pairs spanned by one group (G <= HALF)
   constexpr int NGH = HALF / GX;                 // groups per half-lane
-  extern __shared__ __align__(128) uint8_t smem[];
-  const float4* tab = reinterpret_cast<const float4*>(smem + 2 * T::STAGE);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float4* tabw = reinterpret_cast<float4*>(smem + 2 * T::STAGE);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 2 * T::STAGE + T::TAB);
   const int tid = threadIdx.x;
   const int sub = tid % LANES;
   const int rin = tid / LANES;
-  fill_tab<D>(reinterpret_cast<float4*>(smem + 2 * T::STAGE), lam, sgn, false);
+  fill_tab<D>(tabw, lam, sgn, false);
   if (tid == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   __syncthreads();
 
   const int64_t ntiles = (n + ROWS - 1) / ROWS;
-  // tile k of this block -> stage k & 1; every lane copies its own segment
-  auto issue = [&](int64_t k) {
-    const int64_t tile = blockIdx.x + k * gridDim.x;
-    if (tile >= ntiles) return;
-    const int64_t row0 = tile * ROWS;
-    const int valid = static_cast<int>(n - row0 < ROWS ? n - row0 : ROWS);
-    uint64_t* b = &bar[k & 1];
-    if (tid == 0) mbar_expect_tx(b, static_cast<uint32_t>(valid) * 2 * D);
-    if (rin < valid)
-      bulk_g2s(smem + (k & 1) * T::STAGE + rin * T::RS + sub * T::HS,
-               x + (row0 + rin) * D + sub * EPT, T::SEG, b);
+  const int tstride = gridDim.x;
+  // tile -> stage: one thread issues the Q quarter copies of the whole tile
+  auto issue = [&](int64_t tile, int stage) {
+    if (tile >= ntiles || tid != 0) return;
+    mbar_expect_tx(&bar[stage], T::STAGE);
+#pragma unroll
+    for (int q = 0; q < T::Q; ++q)
+      tensor_g2s(smem + stage * T::STAGE + q * T::QB, &maps.q[q], 0, static_cast<int>(tile * ROWS), &bar[stage]);
   };
-  issue(0);
-  issue(1);
+  issue(blockIdx.x, 0);
+  issue(static_cast<int64_t>(blockIdx.x) + tstride, 1);
   const float2 c2 = make_float2(c, c);
-  const float4* mytab = tab + sub * (NP / 2);
-  for (int64_t k = 0;; ++k) {
-    const int64_t tile = blockIdx.x + k * gridDim.x;
-    if (tile >= ntiles) break;
-    const bool ok = mbar_wait(&bar[k & 1], static_cast<uint32_t>((k >> 1) & 1), kSpinLimit);
+  const float4* mytab = tabw + sub * (NP / 2);
+  int64_t tile = blockIdx.x;
+  for (uint32_t k = 0; tile < ntiles; ++k, tile += tstride) {
+    const int stage = k & 1;
+    const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);
     if (__syncthreads_or(!ok)) {
       if (tid == 0) atomicOr(&g_kvq_fault, 1u);
-      if (blockIdx.x + (k + 1) * gridDim.x < ntiles)
-        mbar_wait(&bar[(k + 1) & 1], static_cast<uint32_t>(((k + 1) >> 1) & 1), kSpinLimit);
+      if (tile + tstride < ntiles) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
       return;
     }
     const int64_t row = tile * ROWS + rin;
     const bool active = row < n;
 
     // a1: widen fp16 and multiply by lambda*s (one rounding per element).
-    const uint4* seg = reinterpret_cast<const uint4*>(smem + (k & 1) * T::STAGE + rin * T::RS + sub * T::HS);
+    const uint8_t* st = smem + stage * T::STAGE;
     float2 p[NP];
 #pragma unroll
     for (int j = 0; j < NP / 8; ++j) {
-      const uint4 a = seg[j];                // channels 8j .. 8j+7
-      const uint4 b = seg[j + HALF / 8];     // channels HALF+8j .. HALF+8j+7
+      constexpr int QL = EPT / 64;               // quarters per lane
+      const int ea = 8 * j, eb = HALF + 8 * j;    // first channel of each chunk
+      const uint4 a = *reinterpret_cast<const uint4*>(st + tile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8));
+      const uint4 b = *reinterpret_cast<const uint4*>(st + tile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8));
       const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -338,6 +361,9 @@ kvq_quantize_kernel(const uint16_t* __restrict__ x, const float* __restrict__ la
         p[8 * j + 2 * t + 1] = __fmul2_rn(make_float2(fa.y, fb.y), make_float2(l.z, l.w));
       }
     }
+    __syncthreads();          // everyone has its inputs: the stage can be refilled
+    issue(tile + 2 * static_cast<int64_t>(tstride), stage);
+
     // a2, a3: transform, normalise.
     fwht_pairs<EPT, LANES>(p, sub);
 #pragma unroll
@@ -403,8 +429,6 @@ kvq_quantize_kernel(const uint16_t* __restrict__ x, const float* __restrict__ la
         if (sub % (G / EPT) == 0) srow[sub / (G / EPT)] = bx[0];
       }
     }
-    __syncthreads();          // everyone is done with stage k & 1
-    issue(k + 2);
   }
 }
 
@@ -415,47 +439,48 @@ template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 3)
 kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
                       const float* __restrict__ lam, const int8_t* __restrict__ sgn,
-                      int64_t n, float c, uint16_t* __restrict__ x_out) {
+                      int64_t n, float c, const __grid_constant__ RowMaps maps) {
   using T = Tile<D>;
   constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF, ROWS = T::ROWS;
   constexpr int PIN = T::PIN;
   constexpr int GX = (G < HALF) ? G : HALF;
   constexpr int NGH = HALF / GX;
   constexpr int HG = (G < NP) ? G : NP;          // butterfly stages h < HG stay inside a group
-  extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* stage_out = smem + 2 * PIN;
-  const float4* tab = reinterpret_cast<const float4*>(smem + 2 * PIN + T::STAGE);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 2 * PIN + T::STAGE + T::TAB);
+  constexpr int QL = EPT / 64;                   // quarters per lane
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_out = smem;                                  // one swizzled fp16 tile
+  uint8_t* stage_in = smem + T::STAGE;                        // two packed tiles
+  float4* tabw = reinterpret_cast<float4*>(smem + T::STAGE + 2 * PIN);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + T::STAGE + 2 * PIN + T::TAB);
   const int tid = threadIdx.x;
   const int sub = tid % LANES;
   const int rin = tid / LANES;
-  fill_tab<D>(reinterpret_cast<float4*>(smem + 2 * PIN + T::STAGE), lam, sgn, true);
+  fill_tab<D>(tabw, lam, sgn, true);
   if (tid == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   __syncthreads();
 
   const int64_t ntiles = (n + ROWS - 1) / ROWS;
-  auto issue = [&](int64_t k) {
-    const int64_t tile = blockIdx.x + k * gridDim.x;
+  const int tstride = gridDim.x;
+  auto issue = [&](int64_t tile, int stage) {
     if (tile >= ntiles || tid != 0) return;
     const int64_t row0 = tile * ROWS;
     const int valid = static_cast<int>(n - row0 < ROWS ? n - row0 : ROWS);
-    uint64_t* b = &bar[k & 1];
-    mbar_expect_tx(b, static_cast<uint32_t>(valid) * (D / 2));
-    bulk_g2s(smem + (k & 1) * PIN, packed + row0 * (D / 2), static_cast<uint32_t>(valid) * (D / 2), b);
+    mbar_expect_tx(&bar[stage], static_cast<uint32_t>(valid) * (D / 2));
+    bulk_g2s(stage_in + stage * PIN, packed + row0 * (D / 2), static_cast<uint32_t>(valid) * (D / 2), &bar[stage]);
   };
-  issue(0);
-  issue(1);
+  issue(blockIdx.x, 0);
+  issue(static_cast<int64_t>(blockIdx.x) + tstride, 1);
   const float2 c2 = make_float2(c, c);
-  const float4* mytab = tab + sub * (NP / 2);
+  const float4* mytab = tabw + sub * (NP / 2);
   const __half2 k1032 = __floats2half2_rn(1032.0f, 1032.0f);
   const __half2 k16th = __floats2half2_rn(0.0625f, 0.0625f);
   const __half2 km72 = __floats2half2_rn(-72.0f, -72.0f);
-  for (int64_t k = 0;; ++k) {
-    const int64_t tile = blockIdx.x + k * gridDim.x;
-    if (tile >= ntiles) break;
+  int64_t tile = blockIdx.x;
+  for (uint32_t k = 0; tile < ntiles; ++k, tile += tstride) {
+    const int stage = k & 1;
     const int64_t row = tile * ROWS + rin;
-    const bool active = row < n;
-    const int64_t rrow = active ? row : n - 1;
+    const int64_t rrow = row < n ? row : n - 1;
     const uint16_t* srow = scales + rrow * (D / G);
     uint16_t sx[NGH], sy[NGH];
     if constexpr (G <= HALF) {
@@ -468,16 +493,15 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
       sx[0] = srow[sub / (G / EPT)];
       sy[0] = sx[0];
     }
-    const bool ok = mbar_wait(&bar[k & 1], static_cast<uint32_t>((k >> 1) & 1), kSpinLimit);
+    const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);
     if (__syncthreads_or(!ok)) {
       if (tid == 0) atomicOr(&g_kvq_fault, 1u);
-      if (blockIdx.x + (k + 1) * gridDim.x < ntiles)
-        mbar_wait(&bar[(k + 1) & 1], static_cast<uint32_t>(((k + 1) >> 1) & 1), kSpinLimit);
-      bulk_wait0();
+      if (tile + tstride < ntiles) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
+      if (tid == 0) bulk_wait0();
       return;
     }
     // a8: the lane's EPT/2 bytes of codes; nibbles biased to n = q + 8.
-    const uint4* seg = reinterpret_cast<const uint4*>(smem + (k & 1) * PIN + rin * (D / 2) + sub * (EPT / 2));
+    const uint4* seg = reinterpret_cast<const uint4*>(stage_in + stage * PIN + rin * (D / 2) + sub * (EPT / 2));
     uint32_t w[EPT / 8];
 #pragma unroll
     for (int j = 0; j < EPT / 32; ++j) {
@@ -494,7 +518,6 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
     for (int kw = 0; kw < NP / 8; ++kw) {
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        // byte t of word kw to byte 0, byte t of word kw + HALF/8 to byte 2
         const uint32_t xb = __byte_perm(w[kw], w[kw + HALF / 8], 0x0400u | (t << 8) | t);
         const uint32_t lo = (xb & 0x000F000Fu) | 0x64006400u;
         const uint32_t hi = (xb & 0x00F000F0u) | 0x64006400u;
@@ -502,9 +525,7 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
         hq[8 * kw + 2 * t + 1] = __hfma2(*reinterpret_cast<const __half2*>(&hi), k16th, km72);
       }
     }
-    // a9 (first part): butterfly stages inside a group act on integers of
-    // magnitude <= 8 * 2^stage <= 512, exact in fp16; u = W * S is then exact
-    // in fp32 and equal, stage for stage, to the fp32 butterfly of q * S.
+    // a9 (first part): in-group stages on exact fp16 integers.
 #pragma unroll
     for (int h = 1; h < HG; h <<= 1) {
 #pragma unroll
@@ -524,9 +545,11 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
     // a9 (rest): the stages that cross groups, in fp32.
     fwht_pairs<EPT, LANES, HG>(p, sub);
 
-    // a10: normalise, s / lambda, fp16; stage the row and bulk-store it.
-    bulk_wait_read0();        // this lane's previous store has read its row
-    uint4* orow = reinterpret_cast<uint4*>(stage_out + rin * T::RS + sub * T::HS);
+    // a10: normalise, s / lambda, fp16 into the swizzled staging tile, which
+    // the tensor store of the previous tile must have finished reading.
+    if (tid == 0) bulk_wait_read0();
+    __syncthreads();          // staging tile free; everyone done with packed stage
+    issue(tile + 2 * static_cast<int64_t>(tstride), stage);
 #pragma unroll
     for (int j = 0; j < NP / 8; ++j) {
       uint32_t lo[4], hi[4];
@@ -538,18 +561,22 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
         lo[t] = float2_to_half2_bits(a.x, b.x);   // channels 8j+2t, +1
         hi[t] = float2_to_half2_bits(a.y, b.y);   // channels HALF+8j+2t, +1
       }
-      orow[j] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      orow[j + HALF / 8] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      const int ea = 8 * j, eb = HALF + 8 * j;
+      *reinterpret_cast<uint4*>(stage_out + tile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8)) =
+          make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(stage_out + tile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8)) =
+          make_uint4(hi[0], hi[1], hi[2], hi[3]);
     }
-    fence_proxy_async();
-    if (active) {
-      bulk_s2g(x_out + row * D + sub * EPT, orow, T::SEG);
+    fence_proxy_async();      // generic-proxy writes -> visible to the tensor store
+    __syncthreads();
+    if (tid == 0) {
+#pragma unroll
+      for (int q = 0; q < T::Q; ++q)
+        tensor_s2g(&maps.q[q], 0, static_cast<int>(tile * ROWS), stage_out + q * T::QB);
       bulk_commit();
     }
-    __syncthreads();          // everyone is done with packed stage k & 1
-    issue(k + 2);
   }
-  bulk_wait0();
+  if (tid == 0) bulk_wait0();
 }
 
 // A barrier that nothing completes, waited on with a short limit: exercises
@@ -604,6 +631,50 @@ int grid_for(Kernel k, int64_t n, int smem) {
   return static_cast<int>(need < cap ? need : cap);
 }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled, resolved once through the runtime (no libcuda link).
+EncodeTiledFn encode_tiled() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (f == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && p != nullptr) {
+      f = reinterpret_cast<EncodeTiledFn>(p);
+      fn.store(f, std::memory_order_release);
+    }
+  }
+  return f;
+}
+
+// One 2-D map per 64-channel quarter of the fp16 rows at `base`: 64 channels
+// x n rows, row stride 2D bytes, box 64 x ROWS, 128-byte swizzle.
+template <int D>
+int make_row_maps(RowMaps& m, const void* base, int64_t n) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return KVQ_ERR_LAUNCH;
+  for (int q = 0; q < D / 64; ++q) {
+    const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(n)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(2 * D)};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(Tile<D>::ROWS)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(&m.q[q], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+                           const_cast<char*>(static_cast<const char*>(base)) + 128 * q, dims, strides,
+                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+      g_last_cuda_error = static_cast<int>(r);
+      return KVQ_ERR_LAUNCH;
+    }
+  }
+  return KVQ_OK;
+}
+
 inline bool aligned(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }
@@ -611,7 +682,7 @@ inline bool aligned(const void* p, uintptr_t a) {
 int check_shape(int D, int G, int64_t n) {
   if (D != 64 && D != 128 && D != 256) return KVQ_ERR_DIM;
   if (G < 16 || G > D || (G & (G - 1)) != 0) return KVQ_ERR_GROUP;
-  if (n < 0) return KVQ_ERR_COUNT;
+  if (n < 0 || n > kMaxVectors) return KVQ_ERR_COUNT;
   return KVQ_OK;
 }
 
@@ -631,9 +702,12 @@ int launch_quantize(const uint16_t* x, const float* lam, const int8_t* s, int64_
                     uint8_t* packed, uint16_t* scales, cudaStream_t st) {
   auto k = kvq_quantize_kernel<D, G>;
   constexpr int smem = quantize_smem_bytes<D>();
+  RowMaps maps;
+  const int rc = make_row_maps<D>(maps, x, n);
+  if (rc != KVQ_OK) return rc;
   const int grid = grid_for<0, D, G>(k, n, smem);
   (void)cudaGetLastError();
-  k<<<grid, kThreads, smem, st>>>(x, lam, s, n, norm_const(D), packed, scales);
+  k<<<grid, kThreads, smem, st>>>(maps, lam, s, n, norm_const(D), packed, scales);
   return finish_launch();
 }
 
@@ -642,9 +716,12 @@ int launch_dequantize(const uint8_t* packed, const uint16_t* scales, const float
                       const int8_t* s, int64_t n, uint16_t* out, cudaStream_t st) {
   auto k = kvq_dequantize_kernel<D, G>;
   constexpr int smem = dequantize_smem_bytes<D>();
+  RowMaps maps;
+  const int rc = make_row_maps<D>(maps, out, n);
+  if (rc != KVQ_OK) return rc;
   const int grid = grid_for<1, D, G>(k, n, smem);
   (void)cudaGetLastError();
-  k<<<grid, kThreads, smem, st>>>(packed, scales, lam, s, n, norm_const(D), out);
+  k<<<grid, kThreads, smem, st>>>(packed, scales, lam, s, n, norm_const(D), maps);
   return finish_launch();
 }
 
@@ -732,7 +809,7 @@ const char* kvq_status_string(int status) {
     case KVQ_ERR_ALIGN: return "KVQ_ERR_ALIGN: a pointer is misaligned";
     case KVQ_ERR_DIM: return "KVQ_ERR_DIM: D must be 64, 128 or 256";
     case KVQ_ERR_GROUP: return "KVQ_ERR_GROUP: group must be a power of two in [16, D]";
-    case KVQ_ERR_COUNT: return "KVQ_ERR_COUNT: n_vec must be >= 0";
+    case KVQ_ERR_COUNT: return "KVQ_ERR_COUNT: n_vec must be in [0, 2^31 - 256]";
     case KVQ_ERR_LAUNCH: return "KVQ_ERR_LAUNCH: the kernel launch failed";
     default: return "unknown kvq status";
   }
@@ -740,6 +817,6 @@ const char* kvq_status_string(int status) {
 
 int kvq_last_cuda_error(void) { return g_last_cuda_error; }
 
-int kvq_version(void) { return (1 << 16) | 1; }
+int kvq_version(void) { return (1 << 16) | 2; }
 
 }  // extern "C"

@@ -58,7 +58,7 @@ A = 0x7F0000000000          # 256-byte aligned
 @pytest.mark.parametrize("D,G,n,want", [
     (96, 32, 10, -3), (32, 32, 10, -3), (512, 32, 10, -3),
     (128, 8, 10, -4), (128, 24, 10, -4), (128, 256, 10, -4), (64, 128, 10, -4),
-    (128, 32, -1, -5),
+    (128, 32, -1, -5), (128, 32, 1 << 31, -5), (64, 16, (1 << 40), -5),
 ])
 def test_shape_errors(kvq, D, G, n, want):
     assert kvq.kvq_quantize(A, A, A, n, D, G, A, A, 0) == want
