@@ -473,9 +473,7 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
   issue(static_cast<int64_t>(blockIdx.x) + tstride, 1);
   const float2 c2 = make_float2(c, c);
   const float4* mytab = tabw + sub * (NP / 2);
-  const __half2 k1032 = __floats2half2_rn(1032.0f, 1032.0f);
-  const __half2 k16th = __floats2half2_rn(0.0625f, 0.0625f);
-  const __half2 km72 = __floats2half2_rn(-72.0f, -72.0f);
+  const __half2 k1544 = __floats2half2_rn(1544.0f, 1544.0f);
   int64_t tile = blockIdx.x;
   for (uint32_t k = 0; tile < ntiles; ++k, tile += tstride) {
     const int stage = k & 1;
@@ -511,23 +509,48 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
       w[4 * j + 2] = a.z ^ 0x88888888u;
       w[4 * j + 3] = a.w ^ 0x88888888u;
     }
-    // Codes as exact fp16 integers in pairs hq[m] = (q[m], q[m+HALF]):
-    // (n | 0x6400) is the fp16 value 1024 + n, (16 n | 0x6400) is 1024 + 16 n.
-    __half2 hq[NP];
+    // Codes in pairs (q[m], q[m+HALF]) as two 16-bit integer lanes holding
+    // W + 0x6608, whose bit pattern is the fp16 encoding of the exact integer
+    // W + 1544 (|W| <= 512).  Unpack: biased nibble n = q + 8 in the low bits
+    // of 0x6600 gives 0x6600 + n = q + 0x6608.
+    uint32_t iq[NP];
 #pragma unroll
     for (int kw = 0; kw < NP / 8; ++kw) {
+      const uint32_t wa = w[kw], wb = w[kw + HALF / 8];
+      const uint32_t wa4 = wa >> 4, wb4 = wb >> 4;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const uint32_t xb = __byte_perm(w[kw], w[kw + HALF / 8], 0x0400u | (t << 8) | t);
-        const uint32_t lo = (xb & 0x000F000Fu) | 0x64006400u;
-        const uint32_t hi = (xb & 0x00F000F0u) | 0x64006400u;
-        hq[8 * kw + 2 * t] = __hsub2(*reinterpret_cast<const __half2*>(&lo), k1032);
-        hq[8 * kw + 2 * t + 1] = __hfma2(*reinterpret_cast<const __half2*>(&hi), k16th, km72);
+        const uint32_t sel = 0x0400u | (t << 8) | t;   // byte t of a -> byte 0, of b -> byte 2
+        iq[8 * kw + 2 * t] = (__byte_perm(wa, wb, sel) & 0x000F000Fu) | 0x66006600u;
+        iq[8 * kw + 2 * t + 1] = (__byte_perm(wa4, wb4, sel) & 0x000F000Fu) | 0x66006600u;
       }
     }
-    // a9 (first part): in-group stages on exact fp16 integers.
+    // a9 (first part): butterfly stages inside a group act on integers of
+    // magnitude <= 8 * 2^stage <= 512, so they are exact in any arithmetic.
+    // The first kIntStages run on the integer lanes (a + b - bias, a - b +
+    // bias in one 32-bit add for both lanes; each lane stays in [0, 65535],
+    // so nothing carries across), the rest in fp16x2 -- which splits the work
+    // between the integer and the FMA pipes.  u = W * S is then exact in fp32
+    // and equal, stage for stage, to the fp32 butterfly of q * S.
+    constexpr int kIntStages = 4;
+    constexpr uint32_t kBias2 = 0x66086608u;
+    constexpr int HI = (1 << kIntStages) < HG ? (1 << kIntStages) : HG;
 #pragma unroll
-    for (int h = 1; h < HG; h <<= 1) {
+    for (int h = 1; h < HI; h <<= 1) {
+#pragma unroll
+      for (int m = 0; m < NP; ++m) {
+        if ((m & h) == 0) {
+          const uint32_t a = iq[m], b = iq[m + h];
+          iq[m] = a + b - kBias2;
+          iq[m + h] = a - b + kBias2;
+        }
+      }
+    }
+    __half2 hq[NP];
+#pragma unroll
+    for (int m = 0; m < NP; ++m) hq[m] = __hsub2(*reinterpret_cast<const __half2*>(&iq[m]), k1544);
+#pragma unroll
+    for (int h = HI; h < HG; h <<= 1) {
 #pragma unroll
       for (int m = 0; m < NP; ++m) {
         if ((m & h) == 0) {
