@@ -291,6 +291,10 @@ def run_gpu(args):
     q_ms = max_over_ranks(q_ms, world, dev)
     d_ms = max_over_ranks(d_ms, world, dev)
 
+    extra = {}
+    if not args.no_extra:
+        extra = run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w)
+
     bpv = bytes_per_vector(D, G)
     total_vec = n * world
     value = total_vec * K / (elapsed_ms / 1e3) / 1e9
@@ -339,6 +343,7 @@ def run_gpu(args):
             "bytes_per_vector": bpv,
             "frac_of_8tbs": {"kvq_quantize": round(bpv * n / (q_ms / 1e3) / 1e9 / 8000, 4),
                              "kvq_dequantize": round(bpv * n / (d_ms / 1e3) / 1e9 / 8000, 4)},
+            **extra,
         },
         "roofline": {
             "kernel": top, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
@@ -352,6 +357,45 @@ def run_gpu(args):
         "cpu_baseline": cpu,
     }
     return line
+
+
+def _event_ms(torch, stream, fn, reps):
+    fn()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    ev[0].record(stream)
+    for i in range(reps):
+        fn()
+        ev[i + 1].record(stream)
+    torch.cuda.synchronize()
+    t = sorted(ev[i].elapsed_time(ev[i + 1]) for i in range(reps))
+    return t[len(t) // 2]
+
+
+def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w):
+    """Secondary figures, outside the timed steps: the fused round trip on the
+    same batch, and the decode-time append of one new K and V token for 64
+    sequences x 36 layers x 8 KV heads into their rows of a cache."""
+    n, D = x.shape
+    rt_ms = _event_ms(torch, stream,
+                      lambda: kvq.roundtrip(x, lam_t, s_t, G, out=out, stream=stream), 10)
+    a = workloads.WORKLOADS["decode-append"]
+    na = a.n_vec
+    T = 64                                        # cache slots per (sequence, layer, head)
+    xa = workloads.device_rows(a, na, dev)
+    idx = torch.arange(na, device=dev, dtype=torch.int64) * T + (T - 1)
+    cpk = torch.empty((na * T, D // 2), dtype=torch.uint8, device=dev)
+    csc = torch.empty((na * T, D // G), dtype=torch.float16, device=dev)
+    ap_ms = _event_ms(torch, stream, lambda: kvq.quantize_rows(
+        xa, lam_t, s_t, G, idx, cpk, csc, stream=stream), 50)
+    del xa, cpk, csc
+    return {
+        "roundtrip_ms": round(rt_ms, 5),
+        "roundtrip_gbs": round(n * 4 * D / (rt_ms / 1e3) / 1e9, 1),
+        "decode_append_vectors": na,
+        "decode_append_us": round(ap_ms * 1e3, 2),
+        "decode_append_gvec_s": round(na / (ap_ms / 1e3) / 1e9, 3),
+    }
 
 
 def run_e2e(args, torch, kvq, dev, x_dev, lam_t, s_t, G, world):
@@ -453,6 +497,7 @@ def parse(argv=None):
     p.add_argument("--n-vec", type=int, default=None, help="override vectors per GPU (profiling)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--no-extra", action="store_true", help="skip round-trip and append figures")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--e2e-chunks", type=int, default=16)
     p.add_argument("--cpu-seconds", type=float, default=10.0)

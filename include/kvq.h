@@ -98,6 +98,24 @@ int kvq_quantize(const uint16_t *x, const float *lambda, const int8_t *signs,
                  uint8_t *packed, uint16_t *scales, void *stream);
 
 /*
+ * kvq_quantize_rows -- kvq_quantize with a row map: vector r of x is encoded
+ * into row row_idx[r] of packed / scales, whose rows 0 .. cache_rows-1
+ * belong to the caller (e.g. one new token per sequence appended into its
+ * slot of a decode cache).  Rows not named in row_idx are left untouched.
+ *
+ *   row_idx     [in] int64 [n_vec], device memory, 8-byte aligned.  An index
+ *               outside [0, cache_rows) is skipped (nothing is written for
+ *               that vector) and sets bit 2 of the fault word.  Two vectors
+ *               with the same index race; either result may remain.
+ *   cache_rows  number of rows of packed / scales (>= 0).
+ *   Other arguments as for kvq_quantize.
+ */
+int kvq_quantize_rows(const uint16_t *x, const float *lambda, const int8_t *signs,
+                      int64_t n_vec, int D, int group,
+                      const int64_t *row_idx, int64_t cache_rows,
+                      uint8_t *packed, uint16_t *scales, void *stream);
+
+/*
  * kvq_dequantize -- unpack, rescale, inverse-rotate and un-scale n_vec
  * vectors.  Same layouts and conventions as kvq_quantize.
  *
@@ -114,10 +132,25 @@ int kvq_dequantize(const uint8_t *packed, const uint16_t *scales,
                    uint16_t *x_out, void *stream);
 
 /*
+ * kvq_roundtrip -- x_hat = kvq_dequantize(kvq_quantize(x)) in one pass over
+ * x (the quantise-then-dequantise shape used to simulate the cache's error
+ * on the fly), bit-identical to the two calls back to back.
+ *
+ *   x, lambda, signs, n_vec, D, group: as for kvq_quantize.
+ *   x_hat   [out] fp16 bits [n_vec][D]; 16-byte aligned; must not overlap x.
+ *   packed, scales [out, optional] the codes and scales as kvq_quantize
+ *                  writes them; pass both or neither (NULL).
+ */
+int kvq_roundtrip(const uint16_t *x, const float *lambda, const int8_t *signs,
+                  int64_t n_vec, int D, int group, uint16_t *x_hat,
+                  uint8_t *packed, uint16_t *scales, void *stream);
+
+/*
  * kvq_fault_status -- the current device's fault word: 0 when every bounded
  * wait of every kernel so far completed; bit 0 set when a quantize or
  * dequantize block gave up waiting for its bulk copies (its outputs are then
- * incomplete); bit 1 set by kvq_selftest_wait_timeout.  Non-zero `clear`
+ * incomplete); bit 1 set by kvq_selftest_wait_timeout; bit 2 set when
+ * kvq_quantize_rows skipped an out-of-range row index.  Non-zero `clear`
  * resets the word.  Synchronous (it copies the word to the host, which waits
  * for prior work on the device's legacy default stream).  Returns -1 if the
  * word cannot be read.

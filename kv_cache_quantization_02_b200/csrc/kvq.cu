@@ -99,6 +99,8 @@ struct RowMaps {
 template <int D>
 constexpr int quantize_smem_bytes() { return 1024 + 2 * Tile<D>::STAGE + Tile<D>::TAB + 16; }
 template <int D>
+constexpr int roundtrip_smem_bytes() { return 1024 + 3 * Tile<D>::STAGE + 2 * Tile<D>::TAB + 16; }
+template <int D>
 constexpr int dequantize_smem_bytes() { return 1024 + Tile<D>::STAGE + 2 * Tile<D>::PIN + Tile<D>::TAB + 16; }
 
 // ---------------------------------------------------------------------------
@@ -296,11 +298,12 @@ __device__ __forceinline__ void fill_tab(float4* tab, const float* __restrict__ 
 // ---------------------------------------------------------------------------
 // Quantize: fp16 [n][D] -> packed u8 [n][D/2] + fp16 scales [n][D/G].
 // ---------------------------------------------------------------------------
-template <int D, int G>
+template <int D, int G, bool INDEXED>
 __global__ void __launch_bounds__(kThreads, 3)
 kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restrict__ lam,
                     const int8_t* __restrict__ sgn, int64_t n, float c,
-                    uint8_t* __restrict__ packed, uint16_t* __restrict__ scales) {
+                    uint8_t* __restrict__ packed, uint16_t* __restrict__ scales,
+                    const int64_t* __restrict__ row_idx, int64_t cache_rows) {
   using T = Tile<D>;
   constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF, ROWS = T::ROWS;
   constexpr int GX = (G < HALF) ? G : HALF;      // pairs spanned by one group (G <= HALF)
@@ -340,7 +343,15 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
       return;
     }
     const int64_t row = tile * ROWS + rin;
-    const bool active = row < n;
+    bool active = row < n;
+    int64_t orow = row;                          // destination row of the codes
+    if constexpr (INDEXED) {
+      orow = active ? row_idx[row] : 0;
+      if (active && (orow < 0 || orow >= cache_rows)) {
+        atomicOr(&g_kvq_fault, 4u);              // out-of-range index: skipped
+        active = false;
+      }
+    }
 
     // a1: widen fp16 and multiply by lambda*s (one rounding per element).
     const uint8_t* st = smem + stage * T::STAGE;
@@ -412,13 +423,13 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
       out[k8 + NP / 8] = pack8(qb);
     }
     if (active) {
-      uint8_t* dst = packed + row * (D / 2) + sub * (EPT / 2);
+      uint8_t* dst = packed + orow * (D / 2) + sub * (EPT / 2);
 #pragma unroll
       for (int k4 = 0; k4 < EPT / 32; ++k4) {
         const uint32_t t4[4] = {out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]};
         st_v4(dst + 16 * k4, t4);
       }
-      uint16_t* srow = scales + row * (D / G);
+      uint16_t* srow = scales + orow * (D / G);
       if constexpr (G <= HALF) {
 #pragma unroll
         for (int j = 0; j < NGH; ++j) {
@@ -602,6 +613,177 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
   if (tid == 0) bulk_wait0();
 }
 
+
+// ---------------------------------------------------------------------------
+// Round trip: fp16 [n][D] -> x_hat = dequantize(quantize(x)) fp16 [n][D], and
+// optionally the codes and scales, in one pass (the quantise-then-dequantise
+// shape used to simulate the cache's error).  Same arithmetic as the two
+// kernels back to back: u = q * S is exact, then the same butterfly order.
+// ---------------------------------------------------------------------------
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads, 2)
+kvq_roundtrip_kernel(const __grid_constant__ RowMaps in_maps, const __grid_constant__ RowMaps out_maps,
+                     const float* __restrict__ lam, const int8_t* __restrict__ sgn, int64_t n,
+                     float c, uint8_t* __restrict__ packed, uint16_t* __restrict__ scales) {
+  using T = Tile<D>;
+  constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF, ROWS = T::ROWS;
+  constexpr int GX = (G < HALF) ? G : HALF;
+  constexpr int NGH = HALF / GX;
+  constexpr int QL = EPT / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_out = smem + 2 * T::STAGE;
+  float4* tab_q = reinterpret_cast<float4*>(smem + 3 * T::STAGE);
+  float4* tab_d = reinterpret_cast<float4*>(smem + 3 * T::STAGE + T::TAB);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 3 * T::STAGE + 2 * T::TAB);
+  const int tid = threadIdx.x;
+  const int sub = tid % LANES;
+  const int rin = tid / LANES;
+  fill_tab<D>(tab_q, lam, sgn, false);
+  fill_tab<D>(tab_d, lam, sgn, true);
+  if (tid == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
+  __syncthreads();
+
+  const int64_t ntiles = (n + ROWS - 1) / ROWS;
+  const int tstride = gridDim.x;
+  auto issue = [&](int64_t tile, int stage) {
+    if (tile >= ntiles || tid != 0) return;
+    mbar_expect_tx(&bar[stage], T::STAGE);
+#pragma unroll
+    for (int q = 0; q < T::Q; ++q)
+      tensor_g2s(smem + stage * T::STAGE + q * T::QB, &in_maps.q[q], 0, static_cast<int>(tile * ROWS), &bar[stage]);
+  };
+  issue(blockIdx.x, 0);
+  issue(static_cast<int64_t>(blockIdx.x) + tstride, 1);
+  const float2 c2 = make_float2(c, c);
+  const float4* tq = tab_q + sub * (NP / 2);
+  const float4* td = tab_d + sub * (NP / 2);
+  int64_t tile = blockIdx.x;
+  for (uint32_t k = 0; tile < ntiles; ++k, tile += tstride) {
+    const int stage = k & 1;
+    const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);
+    if (__syncthreads_or(!ok)) {
+      if (tid == 0) atomicOr(&g_kvq_fault, 1u);
+      if (tile + tstride < ntiles) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
+      if (tid == 0) bulk_wait0();
+      return;
+    }
+    const int64_t row = tile * ROWS + rin;
+    const bool active = row < n;
+    const uint8_t* st = smem + stage * T::STAGE;
+    float2 p[NP];
+#pragma unroll
+    for (int j = 0; j < NP / 8; ++j) {
+      const int ea = 8 * j, eb = HALF + 8 * j;
+      const uint4 a = *reinterpret_cast<const uint4*>(st + tile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8));
+      const uint4 b = *reinterpret_cast<const uint4*>(st + tile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8));
+      const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float2 fa = half2_bits_to_float2(aw[t]);
+        const float2 fb = half2_bits_to_float2(bw[t]);
+        const float4 l = tq[4 * j + t];
+        p[8 * j + 2 * t] = __fmul2_rn(make_float2(fa.x, fb.x), make_float2(l.x, l.y));
+        p[8 * j + 2 * t + 1] = __fmul2_rn(make_float2(fa.y, fb.y), make_float2(l.z, l.w));
+      }
+    }
+    __syncthreads();
+    issue(tile + 2 * static_cast<int64_t>(tstride), stage);
+    fwht_pairs<EPT, LANES>(p, sub);
+#pragma unroll
+    for (int m = 0; m < NP; ++m) p[m] = __fmul2_rn(p[m], c2);
+    float rx[NGH], ry[NGH];
+    uint16_t bx[NGH], by[NGH];
+    if constexpr (G <= HALF) {
+#pragma unroll
+      for (int j = 0; j < NGH; ++j) {
+        float ax = 0.f, ay = 0.f;
+#pragma unroll
+        for (int m = 0; m < GX; m += 2) {
+          ax = amax3(ax, p[j * GX + m].x, p[j * GX + m + 1].x);
+          ay = amax3(ay, p[j * GX + m].y, p[j * GX + m + 1].y);
+        }
+        bx[j] = group_scale(ax, rx[j]);
+        by[j] = group_scale(ay, ry[j]);
+      }
+    } else {
+      float a = 0.f;
+#pragma unroll
+      for (int m = 0; m < NP; ++m) a = amax3(a, p[m].x, p[m].y);
+#pragma unroll
+      for (int bit = 1; bit < G / EPT; bit <<= 1) a = fmaxf(a, __shfl_xor_sync(kFullMask, a, bit));
+      bx[0] = group_scale(a, rx[0]);
+      ry[0] = rx[0];
+      by[0] = bx[0];
+    }
+    // codes (saturated to [-8, 7]), then u = q * S, exact in fp32
+    uint32_t out[EPT / 8];
+#pragma unroll
+    for (int k8 = 0; k8 < NP / 8; ++k8) {
+      int qa[8], qb[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int m = 8 * k8 + t;
+        const float2 v = __fmul2_rn(p[m], make_float2(rx[m / GX], ry[m / GX]));
+        qa[t] = min(max(__float2int_rn(v.x), -8), 7);
+        qb[t] = min(max(__float2int_rn(v.y), -8), 7);
+        p[m] = __fmul2_rn(make_float2(__int2float_rn(qa[t]), __int2float_rn(qb[t])),
+                          make_float2(half_bits_to_float(bx[m / GX]), half_bits_to_float(by[m / GX])));
+      }
+      out[k8] = pack8(qa);
+      out[k8 + NP / 8] = pack8(qb);
+    }
+    if (active && packed != nullptr) {
+      uint8_t* dst = packed + row * (D / 2) + sub * (EPT / 2);
+#pragma unroll
+      for (int k4 = 0; k4 < EPT / 32; ++k4) {
+        const uint32_t t4[4] = {out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]};
+        st_v4(dst + 16 * k4, t4);
+      }
+      uint16_t* srow = scales + row * (D / G);
+      if constexpr (G <= HALF) {
+#pragma unroll
+        for (int j = 0; j < NGH; ++j) {
+          srow[sub * (EPT / G) + j] = bx[j];
+          srow[sub * (EPT / G) + NGH + j] = by[j];
+        }
+      } else {
+        if (sub % (G / EPT) == 0) srow[sub / (G / EPT)] = bx[0];
+      }
+    }
+    // inverse: the same butterfly, normalise, s / lambda, fp16
+    fwht_pairs<EPT, LANES>(p, sub);
+    if (tid == 0) bulk_wait_read0();
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < NP / 8; ++j) {
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float4 l = td[4 * j + t];
+        const float2 a = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t], c2), make_float2(l.x, l.y));
+        const float2 b = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t + 1], c2), make_float2(l.z, l.w));
+        lo[t] = float2_to_half2_bits(a.x, b.x);
+        hi[t] = float2_to_half2_bits(a.y, b.y);
+      }
+      const int ea = 8 * j, eb = HALF + 8 * j;
+      *reinterpret_cast<uint4*>(stage_out + tile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8)) =
+          make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(stage_out + tile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8)) =
+          make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    }
+    fence_proxy_async();
+    __syncthreads();
+    if (tid == 0) {
+#pragma unroll
+      for (int q = 0; q < T::Q; ++q)
+        tensor_s2g(&out_maps.q[q], 0, static_cast<int>(tile * ROWS), stage_out + q * T::QB);
+      bulk_commit();
+    }
+  }
+  if (tid == 0) bulk_wait0();
+}
+
 // A barrier that nothing completes, waited on with a short limit: exercises
 // the bounded-wait give-up path (fault word) without any real copy.
 __global__ void kvq_wait_timeout_kernel(uint32_t limit) {
@@ -720,18 +902,32 @@ int finish_launch() {
   return KVQ_OK;
 }
 
-template <int D, int G>
-int launch_quantize(const uint16_t* x, const float* lam, const int8_t* s, int64_t n,
-                    uint8_t* packed, uint16_t* scales, cudaStream_t st) {
-  auto k = kvq_quantize_kernel<D, G>;
+template <int D, int G, bool INDEXED>
+int launch_quantize_t(const uint16_t* x, const float* lam, const int8_t* s, int64_t n,
+                      uint8_t* packed, uint16_t* scales, const int64_t* row_idx,
+                      int64_t cache_rows, cudaStream_t st) {
+  auto k = kvq_quantize_kernel<D, G, INDEXED>;
   constexpr int smem = quantize_smem_bytes<D>();
   RowMaps maps;
   const int rc = make_row_maps<D>(maps, x, n);
   if (rc != KVQ_OK) return rc;
-  const int grid = grid_for<0, D, G>(k, n, smem);
+  const int grid = grid_for<INDEXED ? 2 : 0, D, G>(k, n, smem);
   (void)cudaGetLastError();
-  k<<<grid, kThreads, smem, st>>>(maps, lam, s, n, norm_const(D), packed, scales);
+  k<<<grid, kThreads, smem, st>>>(maps, lam, s, n, norm_const(D), packed, scales, row_idx, cache_rows);
   return finish_launch();
+}
+
+template <int D, int G>
+int launch_quantize(const uint16_t* x, const float* lam, const int8_t* s, int64_t n,
+                    uint8_t* packed, uint16_t* scales, cudaStream_t st) {
+  return launch_quantize_t<D, G, false>(x, lam, s, n, packed, scales, nullptr, n, st);
+}
+
+template <int D, int G>
+int launch_quantize_rows(const uint16_t* x, const float* lam, const int8_t* s, int64_t n,
+                         uint8_t* packed, uint16_t* scales, const int64_t* row_idx,
+                         int64_t cache_rows, cudaStream_t st) {
+  return launch_quantize_t<D, G, true>(x, lam, s, n, packed, scales, row_idx, cache_rows, st);
 }
 
 template <int D, int G>
@@ -745,6 +941,21 @@ int launch_dequantize(const uint8_t* packed, const uint16_t* scales, const float
   const int grid = grid_for<1, D, G>(k, n, smem);
   (void)cudaGetLastError();
   k<<<grid, kThreads, smem, st>>>(packed, scales, lam, s, n, norm_const(D), maps);
+  return finish_launch();
+}
+
+template <int D, int G>
+int launch_roundtrip(const uint16_t* x, const float* lam, const int8_t* s, int64_t n,
+                     uint16_t* x_hat, uint8_t* packed, uint16_t* scales, cudaStream_t st) {
+  auto k = kvq_roundtrip_kernel<D, G>;
+  constexpr int smem = roundtrip_smem_bytes<D>();
+  RowMaps in_maps, out_maps;
+  int rc = make_row_maps<D>(in_maps, x, n);
+  if (rc == KVQ_OK) rc = make_row_maps<D>(out_maps, x_hat, n);
+  if (rc != KVQ_OK) return rc;
+  const int grid = grid_for<3, D, G>(k, n, smem);
+  (void)cudaGetLastError();
+  k<<<grid, kThreads, smem, st>>>(in_maps, out_maps, lam, s, n, norm_const(D), packed, scales);
   return finish_launch();
 }
 
@@ -796,6 +1007,22 @@ int kvq_quantize(const uint16_t* x, const float* lambda, const int8_t* signs,
   KVQ_DISPATCH(launch_quantize, D, group, x, lambda, signs, n_vec, packed, scales, st);
 }
 
+int kvq_quantize_rows(const uint16_t* x, const float* lambda, const int8_t* signs,
+                      int64_t n_vec, int D, int group, const int64_t* row_idx,
+                      int64_t cache_rows, uint8_t* packed, uint16_t* scales, void* stream) {
+  const int rc = check_shape(D, group, n_vec);
+  if (rc != KVQ_OK) return rc;
+  if (cache_rows < 0) return KVQ_ERR_COUNT;
+  if (n_vec == 0) return KVQ_OK;
+  if (!x || !lambda || !signs || !row_idx || !packed || !scales) return KVQ_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(packed, 16) || !aligned(scales, 2) || !aligned(lambda, 4) ||
+      !aligned(row_idx, 8))
+    return KVQ_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  KVQ_DISPATCH(launch_quantize_rows, D, group, x, lambda, signs, n_vec, packed, scales, row_idx,
+               cache_rows, st);
+}
+
 int kvq_dequantize(const uint8_t* packed, const uint16_t* scales, const float* lambda,
                    const int8_t* signs, int64_t n_vec, int D, int group, uint16_t* x_out,
                    void* stream) {
@@ -807,6 +1034,21 @@ int kvq_dequantize(const uint8_t* packed, const uint16_t* scales, const float* l
     return KVQ_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   KVQ_DISPATCH(launch_dequantize, D, group, packed, scales, lambda, signs, n_vec, x_out, st);
+}
+
+int kvq_roundtrip(const uint16_t* x, const float* lambda, const int8_t* signs, int64_t n_vec,
+                  int D, int group, uint16_t* x_hat, uint8_t* packed, uint16_t* scales,
+                  void* stream) {
+  const int rc = check_shape(D, group, n_vec);
+  if (rc != KVQ_OK) return rc;
+  if (n_vec == 0) return KVQ_OK;
+  if (!x || !lambda || !signs || !x_hat) return KVQ_ERR_NULL;
+  if ((packed == nullptr) != (scales == nullptr)) return KVQ_ERR_NULL;
+  if (!aligned(x, 16) || !aligned(x_hat, 16) || !aligned(lambda, 4) ||
+      (packed && (!aligned(packed, 16) || !aligned(scales, 2))))
+    return KVQ_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  KVQ_DISPATCH(launch_roundtrip, D, group, x, lambda, signs, n_vec, x_hat, packed, scales, st);
 }
 
 int kvq_fault_status(int clear) {

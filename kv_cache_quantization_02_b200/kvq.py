@@ -33,6 +33,10 @@ _I = ctypes.c_int
 
 _lib.kvq_quantize.restype = _I
 _lib.kvq_quantize.argtypes = [_P, _P, _P, _I64, _I, _I, _P, _P, _P]
+_lib.kvq_quantize_rows.restype = _I
+_lib.kvq_quantize_rows.argtypes = [_P, _P, _P, _I64, _I, _I, _P, _I64, _P, _P, _P]
+_lib.kvq_roundtrip.restype = _I
+_lib.kvq_roundtrip.argtypes = [_P, _P, _P, _I64, _I, _I, _P, _P, _P, _P]
 _lib.kvq_dequantize.restype = _I
 _lib.kvq_dequantize.argtypes = [_P, _P, _P, _P, _I64, _I, _I, _P, _P]
 _lib.kvq_status_string.restype = ctypes.c_char_p
@@ -69,6 +73,18 @@ class KvqError(RuntimeError):
 def kvq_quantize(x: int, lam: int, signs: int, n_vec: int, D: int, group: int,
                  packed: int, scales: int, stream: int = 0) -> int:
     return _lib.kvq_quantize(x, lam, signs, n_vec, D, group, packed, scales, stream)
+
+
+def kvq_quantize_rows(x: int, lam: int, signs: int, n_vec: int, D: int, group: int,
+                      row_idx: int, cache_rows: int, packed: int, scales: int,
+                      stream: int = 0) -> int:
+    return _lib.kvq_quantize_rows(x, lam, signs, n_vec, D, group, row_idx, cache_rows,
+                                  packed, scales, stream)
+
+
+def kvq_roundtrip(x: int, lam: int, signs: int, n_vec: int, D: int, group: int,
+                  x_hat: int, packed: int = 0, scales: int = 0, stream: int = 0) -> int:
+    return _lib.kvq_roundtrip(x, lam, signs, n_vec, D, group, x_hat, packed, scales, stream)
 
 
 def kvq_dequantize(packed: int, scales: int, lam: int, signs: int, n_vec: int,
@@ -136,6 +152,56 @@ def quantize(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: int
     if rc != KVQ_OK:
         raise KvqError(rc)
     return packed, scales
+
+
+def quantize_rows(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: int,
+                  row_idx: torch.Tensor, packed: torch.Tensor, scales: torch.Tensor,
+                  stream=None):
+    """Encode x: fp16 [n, D] into rows row_idx (int64 [n]) of the cache
+    (packed uint8 [N, D/2], scales fp16 [N, D/group]); other rows untouched."""
+    if x.dim() != 2:
+        raise ValueError("x must be [n_vec, D]")
+    n, D = x.shape
+    _need(x, torch.float16, (n, D), "x")
+    _need(lam, torch.float32, (D,), "lambda")
+    _need(signs, torch.int8, (D,), "signs")
+    _need(row_idx, torch.int64, (n,), "row_idx")
+    N = packed.shape[0]
+    _need(packed, torch.uint8, (N, D // 2), "packed")
+    _need(scales, torch.float16, (N, max(D // group, 1)), "scales")
+    rc = kvq_quantize_rows(x.data_ptr(), lam.data_ptr(), signs.data_ptr(), n, D, group,
+                           row_idx.data_ptr(), N, packed.data_ptr(), scales.data_ptr(),
+                           _stream_handle(stream))
+    if rc != KVQ_OK:
+        raise KvqError(rc)
+    return packed, scales
+
+
+def roundtrip(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: int,
+              out: torch.Tensor | None = None, packed: torch.Tensor | None = None,
+              scales: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """x_hat = dequantize(quantize(x)) in one kernel; codes/scales optional."""
+    if x.dim() != 2:
+        raise ValueError("x must be [n_vec, D]")
+    n, D = x.shape
+    _need(x, torch.float16, (n, D), "x")
+    _need(lam, torch.float32, (D,), "lambda")
+    _need(signs, torch.int8, (D,), "signs")
+    if out is None:
+        out = torch.empty((n, D), dtype=torch.float16, device=x.device)
+    _need(out, torch.float16, (n, D), "out")
+    if (packed is None) != (scales is None):
+        raise ValueError("pass both packed and scales, or neither")
+    pk = sc = 0
+    if packed is not None:
+        _need(packed, torch.uint8, (n, D // 2), "packed")
+        _need(scales, torch.float16, (n, max(D // group, 1)), "scales")
+        pk, sc = packed.data_ptr(), scales.data_ptr()
+    rc = kvq_roundtrip(x.data_ptr(), lam.data_ptr(), signs.data_ptr(), n, D, group,
+                       out.data_ptr(), pk, sc, _stream_handle(stream))
+    if rc != KVQ_OK:
+        raise KvqError(rc)
+    return out
 
 
 def dequantize(packed: torch.Tensor, scales: torch.Tensor, lam: torch.Tensor,

@@ -103,3 +103,19 @@ def test_binding_fails_loudly_without_the_library(tmp_path):
     mod = importlib.util.module_from_spec(spec)
     with pytest.raises(ImportError):
         spec.loader.exec_module(mod)
+
+
+def test_quantize_rows_errors(kvq):
+    assert kvq.kvq_quantize_rows(A, A, A, 4, 128, 32, 0, 100, A, A, 0) == -1     # row_idx NULL
+    assert kvq.kvq_quantize_rows(A, A, A, 4, 128, 32, A + 4, 100, A, A, 0) == -2  # row_idx needs 8
+    assert kvq.kvq_quantize_rows(A, A, A, 4, 128, 32, A, -1, A, A, 0) == -5       # cache_rows < 0
+    assert kvq.kvq_quantize_rows(A, A, A, 4, 96, 32, A, 100, A, A, 0) == -3
+    assert kvq.kvq_quantize_rows(0, 0, 0, 0, 128, 32, 0, 0, 0, 0, 0) == 0
+
+
+def test_roundtrip_errors(kvq):
+    assert kvq.kvq_roundtrip(A, A, A, 4, 128, 32, 0, 0, 0, 0) == -1       # x_hat NULL
+    assert kvq.kvq_roundtrip(A, A, A, 4, 128, 32, A, A, 0, 0) == -1       # packed without scales
+    assert kvq.kvq_roundtrip(A, A, A, 4, 128, 32, A + 8, 0, 0, 0) == -2   # x_hat needs 16
+    assert kvq.kvq_roundtrip(A, A, A, 4, 128, 8, A, 0, 0, 0) == -4
+    assert kvq.kvq_roundtrip(0, 0, 0, 0, 128, 32, 0, 0, 0, 0) == 0
