@@ -81,6 +81,8 @@ class Oracle:
             "kvqo_dequantize_f32": (_I, [_P, _P, _P, _P, _I64, _I, _I, _P]),
             "kvqo_pack": (None, [_P, _I64, _P]),
             "kvqo_unpack": (None, [_P, _I64, _P]),
+            "kvqo_attention_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                           _I, _I, _I, _I, _I, _I, ctypes.c_double, _P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -205,6 +207,34 @@ class Oracle:
         packed = np.ascontiguousarray(packed, dtype=np.uint8)
         out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), dtype=np.int8)
         self._lib.kvqo_unpack(_ptr(packed), packed.size * 2, _ptr(out))
+        return out
+
+
+    def attention_decode(self, q, k_packed, k_scales, v_packed, v_scales, seq_len,
+                         lam_k, s_k, lam_v, s_v, group: int, sm_scale: float) -> np.ndarray:
+        """Decode attention over the int4 cache, float64 [B, Hq, D].
+
+        q fp16 [B, Hq, D]; packed u8 [B, Hkv, T, D/2]; scales fp16
+        [B, Hkv, T, D/group]; seq_len int [B]."""
+        q = np.ascontiguousarray(q)
+        if q.dtype != np.float16 or q.ndim != 3:
+            raise TypeError("q must be float16 [B, Hq, D]")
+        B, Hq, D = q.shape
+        kp = np.ascontiguousarray(k_packed, dtype=np.uint8)
+        vp = np.ascontiguousarray(v_packed, dtype=np.uint8)
+        ks = np.ascontiguousarray(k_scales).view(np.uint16)
+        vs = np.ascontiguousarray(v_scales).view(np.uint16)
+        if kp.ndim != 4 or kp.shape[0] != B or kp.shape[3] * 2 != D or vp.shape != kp.shape:
+            raise ValueError("packed caches must be [B, Hkv, T, D/2]")
+        Hkv, T = kp.shape[1], kp.shape[2]
+        sl = np.ascontiguousarray(seq_len, dtype=np.int32)
+        lk, sk = _params(lam_k, s_k)
+        lv, sv = _params(lam_v, s_v)
+        out = np.empty((B, Hq, D), dtype=np.float64)
+        _check(self._lib.kvqo_attention_decode(
+            _ptr(q.view(np.uint16)), _ptr(kp), _ptr(ks), _ptr(vp), _ptr(vs), _ptr(sl),
+            _ptr(lk), _ptr(sk), _ptr(lv), _ptr(sv), B, Hq, Hkv, T, D, group,
+            float(sm_scale), _ptr(out)))
         return out
 
 

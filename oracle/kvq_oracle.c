@@ -50,6 +50,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #define KVQO_DMAX 4096
@@ -370,5 +371,94 @@ int kvqo_quantize_codes_divform(const uint16_t *x, const float *lam,
             }
         }
     }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Decode attention over the int4 cache: one query token per sequence.  */
+/* [P1] "Fused group-affine (KIVI-style) attention": the quantised K    */
+/* and V are reconstructed and attended with a numerically stable       */
+/* softmax in place of a dequantize -> memory -> SDPA round trip.  This */
+/* is the plain definition the fused kernel has to reproduce, in double */
+/* precision and without rounding the reconstructed rows to fp16:       */
+/*   K_t = (diag(s_K) H (codes_t . S_t) / sqrt(D)) / lambda_K, V_t      */
+/*   likewise with (lambda_V, s_V);                                     */
+/*   z_t = sm_scale <q, K_t>;  p = softmax(z) over t < len;             */
+/*   o = sum_t p_t V_t.                                                 */
+/* Query head h reads KV head h / (Hq / Hkv) (grouped-query attention). */
+/* An empty context (len = 0) gives o = 0.                               */
+/* Layouts: q fp16 [B][Hq][D]; packed u8 [B][Hkv][T][D/2]; scales fp16  */
+/* [B][Hkv][T][D/G]; seq_len [B]; out double [B][Hq][D].                */
+/* ------------------------------------------------------------------ */
+
+/* One reconstructed row in double: codes times scales, then the exact   */
+/* inverse rotation.                                                     */
+static void reconstruct_row_f64(const uint8_t *packed, const uint16_t *scales,
+                                const double *lam, const int8_t *s, int D,
+                                int G, double *x)
+{
+    int8_t q[KVQO_DMAX];
+    double y[KVQO_DMAX];
+    kvqo_unpack(packed, D, q);
+    for (int i = 0; i < D; ++i)
+        y[i] = (double)q[i] * (double)kvqo_f16_to_f32(scales[i / G]);
+    kvqo_unrotate_f64(y, lam, s, D, x);
+}
+
+int kvqo_attention_decode(const uint16_t *q, const uint8_t *k_packed,
+                          const uint16_t *k_scales, const uint8_t *v_packed,
+                          const uint16_t *v_scales, const int32_t *seq_len,
+                          const float *lam_k, const int8_t *s_k,
+                          const float *lam_v, const int8_t *s_v, int B, int Hq,
+                          int Hkv, int T, int D, int G, double sm_scale,
+                          double *out)
+{
+    int rc = check_shape(D, G);
+    if (rc) return rc;
+    if (B < 0 || T < 0 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0) return -5;
+    for (int b = 0; b < B; ++b)
+        if (seq_len[b] < 0 || seq_len[b] > T) return -5;
+    int R = Hq / Hkv;
+    double lk[KVQO_DMAX], lv[KVQO_DMAX], qd[KVQO_DMAX], row[KVQO_DMAX];
+    for (int i = 0; i < D; ++i) {
+        lk[i] = (double)lam_k[i];
+        lv[i] = (double)lam_v[i];
+    }
+    double *z = (double *)malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    if (z == NULL) return -6;
+    for (int b = 0; b < B; ++b) {
+        int len = seq_len[b];
+        for (int h = 0; h < Hq; ++h) {
+            int kv = h / R;
+            int64_t base = ((int64_t)b * Hkv + kv) * T;
+            double *o = out + ((int64_t)b * Hq + h) * D;
+            for (int i = 0; i < D; ++i) {
+                qd[i] = (double)kvqo_f16_to_f32(q[((int64_t)b * Hq + h) * D + i]);
+                o[i] = 0.0;
+            }
+            if (len == 0) continue;
+            double m = -INFINITY;
+            for (int t = 0; t < len; ++t) {
+                reconstruct_row_f64(k_packed + (base + t) * (D / 2),
+                                    k_scales + (base + t) * (D / G), lk, s_k,
+                                    D, G, row);
+                double dot = 0.0;
+                for (int i = 0; i < D; ++i) dot += qd[i] * row[i];
+                z[t] = sm_scale * dot;
+                if (z[t] > m) m = z[t];
+            }
+            double l = 0.0;
+            for (int t = 0; t < len; ++t) {
+                double p = exp(z[t] - m);
+                l += p;
+                reconstruct_row_f64(v_packed + (base + t) * (D / 2),
+                                    v_scales + (base + t) * (D / G), lv, s_v,
+                                    D, G, row);
+                for (int i = 0; i < D; ++i) o[i] += p * row[i];
+            }
+            for (int i = 0; i < D; ++i) o[i] /= l;
+        }
+    }
+    free(z);
     return 0;
 }

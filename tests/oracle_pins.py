@@ -11,7 +11,11 @@ check the oracle against what the pages and the mathematics fix:
 * the quantiser's error bound |y - q S| <= S/2 and the codes' range;
 * library routines: fp16 conversion against numpy's IEEE cast;
 * hand-worked examples (tests/golden/worked_examples.json) and the pages'
-  printed compression figure (tests/golden/accounting.json).
+  printed compression figure (tests/golden/accounting.json);
+* decode attention: against torch's scaled_dot_product_attention (float64)
+  on caches rebuilt with numpy and scipy's Hadamard matrix, and against the
+  closed forms one key (o = V_0), zero scale (o = mean V), a huge scale
+  (o = V at the arg-max) and masking (entries past the length are ignored).
 
 ``tests/test_oracle.py`` runs every pin on the oracle; ``tests/
 test_oracle_mutants.py`` plants plausible mistakes in copies of the oracle's
@@ -362,10 +366,117 @@ def pin_accounting(o):
         assert abs(fp16_bytes / stored - 16.0 / (4.0 + 16.0 / G)) < 1e-12
 
 
+# ---- decode attention over the int4 cache ------------------------------
+
+def _nibbles(packed):
+    """Independent unpack: low nibble first, 4-bit two's complement."""
+    p = np.asarray(packed, dtype=np.uint8)
+    lo = (p & 0xF).astype(np.int16)
+    hi = (p >> 4).astype(np.int16)
+    q = np.stack([lo, hi], axis=-1).reshape(p.shape[:-1] + (p.shape[-1] * 2,))
+    return np.where(q >= 8, q - 16, q).astype(np.float64)
+
+
+def _rebuild(packed, scales, lam, s, G):
+    """Rows of the cache in float64: (diag(s) H (codes . S) / sqrt D) / lambda,
+    with scipy's Sylvester-Hadamard matrix."""
+    import scipy.linalg
+    q = _nibbles(packed)
+    D = q.shape[-1]
+    S = np.repeat(np.asarray(scales, dtype=np.float16).astype(np.float64), G, axis=-1)
+    H = scipy.linalg.hadamard(D).astype(np.float64)
+    y = q * S
+    return (y @ H.T) / math.sqrt(D) * s.astype(np.float64) / lam.astype(np.float64)
+
+
+def _attn_case(rng, B, Hq, Hkv, T, D, G, smax=2.0):
+    q = rng.standard_normal((B, Hq, D)).astype(np.float16)
+    kp = rng.integers(0, 256, (B, Hkv, T, D // 2), dtype=np.uint8)
+    vp = rng.integers(0, 256, (B, Hkv, T, D // 2), dtype=np.uint8)
+    ks = rng.uniform(0.01, smax, (B, Hkv, T, D // G)).astype(np.float16)
+    vs = rng.uniform(0.01, smax, (B, Hkv, T, D // G)).astype(np.float16)
+    lk, sk = _rand_params(rng, D)
+    lv, sv = _rand_params(rng, D)
+    return q, kp, ks, vp, vs, lk, sk, lv, sv
+
+
+def pin_attention_vs_sdpa(o):
+    """The oracle equals torch's SDPA (float64) on independently rebuilt K, V,
+    with grouped-query head mapping and per-sequence lengths."""
+    import torch
+    rng = np.random.default_rng(21)
+    for B, Hq, Hkv, T, D, G, scale in ((2, 8, 2, 37, 32, 8, 0.3), (3, 4, 4, 20, 64, 32, 0.125),
+                                       (1, 6, 1, 9, 16, 16, 1.7)):
+        q, kp, ks, vp, vs, lk, sk, lv, sv = _attn_case(rng, B, Hq, Hkv, T, D, G)
+        lens = rng.integers(1, T + 1, B)
+        lens[0] = T
+        got = o.attention_decode(q, kp, ks, vp, vs, lens, lk, sk, lv, sv, G, scale)
+        K = _rebuild(kp, ks, lk, sk, G)
+        V = _rebuild(vp, vs, lv, sv, G)
+        R = Hq // Hkv
+        for b in range(B):
+            L = int(lens[b])
+            kt = torch.from_numpy(K[b, :, :L]).repeat_interleave(R, dim=0)[None]
+            vt = torch.from_numpy(V[b, :, :L]).repeat_interleave(R, dim=0)[None]
+            qt = torch.from_numpy(q[b].astype(np.float64))[None, :, None, :]
+            ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)
+            ref = ref[0, :, 0, :].numpy()
+            err = np.abs(got[b] - ref).max()
+            assert err <= 1e-12 * max(1.0, np.abs(ref).max()), f"attention off by {err}"
+
+
+def pin_attention_closed_forms(o):
+    """One key: o = V_0.  Zero scale: o = mean of V.  Huge scale: o = V at the
+    key with the largest score.  Both compared with the fp32 inverse path."""
+    rng = np.random.default_rng(22)
+    B, Hq, Hkv, T, D, G = 2, 4, 2, 16, 64, 16
+    q, kp, ks, vp, vs, lk, sk, lv, sv = _attn_case(rng, B, Hq, Hkv, T, D, G)
+    def deq(b, kv, t, packed, scales, lam, s):
+        return o.dequantize_f32(o.unpack(packed[b, kv, t]), scales[b, kv, t], lam, s, G)[0]
+    one = o.attention_decode(q, kp, ks, vp, vs, [1, 1], lk, sk, lv, sv, G, 0.5)
+    for b in range(B):
+        for h in range(Hq):
+            ref = deq(b, h // 2, 0, vp, vs, lv, sv).astype(np.float64)
+            assert np.abs(one[b, h] - ref).max() <= 1e-5 * np.abs(ref).max()
+    mean = o.attention_decode(q, kp, ks, vp, vs, [T, 5], lk, sk, lv, sv, G, 0.0)
+    for b, L in ((0, T), (1, 5)):
+        for h in range(Hq):
+            ref = np.mean([deq(b, h // 2, t, vp, vs, lv, sv) for t in range(L)], axis=0)
+            assert np.abs(mean[b, h] - ref).max() <= 1e-5 * np.abs(ref).max()
+    # huge scale: the softmax is one-hot at the arg-max of the scores
+    K = _rebuild(kp, ks, lk, sk, G)
+    hard = o.attention_decode(q, kp, ks, vp, vs, [T, T], lk, sk, lv, sv, G, 1e4)
+    for b in range(B):
+        for h in range(Hq):
+            z = K[b, h // 2] @ q[b, h].astype(np.float64)
+            top = np.sort(z)[-2:]
+            if top[1] - top[0] < 1e-2:
+                continue
+            ref = deq(b, h // 2, int(np.argmax(z)), vp, vs, lv, sv)
+            assert np.all(np.isfinite(hard[b, h]))
+            assert np.abs(hard[b, h] - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+def pin_attention_masking(o):
+    """Entries past a sequence's length do not matter; length 0 gives 0."""
+    rng = np.random.default_rng(23)
+    B, Hq, Hkv, T, D, G = 2, 2, 1, 12, 32, 32
+    q, kp, ks, vp, vs, lk, sk, lv, sv = _attn_case(rng, B, Hq, Hkv, T, D, G)
+    a = o.attention_decode(q, kp, ks, vp, vs, [7, 0], lk, sk, lv, sv, G, 0.4)
+    kp2, vp2, ks2 = kp.copy(), vp.copy(), ks.copy()
+    kp2[:, :, 7:] ^= 0x5A
+    vp2[:, :, 7:] ^= 0xA5
+    ks2[:, :, 7:] = np.float16(60000.0)
+    b = o.attention_decode(q, kp2, ks2, vp2, vs, [7, 0], lk, sk, lv, sv, G, 0.4)
+    assert np.array_equal(a, b)
+    assert np.all(a[1] == 0.0)
+
+
 ALL_PINS = [
     pin_f16_conversion, pin_norm_const, pin_fwht_dense, pin_rotation_dense,
     pin_rotate_f32, pin_norm_preservation, pin_roundtrip_unquantized,
     pin_code_invariants, pin_error_bound, pin_dequant_vs_f64,
     pin_special_cases, pin_worked_examples, pin_divform_near_ties,
     pin_pack_layout, pin_accounting,
+    pin_attention_vs_sdpa, pin_attention_closed_forms, pin_attention_masking,
 ]

@@ -36,6 +36,14 @@ MUTANTS = [
     ("deq_lambda_mult", "float il = 1.0f / lam[i];", "float il = lam[i];", 0),
     ("unrotate_f64_lambda", "(double)s[i] / lam[i];", "(double)s[i] * lam[i];", 0),
     ("f16_round_trunc", "_Float16 h = (_Float16)f;", "_Float16 h = (_Float16)(f - f * 0x1p-12f);", 0),
+    ("attn_gqa_index", "int kv = h / R;", "int kv = h % Hkv;", 0),
+    ("attn_no_max_shift", "double p = exp(z[t] - m);", "double p = exp(z[t]);", 0),
+    ("attn_len_ignored", "for (int t = 0; t < len; ++t) {\n                double p", "for (int t = 0; t < T; ++t) {\n                double p", 0),
+    ("attn_scale_unused", "z[t] = sm_scale * dot;", "z[t] = dot;", 0),
+    ("attn_v_uses_k_lambda", "D, G, row);\n                for (int i = 0; i < D; ++i) o[i] += p * row[i];",
+     "D, G, row);\n                (void)lv; for (int i = 0; i < D; ++i) o[i] += p * row[i] * lv[i] / lk[i];", 0),
+    ("attn_not_normalised", "for (int i = 0; i < D; ++i) o[i] /= l;", "(void)l;", 0),
+    ("attn_scale_index", "(double)kvqo_f16_to_f32(scales[i / G]);", "(double)kvqo_f16_to_f32(scales[0]);", 0),
 ]
 
 
