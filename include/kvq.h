@@ -146,11 +146,72 @@ int kvq_roundtrip(const uint16_t *x, const float *lambda, const int8_t *signs,
                   uint8_t *packed, uint16_t *scales, void *stream);
 
 /*
+ * kvq_attention_decode -- one decode step of attention over the int4 cache:
+ * for every sequence b and query head h,
+ *     o[b][h] = sum_t p_t V_t,  p = softmax_t(sm_scale <q[b][h], K_t>),
+ * over the keys t < seq_len[b] of KV head h / (Hq / Hkv) (grouped-query
+ * attention), where K_t and V_t are the rows kvq_dequantize would rebuild
+ * from the codes, but never rounded to fp16 nor written anywhere.  The
+ * operation is the fused group-quantised attention of "The Kernel That
+ * Finally Did Something -- And Didn't Quite Agree With Itself" (VeloxQuant-MLX
+ * blog), "Fused group-affine (KIVI-style) attention", taken to the rotated
+ * domain of "When Quantization Is Free" (Methodologie 1): the query is
+ * rotated once, q~ = H diag(s_K)(q / lambda_K)/sqrt(D), scores are
+ * <q~, codes * S>, the values are summed in the rotated domain and rotated
+ * back once per head.  An empty context (seq_len[b] = 0) gives zeros.
+ *
+ *   q         [in]  fp16 bits [B][Hq][D]; 16-byte aligned.
+ *   k_packed, v_packed  [in] uint8 [B][Hkv][T][D/2] (kvq_quantize rows, one
+ *                   cache row per (sequence, KV head, position)); 16-byte
+ *                   aligned.
+ *   k_scales, v_scales  [in] fp16 bits [B][Hkv][T][D/group]; 16-byte aligned.
+ *   seq_len   [in]  int32 [B], device memory, 4-byte aligned; each in [0, T]
+ *                   (a value outside is clamped and sets bit 3 of the fault
+ *                   word).
+ *   lambda_k, signs_k, lambda_v, signs_v  [in] the parameters the K and V
+ *                   rows were quantised with (fp32 [D], 4-byte aligned;
+ *                   int8 [D] with values +-1).
+ *   B, Hq, Hkv, T  sequences, query heads, KV heads, cache positions:
+ *                   B >= 0, Hkv >= 1, Hq a multiple of Hkv with Hq / Hkv <= 8,
+ *                   T >= 0 a multiple of 16 (else KVQ_ERR_COUNT).
+ *   D, group  D in {64, 128} (else KVQ_ERR_DIM); group in {32, 64, 128},
+ *                   group <= D (else KVQ_ERR_GROUP).
+ *   sm_scale  softmax scale, finite (usually 1/sqrt(D)).
+ *   out       [out] fp16 bits [B][Hq][D]; 16-byte aligned; must not overlap
+ *                   the inputs.
+ *   workspace, workspace_bytes  optional device scratch for splitting the
+ *                   key axis when B * Hkv is too small to fill the GPU; give
+ *                   at least kvq_attention_workspace_bytes() bytes, 16-byte
+ *                   aligned.  With less (or NULL) the call runs unsplit: same
+ *                   result up to fp32 summation order, possibly slower.  The
+ *                   library allocates nothing.
+ *   stream    cudaStream_t (NULL: legacy default stream); asynchronous.
+ * B = 0 is a no-op.  Preconditions are checked in the order shape, NULL,
+ * alignment.
+ */
+int kvq_attention_decode(const uint16_t *q, const uint8_t *k_packed,
+                         const uint16_t *k_scales, const uint8_t *v_packed,
+                         const uint16_t *v_scales, const int32_t *seq_len,
+                         const float *lambda_k, const int8_t *signs_k,
+                         const float *lambda_v, const int8_t *signs_v,
+                         int B, int Hq, int Hkv, int T, int D, int group,
+                         float sm_scale, uint16_t *out, void *workspace,
+                         int64_t workspace_bytes, void *stream);
+
+/*
+ * kvq_attention_workspace_bytes -- bytes of workspace kvq_attention_decode
+ * uses for these shapes on the current device (0: it does not split), or -1
+ * if the shapes are invalid.  Host-only; launches nothing.
+ */
+int64_t kvq_attention_workspace_bytes(int B, int Hq, int Hkv, int T, int D, int group);
+
+/*
  * kvq_fault_status -- the current device's fault word: 0 when every bounded
- * wait of every kernel so far completed; bit 0 set when a quantize or
- * dequantize block gave up waiting for its bulk copies (its outputs are then
- * incomplete); bit 1 set by kvq_selftest_wait_timeout; bit 2 set when
- * kvq_quantize_rows skipped an out-of-range row index.  Non-zero `clear`
+ * wait of every kernel so far completed; bit 0 set when a quantize,
+ * dequantize or attention block gave up waiting for its bulk copies (its
+ * outputs are then incomplete); bit 1 set by kvq_selftest_wait_timeout; bit 2 set when
+ * kvq_quantize_rows skipped an out-of-range row index; bit 3 set when
+ * kvq_attention_decode met a sequence length outside [0, T].  Non-zero `clear`
  * resets the word.  Synchronous (it copies the word to the host, which waits
  * for prior work on the device's legacy default stream).  Returns -1 if the
  * word cannot be read.

@@ -22,18 +22,23 @@
 // same ascending-h order as the plain sequential loop, so the result is
 // bit-identical to it.
 //
-// Data movement.  A persistent block of 128 lanes walks tiles of 128 / LANES
-// vectors, double-buffered in shared memory.  Each fp16 tile moves as Q = D/64
-// tensor copies (one per 64-channel quarter of the rows, 2-D maps of 64
-// channels x n rows with the 128-byte swizzle), issued by one thread; chunk c
-// of tile row t lands at chunk c ^ (t mod 8), so lanes reading consecutive
-// rows hit distinct bank groups.  Quantize: tensor loads in, 16-byte code
-// stores and 2-byte scale stores out.  Dequantize: the tile's packed codes
-// arrive as one bulk copy; the lanes write their fp16 rows into a swizzled
-// staging tile that leaves as Q tensor stores (rows past n are clipped by the
-// copy engine).  No copy uses multicast.  Every mbarrier wait is bounded; a
-// block that gives up sets a device fault word, drains its own copies and
-// returns (kvq_fault_status reads the word).
+// Data movement.  Each warp streams its own warp tiles (32 / LANES vectors,
+// one per lane or lane pair) through a private double-buffered ring in
+// shared memory, so no block-wide barrier couples the warps.  The warps of a
+// block draw their next tile from a shared-memory counter over the block's
+// tiles (blockIdx.x + i * gridDim.x): a warp that the scheduler favours takes
+// more tiles, and all warps finish together.  Large batches run one block of
+// 12 warps per SM; small ones run 4-warp blocks, three per SM.  Each fp16
+// tile moves as Q = D/64 tensor copies (one per 64-channel quarter of the
+// rows, 2-D maps of 64 channels x n rows with the 128-byte swizzle), issued by
+// one lane; chunk c of tile row t lands at chunk c ^ (t mod 8), so lanes
+// reading consecutive rows hit distinct bank groups.  Quantize: tensor loads
+// in, 16-byte code stores and 2-byte scale stores out.  Dequantize: a tile's
+// packed codes and its scales arrive as bulk copies; the lanes write their
+// fp16 rows into a swizzled staging tile that leaves as Q tensor stores (rows
+// past n are clipped by the copy engine).  No copy uses multicast.  Every
+// mbarrier wait is bounded; a warp that gives up sets a device fault word,
+// drains its own copies and returns (kvq_fault_status reads the word).
 //
 // This translation unit is compiled with --fmad=false and uses only _rn
 // intrinsics on the contract-sensitive steps, so no multiply is ever fused
@@ -49,9 +54,14 @@
 
 #include "kvq.h"
 
+// The attention translation unit's fault word and last CUDA error.
+unsigned int kvq_attn_fault_word(int clear);
+int kvq_attn_last_cuda_error();
+
 namespace {
 
 constexpr int kThreads = 128;              // lanes per block (4 warps)
+constexpr int kWarps = 12;                 // warps of a streaming block (one block per SM)
 constexpr unsigned kFullMask = 0xffffffffu;
 constexpr uint32_t kSpinLimit = 1u << 22;  // bounded mbarrier waits
 constexpr int kMaxDevices = 64;
@@ -77,7 +87,6 @@ struct Tile {
   static constexpr int QB = ROWS * 128;             // bytes of one quarter of a tile
   static constexpr int STAGE = Q * QB;              // bytes of one fp16 tile (= ROWS * 2D)
   static constexpr int TAB = LANES * NP * 8;        // per-channel pair table
-  static constexpr int PIN = ROWS * (D / 2);        // bytes of one packed tile
 };
 
 // Byte offset, inside one fp16 tile, of 16-byte chunk c (channels 8c..8c+7) of
@@ -96,61 +105,46 @@ struct RowMaps {
   CUtensorMap q[4];
 };
 
+// A warp tile: the 32 / LANES vectors one warp holds, one per lane (team).
 template <int D>
-constexpr int quantize_smem_bytes() { return 1024 + 2 * Tile<D>::STAGE + Tile<D>::TAB + 16; }
+struct WTile {
+  static constexpr int WROWS = 32 / Tile<D>::LANES;   // vectors per warp tile
+  static constexpr int WQB = WROWS * 128;             // bytes of one quarter of a warp tile
+  static constexpr int WSTAGE = Tile<D>::Q * WQB;     // bytes of one fp16 warp tile
+  static constexpr int WPIN = WROWS * (D / 2);        // bytes of one packed warp tile
+};
+// Byte offset of chunk c of quarter q of row t inside a swizzled warp tile.
+template <int D>
+__device__ __forceinline__ int wtile_off(int q, int t, int c) {
+  return q * WTile<D>::WQB + t * 128 + ((c ^ (t & 7)) << 4);
+}
+
+constexpr int kScaleBlock = 512;   // bytes reserved for one warp tile's scales (>= 32 rows x 16 B)
+
+// Shared memory of a streaming block (quantize, dequantize) of NW warps: one
+// private buffer per warp (a multiple of 1 KiB, so every tensor-copy
+// destination keeps the 1 KiB swizzle alignment), then a header holding the
+// per-channel table, two mbarriers and two stage tile ids per warp and the
+// tile-claim counter.
+template <int D>
+struct Stream {
+  static constexpr int BARS = Tile<D>::TAB;                 // header offsets
+  static constexpr int TQ = BARS + 16 * kWarps;
+  static constexpr int NEXT = TQ + 8 * kWarps;
+  static constexpr int HDR = NEXT + 16;
+  static constexpr int QWARP = 2 * WTile<D>::WSTAGE;        // quantize: two fp16 input stages
+  static constexpr int DWARP =                              // dequantize: output tile, 2 x (codes, scales)
+      (WTile<D>::WSTAGE + 2 * WTile<D>::WPIN + 2 * kScaleBlock + 1023) / 1024 * 1024;
+  static constexpr int smem(int per_warp, int warps) { return 1024 + warps * per_warp + HDR; }
+};
 template <int D>
 constexpr int roundtrip_smem_bytes() { return 1024 + 3 * Tile<D>::STAGE + 2 * Tile<D>::TAB + 16; }
-template <int D>
-constexpr int dequantize_smem_bytes() { return 1024 + Tile<D>::STAGE + 2 * Tile<D>::PIN + Tile<D>::TAB + 16; }
 
 // ---------------------------------------------------------------------------
 // Asynchronous copies and barriers.
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_addr(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_fence_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
-               :: "r"(smem_addr(bar)), "r"(bytes) : "memory");
-}
-// Waits for the phase with the given parity; false if `limit` polls passed.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
-  const uint32_t a = smem_addr(bar);
-  for (uint32_t it = 0; it < limit; ++it) {
-    uint32_t ok;
-    asm volatile("{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-                 " selp.u32 %0, 1, 0, p;\n}" : "=r"(ok) : "r"(a), "r"(parity) : "memory");
-    if (ok) return true;
-  }
-  return false;
-}
-// global -> shared bulk copy completing on an mbarrier (no multicast)
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-               :: "r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
-}
-// 2-D tensor tile load (128B swizzle via the map), completing on an mbarrier
-__device__ __forceinline__ void tensor_g2s(void* dst, const CUtensorMap* map, int x0, int y0, uint64_t* bar) {
-  asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-               :: "r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x0), "r"(y0), "r"(smem_addr(bar))
-               : "memory");
-}
-// 2-D tensor tile store, tracked in bulk groups; rows outside the tensor are skipped
-__device__ __forceinline__ void tensor_s2g(const CUtensorMap* map, int x0, int y0, const void* src) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%1, %2}], [%3];"
-               :: "l"(reinterpret_cast<uint64_t>(map)), "r"(x0), "r"(y0), "r"(smem_addr(src)) : "memory");
-}
-__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+#include "kvq_async.cuh"
 
 __device__ __forceinline__ void st_v4(void* p, const uint32_t (&r)[4]) {
   asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};"
@@ -298,51 +292,74 @@ __device__ __forceinline__ void fill_tab(float4* tab, const float* __restrict__ 
 // ---------------------------------------------------------------------------
 // Quantize: fp16 [n][D] -> packed u8 [n][D/2] + fp16 scales [n][D/G].
 // ---------------------------------------------------------------------------
-template <int D, int G, bool INDEXED>
-__global__ void __launch_bounds__(kThreads, 3)
+template <int D, int G, bool INDEXED, int NW>
+__global__ void __launch_bounds__(NW * 32, NW == kWarps ? 1 : 3)
 kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restrict__ lam,
                     const int8_t* __restrict__ sgn, int64_t n, float c,
                     uint8_t* __restrict__ packed, uint16_t* __restrict__ scales,
                     const int64_t* __restrict__ row_idx, int64_t cache_rows) {
   using T = Tile<D>;
-  constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF, ROWS = T::ROWS;
+  using W = WTile<D>;
+  constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF;
   constexpr int GX = (G < HALF) ? G : HALF;      // pairs spanned by one group (G <= HALF)
   constexpr int NGH = HALF / GX;                 // groups per half-lane
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float4* tabw = reinterpret_cast<float4*>(smem + 2 * T::STAGE);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 2 * T::STAGE + T::TAB);
   const int tid = threadIdx.x;
-  const int sub = tid % LANES;
-  const int rin = tid / LANES;
+  const int warp = tid >> 5, lane = tid & 31;
+  using L = Stream<D>;
+  uint8_t* hdr = smem + NW * L::QWARP;
+  float4* tabw = reinterpret_cast<float4*>(hdr);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + L::BARS) + 2 * warp;
+  int* tq = reinterpret_cast<int*>(hdr + L::TQ) + 2 * warp;   // tile in each stage, -1: none
+  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + L::NEXT);
+  uint8_t* wsm = smem + warp * L::QWARP;
+  const int sub = lane % LANES;
+  const int rin = lane / LANES;
   fill_tab<D>(tabw, lam, sgn, false);
-  if (tid == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
+  if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
+  if (tid == 0) *next = 0;
   __syncthreads();
 
-  const int64_t ntiles = (n + ROWS - 1) / ROWS;
-  const int tstride = gridDim.x;
-  // tile -> stage: one thread issues the Q quarter copies of the whole tile
+  // The block owns warp tiles blockIdx.x + i * gridDim.x; its warps claim the
+  // next i from a shared counter, so a warp that runs ahead takes more tiles.
+  const int64_t ntiles = (n + W::WROWS - 1) / W::WROWS;
+  // (ntiles < 2^31: n < 2^31 and a warp tile holds at least 16 rows)
+  const unsigned int mine = static_cast<unsigned int>((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  auto claim = [&]() -> int {
+    unsigned int i = 0;
+    if (lane == 0) i = atomicAdd(next, 1u);
+    i = __shfl_sync(kFullMask, i, 0);
+    return i < mine ? static_cast<int>(blockIdx.x + i * gridDim.x) : -1;
+  };
   auto issue = [&](int64_t tile, int stage) {
-    if (tile >= ntiles || tid != 0) return;
-    mbar_expect_tx(&bar[stage], T::STAGE);
+    if (tile < 0 || lane != 0) return;
+    mbar_expect_tx(&bar[stage], W::WSTAGE);
 #pragma unroll
     for (int q = 0; q < T::Q; ++q)
-      tensor_g2s(smem + stage * T::STAGE + q * T::QB, &maps.q[q], 0, static_cast<int>(tile * ROWS), &bar[stage]);
+      tensor_g2s(wsm + stage * W::WSTAGE + q * W::WQB, &maps.q[q], 0, static_cast<int>(tile * W::WROWS), &bar[stage]);
   };
-  issue(blockIdx.x, 0);
-  issue(static_cast<int64_t>(blockIdx.x) + tstride, 1);
+  auto refill = [&](int stage) {
+    const int t = claim();
+    if (lane == 0) tq[stage] = t;
+    issue(t, stage);
+  };
+  refill(0);
+  refill(1);
   const float2 c2 = make_float2(c, c);
   const float4* mytab = tabw + sub * (NP / 2);
-  int64_t tile = blockIdx.x;
-  for (uint32_t k = 0; tile < ntiles; ++k, tile += tstride) {
+  for (uint32_t k = 0;; ++k) {
     const int stage = k & 1;
+    __syncwarp();
+    const int64_t tile = tq[stage];
+    if (tile < 0) break;                         // later claims failed too
     const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) atomicOr(&g_kvq_fault, 1u);
-      if (tile + tstride < ntiles) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
+    if (__any_sync(kFullMask, !ok)) {
+      if (lane == 0) atomicOr(&g_kvq_fault, 1u);
+      if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
       return;
     }
-    const int64_t row = tile * ROWS + rin;
+    const int64_t row = tile * W::WROWS + rin;
     bool active = row < n;
     int64_t orow = row;                          // destination row of the codes
     if constexpr (INDEXED) {
@@ -354,14 +371,14 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
     }
 
     // a1: widen fp16 and multiply by lambda*s (one rounding per element).
-    const uint8_t* st = smem + stage * T::STAGE;
+    const uint8_t* st = wsm + stage * W::WSTAGE;
     float2 p[NP];
 #pragma unroll
     for (int j = 0; j < NP / 8; ++j) {
       constexpr int QL = EPT / 64;               // quarters per lane
       const int ea = 8 * j, eb = HALF + 8 * j;    // first channel of each chunk
-      const uint4 a = *reinterpret_cast<const uint4*>(st + tile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8));
-      const uint4 b = *reinterpret_cast<const uint4*>(st + tile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8));
+      const uint4 a = *reinterpret_cast<const uint4*>(st + wtile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8));
+      const uint4 b = *reinterpret_cast<const uint4*>(st + wtile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8));
       const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -372,8 +389,8 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
         p[8 * j + 2 * t + 1] = __fmul2_rn(make_float2(fa.y, fb.y), make_float2(l.z, l.w));
       }
     }
-    __syncthreads();          // everyone has its inputs: the stage can be refilled
-    issue(tile + 2 * static_cast<int64_t>(tstride), stage);
+    __syncwarp();             // the warp has its inputs: the stage can be refilled
+    refill(stage);
 
     // a2, a3: transform, normalise.
     fwht_pairs<EPT, LANES>(p, sub);
@@ -446,51 +463,95 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
 // ---------------------------------------------------------------------------
 // Dequantize: packed u8 [n][D/2] + fp16 scales [n][D/G] -> fp16 [n][D].
 // ---------------------------------------------------------------------------
-template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 3)
+template <int D, int G, int NW>
+__global__ void __launch_bounds__(NW * 32, NW == kWarps ? 1 : 3)
 kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
                       const float* __restrict__ lam, const int8_t* __restrict__ sgn,
-                      int64_t n, float c, const __grid_constant__ RowMaps maps) {
+                      int64_t n, float c, const __grid_constant__ RowMaps maps, int scale_copy) {
   using T = Tile<D>;
-  constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF, ROWS = T::ROWS;
-  constexpr int PIN = T::PIN;
+  using W = WTile<D>;
+  constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF;
+  constexpr int WROWS = W::WROWS;
+  constexpr int WPIN = W::WPIN;
+  constexpr int SPR = (D / G) * 2;               // scale bytes per row
+  constexpr int WSC = kScaleBlock;
+  static_assert(WROWS * SPR <= WSC, "scale block");
   constexpr int GX = (G < HALF) ? G : HALF;
   constexpr int NGH = HALF / GX;
   constexpr int HG = (G < NP) ? G : NP;          // butterfly stages h < HG stay inside a group
   constexpr int QL = EPT / 64;                   // quarters per lane
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* stage_out = smem;                                  // one swizzled fp16 tile
-  uint8_t* stage_in = smem + T::STAGE;                        // two packed tiles
-  float4* tabw = reinterpret_cast<float4*>(smem + T::STAGE + 2 * PIN);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + T::STAGE + 2 * PIN + T::TAB);
   const int tid = threadIdx.x;
-  const int sub = tid % LANES;
-  const int rin = tid / LANES;
+  const int warp = tid >> 5, lane = tid & 31;
+  using L = Stream<D>;
+  uint8_t* hdr = smem + NW * L::DWARP;
+  float4* tabw = reinterpret_cast<float4*>(hdr);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + L::BARS) + 2 * warp;
+  int* tq = reinterpret_cast<int*>(hdr + L::TQ) + 2 * warp;   // tile in each stage, -1: none
+  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + L::NEXT);
+  uint8_t* stage_out = smem + warp * L::DWARP;                // swizzled fp16 warp tile
+  uint8_t* stage_in = stage_out + W::WSTAGE;                  // two packed warp tiles
+  uint8_t* stage_sc = stage_in + 2 * WPIN;                    // two scale blocks
+  const int sub = lane % LANES;
+  const int rin = lane / LANES;
   fill_tab<D>(tabw, lam, sgn, true);
-  if (tid == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
+  if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
+  if (tid == 0) *next = 0;
   __syncthreads();
 
-  const int64_t ntiles = (n + ROWS - 1) / ROWS;
-  const int tstride = gridDim.x;
-  auto issue = [&](int64_t tile, int stage) {
-    if (tile >= ntiles || tid != 0) return;
-    const int64_t row0 = tile * ROWS;
-    const int valid = static_cast<int>(n - row0 < ROWS ? n - row0 : ROWS);
-    mbar_expect_tx(&bar[stage], static_cast<uint32_t>(valid) * (D / 2));
-    bulk_g2s(stage_in + stage * PIN, packed + row0 * (D / 2), static_cast<uint32_t>(valid) * (D / 2), &bar[stage]);
+  const int64_t ntiles = (n + WROWS - 1) / WROWS;
+  // (ntiles < 2^31: n < 2^31 and a warp tile holds at least 16 rows)
+  const unsigned int mine = static_cast<unsigned int>((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  auto claim = [&]() -> int {
+    unsigned int i = 0;
+    if (lane == 0) i = atomicAdd(next, 1u);
+    i = __shfl_sync(kFullMask, i, 0);
+    return i < mine ? static_cast<int>(blockIdx.x + i * gridDim.x) : -1;
   };
-  issue(blockIdx.x, 0);
-  issue(static_cast<int64_t>(blockIdx.x) + tstride, 1);
+  // bytes of the scale block moved by the copy engine (a multiple of 16)
+  auto scale_bytes = [&](int64_t tile) -> uint32_t {
+    if (!scale_copy) return 0;
+    const int64_t row0 = tile * WROWS;
+    const int valid = static_cast<int>(n - row0 < WROWS ? n - row0 : WROWS);
+    return static_cast<uint32_t>(valid * SPR) & ~15u;
+  };
+  auto issue = [&](int64_t tile, int stage) {
+    if (tile < 0 || lane != 0) return;
+    const int64_t row0 = tile * WROWS;
+    const int valid = static_cast<int>(n - row0 < WROWS ? n - row0 : WROWS);
+    const uint32_t sb = scale_bytes(tile);
+    mbar_expect_tx(&bar[stage], static_cast<uint32_t>(valid) * (D / 2) + sb);
+    bulk_g2s(stage_in + stage * WPIN, packed + row0 * (D / 2), static_cast<uint32_t>(valid) * (D / 2), &bar[stage]);
+    if (sb) bulk_g2s(stage_sc + stage * WSC, reinterpret_cast<const uint8_t*>(scales) + row0 * SPR, sb, &bar[stage]);
+  };
+  auto refill = [&](int stage) {
+    const int t = claim();
+    if (lane == 0) tq[stage] = t;
+    issue(t, stage);
+  };
+  refill(0);
+  refill(1);
   const float2 c2 = make_float2(c, c);
   const float4* mytab = tabw + sub * (NP / 2);
   const __half2 k1544 = __floats2half2_rn(1544.0f, 1544.0f);
-  int64_t tile = blockIdx.x;
-  for (uint32_t k = 0; tile < ntiles; ++k, tile += tstride) {
+  for (uint32_t k = 0;; ++k) {
     const int stage = k & 1;
-    const int64_t row = tile * ROWS + rin;
+    __syncwarp();
+    const int64_t tile = tq[stage];
+    if (tile < 0) break;                         // later claims failed too
+    const int64_t row = tile * WROWS + rin;
     const int64_t rrow = row < n ? row : n - 1;
-    const uint16_t* srow = scales + rrow * (D / G);
+    const bool sc_smem = static_cast<uint32_t>((rin + 1) * SPR) <= scale_bytes(tile);
+    const uint16_t* srow = sc_smem ? reinterpret_cast<const uint16_t*>(stage_sc + stage * WSC + rin * SPR)
+                                   : scales + rrow * (D / G);
+    const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);
+    if (__any_sync(kFullMask, !ok)) {
+      if (lane == 0) atomicOr(&g_kvq_fault, 1u);
+      if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
+      if (lane == 0) bulk_wait0();
+      return;
+    }
     uint16_t sx[NGH], sy[NGH];
     if constexpr (G <= HALF) {
 #pragma unroll
@@ -502,15 +563,8 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
       sx[0] = srow[sub / (G / EPT)];
       sy[0] = sx[0];
     }
-    const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) atomicOr(&g_kvq_fault, 1u);
-      if (tile + tstride < ntiles) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
-      if (tid == 0) bulk_wait0();
-      return;
-    }
     // a8: the lane's EPT/2 bytes of codes; nibbles biased to n = q + 8.
-    const uint4* seg = reinterpret_cast<const uint4*>(stage_in + stage * PIN + rin * (D / 2) + sub * (EPT / 2));
+    const uint4* seg = reinterpret_cast<const uint4*>(stage_in + stage * WPIN + rin * (D / 2) + sub * (EPT / 2));
     uint32_t w[EPT / 8];
 #pragma unroll
     for (int j = 0; j < EPT / 32; ++j) {
@@ -520,10 +574,6 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
       w[4 * j + 2] = a.z ^ 0x88888888u;
       w[4 * j + 3] = a.w ^ 0x88888888u;
     }
-    // Codes in pairs (q[m], q[m+HALF]) as two 16-bit integer lanes holding
-    // W + 0x6608, whose bit pattern is the fp16 encoding of the exact integer
-    // W + 1544 (|W| <= 512).  Unpack: biased nibble n = q + 8 in the low bits
-    // of 0x6600 gives 0x6600 + n = q + 0x6608.
     uint32_t iq[NP];
 #pragma unroll
     for (int kw = 0; kw < NP / 8; ++kw) {
@@ -536,13 +586,6 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
         iq[8 * kw + 2 * t + 1] = (__byte_perm(wa4, wb4, sel) & 0x000F000Fu) | 0x66006600u;
       }
     }
-    // a9 (first part): butterfly stages inside a group act on integers of
-    // magnitude <= 8 * 2^stage <= 512, so they are exact in any arithmetic.
-    // The first kIntStages run on the integer lanes (a + b - bias, a - b +
-    // bias in one 32-bit add for both lanes; each lane stays in [0, 65535],
-    // so nothing carries across), the rest in fp16x2 -- which splits the work
-    // between the integer and the FMA pipes.  u = W * S is then exact in fp32
-    // and equal, stage for stage, to the fp32 butterfly of q * S.
     constexpr int kIntStages = 4;
     constexpr uint32_t kBias2 = 0x66086608u;
     constexpr int HI = (1 << kIntStages) < HG ? (1 << kIntStages) : HG;
@@ -576,14 +619,12 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
     for (int m = 0; m < NP; ++m)
       p[m] = make_float2(mul_f16_f32(__low2half(hq[m]), sx[m / GX]),
                          mul_f16_f32(__high2half(hq[m]), sy[m / GX]));
-    // a9 (rest): the stages that cross groups, in fp32.
+    __syncwarp();             // codes and scales consumed: the input stage can be refilled
+    refill(stage);
     fwht_pairs<EPT, LANES, HG>(p, sub);
 
-    // a10: normalise, s / lambda, fp16 into the swizzled staging tile, which
-    // the tensor store of the previous tile must have finished reading.
-    if (tid == 0) bulk_wait_read0();
-    __syncthreads();          // staging tile free; everyone done with packed stage
-    issue(tile + 2 * static_cast<int64_t>(tstride), stage);
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();             // the warp's staging tile is free
 #pragma unroll
     for (int j = 0; j < NP / 8; ++j) {
       uint32_t lo[4], hi[4];
@@ -592,25 +633,25 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
         const float4 l = mytab[4 * j + t];
         const float2 a = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t], c2), make_float2(l.x, l.y));
         const float2 b = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t + 1], c2), make_float2(l.z, l.w));
-        lo[t] = float2_to_half2_bits(a.x, b.x);   // channels 8j+2t, +1
-        hi[t] = float2_to_half2_bits(a.y, b.y);   // channels HALF+8j+2t, +1
+        lo[t] = float2_to_half2_bits(a.x, b.x);
+        hi[t] = float2_to_half2_bits(a.y, b.y);
       }
       const int ea = 8 * j, eb = HALF + 8 * j;
-      *reinterpret_cast<uint4*>(stage_out + tile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8)) =
+      *reinterpret_cast<uint4*>(stage_out + wtile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8)) =
           make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      *reinterpret_cast<uint4*>(stage_out + tile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8)) =
+      *reinterpret_cast<uint4*>(stage_out + wtile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8)) =
           make_uint4(hi[0], hi[1], hi[2], hi[3]);
     }
-    fence_proxy_async();      // generic-proxy writes -> visible to the tensor store
-    __syncthreads();
-    if (tid == 0) {
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) {
 #pragma unroll
       for (int q = 0; q < T::Q; ++q)
-        tensor_s2g(&maps.q[q], 0, static_cast<int>(tile * ROWS), stage_out + q * T::QB);
+        tensor_s2g(&maps.q[q], 0, static_cast<int>(tile * WROWS), stage_out + q * W::WQB);
       bulk_commit();
     }
   }
-  if (tid == 0) bulk_wait0();
+  if (lane == 0) bulk_wait0();
 }
 
 
@@ -810,20 +851,51 @@ int sm_count(int dev) {
   return v;
 }
 
-// Resident blocks per SM of one kernel instance on one device; the first call
-// also raises the instance's dynamic shared-memory limit.
-template <int KIND, int D, int G, typename Kernel>
-int blocks_per_sm(Kernel k, int dev, int smem) {
+// Resident blocks per SM of one kernel instance at one block shape on one
+// device.  The first call for an instance raises its dynamic shared-memory
+// limit to `attr_smem` (the largest shape it is launched with) and asks for
+// the largest shared-memory carveout, so kernels launched back to back do not
+// make the SMs repartition L1.
+template <int KIND, int D, int G, int SHAPE = 0, typename Kernel>
+int blocks_per_sm(Kernel k, int dev, int attr_smem, int smem, int threads) {
   static std::atomic<int> cache[kMaxDevices];
   if (dev < 0 || dev >= kMaxDevices) return 1;
   int v = cache[dev].load(std::memory_order_relaxed);
   if (v == 0) {
-    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k, kThreads, smem) != cudaSuccess || v < 1)
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, attr_smem);
+    cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k, threads, smem) != cudaSuccess || v < 1)
       v = 1;
     cache[dev].store(v, std::memory_order_relaxed);
   }
   return v;
+}
+
+// Launch shape of a streaming kernel (quantize, dequantize) for n vectors.
+// Large batches run one block of kWarps warps per SM, whose warps share one
+// tile counter.  Batches with fewer than two tiles per such warp run blocks of
+// kSmallWarps warps, several per SM, which spreads the few tiles over more SMs
+// and starts sooner.  Never more blocks than warp tiles.
+constexpr int kSmallWarps = 4;
+
+template <int D>
+bool stream_big(int64_t n, int sms) {
+  const int64_t tiles = (n + WTile<D>::WROWS - 1) / WTile<D>::WROWS;
+  return tiles >= static_cast<int64_t>(sms) * kWarps * 2;
+}
+
+template <int KIND, int D, int G, int NW, typename Kernel>
+int stream_grid(Kernel k, int dev, int sms, int64_t n, int smem) {
+  const int64_t tiles = (n + WTile<D>::WROWS - 1) / WTile<D>::WROWS;
+  const int64_t cap = static_cast<int64_t>(sms) * blocks_per_sm<KIND, D, G, NW>(k, dev, smem, smem, NW * 32);
+  return static_cast<int>(tiles < cap ? tiles : cap);
+}
+
+inline int current_device_sms(int& dev) {
+  dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  const int sms = sm_count(dev);
+  return sms < 1 ? 1 : sms;
 }
 
 template <int KIND, int D, int G, typename Kernel>
@@ -831,7 +903,7 @@ int grid_for(Kernel k, int64_t n, int smem) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
   const int64_t need = (n + Tile<D>::ROWS - 1) / Tile<D>::ROWS;
-  int64_t cap = static_cast<int64_t>(sm_count(dev)) * blocks_per_sm<KIND, D, G>(k, dev, smem);
+  int64_t cap = static_cast<int64_t>(sm_count(dev)) * blocks_per_sm<KIND, D, G, 0>(k, dev, smem, smem, kThreads);
   if (cap < 1) cap = 1;
   return static_cast<int>(need < cap ? need : cap);
 }
@@ -860,13 +932,13 @@ EncodeTiledFn encode_tiled() {
 // One 2-D map per 64-channel quarter of the fp16 rows at `base`: 64 channels
 // x n rows, row stride 2D bytes, box 64 x ROWS, 128-byte swizzle.
 template <int D>
-int make_row_maps(RowMaps& m, const void* base, int64_t n) {
+int make_row_maps(RowMaps& m, const void* base, int64_t n, int box_rows = Tile<D>::ROWS) {
   const EncodeTiledFn enc = encode_tiled();
   if (enc == nullptr) return KVQ_ERR_LAUNCH;
   for (int q = 0; q < D / 64; ++q) {
     const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(n)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(2 * D)};
-    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(Tile<D>::ROWS)};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
     const cuuint32_t estr[2] = {1, 1};
     const CUresult r = enc(&m.q[q], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
                            const_cast<char*>(static_cast<const char*>(base)) + 128 * q, dims, strides,
@@ -902,19 +974,32 @@ int finish_launch() {
   return KVQ_OK;
 }
 
+template <int D, int G, bool INDEXED, int NW>
+int launch_quantize_nw(const RowMaps& maps, int dev, int sms, const float* lam, const int8_t* s,
+                       int64_t n, uint8_t* packed, uint16_t* scales, const int64_t* row_idx,
+                       int64_t cache_rows, cudaStream_t st) {
+  auto k = kvq_quantize_kernel<D, G, INDEXED, NW>;
+  constexpr int smem = Stream<D>::smem(Stream<D>::QWARP, NW);
+  const int grid = stream_grid<INDEXED ? 2 : 0, D, G, NW>(k, dev, sms, n, smem);
+  (void)cudaGetLastError();
+  k<<<grid, NW * 32, smem, st>>>(maps, lam, s, n, norm_const(D), packed, scales, row_idx, cache_rows);
+  return finish_launch();
+}
+
 template <int D, int G, bool INDEXED>
 int launch_quantize_t(const uint16_t* x, const float* lam, const int8_t* s, int64_t n,
                       uint8_t* packed, uint16_t* scales, const int64_t* row_idx,
                       int64_t cache_rows, cudaStream_t st) {
-  auto k = kvq_quantize_kernel<D, G, INDEXED>;
-  constexpr int smem = quantize_smem_bytes<D>();
   RowMaps maps;
-  const int rc = make_row_maps<D>(maps, x, n);
+  const int rc = make_row_maps<D>(maps, x, n, WTile<D>::WROWS);
   if (rc != KVQ_OK) return rc;
-  const int grid = grid_for<INDEXED ? 2 : 0, D, G>(k, n, smem);
-  (void)cudaGetLastError();
-  k<<<grid, kThreads, smem, st>>>(maps, lam, s, n, norm_const(D), packed, scales, row_idx, cache_rows);
-  return finish_launch();
+  int dev = 0;
+  const int sms = current_device_sms(dev);
+  if (stream_big<D>(n, sms))
+    return launch_quantize_nw<D, G, INDEXED, kWarps>(maps, dev, sms, lam, s, n, packed, scales,
+                                                     row_idx, cache_rows, st);
+  return launch_quantize_nw<D, G, INDEXED, kSmallWarps>(maps, dev, sms, lam, s, n, packed, scales,
+                                                        row_idx, cache_rows, st);
 }
 
 template <int D, int G>
@@ -930,18 +1015,30 @@ int launch_quantize_rows(const uint16_t* x, const float* lam, const int8_t* s, i
   return launch_quantize_t<D, G, true>(x, lam, s, n, packed, scales, row_idx, cache_rows, st);
 }
 
+template <int D, int G, int NW>
+int launch_dequantize_nw(const RowMaps& maps, int dev, int sms, const uint8_t* packed,
+                         const uint16_t* scales, const float* lam, const int8_t* s, int64_t n,
+                         cudaStream_t st) {
+  auto k = kvq_dequantize_kernel<D, G, NW>;
+  constexpr int smem = Stream<D>::smem(Stream<D>::DWARP, NW);
+  const int grid = stream_grid<1, D, G, NW>(k, dev, sms, n, smem);
+  (void)cudaGetLastError();
+  k<<<grid, NW * 32, smem, st>>>(packed, scales, lam, s, n, norm_const(D), maps,
+                                 (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
+  return finish_launch();
+}
+
 template <int D, int G>
 int launch_dequantize(const uint8_t* packed, const uint16_t* scales, const float* lam,
                       const int8_t* s, int64_t n, uint16_t* out, cudaStream_t st) {
-  auto k = kvq_dequantize_kernel<D, G>;
-  constexpr int smem = dequantize_smem_bytes<D>();
   RowMaps maps;
-  const int rc = make_row_maps<D>(maps, out, n);
+  const int rc = make_row_maps<D>(maps, out, n, WTile<D>::WROWS);
   if (rc != KVQ_OK) return rc;
-  const int grid = grid_for<1, D, G>(k, n, smem);
-  (void)cudaGetLastError();
-  k<<<grid, kThreads, smem, st>>>(packed, scales, lam, s, n, norm_const(D), maps);
-  return finish_launch();
+  int dev = 0;
+  const int sms = current_device_sms(dev);
+  if (stream_big<D>(n, sms))
+    return launch_dequantize_nw<D, G, kWarps>(maps, dev, sms, packed, scales, lam, s, n, st);
+  return launch_dequantize_nw<D, G, kSmallWarps>(maps, dev, sms, packed, scales, lam, s, n, st);
 }
 
 template <int D, int G>
@@ -1058,7 +1155,7 @@ int kvq_fault_status(int clear) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_kvq_fault, &zero, sizeof zero) != cudaSuccess) return -1;
   }
-  return static_cast<int>(v);
+  return static_cast<int>(v | kvq_attn_fault_word(clear));
 }
 
 int kvq_selftest_wait_timeout(uint32_t limit, void* stream) {
@@ -1080,7 +1177,7 @@ const char* kvq_status_string(int status) {
   }
 }
 
-int kvq_last_cuda_error(void) { return g_last_cuda_error; }
+int kvq_last_cuda_error(void) { return g_last_cuda_error ? g_last_cuda_error : kvq_attn_last_cuda_error(); }
 
 int kvq_version(void) { return (1 << 16) | 2; }
 

@@ -1,0 +1,611 @@
+// kvq_attn.cu -- fused decode attention over the int4 rotated-domain KV cache
+// for B200 (sm_100a): kernels and the C-ABI launcher of kvq_attention_decode
+// (include/kvq.h).
+//
+// Method: "The Kernel That Finally Did Something -- And Didn't Quite Agree
+// With Itself" (VeloxQuant-MLX blog), "Fused group-affine (KIVI-style)
+// attention": the quantised keys and values are reconstructed in registers
+// inside a FlashAttention-style online softmax, so no dequantised K or V ever
+// reaches memory, and the key axis is split flash-decoding style when there
+// are few sequences.  The cache rows here are int4 codes of the rotated vector
+// y = H diag(s) (lambda . x) / sqrt(D) with fp16 group scales ("When
+// Quantization Is Free", technical summary, Methodologie 1-3), so the rotation
+// moves to the query, once per head, instead of running once per key:
+//     <q, x_t> = <q~, y_t>,   q~ = H diag(s_K) (q / lambda_K) / sqrt(D),
+// and the values are summed in the rotated domain and rotated back once:
+//     o = (diag(s_V) H (sum_t p_t y_t) / sqrt(D)) / lambda_V
+// (H is symmetric with H H = D I, and s_i^2 = 1).
+//
+// Work decomposition.  A block of four warps owns one (sequence, KV head,
+// key split); each warp streams 64-key blocks (codes and scales of K and V,
+// four bulk copies into a private double-buffered ring) and keeps its own
+// online-softmax state; the block merges the four states at the end.  Both
+// products run on the tensor cores as m16n8k16 fp16 MMAs with fp32
+// accumulation, the query heads of the KV head on the M rows:
+//   * scores: rows 0..R-1 hold the fp16 high parts of q~, rows 8..8+R-1 the
+//     fp16 residuals (q~ = hi + lo to ~2^-22), the N columns are 8 keys and
+//     the K dimension 16 channels.  The channel order inside each 32-channel
+//     block is permuted so that a lane's B fragment for one k-step is the two
+//     nibbles of each of two consecutive code bytes, and every k-step stays
+//     inside one scale group: the group's scale multiplies the per-group
+//     partial sums, key by key, after the MMA.
+//   * values: the score fragments are already in the A layout of the value
+//     product (rows = heads, K dimension = 16 keys), so p * S_V (split hi/lo
+//     the same way) feeds it directly, one A fragment per scale group; the B
+//     fragments pair the same channel of two keys.
+// Codes become exact fp16 integers with a byte permute, a mask and one fp16
+// subtraction (the biased nibble n sits in the low bits of 1024's encoding).
+//
+// Every mbarrier wait is bounded; a warp that gives up sets the fault word
+// and the block still finishes (its output is then meaningless).  A sequence
+// length outside [0, T] is clamped and flagged.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+
+#include "kvq.h"
+
+namespace {
+
+#include "kvq_async.cuh"
+
+constexpr int kAW = 4;                       // warps per block
+constexpr int kBK = 64;                      // keys per streamed block
+constexpr int kAStages = 2;                  // ring depth per warp
+constexpr unsigned kFull = 0xffffffffu;
+constexpr uint32_t kSpin = 1u << 22;         // bounded mbarrier waits
+constexpr int kMaxRows = 8;                  // query heads per KV head (M rows of one MMA half)
+
+__device__ unsigned int g_attn_fault = 0;    // bit 0: a wait gave up; bit 3: bad sequence length
+thread_local int g_attn_cuda_error = 0;
+
+struct AttnParams {
+  const uint16_t* q;            // fp16 [B][Hq][D]
+  const uint8_t* kp;            // [B][Hkv][T][D/2]
+  const uint16_t* ks;           // fp16 [B][Hkv][T][D/G]
+  const uint8_t* vp;
+  const uint16_t* vs;
+  const int32_t* seq_len;       // [B]
+  const float* lam_k;
+  const int8_t* s_k;
+  const float* lam_v;
+  const int8_t* s_v;
+  uint16_t* out;                // fp16 [B][Hq][D]
+  float* part;                  // [B*Hkv*nsplit][R][D + 4] when nsplit > 1
+  int Hkv, T, R, nsplit, chunk;
+  float scale_log2;             // sm_scale * log2(e)
+  float c;                      // fp32 1/sqrt(D)
+};
+
+template <int D, int G>
+struct Attn {
+  static constexpr int NB = D / 32;                 // 32-channel blocks of a row
+  static constexpr int KS = D / 16;                 // k-steps of the score product
+  static constexpr int NT = D / 8;                  // n-tiles of the value product
+  static constexpr int NG = D / G;                  // scale groups of a row
+  static constexpr int W32 = D / 8;                 // 32-bit words of one code row
+  static constexpr int CB = kBK * D / 2;            // code bytes of one block
+  static constexpr int SB = kBK * NG * 2;           // scale bytes of one block
+  static constexpr int STAGE = 2 * CB + 2 * SB;     // K codes, V codes, K scales, V scales
+  static constexpr int QT = 2 * kMaxRows * D * 2;   // q~ hi and lo rows, fp16
+  static constexpr int COMB = kAW * kMaxRows * D * 4;
+  static constexpr int RING = kAW * kAStages * STAGE;
+  static constexpr int AREA = RING > COMB ? RING : COMB;   // the merge reuses the ring
+  static constexpr int SMEM = AREA + QT + kAW * kAStages * 8 + kAW * kMaxRows * 8;
+  static constexpr int DPL = D / 32;                // channels per lane in the row transforms
+};
+
+// fp16x2 (low nibble, high nibble) of byte `beta` of a code word, as exact
+// fp16 integers q in [-8, 7]: w holds the codes xor 0x88 (n = q + 8), w4 = w >> 4.
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w, uint32_t w4, int beta) {
+  const uint32_t x = (__byte_perm(w, w4, static_cast<uint32_t>(beta | ((4 + beta) << 8))) & 0x000F000Fu) | 0x64006400u;
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&x), __floats2half2_rn(1032.0f, 1032.0f));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+// fp16x2 (code of key a, code of key b) at the same nibble of byte `beta`.
+__device__ __forceinline__ uint32_t key_pair(uint32_t wa, uint32_t wb, int beta) {
+  const uint32_t x = (__byte_perm(wa, wb, static_cast<uint32_t>(beta | ((4 + beta) << 8))) & 0x000F000Fu) | 0x64006400u;
+  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&x), __floats2half2_rn(1032.0f, 1032.0f));
+  return *reinterpret_cast<const uint32_t*>(&r);
+}
+
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t h2bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+
+// Unnormalised Walsh-Hadamard transform of one D-vector held by a warp, lane
+// l holding channels DPL*l .. DPL*l + DPL-1 (ascending half-width h).
+template <int D>
+__device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
+  constexpr int DPL = D / 32;
+#pragma unroll
+  for (int h = 1; h < DPL; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+    }
+  }
+#pragma unroll
+  for (int h = DPL; h < D; h <<= 1) {
+    const int lb = h / DPL;
+    const bool upper = (lane & lb) != 0;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      const float o = __shfl_xor_sync(kFull, v[i], lb);
+      v[i] = upper ? o - v[i] : v[i] + o;
+    }
+  }
+}
+
+// out[d] = fp16((s_V[d] * c * (H y)[d]) / lambda_V[d]) for one head, y = o / l.
+template <int D>
+__device__ __forceinline__ void finish_head(const AttnParams& P, float (&v)[D / 32], float l,
+                                            uint16_t* out_row, int lane) {
+  constexpr int DPL = D / 32;
+  const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) v[i] *= inv;
+  warp_fwht<D>(v, lane);
+  uint16_t h[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) {
+    const int d = DPL * lane + i;
+    const float z = v[i] * P.c;
+    const float zs = P.s_v[d] < 0 ? -z : z;
+    h[i] = __half_as_ushort(__float2half_rn(zs / P.lam_v[d]));
+  }
+  if constexpr (DPL == 4) {
+    *reinterpret_cast<uint2*>(out_row + DPL * lane) =
+        make_uint2(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16));
+  } else {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) out_row[DPL * lane + i] = h[i];
+  }
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kAW * 32, 2)
+kvq_attn_kernel(const __grid_constant__ AttnParams P) {
+  using A = Attn<D, G>;
+  constexpr int NB = A::NB, KS = A::KS, NT = A::NT, NG = A::NG, W32 = A::W32, DPL = A::DPL;
+  extern __shared__ __align__(128) uint8_t sm[];
+  uint8_t* ring = sm;                                            // [warp][stage][STAGE]
+  __half* qt = reinterpret_cast<__half*>(sm + A::AREA);           // [2][8][D]: hi rows, lo rows
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + A::AREA + A::QT);
+  float* ml = reinterpret_cast<float*>(bars + kAW * kAStages);    // [warp][8][2]: m, l
+  float* comb = reinterpret_cast<float*>(sm);                     // [warp][8][D], after the key loop
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int item = blockIdx.x;
+  const int split = item % P.nsplit;
+  const int bh = item / P.nsplit;                                 // b * Hkv + kv head
+  const int b = bh / P.Hkv, kvh = bh % P.Hkv;
+  const int R = P.R;
+  int L = P.seq_len[b];
+  if (L < 0 || L > P.T) {
+    if (tid == 0) atomicOr(&g_attn_fault, 8u);
+    L = L < 0 ? 0 : P.T;
+  }
+  const int k0 = split * P.chunk;
+  const int k1 = min(L, k0 + P.chunk);
+  const int nkeys = k1 > k0 ? k1 - k0 : 0;
+  const int nblk = (nkeys + kBK - 1) / kBK;
+
+  uint64_t* bar = bars + kAStages * warp;
+  if (lane == 0) {
+    for (int s = 0; s < kAStages; ++s) mbar_init(&bar[s], 1);
+    mbar_fence_init();
+  }
+  // q~ = H diag(s_K) (q / lambda_K) / sqrt(D), split into fp16 hi + lo.
+  for (int r = warp; r < kMaxRows; r += kAW) {
+    float v[DPL];
+    if (r < R) {
+      const uint16_t* qr = P.q + (static_cast<int64_t>(b) * P.Hkv * R + kvh * R + r) * D;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        const int d = DPL * lane + i;
+        const float x = __half2float(__ushort_as_half(qr[d])) / P.lam_k[d];
+        v[i] = P.s_k[d] < 0 ? -x : x;
+      }
+      warp_fwht<D>(v, lane);
+    } else {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) v[i] = 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      const int d = DPL * lane + i;
+      const float y = v[i] * P.c;
+      const __half hi = __float2half_rn(y);
+      const __half lo = __float2half_rn(y - __half2float(hi));
+      qt[r * D + d] = hi;
+      qt[(kMaxRows + r) * D + d] = lo;
+    }
+  }
+  __syncthreads();
+
+  // Score-product A fragments, k-step j = (32-channel block j/2, half j%2):
+  // k-index 2t, 2t+1 <-> channels 32(j/2) + 8t + 4(j%2) + {0,1}; 2t+8, 2t+9 <-> +{2,3}.
+  uint32_t Aq[KS][4];
+#pragma unroll
+  for (int j = 0; j < KS; ++j) {
+    const int d0 = 32 * (j >> 1) + 8 * t + 4 * (j & 1);
+    Aq[j][0] = *reinterpret_cast<const uint32_t*>(qt + g * D + d0);
+    Aq[j][1] = *reinterpret_cast<const uint32_t*>(qt + (kMaxRows + g) * D + d0);
+    Aq[j][2] = *reinterpret_cast<const uint32_t*>(qt + g * D + d0 + 2);
+    Aq[j][3] = *reinterpret_cast<const uint32_t*>(qt + (kMaxRows + g) * D + d0 + 2);
+  }
+
+  const int64_t row_base = static_cast<int64_t>(bh) * P.T;
+  auto issue = [&](int blk, int stage) {
+    if (blk >= nblk || lane != 0) return;
+    const int kb = k0 + blk * kBK;
+    const int nk = min(kBK, k1 - kb);
+    const int nk16 = (nk + 15) & ~15;                            // stays inside T (T % 16 == 0)
+    const int64_t row0 = row_base + kb;
+    uint8_t* st = ring + (warp * kAStages + stage) * A::STAGE;
+    const uint32_t cb = static_cast<uint32_t>(nk16 * (D / 2));
+    const uint32_t sb = static_cast<uint32_t>(nk16 * NG * 2);
+    mbar_expect_tx(&bar[stage], 2 * cb + 2 * sb);
+    bulk_g2s(st, P.kp + row0 * (D / 2), cb, &bar[stage]);
+    bulk_g2s(st + A::CB, P.vp + row0 * (D / 2), cb, &bar[stage]);
+    bulk_g2s(st + 2 * A::CB, P.ks + row0 * NG, sb, &bar[stage]);
+    bulk_g2s(st + 2 * A::CB + A::SB, P.vs + row0 * NG, sb, &bar[stage]);
+  };
+  for (int s = 0; s < kAStages; ++s) issue(warp + s * kAW, s);
+
+  float O[NT][4];
+#pragma unroll
+  for (int n = 0; n < NT; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.0f;
+  float m = -INFINITY, l = 0.0f;
+  bool failed = false;
+  int k = 0;
+  for (int blk = warp; blk < nblk; blk += kAW, ++k) {
+    const int stage = k % kAStages;
+    const bool ok = mbar_wait(&bar[stage], (k / kAStages) & 1, kSpin);
+    if (__any_sync(kFull, !ok)) {
+      failed = true;
+      break;
+    }
+    const uint8_t* st = ring + (warp * kAStages + stage) * A::STAGE;
+    const uint32_t* kc = reinterpret_cast<const uint32_t*>(st);
+    const uint32_t* vc = reinterpret_cast<const uint32_t*>(st + A::CB);
+    const __half* ksc = reinterpret_cast<const __half*>(st + 2 * A::CB);
+    const __half* vsc = reinterpret_cast<const __half*>(st + 2 * A::CB + A::SB);
+    const int nk = min(kBK, k1 - (k0 + blk * kBK));
+
+    // Scores of the block's 64 keys, in log2 units: z[sb][nt][e] for key
+    // 16 sb + 8 nt + 2 t + e of head g.
+    float z[kBK / 16][2][2];
+#pragma unroll
+    for (int sb = 0; sb < kBK / 16; ++sb) {
+      float acc[NG][2][4];
+#pragma unroll
+      for (int gi = 0; gi < NG; ++gi)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) acc[gi][nt][0] = acc[gi][nt][1] = acc[gi][nt][2] = acc[gi][nt][3] = 0.0f;
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int kk = 16 * sb + 8 * nt + g;
+        uint32_t w[NB], w4[NB];
+#pragma unroll
+        for (int bb = 0; bb < NB; ++bb) {
+          w[bb] = kc[kk * W32 + 4 * bb + t] ^ 0x88888888u;
+          w4[bb] = w[bb] >> 4;
+        }
+#pragma unroll
+        for (int j = 0; j < KS; ++j) {
+          const int bb = j >> 1, h = j & 1;
+          mma16816(acc[(32 * bb) / G][nt], Aq[j], nib_pair(w[bb], w4[bb], 2 * h), nib_pair(w[bb], w4[bb], 2 * h + 1));
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int key = 16 * sb + 8 * nt + 2 * t + e;
+          float zz = 0.0f;
+#pragma unroll
+          for (int gi = 0; gi < NG; ++gi)
+            zz += __half2float(ksc[key * NG + gi]) * (acc[gi][nt][e] + acc[gi][nt][2 + e]);
+          z[sb][nt][e] = (key < nk && g < R) ? zz * P.scale_log2 : -INFINITY;
+        }
+      }
+    }
+    // Online softmax: new running max, rescale what is accumulated.
+    float mx = -INFINITY;
+#pragma unroll
+    for (int sb = 0; sb < kBK / 16; ++sb)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) mx = fmaxf(mx, fmaxf(z[sb][nt][0], z[sb][nt][1]));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+    const float mnew = fmaxf(m, mx);
+    const float alpha = (mnew == -INFINITY) ? 1.0f : exp2f(m - mnew);
+    m = mnew;
+    l *= alpha;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      O[n][0] *= alpha; O[n][1] *= alpha; O[n][2] *= alpha; O[n][3] *= alpha;
+    }
+#pragma unroll
+    for (int sb = 0; sb < kBK / 16; ++sb) {
+      float p[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          p[nt][e] = (z[sb][nt][e] == -INFINITY) ? 0.0f : exp2f(z[sb][nt][e] - m);
+          l += p[nt][e];
+        }
+      // A fragments of the value product, one per scale group: p * S_V as hi + lo.
+      uint32_t Ap[NG][4];
+#pragma unroll
+      for (int gi = 0; gi < NG; ++gi) {
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int key = 16 * sb + 8 * nt + 2 * t;
+          // masked keys may sit on stale scale bytes: keep their weight exactly 0
+          const float pa = p[nt][0] == 0.0f ? 0.0f : p[nt][0] * __half2float(vsc[key * NG + gi]);
+          const float pb = p[nt][1] == 0.0f ? 0.0f : p[nt][1] * __half2float(vsc[(key + 1) * NG + gi]);
+          const __half2 hi = __floats2half2_rn(pa, pb);
+          const float2 hf = __half22float2(hi);
+          Ap[gi][2 * nt] = h2bits(hi);
+          Ap[gi][2 * nt + 1] = h2bits(__floats2half2_rn(pa - hf.x, pb - hf.y));
+        }
+      }
+      // B fragments: n-tile nu = 4 bb + u, column g <-> channel 32 bb + 4 g + u,
+      // i.e. nibble u & 1 of byte 16 bb + 2 g + (u >> 1).
+      const int ka = 16 * sb + 2 * t;
+#pragma unroll
+      for (int bb = 0; bb < NB; ++bb) {
+        const int wi = 4 * bb + (g >> 1);
+        const uint32_t a0 = vc[ka * W32 + wi] ^ 0x88888888u;
+        const uint32_t a1 = vc[(ka + 1) * W32 + wi] ^ 0x88888888u;
+        const uint32_t c0 = vc[(ka + 8) * W32 + wi] ^ 0x88888888u;
+        const uint32_t c1 = vc[(ka + 9) * W32 + wi] ^ 0x88888888u;
+        const uint32_t a04 = a0 >> 4, a14 = a1 >> 4, c04 = c0 >> 4, c14 = c1 >> 4;
+        const int gi = (32 * bb) / G;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int beta = 2 * (g & 1) + (u >> 1);
+          const uint32_t b0 = (u & 1) ? key_pair(a04, a14, beta) : key_pair(a0, a1, beta);
+          const uint32_t b1 = (u & 1) ? key_pair(c04, c14, beta) : key_pair(c0, c1, beta);
+          mma16816(O[4 * bb + u], Ap[gi], b0, b1);
+        }
+      }
+    }
+    __syncwarp();                      // the stage is consumed: refill it
+    issue(blk + kAStages * kAW, stage);
+  }
+  if (failed) {
+    if (lane == 0) atomicOr(&g_attn_fault, 1u);
+    // drain whatever this warp still has in flight before the ring is reused
+    for (int s = 1; s < kAStages; ++s) {
+      const int kk2 = k + s;
+      if (warp + kk2 * kAW < nblk) mbar_wait(&bar[kk2 % kAStages], (kk2 / kAStages) & 1, kSpin);
+    }
+  }
+  l += __shfl_xor_sync(kFull, l, 1);
+  l += __shfl_xor_sync(kFull, l, 2);
+  __syncthreads();                     // every warp is out of the ring: reuse it for the merge
+  if (g < R) {
+    float* cw = comb + (warp * kMaxRows + g) * D;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int bb = n >> 2, u = n & 3;
+      cw[32 * bb + 8 * t + u] = O[n][0] + O[n][2];
+      cw[32 * bb + 8 * t + 4 + u] = O[n][1] + O[n][3];
+    }
+    if (t == 0) {
+      ml[(warp * kMaxRows + g) * 2] = m;
+      ml[(warp * kMaxRows + g) * 2 + 1] = l;
+    }
+  }
+  __syncthreads();
+  for (int r = warp; r < R; r += kAW) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w2 = 0; w2 < kAW; ++w2) M = fmaxf(M, ml[(w2 * kMaxRows + r) * 2]);
+    float lsum = 0.0f, v[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) v[i] = 0.0f;
+#pragma unroll
+    for (int w2 = 0; w2 < kAW; ++w2) {
+      const float mw = ml[(w2 * kMaxRows + r) * 2];
+      const float e = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
+      lsum += e * ml[(w2 * kMaxRows + r) * 2 + 1];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) v[i] += e * comb[(w2 * kMaxRows + r) * D + DPL * lane + i];
+    }
+    if (P.nsplit == 1) {
+      uint16_t* orow = P.out + (static_cast<int64_t>(b) * P.Hkv * R + kvh * R + r) * D;
+      finish_head<D>(P, v, lsum, orow, lane);
+    } else {
+      float* pr = P.part + (static_cast<int64_t>(item) * R + r) * (D + 4);
+      if (lane == 0) { pr[0] = M; pr[1] = lsum; }
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) pr[4 + DPL * lane + i] = v[i];
+    }
+  }
+}
+
+// Merge of the key splits of one (sequence, KV head): one warp per head.
+template <int D>
+__global__ void __launch_bounds__(kMaxRows * 32)
+kvq_attn_combine_kernel(const __grid_constant__ AttnParams P) {
+  constexpr int DPL = D / 32;
+  const int bh = blockIdx.x, b = bh / P.Hkv, kvh = bh % P.Hkv;
+  const int r = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (r >= P.R) return;
+  const int64_t stride = static_cast<int64_t>(P.R) * (D + 4);
+  const float* base = P.part + (static_cast<int64_t>(bh) * P.nsplit * P.R + r) * (D + 4);
+  float M = -INFINITY;
+  for (int s = 0; s < P.nsplit; ++s) M = fmaxf(M, base[s * stride]);
+  float lsum = 0.0f, v[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) v[i] = 0.0f;
+  for (int s = 0; s < P.nsplit; ++s) {
+    const float* pr = base + s * stride;
+    const float e = (pr[0] == -INFINITY) ? 0.0f : exp2f(pr[0] - M);
+    lsum += e * pr[1];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) v[i] += e * pr[4 + DPL * lane + i];
+  }
+  uint16_t* orow = P.out + (static_cast<int64_t>(b) * P.Hkv * P.R + kvh * P.R + r) * D;
+  finish_head<D>(P, v, lsum, orow, lane);
+}
+
+// ---------------------------------------------------------------------------
+// Launch plumbing.
+// ---------------------------------------------------------------------------
+
+int attn_sms() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1) v = 148;
+    cache[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
+// Key-axis split: enough blocks for about four waves of two blocks per SM,
+// but at least one 64-key block per warp in every split.
+struct Split {
+  int nsplit, chunk;
+};
+Split choose_split(int64_t pairs, int T) {
+  if (T <= 0 || pairs <= 0) return Split{1, T > 0 ? T : kBK};
+  const int64_t target = static_cast<int64_t>(attn_sms()) * 2 * 4;
+  int64_t ns = (target + pairs - 1) / pairs;
+  const int64_t max_ns = (T + kBK * kAW - 1) / (kBK * kAW);
+  if (ns > max_ns) ns = max_ns;
+  if (ns < 1) ns = 1;
+  int64_t chunk = (T + ns - 1) / ns;
+  chunk = (chunk + kBK - 1) / kBK * kBK;
+  ns = (T + chunk - 1) / chunk;
+  return Split{static_cast<int>(ns), static_cast<int>(chunk)};
+}
+
+int64_t part_bytes(int64_t pairs, int R, int D, int nsplit) {
+  return nsplit > 1 ? pairs * nsplit * R * (D + 4) * static_cast<int64_t>(sizeof(float)) : 0;
+}
+
+int check_attn(int B, int Hq, int Hkv, int T, int D, int G) {
+  if (D != 64 && D != 128) return KVQ_ERR_DIM;
+  if ((G != 32 && G != 64 && G != 128) || G > D) return KVQ_ERR_GROUP;
+  if (B < 0 || T < 0 || (T % 16) != 0 || Hkv < 1 || Hq < Hkv || (Hq % Hkv) != 0 ||
+      Hq / Hkv > kMaxRows)
+    return KVQ_ERR_COUNT;
+  if (static_cast<int64_t>(B) * Hkv * T >= (int64_t{1} << 40)) return KVQ_ERR_COUNT;
+  return KVQ_OK;
+}
+
+template <int D, int G>
+int launch_attn(AttnParams P, int64_t pairs, cudaStream_t st) {
+  using A = Attn<D, G>;
+  auto k = kvq_attn_kernel<D, G>;
+  static std::atomic<int> ready[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (dev >= 0 && dev < 64 && ready[dev].load(std::memory_order_relaxed) == 0) {
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, A::SMEM);
+    ready[dev].store(1, std::memory_order_relaxed);
+  }
+  const int64_t items = pairs * P.nsplit;
+  (void)cudaGetLastError();
+  k<<<static_cast<unsigned>(items), kAW * 32, A::SMEM, st>>>(P);
+  if (P.nsplit > 1)
+    kvq_attn_combine_kernel<D><<<static_cast<unsigned>(pairs), kMaxRows * 32, 0, st>>>(P);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    g_attn_cuda_error = static_cast<int>(e);
+    return KVQ_ERR_LAUNCH;
+  }
+  return KVQ_OK;
+}
+
+}  // namespace
+
+// Read (and optionally clear) the attention kernels' fault word; used by
+// kvq_fault_status.
+__attribute__((visibility("hidden"))) unsigned int kvq_attn_fault_word(int clear) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_attn_fault, sizeof(v)) != cudaSuccess) return 0;
+  if (clear && v) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(g_attn_fault, &zero, sizeof(zero));
+  }
+  return v;
+}
+__attribute__((visibility("hidden"))) int kvq_attn_last_cuda_error() { return g_attn_cuda_error; }
+
+extern "C" {
+
+int64_t kvq_attention_workspace_bytes(int B, int Hq, int Hkv, int T, int D, int group) {
+  if (check_attn(B, Hq, Hkv, T, D, group) != KVQ_OK) return -1;
+  const int64_t pairs = static_cast<int64_t>(B) * Hkv;
+  const Split sp = choose_split(pairs, T);
+  return part_bytes(pairs, Hq / Hkv, D, sp.nsplit);
+}
+
+int kvq_attention_decode(const uint16_t* q, const uint8_t* k_packed, const uint16_t* k_scales,
+                         const uint8_t* v_packed, const uint16_t* v_scales, const int32_t* seq_len,
+                         const float* lambda_k, const int8_t* signs_k, const float* lambda_v,
+                         const int8_t* signs_v, int B, int Hq, int Hkv, int T, int D, int group,
+                         float sm_scale, uint16_t* out, void* workspace, int64_t workspace_bytes,
+                         void* stream) {
+  const int rc = check_attn(B, Hq, Hkv, T, D, group);
+  if (rc != KVQ_OK) return rc;
+  if (B == 0) return KVQ_OK;
+  if (!q || !k_packed || !k_scales || !v_packed || !v_scales || !seq_len || !lambda_k ||
+      !signs_k || !lambda_v || !signs_v || !out)
+    return KVQ_ERR_NULL;
+  auto al = [](const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; };
+  if (!al(q, 16) || !al(k_packed, 16) || !al(v_packed, 16) || !al(k_scales, 16) ||
+      !al(v_scales, 16) || !al(out, 16) || !al(lambda_k, 4) || !al(lambda_v, 4) || !al(seq_len, 4))
+    return KVQ_ERR_ALIGN;
+  if (!std::isfinite(sm_scale)) return KVQ_ERR_COUNT;
+  const int64_t pairs = static_cast<int64_t>(B) * Hkv;
+  Split sp = choose_split(pairs, T);
+  if (sp.nsplit > 1 && (workspace == nullptr || !al(workspace, 16) ||
+                        workspace_bytes < part_bytes(pairs, Hq / Hkv, D, sp.nsplit)))
+    sp = Split{1, T > 0 ? T : kBK};                      // no room for partials: no split
+  if (pairs * sp.nsplit > 0x7fffffffLL) return KVQ_ERR_COUNT;
+  AttnParams P;
+  P.q = q; P.kp = k_packed; P.ks = k_scales; P.vp = v_packed; P.vs = v_scales;
+  P.seq_len = seq_len; P.lam_k = lambda_k; P.s_k = signs_k; P.lam_v = lambda_v; P.s_v = signs_v;
+  P.out = out;
+  P.part = static_cast<float*>(workspace);
+  P.Hkv = Hkv; P.T = T; P.R = Hq / Hkv; P.nsplit = sp.nsplit; P.chunk = sp.chunk;
+  P.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  P.c = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (D * 1000 + group) {
+    case 64032: return launch_attn<64, 32>(P, pairs, st);
+    case 64064: return launch_attn<64, 64>(P, pairs, st);
+    case 128032: return launch_attn<128, 32>(P, pairs, st);
+    case 128064: return launch_attn<128, 64>(P, pairs, st);
+    case 128128: return launch_attn<128, 128>(P, pairs, st);
+    default: return KVQ_ERR_GROUP;
+  }
+}
+
+}  // extern "C"

@@ -4,6 +4,9 @@ The raw entry points keep the C names and take integer device addresses:
 
     kvq_quantize(x, lam, signs, n_vec, D, group, packed, scales, stream) -> status
     kvq_dequantize(packed, scales, lam, signs, n_vec, D, group, x_out, stream) -> status
+    kvq_attention_decode(q, k_packed, k_scales, v_packed, v_scales, seq_len,
+                         lam_k, s_k, lam_v, s_v, B, Hq, Hkv, T, D, group,
+                         sm_scale, out, workspace, workspace_bytes, stream) -> status
 
 ``quantize`` / ``dequantize`` accept torch CUDA tensors, allocate outputs
 with torch when none are given, call the C entry point on the current (or
@@ -39,6 +42,11 @@ _lib.kvq_roundtrip.restype = _I
 _lib.kvq_roundtrip.argtypes = [_P, _P, _P, _I64, _I, _I, _P, _P, _P, _P]
 _lib.kvq_dequantize.restype = _I
 _lib.kvq_dequantize.argtypes = [_P, _P, _P, _P, _I64, _I, _I, _P, _P]
+_lib.kvq_attention_decode.restype = _I
+_lib.kvq_attention_decode.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                      _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _I64, _P]
+_lib.kvq_attention_workspace_bytes.restype = _I64
+_lib.kvq_attention_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
 _lib.kvq_status_string.restype = ctypes.c_char_p
 _lib.kvq_status_string.argtypes = [_I]
 _lib.kvq_last_cuda_error.restype = _I
@@ -90,6 +98,20 @@ def kvq_roundtrip(x: int, lam: int, signs: int, n_vec: int, D: int, group: int,
 def kvq_dequantize(packed: int, scales: int, lam: int, signs: int, n_vec: int,
                    D: int, group: int, x_out: int, stream: int = 0) -> int:
     return _lib.kvq_dequantize(packed, scales, lam, signs, n_vec, D, group, x_out, stream)
+
+
+def kvq_attention_decode(q: int, k_packed: int, k_scales: int, v_packed: int, v_scales: int,
+                         seq_len: int, lam_k: int, s_k: int, lam_v: int, s_v: int,
+                         B: int, Hq: int, Hkv: int, T: int, D: int, group: int,
+                         sm_scale: float, out: int, workspace: int = 0,
+                         workspace_bytes: int = 0, stream: int = 0) -> int:
+    return _lib.kvq_attention_decode(q, k_packed, k_scales, v_packed, v_scales, seq_len,
+                                     lam_k, s_k, lam_v, s_v, B, Hq, Hkv, T, D, group,
+                                     sm_scale, out, workspace, workspace_bytes, stream)
+
+
+def kvq_attention_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, D: int, group: int) -> int:
+    return _lib.kvq_attention_workspace_bytes(B, Hq, Hkv, T, D, group)
 
 
 def kvq_status_string(status: int) -> str:
@@ -199,6 +221,54 @@ def roundtrip(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: in
         pk, sc = packed.data_ptr(), scales.data_ptr()
     rc = kvq_roundtrip(x.data_ptr(), lam.data_ptr(), signs.data_ptr(), n, D, group,
                        out.data_ptr(), pk, sc, _stream_handle(stream))
+    if rc != KVQ_OK:
+        raise KvqError(rc)
+    return out
+
+
+def attention_decode(q: torch.Tensor, k_packed: torch.Tensor, k_scales: torch.Tensor,
+                     v_packed: torch.Tensor, v_scales: torch.Tensor, seq_len: torch.Tensor,
+                     lam_k: torch.Tensor, s_k: torch.Tensor, lam_v: torch.Tensor,
+                     s_v: torch.Tensor, group: int, sm_scale: float,
+                     out: torch.Tensor | None = None, workspace: torch.Tensor | bool = True,
+                     stream=None) -> torch.Tensor:
+    """Decode attention over the int4 cache.  q fp16 [B, Hq, D]; packed uint8
+    [B, Hkv, T, D/2]; scales fp16 [B, Hkv, T, D/group]; seq_len int32 [B]
+    -> fp16 [B, Hq, D].  ``workspace``: a uint8 CUDA tensor, True to allocate
+    the size the library asks for, or False to run without splitting."""
+    if q.dim() != 3 or k_packed.dim() != 4:
+        raise ValueError("q must be [B, Hq, D] and the caches [B, Hkv, T, D/2]")
+    B, Hq, D = q.shape
+    Hkv, T = k_packed.shape[1], k_packed.shape[2]
+    _need(q, torch.float16, (B, Hq, D), "q")
+    for name, t in (("k_packed", k_packed), ("v_packed", v_packed)):
+        _need(t, torch.uint8, (B, Hkv, T, D // 2), name)
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        _need(t, torch.float16, (B, Hkv, T, max(D // group, 1)), name)
+    _need(seq_len, torch.int32, (B,), "seq_len")
+    for name, t in (("lambda_k", lam_k), ("lambda_v", lam_v)):
+        _need(t, torch.float32, (D,), name)
+    for name, t in (("signs_k", s_k), ("signs_v", s_v)):
+        _need(t, torch.int8, (D,), name)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device=q.device)
+    _need(out, torch.float16, (B, Hq, D), "out")
+    ws, wsb = 0, 0
+    if workspace is True:
+        need = kvq_attention_workspace_bytes(B, Hq, Hkv, T, D, group)
+        if need > 0:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        else:
+            workspace = None
+    if isinstance(workspace, torch.Tensor):
+        if not workspace.is_cuda or workspace.dtype != torch.uint8:
+            raise ValueError("workspace must be a uint8 CUDA tensor")
+        ws, wsb = workspace.data_ptr(), workspace.numel()
+    rc = kvq_attention_decode(q.data_ptr(), k_packed.data_ptr(), k_scales.data_ptr(),
+                              v_packed.data_ptr(), v_scales.data_ptr(), seq_len.data_ptr(),
+                              lam_k.data_ptr(), s_k.data_ptr(), lam_v.data_ptr(), s_v.data_ptr(),
+                              B, Hq, Hkv, T, D, group, float(sm_scale), out.data_ptr(),
+                              ws, wsb, _stream_handle(stream))
     if rc != KVQ_OK:
         raise KvqError(rc)
     return out

@@ -119,3 +119,22 @@ def test_roundtrip_errors(kvq):
     assert kvq.kvq_roundtrip(A, A, A, 4, 128, 32, A + 8, 0, 0, 0) == -2   # x_hat needs 16
     assert kvq.kvq_roundtrip(A, A, A, 4, 128, 8, A, 0, 0, 0) == -4
     assert kvq.kvq_roundtrip(0, 0, 0, 0, 128, 32, 0, 0, 0, 0) == 0
+
+
+def test_attention_errors(kvq):
+    A_ = A
+    args = lambda **kw: dict(dict(B=1, Hq=32, Hkv=8, T=4096, D=128, G=32), **kw)
+    def call(q=A_, B=1, Hq=32, Hkv=8, T=4096, D=128, G=32, out=A_, lens=A_):
+        return kvq.kvq_attention_decode(q, A_, A_, A_, A_, lens, A_, A_, A_, A_,
+                                        B, Hq, Hkv, T, D, G, 0.1, out)
+    assert call(D=256) == -3 and call(D=96) == -3
+    assert call(G=16) == -4 and call(D=64, G=128) == -4
+    assert call(Hq=40, Hkv=4) == -5          # 10 query heads per KV head
+    assert call(Hq=30) == -5                 # not a multiple of Hkv
+    assert call(T=4000 + 8) == -5            # T % 16 != 0
+    assert call(B=-1) == -5
+    assert call(q=0) == -1 and call(out=0) == -1 and call(lens=0) == -1
+    assert call(q=A_ + 8) == -2 and call(out=A_ + 8) == -2 and call(lens=A_ + 2) == -2
+    assert call(B=0, q=0, out=0, lens=0) == 0
+    assert kvq.kvq_attention_workspace_bytes(1, 32, 8, 4096, 256, 32) == -1
+    assert kvq.kvq_attention_workspace_bytes(4096, 32, 8, 4096, 128, 32) == 0

@@ -1,0 +1,167 @@
+"""Fused decode attention over the int4 cache (kvq_attention_decode) against
+the oracle's double-precision definition.
+
+Tolerance.  The kernel computes the same attention in fp32 with tensor-core
+products: the rotated query is split into fp16 hi + lo parts (relative error
+~2^-22), codes are exact, the scores and the weighted value sums accumulate in
+fp32, p * S_V is split hi + lo again, and the result is rounded once to fp16
+(half an fp16 ulp, 2^-11 relative).  The fp32 parts stay below ~1e-5 of a
+row's largest output, so every output must lie within
+    |out - o| <= 2^-10 |o| + 1e-4 max|o_row|,
+one fp16 ulp plus a small absolute floor for near-zero outputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_quantization_02_b200 import kvq, workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(B, Hq, Hkv, T, D, G, seed, lens=None, dist="uniform"):
+    """Random caches: codes uniform over all nibbles, scales in a realistic
+    range; or, with dist="quantized", rows that are the codes of real
+    quantize calls on Gaussian K/V with outliers."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, Hq, D)).astype(np.float16)
+    lk, sk = workloads.params(D, seed)
+    lv, sv = workloads.params(D, seed + 1)
+    if dist == "uniform":
+        kp = rng.integers(0, 256, (B, Hkv, T, D // 2), dtype=np.uint8)
+        vp = rng.integers(0, 256, (B, Hkv, T, D // 2), dtype=np.uint8)
+        ks = rng.uniform(0.02, 0.5, (B, Hkv, T, D // G)).astype(np.float16)
+        vs = rng.uniform(0.02, 0.5, (B, Hkv, T, D // G)).astype(np.float16)
+    else:
+        o = oracle.get()
+        x = rng.standard_normal((2, B * Hkv * T, D))
+        x[:, :, rng.permutation(D)[:4]] *= 20.0
+        x = x.astype(np.float16)
+        kp, ks = o.quantize(x[0], lk, sk, G)
+        vp, vs = o.quantize(x[1], lv, sv, G)
+        kp = kp.reshape(B, Hkv, T, D // 2)
+        vp = vp.reshape(B, Hkv, T, D // 2)
+        ks = ks.reshape(B, Hkv, T, D // G)
+        vs = vs.reshape(B, Hkv, T, D // G)
+    if lens is None:
+        lens = rng.integers(0, T + 1, B)
+    lens = np.asarray(lens, dtype=np.int32)
+    return dict(q=q, kp=kp, ks=ks, vp=vp, vs=vs, lens=lens, lk=lk, sk=sk, lv=lv, sv=sv, G=G)
+
+
+def _gpu(c, scale, workspace=True):
+    dev = torch.device("cuda")
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    out = kvq.attention_decode(t(c["q"]), t(c["kp"]), t(c["ks"]), t(c["vp"]), t(c["vs"]),
+                               t(c["lens"]), t(c["lk"]), t(c["sk"]), t(c["lv"]), t(c["sv"]),
+                               c["G"], scale, workspace=workspace)
+    torch.cuda.synchronize()
+    return out.cpu().numpy().astype(np.float64)
+
+
+def _oracle(c, scale):
+    return oracle.get().attention_decode(c["q"], c["kp"], c["ks"], c["vp"], c["vs"], c["lens"],
+                                         c["lk"], c["sk"], c["lv"], c["sv"], c["G"], scale)
+
+
+def _check(got, ref):
+    row = np.abs(ref).max(axis=-1, keepdims=True)
+    bound = 2.0 ** -10 * np.abs(ref) + 1e-4 * row
+    err = np.abs(got - ref)
+    worst = float((err - bound).max())
+    assert np.all(err <= bound), f"max excess {worst}, max err {err.max()}"
+    return float(err.max())
+
+
+CASES = [
+    # B, Hq, Hkv, T, D, G, lens
+    (2, 8, 2, 64, 128, 32, [64, 37]),
+    (3, 4, 4, 160, 64, 32, [0, 1, 160]),
+    (2, 16, 2, 96, 128, 64, [17, 96]),
+    (1, 6, 1, 48, 128, 128, [48]),
+    (4, 8, 8, 16, 64, 64, [15, 16, 1, 0]),
+    (2, 32, 8, 208, 128, 32, [65, 208]),
+    (1, 2, 2, 1024, 128, 32, [1000]),          # few pairs: the key axis splits
+    (1, 8, 1, 4096, 64, 32, [4095]),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,D,G,lens", CASES)
+def test_attention_matches_oracle(B, Hq, Hkv, T, D, G, lens):
+    c = _case(B, Hq, Hkv, T, D, G, seed=B * 7 + T, lens=lens)
+    scale = 1.0 / math.sqrt(D)
+    _check(_gpu(c, scale), _oracle(c, scale))
+
+
+@pytest.mark.parametrize("dist", ["quantized"])
+def test_attention_on_quantized_rows(dist):
+    """Rows that are real quantize outputs (peaked softmax from outliers)."""
+    c = _case(2, 8, 2, 256, 128, 32, seed=5, lens=[256, 131], dist=dist)
+    for scale in (1.0 / math.sqrt(128), 0.3):
+        _check(_gpu(c, scale), _oracle(c, scale))
+
+
+def test_split_and_unsplit_agree():
+    """With and without workspace (split key axis vs one pass): both match
+    the oracle; they differ only in fp32 summation order."""
+    c = _case(1, 4, 2, 2048, 128, 32, seed=11, lens=[1999])
+    assert kvq.kvq_attention_workspace_bytes(1, 4, 2, 2048, 128, 32) > 0
+    ref = _oracle(c, 0.1)
+    a = _gpu(c, 0.1, workspace=True)
+    b = _gpu(c, 0.1, workspace=False)
+    _check(a, ref)
+    _check(b, ref)
+
+
+def test_extreme_scales_and_zero_length():
+    c = _case(3, 4, 1, 64, 128, 32, seed=13, lens=[64, 0, 9])
+    for scale in (0.0, 1e-3, 5.0):
+        got = _gpu(c, scale)
+        _check(got, _oracle(c, scale))
+    assert np.all(got[1] == 0.0)
+
+
+def test_bad_length_is_clamped_and_flagged():
+    kvq.kvq_fault_status(True)
+    c = _case(2, 4, 2, 32, 128, 32, seed=17, lens=[40, 32])
+    got = _gpu(c, 0.2)
+    assert kvq.kvq_fault_status(True) & 8
+    c["lens"] = np.array([32, 32], dtype=np.int32)
+    _check(got, _oracle(c, 0.2))
+    assert kvq.kvq_fault_status(False) == 0
+
+
+def test_decode_config_sampled():
+    """The bench's decode shape (a 64-sequence batch x 36 layers folded into
+    B, 8 KV heads, 32 query heads, 4096 positions) on a slice of sequences,
+    sampled rows checked against the oracle one (sequence, KV head) at a time."""
+    B, Hq, Hkv, T, D, G = 48, 32, 8, 4096, 128, 32
+    dev = torch.device("cuda")
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4)
+    kp = torch.randint(0, 256, (B, Hkv, T, D // 2), dtype=torch.uint8, device=dev, generator=gen)
+    vp = torch.randint(0, 256, (B, Hkv, T, D // 2), dtype=torch.uint8, device=dev, generator=gen)
+    ks = (torch.rand((B, Hkv, T, D // G), device=dev, generator=gen) * 0.4 + 0.02).half()
+    vs = (torch.rand((B, Hkv, T, D // G), device=dev, generator=gen) * 0.4 + 0.02).half()
+    q = torch.randn((B, Hq, D), device=dev, generator=gen).half()
+    lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+    lens[::5] = 1234
+    lk, sk = workloads.params(D, 4)
+    lv, sv = workloads.params(D, 5)
+    t = lambda a: torch.from_numpy(a).to(dev)
+    out = kvq.attention_decode(q, kp, ks, vp, vs, lens, t(lk), t(sk), t(lv), t(sv), G,
+                               1.0 / math.sqrt(D))
+    torch.cuda.synchronize()
+    R = Hq // Hkv
+    for b, kvh in ((0, 0), (5, 7), (47, 3)):
+        L = int(lens[b])
+        sub = dict(q=q[b:b + 1, kvh * R:(kvh + 1) * R].cpu().numpy(),
+                   kp=kp[b:b + 1, kvh:kvh + 1].cpu().numpy(), ks=ks[b:b + 1, kvh:kvh + 1].cpu().numpy(),
+                   vp=vp[b:b + 1, kvh:kvh + 1].cpu().numpy(), vs=vs[b:b + 1, kvh:kvh + 1].cpu().numpy(),
+                   lens=np.array([L], dtype=np.int32), lk=lk, sk=sk, lv=lv, sv=sv, G=G)
+        ref = _oracle(sub, 1.0 / math.sqrt(D))[0]
+        got = out[b, kvh * R:(kvh + 1) * R].cpu().numpy().astype(np.float64)
+        _check(got, ref)
