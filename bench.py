@@ -389,12 +389,64 @@ def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w):
     ap_ms = _event_ms(torch, stream, lambda: kvq.quantize_rows(
         xa, lam_t, s_t, G, idx, cpk, csc, stream=stream), 50)
     del xa, cpk, csc
-    return {
+    res = {
         "roundtrip_ms": round(rt_ms, 5),
         "roundtrip_gbs": round(n * 4 * D / (rt_ms / 1e3) / 1e9, 1),
         "decode_append_vectors": na,
         "decode_append_us": round(ap_ms * 1e3, 2),
         "decode_append_gvec_s": round(na / (ap_ms / 1e3) / 1e9, 3),
+    }
+    if D == 128:
+        res["attention_decode"] = run_attention(torch, kvq, dev, stream, lam_t, s_t, G)
+    return res
+
+
+def run_attention(torch, kvq, dev, stream, lam_t, s_t, G):
+    """One decode step of attention over the whole int4 cache of the decode
+    configuration: 64 sequences x 36 layers (folded into the batch) x 8 KV
+    heads x 4096 positions, 32 query heads (Qwen3-8B's grouping), D = 128.
+    The cache holds real quantize output of N(0,1) rows.  Algorithmic bytes:
+    every K and V code and scale once, plus q and the output."""
+    c = workloads.WORKLOADS["decode-cache"]
+    B, Hq, Hkv, T, D = 64 * 36, 32, 8, 4096, 128
+    rows = B * Hkv * T
+    kp = torch.empty((B, Hkv, T, D // 2), dtype=torch.uint8, device=dev)
+    vp = torch.empty_like(kp)
+    ks = torch.empty((B, Hkv, T, D // G), dtype=torch.float16, device=dev)
+    vs = torch.empty_like(ks)
+    chunk = 1 << 23
+    buf = torch.empty((chunk, D), dtype=torch.float16, device=dev)
+    for j, (pk, sc) in enumerate(((kp, ks), (vp, vs))):
+        pk2, sc2 = pk.view(rows, D // 2), sc.view(rows, D // G)
+        for i, a in enumerate(range(0, rows, chunk)):
+            b = min(rows, a + chunk)
+            xr = workloads.device_rows(c, b - a, dev, seed_offset=2 * i + j, out=buf[: b - a])
+            kvq.quantize(xr, lam_t, s_t, G, packed=pk2[a:b], scales=sc2[a:b], stream=stream)
+    del buf
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(c.seed)
+    q = torch.randn((B, Hq, D), device=dev, generator=gen).half()
+    lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    need = kvq.kvq_attention_workspace_bytes(B, Hq, Hkv, T, D, G)
+    ws = torch.empty(max(need, 0), dtype=torch.uint8, device=dev) if need > 0 else False
+    scale = 1.0 / math.sqrt(D)
+    ms = _event_ms(torch, stream, lambda: kvq.attention_decode(
+        q, kp, ks, vp, vs, lens, lam_t, s_t, lam_t, s_t, G, scale, out=out,
+        workspace=ws, stream=stream), 10)
+    byts = 2 * rows * (D // 2 + 2 * (D // G)) + 2 * q.numel() * 2
+    peak, kind = hbm_peak()
+    gbs = byts / (ms / 1e3) / 1e9
+    del kp, vp, ks, vs, q, out
+    torch.cuda.empty_cache()
+    return {
+        "shape": f"B={B} (64 sequences x 36 layers), Hq={Hq}, Hkv={Hkv}, T={T}, D={D}, G={G}",
+        "ms": round(ms, 4),
+        "algorithmic_bytes": byts,
+        "gbs": round(gbs, 1),
+        "gkeys_s": round(B * Hkv * T / (ms / 1e3) / 1e9, 2),
+        "frac_of_peak": round(gbs / peak, 4),
+        "peak_kind": kind,
     }
 
 

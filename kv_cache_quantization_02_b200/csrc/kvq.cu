@@ -908,26 +908,6 @@ int grid_for(Kernel k, int64_t n, int smem) {
   return static_cast<int>(need < cap ? need : cap);
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// cuTensorMapEncodeTiled, resolved once through the runtime (no libcuda link).
-EncodeTiledFn encode_tiled() {
-  static std::atomic<EncodeTiledFn> fn{nullptr};
-  EncodeTiledFn f = fn.load(std::memory_order_acquire);
-  if (f == nullptr) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess && p != nullptr) {
-      f = reinterpret_cast<EncodeTiledFn>(p);
-      fn.store(f, std::memory_order_release);
-    }
-  }
-  return f;
-}
 
 // One 2-D map per 64-channel quarter of the fp16 rows at `base`: 64 channels
 // x n rows, row stride 2D bytes, box 64 x ROWS, 128-byte swizzle.

@@ -1,6 +1,7 @@
-// kvq_async.cuh -- inline-PTX helpers shared by the library's kernels:
-// mbarriers with bounded waits, bulk and tensor copies between global and
-// shared memory (never with multicast), and the async-proxy fence.
+// kvq_async.cuh -- helpers shared by the library's translation units: inline
+// PTX for mbarriers with bounded waits, bulk and tensor copies between global
+// and shared memory (never with multicast) and the async-proxy fence; on the
+// host, the driver's tensor-map encoder resolved through the runtime.
 // Included inside each translation unit's anonymous namespace.
 #pragma once
 
@@ -49,3 +50,23 @@ __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled, resolved once through the runtime (no libcuda link).
+EncodeTiledFn encode_tiled() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (f == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && p != nullptr) {
+      f = reinterpret_cast<EncodeTiledFn>(p);
+      fn.store(f, std::memory_order_release);
+    }
+  }
+  return f;
+}

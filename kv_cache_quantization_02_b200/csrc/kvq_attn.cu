@@ -19,22 +19,26 @@
 // Work decomposition.  A block of four warps owns one (sequence, KV head,
 // key split); each warp streams 64-key blocks (codes and scales of K and V,
 // four bulk copies into a private double-buffered ring) and keeps its own
-// online-softmax state; the block merges the four states at the end.  Both
-// products run on the tensor cores as m16n8k16 fp16 MMAs with fp32
+// online-softmax state, updated once per block; the block merges the four
+// states at the end.
+// Both products run on the tensor cores as m16n8k16 fp16 MMAs with fp32
 // accumulation, the query heads of the KV head on the M rows:
 //   * scores: rows 0..R-1 hold the fp16 high parts of q~, rows 8..8+R-1 the
 //     fp16 residuals (q~ = hi + lo to ~2^-22), the N columns are 8 keys and
 //     the K dimension 16 channels.  The channel order inside each 32-channel
-//     block is permuted so that a lane's B fragment for one k-step is the two
-//     nibbles of each of two consecutive code bytes, and every k-step stays
-//     inside one scale group: the group's scale multiplies the per-group
-//     partial sums, key by key, after the MMA.
+//     block is permuted so that a lane's B fragments for two k-steps are the
+//     four nibble pairs of one 32-bit word of codes (nibbles k and k + 16 of
+//     the word), and every k-step stays inside one scale group: the group's
+//     scale multiplies the per-group partial sums, key by key, after the MMA.
 //   * values: the score fragments are already in the A layout of the value
 //     product (rows = heads, K dimension = 16 keys), so p * S_V (split hi/lo
 //     the same way) feeds it directly, one A fragment per scale group; the B
 //     fragments pair the same channel of two keys.
-// Codes become exact fp16 integers with a byte permute, a mask and one fp16
-// subtraction (the biased nibble n sits in the low bits of 1024's encoding).
+// A biased code n = q + 8 in [0, 15] is used as the fp16 subnormal n 2^-24,
+// exact and made by one mask-and-xor: sum_k a_k q_k = 2^24 sum_k a_k n_k 2^-24
+// - 8 sum_k a_k.  The key side starts its accumulators at -8 2^-24 sum a (a
+// constant of the query); the value side keeps the running sum of p * S_V per
+// group and subtracts it once at the end.
 //
 // Every mbarrier wait is bounded; a warp that gives up sets the fault word
 // and the block still finishes (its output is then meaningless).  A sequence
@@ -62,6 +66,7 @@ constexpr uint32_t kSpin = 1u << 22;         // bounded mbarrier waits
 constexpr int kMaxRows = 8;                  // query heads per KV head (M rows of one MMA half)
 
 __device__ unsigned int g_attn_fault = 0;    // bit 0: a wait gave up; bit 3: bad sequence length
+
 thread_local int g_attn_cuda_error = 0;
 
 struct AttnParams {
@@ -78,7 +83,7 @@ struct AttnParams {
   uint16_t* out;                // fp16 [B][Hq][D]
   float* part;                  // [B*Hkv*nsplit][R][D + 4] when nsplit > 1
   int Hkv, T, R, nsplit, chunk;
-  float scale_log2;             // sm_scale * log2(e)
+  float scale_log2;             // sm_scale * log2(e) * 2^24 (the key product comes out scaled by 2^-24)
   float c;                      // fp32 1/sqrt(D)
 };
 
@@ -100,20 +105,11 @@ struct Attn {
   static constexpr int DPL = D / 32;                // channels per lane in the row transforms
 };
 
-// fp16x2 (low nibble, high nibble) of byte `beta` of a code word, as exact
-// fp16 integers q in [-8, 7]: w holds the codes xor 0x88 (n = q + 8), w4 = w >> 4.
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w, uint32_t w4, int beta) {
-  const uint32_t x = (__byte_perm(w, w4, static_cast<uint32_t>(beta | ((4 + beta) << 8))) & 0x000F000Fu) | 0x64006400u;
-  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&x), __floats2half2_rn(1032.0f, 1032.0f));
-  return *reinterpret_cast<const uint32_t*>(&r);
+// A biased code pair as fp16 subnormals: nibbles at bits 0-3 and 16-19 of x,
+// n = q + 8 (xor 8 of the two's-complement nibble), value n 2^-24, exact.
+__device__ __forceinline__ uint32_t sub_pair(uint32_t x) {
+  return (x & 0x000F000Fu) ^ 0x00080008u;
 }
-// fp16x2 (code of key a, code of key b) at the same nibble of byte `beta`.
-__device__ __forceinline__ uint32_t key_pair(uint32_t wa, uint32_t wb, int beta) {
-  const uint32_t x = (__byte_perm(wa, wb, static_cast<uint32_t>(beta | ((4 + beta) << 8))) & 0x000F000Fu) | 0x64006400u;
-  const __half2 r = __hsub2(*reinterpret_cast<const __half2*>(&x), __floats2half2_rn(1032.0f, 1032.0f));
-  return *reinterpret_cast<const uint32_t*>(&r);
-}
-
 __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
                : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -238,16 +234,34 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   }
   __syncthreads();
 
-  // Score-product A fragments, k-step j = (32-channel block j/2, half j%2):
-  // k-index 2t, 2t+1 <-> channels 32(j/2) + 8t + 4(j%2) + {0,1}; 2t+8, 2t+9 <-> +{2,3}.
+  // Score-product A fragments.  k-step j = (32-channel block bb = j/2, half
+  // h = j%2); with c0 = 32 bb + 8 t + 2 h, k-indices (2t, 2t+1) are channels
+  // (c0, c0 + 4) and (2t+8, 2t+9) are (c0 + 1, c0 + 5): nibbles (k, k + 16)
+  // of the lane's code word 4 bb + t, k = 0, 4 (h = 0) or 8, 12 (h = 1).
+  auto qpair = [&](int row, int d0, int d1) -> uint32_t {
+    return static_cast<uint32_t>(__half_as_ushort(qt[row * D + d0])) |
+           (static_cast<uint32_t>(__half_as_ushort(qt[row * D + d1])) << 16);
+  };
   uint32_t Aq[KS][4];
 #pragma unroll
   for (int j = 0; j < KS; ++j) {
-    const int d0 = 32 * (j >> 1) + 8 * t + 4 * (j & 1);
-    Aq[j][0] = *reinterpret_cast<const uint32_t*>(qt + g * D + d0);
-    Aq[j][1] = *reinterpret_cast<const uint32_t*>(qt + (kMaxRows + g) * D + d0);
-    Aq[j][2] = *reinterpret_cast<const uint32_t*>(qt + g * D + d0 + 2);
-    Aq[j][3] = *reinterpret_cast<const uint32_t*>(qt + (kMaxRows + g) * D + d0 + 2);
+    const int c0 = 32 * (j >> 1) + 8 * t + 2 * (j & 1);
+    Aq[j][0] = qpair(g, c0, c0 + 4);
+    Aq[j][1] = qpair(kMaxRows + g, c0, c0 + 4);
+    Aq[j][2] = qpair(g, c0 + 1, c0 + 5);
+    Aq[j][3] = qpair(kMaxRows + g, c0 + 1, c0 + 5);
+  }
+  // Bias of the biased codes: -8 2^-24 times each row's sum over a group.
+  float bias_hi[NG], bias_lo[NG];
+#pragma unroll
+  for (int gi = 0; gi < NG; ++gi) {
+    float sh = 0.0f, sl = 0.0f;
+    for (int d = gi * G; d < (gi + 1) * G; ++d) {
+      sh += __half2float(qt[g * D + d]);
+      sl += __half2float(qt[(kMaxRows + g) * D + d]);
+    }
+    bias_hi[gi] = -8.0f * 0x1p-24f * sh;
+    bias_lo[gi] = -8.0f * 0x1p-24f * sl;
   }
 
   const int64_t row_base = static_cast<int64_t>(bh) * P.T;
@@ -271,6 +285,9 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   float O[NT][4];
 #pragma unroll
   for (int n = 0; n < NT; ++n) O[n][0] = O[n][1] = O[n][2] = O[n][3] = 0.0f;
+  float psum[NG];                      // running sum of p * S_V per group (this lane's keys)
+#pragma unroll
+  for (int gi = 0; gi < NG; ++gi) psum[gi] = 0.0f;
   float m = -INFINITY, l = 0.0f;
   bool failed = false;
   int k = 0;
@@ -297,20 +314,18 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
 #pragma unroll
       for (int gi = 0; gi < NG; ++gi)
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) acc[gi][nt][0] = acc[gi][nt][1] = acc[gi][nt][2] = acc[gi][nt][3] = 0.0f;
+        for (int nt = 0; nt < 2; ++nt) {
+          acc[gi][nt][0] = acc[gi][nt][1] = bias_hi[gi];
+          acc[gi][nt][2] = acc[gi][nt][3] = bias_lo[gi];
+        }
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         const int kk = 16 * sb + 8 * nt + g;
-        uint32_t w[NB], w4[NB];
 #pragma unroll
         for (int bb = 0; bb < NB; ++bb) {
-          w[bb] = kc[kk * W32 + 4 * bb + t] ^ 0x88888888u;
-          w4[bb] = w[bb] >> 4;
-        }
-#pragma unroll
-        for (int j = 0; j < KS; ++j) {
-          const int bb = j >> 1, h = j & 1;
-          mma16816(acc[(32 * bb) / G][nt], Aq[j], nib_pair(w[bb], w4[bb], 2 * h), nib_pair(w[bb], w4[bb], 2 * h + 1));
+          const uint32_t w = kc[kk * W32 + 4 * bb + t];
+          mma16816(acc[(32 * bb) / G][nt], Aq[2 * bb], sub_pair(w), sub_pair(w >> 4));
+          mma16816(acc[(32 * bb) / G][nt], Aq[2 * bb + 1], sub_pair(w >> 8), sub_pair(w >> 12));
         }
       }
 #pragma unroll
@@ -337,10 +352,14 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     const float mnew = fmaxf(m, mx);
     const float alpha = (mnew == -INFINITY) ? 1.0f : exp2f(m - mnew);
     m = mnew;
-    l *= alpha;
+    if (__any_sync(kFull, alpha != 1.0f)) {     // skipped once the running maxima settle
+      l *= alpha;
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      O[n][0] *= alpha; O[n][1] *= alpha; O[n][2] *= alpha; O[n][3] *= alpha;
+      for (int gi = 0; gi < NG; ++gi) psum[gi] *= alpha;
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        O[n][0] *= alpha; O[n][1] *= alpha; O[n][2] *= alpha; O[n][3] *= alpha;
+      }
     }
 #pragma unroll
     for (int sb = 0; sb < kBK / 16; ++sb) {
@@ -362,6 +381,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
           // masked keys may sit on stale scale bytes: keep their weight exactly 0
           const float pa = p[nt][0] == 0.0f ? 0.0f : p[nt][0] * __half2float(vsc[key * NG + gi]);
           const float pb = p[nt][1] == 0.0f ? 0.0f : p[nt][1] * __half2float(vsc[(key + 1) * NG + gi]);
+          psum[gi] += pa + pb;
           const __half2 hi = __floats2half2_rn(pa, pb);
           const float2 hf = __half22float2(hi);
           Ap[gi][2 * nt] = h2bits(hi);
@@ -374,19 +394,17 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
 #pragma unroll
       for (int bb = 0; bb < NB; ++bb) {
         const int wi = 4 * bb + (g >> 1);
-        const uint32_t a0 = vc[ka * W32 + wi] ^ 0x88888888u;
-        const uint32_t a1 = vc[(ka + 1) * W32 + wi] ^ 0x88888888u;
-        const uint32_t c0 = vc[(ka + 8) * W32 + wi] ^ 0x88888888u;
-        const uint32_t c1 = vc[(ka + 9) * W32 + wi] ^ 0x88888888u;
-        const uint32_t a04 = a0 >> 4, a14 = a1 >> 4, c04 = c0 >> 4, c14 = c1 >> 4;
+        const uint32_t a0 = vc[ka * W32 + wi], a1 = vc[(ka + 1) * W32 + wi];
+        const uint32_t c0 = vc[(ka + 8) * W32 + wi], c1 = vc[(ka + 9) * W32 + wi];
+        const uint32_t sel0 = static_cast<uint32_t>(2 * (g & 1)) | ((4u + 2 * (g & 1)) << 8);
+        const uint32_t sel1 = sel0 + 0x101u;
+        const uint32_t xa0 = __byte_perm(a0, a1, sel0), xa1 = __byte_perm(a0, a1, sel1);
+        const uint32_t xc0 = __byte_perm(c0, c1, sel0), xc1 = __byte_perm(c0, c1, sel1);
         const int gi = (32 * bb) / G;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int beta = 2 * (g & 1) + (u >> 1);
-          const uint32_t b0 = (u & 1) ? key_pair(a04, a14, beta) : key_pair(a0, a1, beta);
-          const uint32_t b1 = (u & 1) ? key_pair(c04, c14, beta) : key_pair(c0, c1, beta);
-          mma16816(O[4 * bb + u], Ap[gi], b0, b1);
-        }
+        mma16816(O[4 * bb + 0], Ap[gi], sub_pair(xa0), sub_pair(xc0));
+        mma16816(O[4 * bb + 1], Ap[gi], sub_pair(xa0 >> 4), sub_pair(xc0 >> 4));
+        mma16816(O[4 * bb + 2], Ap[gi], sub_pair(xa1), sub_pair(xc1));
+        mma16816(O[4 * bb + 3], Ap[gi], sub_pair(xa1 >> 4), sub_pair(xc1 >> 4));
       }
     }
     __syncwarp();                      // the stage is consumed: refill it
@@ -402,14 +420,20 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   }
   l += __shfl_xor_sync(kFull, l, 1);
   l += __shfl_xor_sync(kFull, l, 2);
+#pragma unroll
+  for (int gi = 0; gi < NG; ++gi) {
+    psum[gi] += __shfl_xor_sync(kFull, psum[gi], 1);
+    psum[gi] += __shfl_xor_sync(kFull, psum[gi], 2);
+  }
   __syncthreads();                     // every warp is out of the ring: reuse it for the merge
   if (g < R) {
     float* cw = comb + (warp * kMaxRows + g) * D;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
       const int bb = n >> 2, u = n & 3;
-      cw[32 * bb + 8 * t + u] = O[n][0] + O[n][2];
-      cw[32 * bb + 8 * t + 4 + u] = O[n][1] + O[n][3];
+      const float corr = 8.0f * psum[(32 * bb) / G];
+      cw[32 * bb + 8 * t + u] = __fmaf_rn(O[n][0] + O[n][2], 0x1p24f, -corr);
+      cw[32 * bb + 8 * t + 4 + u] = __fmaf_rn(O[n][1] + O[n][3], 0x1p24f, -corr);
     }
     if (t == 0) {
       ml[(warp * kMaxRows + g) * 2] = m;
@@ -595,7 +619,8 @@ int kvq_attention_decode(const uint16_t* q, const uint8_t* k_packed, const uint1
   P.out = out;
   P.part = static_cast<float*>(workspace);
   P.Hkv = Hkv; P.T = T; P.R = Hq / Hkv; P.nsplit = sp.nsplit; P.chunk = sp.chunk;
-  P.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  // scores come out of the key product scaled by 2^-24 (subnormal codes)
+  P.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634 * 16777216.0);
   P.c = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (D * 1000 + group) {
