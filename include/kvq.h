@@ -206,6 +206,25 @@ int kvq_attention_decode(const uint16_t *q, const uint8_t *k_packed,
 int64_t kvq_attention_workspace_bytes(int B, int Hq, int Hkv, int T, int D, int group);
 
 /*
+ * kvq_attention_decode_static -- kvq_attention_decode without a caller
+ * workspace and without any allocation: the key-split scratch is a static
+ * 8 MiB device array inside the library (one per device, its address looked
+ * up once).  The pages have no counterpart of this entry point; it exists for
+ * callers that cannot hand out device memory.  Same arguments, results and
+ * checks as kvq_attention_decode; returns KVQ_ERR_COUNT when the shapes need
+ * more split scratch than 8 MiB (kvq_attention_workspace_bytes() > 8 MiB).
+ * Calls that overlap in time share the scratch and race: serialise them (one
+ * stream, or events between streams and host threads).
+ */
+int kvq_attention_decode_static(const uint16_t *q, const uint8_t *k_packed,
+                                const uint16_t *k_scales, const uint8_t *v_packed,
+                                const uint16_t *v_scales, const int32_t *seq_len,
+                                const float *lambda_k, const int8_t *signs_k,
+                                const float *lambda_v, const int8_t *signs_v,
+                                int B, int Hq, int Hkv, int T, int D, int group,
+                                float sm_scale, uint16_t *out, void *stream);
+
+/*
  * kvq_fault_status -- the current device's fault word: 0 when every bounded
  * wait of every kernel so far completed; bit 0 set when a quantize,
  * dequantize or attention block gave up waiting for its bulk copies (its

@@ -67,6 +67,13 @@ constexpr int kMaxRows = 8;                  // query heads per KV head (M rows 
 
 __device__ unsigned int g_attn_fault = 0;    // bit 0: a wait gave up; bit 3: bad sequence length
 
+// Scratch of kvq_attention_decode_static: the partial (max, sum, rotated
+// output) rows of the key splits, 8 MiB per device.  Nothing in it has to
+// start at zero: every split writes its own slots before the merge kernel,
+// later on the same stream, reads them.  Calls that overlap in time (other
+// streams, other host threads) share it and race.
+constexpr int64_t kStaticScratchBytes = int64_t{8} << 20;
+static __device__ __align__(256) unsigned char g_attn_static_scratch[kStaticScratchBytes];
 thread_local int g_attn_cuda_error = 0;
 
 struct AttnParams {
@@ -581,6 +588,28 @@ __attribute__((visibility("hidden"))) unsigned int kvq_attn_fault_word(int clear
 }
 __attribute__((visibility("hidden"))) int kvq_attn_last_cuda_error() { return g_attn_cuda_error; }
 
+// Device address of the static scratch, looked up once per device.
+void* static_scratch(int& rc) {
+  static std::atomic<void*> cache[64];
+  int dev = 0;
+  rc = KVQ_OK;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    rc = KVQ_ERR_LAUNCH;
+    return nullptr;
+  }
+  void* p = cache[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_attn_static_scratch);
+    if (e != cudaSuccess || p == nullptr) {
+      g_attn_cuda_error = static_cast<int>(e);
+      rc = KVQ_ERR_LAUNCH;
+      return nullptr;
+    }
+    cache[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
+
 extern "C" {
 
 int64_t kvq_attention_workspace_bytes(int B, int Hq, int Hkv, int T, int D, int group) {
@@ -631,6 +660,28 @@ int kvq_attention_decode(const uint16_t* q, const uint8_t* k_packed, const uint1
     case 128128: return launch_attn<128, 128>(P, pairs, st);
     default: return KVQ_ERR_GROUP;
   }
+}
+
+int kvq_attention_decode_static(const uint16_t* q, const uint8_t* k_packed, const uint16_t* k_scales,
+                                const uint8_t* v_packed, const uint16_t* v_scales,
+                                const int32_t* seq_len, const float* lambda_k,
+                                const int8_t* signs_k, const float* lambda_v,
+                                const int8_t* signs_v, int B, int Hq, int Hkv, int T, int D,
+                                int group, float sm_scale, uint16_t* out, void* stream) {
+  const int rc = check_attn(B, Hq, Hkv, T, D, group);
+  if (rc != KVQ_OK) return rc;
+  const int64_t pairs = static_cast<int64_t>(B) * Hkv;
+  const int64_t need = part_bytes(pairs, Hq / Hkv, D, choose_split(pairs, T).nsplit);
+  if (need > kStaticScratchBytes) return KVQ_ERR_COUNT;      // more than the static scratch holds
+  void* ws = nullptr;
+  if (need > 0 && B > 0) {
+    int src = KVQ_OK;
+    ws = static_scratch(src);
+    if (src != KVQ_OK) return src;
+  }
+  return kvq_attention_decode(q, k_packed, k_scales, v_packed, v_scales, seq_len, lambda_k, signs_k,
+                              lambda_v, signs_v, B, Hq, Hkv, T, D, group, sm_scale, out, ws, need,
+                              stream);
 }
 
 }  // extern "C"

@@ -45,6 +45,9 @@ _lib.kvq_dequantize.argtypes = [_P, _P, _P, _P, _I64, _I, _I, _P, _P]
 _lib.kvq_attention_decode.restype = _I
 _lib.kvq_attention_decode.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _I64, _P]
+_lib.kvq_attention_decode_static.restype = _I
+_lib.kvq_attention_decode_static.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                             _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P]
 _lib.kvq_attention_workspace_bytes.restype = _I64
 _lib.kvq_attention_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
 _lib.kvq_status_string.restype = ctypes.c_char_p
@@ -108,6 +111,15 @@ def kvq_attention_decode(q: int, k_packed: int, k_scales: int, v_packed: int, v_
     return _lib.kvq_attention_decode(q, k_packed, k_scales, v_packed, v_scales, seq_len,
                                      lam_k, s_k, lam_v, s_v, B, Hq, Hkv, T, D, group,
                                      sm_scale, out, workspace, workspace_bytes, stream)
+
+
+def kvq_attention_decode_static(q: int, k_packed: int, k_scales: int, v_packed: int,
+                                v_scales: int, seq_len: int, lam_k: int, s_k: int, lam_v: int,
+                                s_v: int, B: int, Hq: int, Hkv: int, T: int, D: int, group: int,
+                                sm_scale: float, out: int, stream: int = 0) -> int:
+    return _lib.kvq_attention_decode_static(q, k_packed, k_scales, v_packed, v_scales, seq_len,
+                                            lam_k, s_k, lam_v, s_v, B, Hq, Hkv, T, D, group,
+                                            sm_scale, out, stream)
 
 
 def kvq_attention_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, D: int, group: int) -> int:
