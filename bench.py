@@ -44,8 +44,7 @@ from kv_cache_quantization_02_b200 import workloads  # noqa: E402
 METRIC = "Gvec/s quantize+pack and dequant at D=128; achieved HBM GB/s vs B200 peak"
 UNIT = "Gvec/s"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCE = os.path.join(ROOT, "kv_cache_quantization_02_b200", "csrc", "kvq.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "kvq_traffic_qwen3_8b.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "kvq_traffic_full_size.json")
 
 
 def bytes_per_vector(D: int, G: int) -> int:
@@ -162,25 +161,27 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_sha() -> str:
-    with open(KERNEL_SOURCE, "rb") as f:
+def source_sha(path: str) -> str:
+    with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()
 
 
-def traffic_per_launch(kernel: str, n_vec: int):
-    """DRAM bytes per launch from the committed ncu summary, scaled by vectors,
-    or None when the kernel source changed since those counters were taken."""
+def traffic_per_launch(kernel: str, units: int):
+    """DRAM bytes per launch from the committed ncu summary, scaled by the
+    units one launch processes (vectors, or cache rows for the attention), or
+    None when that kernel's source changed since the counters were taken."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
     except Exception:  # noqa: BLE001
         return None
-    if t.get("kernel_source_sha256") != kernel_source_sha():
-        return None
     k = t.get("kernels", {}).get(kernel)
     if not k:
         return None
-    return k["dram_bytes_per_vector"] * n_vec
+    src = os.path.join(ROOT, k.get("source", ""))
+    if not os.path.isfile(src) or k.get("source_sha256") != source_sha(src):
+        return None
+    return k["dram_bytes_per_unit"] * units
 
 
 # ---------------------------------------------------------------------------
@@ -293,7 +294,7 @@ def run_gpu(args):
 
     extra = {}
     if not args.no_extra:
-        extra = run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w)
+        extra = run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, args.attn_seqs)
 
     bpv = bytes_per_vector(D, G)
     total_vec = n * world
@@ -372,7 +373,7 @@ def _event_ms(torch, stream, fn, reps):
     return t[len(t) // 2]
 
 
-def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w):
+def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, attn_seqs=64):
     """Secondary figures, outside the timed steps: the fused round trip on the
     same batch, and the decode-time append of one new K and V token for 64
     sequences x 36 layers x 8 KV heads into their rows of a cache."""
@@ -397,18 +398,19 @@ def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w):
         "decode_append_gvec_s": round(na / (ap_ms / 1e3) / 1e9, 3),
     }
     if D == 128:
-        res["attention_decode"] = run_attention(torch, kvq, dev, stream, lam_t, s_t, G)
+        res["attention_decode"] = run_attention(torch, kvq, dev, stream, lam_t, s_t, G, attn_seqs)
     return res
 
 
-def run_attention(torch, kvq, dev, stream, lam_t, s_t, G):
+def run_attention(torch, kvq, dev, stream, lam_t, s_t, G, seqs=64):
     """One decode step of attention over the whole int4 cache of the decode
     configuration: 64 sequences x 36 layers (folded into the batch) x 8 KV
-    heads x 4096 positions, 32 query heads (Qwen3-8B's grouping), D = 128.
-    The cache holds real quantize output of N(0,1) rows.  Algorithmic bytes:
-    every K and V code and scale once, plus q and the output."""
+    heads x 4096 positions, 32 query heads (Qwen3-8B's grouping), D = 128
+    (`seqs` other than 64 only for small profiling runs).  The cache holds
+    real quantize output of N(0,1) rows.  Algorithmic bytes: every K and V
+    code and scale once, plus q and the output."""
     c = workloads.WORKLOADS["decode-cache"]
-    B, Hq, Hkv, T, D = 64 * 36, 32, 8, 4096, 128
+    B, Hq, Hkv, T, D = seqs * 36, 32, 8, 4096, 128
     rows = B * Hkv * T
     kp = torch.empty((B, Hkv, T, D // 2), dtype=torch.uint8, device=dev)
     vp = torch.empty_like(kp)
@@ -440,13 +442,14 @@ def run_attention(torch, kvq, dev, stream, lam_t, s_t, G):
     del kp, vp, ks, vs, q, out
     torch.cuda.empty_cache()
     return {
-        "shape": f"B={B} (64 sequences x 36 layers), Hq={Hq}, Hkv={Hkv}, T={T}, D={D}, G={G}",
+        "shape": f"B={B} ({seqs} sequences x 36 layers), Hq={Hq}, Hkv={Hkv}, T={T}, D={D}, G={G}",
         "ms": round(ms, 4),
         "algorithmic_bytes": byts,
         "gbs": round(gbs, 1),
         "gkeys_s": round(B * Hkv * T / (ms / 1e3) / 1e9, 2),
         "frac_of_peak": round(gbs / peak, 4),
         "peak_kind": kind,
+        "traffic": traffic_per_launch("kvq_attention", rows),
     }
 
 
@@ -549,7 +552,8 @@ def parse(argv=None):
     p.add_argument("--n-vec", type=int, default=None, help="override vectors per GPU (profiling)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
-    p.add_argument("--no-extra", action="store_true", help="skip round-trip and append figures")
+    p.add_argument("--no-extra", action="store_true", help="skip round-trip, append and attention figures")
+    p.add_argument("--attn-seqs", type=int, default=64, help="sequences of the attention figure (profiling)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--e2e-chunks", type=int, default=16)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
