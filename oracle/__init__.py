@@ -81,6 +81,8 @@ class Oracle:
             "kvqo_dequantize_f32": (_I, [_P, _P, _P, _P, _I64, _I, _I, _P]),
             "kvqo_pack": (None, [_P, _I64, _P]),
             "kvqo_unpack": (None, [_P, _I64, _P]),
+            "kvqo_quantize_ex": (_I, [_P, _P, _P, _I64, _I, _I, _I, _I, _I64, _I, _P, _P]),
+            "kvqo_dequantize_ex": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _I64, _I, _P]),
             "kvqo_attention_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            _I, _I, _I, _I, _I, _I, ctypes.c_double, _P]),
         }
@@ -209,6 +211,39 @@ class Oracle:
         self._lib.kvqo_unpack(_ptr(packed), packed.size * 2, _ptr(out))
         return out
 
+
+    def quantize_ex(self, x_f16, lam, signs, group: int, bits: int = 4, lambda_after: bool = False,
+                    lambda_rows: int | None = None):
+        """Format variants: lam is [n_lambda, D] (or [D]); row r uses table
+        (r // lambda_rows) % n_lambda.  Returns (codes uint8 [n, D/2 or D],
+        scales fp16 [n, D/group])."""
+        x = _rows_f16(x_f16)
+        n, D = x.shape
+        lam = np.ascontiguousarray(np.atleast_2d(lam), dtype=np.float32)
+        s = np.ascontiguousarray(signs, dtype=np.int8)
+        nl = lam.shape[0]
+        rows = lambda_rows if lambda_rows is not None else max(n, 1)
+        codes = np.empty((n, D // 2 if bits == 4 else D), dtype=np.uint8)
+        scales = np.empty((n, D // group), dtype=np.uint16)
+        _check(self._lib.kvqo_quantize_ex(_ptr(x), _ptr(lam), _ptr(s), n, D, group, bits,
+                                          1 if lambda_after else 0, rows, nl,
+                                          _ptr(codes), _ptr(scales)))
+        return codes, scales.view(np.float16)
+
+    def dequantize_ex(self, codes, scales, lam, signs, group: int, bits: int = 4,
+                      lambda_after: bool = False, lambda_rows: int | None = None) -> np.ndarray:
+        codes = np.ascontiguousarray(np.atleast_2d(codes), dtype=np.uint8)
+        sc = np.ascontiguousarray(np.atleast_2d(scales)).view(np.uint16)
+        lam = np.ascontiguousarray(np.atleast_2d(lam), dtype=np.float32)
+        s = np.ascontiguousarray(signs, dtype=np.int8)
+        n = codes.shape[0]
+        D = codes.shape[1] * (2 if bits == 4 else 1)
+        rows = lambda_rows if lambda_rows is not None else max(n, 1)
+        out = np.empty((n, D), dtype=np.uint16)
+        _check(self._lib.kvqo_dequantize_ex(_ptr(codes), _ptr(sc), _ptr(lam), _ptr(s), n, D,
+                                            group, bits, 1 if lambda_after else 0, rows,
+                                            lam.shape[0], _ptr(out)))
+        return out.view(np.float16)
 
     def attention_decode(self, q, k_packed, k_scales, v_packed, v_scales, seq_len,
                          lam_k, s_k, lam_v, s_v, group: int, sm_scale: float) -> np.ndarray:

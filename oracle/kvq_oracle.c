@@ -462,3 +462,130 @@ int kvqo_attention_decode(const uint16_t *q, const uint8_t *k_packed,
     free(z);
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Format variants of the codec: lambda after the rotation, 8-bit      */
+/* codes, and one lambda table per range of rows.                      */
+/*   lambda_after 0: y = H diag(s) (lambda . x) / sqrt(D), as above;    */
+/*                1: y = lambda . (H diag(s) x / sqrt(D)), the paper's  */
+/*                   order ([P5] Methodologie 2: transform of diag(s)x, */
+/*                   then the per-channel lambda rescale);              */
+/*   bits 4: codes in [-8, 7], S = fp16(max|y| / 7), nibbles packed     */
+/*           as kvqo_pack;                                              */
+/*   bits 8: codes in [-128, 127], S = fp16(max|y| / 127), one two's-   */
+/*           complement byte per code;                                  */
+/*   row r uses lambda table (r / lambda_rows) % n_lambda, a table      */
+/*   being D floats (per-(layer, head) smoothing).                      */
+/* The inverse mirrors each order: lambda before -> dequantize_row;     */
+/* lambda after -> w = (q S) * (1/lambda), transform, * c, * s.         */
+/* ------------------------------------------------------------------ */
+
+static int check_ex(int D, int G, int bits, int64_t lambda_rows, int n_lambda)
+{
+    int rc = check_shape(D, G);
+    if (rc) return rc;
+    if (bits != 4 && bits != 8) return -4;
+    if (lambda_rows < 1 || n_lambda < 1) return -5;
+    return 0;
+}
+
+static const float *table_of(const float *lam, int64_t r, int64_t lambda_rows,
+                             int n_lambda, int D)
+{
+    return lam + ((r / lambda_rows) % n_lambda) * (int64_t)D;
+}
+
+int kvqo_quantize_ex(const uint16_t *x, const float *lam, const int8_t *s,
+                     int64_t n, int D, int G, int bits, int lambda_after,
+                     int64_t lambda_rows, int n_lambda, uint8_t *codes,
+                     uint16_t *scales)
+{
+    int rc = check_ex(D, G, bits, lambda_rows, n_lambda);
+    if (rc) return rc;
+    if (n < 0) return -5;
+    float c = kvqo_norm_const(D);
+    float qmax = (bits == 4) ? 7.0f : 127.0f;
+    float qmin = (bits == 4) ? -8.0f : -128.0f;
+    int row_bytes = (bits == 4) ? D / 2 : D;
+    float y[KVQO_DMAX];
+    int8_t q[KVQO_DMAX];
+    for (int64_t r = 0; r < n; ++r) {
+        const uint16_t *xr = x + r * D;
+        const float *lr = table_of(lam, r, lambda_rows, n_lambda, D);
+        if (!lambda_after) {
+            rotate_row_f32(xr, lr, s, D, c, y);
+        } else {
+            for (int i = 0; i < D; ++i) {
+                float t = kvqo_f16_to_f32(xr[i]);
+                y[i] = (s[i] < 0) ? -t : t;                    /* exact  */
+            }
+            kvqo_fwht_f32(y, D);
+            for (int i = 0; i < D; ++i) y[i] = y[i] * c;
+            for (int i = 0; i < D; ++i) y[i] = y[i] * lr[i];   /* lambda */
+        }
+        uint16_t *sc = scales + r * (D / G);
+        for (int j = 0; j < D / G; ++j) {
+            const float *yg = y + j * G;
+            float a = 0.0f;
+            for (int i = 0; i < G; ++i) {
+                float m = fabsf(yg[i]);
+                if (m > a) a = m;
+            }
+            uint16_t sb = kvqo_f32_to_f16(a / qmax);
+            if (sb == 0x7C00u) sb = 0x7BFFu;
+            sc[j] = sb;
+            float sf = kvqo_f16_to_f32(sb);
+            float rcp = (sf == 0.0f) ? 0.0f : 1.0f / sf;
+            for (int i = 0; i < G; ++i) {
+                float t = (sf == 0.0f) ? 0.0f : rintf(yg[i] * rcp);
+                if (t > qmax) t = qmax;
+                if (t < qmin) t = qmin;
+                q[j * G + i] = (int8_t)t;
+            }
+        }
+        uint8_t *cr = codes + r * row_bytes;
+        if (bits == 4)
+            kvqo_pack(q, D, cr);
+        else
+            for (int i = 0; i < D; ++i) cr[i] = (uint8_t)q[i];
+    }
+    return 0;
+}
+
+int kvqo_dequantize_ex(const uint8_t *codes, const uint16_t *scales,
+                       const float *lam, const int8_t *s, int64_t n, int D,
+                       int G, int bits, int lambda_after, int64_t lambda_rows,
+                       int n_lambda, uint16_t *out)
+{
+    int rc = check_ex(D, G, bits, lambda_rows, n_lambda);
+    if (rc) return rc;
+    if (n < 0) return -5;
+    float c = kvqo_norm_const(D);
+    int row_bytes = (bits == 4) ? D / 2 : D;
+    int8_t q[KVQO_DMAX];
+    float w[KVQO_DMAX];
+    for (int64_t r = 0; r < n; ++r) {
+        const uint8_t *cr = codes + r * row_bytes;
+        const float *lr = table_of(lam, r, lambda_rows, n_lambda, D);
+        if (bits == 4)
+            kvqo_unpack(cr, D, q);
+        else
+            for (int i = 0; i < D; ++i) q[i] = (int8_t)cr[i];
+        const uint16_t *sc = scales + r * (D / G);
+        if (!lambda_after) {
+            dequantize_row(q, sc, lr, s, D, G, c, w);
+        } else {
+            for (int i = 0; i < D; ++i) {
+                float u = (float)q[i] * kvqo_f16_to_f32(sc[i / G]);   /* exact */
+                w[i] = u * (1.0f / lr[i]);                             /* 1/lambda */
+            }
+            kvqo_fwht_f32(w, D);
+            for (int i = 0; i < D; ++i) {
+                float z = w[i] * c;
+                w[i] = (s[i] < 0) ? -z : z;                            /* exact */
+            }
+        }
+        for (int i = 0; i < D; ++i) out[r * D + i] = kvqo_f32_to_f16(w[i]);
+    }
+    return 0;
+}

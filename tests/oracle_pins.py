@@ -12,6 +12,9 @@ check the oracle against what the pages and the mathematics fix:
 * library routines: fp16 conversion against numpy's IEEE cast;
 * hand-worked examples (tests/golden/worked_examples.json) and the pages'
   printed compression figure (tests/golden/accounting.json);
+* format variants (lambda after the rotation, int8 codes, lambda tables):
+  the float64 definition with the dense matrix, the int8 code invariants, the
+  table indexing, the round-trip bound and the impulse closed form;
 * decode attention: against torch's scaled_dot_product_attention (float64)
   on caches rebuilt with numpy and scipy's Hadamard matrix, and against the
   closed forms one key (o = V_0), zero scale (o = mean V), a huge scale
@@ -366,6 +369,144 @@ def pin_accounting(o):
         assert abs(fp16_bytes / stored - 16.0 / (4.0 + 16.0 / G)) < 1e-12
 
 
+# ---- format variants: lambda after the rotation, int8 codes, lambda tables ----
+
+def _y_def(x, lam, s, lambda_after):
+    """The rotation's definition in float64 with the dense Sylvester matrix."""
+    D = x.shape[1]
+    H = sylvester_kron(D)
+    x64 = x.astype(np.float64)
+    l64 = lam.astype(np.float64)
+    s64 = s.astype(np.float64)
+    if lambda_after:
+        return l64 * ((x64 * s64) @ H.T) / math.sqrt(D)
+    return ((x64 * l64 * s64) @ H.T) / math.sqrt(D)
+
+
+def _codes_ex(o, codes, bits, D):
+    if bits == 4:
+        return o.unpack(codes).astype(np.int64)
+    return codes.view(np.int8).astype(np.int64)
+
+
+def pin_ex_matches_base(o):
+    """bits 4, lambda before, one table: the variant path is the base codec."""
+    rng = np.random.default_rng(31)
+    for D, G in ((16, 16), (128, 32), (256, 64)):
+        lam, s = _rand_params(rng, D)
+        x = _rows(rng, 9, D)
+        p1, s1 = o.quantize(x, lam, s, G)
+        p2, s2 = o.quantize_ex(x, lam, s, G)
+        assert np.array_equal(p1, p2) and np.array_equal(s1.view(np.uint16), s2.view(np.uint16))
+        assert np.array_equal(o.dequantize(p1, s1, lam, s, G).view(np.uint16),
+                              o.dequantize_ex(p2, s2, lam, s, G).view(np.uint16))
+
+
+def pin_ex_definition(o):
+    """Scales and codes against the float64 definition of each order: S within
+    one fp16 ulp of fp16(max|y|/qmax) and every code within rounding of y/S."""
+    rng = np.random.default_rng(32)
+    for D, G in ((16, 16), (64, 32), (128, 32)):
+        for bits in (4, 8):
+            for after in (False, True):
+                lam, s = _rand_params(rng, D)
+                x = _rows(rng, 16, D)
+                codes, S = o.quantize_ex(x, lam, s, G, bits=bits, lambda_after=after)
+                y = _y_def(x, lam, s, after)
+                qmax = 7.0 if bits == 4 else 127.0
+                a = np.abs(y).reshape(16, D // G, G).max(axis=2)
+                Sf = S.astype(np.float64)
+                ref = (a / qmax).astype(np.float16).astype(np.float64)
+                ulp = np.spacing(ref.astype(np.float16)).astype(np.float64)
+                assert np.all(np.abs(Sf - ref) <= ulp), f"scale off bits={bits} after={after}"
+                q = _codes_ex(o, codes, bits, D)
+                t = y / np.repeat(Sf, G, axis=1)
+                lo = -8 if bits == 4 else -128
+                assert np.all(np.abs(q - np.clip(t, lo, qmax)) <= 0.5 + 1e-3), \
+                    f"codes off bits={bits} after={after}"
+
+
+def pin_ex_int8_codes(o):
+    """8-bit codes lie in [-128, 127], every normal-scale group reaches 127,
+    and |y - q S| <= S / 2 (no clamping inside the range)."""
+    rng = np.random.default_rng(33)
+    D, G = 128, 32
+    for after in (False, True):
+        lam, s = _rand_params(rng, D)
+        x = _rows(rng, 32, D)
+        codes, S = o.quantize_ex(x, lam, s, G, bits=8, lambda_after=after)
+        q = _codes_ex(o, codes, 8, D).reshape(32, D // G, G)
+        Sf = S.astype(np.float64)
+        assert q.min() >= -128 and q.max() <= 127
+        normal = Sf >= 2.0 ** -14
+        assert np.all(np.abs(q).max(axis=2)[normal] == 127)
+        y = _y_def(x, lam, s, after).reshape(32, D // G, G)
+        err = np.abs(y - q * Sf[..., None])
+        assert np.all(err <= Sf[..., None] * (0.5 + 1e-4) + 1e-6)
+
+
+def pin_ex_tables(o):
+    """Row r uses table (r // lambda_rows) % n_lambda."""
+    rng = np.random.default_rng(34)
+    D, G = 64, 16
+    tables = rng.uniform(0.5, 2.0, (3, D)).astype(np.float32)
+    s = np.where(rng.random(D) < 0.5, -1, 1).astype(np.int8)
+    x = _rows(rng, 11, D)
+    for bits in (4, 8):
+        for after in (False, True):
+            codes, S = o.quantize_ex(x, tables, s, G, bits=bits, lambda_after=after, lambda_rows=2)
+            back = o.dequantize_ex(codes, S, tables, s, G, bits=bits, lambda_after=after, lambda_rows=2)
+            for r in range(11):
+                t = tables[(r // 2) % 3]
+                c1, s1 = o.quantize_ex(x[r:r + 1], t, s, G, bits=bits, lambda_after=after)
+                assert np.array_equal(codes[r:r + 1], c1)
+                assert np.array_equal(S[r:r + 1].view(np.uint16), s1.view(np.uint16))
+                b1 = o.dequantize_ex(c1, s1, t, s, G, bits=bits, lambda_after=after)
+                assert np.array_equal(back[r:r + 1].view(np.uint16), b1.view(np.uint16))
+
+
+def pin_ex_roundtrip_bound(o):
+    """dequantize(quantize(x)) obeys the quantiser's closed-form bound in the
+    space where the scales act: |lambda (x - x^)| (before) or |(x - x^) /
+    lambda-weighted| (after) <= 1/2 sqrt(sum S^2), plus output rounding."""
+    rng = np.random.default_rng(35)
+    for D, G in ((64, 16), (128, 32)):
+        for bits in (4, 8):
+            for after in (False, True):
+                lam, s = _rand_params(rng, D)
+                x = _rows(rng, 12, D, outliers=0)
+                codes, S = o.quantize_ex(x, lam, s, G, bits=bits, lambda_after=after)
+                xh = o.dequantize_ex(codes, S, lam, s, G, bits=bits, lambda_after=after)
+                d = x.astype(np.float64) - xh.astype(np.float64)
+                Sg = np.repeat(S.astype(np.float64), G, axis=1)
+                l64 = lam.astype(np.float64)
+                if after:
+                    # x - x^ = s H (lambda^-1 (y - y^)) / sqrt(D): an isometry of lambda^-1 (y - y^)
+                    bound = 0.5 * np.sqrt((Sg ** 2 / l64 ** 2).sum(axis=1))
+                    lhs = np.sqrt((d ** 2).sum(axis=1))
+                else:
+                    bound = 0.5 * np.sqrt((Sg ** 2).sum(axis=1))
+                    lhs = np.sqrt(((d * l64) ** 2).sum(axis=1))
+                slack = 2.0 ** -10 * np.sqrt((x.astype(np.float64) ** 2).sum(axis=1)) * (l64.max() if not after else 1.0)
+                assert np.all(lhs <= bound * 1.001 + slack), f"bits={bits} after={after}"
+
+
+def pin_ex_impulse(o):
+    """x = alpha e_k, lambda = 1: every code is +-qmax with the Hadamard sign
+    pattern of row k, in both orders and both widths."""
+    D, G = 32, 8
+    s = np.where(np.arange(D) % 3 == 0, -1, 1).astype(np.int8)
+    H = sylvester_kron(D)
+    for k in (0, 5, 31):
+        x = np.zeros((1, D), dtype=np.float16)
+        x[0, k] = 3.0
+        for bits, qmax in ((4, 7), (8, 127)):
+            for after in (False, True):
+                codes, S = o.quantize_ex(x, np.ones(D, np.float32), s, G, bits=bits, lambda_after=after)
+                q = _codes_ex(o, codes, bits, D)[0]
+                assert np.array_equal(q, (qmax * s[k] * H[k]).astype(np.int64))
+
+
 # ---- decode attention over the int4 cache ------------------------------
 
 def _nibbles(packed):
@@ -479,4 +620,6 @@ ALL_PINS = [
     pin_special_cases, pin_worked_examples, pin_divform_near_ties,
     pin_pack_layout, pin_accounting,
     pin_attention_vs_sdpa, pin_attention_closed_forms, pin_attention_masking,
+    pin_ex_matches_base, pin_ex_definition, pin_ex_int8_codes, pin_ex_tables,
+    pin_ex_roundtrip_bound, pin_ex_impulse,
 ]

@@ -36,6 +36,15 @@ MUTANTS = [
     ("deq_lambda_mult", "float il = 1.0f / lam[i];", "float il = lam[i];", 0),
     ("unrotate_f64_lambda", "(double)s[i] / lam[i];", "(double)s[i] * lam[i];", 0),
     ("f16_round_trunc", "_Float16 h = (_Float16)f;", "_Float16 h = (_Float16)(f - f * 0x1p-12f);", 0),
+    ("ex_int8_qmax", "float qmax = (bits == 4) ? 7.0f : 127.0f;", "float qmax = (bits == 4) ? 7.0f : 126.0f;", 0),
+    ("ex_int8_clamp", "float qmin = (bits == 4) ? -8.0f : -128.0f;", "float qmin = (bits == 4) ? -8.0f : -8.0f;", 0),
+    ("ex_after_lambda_dropped", "for (int i = 0; i < D; ++i) y[i] = y[i] * lr[i];   /* lambda */", "(void)lr;", 0),
+    ("ex_after_sign_dropped", "                y[i] = (s[i] < 0) ? -t : t;                    /* exact  */", "                y[i] = t;", 0),
+    ("ex_table_index", "return lam + ((r / lambda_rows) % n_lambda) * (int64_t)D;", "return lam + (r % n_lambda) * (int64_t)D;", 0),
+    ("ex_int8_store", "for (int i = 0; i < D; ++i) cr[i] = (uint8_t)q[i];", "for (int i = 0; i < D; ++i) cr[i] = (uint8_t)(q[i] & 0x7F);", 0),
+    ("ex_deq_lambda_mult", "w[i] = u * (1.0f / lr[i]);                             /* 1/lambda */", "w[i] = u * lr[i];", 0),
+    ("ex_deq_sign_dropped", "                w[i] = (s[i] < 0) ? -z : z;                            /* exact */", "                w[i] = z;", 0),
+    ("ex_deq_int8_unsigned", "for (int i = 0; i < D; ++i) q[i] = (int8_t)cr[i];", "for (int i = 0; i < D; ++i) q[i] = (int8_t)(cr[i] & 0x7F);", 0),
     ("attn_gqa_index", "int kv = h / R;", "int kv = h % Hkv;", 0),
     ("attn_no_max_shift", "double p = exp(z[t] - m);", "double p = exp(z[t]);", 0),
     ("attn_len_ignored", "for (int t = 0; t < len; ++t) {\n                double p", "for (int t = 0; t < T; ++t) {\n                double p", 0),
