@@ -146,6 +146,42 @@ int kvq_roundtrip(const uint16_t *x, const float *lambda, const int8_t *signs,
                   uint8_t *packed, uint16_t *scales, void *stream);
 
 /*
+ * kvq_quantize_ex / kvq_dequantize_ex -- the codec with format options:
+ *   lambda_after  0: lambda before the rotation, y = H diag(s)(lambda . x)/sqrt(D)
+ *                    (as kvq_quantize); 1: after it, y = lambda . (H diag(s) x
+ *                    / sqrt(D)), the order of "When Quantization Is Free",
+ *                    technical summary, Methodologie 2 (transform of diag(s) x,
+ *                    then the per-channel lambda rescale).  The inverse divides
+ *                    by lambda (fp32 multiply by IEEE 1/lambda) before its
+ *                    transform instead of after.
+ *   bits          4: int4 codes packed two per byte as kvq_quantize, S =
+ *                    fp16(max|y| / 7); 8: one int8 code per byte (two's
+ *                    complement), S = fp16(max|y| / 127), codes in [-128, 127].
+ *   lambda        n_lambda tables of D floats, fp32, 4-byte aligned; vector r
+ *                 uses table (r / lambda_rows) % n_lambda (per-(layer, head)
+ *                 smoothing: for a [layers][K,V][heads][T][D] cache,
+ *                 lambda_rows = T and n_lambda = layers * 2 * heads).  With
+ *                 n_lambda > 1, lambda_rows must be a multiple of 32.
+ *   codes         uint8 [n_vec][D/2] (bits 4) or [n_vec][D] (bits 8),
+ *                 16-byte aligned.  Other arguments as for kvq_quantize /
+ *                 kvq_dequantize.
+ * D must be 128 (else KVQ_ERR_DIM); group in {16, 32, 64} and bits in {4, 8}
+ * (else KVQ_ERR_GROUP); n_vec, lambda_rows, n_lambda out of range ->
+ * KVQ_ERR_COUNT.  Results are bit-identical to the oracle's definition of each
+ * option; bits = 4, lambda_after = 0 and one table reproduce kvq_quantize /
+ * kvq_dequantize exactly.
+ */
+int kvq_quantize_ex(const uint16_t *x, const float *lambda, const int8_t *signs,
+                    int64_t n_vec, int D, int group, int bits, int lambda_after,
+                    int64_t lambda_rows, int n_lambda, uint8_t *codes,
+                    uint16_t *scales, void *stream);
+int kvq_dequantize_ex(const uint8_t *codes, const uint16_t *scales,
+                      const float *lambda, const int8_t *signs, int64_t n_vec,
+                      int D, int group, int bits, int lambda_after,
+                      int64_t lambda_rows, int n_lambda, uint16_t *x_out,
+                      void *stream);
+
+/*
  * kvq_attention_decode -- one decode step of attention over the int4 cache:
  * for every sequence b and query head h,
  *     o[b][h] = sum_t p_t V_t,  p = softmax_t(sm_scale <q[b][h], K_t>),
@@ -227,8 +263,8 @@ int kvq_attention_decode_static(const uint16_t *q, const uint8_t *k_packed,
 /*
  * kvq_fault_status -- the current device's fault word: 0 when every bounded
  * wait of every kernel so far completed; bit 0 set when a quantize,
- * dequantize or attention block gave up waiting for its bulk copies (its
- * outputs are then incomplete); bit 1 set by kvq_selftest_wait_timeout; bit 2 set when
+ * dequantize (base or _ex) or attention warp gave up waiting for its bulk
+ * copies (its outputs are then incomplete); bit 1 set by kvq_selftest_wait_timeout; bit 2 set when
  * kvq_quantize_rows skipped an out-of-range row index; bit 3 set when
  * kvq_attention_decode met a sequence length outside [0, T].  Non-zero `clear`
  * resets the word.  Synchronous (it copies the word to the host, which waits

@@ -14,7 +14,7 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SOURCES = [os.path.join(PKG, "csrc", "kvq.cu"), os.path.join(PKG, "csrc", "kvq_attn.cu")]
+SOURCES = [os.path.join(PKG, "csrc", n) for n in ("kvq.cu", "kvq_attn.cu", "kvq_ex.cu")]
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libkvq.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -54,9 +54,11 @@
 
 #include "kvq.h"
 
-// The attention translation unit's fault word and last CUDA error.
+// The other translation units' fault words and last CUDA errors.
 unsigned int kvq_attn_fault_word(int clear);
 int kvq_attn_last_cuda_error();
+unsigned int kvq_ex_fault_word(int clear);
+int kvq_ex_last_cuda_error();
 
 namespace {
 
@@ -146,126 +148,7 @@ constexpr int roundtrip_smem_bytes() { return 1024 + 3 * Tile<D>::STAGE + 2 * Ti
 
 #include "kvq_async.cuh"
 
-__device__ __forceinline__ void st_v4(void* p, const uint32_t (&r)[4]) {
-  asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};"
-               :: "l"(p), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]) : "memory");
-}
-
-// ---------------------------------------------------------------------------
-// Arithmetic helpers.
-// ---------------------------------------------------------------------------
-
-__device__ __forceinline__ float2 half2_bits_to_float2(uint32_t w) {
-  __half2 h = *reinterpret_cast<__half2*>(&w);
-  return __half22float2(h);
-}
-__device__ __forceinline__ uint32_t float2_to_half2_bits(float lo, float hi) {
-  __half2 h = __floats2half2_rn(lo, hi);   // .x (low 16 bits) = lo
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-__device__ __forceinline__ float half_bits_to_float(uint16_t b) {
-  return __half2float(__ushort_as_half(b));
-}
-// a - b with one rounding: fma(b, -1, a).
-__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
-  return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a);
-}
-// max(a, |b|, |c|)
-__device__ __forceinline__ float amax3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(fabsf(b)), "f"(fabsf(c)));
-  return d;
-}
-
-// fp32 quotient a / 7, correctly rounded: q0 = a * RN(1/7), then one residual
-// correction r = a - 7 q0 (exact by fma), q = q0 + r * RN(1/7) (Markstein's
-// division by a known divisor; equal to IEEE a / 7.0f for every positive
-// finite fp32 a, checked exhaustively).
-__device__ __forceinline__ float div7_rn(float a) {
-  const float zh = 0x1.24924ap-3f;               // RN(1/7)
-  const float q0 = __fmul_rn(a, zh);
-  const float r = __fmaf_rn(-q0, 7.0f, a);
-  return __fmaf_rn(r, zh, q0);
-}
-// fp32 reciprocal of a positive fp16 value s, correctly rounded: approximate
-// reciprocal plus one Newton-Raphson step.  1/s lies at least 2^-35 (relative)
-// away from every rounding midpoint because s has an 11-bit significand, far
-// beyond the step's error; checked against IEEE 1/s for every positive
-// finite fp16 s.
-__device__ __forceinline__ float rcp_f16val(float s) {
-  float r0;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(s));
-  const float e = __fmaf_rn(-s, r0, 1.0f);
-  return __fmaf_rn(r0, e, r0);
-}
-// Scale of one group: S = fp16_rne(a / 7) saturated to 65504 (satfinite);
-// r = 1/S, or 0 when S = 0 (which makes every code of the group 0).
-__device__ __forceinline__ uint16_t group_scale(float a, float& r) {
-  uint16_t b;
-  asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(b) : "f"(div7_rn(a)));
-  const float sf = half_bits_to_float(b);
-  r = (sf == 0.0f) ? 0.0f : rcp_f16val(sf);
-  return b;
-}
-// Eight codes -> one 32-bit word, code k in bits [4k, 4k+4), each saturated
-// to [-8, 7] by the packing conversion.
-__device__ __forceinline__ uint32_t pack8(const int (&q)[8]) {
-  uint32_t d;
-  asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(q[7]), "r"(q[6]), "r"(0u));
-  asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(q[5]), "r"(q[4]), "r"(d));
-  asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(q[3]), "r"(q[2]), "r"(d));
-  asm("cvt.pack.sat.s4.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(q[1]), "r"(q[0]), "r"(d));
-  return d;
-}
-// w * s for fp16 operands, exact in fp32 (a product of two fp16 values has at
-// most 22 significant bits); the -0.0 addend keeps the sign of a zero product.
-__device__ __forceinline__ float mul_f16_f32(__half w, uint16_t s) {
-  float d;
-  asm("fma.rn.f32.f16 %0, %1, %2, %3;" : "=f"(d) : "h"(__half_as_ushort(w)), "h"(s), "f"(-0.0f));
-  return d;
-}
-
-// ---------------------------------------------------------------------------
-// Walsh-Hadamard butterflies (unnormalised, Sylvester order) on one vector
-// held as pairs p[m] = (v[m], v[m+HALF]) by LANES lanes, from half-width H0
-// upwards (stages below H0 already applied).
-// ---------------------------------------------------------------------------
-template <int EPT, int LANES, int H0 = 1>
-__device__ __forceinline__ void fwht_pairs(float2 (&p)[EPT / 2], int sub) {
-  constexpr int NP = EPT / 2;
-#pragma unroll
-  for (int h = H0; h < NP; h <<= 1) {
-#pragma unroll
-    for (int m = 0; m < NP; ++m) {
-      if ((m & h) == 0) {
-        const float2 a = p[m];
-        const float2 b = p[m + h];
-        p[m] = __fadd2_rn(a, b);
-        p[m + h] = fsub2(a, b);
-      }
-    }
-  }
-  // h = HALF: the two halves of each pair
-#pragma unroll
-  for (int m = 0; m < NP; ++m) {
-    const float a = p[m].x, b = p[m].y;
-    p[m] = make_float2(__fadd_rn(a, b), __fsub_rn(a, b));
-  }
-  // h = EPT (two lanes per vector): the lower lane keeps a + b, the upper one
-  // a_partner - b_own = fma(-1, own, partner).
-#pragma unroll
-  for (int bit = 1; bit < LANES; bit <<= 1) {
-    const float sg = (sub & bit) ? -1.0f : 1.0f;
-    const float2 sg2 = make_float2(sg, sg);
-#pragma unroll
-    for (int m = 0; m < NP; ++m) {
-      float2 o;
-      o.x = __shfl_xor_sync(kFullMask, p[m].x, bit);
-      o.y = __shfl_xor_sync(kFullMask, p[m].y, bit);
-      p[m] = __ffma2_rn(sg2, p[m], o);
-    }
-  }
-}
+#include "kvq_arith.cuh"
 
 // Per-channel table: tab[sub * NP/2 + q] = (c[2q], c[2q+HALF], c[2q+1],
 // c[2q+1+HALF]) over lane `sub`'s channels, c = lambda*s (quantize) or
@@ -1135,7 +1018,7 @@ int kvq_fault_status(int clear) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_kvq_fault, &zero, sizeof zero) != cudaSuccess) return -1;
   }
-  return static_cast<int>(v | kvq_attn_fault_word(clear));
+  return static_cast<int>(v | kvq_attn_fault_word(clear) | kvq_ex_fault_word(clear));
 }
 
 int kvq_selftest_wait_timeout(uint32_t limit, void* stream) {
@@ -1157,7 +1040,11 @@ const char* kvq_status_string(int status) {
   }
 }
 
-int kvq_last_cuda_error(void) { return g_last_cuda_error ? g_last_cuda_error : kvq_attn_last_cuda_error(); }
+int kvq_last_cuda_error(void) {
+  if (g_last_cuda_error) return g_last_cuda_error;
+  if (const int e = kvq_attn_last_cuda_error()) return e;
+  return kvq_ex_last_cuda_error();
+}
 
 int kvq_version(void) { return (1 << 16) | 2; }
 

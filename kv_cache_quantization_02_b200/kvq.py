@@ -42,6 +42,10 @@ _lib.kvq_roundtrip.restype = _I
 _lib.kvq_roundtrip.argtypes = [_P, _P, _P, _I64, _I, _I, _P, _P, _P, _P]
 _lib.kvq_dequantize.restype = _I
 _lib.kvq_dequantize.argtypes = [_P, _P, _P, _P, _I64, _I, _I, _P, _P]
+_lib.kvq_quantize_ex.restype = _I
+_lib.kvq_quantize_ex.argtypes = [_P, _P, _P, _I64, _I, _I, _I, _I, _I64, _I, _P, _P, _P]
+_lib.kvq_dequantize_ex.restype = _I
+_lib.kvq_dequantize_ex.argtypes = [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _I64, _I, _P, _P]
 _lib.kvq_attention_decode.restype = _I
 _lib.kvq_attention_decode.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _I64, _P]
@@ -101,6 +105,20 @@ def kvq_roundtrip(x: int, lam: int, signs: int, n_vec: int, D: int, group: int,
 def kvq_dequantize(packed: int, scales: int, lam: int, signs: int, n_vec: int,
                    D: int, group: int, x_out: int, stream: int = 0) -> int:
     return _lib.kvq_dequantize(packed, scales, lam, signs, n_vec, D, group, x_out, stream)
+
+
+def kvq_quantize_ex(x: int, lam: int, signs: int, n_vec: int, D: int, group: int, bits: int,
+                    lambda_after: int, lambda_rows: int, n_lambda: int, codes: int, scales: int,
+                    stream: int = 0) -> int:
+    return _lib.kvq_quantize_ex(x, lam, signs, n_vec, D, group, bits, lambda_after, lambda_rows,
+                                n_lambda, codes, scales, stream)
+
+
+def kvq_dequantize_ex(codes: int, scales: int, lam: int, signs: int, n_vec: int, D: int,
+                      group: int, bits: int, lambda_after: int, lambda_rows: int, n_lambda: int,
+                      x_out: int, stream: int = 0) -> int:
+    return _lib.kvq_dequantize_ex(codes, scales, lam, signs, n_vec, D, group, bits, lambda_after,
+                                  lambda_rows, n_lambda, x_out, stream)
 
 
 def kvq_attention_decode(q: int, k_packed: int, k_scales: int, v_packed: int, v_scales: int,
@@ -233,6 +251,62 @@ def roundtrip(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: in
         pk, sc = packed.data_ptr(), scales.data_ptr()
     rc = kvq_roundtrip(x.data_ptr(), lam.data_ptr(), signs.data_ptr(), n, D, group,
                        out.data_ptr(), pk, sc, _stream_handle(stream))
+    if rc != KVQ_OK:
+        raise KvqError(rc)
+    return out
+
+
+def quantize_ex(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: int,
+                bits: int = 4, lambda_after: bool = False, lambda_rows: int | None = None,
+                codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                stream=None):
+    """Format variants.  x fp16 [n, 128]; lam fp32 [n_lambda, 128] (or [128]);
+    row r uses table (r // lambda_rows) % n_lambda.  -> (codes uint8 [n, 64 or
+    128], scales fp16 [n, 128/group])."""
+    if x.dim() != 2:
+        raise ValueError("x must be [n_vec, D]")
+    n, D = x.shape
+    _need(x, torch.float16, (n, D), "x")
+    lam2 = lam.reshape(-1, D)
+    _need(lam2, torch.float32, (lam2.shape[0], D), "lambda")
+    _need(signs, torch.int8, (D,), "signs")
+    cb = D // 2 if bits == 4 else D
+    if codes is None:
+        codes = torch.empty((n, cb), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((n, D // group), dtype=torch.float16, device=x.device)
+    _need(codes, torch.uint8, (n, cb), "codes")
+    _need(scales, torch.float16, (n, D // group), "scales")
+    rows = lambda_rows if lambda_rows is not None else max(n, 1)
+    rc = kvq_quantize_ex(x.data_ptr(), lam2.data_ptr(), signs.data_ptr(), n, D, group, bits,
+                         1 if lambda_after else 0, rows, lam2.shape[0], codes.data_ptr(),
+                         scales.data_ptr(), _stream_handle(stream))
+    if rc != KVQ_OK:
+        raise KvqError(rc)
+    return codes, scales
+
+
+def dequantize_ex(codes: torch.Tensor, scales: torch.Tensor, lam: torch.Tensor,
+                  signs: torch.Tensor, group: int, bits: int = 4, lambda_after: bool = False,
+                  lambda_rows: int | None = None, out: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """Inverse of quantize_ex -> fp16 [n, 128]."""
+    if codes.dim() != 2:
+        raise ValueError("codes must be [n_vec, bytes]")
+    n = codes.shape[0]
+    D = codes.shape[1] * (2 if bits == 4 else 1)
+    _need(codes, torch.uint8, (n, codes.shape[1]), "codes")
+    _need(scales, torch.float16, (n, D // group), "scales")
+    lam2 = lam.reshape(-1, D)
+    _need(lam2, torch.float32, (lam2.shape[0], D), "lambda")
+    _need(signs, torch.int8, (D,), "signs")
+    if out is None:
+        out = torch.empty((n, D), dtype=torch.float16, device=codes.device)
+    _need(out, torch.float16, (n, D), "out")
+    rows = lambda_rows if lambda_rows is not None else max(n, 1)
+    rc = kvq_dequantize_ex(codes.data_ptr(), scales.data_ptr(), lam2.data_ptr(), signs.data_ptr(),
+                           n, D, group, bits, 1 if lambda_after else 0, rows, lam2.shape[0],
+                           out.data_ptr(), _stream_handle(stream))
     if rc != KVQ_OK:
         raise KvqError(rc)
     return out

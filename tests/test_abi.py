@@ -138,3 +138,20 @@ def test_attention_errors(kvq):
     assert call(B=0, q=0, out=0, lens=0) == 0
     assert kvq.kvq_attention_workspace_bytes(1, 32, 8, 4096, 256, 32) == -1
     assert kvq.kvq_attention_workspace_bytes(4096, 32, 8, 4096, 128, 32) == 0
+
+
+def test_codec_ex_errors(kvq):
+    q = lambda **kw: kvq.kvq_quantize_ex(kw.get("x", A), kw.get("lam", A), A, kw.get("n", 64),
+                                         kw.get("D", 128), kw.get("G", 32), kw.get("bits", 4),
+                                         0, kw.get("rows", 64), kw.get("nl", 1), kw.get("codes", A), A)
+    d = lambda **kw: kvq.kvq_dequantize_ex(kw.get("codes", A), A, A, A, kw.get("n", 64),
+                                           kw.get("D", 128), kw.get("G", 32), kw.get("bits", 4),
+                                           1, kw.get("rows", 64), kw.get("nl", 1), kw.get("out", A))
+    for f in (q, d):
+        assert f(D=64) == -3 and f(D=256) == -3
+        assert f(G=128) == -4 and f(G=8) == -4 and f(bits=5) == -4
+        assert f(n=-1) == -5 and f(nl=0) == -5 and f(rows=0) == -5
+        assert f(nl=3, rows=48) == -5            # several tables: rows a multiple of 32
+        assert f(n=0) == 0
+    assert q(x=0) == -1 and q(codes=0) == -1 and d(codes=0) == -1 and d(out=0) == -1
+    assert q(x=A + 8) == -2 and q(lam=A + 2) == -2 and d(codes=A + 8) == -2 and d(out=A + 8) == -2
