@@ -83,6 +83,10 @@ class Oracle:
             "kvqo_unpack": (None, [_P, _I64, _P]),
             "kvqo_quantize_ex": (_I, [_P, _P, _P, _I64, _I, _I, _I, _I, _I64, _I, _P, _P]),
             "kvqo_dequantize_ex": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _I64, _I, _P]),
+            "kvqo_srft_f32": (None, [_P, _I, _P]),
+            "kvqo_isrft_f32": (None, [_P, _I, _P]),
+            "kvqo_srft_f64": (None, [_P, _I, _P]),
+            "kvqo_isrft_f64": (None, [_P, _I, _P]),
             "kvqo_attention_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            _I, _I, _I, _I, _I, _I, ctypes.c_double, _P]),
         }
@@ -212,8 +216,37 @@ class Oracle:
         return out
 
 
+    def srft_f32(self, v) -> np.ndarray:
+        """fp32 SRFT (packed unitary real DFT) of rows v [n, D]."""
+        v = np.ascontiguousarray(np.atleast_2d(v), dtype=np.float32)
+        out = np.empty_like(v)
+        for r in range(v.shape[0]):
+            self._lib.kvqo_srft_f32(_ptr(v[r]), v.shape[1], _ptr(out[r]))
+        return out
+
+    def isrft_f32(self, y) -> np.ndarray:
+        y = np.ascontiguousarray(np.atleast_2d(y), dtype=np.float32)
+        out = np.empty_like(y)
+        for r in range(y.shape[0]):
+            self._lib.kvqo_isrft_f32(_ptr(y[r]), y.shape[1], _ptr(out[r]))
+        return out
+
+    def srft_f64(self, v) -> np.ndarray:
+        v = np.ascontiguousarray(np.atleast_2d(v), dtype=np.float64)
+        out = np.empty_like(v)
+        for r in range(v.shape[0]):
+            self._lib.kvqo_srft_f64(_ptr(v[r]), v.shape[1], _ptr(out[r]))
+        return out
+
+    def isrft_f64(self, y) -> np.ndarray:
+        y = np.ascontiguousarray(np.atleast_2d(y), dtype=np.float64)
+        out = np.empty_like(y)
+        for r in range(y.shape[0]):
+            self._lib.kvqo_isrft_f64(_ptr(y[r]), y.shape[1], _ptr(out[r]))
+        return out
+
     def quantize_ex(self, x_f16, lam, signs, group: int, bits: int = 4, lambda_after: bool = False,
-                    lambda_rows: int | None = None):
+                    lambda_rows: int | None = None, srft: bool = False):
         """Format variants: lam is [n_lambda, D] (or [D]); row r uses table
         (r // lambda_rows) % n_lambda.  Returns (codes uint8 [n, D/2 or D],
         scales fp16 [n, D/group])."""
@@ -226,12 +259,13 @@ class Oracle:
         codes = np.empty((n, D // 2 if bits == 4 else D), dtype=np.uint8)
         scales = np.empty((n, D // group), dtype=np.uint16)
         _check(self._lib.kvqo_quantize_ex(_ptr(x), _ptr(lam), _ptr(s), n, D, group, bits,
-                                          1 if lambda_after else 0, rows, nl,
+                                          _flags(lambda_after, srft), rows, nl,
                                           _ptr(codes), _ptr(scales)))
         return codes, scales.view(np.float16)
 
     def dequantize_ex(self, codes, scales, lam, signs, group: int, bits: int = 4,
-                      lambda_after: bool = False, lambda_rows: int | None = None) -> np.ndarray:
+                      lambda_after: bool = False, lambda_rows: int | None = None,
+                      srft: bool = False) -> np.ndarray:
         codes = np.ascontiguousarray(np.atleast_2d(codes), dtype=np.uint8)
         sc = np.ascontiguousarray(np.atleast_2d(scales)).view(np.uint16)
         lam = np.ascontiguousarray(np.atleast_2d(lam), dtype=np.float32)
@@ -241,7 +275,7 @@ class Oracle:
         rows = lambda_rows if lambda_rows is not None else max(n, 1)
         out = np.empty((n, D), dtype=np.uint16)
         _check(self._lib.kvqo_dequantize_ex(_ptr(codes), _ptr(sc), _ptr(lam), _ptr(s), n, D,
-                                            group, bits, 1 if lambda_after else 0, rows,
+                                            group, bits, _flags(lambda_after, srft), rows,
                                             lam.shape[0], _ptr(out)))
         return out.view(np.float16)
 
@@ -271,6 +305,10 @@ class Oracle:
             _ptr(lk), _ptr(sk), _ptr(lv), _ptr(sv), B, Hq, Hkv, T, D, group,
             float(sm_scale), _ptr(out)))
         return out
+
+
+def _flags(lambda_after: bool, srft: bool) -> int:
+    return (1 if lambda_after else 0) | (2 if srft else 0)
 
 
 def _rows_f16(x) -> np.ndarray:

@@ -464,12 +464,171 @@ int kvqo_attention_decode(const uint16_t *q, const uint8_t *k_packed,
 }
 
 /* ------------------------------------------------------------------ */
-/* Format variants of the codec: lambda after the rotation, 8-bit      */
-/* codes, and one lambda table per range of rows.                      */
-/*   lambda_after 0: y = H diag(s) (lambda . x) / sqrt(D), as above;    */
-/*                1: y = lambda . (H diag(s) x / sqrt(D)), the paper's  */
-/*                   order ([P5] Methodologie 2: transform of diag(s)x, */
+/* The SRFT rotation: SRFT(x) = pack(F diag(s) x), F the unitary DFT    */
+/* of length D ([P5] Methodologie 1), computed as in the paper's        */
+/* kernel ([P5] Methodologie 2): a length-N = D/2 complex FFT of        */
+/* z_n = v_2n + i v_2n+1 in log2(N) radix-2 Stockham stages, then the   */
+/* Hermitian unpacking to a real representation.  The packing read     */
+/* here (orthonormal, so the inverse is the transpose):                 */
+/*   y0 = X_0 / sqrt(D),  y1 = X_N / sqrt(D),                            */
+/*   y_2k = sqrt(2) Re X_k / sqrt(D),  y_2k+1 = sqrt(2) Im X_k / sqrt(D), */
+/*   k = 1 .. N-1, X = DFT(v).                                          */
+/* Twiddles are cos / sin in double, rounded to fp32; every complex     */
+/* product is four fp32 products and two fp32 sums in the order below.  */
+/* ------------------------------------------------------------------ */
+
+/* omega_M^k = (cos(2 pi k / M), -sin(2 pi k / M)) rounded to fp32. */
+static void twiddle(int k, int M, float *wr, float *wi)
+{
+    const double a = 2.0 * 3.14159265358979323846 * (double)k / (double)M;
+    *wr = (float)cos(a);
+    *wi = (float)(-sin(a));
+}
+
+/* Stockham radix-2 FFT of length N (a power of two), unnormalised, in
+ * place through a scratch copy.  sign = -1: forward (omega), +1: inverse
+ * (conjugate twiddles).  Stage: n = N, N/2, ..., 2 with stride s = N / n:
+ *   a = x[q + s p], b = x[q + s (p + n/2)],
+ *   y[q + s 2p] = a + b,  y[q + s (2p + 1)] = (a - b) * omega_n^p. */
+static void stockham(float *re, float *im, int N, int sign)
+{
+    float tr[KVQO_DMAX / 2], ti[KVQO_DMAX / 2];
+    float *xr = re, *xi = im, *yr = tr, *yi = ti;
+    int s = 1;
+    for (int n = N; n > 1; n >>= 1) {
+        int m = n / 2;
+        for (int p = 0; p < m; ++p) {
+            float wr, wi;
+            twiddle(p * s, N, &wr, &wi);      /* omega_n^p = omega_N^(p s) */
+            if (sign > 0) wi = -wi;
+            for (int q = 0; q < s; ++q) {
+                float ar = xr[q + s * p], ai = xi[q + s * p];
+                float br = xr[q + s * (p + m)], bi = xi[q + s * (p + m)];
+                yr[q + s * 2 * p] = ar + br;
+                yi[q + s * 2 * p] = ai + bi;
+                float dr = ar - br, di = ai - bi;
+                float pr = dr * wr, pi_ = di * wi, qr = dr * wi, qi = di * wr;
+                yr[q + s * (2 * p + 1)] = pr - pi_;
+                yi[q + s * (2 * p + 1)] = qr + qi;
+            }
+        }
+        float *t;
+        t = xr; xr = yr; yr = t;
+        t = xi; xi = yi; yi = t;
+        s *= 2;
+    }
+    if (xr != re) {
+        for (int i = 0; i < N; ++i) { re[i] = xr[i]; im[i] = xi[i]; }
+    }
+}
+
+/* One spectrum bin of the real input from the half-length spectrum:
+ * X_k = E_k + omega_D^k O_k, E_k = (Z_k + conj Z_(N-k)) / 2,
+ * O_k = (Z_k - conj Z_(N-k)) / 2i   (indices mod N). */
+static void real_bin(const float *zr, const float *zi, int N, int k,
+                     float *xr, float *xi)
+{
+    int a = k % N, b = (N - k) % N;
+    float Ar = zr[a], Ai = zi[a], Br = zr[b], Bi = -zi[b];
+    float Er = (Ar + Br) * 0.5f, Ei = (Ai + Bi) * 0.5f;
+    float Dr = Ar - Br, Di = Ai - Bi;
+    float Or = Di * 0.5f, Oi = -(Dr * 0.5f);
+    float wr, wi;
+    twiddle(k, 2 * N, &wr, &wi);
+    float Tr = Or * wr - Oi * wi, Ti = Or * wi + Oi * wr;
+    *xr = Er + Tr;
+    *xi = Ei + Ti;
+}
+
+/* fp32 forward SRFT of one sign-flipped (and scaled) row v[D] -> y[D]. */
+void kvqo_srft_f32(const float *v, int D, float *y)
+{
+    int N = D / 2;
+    float zr[KVQO_DMAX / 2], zi[KVQO_DMAX / 2];
+    for (int n = 0; n < N; ++n) { zr[n] = v[2 * n]; zi[n] = v[2 * n + 1]; }
+    stockham(zr, zi, N, -1);
+    const float c0 = (float)(1.0 / sqrt((double)D));
+    const float c1 = (float)(sqrt(2.0 / (double)D));
+    float xr, xi;
+    real_bin(zr, zi, N, 0, &xr, &xi);
+    y[0] = xr * c0;
+    real_bin(zr, zi, N, N, &xr, &xi);
+    y[1] = xr * c0;
+    for (int k = 1; k < N; ++k) {
+        real_bin(zr, zi, N, k, &xr, &xi);
+        y[2 * k] = xr * c1;
+        y[2 * k + 1] = xi * c1;
+    }
+}
+
+/* fp32 inverse SRFT (the transpose): y[D] -> v[D] = P^T y. */
+void kvqo_isrft_f32(const float *y, int D, float *v)
+{
+    int N = D / 2;
+    const float c0 = (float)(1.0 / sqrt((double)D));
+    const float c1 = (float)(sqrt(2.0 / (double)D));
+    /* U_0 = 2 c0 y0, U_N = 2 c0 y1, U_k = c1 (y_2k + i y_2k+1) */
+    float Ur[KVQO_DMAX / 2 + 1], Ui[KVQO_DMAX / 2 + 1];
+    Ur[0] = (y[0] * c0) * 2.0f; Ui[0] = 0.0f;
+    Ur[N] = (y[1] * c0) * 2.0f; Ui[N] = 0.0f;
+    for (int k = 1; k < N; ++k) { Ur[k] = y[2 * k] * c1; Ui[k] = y[2 * k + 1] * c1; }
+    float zr[KVQO_DMAX / 2], zi[KVQO_DMAX / 2];
+    for (int k = 0; k < N; ++k) {
+        float Ar = Ur[k], Ai = Ui[k], Br = Ur[N - k], Bi = -Ui[N - k];
+        float Er = (Ar + Br) * 0.5f, Ei = (Ai + Bi) * 0.5f;
+        float Dr = Ar - Br, Di = Ai - Bi;
+        float wr, wi;
+        twiddle(k, D, &wr, &wi);
+        wi = -wi;                                         /* conj(omega_D^k) */
+        float Tr = Dr * wr - Di * wi, Ti = Dr * wi + Di * wr;
+        float Or = Tr * 0.5f, Oi = Ti * 0.5f;
+        zr[k] = Er - Oi;                                  /* E + i O */
+        zi[k] = Ei + Or;
+    }
+    stockham(zr, zi, N, +1);
+    for (int n = 0; n < N; ++n) { v[2 * n] = zr[n]; v[2 * n + 1] = zi[n]; }
+}
+
+/* Definitions in double, for the pins: the packed unitary DFT and its
+ * transpose, by direct sums. */
+void kvqo_srft_f64(const double *v, int D, double *y)
+{
+    int N = D / 2;
+    for (int k = 0; k <= N; ++k) {
+        double xr = 0.0, xi = 0.0;
+        for (int n = 0; n < D; ++n) {
+            double a = 2.0 * 3.14159265358979323846 * (double)k * (double)n / (double)D;
+            xr += v[n] * cos(a);
+            xi -= v[n] * sin(a);
+        }
+        if (k == 0) y[0] = xr / sqrt((double)D);
+        else if (k == N) y[1] = xr / sqrt((double)D);
+        else { y[2 * k] = xr * sqrt(2.0 / D); y[2 * k + 1] = xi * sqrt(2.0 / D); }
+    }
+}
+
+void kvqo_isrft_f64(const double *y, int D, double *v)
+{
+    int N = D / 2;
+    for (int n = 0; n < D; ++n) {
+        double acc = y[0] / sqrt((double)D) + y[1] * ((n & 1) ? -1.0 : 1.0) / sqrt((double)D);
+        for (int k = 1; k < N; ++k) {
+            double a = 2.0 * 3.14159265358979323846 * (double)k * (double)n / (double)D;
+            acc += sqrt(2.0 / D) * (y[2 * k] * cos(a) - y[2 * k + 1] * sin(a));
+        }
+        v[n] = acc;
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Format variants of the codec: lambda after the rotation, the SRFT,  */
+/* 8-bit codes, and one lambda table per range of rows.  flags:         */
+/*   bit 0 (lambda after) 0: y = R (lambda . x), as above;              */
+/*                        1: y = lambda . (R x), the paper's order      */
+/*                   ([P5] Methodologie 2: transform of diag(s) x,      */
 /*                   then the per-channel lambda rescale);              */
+/*   bit 1 (SRFT)  R = H diag(s) / sqrt(D) (0) or the SRFT pack(F       */
+/*                 diag(s) .) above (1);                                */
 /*   bits 4: codes in [-8, 7], S = fp16(max|y| / 7), nibbles packed     */
 /*           as kvqo_pack;                                              */
 /*   bits 8: codes in [-128, 127], S = fp16(max|y| / 127), one two's-   */
@@ -496,10 +655,11 @@ static const float *table_of(const float *lam, int64_t r, int64_t lambda_rows,
 }
 
 int kvqo_quantize_ex(const uint16_t *x, const float *lam, const int8_t *s,
-                     int64_t n, int D, int G, int bits, int lambda_after,
+                     int64_t n, int D, int G, int bits, int flags,
                      int64_t lambda_rows, int n_lambda, uint8_t *codes,
                      uint16_t *scales)
 {
+    const int lambda_after = flags & 1, srft = (flags >> 1) & 1;
     int rc = check_ex(D, G, bits, lambda_rows, n_lambda);
     if (rc) return rc;
     if (n < 0) return -5;
@@ -512,16 +672,23 @@ int kvqo_quantize_ex(const uint16_t *x, const float *lam, const int8_t *s,
     for (int64_t r = 0; r < n; ++r) {
         const uint16_t *xr = x + r * D;
         const float *lr = table_of(lam, r, lambda_rows, n_lambda, D);
-        if (!lambda_after) {
+        if (!lambda_after && !srft) {
             rotate_row_f32(xr, lr, s, D, c, y);
         } else {
+            float v[KVQO_DMAX];
             for (int i = 0; i < D; ++i) {
                 float t = kvqo_f16_to_f32(xr[i]);
-                y[i] = (s[i] < 0) ? -t : t;                    /* exact  */
+                if (!lambda_after) t = t * lr[i];              /* lambda */
+                v[i] = (s[i] < 0) ? -t : t;                    /* exact  */
             }
-            kvqo_fwht_f32(y, D);
-            for (int i = 0; i < D; ++i) y[i] = y[i] * c;
-            for (int i = 0; i < D; ++i) y[i] = y[i] * lr[i];   /* lambda */
+            if (srft) {
+                kvqo_srft_f32(v, D, y);
+            } else {
+                kvqo_fwht_f32(v, D);
+                for (int i = 0; i < D; ++i) y[i] = v[i] * c;
+            }
+            if (lambda_after)
+                for (int i = 0; i < D; ++i) y[i] = y[i] * lr[i];   /* lambda */
         }
         uint16_t *sc = scales + r * (D / G);
         for (int j = 0; j < D / G; ++j) {
@@ -554,9 +721,10 @@ int kvqo_quantize_ex(const uint16_t *x, const float *lam, const int8_t *s,
 
 int kvqo_dequantize_ex(const uint8_t *codes, const uint16_t *scales,
                        const float *lam, const int8_t *s, int64_t n, int D,
-                       int G, int bits, int lambda_after, int64_t lambda_rows,
+                       int G, int bits, int flags, int64_t lambda_rows,
                        int n_lambda, uint16_t *out)
 {
+    const int lambda_after = flags & 1, srft = (flags >> 1) & 1;
     int rc = check_ex(D, G, bits, lambda_rows, n_lambda);
     if (rc) return rc;
     if (n < 0) return -5;
@@ -572,20 +740,27 @@ int kvqo_dequantize_ex(const uint8_t *codes, const uint16_t *scales,
         else
             for (int i = 0; i < D; ++i) q[i] = (int8_t)cr[i];
         const uint16_t *sc = scales + r * (D / G);
-        if (!lambda_after) {
+        if (!lambda_after && !srft) {
             dequantize_row(q, sc, lr, s, D, G, c, w);
         } else {
+            float u[KVQO_DMAX];
             for (int i = 0; i < D; ++i) {
-                float u = (float)q[i] * kvqo_f16_to_f32(sc[i / G]);   /* exact */
-                w[i] = u * (1.0f / lr[i]);                             /* 1/lambda */
+                u[i] = (float)q[i] * kvqo_f16_to_f32(sc[i / G]);      /* exact */
+                if (lambda_after) u[i] = u[i] * (1.0f / lr[i]);        /* 1/lambda */
             }
-            kvqo_fwht_f32(w, D);
+            if (srft) {
+                kvqo_isrft_f32(u, D, w);
+            } else {
+                kvqo_fwht_f32(u, D);
+                for (int i = 0; i < D; ++i) w[i] = u[i] * c;
+            }
             for (int i = 0; i < D; ++i) {
-                float z = w[i] * c;
-                w[i] = (s[i] < 0) ? -z : z;                            /* exact */
+                float z = (s[i] < 0) ? -w[i] : w[i];                   /* exact */
+                w[i] = lambda_after ? z : z * (1.0f / lr[i]);
             }
         }
         for (int i = 0; i < D; ++i) out[r * D + i] = kvqo_f32_to_f16(w[i]);
     }
     return 0;
 }
+

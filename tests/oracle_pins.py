@@ -12,6 +12,9 @@ check the oracle against what the pages and the mathematics fix:
 * library routines: fp16 conversion against numpy's IEEE cast;
 * hand-worked examples (tests/golden/worked_examples.json) and the pages'
   printed compression figure (tests/golden/accounting.json);
+* the SRFT rotation: numpy's rfft (unitary, packed), orthogonality of its
+  dense matrix, the fp32 Stockham path within its bound of the float64
+  definition, closed forms, and the codec built on it;
 * format variants (lambda after the rotation, int8 codes, lambda tables):
   the float64 definition with the dense matrix, the int8 code invariants, the
   table indexing, the round-trip bound and the impulse closed form;
@@ -507,6 +510,117 @@ def pin_ex_impulse(o):
                 assert np.array_equal(q, (qmax * s[k] * H[k]).astype(np.int64))
 
 
+# ---- the SRFT rotation ---------------------------------------------------
+
+def _rfft_packed(v):
+    """numpy's rfft, unitary-scaled and packed (y0 = X_0, y1 = X_N, then
+    sqrt(2) (Re, Im) X_k): the pages' pack(F v) read as an orthonormal map."""
+    D = v.shape[-1]
+    N = D // 2
+    X = np.fft.rfft(v, axis=-1) / math.sqrt(D)
+    y = np.empty(v.shape, dtype=np.float64)
+    y[..., 0] = X[..., 0].real
+    y[..., 1] = X[..., N].real
+    y[..., 2::2] = 0.0
+    for k in range(1, N):
+        y[..., 2 * k] = math.sqrt(2.0) * X[..., k].real
+        y[..., 2 * k + 1] = math.sqrt(2.0) * X[..., k].imag
+    return y
+
+
+def pin_srft_definition(o):
+    """The f64 SRFT equals numpy's rfft packed and scaled; it is orthogonal
+    (its dense matrix P has P^T P = I) and the f64 inverse is P^T."""
+    rng = np.random.default_rng(41)
+    for D in (4, 8, 32, 128, 256):
+        v = rng.standard_normal((5, D))
+        assert np.abs(o.srft_f64(v) - _rfft_packed(v)).max() < 1e-12 * math.sqrt(D)
+        P = o.srft_f64(np.eye(D)).T                    # column j = P e_j
+        assert np.abs(P.T @ P - np.eye(D)).max() < 1e-12
+        y = rng.standard_normal((5, D))
+        assert np.abs(o.isrft_f64(y) - y @ P).max() < 1e-12 * math.sqrt(D)
+
+
+def pin_srft_f32(o):
+    """The fp32 Stockham path lies within its error bound of the f64
+    definition, preserves the norm, and its inverse undoes it."""
+    rng = np.random.default_rng(42)
+    U = 2.0 ** -24
+    for D in (8, 64, 128, 256):
+        v = rng.standard_normal((16, D)).astype(np.float32)
+        v[:, 3] *= 30.0
+        y32 = o.srft_f32(v).astype(np.float64)
+        y64 = o.srft_f64(v.astype(np.float64))
+        bound = 6.0 * math.log2(D) * U * np.abs(v.astype(np.float64)).sum(axis=1, keepdims=True) / math.sqrt(D) * 2
+        assert np.all(np.abs(y32 - y64) <= bound)
+        nv = np.linalg.norm(v.astype(np.float64), axis=1)
+        assert np.all(np.abs(np.linalg.norm(y32, axis=1) - nv) <= 1e-6 * nv)
+        b32 = o.isrft_f32(y64.astype(np.float32)).astype(np.float64)
+        b64 = o.isrft_f64(y64)
+        assert np.all(np.abs(b32 - b64) <= bound * 2)
+        assert np.abs(b64 - v).max() <= 1e-12 * np.abs(v).max()
+
+
+def pin_srft_closed_forms(o):
+    """signs +1, lambda 1: a constant row puts everything in y0 (code 7 there,
+    0 elsewhere); an impulse at channel 0 gives y = (1, 1, sqrt2, 0, sqrt2, 0,
+    ...) / sqrt(D): codes (5, 5, 7, 0, 7, 0, ...) at int4, (90, 90, 127, 0,
+    ...) at int8."""
+    D, G = 32, 8
+    one = np.ones(D, np.float32)
+    s = np.ones(D, np.int8)
+    x = np.full((1, D), 0.5, dtype=np.float16)
+    codes, S = o.quantize_ex(x, one, s, G, srft=True)
+    q = o.unpack(codes)[0]
+    assert q[0] == 7 and np.all(q[1:] == 0)
+    x = np.zeros((1, D), dtype=np.float16)
+    x[0, 0] = 1.0
+    for bits, top, edge in ((4, 7, 5), (8, 127, 90)):
+        codes, S = o.quantize_ex(x, one, s, G, bits=bits, srft=True)
+        q = _codes_ex(o, codes, bits, D)[0]
+        want = np.zeros(D, np.int64)
+        want[0::2] = top
+        want[0] = want[1] = edge
+        assert np.array_equal(q, want), (bits, q)
+
+
+def pin_srft_codec(o):
+    """The codec with the SRFT: scales and codes against the float64 definition
+    y = R(lambda . x) or lambda . R(x) with R = P diag(s), and the round trip
+    obeys the quantiser bound."""
+    rng = np.random.default_rng(43)
+    for D, G in ((16, 16), (128, 32)):
+        for bits in (4, 8):
+            for after in (False, True):
+                lam, s = _rand_params(rng, D)
+                x = _rows(rng, 12, D, outliers=0)
+                codes, S = o.quantize_ex(x, lam, s, G, bits=bits, lambda_after=after, srft=True)
+                x64 = x.astype(np.float64)
+                l64 = lam.astype(np.float64)
+                v = x64 * s.astype(np.float64) * (1.0 if after else l64)
+                y = o.srft_f64(v) * (l64 if after else 1.0)
+                qmax = 7.0 if bits == 4 else 127.0
+                a = np.abs(y).reshape(12, D // G, G).max(axis=2)
+                Sf = S.astype(np.float64)
+                ref = (a / qmax).astype(np.float16).astype(np.float64)
+                ulp = np.spacing(ref.astype(np.float16)).astype(np.float64)
+                assert np.all(np.abs(Sf - ref) <= ulp)
+                q = _codes_ex(o, codes, bits, D)
+                t = y / np.repeat(Sf, G, axis=1)
+                assert np.all(np.abs(q - np.clip(t, -qmax - 1, qmax)) <= 0.5 + 1e-3)
+                xh = o.dequantize_ex(codes, S, lam, s, G, bits=bits, lambda_after=after, srft=True)
+                d = x64 - xh.astype(np.float64)
+                Sg = np.repeat(Sf, G, axis=1)
+                if after:
+                    bound = 0.5 * np.sqrt((Sg ** 2 / l64 ** 2).sum(axis=1))
+                    lhs = np.linalg.norm(d, axis=1)
+                else:
+                    bound = 0.5 * np.sqrt((Sg ** 2).sum(axis=1))
+                    lhs = np.linalg.norm(d * l64, axis=1)
+                slack = 2.0 ** -10 * np.linalg.norm(x64, axis=1) * (1.0 if after else l64.max())
+                assert np.all(lhs <= bound * 1.001 + slack)
+
+
 # ---- decode attention over the int4 cache ------------------------------
 
 def _nibbles(packed):
@@ -622,4 +736,5 @@ ALL_PINS = [
     pin_attention_vs_sdpa, pin_attention_closed_forms, pin_attention_masking,
     pin_ex_matches_base, pin_ex_definition, pin_ex_int8_codes, pin_ex_tables,
     pin_ex_roundtrip_bound, pin_ex_impulse,
+    pin_srft_definition, pin_srft_f32, pin_srft_closed_forms, pin_srft_codec,
 ]

@@ -45,6 +45,14 @@ MUTANTS = [
     ("ex_deq_lambda_mult", "w[i] = u * (1.0f / lr[i]);                             /* 1/lambda */", "w[i] = u * lr[i];", 0),
     ("ex_deq_sign_dropped", "                w[i] = (s[i] < 0) ? -z : z;                            /* exact */", "                w[i] = z;", 0),
     ("ex_deq_int8_unsigned", "for (int i = 0; i < D; ++i) q[i] = (int8_t)cr[i];", "for (int i = 0; i < D; ++i) q[i] = (int8_t)(cr[i] & 0x7F);", 0),
+    ("srft_twiddle_sign", "*wi = (float)(-sin(a));", "*wi = (float)(sin(a));", 0),
+    ("srft_no_sqrt2", "const float c1 = (float)(sqrt(2.0 / (double)D));", "const float c1 = (float)(sqrt(1.0 / (double)D));", 0),
+    ("srft_stage_stride", "twiddle(p * s, N, &wr, &wi);      /* omega_n^p = omega_N^(p s) */", "twiddle(p, N, &wr, &wi);", 0),
+    ("srft_butterfly_sign", "yr[q + s * 2 * p] = ar + br;", "yr[q + s * 2 * p] = ar - br;", 0),
+    ("srft_odd_part_sign", "float Or = Di * 0.5f, Oi = -(Dr * 0.5f);", "float Or = Di * 0.5f, Oi = (Dr * 0.5f);", 0),
+    ("srft_nyquist_slot", "y[1] = xr * c0;", "y[1] = xr * c1;", 0),
+    ("isrft_no_conj", "wi = -wi;                                         /* conj(omega_D^k) */", "wi = wi;", 0),
+    ("isrft_pairing", "zr[k] = Er - Oi;                                  /* E + i O */", "zr[k] = Er + Oi;", 0),
     ("attn_gqa_index", "int kv = h / R;", "int kv = h % Hkv;", 0),
     ("attn_no_max_shift", "double p = exp(z[t] - m);", "double p = exp(z[t]);", 0),
     ("attn_len_ignored", "for (int t = 0; t < len; ++t) {\n                double p", "for (int t = 0; t < T; ++t) {\n                double p", 0),
