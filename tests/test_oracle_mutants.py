@@ -39,11 +39,12 @@ MUTANTS = [
     ("ex_int8_qmax", "float qmax = (bits == 4) ? 7.0f : 127.0f;", "float qmax = (bits == 4) ? 7.0f : 126.0f;", 0),
     ("ex_int8_clamp", "float qmin = (bits == 4) ? -8.0f : -128.0f;", "float qmin = (bits == 4) ? -8.0f : -8.0f;", 0),
     ("ex_after_lambda_dropped", "for (int i = 0; i < D; ++i) y[i] = y[i] * lr[i];   /* lambda */", "(void)lr;", 0),
-    ("ex_after_sign_dropped", "                y[i] = (s[i] < 0) ? -t : t;                    /* exact  */", "                y[i] = t;", 0),
+    ("ex_variant_sign_dropped", "v[i] = (s[i] < 0) ? -t : t;                    /* exact  */", "v[i] = t;", 0),
     ("ex_table_index", "return lam + ((r / lambda_rows) % n_lambda) * (int64_t)D;", "return lam + (r % n_lambda) * (int64_t)D;", 0),
     ("ex_int8_store", "for (int i = 0; i < D; ++i) cr[i] = (uint8_t)q[i];", "for (int i = 0; i < D; ++i) cr[i] = (uint8_t)(q[i] & 0x7F);", 0),
-    ("ex_deq_lambda_mult", "w[i] = u * (1.0f / lr[i]);                             /* 1/lambda */", "w[i] = u * lr[i];", 0),
-    ("ex_deq_sign_dropped", "                w[i] = (s[i] < 0) ? -z : z;                            /* exact */", "                w[i] = z;", 0),
+    ("ex_deq_lambda_mult", "if (lambda_after) u[i] = u[i] * (1.0f / lr[i]);        /* 1/lambda */", "if (lambda_after) u[i] = u[i] * lr[i];", 0),
+    ("ex_deq_sign_dropped", "float z = (s[i] < 0) ? -w[i] : w[i];                   /* exact */", "float z = w[i];", 0),
+    ("ex_deq_before_lambda_mult", "w[i] = lambda_after ? z : z * (1.0f / lr[i]);", "w[i] = lambda_after ? z : z * lr[i];", 0),
     ("ex_deq_int8_unsigned", "for (int i = 0; i < D; ++i) q[i] = (int8_t)cr[i];", "for (int i = 0; i < D; ++i) q[i] = (int8_t)(cr[i] & 0x7F);", 0),
     ("srft_twiddle_sign", "*wi = (float)(-sin(a));", "*wi = (float)(sin(a));", 0),
     ("srft_no_sqrt2", "const float c1 = (float)(sqrt(2.0 / (double)D));", "const float c1 = (float)(sqrt(1.0 / (double)D));", 0),
