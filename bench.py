@@ -404,7 +404,8 @@ def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, attn_seqs=64):
 
 
 def run_variants(torch, kvq, dev, stream, x, out, s_t, G, w):
-    """The codec's format variants on the same batch, with one lambda table per
+    """The codec's format variants (and the SRFT rotation with lambda after it,
+    the paper's configuration) on the same batch, with one lambda table per
     (layer, K/V, head): 36 x 2 x 8 = 576 tables of 128 channels, each over the
     32,768 rows of its tokens.  Algorithmic bytes per vector: 2D (fp16 row) +
     code bytes (D/2 or D) + 2D/G (scales), read once and written once."""
@@ -417,19 +418,21 @@ def run_variants(torch, kvq, dev, stream, x, out, s_t, G, w):
     tables = torch.from_numpy(gen.uniform(0.5, 2.0, (ntab, D)).astype(np.float32)).to(dev)
     peak, _ = hbm_peak()
     res = {"lambda_tables": ntab, "rows_per_table": rows}
-    for bits, after in ((4, True), (8, False), (8, True)):
+    for bits, after, srft in ((4, True, False), (8, False, False), (8, True, False),
+                              (4, True, True)):
         cb = D // 2 if bits == 4 else D
         codes = torch.empty((n, cb), dtype=torch.uint8, device=dev)
         scales = torch.empty((n, D // G), dtype=torch.float16, device=dev)
         q_ms = _event_ms(torch, stream, lambda: kvq.quantize_ex(
             x, tables, s_t, G, bits=bits, lambda_after=after, lambda_rows=rows,
-            codes=codes, scales=scales, stream=stream), 10)
+            codes=codes, scales=scales, stream=stream, srft=srft), 10)
         d_ms = _event_ms(torch, stream, lambda: kvq.dequantize_ex(
             codes, scales, tables, s_t, G, bits=bits, lambda_after=after, lambda_rows=rows,
-            out=out, stream=stream), 10)
+            out=out, stream=stream, srft=srft), 10)
         bpv = 2 * D + cb + 2 * (D // G)
         qg, dg = bpv * n / (q_ms / 1e3) / 1e9, bpv * n / (d_ms / 1e3) / 1e9
-        res[f"int{bits}_lambda_{'after' if after else 'before'}"] = {
+        name = f"int{bits}_lambda_{'after' if after else 'before'}" + ("_srft" if srft else "")
+        res[name] = {
             "bytes_per_vector": bpv,
             "quantize_ms": round(q_ms, 4), "quantize_gbs": round(qg, 1),
             "quantize_frac_of_peak": round(qg / peak, 4),

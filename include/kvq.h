@@ -146,14 +146,20 @@ int kvq_roundtrip(const uint16_t *x, const float *lambda, const int8_t *signs,
                   uint8_t *packed, uint16_t *scales, void *stream);
 
 /*
- * kvq_quantize_ex / kvq_dequantize_ex -- the codec with format options:
- *   lambda_after  0: lambda before the rotation, y = H diag(s)(lambda . x)/sqrt(D)
- *                    (as kvq_quantize); 1: after it, y = lambda . (H diag(s) x
- *                    / sqrt(D)), the order of "When Quantization Is Free",
- *                    technical summary, Methodologie 2 (transform of diag(s) x,
- *                    then the per-channel lambda rescale).  The inverse divides
- *                    by lambda (fp32 multiply by IEEE 1/lambda) before its
- *                    transform instead of after.
+ * kvq_quantize_ex / kvq_dequantize_ex -- the codec with format options.
+ *   flags bit 0 (KVQ_LAMBDA_AFTER)  0: lambda before the rotation, y =
+ *                    R (lambda . x) (as kvq_quantize); 1: after it, y =
+ *                    lambda . (R x), the order of "When Quantization Is
+ *                    Free", technical summary, Methodologie 2 (transform of
+ *                    diag(s) x, then the per-channel lambda rescale).  The
+ *                    inverse divides by lambda (fp32 multiply by IEEE
+ *                    1/lambda) before its transform instead of after.
+ *   flags bit 1 (KVQ_SRFT)  R = H diag(s) / sqrt(D) (0), or the SRFT (1):
+ *                    pack(F diag(s) .), F the unitary DFT (same summary,
+ *                    Methodologie 1), computed as a length-D/2 complex FFT
+ *                    in radix-2 Stockham stages with the Hermitian unpacking
+ *                    y0 = X_0, y1 = X_D/2, (y_2k, y_2k+1) = sqrt(2) (Re, Im)
+ *                    X_k, all divided by sqrt(D).
  *   bits          4: int4 codes packed two per byte as kvq_quantize, S =
  *                    fp16(max|y| / 7); 8: one int8 code per byte (two's
  *                    complement), S = fp16(max|y| / 127), codes in [-128, 127].
@@ -165,19 +171,21 @@ int kvq_roundtrip(const uint16_t *x, const float *lambda, const int8_t *signs,
  *   codes         uint8 [n_vec][D/2] (bits 4) or [n_vec][D] (bits 8),
  *                 16-byte aligned.  Other arguments as for kvq_quantize /
  *                 kvq_dequantize.
- * D must be 128 (else KVQ_ERR_DIM); group in {16, 32, 64} and bits in {4, 8}
- * (else KVQ_ERR_GROUP); n_vec, lambda_rows, n_lambda out of range ->
- * KVQ_ERR_COUNT.  Results are bit-identical to the oracle's definition of each
- * option; bits = 4, lambda_after = 0 and one table reproduce kvq_quantize /
+ * D must be 128 (else KVQ_ERR_DIM); group in {16, 32, 64}, bits in {4, 8} and
+ * no other flag bits (else KVQ_ERR_GROUP); n_vec, lambda_rows, n_lambda out of
+ * range -> KVQ_ERR_COUNT.  Results are bit-identical to the oracle's definition
+ * of each option; bits = 4, flags = 0 and one table reproduce kvq_quantize /
  * kvq_dequantize exactly.
  */
+#define KVQ_LAMBDA_AFTER 1
+#define KVQ_SRFT 2
 int kvq_quantize_ex(const uint16_t *x, const float *lambda, const int8_t *signs,
-                    int64_t n_vec, int D, int group, int bits, int lambda_after,
+                    int64_t n_vec, int D, int group, int bits, int flags,
                     int64_t lambda_rows, int n_lambda, uint8_t *codes,
                     uint16_t *scales, void *stream);
 int kvq_dequantize_ex(const uint8_t *codes, const uint16_t *scales,
                       const float *lambda, const int8_t *signs, int64_t n_vec,
-                      int D, int group, int bits, int lambda_after,
+                      int D, int group, int bits, int flags,
                       int64_t lambda_rows, int n_lambda, uint16_t *x_out,
                       void *stream);
 

@@ -30,14 +30,34 @@ FLAGS = [
 
 
 def build(verbose: bool = False, extra: list[str] | None = None) -> str:
-    cmd = [NVCC, *FLAGS, *(extra or []), "-I", INCLUDE, *SOURCES, "-o", LIBRARY]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if res.returncode != 0:
-        raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
-    if verbose:
-        sys.stderr.write(res.stderr)
+    """Compile every translation unit to an object in parallel, then link."""
+    import concurrent.futures
+    import tempfile
+
+    compile_flags = [f for f in FLAGS if f not in ("-shared", "-cudart", "shared")
+                     and not f.startswith("-rpath")]
+    compile_flags = [f for f in compile_flags if f != "-Xlinker"]
+    with tempfile.TemporaryDirectory() as td:
+        objs = [os.path.join(td, os.path.basename(src) + ".o") for src in SOURCES]
+
+        def one(src, obj):
+            cmd = [NVCC, *compile_flags, *(extra or []), "-I", INCLUDE, "-c", src, "-o", obj]
+            if verbose:
+                cmd.insert(1, "-Xptxas=-v")
+            return subprocess.run(cmd, capture_output=True, text=True)
+
+        with concurrent.futures.ThreadPoolExecutor(len(SOURCES)) as ex:
+            results = list(ex.map(one, SOURCES, objs))
+        for res in results:
+            if res.returncode != 0:
+                raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
+            if verbose:
+                sys.stderr.write(res.stderr)
+        link = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "shared",
+                "-Xlinker", "-rpath,/usr/local/cuda/lib64", *objs, "-o", LIBRARY]
+        res = subprocess.run(link, capture_output=True, text=True)
+        if res.returncode != 0:
+            raise RuntimeError("nvcc link failed:\n" + res.stdout + res.stderr)
     return LIBRARY
 
 

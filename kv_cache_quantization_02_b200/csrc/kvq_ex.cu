@@ -457,6 +457,410 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const uint16_t* __re
 }
 
 // ---------------------------------------------------------------------------
+// The SRFT variants.  SRFT(x) = pack(F diag(s) x), F the unitary DFT ("When
+// Quantization Is Free", technical summary, Methodologie 1), computed as the
+// paper's kernel does (Methodologie 2): the length-64 complex FFT of
+// z_n = v_2n + i v_2n+1 in six radix-2 Stockham stages, then the Hermitian
+// unpacking into the orthonormal real packing y0 = X_0, y1 = X_64,
+// (y_2k, y_2k+1) = sqrt(2) (Re, Im) X_k, all / sqrt(128).  The lane holds its
+// vector in the natural pair layout z[n] = (v[2n], v[2n+1]) (two fp16
+// channels of one 32-bit word), every complex product is the oracle's four
+// products and two sums, and the twiddles are the host's double cos / sin
+// rounded to fp32, so the results are bit-identical.
+// ---------------------------------------------------------------------------
+
+constexpr int kFN = kD / 2;             // complex FFT length (64)
+
+struct SrftTw {
+  float2 wn[kFN / 2];                   // omega_64^k, k < 32
+  float2 wd[kFN + 1];                   // omega_128^k, k <= 64
+};
+
+// (a - b) * w with the oracle's operation order: re = d.x w.x - d.y w.y,
+// im = d.x w.y + d.y w.x, each product and sum rounded once.
+__device__ __forceinline__ float2 cmul_rn(float2 d, float2 w) {
+  const float2 p0 = __fmul2_rn(d, make_float2(w.x, w.x));              // (d.x w.x, d.y w.x)
+  const float2 p1 = __fmul2_rn(make_float2(d.y, d.x), make_float2(w.y, w.y));   // (d.y w.y, d.x w.y)
+  return make_float2(__fsub_rn(p0.x, p1.x), __fadd_rn(p1.y, p0.y));
+}
+
+// Stockham radix-2 FFT of 64 points in registers; INV: conjugate twiddles.
+template <bool INV>
+__device__ __forceinline__ void stockham64(float2 (&x)[kFN], const SrftTw& tw) {
+  float2 y[kFN];
+#pragma unroll
+  for (int st = 0; st < 6; ++st) {
+    const int n = kFN >> st, m = n / 2, sstr = 1 << st;
+#pragma unroll
+    for (int p = 0; p < m; ++p) {
+      float2 w = tw.wn[p * sstr];
+      if (INV) w.y = -w.y;
+#pragma unroll
+      for (int q = 0; q < sstr; ++q) {
+        const float2 a = x[q + sstr * p], b = x[q + sstr * (p + m)];
+        y[q + sstr * 2 * p] = __fadd2_rn(a, b);
+        y[q + sstr * (2 * p + 1)] = cmul_rn(fsub2(a, b), w);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kFN; ++i) x[i] = y[i];
+  }
+}
+
+// Forward extraction: X_k from Z_k and Z_(64-k) (indices mod 64).
+__device__ __forceinline__ float2 real_bin(const float2 (&z)[kFN], int k, const SrftTw& tw) {
+  const float2 A = z[k % kFN];
+  const float2 zb = z[(kFN - k) % kFN];
+  const float2 B = make_float2(zb.x, -zb.y);
+  const float2 E = __fmul2_rn(__fadd2_rn(A, B), make_float2(0.5f, 0.5f));
+  const float2 Dd = fsub2(A, B);
+  const float2 O = __fmul2_rn(make_float2(Dd.y, Dd.x), make_float2(0.5f, -0.5f));   // (A - B) / 2i
+  return __fadd2_rn(E, cmul_rn(O, tw.wd[k]));
+}
+
+// Bins k and 64 - k read the same two spectrum values, so they are computed
+// together and written back in place (each Z is then dead).
+__device__ __forceinline__ void srft_fwd(float2 (&z)[kFN], const SrftTw& tw, float c0, float c1) {
+  stockham64<false>(z, tw);
+  const float2 x0 = real_bin(z, 0, tw), xn = real_bin(z, kFN, tw);
+#pragma unroll
+  for (int k = 1; k < kFN / 2; ++k) {
+    const float2 xk = real_bin(z, k, tw), xm = real_bin(z, kFN - k, tw);
+    z[k] = __fmul2_rn(xk, make_float2(c1, c1));
+    z[kFN - k] = __fmul2_rn(xm, make_float2(c1, c1));
+  }
+  z[kFN / 2] = __fmul2_rn(real_bin(z, kFN / 2, tw), make_float2(c1, c1));
+  z[0] = make_float2(__fmul_rn(x0.x, c0), __fmul_rn(xn.x, c0));
+}
+
+// Inverse (the transpose): packed pairs u[k] = (y_2k, y_2k+1), u[0] = (y0, y1).
+// Z'_k = E + i O from U_k and conj U_(64-k), E = (U_k + conj U_(64-k)) / 2,
+// O = (U_k - conj U_(64-k)) conj(omega_128^k) / 2.
+__device__ __forceinline__ float2 inv_bin(float2 A, float2 Bc, int k, const SrftTw& tw) {
+  const float2 B = make_float2(Bc.x, -Bc.y);
+  const float2 E = __fmul2_rn(__fadd2_rn(A, B), make_float2(0.5f, 0.5f));
+  const float2 w = make_float2(tw.wd[k].x, -tw.wd[k].y);
+  const float2 O = __fmul2_rn(cmul_rn(fsub2(A, B), w), make_float2(0.5f, 0.5f));
+  return make_float2(__fsub_rn(E.x, O.y), __fadd_rn(E.y, O.x));
+}
+
+// Inverse (the transpose): packed pairs z[k] = (y_2k, y_2k+1), z[0] = (y0, y1).
+// U_0 = 2 c0 y0, U_64 = 2 c0 y1, U_k = c1 (y_2k, y_2k+1); bins k and 64 - k
+// are again formed together, in place.
+__device__ __forceinline__ void srft_inv(float2 (&z)[kFN], const SrftTw& tw, float c0, float c1) {
+  const float2 u0 = make_float2(__fmul_rn(__fmul_rn(z[0].x, c0), 2.0f), 0.0f);
+  const float2 un = make_float2(__fmul_rn(__fmul_rn(z[0].y, c0), 2.0f), 0.0f);
+  z[0] = inv_bin(u0, un, 0, tw);
+#pragma unroll
+  for (int k = 1; k < kFN / 2; ++k) {
+    const float2 uk = __fmul2_rn(z[k], make_float2(c1, c1));
+    const float2 um = __fmul2_rn(z[kFN - k], make_float2(c1, c1));
+    z[k] = inv_bin(uk, um, k, tw);
+    z[kFN - k] = inv_bin(um, uk, kFN - k, tw);
+  }
+  {
+    const float2 uh = __fmul2_rn(z[kFN / 2], make_float2(c1, c1));
+    z[kFN / 2] = inv_bin(uh, uh, kFN / 2, tw);
+  }
+  stockham64<true>(z, tw);
+}
+
+// The warp's per-channel table in natural order: tab[q] = (t[4q] .. t[4q+3]).
+__device__ __forceinline__ void build_table_nat(float4* tab, const ExArgs& a, int id, int mode, int lane) {
+  const float* lr = a.lam + static_cast<int64_t>(id) * kD;
+  float v[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int ch = 4 * lane + k;
+    float l = lr[ch];
+    if (mode >= 2) l = __frcp_rn(l);
+    v[k] = ((mode == 0 || mode == 2) && a.sgn[ch] < 0) ? -l : l;
+  }
+  tab[lane] = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void build_signs_nat(float4* stab, const ExArgs& a, int q) {
+  float v[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) v[k] = a.sgn[4 * q + k] < 0 ? -1.0f : 1.0f;
+  stab[q] = make_float4(v[0], v[1], v[2], v[3]);
+}
+
+template <int G, int BITS, bool AFTER>
+__global__ void __launch_bounds__(kXW * 32, 2)
+kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
+                         const __grid_constant__ SrftTw tw, float c0, float c1,
+                         uint8_t* __restrict__ codes, uint16_t* __restrict__ scales) {
+  using F = Fmt<BITS>;
+  constexpr int GP = G / 2;             // pairs per group
+  constexpr int NG = kD / G;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint8_t* wsm = smem + warp * 2 * kXStage;
+  uint8_t* hdr = smem + kXW * 2 * kXStage;
+  float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
+  float4* stab = reinterpret_cast<float4*>(hdr + kXW * 512);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + kHdrBars) + 2 * warp;
+  int* tq = reinterpret_cast<int*>(hdr + kHdrBars + 16 * kXW) + 2 * warp;
+  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + kHdrBars + 24 * kXW);
+  if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
+  if (tid == 0) *next = 0;
+  if (tid < 32) build_signs_nat(stab, a, tid);
+  __syncthreads();
+
+  const int64_t ntiles = (a.n + kWR - 1) / kWR;
+  const unsigned int mine = static_cast<unsigned int>((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  auto claim = [&]() -> int {
+    unsigned int i = 0;
+    if (lane == 0) i = atomicAdd(next, 1u);
+    i = __shfl_sync(kFullMask, i, 0);
+    return i < mine ? static_cast<int>(blockIdx.x + i * gridDim.x) : -1;
+  };
+  auto refill = [&](int stage) {
+    const int t = claim();
+    if (lane == 0) tq[stage] = t;
+    if (t < 0 || lane != 0) return;
+    mbar_expect_tx(&bar[stage], kXStage);
+    tensor_g2s(wsm + stage * kXStage, &maps.q[0], 0, t * kWR, &bar[stage]);
+    tensor_g2s(wsm + stage * kXStage + kQB, &maps.q[1], 0, t * kWR, &bar[stage]);
+  };
+  refill(0);
+  refill(1);
+  int cached = -1;
+  for (uint32_t k = 0;; ++k) {
+    const int stage = k & 1;
+    __syncwarp();
+    const int64_t tile = tq[stage];
+    if (tile < 0) break;
+    const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);
+    if (__any_sync(kFullMask, !ok)) {
+      if (lane == 0) atomicOr(&g_ex_fault, 1u);
+      if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinX);
+      return;
+    }
+    const int id = table_id(a, tile * kWR);
+    if (id != cached) {
+      build_table_nat(tab, a, id, AFTER ? 1 : 0, lane);
+      cached = id;
+      __syncwarp();
+    }
+    const int64_t row = tile * kWR + lane;
+    const bool active = row < a.n;
+    const uint8_t* st = wsm + stage * kXStage;
+    float2 z[kFN];
+#pragma unroll
+    for (int c = 0; c < kD / 8; ++c) {                 // 16-byte chunk c: channels 8c .. 8c+7
+      const uint4 xv = *reinterpret_cast<const uint4*>(st + xtile_off(c / 8, lane, c % 8));
+      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+      const float4 l0 = AFTER ? stab[2 * c] : tab[2 * c];          // channels 8c .. 8c+3
+      const float4 l1 = AFTER ? stab[2 * c + 1] : tab[2 * c + 1];  // 8c+4 .. 8c+7
+      z[4 * c] = __fmul2_rn(half2_bits_to_float2(xw[0]), make_float2(l0.x, l0.y));
+      z[4 * c + 1] = __fmul2_rn(half2_bits_to_float2(xw[1]), make_float2(l0.z, l0.w));
+      z[4 * c + 2] = __fmul2_rn(half2_bits_to_float2(xw[2]), make_float2(l1.x, l1.y));
+      z[4 * c + 3] = __fmul2_rn(half2_bits_to_float2(xw[3]), make_float2(l1.z, l1.w));
+    }
+    __syncwarp();
+    refill(stage);
+
+    srft_fwd(z, tw, c0, c1);
+    if constexpr (AFTER) {
+#pragma unroll
+      for (int q = 0; q < kFN / 2; ++q) {
+        const float4 l = tab[q];                      // lambda, channels 4q .. 4q+3
+        z[2 * q] = __fmul2_rn(z[2 * q], make_float2(l.x, l.y));
+        z[2 * q + 1] = __fmul2_rn(z[2 * q + 1], make_float2(l.z, l.w));
+      }
+    }
+    float r[NG];
+    uint16_t b[NG];
+#pragma unroll
+    for (int j = 0; j < NG; ++j) {
+      float am = 0.f;
+#pragma unroll
+      for (int m = 0; m < GP; ++m) am = amax3(am, z[j * GP + m].x, z[j * GP + m].y);
+      asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(b[j]) : "f"(__fdiv_rn(am, F::QMAX)));
+      const float sf = half_bits_to_float(b[j]);
+      r[j] = sf == 0.0f ? 0.0f : __frcp_rn(sf);
+    }
+    uint32_t out[F::CB / 4];
+    if constexpr (BITS == 4) {
+#pragma unroll
+      for (int k8 = 0; k8 < kD / 8; ++k8) {
+        int qv[8];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int m = 4 * k8 + t;
+          const float2 v = __fmul2_rn(z[m], make_float2(r[m / GP], r[m / GP]));
+          qv[2 * t] = __float2int_rn(v.x);
+          qv[2 * t + 1] = __float2int_rn(v.y);
+        }
+        out[k8] = pack8(qv);
+      }
+    } else {
+#pragma unroll
+      for (int k4 = 0; k4 < kD / 4; ++k4) {
+        const float2 v0 = __fmul2_rn(z[2 * k4], make_float2(r[(2 * k4) / GP], r[(2 * k4) / GP]));
+        const float2 v1 = __fmul2_rn(z[2 * k4 + 1], make_float2(r[(2 * k4 + 1) / GP], r[(2 * k4 + 1) / GP]));
+        out[k4] = pack4_s8(__float2int_rn(v0.x), __float2int_rn(v0.y), __float2int_rn(v1.x), __float2int_rn(v1.y));
+      }
+    }
+    if (active) {
+      uint8_t* dst = codes + row * F::CB;
+#pragma unroll
+      for (int k4 = 0; k4 < F::CB / 16; ++k4) {
+        const uint32_t t4[4] = {out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]};
+        st_v4(dst + 16 * k4, t4);
+      }
+      uint16_t* srow = scales + row * NG;
+#pragma unroll
+      for (int j = 0; j < NG; ++j) srow[j] = b[j];
+    }
+  }
+}
+
+template <int G, int BITS, bool AFTER>
+__global__ void __launch_bounds__(kXW * 32, 2)
+kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
+                           const ExArgs a, const __grid_constant__ SrftTw tw, float c0, float c1,
+                           uint16_t* __restrict__ out, int scale_copy) {
+  using F = Fmt<BITS>;
+  using L = DeqLayout<G, BITS>;
+  constexpr int GP = G / 2;
+  constexpr int NG = kD / G;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint8_t* wsm = smem + warp * L::WARP;
+  uint8_t* hdr = smem + kXW * L::WARP;
+  float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
+  float4* stab = reinterpret_cast<float4*>(hdr + kXW * 512);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + kHdrBars) + 2 * warp;
+  int* tq = reinterpret_cast<int*>(hdr + kHdrBars + 16 * kXW) + 2 * warp;
+  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + kHdrBars + 24 * kXW);
+  if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
+  if (tid == 0) *next = 0;
+  if (tid < 32) build_signs_nat(stab, a, tid);
+  __syncthreads();
+
+  const int64_t ntiles = (a.n + kWR - 1) / kWR;
+  const unsigned int mine = static_cast<unsigned int>((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  auto claim = [&]() -> int {
+    unsigned int i = 0;
+    if (lane == 0) i = atomicAdd(next, 1u);
+    i = __shfl_sync(kFullMask, i, 0);
+    return i < mine ? static_cast<int>(blockIdx.x + i * gridDim.x) : -1;
+  };
+  auto scale_bytes = [&](int64_t t) -> uint32_t {
+    if (!scale_copy) return 0;
+    const int64_t row0 = t * kWR;
+    const int valid = static_cast<int>(a.n - row0 < kWR ? a.n - row0 : kWR);
+    return static_cast<uint32_t>(valid * L::SPR) & ~15u;
+  };
+  auto refill = [&](int stage) {
+    const int t = claim();
+    if (lane == 0) tq[stage] = t;
+    if (t < 0 || lane != 0) return;
+    const int64_t row0 = static_cast<int64_t>(t) * kWR;
+    const int valid = static_cast<int>(a.n - row0 < kWR ? a.n - row0 : kWR);
+    const uint32_t sb = scale_bytes(t);
+    mbar_expect_tx(&bar[stage], static_cast<uint32_t>(valid) * F::CB + sb);
+    bulk_g2s(wsm + stage * L::STAGE, codes + row0 * F::CB, static_cast<uint32_t>(valid) * F::CB, &bar[stage]);
+    if (sb) bulk_g2s(wsm + stage * L::STAGE + L::WC, reinterpret_cast<const uint8_t*>(scales) + row0 * L::SPR, sb, &bar[stage]);
+  };
+  refill(0);
+  refill(1);
+  int cached = -1;
+  for (uint32_t k = 0;; ++k) {
+    const int stage = k & 1;
+    __syncwarp();
+    const int64_t tile = tq[stage];
+    if (tile < 0) break;
+    const int64_t row = tile * kWR + lane;
+    const int64_t rrow = row < a.n ? row : a.n - 1;
+    const bool sc_smem = static_cast<uint32_t>((lane + 1) * L::SPR) <= scale_bytes(tile);
+    const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);
+    if (__any_sync(kFullMask, !ok)) {
+      if (lane == 0) atomicOr(&g_ex_fault, 1u);
+      if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinX);
+      return;
+    }
+    const int id = table_id(a, tile * kWR);
+    if (id != cached) {
+      build_table_nat(tab, a, id, AFTER ? 3 : 2, lane);
+      cached = id;
+      __syncwarp();
+    }
+    const uint8_t* st = wsm + stage * L::STAGE;
+    const uint16_t* srow = sc_smem ? reinterpret_cast<const uint16_t*>(st + L::WC + lane * L::SPR)
+                                   : scales + rrow * NG;
+    uint16_t sv[NG];
+#pragma unroll
+    for (int j = 0; j < NG; ++j) sv[j] = srow[j];
+    const uint32_t* seg = reinterpret_cast<const uint32_t*>(st + lane * F::CB);
+    float2 z[kFN];
+    if constexpr (BITS == 4) {
+      const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
+#pragma unroll
+      for (int j = 0; j < kD / 8; ++j) {               // word j: channels 8j .. 8j+7
+        const uint32_t w = seg[j] ^ 0x88888888u, w4 = w >> 4;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const uint32_t sel = 0x0400u | (t << 8) | t;
+          const uint32_t e = (__byte_perm(w, w4, sel) & 0x000F000Fu) | 0x64006400u;
+          const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&e), bias);
+          const int m = 4 * j + t;                     // pair (2m, 2m+1)
+          z[m] = make_float2(mul_f16_f32(__low2half(h), sv[m / GP]), mul_f16_f32(__high2half(h), sv[m / GP]));
+        }
+      }
+    } else {
+      const __half2 bias = __floats2half2_rn(1152.0f, 1152.0f);
+#pragma unroll
+      for (int j = 0; j < kD / 4; ++j) {               // word j: channels 4j .. 4j+3
+        const uint32_t w = seg[j] ^ 0x80808080u;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const uint32_t sel = static_cast<uint32_t>(2 * t) | ((2u * t + 1) << 8);   // bytes 2t, 2t+1
+          const uint32_t e = (__byte_perm(w, 0u, sel) & 0x00FF00FFu) | 0x64006400u;
+          const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&e), bias);
+          const int m = 2 * j + t;
+          z[m] = make_float2(mul_f16_f32(__low2half(h), sv[m / GP]), mul_f16_f32(__high2half(h), sv[m / GP]));
+        }
+      }
+    }
+    __syncwarp();
+    refill(stage);
+    if constexpr (AFTER) {
+#pragma unroll
+      for (int q = 0; q < kFN / 2; ++q) {
+        const float4 l = tab[q];                      // 1/lambda
+        z[2 * q] = __fmul2_rn(z[2 * q], make_float2(l.x, l.y));
+        z[2 * q + 1] = __fmul2_rn(z[2 * q + 1], make_float2(l.z, l.w));
+      }
+    }
+    srft_inv(z, tw, c0, c1);
+    uint16_t* dst = out + (row < a.n ? row : 0) * kD;
+#pragma unroll
+    for (int c = 0; c < kD / 8; ++c) {
+      uint32_t hv[4];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float4 sg = stab[2 * c + t];
+        float2 v0 = __fmul2_rn(z[4 * c + 2 * t], make_float2(sg.x, sg.y));
+        float2 v1 = __fmul2_rn(z[4 * c + 2 * t + 1], make_float2(sg.z, sg.w));
+        if constexpr (!AFTER) {
+          const float4 l = tab[2 * c + t];            // s * (1/lambda): the sign again, exact
+          v0 = __fmul2_rn(z[4 * c + 2 * t], make_float2(l.x, l.y));
+          v1 = __fmul2_rn(z[4 * c + 2 * t + 1], make_float2(l.z, l.w));
+        }
+        hv[2 * t] = float2_to_half2_bits(v0.x, v0.y);
+        hv[2 * t + 1] = float2_to_half2_bits(v1.x, v1.y);
+      }
+      if (row < a.n) st_v4(dst + 8 * c, hv);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Launch plumbing.
 // ---------------------------------------------------------------------------
 
@@ -506,25 +910,13 @@ int check_ex(int D, int G, int bits, int64_t n, int64_t lambda_rows, int n_lambd
   return KVQ_OK;
 }
 
+int encode_x_maps(ExMaps& maps, const uint16_t* x, int64_t n);
+
 template <int G, int BITS, bool AFTER>
 int launch_qex(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* scales, cudaStream_t st) {
   ExMaps maps;
-  const EncodeTiledFn enc = encode_tiled();
-  if (enc == nullptr) return KVQ_ERR_LAUNCH;
-  for (int q = 0; q < 2; ++q) {
-    const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(a.n)};
-    const cuuint64_t strides[1] = {2 * kD};
-    const cuuint32_t box[2] = {64, kWR};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(&maps.q[q], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
-                           const_cast<char*>(reinterpret_cast<const char*>(x)) + 128 * q, dims, strides,
-                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-      g_ex_cuda_error = static_cast<int>(r);
-      return KVQ_ERR_LAUNCH;
-    }
-  }
+  const int rc = encode_x_maps(maps, x, a.n);
+  if (rc != KVQ_OK) return rc;
   auto k = kvq_quantize_ex_kernel<G, BITS, AFTER>;
   constexpr int smem = 1024 + kXW * 2 * kXStage + kHdrBytes;
   static std::atomic<int> ready[64];
@@ -544,6 +936,72 @@ int launch_dex(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, ui
   const int grid = ex_grid(k, a.n, smem, ready);
   (void)cudaGetLastError();
   k<<<grid, kXW * 32, smem, st>>>(codes, scales, a, out,
+                                  (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
+  return finish_ex();
+}
+
+// Twiddles of the SRFT: omega_M^k = (cos(2 pi k / M), -sin(2 pi k / M)) in
+// double, rounded to fp32 (built once).
+const SrftTw& srft_twiddles() {
+  static const SrftTw tw = [] {
+    SrftTw t{};
+    auto om = [](int k, int M) {
+      const double a = 2.0 * 3.14159265358979323846 * static_cast<double>(k) / static_cast<double>(M);
+      return make_float2(static_cast<float>(std::cos(a)), static_cast<float>(-std::sin(a)));
+    };
+    for (int k = 0; k < kFN / 2; ++k) t.wn[k] = om(k, kFN);
+    for (int k = 0; k <= kFN; ++k) t.wd[k] = om(k, kD);
+    return t;
+  }();
+  return tw;
+}
+const float kSrftC0 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kD)));
+const float kSrftC1 = static_cast<float>(std::sqrt(2.0 / static_cast<double>(kD)));
+
+int encode_x_maps(ExMaps& maps, const uint16_t* x, int64_t n) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return KVQ_ERR_LAUNCH;
+  for (int q = 0; q < 2; ++q) {
+    const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(n)};
+    const cuuint64_t strides[1] = {2 * kD};
+    const cuuint32_t box[2] = {64, kWR};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(&maps.q[q], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+                           const_cast<char*>(reinterpret_cast<const char*>(x)) + 128 * q, dims, strides,
+                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+      g_ex_cuda_error = static_cast<int>(r);
+      return KVQ_ERR_LAUNCH;
+    }
+  }
+  return KVQ_OK;
+}
+
+template <int G, int BITS, bool AFTER>
+int launch_qsrft(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* scales, cudaStream_t st) {
+  ExMaps maps;
+  const int rc = encode_x_maps(maps, x, a.n);
+  if (rc != KVQ_OK) return rc;
+  auto k = kvq_quantize_srft_kernel<G, BITS, AFTER>;
+  constexpr int smem = 1024 + kXW * 2 * kXStage + kHdrBytes;
+  static std::atomic<int> ready[64];
+  const int grid = ex_grid(k, a.n, smem, ready);
+  (void)cudaGetLastError();
+  k<<<grid, kXW * 32, smem, st>>>(maps, a, srft_twiddles(), kSrftC0, kSrftC1, codes, scales);
+  return finish_ex();
+}
+
+template <int G, int BITS, bool AFTER>
+int launch_dsrft(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, uint16_t* out,
+                 cudaStream_t st) {
+  using L = DeqLayout<G, BITS>;
+  auto k = kvq_dequantize_srft_kernel<G, BITS, AFTER>;
+  constexpr int smem = 128 + kXW * L::WARP + kHdrBytes;
+  static std::atomic<int> ready[64];
+  const int grid = ex_grid(k, a.n, smem, ready);
+  (void)cudaGetLastError();
+  k<<<grid, kXW * 32, smem, st>>>(codes, scales, a, srft_twiddles(), kSrftC0, kSrftC1, out,
                                   (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
   return finish_ex();
 }
@@ -585,10 +1043,11 @@ __attribute__((visibility("hidden"))) int kvq_ex_last_cuda_error() { return g_ex
 extern "C" {
 
 int kvq_quantize_ex(const uint16_t* x, const float* lambda, const int8_t* signs, int64_t n_vec,
-                    int D, int group, int bits, int lambda_after, int64_t lambda_rows,
+                    int D, int group, int bits, int flags, int64_t lambda_rows,
                     int n_lambda, uint8_t* codes, uint16_t* scales, void* stream) {
   const int rc = check_ex(D, group, bits, n_vec, lambda_rows, n_lambda);
   if (rc != KVQ_OK) return rc;
+  if ((flags & ~3) != 0) return KVQ_ERR_GROUP;
   if (n_vec == 0) return KVQ_OK;
   if (!x || !lambda || !signs || !codes || !scales) return KVQ_ERR_NULL;
   if (!aligned_to(x, 16) || !aligned_to(codes, 16) || !aligned_to(scales, 2) || !aligned_to(lambda, 4))
@@ -596,15 +1055,20 @@ int kvq_quantize_ex(const uint16_t* x, const float* lambda, const int8_t* signs,
   ExArgs a{lambda, signs, n_vec, lambda_rows, n_lambda,
            static_cast<float>(1.0 / std::sqrt(static_cast<double>(kD)))};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool lambda_after = (flags & 1) != 0;
+  if (flags & 2) {
+    KVQ_EX_DISPATCH(launch_qsrft, x, a, codes, scales, st)
+  }
   KVQ_EX_DISPATCH(launch_qex, x, a, codes, scales, st)
 }
 
 int kvq_dequantize_ex(const uint8_t* codes, const uint16_t* scales, const float* lambda,
                       const int8_t* signs, int64_t n_vec, int D, int group, int bits,
-                      int lambda_after, int64_t lambda_rows, int n_lambda, uint16_t* x_out,
+                      int flags, int64_t lambda_rows, int n_lambda, uint16_t* x_out,
                       void* stream) {
   const int rc = check_ex(D, group, bits, n_vec, lambda_rows, n_lambda);
   if (rc != KVQ_OK) return rc;
+  if ((flags & ~3) != 0) return KVQ_ERR_GROUP;
   if (n_vec == 0) return KVQ_OK;
   if (!codes || !scales || !lambda || !signs || !x_out) return KVQ_ERR_NULL;
   if (!aligned_to(codes, 16) || !aligned_to(x_out, 16) || !aligned_to(scales, 2) || !aligned_to(lambda, 4))
@@ -612,6 +1076,10 @@ int kvq_dequantize_ex(const uint8_t* codes, const uint16_t* scales, const float*
   ExArgs a{lambda, signs, n_vec, lambda_rows, n_lambda,
            static_cast<float>(1.0 / std::sqrt(static_cast<double>(kD)))};
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool lambda_after = (flags & 1) != 0;
+  if (flags & 2) {
+    KVQ_EX_DISPATCH(launch_dsrft, codes, scales, a, x_out, st)
+  }
   KVQ_EX_DISPATCH(launch_dex, codes, scales, a, x_out, st)
 }
 

@@ -107,18 +107,26 @@ def kvq_dequantize(packed: int, scales: int, lam: int, signs: int, n_vec: int,
     return _lib.kvq_dequantize(packed, scales, lam, signs, n_vec, D, group, x_out, stream)
 
 
+KVQ_LAMBDA_AFTER = 1
+KVQ_SRFT = 2
+
+
 def kvq_quantize_ex(x: int, lam: int, signs: int, n_vec: int, D: int, group: int, bits: int,
-                    lambda_after: int, lambda_rows: int, n_lambda: int, codes: int, scales: int,
+                    flags: int, lambda_rows: int, n_lambda: int, codes: int, scales: int,
                     stream: int = 0) -> int:
-    return _lib.kvq_quantize_ex(x, lam, signs, n_vec, D, group, bits, lambda_after, lambda_rows,
+    return _lib.kvq_quantize_ex(x, lam, signs, n_vec, D, group, bits, flags, lambda_rows,
                                 n_lambda, codes, scales, stream)
 
 
 def kvq_dequantize_ex(codes: int, scales: int, lam: int, signs: int, n_vec: int, D: int,
-                      group: int, bits: int, lambda_after: int, lambda_rows: int, n_lambda: int,
+                      group: int, bits: int, flags: int, lambda_rows: int, n_lambda: int,
                       x_out: int, stream: int = 0) -> int:
-    return _lib.kvq_dequantize_ex(codes, scales, lam, signs, n_vec, D, group, bits, lambda_after,
+    return _lib.kvq_dequantize_ex(codes, scales, lam, signs, n_vec, D, group, bits, flags,
                                   lambda_rows, n_lambda, x_out, stream)
+
+
+def _ex_flags(lambda_after: bool, srft: bool) -> int:
+    return (KVQ_LAMBDA_AFTER if lambda_after else 0) | (KVQ_SRFT if srft else 0)
 
 
 def kvq_attention_decode(q: int, k_packed: int, k_scales: int, v_packed: int, v_scales: int,
@@ -259,7 +267,7 @@ def roundtrip(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: in
 def quantize_ex(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: int,
                 bits: int = 4, lambda_after: bool = False, lambda_rows: int | None = None,
                 codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
-                stream=None):
+                stream=None, srft: bool = False):
     """Format variants.  x fp16 [n, 128]; lam fp32 [n_lambda, 128] (or [128]);
     row r uses table (r // lambda_rows) % n_lambda.  -> (codes uint8 [n, 64 or
     128], scales fp16 [n, 128/group])."""
@@ -279,7 +287,7 @@ def quantize_ex(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: 
     _need(scales, torch.float16, (n, D // group), "scales")
     rows = lambda_rows if lambda_rows is not None else max(n, 1)
     rc = kvq_quantize_ex(x.data_ptr(), lam2.data_ptr(), signs.data_ptr(), n, D, group, bits,
-                         1 if lambda_after else 0, rows, lam2.shape[0], codes.data_ptr(),
+                         _ex_flags(lambda_after, srft), rows, lam2.shape[0], codes.data_ptr(),
                          scales.data_ptr(), _stream_handle(stream))
     if rc != KVQ_OK:
         raise KvqError(rc)
@@ -289,7 +297,7 @@ def quantize_ex(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: 
 def dequantize_ex(codes: torch.Tensor, scales: torch.Tensor, lam: torch.Tensor,
                   signs: torch.Tensor, group: int, bits: int = 4, lambda_after: bool = False,
                   lambda_rows: int | None = None, out: torch.Tensor | None = None,
-                  stream=None) -> torch.Tensor:
+                  stream=None, srft: bool = False) -> torch.Tensor:
     """Inverse of quantize_ex -> fp16 [n, 128]."""
     if codes.dim() != 2:
         raise ValueError("codes must be [n_vec, bytes]")
@@ -305,7 +313,7 @@ def dequantize_ex(codes: torch.Tensor, scales: torch.Tensor, lam: torch.Tensor,
     _need(out, torch.float16, (n, D), "out")
     rows = lambda_rows if lambda_rows is not None else max(n, 1)
     rc = kvq_dequantize_ex(codes.data_ptr(), scales.data_ptr(), lam2.data_ptr(), signs.data_ptr(),
-                           n, D, group, bits, 1 if lambda_after else 0, rows, lam2.shape[0],
+                           n, D, group, bits, _ex_flags(lambda_after, srft), rows, lam2.shape[0],
                            out.data_ptr(), _stream_handle(stream))
     if rc != KVQ_OK:
         raise KvqError(rc)

@@ -147,6 +147,8 @@ def test_codec_ex_errors(kvq):
     d = lambda **kw: kvq.kvq_dequantize_ex(kw.get("codes", A), A, A, A, kw.get("n", 64),
                                            kw.get("D", 128), kw.get("G", 32), kw.get("bits", 4),
                                            1, kw.get("rows", 64), kw.get("nl", 1), kw.get("out", A))
+    flag = lambda **kw: kvq.kvq_quantize_ex(A, A, A, 64, 128, 32, 4, kw["flags"], 64, 1, A, A)
+    assert flag(flags=4) == -4 and flag(flags=-1) == -4
     for f in (q, d):
         assert f(D=64) == -3 and f(D=256) == -3
         assert f(G=128) == -4 and f(G=8) == -4 and f(bits=5) == -4
