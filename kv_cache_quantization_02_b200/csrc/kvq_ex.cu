@@ -287,26 +287,29 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
 // ---------------------------------------------------------------------------
 // Dequantize variants: codes [n][CB] + fp16 scales [n][128/G] -> fp16 [n][128].
 // ---------------------------------------------------------------------------
+// A warp's shared memory: the swizzled fp16 staging tile its tensor stores
+// read (first, 1 KiB aligned), then two stages of codes and scales.
 template <int G, int BITS>
 struct DeqLayout {
   static constexpr int WC = kWR * Fmt<BITS>::CB;          // codes of one warp tile
   static constexpr int SPR = (kD / G) * 2;                // scale bytes per row
   static constexpr int WS = kWR * SPR;                    // scales of one warp tile (<= 512)
   static constexpr int STAGE = WC + WS;
-  static constexpr int WARP = 2 * STAGE;
+  static constexpr int WARP = (kXStage + 2 * STAGE + 1023) / 1024 * 1024;
 };
 
 template <int G, int BITS, bool AFTER>
 __global__ void __launch_bounds__(kXW * 32, 2)
 kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
-                         const ExArgs a, uint16_t* __restrict__ out, int scale_copy) {
+                         const ExArgs a, const __grid_constant__ ExMaps omaps, int scale_copy) {
   using F = Fmt<BITS>;
   using L = DeqLayout<G, BITS>;
   constexpr int NGH = kNP / G;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint8_t* wsm = smem + warp * L::WARP;
+  uint8_t* stage_out = smem + warp * L::WARP;              // swizzled fp16 staging tile
+  uint8_t* wsm = stage_out + kXStage;                      // two stages of codes and scales
   uint8_t* hdr = smem + kXW * L::WARP;
   float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
   float4* stab = reinterpret_cast<float4*>(hdr + kXW * 512);
@@ -359,6 +362,7 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const uint16_t* __re
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_ex_fault, 1u);
       if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinX);
+      if (lane == 0) bulk_wait0();
       return;
     }
     const int id = table_id(a, tile * kWR);
@@ -427,7 +431,8 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const uint16_t* __re
       }
     }
     fwht_pairs<kD, 1>(p, 0);
-    uint16_t* dst = out + (row < a.n ? row : 0) * kD;
+    if (lane == 0) bulk_wait_read0();   // the previous tile's stores have read the staging tile
+    __syncwarp();
 #pragma unroll
     for (int k4 = 0; k4 < kNP / 8; ++k4) {
       uint32_t lo[4], hi[4];
@@ -448,12 +453,18 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const uint16_t* __re
         lo[t] = float2_to_half2_bits(a0.x, a1.x);    // channels 2q, 2q+1
         hi[t] = float2_to_half2_bits(a0.y, a1.y);    // channels 64+2q, 64+2q+1
       }
-      if (row < a.n) {
-        st_v4(dst + 8 * k4, lo);
-        st_v4(dst + kNP + 8 * k4, hi);
-      }
+      *reinterpret_cast<uint4*>(stage_out + xtile_off(0, lane, k4)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      *reinterpret_cast<uint4*>(stage_out + xtile_off(1, lane, k4)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    }
+    fence_proxy_async();                // generic-proxy writes -> visible to the tensor stores
+    __syncwarp();
+    if (lane == 0) {
+      tensor_s2g(&omaps.q[0], 0, static_cast<int>(tile * kWR), stage_out);
+      tensor_s2g(&omaps.q[1], 0, static_cast<int>(tile * kWR), stage_out + kQB);
+      bulk_commit();
     }
   }
+  if (lane == 0) bulk_wait0();
 }
 
 // ---------------------------------------------------------------------------
@@ -722,15 +733,16 @@ template <int G, int BITS, bool AFTER>
 __global__ void __launch_bounds__(kXW * 32, 2)
 kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
                            const ExArgs a, const __grid_constant__ SrftTw tw, float c0, float c1,
-                           uint16_t* __restrict__ out, int scale_copy) {
+                           const __grid_constant__ ExMaps omaps, int scale_copy) {
   using F = Fmt<BITS>;
   using L = DeqLayout<G, BITS>;
   constexpr int GP = G / 2;
   constexpr int NG = kD / G;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint8_t* wsm = smem + warp * L::WARP;
+  uint8_t* stage_out = smem + warp * L::WARP;              // swizzled fp16 staging tile
+  uint8_t* wsm = stage_out + kXStage;                      // two stages of codes and scales
   uint8_t* hdr = smem + kXW * L::WARP;
   float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
   float4* stab = reinterpret_cast<float4*>(hdr + kXW * 512);
@@ -782,6 +794,7 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_ex_fault, 1u);
       if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinX);
+      if (lane == 0) bulk_wait0();
       return;
     }
     const int id = table_id(a, tile * kWR);
@@ -838,7 +851,8 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
       }
     }
     srft_inv(z, tw, c0, c1);
-    uint16_t* dst = out + (row < a.n ? row : 0) * kD;
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();
 #pragma unroll
     for (int c = 0; c < kD / 8; ++c) {
       uint32_t hv[4];
@@ -855,9 +869,17 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
         hv[2 * t] = float2_to_half2_bits(v0.x, v0.y);
         hv[2 * t + 1] = float2_to_half2_bits(v1.x, v1.y);
       }
-      if (row < a.n) st_v4(dst + 8 * c, hv);
+      *reinterpret_cast<uint4*>(stage_out + xtile_off(c / 8, lane, c % 8)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+    }
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) {
+      tensor_s2g(&omaps.q[0], 0, static_cast<int>(tile * kWR), stage_out);
+      tensor_s2g(&omaps.q[1], 0, static_cast<int>(tile * kWR), stage_out + kQB);
+      bulk_commit();
     }
   }
+  if (lane == 0) bulk_wait0();
 }
 
 // ---------------------------------------------------------------------------
@@ -930,12 +952,15 @@ template <int G, int BITS, bool AFTER>
 int launch_dex(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, uint16_t* out,
                cudaStream_t st) {
   using L = DeqLayout<G, BITS>;
+  ExMaps omaps;
+  const int rc = encode_x_maps(omaps, out, a.n);
+  if (rc != KVQ_OK) return rc;
   auto k = kvq_dequantize_ex_kernel<G, BITS, AFTER>;
-  constexpr int smem = 128 + kXW * L::WARP + kHdrBytes;
+  constexpr int smem = 1024 + kXW * L::WARP + kHdrBytes;
   static std::atomic<int> ready[64];
   const int grid = ex_grid(k, a.n, smem, ready);
   (void)cudaGetLastError();
-  k<<<grid, kXW * 32, smem, st>>>(codes, scales, a, out,
+  k<<<grid, kXW * 32, smem, st>>>(codes, scales, a, omaps,
                                   (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
   return finish_ex();
 }
@@ -996,12 +1021,15 @@ template <int G, int BITS, bool AFTER>
 int launch_dsrft(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, uint16_t* out,
                  cudaStream_t st) {
   using L = DeqLayout<G, BITS>;
+  ExMaps omaps;
+  const int rc = encode_x_maps(omaps, out, a.n);
+  if (rc != KVQ_OK) return rc;
   auto k = kvq_dequantize_srft_kernel<G, BITS, AFTER>;
-  constexpr int smem = 128 + kXW * L::WARP + kHdrBytes;
+  constexpr int smem = 1024 + kXW * L::WARP + kHdrBytes;
   static std::atomic<int> ready[64];
   const int grid = ex_grid(k, a.n, smem, ready);
   (void)cudaGetLastError();
-  k<<<grid, kXW * 32, smem, st>>>(codes, scales, a, srft_twiddles(), kSrftC0, kSrftC1, out,
+  k<<<grid, kXW * 32, smem, st>>>(codes, scales, a, srft_twiddles(), kSrftC0, kSrftC1, omaps,
                                   (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
   return finish_ex();
 }
