@@ -51,6 +51,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 
 #include "kvq.h"
 
@@ -135,6 +136,8 @@ struct Stream {
   static constexpr int NEXT = TQ + 8 * kWarps;
   static constexpr int HDR = NEXT + 16;
   static constexpr int QWARP = 2 * WTile<D>::WSTAGE;        // quantize: two fp16 input stages
+  static constexpr int QWARP_S =                            // ... plus the staged codes of one warp tile
+      QWARP + (WTile<D>::WROWS * (D / 2) + 1023) / 1024 * 1024;
   static constexpr int DWARP =                              // dequantize: output tile, 2 x (codes, scales)
       (WTile<D>::WSTAGE + 2 * WTile<D>::WPIN + 2 * kScaleBlock + 1023) / 1024 * 1024;
   static constexpr int smem(int per_warp, int warps) { return 1024 + warps * per_warp + HDR; }
@@ -180,10 +183,13 @@ __global__ void __launch_bounds__(NW * 32, NW == kWarps ? 1 : 3)
 kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restrict__ lam,
                     const int8_t* __restrict__ sgn, int64_t n, float c,
                     uint8_t* __restrict__ packed, uint16_t* __restrict__ scales,
-                    const int64_t* __restrict__ row_idx, int64_t cache_rows) {
+                    const int64_t* __restrict__ row_idx, int64_t cache_rows, int scale_vec,
+                    const __grid_constant__ CUtensorMap cmap) {
   using T = Tile<D>;
   using W = WTile<D>;
   constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF;
+  constexpr bool STG = !INDEXED;                // codes leave through a staged tensor store
+  constexpr int QW = STG ? Stream<D>::QWARP_S : Stream<D>::QWARP;
   constexpr int GX = (G < HALF) ? G : HALF;      // pairs spanned by one group (G <= HALF)
   constexpr int NGH = HALF / GX;                 // groups per half-lane
   extern __shared__ uint8_t smem_raw[];
@@ -191,12 +197,13 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   using L = Stream<D>;
-  uint8_t* hdr = smem + NW * L::QWARP;
+  uint8_t* hdr = smem + NW * QW;
   float4* tabw = reinterpret_cast<float4*>(hdr);
   uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + L::BARS) + 2 * warp;
   int* tq = reinterpret_cast<int*>(hdr + L::TQ) + 2 * warp;   // tile in each stage, -1: none
   unsigned int* next = reinterpret_cast<unsigned int*>(hdr + L::NEXT);
-  uint8_t* wsm = smem + warp * L::QWARP;
+  uint8_t* wsm = smem + warp * QW;
+  uint8_t* cst = wsm + 2 * W::WSTAGE;            // the warp tile's codes, swizzled (STG)
   const int sub = lane % LANES;
   const int rin = lane / LANES;
   fill_tab<D>(tabw, lam, sgn, false);
@@ -240,6 +247,7 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_kvq_fault, 1u);
       if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
+      if (STG && lane == 0) bulk_wait0();
       return;
     }
     const int64_t row = tile * W::WROWS + rin;
@@ -322,15 +330,59 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
       out[k8] = pack8(qa);
       out[k8 + NP / 8] = pack8(qb);
     }
-    if (active) {
-      uint8_t* dst = packed + orow * (D / 2) + sub * (EPT / 2);
+    // The codes of a warp tile are one contiguous block: each lane writes its
+    // row into the staging tile, laid out as the swizzled tensor store reads
+    // it (16-byte chunk c of row t at chunk c ^ ((t * D/2 / 128) mod D/32),
+    // so a quarter-warp's chunks fall in distinct banks), and lane 0 stores
+    // the tile with one tensor copy that skips rows past n.  Rows scattered
+    // by an index are stored by each lane.
+    if constexpr (STG) {
+      if (lane == 0) bulk_wait_read0();
+      __syncwarp();                              // the staging tile is free
+      constexpr int RB = D / 2;                  // code bytes per row
+      const int swz = ((rin * RB) >> 7) & (D / 32 - 1);
 #pragma unroll
       for (int k4 = 0; k4 < EPT / 32; ++k4) {
-        const uint32_t t4[4] = {out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]};
-        st_v4(dst + 16 * k4, t4);
+        const int cidx = sub * (EPT / 32) + k4;
+        *reinterpret_cast<uint4*>(cst + rin * RB + ((cidx ^ swz) << 4)) =
+            make_uint4(out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]);
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        tensor_s2g(&cmap, 0, static_cast<int>(tile * W::WROWS), cst);
+        bulk_commit();
+      }
+    }
+    if (active) {
+      if constexpr (!STG) {
+        uint8_t* dst = packed + orow * (D / 2) + sub * (EPT / 2);
+#pragma unroll
+        for (int k4 = 0; k4 < EPT / 32; ++k4) {
+          const uint32_t t4[4] = {out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]};
+          st_v4(dst + 16 * k4, t4);
+        }
       }
       uint16_t* srow = scales + orow * (D / G);
-      if constexpr (G <= HALF) {
+      if constexpr (G <= HALF && LANES == 1) {     // the row's D/G scales: one store when aligned
+        uint16_t sa[D / G];
+#pragma unroll
+        for (int j = 0; j < NGH; ++j) { sa[j] = bx[j]; sa[NGH + j] = by[j]; }
+        uint32_t sw[D / G / 2];
+#pragma unroll
+        for (int i = 0; i < D / G / 2; ++i) sw[i] = uint32_t(sa[2 * i]) | (uint32_t(sa[2 * i + 1]) << 16);
+        if (scale_vec) {
+          if constexpr (D / G == 2) *reinterpret_cast<uint32_t*>(srow) = sw[0];
+          else if constexpr (D / G == 4) *reinterpret_cast<uint2*>(srow) = make_uint2(sw[0], sw[1]);
+          else *reinterpret_cast<uint4*>(srow) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < NGH; ++j) {
+            srow[j] = bx[j];
+            srow[NGH + j] = by[j];
+          }
+        }
+      } else if constexpr (G <= HALF) {
 #pragma unroll
         for (int j = 0; j < NGH; ++j) {
           srow[sub * (EPT / G) + j] = bx[j];
@@ -341,6 +393,7 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
       }
     }
   }
+  if (STG && lane == 0) bulk_wait0();
 }
 
 // ---------------------------------------------------------------------------
@@ -815,6 +868,28 @@ int make_row_maps(RowMaps& m, const void* base, int64_t n, int box_rows = Tile<D
   return KVQ_OK;
 }
 
+// The packed codes at `base` as one 2-D map: D/2 bytes x n rows, box
+// D/2 x (one warp tile), swizzled over the row's width (32, 64 or 128 bytes).
+template <int D>
+int make_code_map(CUtensorMap& m, void* base, int64_t n) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return KVQ_ERR_LAUNCH;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D / 2), static_cast<cuuint64_t>(n)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D / 2)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(D / 2), static_cast<cuuint32_t>(WTile<D>::WROWS)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_32B
+                               : D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_last_cuda_error = static_cast<int>(r);
+    return KVQ_ERR_LAUNCH;
+  }
+  return KVQ_OK;
+}
+
 inline bool aligned(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }
@@ -842,10 +917,20 @@ int launch_quantize_nw(const RowMaps& maps, int dev, int sms, const float* lam, 
                        int64_t n, uint8_t* packed, uint16_t* scales, const int64_t* row_idx,
                        int64_t cache_rows, cudaStream_t st) {
   auto k = kvq_quantize_kernel<D, G, INDEXED, NW>;
-  constexpr int smem = Stream<D>::smem(Stream<D>::QWARP, NW);
+  constexpr bool STG = !INDEXED;
+  constexpr int smem = Stream<D>::smem(STG ? Stream<D>::QWARP_S : Stream<D>::QWARP, NW);
   const int grid = stream_grid<INDEXED ? 2 : 0, D, G, NW>(k, dev, sms, n, smem);
+  CUtensorMap cmap;
+  memset(&cmap, 0, sizeof(cmap));
+  if (STG) {
+    const int rc = make_code_map<D>(cmap, packed, n);
+    if (rc != KVQ_OK) return rc;
+  }
+  constexpr uintptr_t kScaleRow = (D / G) * 2 < 16 ? (D / G) * 2 : 16;   // bytes of one scale store
+  const int svec = (reinterpret_cast<uintptr_t>(scales) % kScaleRow) == 0;
   (void)cudaGetLastError();
-  k<<<grid, NW * 32, smem, st>>>(maps, lam, s, n, norm_const(D), packed, scales, row_idx, cache_rows);
+  k<<<grid, NW * 32, smem, st>>>(maps, lam, s, n, norm_const(D), packed, scales, row_idx, cache_rows,
+                                 svec, cmap);
   return finish_launch();
 }
 
