@@ -399,7 +399,104 @@ def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, attn_seqs=64):
     }
     if D == 128:
         res["codec_variants"] = run_variants(torch, kvq, dev, stream, x, out, s_t, G, w)
-        res["attention_decode"] = run_attention(torch, kvq, dev, stream, lam_t, s_t, G, attn_seqs)
+        cache = build_decode_cache(torch, kvq, dev, stream, lam_t, s_t, G, attn_seqs)
+        res["attention_decode"] = run_attention(torch, kvq, dev, stream, lam_t, s_t, G, cache)
+        res["decode_step"] = run_decode_step(torch, kvq, dev, stream, lam_t, s_t, G, cache,
+                                             steps=1000 if attn_seqs == 64 else 20)
+        del cache
+        torch.cuda.empty_cache()
+        res["configs"] = run_configs(torch, kvq, dev, stream)
+        res["d256"] = run_d256(torch, kvq, dev, stream)
+    return res
+
+
+def _flushed_ms(torch, stream, fn, reps, flush):
+    """Per-rep CUDA-event times of fn, the L2 flushed before each rep by a
+    write of `flush` (twice the L2's 126 MB).  (median, min, max) in ms."""
+    fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for a, b in ev:
+        flush.zero_()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    t = sorted(a.elapsed_time(b) for a, b in ev)
+    return t[len(t) // 2], t[0], t[-1]
+
+
+CONFIG_CASES = (("tiny", 32), ("qwen2.5-1.5b", 32), ("gemma-3-1b", 32), ("gemma-3-1b", 64))
+
+
+def run_configs(torch, kvq, dev, stream, reps=20):
+    """The smaller configurations (each batch fits in L2): quantize and
+    dequantize timed one rep at a time with the L2 flushed before each rep;
+    median, min and max in microseconds."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    peak, _ = hbm_peak()
+    res = {"protocol": f"{reps} reps, L2 flushed (256 MB write) before each; median/min/max"}
+    for name, G in CONFIG_CASES:
+        w = workloads.WORKLOADS[name]
+        D, n = w.D, w.n_vec
+        lam, s = workloads.params(D, w.seed)
+        lt, st = torch.from_numpy(lam).to(dev), torch.from_numpy(s).to(dev)
+        x = workloads.device_rows(w, n, dev)
+        pk = torch.empty((n, D // 2), dtype=torch.uint8, device=dev)
+        sc = torch.empty((n, D // G), dtype=torch.float16, device=dev)
+        out = torch.empty_like(x)
+        q = _flushed_ms(torch, stream, lambda: kvq.quantize(
+            x, lt, st, G, packed=pk, scales=sc, stream=stream), reps, flush)
+        d = _flushed_ms(torch, stream, lambda: kvq.dequantize(
+            pk, sc, lt, st, G, out=out, stream=stream), reps, flush)
+        bpv = bytes_per_vector(D, G)
+        res[f"{name}_g{G}"] = {
+            "n_vec": n, "D": D, "G": G, "bytes_per_vector": bpv,
+            "quantize_us": [round(v * 1e3, 2) for v in q],
+            "dequantize_us": [round(v * 1e3, 2) for v in d],
+            "quantize_gvec_s": round(n / (q[0] / 1e3) / 1e9, 3),
+            "dequantize_gvec_s": round(n / (d[0] / 1e3) / 1e9, 3),
+            "quantize_gbs": round(bpv * n / (q[0] / 1e3) / 1e9, 1),
+            "dequantize_gbs": round(bpv * n / (d[0] / 1e3) / 1e9, 1),
+        }
+        del x, pk, sc, out
+    del flush
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_d256(torch, kvq, dev, stream, n=9_437_184):
+    """D = 256 on a batch as large in bytes as the prefill batch: 9,437,184
+    rows of the Gemma-3-1B distribution (6.19 GB per launch at G = 32), far
+    above L2; G = 32 and 64."""
+    w = workloads.WORKLOADS["gemma-3-1b"]
+    D = w.D
+    lam, s = workloads.params(D, w.seed)
+    lt, st = torch.from_numpy(lam).to(dev), torch.from_numpy(s).to(dev)
+    x = workloads.device_rows(w, n, dev)
+    out = torch.empty_like(x)
+    peak, _ = hbm_peak()
+    res = {"n_vec": n, "D": D}
+    for G in (32, 64):
+        pk = torch.empty((n, D // 2), dtype=torch.uint8, device=dev)
+        sc = torch.empty((n, D // G), dtype=torch.float16, device=dev)
+        q_ms = _event_ms(torch, stream, lambda: kvq.quantize(
+            x, lt, st, G, packed=pk, scales=sc, stream=stream), 10)
+        d_ms = _event_ms(torch, stream, lambda: kvq.dequantize(
+            pk, sc, lt, st, G, out=out, stream=stream), 10)
+        bpv = bytes_per_vector(D, G)
+        qg, dg = bpv * n / (q_ms / 1e3) / 1e9, bpv * n / (d_ms / 1e3) / 1e9
+        res[f"g{G}"] = {
+            "bytes_per_vector": bpv,
+            "quantize_ms": round(q_ms, 4), "quantize_gvec_s": round(n / (q_ms / 1e3) / 1e9, 3),
+            "quantize_gbs": round(qg, 1), "quantize_frac_of_peak": round(qg / peak, 4),
+            "dequantize_ms": round(d_ms, 4), "dequantize_gvec_s": round(n / (d_ms / 1e3) / 1e9, 3),
+            "dequantize_gbs": round(dg, 1), "dequantize_frac_of_peak": round(dg / peak, 4),
+        }
+        del pk, sc
+    del x, out
+    torch.cuda.empty_cache()
     return res
 
 
@@ -443,29 +540,42 @@ def run_variants(torch, kvq, dev, stream, x, out, s_t, G, w):
     return res
 
 
-def run_attention(torch, kvq, dev, stream, lam_t, s_t, G, seqs=64):
-    """One decode step of attention over the whole int4 cache of the decode
-    configuration: 64 sequences x 36 layers (folded into the batch) x 8 KV
-    heads x 4096 positions, 32 query heads (Qwen3-8B's grouping), D = 128
-    (`seqs` other than 64 only for small profiling runs).  The cache holds
-    real quantize output of N(0,1) rows.  Algorithmic bytes: every K and V
-    code and scale once, plus q and the output."""
+DECODE_HQ, DECODE_HKV, DECODE_T = 32, 8, 4096
+
+
+def build_decode_cache(torch, kvq, dev, stream, lam_t, s_t, G, seqs=64):
+    """The int4 cache of the decode configuration: 64 sequences x 36 layers
+    (folded into the batch B) x 8 KV heads x 4096 positions, K and V, D = 128,
+    holding real quantize output of N(0,1) rows (`seqs` other than 64 only
+    for small profiling runs).  Codes [2][B][Hkv][T][D/2] and scales
+    [2][B][Hkv][T][D/G], index 0 = K, 1 = V."""
     c = workloads.WORKLOADS["decode-cache"]
-    B, Hq, Hkv, T, D = seqs * 36, 32, 8, 4096, 128
-    rows = B * Hkv * T
-    kp = torch.empty((B, Hkv, T, D // 2), dtype=torch.uint8, device=dev)
-    vp = torch.empty_like(kp)
-    ks = torch.empty((B, Hkv, T, D // G), dtype=torch.float16, device=dev)
-    vs = torch.empty_like(ks)
+    B, Hkv, T, D = seqs * 36, DECODE_HKV, DECODE_T, 128
+    rows = 2 * B * Hkv * T
+    pk = torch.empty((2, B, Hkv, T, D // 2), dtype=torch.uint8, device=dev)
+    sc = torch.empty((2, B, Hkv, T, D // G), dtype=torch.float16, device=dev)
+    pk2, sc2 = pk.view(rows, D // 2), sc.view(rows, D // G)
     chunk = 1 << 23
     buf = torch.empty((chunk, D), dtype=torch.float16, device=dev)
-    for j, (pk, sc) in enumerate(((kp, ks), (vp, vs))):
-        pk2, sc2 = pk.view(rows, D // 2), sc.view(rows, D // G)
-        for i, a in enumerate(range(0, rows, chunk)):
-            b = min(rows, a + chunk)
-            xr = workloads.device_rows(c, b - a, dev, seed_offset=2 * i + j, out=buf[: b - a])
-            kvq.quantize(xr, lam_t, s_t, G, packed=pk2[a:b], scales=sc2[a:b], stream=stream)
+    for i, a in enumerate(range(0, rows, chunk)):
+        b = min(rows, a + chunk)
+        xr = workloads.device_rows(c, b - a, dev, seed_offset=i, out=buf[: b - a])
+        kvq.quantize(xr, lam_t, s_t, G, packed=pk2[a:b], scales=sc2[a:b], stream=stream)
     del buf
+    return pk, sc
+
+
+def run_attention(torch, kvq, dev, stream, lam_t, s_t, G, cache):
+    """One decode step of attention over the whole int4 cache of the decode
+    configuration (32 query heads on 8 KV heads, Qwen3-8B's grouping).
+    Algorithmic bytes: every K and V code and scale once, plus q and the
+    output."""
+    c = workloads.WORKLOADS["decode-cache"]
+    pk, sc = cache
+    _, B, Hkv, T, _ = pk.shape
+    Hq, D = DECODE_HQ, 128
+    kp, vp, ks, vs = pk[0], pk[1], sc[0], sc[1]
+    rows = B * Hkv * T
     gen = torch.Generator(device=dev)
     gen.manual_seed(c.seed)
     q = torch.randn((B, Hq, D), device=dev, generator=gen).half()
@@ -480,10 +590,9 @@ def run_attention(torch, kvq, dev, stream, lam_t, s_t, G, seqs=64):
     byts = 2 * rows * (D // 2 + 2 * (D // G)) + 2 * q.numel() * 2
     peak, kind = hbm_peak()
     gbs = byts / (ms / 1e3) / 1e9
-    del kp, vp, ks, vs, q, out
-    torch.cuda.empty_cache()
+    del q, out
     return {
-        "shape": f"B={B} ({seqs} sequences x 36 layers), Hq={Hq}, Hkv={Hkv}, T={T}, D={D}, G={G}",
+        "shape": f"B={B} ({B // 36} sequences x 36 layers), Hq={Hq}, Hkv={Hkv}, T={T}, D={D}, G={G}",
         "ms": round(ms, 4),
         "algorithmic_bytes": byts,
         "gbs": round(gbs, 1),
@@ -491,6 +600,55 @@ def run_attention(torch, kvq, dev, stream, lam_t, s_t, G, seqs=64):
         "frac_of_peak": round(gbs / peak, 4),
         "peak_kind": kind,
         "traffic": traffic_per_launch("kvq_attention", rows),
+    }
+
+
+def run_decode_step(torch, kvq, dev, stream, lam_t, s_t, G, cache, steps=1000):
+    """The decode step of the dequantize-then-attend path on the same cache:
+    append one new K and V token per (sequence, layer, KV head) into its slot
+    (kvq_quantize_rows, 2 x B x 8 = 36,864 vectors at 64 sequences), then
+    dequantize the whole cache (150,994,944 vectors) into one reused fp16
+    buffer (38.7 GB).  Per-step CUDA-event times, p50 and p99."""
+    pk, sc = cache
+    two, B, Hkv, T, half = pk.shape
+    D = 2 * half
+    rows = two * B * Hkv * T
+    pk2, sc2 = pk.view(rows, D // 2), sc.view(rows, D // G)
+    a = workloads.WORKLOADS["decode-append"]
+    na = two * B * Hkv
+    xa = workloads.device_rows(a, na, dev)
+    base = torch.arange(na, device=dev, dtype=torch.int64) * T
+    idx = [base + (p % T) for p in range(8)]
+    out = torch.empty((rows, D), dtype=torch.float16, device=dev)
+
+    def one(i):
+        kvq.quantize_rows(xa, lam_t, s_t, G, idx[i % 8], pk2, sc2, stream=stream)
+
+    one(0)
+    kvq.dequantize(pk2, sc2, lam_t, s_t, G, out=out, stream=stream)
+    torch.cuda.synchronize()
+    ev = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(steps)]
+    for i, (e0, e1, e2) in enumerate(ev):
+        e0.record(stream)
+        one(i)
+        e1.record(stream)
+        kvq.dequantize(pk2, sc2, lam_t, s_t, G, out=out, stream=stream)
+        e2.record(stream)
+    torch.cuda.synchronize()
+    ap = sorted(e0.elapsed_time(e1) for e0, e1, _ in ev)
+    dq = sorted(e1.elapsed_time(e2) for _, e1, e2 in ev)
+    pct = lambda t, p: t[min(len(t) - 1, int(p * len(t)))]
+    bpv = bytes_per_vector(D, G)
+    peak, _ = hbm_peak()
+    del xa, out
+    torch.cuda.empty_cache()
+    return {
+        "steps": steps, "append_vectors": na, "cache_vectors": rows,
+        "append_us_p50": round(pct(ap, 0.5) * 1e3, 2), "append_us_p99": round(pct(ap, 0.99) * 1e3, 2),
+        "dequant_ms_p50": round(pct(dq, 0.5), 4), "dequant_ms_p99": round(pct(dq, 0.99), 4),
+        "dequant_gvec_s": round(rows / (pct(dq, 0.5) / 1e3) / 1e9, 3),
+        "dequant_gbs": round(bpv * rows / (pct(dq, 0.5) / 1e3) / 1e9, 1),
+        "dequant_frac_of_peak": round(bpv * rows / (pct(dq, 0.5) / 1e3) / 1e9 / peak, 4),
     }
 
 
