@@ -23,7 +23,9 @@
 // bit-identical to it.
 //
 // Data movement.  Each warp streams its own warp tiles (32 / LANES vectors,
-// one per lane or lane pair) through a private double-buffered ring in
+// one per lane or lane pair: lane rin + 16 * sub holds part sub of row rin,
+// so the eight lanes of a quarter-warp phase hold eight different rows)
+// through a private double-buffered ring in
 // shared memory, so no block-wide barrier couples the warps.  The warps of a
 // block draw their next tile from a shared-memory counter over the block's
 // tiles (blockIdx.x + i * gridDim.x): a warp that the scheduler favours takes
@@ -32,11 +34,14 @@
 // tile moves as Q = D/64 tensor copies (one per 64-channel quarter of the
 // rows, 2-D maps of 64 channels x n rows with the 128-byte swizzle), issued by
 // one lane; chunk c of tile row t lands at chunk c ^ (t mod 8), so lanes
-// reading consecutive rows hit distinct bank groups.  Quantize: tensor loads
-// in, 16-byte code stores and 2-byte scale stores out.  Dequantize: a tile's
-// packed codes and its scales arrive as bulk copies; the lanes write their
-// fp16 rows into a swizzled staging tile that leaves as Q tensor stores (rows
-// past n are clipped by the copy engine).  No copy uses multicast.  Every
+// reading consecutive rows hit distinct bank groups.  The packed codes of a
+// warp tile are one 2-D tensor copy (D/2 bytes x the tile's rows) swizzled
+// over the row's 32, 64 or 128 bytes the same way.  Quantize: tensor loads
+// in; codes out through a staging tile and one tensor store, scales by
+// direct stores.  Dequantize: codes by tensor copy and scales by bulk copy
+// in; the lanes write their fp16 rows into a swizzled staging tile that
+// leaves as Q tensor stores (rows past n are clipped by the copy engine,
+// rows past n read as zeros on the way in).  No copy uses multicast.  Every
 // mbarrier wait is bounded; a warp that gives up sets a device fault word,
 // drains its own copies and returns (kvq_fault_status reads the word).
 //
@@ -204,8 +209,8 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
   unsigned int* next = reinterpret_cast<unsigned int*>(hdr + L::NEXT);
   uint8_t* wsm = smem + warp * QW;
   uint8_t* cst = wsm + 2 * W::WSTAGE;            // the warp tile's codes, swizzled (STG)
-  const int sub = lane % LANES;
-  const int rin = lane / LANES;
+  const int sub = lane / W::WROWS;               // which part of the vector
+  const int rin = lane % W::WROWS;               // which row of the warp tile
   fill_tab<D>(tabw, lam, sgn, false);
   if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   if (tid == 0) *next = 0;
@@ -284,7 +289,7 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
     refill(stage);
 
     // a2, a3: transform, normalise.
-    fwht_pairs<EPT, LANES>(p, sub);
+    fwht_pairs<EPT, LANES, 1, W::WROWS>(p, sub);
 #pragma unroll
     for (int m = 0; m < NP; ++m) p[m] = __fmul2_rn(p[m], c2);
 
@@ -309,7 +314,7 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
 #pragma unroll
       for (int m = 0; m < NP; ++m) a = amax3(a, p[m].x, p[m].y);
 #pragma unroll
-      for (int bit = 1; bit < G / EPT; bit <<= 1) a = fmaxf(a, __shfl_xor_sync(kFullMask, a, bit));
+      for (int bit = 1; bit < G / EPT; bit <<= 1) a = fmaxf(a, __shfl_xor_sync(kFullMask, a, bit * W::WROWS));
       bx[0] = group_scale(a, rx[0]);
       ry[0] = rx[0];
       by[0] = bx[0];
@@ -401,7 +406,7 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
 // ---------------------------------------------------------------------------
 template <int D, int G, int NW>
 __global__ void __launch_bounds__(NW * 32, NW == kWarps ? 1 : 3)
-kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __restrict__ scales,
+kvq_dequantize_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restrict__ scales,
                       const float* __restrict__ lam, const int8_t* __restrict__ sgn,
                       int64_t n, float c, const __grid_constant__ RowMaps maps, int scale_copy) {
   using T = Tile<D>;
@@ -429,8 +434,8 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
   uint8_t* stage_out = smem + warp * L::DWARP;                // swizzled fp16 warp tile
   uint8_t* stage_in = stage_out + W::WSTAGE;                  // two packed warp tiles
   uint8_t* stage_sc = stage_in + 2 * WPIN;                    // two scale blocks
-  const int sub = lane % LANES;
-  const int rin = lane / LANES;
+  const int sub = lane / WROWS;
+  const int rin = lane % WROWS;
   fill_tab<D>(tabw, lam, sgn, true);
   if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   if (tid == 0) *next = 0;
@@ -455,10 +460,9 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
   auto issue = [&](int64_t tile, int stage) {
     if (tile < 0 || lane != 0) return;
     const int64_t row0 = tile * WROWS;
-    const int valid = static_cast<int>(n - row0 < WROWS ? n - row0 : WROWS);
     const uint32_t sb = scale_bytes(tile);
-    mbar_expect_tx(&bar[stage], static_cast<uint32_t>(valid) * (D / 2) + sb);
-    bulk_g2s(stage_in + stage * WPIN, packed + row0 * (D / 2), static_cast<uint32_t>(valid) * (D / 2), &bar[stage]);
+    mbar_expect_tx(&bar[stage], static_cast<uint32_t>(WPIN) + sb);
+    tensor_g2s(stage_in + stage * WPIN, &cmap, 0, static_cast<int>(row0), &bar[stage]);
     if (sb) bulk_g2s(stage_sc + stage * WSC, reinterpret_cast<const uint8_t*>(scales) + row0 * SPR, sb, &bar[stage]);
   };
   auto refill = [&](int stage) {
@@ -500,11 +504,12 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
       sy[0] = sx[0];
     }
     // a8: the lane's EPT/2 bytes of codes; nibbles biased to n = q + 8.
-    const uint4* seg = reinterpret_cast<const uint4*>(stage_in + stage * WPIN + rin * (D / 2) + sub * (EPT / 2));
+    const uint8_t* crow = stage_in + stage * WPIN + rin * (D / 2);
+    const int cswz = ((rin * (D / 2)) >> 7) & (D / 32 - 1);
     uint32_t w[EPT / 8];
 #pragma unroll
     for (int j = 0; j < EPT / 32; ++j) {
-      const uint4 a = seg[j];
+      const uint4 a = *reinterpret_cast<const uint4*>(crow + (((sub * (EPT / 32) + j) ^ cswz) << 4));
       w[4 * j] = a.x ^ 0x88888888u;
       w[4 * j + 1] = a.y ^ 0x88888888u;
       w[4 * j + 2] = a.z ^ 0x88888888u;
@@ -557,7 +562,7 @@ kvq_dequantize_kernel(const uint8_t* __restrict__ packed, const uint16_t* __rest
                          mul_f16_f32(__high2half(hq[m]), sy[m / GX]));
     __syncwarp();             // codes and scales consumed: the input stage can be refilled
     refill(stage);
-    fwht_pairs<EPT, LANES, HG>(p, sub);
+    fwht_pairs<EPT, LANES, HG, WROWS>(p, sub);
 
     if (lane == 0) bulk_wait_read0();
     __syncwarp();             // the warp's staging tile is free
@@ -970,8 +975,11 @@ int launch_dequantize_nw(const RowMaps& maps, int dev, int sms, const uint8_t* p
   auto k = kvq_dequantize_kernel<D, G, NW>;
   constexpr int smem = Stream<D>::smem(Stream<D>::DWARP, NW);
   const int grid = stream_grid<1, D, G, NW>(k, dev, sms, n, smem);
+  CUtensorMap cmap;
+  const int rc = make_code_map<D>(cmap, const_cast<uint8_t*>(packed), n);
+  if (rc != KVQ_OK) return rc;
   (void)cudaGetLastError();
-  k<<<grid, NW * 32, smem, st>>>(packed, scales, lam, s, n, norm_const(D), maps,
+  k<<<grid, NW * 32, smem, st>>>(cmap, scales, lam, s, n, norm_const(D), maps,
                                  (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
   return finish_launch();
 }

@@ -87,9 +87,10 @@ __device__ __forceinline__ float mul_f16_f32(__half w, uint16_t s) {
 // ---------------------------------------------------------------------------
 // Walsh-Hadamard butterflies (unnormalised, Sylvester order) on one vector
 // held as pairs p[m] = (v[m], v[m+HALF]) by LANES lanes, from half-width H0
-// upwards (stages below H0 already applied).
+// upwards (stages below H0 already applied).  The vector's lanes are XS lane
+// ids apart: lane `sub` of the vector is lane rin + XS * sub of the warp.
 // ---------------------------------------------------------------------------
-template <int EPT, int LANES, int H0 = 1>
+template <int EPT, int LANES, int H0 = 1, int XS = 1>
 __device__ __forceinline__ void fwht_pairs(float2 (&p)[EPT / 2], int sub) {
   constexpr int NP = EPT / 2;
 #pragma unroll
@@ -119,8 +120,8 @@ __device__ __forceinline__ void fwht_pairs(float2 (&p)[EPT / 2], int sub) {
 #pragma unroll
     for (int m = 0; m < NP; ++m) {
       float2 o;
-      o.x = __shfl_xor_sync(kFullMask, p[m].x, bit);
-      o.y = __shfl_xor_sync(kFullMask, p[m].y, bit);
+      o.x = __shfl_xor_sync(kFullMask, p[m].x, bit * XS);
+      o.y = __shfl_xor_sync(kFullMask, p[m].y, bit * XS);
       p[m] = __ffma2_rn(sg2, p[m], o);
     }
   }
