@@ -32,6 +32,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstring>
 
 #include "kvq.h"
 
@@ -288,19 +289,32 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
 // Dequantize variants: codes [n][CB] + fp16 scales [n][128/G] -> fp16 [n][128].
 // ---------------------------------------------------------------------------
 // A warp's shared memory: the swizzled fp16 staging tile its tensor stores
-// read (first, 1 KiB aligned), then two stages of codes and scales.
+// read (first, 1 KiB aligned), the two stages' code tiles (each a multiple
+// of 1 KiB, so the copy engine's swizzle lines up with code_chunk), then the
+// two stages' scales.
 template <int G, int BITS>
 struct DeqLayout {
-  static constexpr int WC = kWR * Fmt<BITS>::CB;          // codes of one warp tile
+  static constexpr int WC = kWR * Fmt<BITS>::CB;          // codes of one warp tile: 2 or 4 KiB
   static constexpr int SPR = (kD / G) * 2;                // scale bytes per row
   static constexpr int WS = kWR * SPR;                    // scales of one warp tile (<= 512)
-  static constexpr int STAGE = WC + WS;
-  static constexpr int WARP = (kXStage + 2 * STAGE + 1023) / 1024 * 1024;
+  static constexpr int SC = 2 * WC;                       // offset of the scales after the staging tile
+  static constexpr int WARP = (kXStage + 2 * WC + 2 * WS + 1023) / 1024 * 1024;
 };
+
+// 16-byte chunk c of lane `lane`'s row of a code tile written by a tensor copy
+// swizzled over the row's CB bytes (64 or 128): chunk c of row t sits at
+// chunk c ^ ((t * CB / 128) mod CB/16), so the eight rows a quarter-warp
+// reads fall in distinct banks.
+template <int CB>
+__device__ __forceinline__ uint4 code_chunk(const uint8_t* tile, int lane, int c) {
+  const int swz = ((lane * CB) >> 7) & (CB / 16 - 1);
+  return *reinterpret_cast<const uint4*>(tile + lane * CB + ((c ^ swz) << 4));
+}
 
 template <int G, int BITS, bool AFTER>
 __global__ void __launch_bounds__(kXW * 32, 2)
-kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
+kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constant__ CUtensorMap cmap,
+                         const uint16_t* __restrict__ scales,
                          const ExArgs a, const __grid_constant__ ExMaps omaps, int scale_copy) {
   using F = Fmt<BITS>;
   using L = DeqLayout<G, BITS>;
@@ -309,7 +323,7 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const uint16_t* __re
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* stage_out = smem + warp * L::WARP;              // swizzled fp16 staging tile
-  uint8_t* wsm = stage_out + kXStage;                      // two stages of codes and scales
+  uint8_t* wsm = stage_out + kXStage;                      // two code tiles, then two scale blocks
   uint8_t* hdr = smem + kXW * L::WARP;
   float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
   float4* stab = reinterpret_cast<float4*>(hdr + kXW * 512);
@@ -340,11 +354,16 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const uint16_t* __re
     if (lane == 0) tq[stage] = t;
     if (t < 0 || lane != 0) return;
     const int64_t row0 = static_cast<int64_t>(t) * kWR;
-    const int valid = static_cast<int>(a.n - row0 < kWR ? a.n - row0 : kWR);
     const uint32_t sb = scale_bytes(t);
-    mbar_expect_tx(&bar[stage], static_cast<uint32_t>(valid) * F::CB + sb);
-    bulk_g2s(wsm + stage * L::STAGE, codes + row0 * F::CB, static_cast<uint32_t>(valid) * F::CB, &bar[stage]);
-    if (sb) bulk_g2s(wsm + stage * L::STAGE + L::WC, reinterpret_cast<const uint8_t*>(scales) + row0 * L::SPR, sb, &bar[stage]);
+    if constexpr (BITS == 8) {         // swizzled tensor copy: the copy engine fills the whole box
+      mbar_expect_tx(&bar[stage], static_cast<uint32_t>(L::WC) + sb);
+      tensor_g2s(wsm + stage * L::WC, &cmap, 0, static_cast<int>(row0), &bar[stage]);
+    } else {                           // plain bulk copy of the valid rows
+      const uint32_t cbytes = static_cast<uint32_t>(a.n - row0 < kWR ? a.n - row0 : kWR) * F::CB;
+      mbar_expect_tx(&bar[stage], cbytes + sb);
+      bulk_g2s(wsm + stage * L::WC, codes + row0 * F::CB, cbytes, &bar[stage]);
+    }
+    if (sb) bulk_g2s(wsm + L::SC + stage * L::WS, reinterpret_cast<const uint8_t*>(scales) + row0 * L::SPR, sb, &bar[stage]);
   };
   refill(0);
   refill(1);
@@ -371,8 +390,8 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const uint16_t* __re
       cached = id;
       __syncwarp();
     }
-    const uint8_t* st = wsm + stage * L::STAGE;
-    const uint16_t* srow = sc_smem ? reinterpret_cast<const uint16_t*>(st + L::WC + lane * L::SPR)
+    const uint8_t* st = wsm + stage * L::WC;
+    const uint16_t* srow = sc_smem ? reinterpret_cast<const uint16_t*>(wsm + L::SC + stage * L::WS + lane * L::SPR)
                                    : scales + rrow * (kD / G);
     uint16_t sx[NGH], sy[NGH];
 #pragma unroll
@@ -380,10 +399,12 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const uint16_t* __re
       sx[j] = srow[j];
       sy[j] = srow[NGH + j];
     }
-    // codes of the pair (m, m+64) as exact fp16 integers, then u = q S exactly
-    const uint2* seg = reinterpret_cast<const uint2*>(st + lane * F::CB);
+    // codes of the pair (m, m+64) as exact fp16 integers, then u = q S exactly.
+    // int4: the row is linear (64 bytes); int8: word w of the row is word
+    // w % 4 of swizzled chunk w / 4.
     float2 p[kNP];
     if constexpr (BITS == 4) {
+      const uint2* seg = reinterpret_cast<const uint2*>(st + lane * F::CB);
       const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
 #pragma unroll
       for (int kw = 0; kw < kNP / 8; ++kw) {
@@ -407,9 +428,11 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const uint16_t* __re
       const __half2 bias = __floats2half2_rn(1152.0f, 1152.0f);
 #pragma unroll
       for (int kw = 0; kw < kNP / 4; ++kw) {
-        const uint2 da = seg[kw / 2], db = seg[(kw + kNP / 4) / 2];
-        const uint32_t wa = ((kw & 1) ? da.y : da.x) ^ 0x80808080u;
-        const uint32_t wb = ((kw & 1) ? db.y : db.x) ^ 0x80808080u;
+        const uint4 ca = code_chunk<F::CB>(st, lane, kw >> 2);
+        const uint4 cb = code_chunk<F::CB>(st, lane, (kw + kNP / 4) >> 2);
+        const uint32_t ra[4] = {ca.x, ca.y, ca.z, ca.w}, rb[4] = {cb.x, cb.y, cb.z, cb.w};
+        const uint32_t wa = ra[kw & 3] ^ 0x80808080u;
+        const uint32_t wb = rb[kw & 3] ^ 0x80808080u;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const uint32_t sel = 0x0400u | (t << 8) | t;
@@ -731,7 +754,8 @@ kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
 
 template <int G, int BITS, bool AFTER>
 __global__ void __launch_bounds__(kXW * 32, 2)
-kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
+kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const __grid_constant__ CUtensorMap cmap,
+                           const uint16_t* __restrict__ scales,
                            const ExArgs a, const __grid_constant__ SrftTw tw, float c0, float c1,
                            const __grid_constant__ ExMaps omaps, int scale_copy) {
   using F = Fmt<BITS>;
@@ -742,7 +766,7 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* stage_out = smem + warp * L::WARP;              // swizzled fp16 staging tile
-  uint8_t* wsm = stage_out + kXStage;                      // two stages of codes and scales
+  uint8_t* wsm = stage_out + kXStage;                      // two code tiles, then two scale blocks
   uint8_t* hdr = smem + kXW * L::WARP;
   float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
   float4* stab = reinterpret_cast<float4*>(hdr + kXW * 512);
@@ -773,11 +797,16 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
     if (lane == 0) tq[stage] = t;
     if (t < 0 || lane != 0) return;
     const int64_t row0 = static_cast<int64_t>(t) * kWR;
-    const int valid = static_cast<int>(a.n - row0 < kWR ? a.n - row0 : kWR);
     const uint32_t sb = scale_bytes(t);
-    mbar_expect_tx(&bar[stage], static_cast<uint32_t>(valid) * F::CB + sb);
-    bulk_g2s(wsm + stage * L::STAGE, codes + row0 * F::CB, static_cast<uint32_t>(valid) * F::CB, &bar[stage]);
-    if (sb) bulk_g2s(wsm + stage * L::STAGE + L::WC, reinterpret_cast<const uint8_t*>(scales) + row0 * L::SPR, sb, &bar[stage]);
+    if constexpr (BITS == 8) {         // swizzled tensor copy: the copy engine fills the whole box
+      mbar_expect_tx(&bar[stage], static_cast<uint32_t>(L::WC) + sb);
+      tensor_g2s(wsm + stage * L::WC, &cmap, 0, static_cast<int>(row0), &bar[stage]);
+    } else {                           // plain bulk copy of the valid rows
+      const uint32_t cbytes = static_cast<uint32_t>(a.n - row0 < kWR ? a.n - row0 : kWR) * F::CB;
+      mbar_expect_tx(&bar[stage], cbytes + sb);
+      bulk_g2s(wsm + stage * L::WC, codes + row0 * F::CB, cbytes, &bar[stage]);
+    }
+    if (sb) bulk_g2s(wsm + L::SC + stage * L::WS, reinterpret_cast<const uint8_t*>(scales) + row0 * L::SPR, sb, &bar[stage]);
   };
   refill(0);
   refill(1);
@@ -803,19 +832,18 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
       cached = id;
       __syncwarp();
     }
-    const uint8_t* st = wsm + stage * L::STAGE;
-    const uint16_t* srow = sc_smem ? reinterpret_cast<const uint16_t*>(st + L::WC + lane * L::SPR)
+    const uint8_t* st = wsm + stage * L::WC;
+    const uint16_t* srow = sc_smem ? reinterpret_cast<const uint16_t*>(wsm + L::SC + stage * L::WS + lane * L::SPR)
                                    : scales + rrow * NG;
     uint16_t sv[NG];
 #pragma unroll
     for (int j = 0; j < NG; ++j) sv[j] = srow[j];
-    const uint32_t* seg = reinterpret_cast<const uint32_t*>(st + lane * F::CB);
     float2 z[kFN];
     if constexpr (BITS == 4) {
       const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
 #pragma unroll
       for (int j = 0; j < kD / 8; ++j) {               // word j: channels 8j .. 8j+7
-        const uint32_t w = seg[j] ^ 0x88888888u, w4 = w >> 4;
+        const uint32_t w = reinterpret_cast<const uint32_t*>(st + lane * F::CB)[j] ^ 0x88888888u, w4 = w >> 4;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const uint32_t sel = 0x0400u | (t << 8) | t;
@@ -829,7 +857,9 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
       const __half2 bias = __floats2half2_rn(1152.0f, 1152.0f);
 #pragma unroll
       for (int j = 0; j < kD / 4; ++j) {               // word j: channels 4j .. 4j+3
-        const uint32_t w = seg[j] ^ 0x80808080u;
+        const uint4 ch = code_chunk<F::CB>(st, lane, j >> 2);
+        const uint32_t cw[4] = {ch.x, ch.y, ch.z, ch.w};
+        const uint32_t w = cw[j & 3] ^ 0x80808080u;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           const uint32_t sel = static_cast<uint32_t>(2 * t) | ((2u * t + 1) << 8);   // bytes 2t, 2t+1
@@ -933,6 +963,7 @@ int check_ex(int D, int G, int bits, int64_t n, int64_t lambda_rows, int n_lambd
 }
 
 int encode_x_maps(ExMaps& maps, const uint16_t* x, int64_t n);
+int encode_code_map(CUtensorMap& map, const uint8_t* codes, int64_t n, int cb);
 
 template <int G, int BITS, bool AFTER>
 int launch_qex(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* scales, cudaStream_t st) {
@@ -959,8 +990,14 @@ int launch_dex(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, ui
   constexpr int smem = 1024 + kXW * L::WARP + kHdrBytes;
   static std::atomic<int> ready[64];
   const int grid = ex_grid(k, a.n, smem, ready);
+  CUtensorMap cmap;
+  memset(&cmap, 0, sizeof(cmap));
+  if (BITS == 8) {
+    const int rc2 = encode_code_map(cmap, codes, a.n, Fmt<BITS>::CB);
+    if (rc2 != KVQ_OK) return rc2;
+  }
   (void)cudaGetLastError();
-  k<<<grid, kXW * 32, smem, st>>>(codes, scales, a, omaps,
+  k<<<grid, kXW * 32, smem, st>>>(codes, cmap, scales, a, omaps,
                                   (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
   return finish_ex();
 }
@@ -1003,6 +1040,29 @@ int encode_x_maps(ExMaps& maps, const uint16_t* x, int64_t n) {
   return KVQ_OK;
 }
 
+// The codes [n][cb] (cb = 64 or 128 bytes) as one 2-D map with a box of one
+// warp tile, swizzled over the row's cb bytes (the layout code_chunk reads).
+// The int8 dequantisers read their codes through it; the int4 ones, whose
+// arithmetic leaves shared memory idle, measured faster with plain bulk
+// copies of the linear rows.
+int encode_code_map(CUtensorMap& map, const uint8_t* codes, int64_t n, int cb) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return KVQ_ERR_LAUNCH;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cb), static_cast<cuuint64_t>(n)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cb)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(cb), kWR};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         cb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_ex_cuda_error = static_cast<int>(r);
+    return KVQ_ERR_LAUNCH;
+  }
+  return KVQ_OK;
+}
+
 template <int G, int BITS, bool AFTER>
 int launch_qsrft(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* scales, cudaStream_t st) {
   ExMaps maps;
@@ -1028,8 +1088,14 @@ int launch_dsrft(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, 
   constexpr int smem = 1024 + kXW * L::WARP + kHdrBytes;
   static std::atomic<int> ready[64];
   const int grid = ex_grid(k, a.n, smem, ready);
+  CUtensorMap cmap;
+  memset(&cmap, 0, sizeof(cmap));
+  if (BITS == 8) {
+    const int rc2 = encode_code_map(cmap, codes, a.n, Fmt<BITS>::CB);
+    if (rc2 != KVQ_OK) return rc2;
+  }
   (void)cudaGetLastError();
-  k<<<grid, kXW * 32, smem, st>>>(codes, scales, a, srft_twiddles(), kSrftC0, kSrftC1, omaps,
+  k<<<grid, kXW * 32, smem, st>>>(codes, cmap, scales, a, srft_twiddles(), kSrftC0, kSrftC1, omaps,
                                   (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
   return finish_ex();
 }
