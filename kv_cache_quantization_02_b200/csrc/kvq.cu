@@ -68,7 +68,6 @@ int kvq_ex_last_cuda_error();
 
 namespace {
 
-constexpr int kThreads = 128;              // lanes per block (4 warps)
 constexpr int kWarps = 12;                 // warps of a streaming block (one block per SM)
 constexpr unsigned kFullMask = 0xffffffffu;
 constexpr uint32_t kSpinLimit = 1u << 22;  // bounded mbarrier waits
@@ -81,8 +80,8 @@ thread_local int g_last_cuda_error = 0;
 __device__ unsigned int g_kvq_fault = 0;
 
 // ---------------------------------------------------------------------------
-// Tile geometry: ROWS vectors per tile, the fp16 rows split into Q quarters
-// of 64 channels (128 bytes), each quarter a [ROWS][128 B] swizzled block.
+// Lane geometry of a vector: a lane holds EPT channels as NP fp32 pairs, the
+// fp16 rows split into Q quarters of 64 channels (128 bytes).
 // ---------------------------------------------------------------------------
 template <int D>
 struct Tile {
@@ -90,22 +89,9 @@ struct Tile {
   static constexpr int LANES = D / EPT;             // lanes per vector
   static constexpr int NP = EPT / 2;                // fp32 pairs per lane
   static constexpr int HALF = EPT / 2;              // pair (m, m + HALF)
-  static constexpr int ROWS = kThreads / LANES;     // vectors per tile
   static constexpr int Q = D / 64;                  // 64-channel quarters of a row
-  static constexpr int QB = ROWS * 128;             // bytes of one quarter of a tile
-  static constexpr int STAGE = Q * QB;              // bytes of one fp16 tile (= ROWS * 2D)
   static constexpr int TAB = LANES * NP * 8;        // per-channel pair table
 };
-
-// Byte offset, inside one fp16 tile, of 16-byte chunk c (channels 8c..8c+7) of
-// quarter q of tile row t.  Each quarter is a [ROWS][128 B] block written by a
-// 128-byte-swizzled tensor copy: chunk c of row t sits at chunk c ^ (t mod 8),
-// so the 8 lanes of a quarter-warp phase, which read 8 consecutive rows,
-// touch 8 distinct bank groups.
-template <int D>
-__device__ __forceinline__ int tile_off(int q, int t, int c) {
-  return q * Tile<D>::QB + t * 128 + ((c ^ (t & 7)) << 4);
-}
 
 // The kernel arguments that describe a tensor copy of the fp16 rows: one 2-D
 // map (64 channels x n rows, row stride 2D bytes) per quarter.
@@ -147,8 +133,25 @@ struct Stream {
       (WTile<D>::WSTAGE + 2 * WTile<D>::WPIN + 2 * kScaleBlock + 1023) / 1024 * 1024;
   static constexpr int smem(int per_warp, int warps) { return 1024 + warps * per_warp + HDR; }
 };
+// Shared memory of a round-trip block: per warp two fp16 stages (a tile's
+// input, then its output: the output is written over the input it was
+// computed from) and the code block of one warp tile; then a header with the
+// quantize and dequantize tables, two mbarriers and two stage tile ids per
+// warp and the tile-claim counter.  One block of kRtWarps warps per SM, as
+// for the streaming kernels.
+constexpr int kRtWarps = kWarps;
 template <int D>
-constexpr int roundtrip_smem_bytes() { return 1024 + 3 * Tile<D>::STAGE + 2 * Tile<D>::TAB + 16; }
+struct RStream {
+  static constexpr int TABQ = 0;
+  static constexpr int TABD = Tile<D>::TAB;
+  static constexpr int BARS = 2 * Tile<D>::TAB;
+  static constexpr int TQ = BARS + 16 * kRtWarps;
+  static constexpr int NEXT = TQ + 8 * kRtWarps;
+  static constexpr int HDR = NEXT + 16;
+  static constexpr int CST = (WTile<D>::WROWS * (D / 2) + 1023) / 1024 * 1024;
+  static constexpr int WARP = 2 * WTile<D>::WSTAGE + CST;
+  static constexpr int SMEM = 1024 + kRtWarps * WARP + HDR;
+};
 
 // ---------------------------------------------------------------------------
 // Asynchronous copies and barriers.
@@ -180,6 +183,225 @@ __device__ __forceinline__ void fill_tab(float4* tab, const float* __restrict__ 
   }
 }
 
+
+// Group geometry of a lane's pairs: GX pairs per group (G <= EPT/2), NGH
+// groups per half-lane, HG = the butterfly half-widths that stay in a group.
+template <int D, int G>
+struct Grp {
+  static constexpr int GX = (G < Tile<D>::HALF) ? G : Tile<D>::HALF;
+  static constexpr int NGH = Tile<D>::HALF / GX;
+  static constexpr int HG = (G < Tile<D>::NP) ? G : Tile<D>::NP;
+};
+
+// a2-a7 on one lane's part of a vector, p = x * lambda * s as pairs
+// (v[m], v[m + EPT/2]): butterfly, x c, group abs-max, scales, codes.  out:
+// the lane's packed codes in row order (word k: channels 8k .. 8k+7 of the
+// lane's EPT, two's-complement nibbles); bx / by: the scales (fp16 bits) of
+// the groups in pair halves .x / .y.  XS: lane stride between the parts of a
+// vector.
+template <int D, int G, int XS>
+__device__ __forceinline__ void quantize_regs(float2 (&p)[Tile<D>::NP], int sub, float2 c2,
+                                              uint32_t (&out)[Tile<D>::EPT / 8],
+                                              uint16_t (&bx)[Grp<D, G>::NGH],
+                                              uint16_t (&by)[Grp<D, G>::NGH]) {
+  constexpr int EPT = Tile<D>::EPT, LANES = Tile<D>::LANES, NP = Tile<D>::NP, HALF = Tile<D>::HALF;
+  constexpr int GX = Grp<D, G>::GX, NGH = Grp<D, G>::NGH;
+  // a2, a3: transform, normalise.
+  fwht_pairs<EPT, LANES, 1, XS>(p, sub);
+#pragma unroll
+  for (int m = 0; m < NP; ++m) p[m] = __fmul2_rn(p[m], c2);
+
+  // a4, a5: group abs-max and scales.  Pair .x holds channels [0, HALF) of
+  // the lane, .y holds [HALF, EPT).
+  float rx[NGH], ry[NGH];
+  if constexpr (G <= HALF) {
+#pragma unroll
+    for (int j = 0; j < NGH; ++j) {
+      float ax = 0.f, ay = 0.f;
+#pragma unroll
+      for (int m = 0; m < GX; m += 2) {
+        ax = amax3(ax, p[j * GX + m].x, p[j * GX + m + 1].x);
+        ay = amax3(ay, p[j * GX + m].y, p[j * GX + m + 1].y);
+      }
+      bx[j] = group_scale(ax, rx[j]);
+      by[j] = group_scale(ay, ry[j]);
+    }
+  } else {
+    float a = 0.f;
+#pragma unroll
+    for (int m = 0; m < NP; ++m) a = amax3(a, p[m].x, p[m].y);
+#pragma unroll
+    for (int bit = 1; bit < G / EPT; bit <<= 1) a = fmaxf(a, __shfl_xor_sync(kFullMask, a, bit * XS));
+    bx[0] = group_scale(a, rx[0]);
+    ry[0] = rx[0];
+    by[0] = bx[0];
+  }
+
+  // a6, a7: codes = rint(y * r) (half to even), saturated and packed.
+#pragma unroll
+  for (int k8 = 0; k8 < NP / 8; ++k8) {
+    int qa[8], qb[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int m = 8 * k8 + t;
+      const float2 v = __fmul2_rn(p[m], make_float2(rx[m / GX], ry[m / GX]));
+      qa[t] = __float2int_rn(v.x);
+      qb[t] = __float2int_rn(v.y);
+    }
+    out[k8] = pack8(qa);
+    out[k8 + NP / 8] = pack8(qb);
+  }
+}
+
+// The lane's codes into a warp tile's code staging block, laid out as the
+// swizzled tensor store reads it: 16-byte chunk c of row t at chunk
+// c ^ ((t * D/2 / 128) mod D/32), so a quarter-warp's chunks fall in distinct
+// banks.
+template <int D>
+__device__ __forceinline__ void stage_codes(uint8_t* cst, const uint32_t (&out)[Tile<D>::EPT / 8],
+                                            int sub, int rin) {
+  constexpr int EPT = Tile<D>::EPT, RB = D / 2;   // code bytes per row
+  const int swz = ((rin * RB) >> 7) & (D / 32 - 1);
+#pragma unroll
+  for (int k4 = 0; k4 < EPT / 32; ++k4) {
+    const int cidx = sub * (EPT / 32) + k4;
+    *reinterpret_cast<uint4*>(cst + rin * RB + ((cidx ^ swz) << 4)) =
+        make_uint4(out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]);
+  }
+}
+
+// The lane's scales into row `orow` of the scale array: the row's D/G scales
+// in one store when the pointer is aligned for it (vec), else one by one.
+template <int D, int G>
+__device__ __forceinline__ void store_scales(uint16_t* __restrict__ scales, int64_t orow, int sub,
+                                             const uint16_t (&bx)[Grp<D, G>::NGH],
+                                             const uint16_t (&by)[Grp<D, G>::NGH], bool vec) {
+  constexpr int EPT = Tile<D>::EPT, LANES = Tile<D>::LANES, HALF = Tile<D>::HALF;
+  constexpr int NGH = Grp<D, G>::NGH;
+  uint16_t* srow = scales + orow * (D / G);
+  if constexpr (G <= HALF && LANES == 1) {
+    uint16_t sa[D / G];
+#pragma unroll
+    for (int j = 0; j < NGH; ++j) { sa[j] = bx[j]; sa[NGH + j] = by[j]; }
+    uint32_t sw[D / G / 2];
+#pragma unroll
+    for (int i = 0; i < D / G / 2; ++i) sw[i] = uint32_t(sa[2 * i]) | (uint32_t(sa[2 * i + 1]) << 16);
+    if (vec) {
+      if constexpr (D / G == 2) *reinterpret_cast<uint32_t*>(srow) = sw[0];
+      else if constexpr (D / G == 4) *reinterpret_cast<uint2*>(srow) = make_uint2(sw[0], sw[1]);
+      else *reinterpret_cast<uint4*>(srow) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < NGH; ++j) {
+        srow[j] = bx[j];
+        srow[NGH + j] = by[j];
+      }
+    }
+  } else if constexpr (G <= HALF) {
+#pragma unroll
+    for (int j = 0; j < NGH; ++j) {
+      srow[sub * (EPT / G) + j] = bx[j];
+      srow[sub * (EPT / G) + NGH + j] = by[j];
+    }
+  } else {
+    if (sub % (G / EPT) == 0) srow[sub / (G / EPT)] = bx[0];
+  }
+}
+
+// a8 and the butterfly stages inside a group: the lane's code words w (row
+// order, nibbles biased to n = q + 8) and scales -> p = u after the stages
+// h < HG, as fp32 pairs (m, m + EPT/2).  u = q S is exact, and so is every
+// stage inside a group.
+//  * One prmt + lop3 puts the codes of a pair (m, m + EPT/2) into two 16-bit
+//    lanes holding W + 0x6608, the fp16 encoding of the exact integer
+//    W + 1544 (W = n, or its partial butterfly sums).
+//  * The first four stages run on those integer lanes: one 32-bit add does
+//    a + b - bias (or a - b + bias) for both; every lane stays in [0, 65535].
+//  * The remaining in-group stages run in fp16x2 after one hsub2 removes the
+//    bias (integers of magnitude <= 8 * 2^stage <= 512: exact).
+//  * u = W * S by one mixed-precision fma.rn.f32.f16 (a product of two fp16
+//    values is exact in fp32).
+template <int D, int G>
+__device__ __forceinline__ void dequant_front(const uint32_t (&w)[Tile<D>::EPT / 8],
+                                              const uint16_t (&sx)[Grp<D, G>::NGH],
+                                              const uint16_t (&sy)[Grp<D, G>::NGH],
+                                              float2 (&p)[Tile<D>::NP]) {
+  constexpr int NP = Tile<D>::NP, HALF = Tile<D>::HALF;
+  constexpr int GX = Grp<D, G>::GX, HG = Grp<D, G>::HG;
+  uint32_t iq[NP];
+#pragma unroll
+  for (int kw = 0; kw < NP / 8; ++kw) {
+    const uint32_t wa = w[kw], wb = w[kw + HALF / 8];
+    const uint32_t wa4 = wa >> 4, wb4 = wb >> 4;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t sel = 0x0400u | (t << 8) | t;   // byte t of a -> byte 0, of b -> byte 2
+      iq[8 * kw + 2 * t] = (__byte_perm(wa, wb, sel) & 0x000F000Fu) | 0x66006600u;
+      iq[8 * kw + 2 * t + 1] = (__byte_perm(wa4, wb4, sel) & 0x000F000Fu) | 0x66006600u;
+    }
+  }
+  constexpr int kIntStages = 4;
+  constexpr uint32_t kBias2 = 0x66086608u;
+  constexpr int HI = (1 << kIntStages) < HG ? (1 << kIntStages) : HG;
+#pragma unroll
+  for (int h = 1; h < HI; h <<= 1) {
+#pragma unroll
+    for (int m = 0; m < NP; ++m) {
+      if ((m & h) == 0) {
+        const uint32_t a = iq[m], b = iq[m + h];
+        iq[m] = a + b - kBias2;
+        iq[m + h] = a - b + kBias2;
+      }
+    }
+  }
+  const __half2 k1544 = __floats2half2_rn(1544.0f, 1544.0f);
+  __half2 hq[NP];
+#pragma unroll
+  for (int m = 0; m < NP; ++m) hq[m] = __hsub2(*reinterpret_cast<const __half2*>(&iq[m]), k1544);
+#pragma unroll
+  for (int h = HI; h < HG; h <<= 1) {
+#pragma unroll
+    for (int m = 0; m < NP; ++m) {
+      if ((m & h) == 0) {
+        const __half2 a = hq[m], b = hq[m + h];
+        hq[m] = __hadd2(a, b);
+        hq[m + h] = __hsub2(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < NP; ++m)
+    p[m] = make_float2(mul_f16_f32(__low2half(hq[m]), sx[m / GX]),
+                       mul_f16_f32(__high2half(hq[m]), sy[m / GX]));
+}
+
+// a9's normalisation and a10: x c, x s/lambda (per-channel table), fp16,
+// written into the warp's swizzled fp16 staging tile (the input's quarter
+// layout), which Q tensor stores then write out.
+template <int D>
+__device__ __forceinline__ void stage_rows(const float2 (&p)[Tile<D>::NP], float2 c2,
+                                           const float4* mytab, uint8_t* stage_out, int sub, int rin) {
+  constexpr int EPT = Tile<D>::EPT, NP = Tile<D>::NP, HALF = Tile<D>::HALF;
+  constexpr int QL = EPT / 64;                   // quarters per lane
+#pragma unroll
+  for (int j = 0; j < NP / 8; ++j) {
+    uint32_t lo[4], hi[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float4 l = mytab[4 * j + t];
+      const float2 a = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t], c2), make_float2(l.x, l.y));
+      const float2 b = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t + 1], c2), make_float2(l.z, l.w));
+      lo[t] = float2_to_half2_bits(a.x, b.x);
+      hi[t] = float2_to_half2_bits(a.y, b.y);
+    }
+    const int ea = 8 * j, eb = HALF + 8 * j;
+    *reinterpret_cast<uint4*>(stage_out + wtile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8)) =
+        make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    *reinterpret_cast<uint4*>(stage_out + wtile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8)) =
+        make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Quantize: fp16 [n][D] -> packed u8 [n][D/2] + fp16 scales [n][D/G].
 // ---------------------------------------------------------------------------
@@ -192,11 +414,9 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
                     const __grid_constant__ CUtensorMap cmap) {
   using T = Tile<D>;
   using W = WTile<D>;
-  constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF;
+  constexpr int EPT = T::EPT, NP = T::NP, HALF = T::HALF;
   constexpr bool STG = !INDEXED;                // codes leave through a staged tensor store
   constexpr int QW = STG ? Stream<D>::QWARP_S : Stream<D>::QWARP;
-  constexpr int GX = (G < HALF) ? G : HALF;      // pairs spanned by one group (G <= HALF)
-  constexpr int NGH = HALF / GX;                 // groups per half-lane
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
@@ -288,70 +508,17 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
     __syncwarp();             // the warp has its inputs: the stage can be refilled
     refill(stage);
 
-    // a2, a3: transform, normalise.
-    fwht_pairs<EPT, LANES, 1, W::WROWS>(p, sub);
-#pragma unroll
-    for (int m = 0; m < NP; ++m) p[m] = __fmul2_rn(p[m], c2);
-
-    // a4, a5: group abs-max and scales.  Pair .x holds channels [0, HALF) of
-    // the lane, .y holds [HALF, EPT).
-    float rx[NGH], ry[NGH];
-    uint16_t bx[NGH], by[NGH];
-    if constexpr (G <= HALF) {
-#pragma unroll
-      for (int j = 0; j < NGH; ++j) {
-        float ax = 0.f, ay = 0.f;
-#pragma unroll
-        for (int m = 0; m < GX; m += 2) {
-          ax = amax3(ax, p[j * GX + m].x, p[j * GX + m + 1].x);
-          ay = amax3(ay, p[j * GX + m].y, p[j * GX + m + 1].y);
-        }
-        bx[j] = group_scale(ax, rx[j]);
-        by[j] = group_scale(ay, ry[j]);
-      }
-    } else {
-      float a = 0.f;
-#pragma unroll
-      for (int m = 0; m < NP; ++m) a = amax3(a, p[m].x, p[m].y);
-#pragma unroll
-      for (int bit = 1; bit < G / EPT; bit <<= 1) a = fmaxf(a, __shfl_xor_sync(kFullMask, a, bit * W::WROWS));
-      bx[0] = group_scale(a, rx[0]);
-      ry[0] = rx[0];
-      by[0] = bx[0];
-    }
-
-    // a6, a7: codes = rint(y * r) (half to even), saturated and packed.
     uint32_t out[EPT / 8];
-#pragma unroll
-    for (int k8 = 0; k8 < NP / 8; ++k8) {
-      int qa[8], qb[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const int m = 8 * k8 + t;
-        const float2 v = __fmul2_rn(p[m], make_float2(rx[m / GX], ry[m / GX]));
-        qa[t] = __float2int_rn(v.x);
-        qb[t] = __float2int_rn(v.y);
-      }
-      out[k8] = pack8(qa);
-      out[k8 + NP / 8] = pack8(qb);
-    }
-    // The codes of a warp tile are one contiguous block: each lane writes its
-    // row into the staging tile, laid out as the swizzled tensor store reads
-    // it (16-byte chunk c of row t at chunk c ^ ((t * D/2 / 128) mod D/32),
-    // so a quarter-warp's chunks fall in distinct banks), and lane 0 stores
-    // the tile with one tensor copy that skips rows past n.  Rows scattered
-    // by an index are stored by each lane.
+    uint16_t bx[Grp<D, G>::NGH], by[Grp<D, G>::NGH];
+    quantize_regs<D, G, W::WROWS>(p, sub, c2, out, bx, by);
+
+    // The codes of a warp tile are one contiguous block: lane 0 stores the
+    // staged tile with one tensor copy that skips rows past n.  Rows
+    // scattered by an index are stored by each lane.
     if constexpr (STG) {
       if (lane == 0) bulk_wait_read0();
       __syncwarp();                              // the staging tile is free
-      constexpr int RB = D / 2;                  // code bytes per row
-      const int swz = ((rin * RB) >> 7) & (D / 32 - 1);
-#pragma unroll
-      for (int k4 = 0; k4 < EPT / 32; ++k4) {
-        const int cidx = sub * (EPT / 32) + k4;
-        *reinterpret_cast<uint4*>(cst + rin * RB + ((cidx ^ swz) << 4)) =
-            make_uint4(out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]);
-      }
+      stage_codes<D>(cst, out, sub, rin);
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) {
@@ -368,34 +535,7 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
           st_v4(dst + 16 * k4, t4);
         }
       }
-      uint16_t* srow = scales + orow * (D / G);
-      if constexpr (G <= HALF && LANES == 1) {     // the row's D/G scales: one store when aligned
-        uint16_t sa[D / G];
-#pragma unroll
-        for (int j = 0; j < NGH; ++j) { sa[j] = bx[j]; sa[NGH + j] = by[j]; }
-        uint32_t sw[D / G / 2];
-#pragma unroll
-        for (int i = 0; i < D / G / 2; ++i) sw[i] = uint32_t(sa[2 * i]) | (uint32_t(sa[2 * i + 1]) << 16);
-        if (scale_vec) {
-          if constexpr (D / G == 2) *reinterpret_cast<uint32_t*>(srow) = sw[0];
-          else if constexpr (D / G == 4) *reinterpret_cast<uint2*>(srow) = make_uint2(sw[0], sw[1]);
-          else *reinterpret_cast<uint4*>(srow) = make_uint4(sw[0], sw[1], sw[2], sw[3]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < NGH; ++j) {
-            srow[j] = bx[j];
-            srow[NGH + j] = by[j];
-          }
-        }
-      } else if constexpr (G <= HALF) {
-#pragma unroll
-        for (int j = 0; j < NGH; ++j) {
-          srow[sub * (EPT / G) + j] = bx[j];
-          srow[sub * (EPT / G) + NGH + j] = by[j];
-        }
-      } else {
-        if (sub % (G / EPT) == 0) srow[sub / (G / EPT)] = bx[0];
-      }
+      store_scales<D, G>(scales, orow, sub, bx, by, scale_vec != 0);
     }
   }
   if (STG && lane == 0) bulk_wait0();
@@ -417,10 +557,8 @@ kvq_dequantize_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* 
   constexpr int SPR = (D / G) * 2;               // scale bytes per row
   constexpr int WSC = kScaleBlock;
   static_assert(WROWS * SPR <= WSC, "scale block");
-  constexpr int GX = (G < HALF) ? G : HALF;
-  constexpr int NGH = HALF / GX;
-  constexpr int HG = (G < NP) ? G : NP;          // butterfly stages h < HG stay inside a group
-  constexpr int QL = EPT / 64;                   // quarters per lane
+  constexpr int NGH = Grp<D, G>::NGH;
+  constexpr int HG = Grp<D, G>::HG;               // butterfly stages h < HG stay inside a group
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
@@ -474,7 +612,6 @@ kvq_dequantize_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* 
   refill(1);
   const float2 c2 = make_float2(c, c);
   const float4* mytab = tabw + sub * (NP / 2);
-  const __half2 k1544 = __floats2half2_rn(1544.0f, 1544.0f);
   for (uint32_t k = 0;; ++k) {
     const int stage = k & 1;
     __syncwarp();
@@ -515,74 +652,15 @@ kvq_dequantize_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* 
       w[4 * j + 2] = a.z ^ 0x88888888u;
       w[4 * j + 3] = a.w ^ 0x88888888u;
     }
-    uint32_t iq[NP];
-#pragma unroll
-    for (int kw = 0; kw < NP / 8; ++kw) {
-      const uint32_t wa = w[kw], wb = w[kw + HALF / 8];
-      const uint32_t wa4 = wa >> 4, wb4 = wb >> 4;
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const uint32_t sel = 0x0400u | (t << 8) | t;   // byte t of a -> byte 0, of b -> byte 2
-        iq[8 * kw + 2 * t] = (__byte_perm(wa, wb, sel) & 0x000F000Fu) | 0x66006600u;
-        iq[8 * kw + 2 * t + 1] = (__byte_perm(wa4, wb4, sel) & 0x000F000Fu) | 0x66006600u;
-      }
-    }
-    constexpr int kIntStages = 4;
-    constexpr uint32_t kBias2 = 0x66086608u;
-    constexpr int HI = (1 << kIntStages) < HG ? (1 << kIntStages) : HG;
-#pragma unroll
-    for (int h = 1; h < HI; h <<= 1) {
-#pragma unroll
-      for (int m = 0; m < NP; ++m) {
-        if ((m & h) == 0) {
-          const uint32_t a = iq[m], b = iq[m + h];
-          iq[m] = a + b - kBias2;
-          iq[m + h] = a - b + kBias2;
-        }
-      }
-    }
-    __half2 hq[NP];
-#pragma unroll
-    for (int m = 0; m < NP; ++m) hq[m] = __hsub2(*reinterpret_cast<const __half2*>(&iq[m]), k1544);
-#pragma unroll
-    for (int h = HI; h < HG; h <<= 1) {
-#pragma unroll
-      for (int m = 0; m < NP; ++m) {
-        if ((m & h) == 0) {
-          const __half2 a = hq[m], b = hq[m + h];
-          hq[m] = __hadd2(a, b);
-          hq[m + h] = __hsub2(a, b);
-        }
-      }
-    }
     float2 p[NP];
-#pragma unroll
-    for (int m = 0; m < NP; ++m)
-      p[m] = make_float2(mul_f16_f32(__low2half(hq[m]), sx[m / GX]),
-                         mul_f16_f32(__high2half(hq[m]), sy[m / GX]));
+    dequant_front<D, G>(w, sx, sy, p);
     __syncwarp();             // codes and scales consumed: the input stage can be refilled
     refill(stage);
     fwht_pairs<EPT, LANES, HG, WROWS>(p, sub);
 
     if (lane == 0) bulk_wait_read0();
     __syncwarp();             // the warp's staging tile is free
-#pragma unroll
-    for (int j = 0; j < NP / 8; ++j) {
-      uint32_t lo[4], hi[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float4 l = mytab[4 * j + t];
-        const float2 a = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t], c2), make_float2(l.x, l.y));
-        const float2 b = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t + 1], c2), make_float2(l.z, l.w));
-        lo[t] = float2_to_half2_bits(a.x, b.x);
-        hi[t] = float2_to_half2_bits(a.y, b.y);
-      }
-      const int ea = 8 * j, eb = HALF + 8 * j;
-      *reinterpret_cast<uint4*>(stage_out + wtile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8)) =
-          make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      *reinterpret_cast<uint4*>(stage_out + wtile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8)) =
-          make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    }
+    stage_rows<D>(p, c2, mytab, stage_out, sub, rin);
     fence_proxy_async();
     __syncwarp();
     if (lane == 0) {
@@ -599,171 +677,132 @@ kvq_dequantize_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* 
 // ---------------------------------------------------------------------------
 // Round trip: fp16 [n][D] -> x_hat = dequantize(quantize(x)) fp16 [n][D], and
 // optionally the codes and scales, in one pass (the quantise-then-dequantise
-// shape used to simulate the cache's error).  Same arithmetic as the two
-// kernels back to back: u = q * S is exact, then the same butterfly order.
+// shape used to simulate the cache's error).  Each warp streams its tiles as
+// the quantize kernel does, runs the quantize arithmetic, then the
+// dequantize arithmetic straight from the packed code words still in its
+// registers (the same words the dequantize kernel would load), so x_hat is
+// bit-identical to the two kernels back to back.
 // ---------------------------------------------------------------------------
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kRtWarps * 32, 1)
 kvq_roundtrip_kernel(const __grid_constant__ RowMaps in_maps, const __grid_constant__ RowMaps out_maps,
-                     const float* __restrict__ lam, const int8_t* __restrict__ sgn, int64_t n,
-                     float c, uint8_t* __restrict__ packed, uint16_t* __restrict__ scales) {
+                     const __grid_constant__ CUtensorMap cmap, const float* __restrict__ lam,
+                     const int8_t* __restrict__ sgn, int64_t n, float c,
+                     uint16_t* __restrict__ scales, int with_codes, int scale_vec) {
   using T = Tile<D>;
-  constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF, ROWS = T::ROWS;
-  constexpr int GX = (G < HALF) ? G : HALF;
-  constexpr int NGH = HALF / GX;
-  constexpr int QL = EPT / 64;
+  using W = WTile<D>;
+  using L = RStream<D>;
+  constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF;
+  constexpr int NGH = Grp<D, G>::NGH, HG = Grp<D, G>::HG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* stage_out = smem + 2 * T::STAGE;
-  float4* tab_q = reinterpret_cast<float4*>(smem + 3 * T::STAGE);
-  float4* tab_d = reinterpret_cast<float4*>(smem + 3 * T::STAGE + T::TAB);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + 3 * T::STAGE + 2 * T::TAB);
   const int tid = threadIdx.x;
-  const int sub = tid % LANES;
-  const int rin = tid / LANES;
+  const int warp = tid >> 5, lane = tid & 31;
+  uint8_t* hdr = smem + kRtWarps * L::WARP;
+  float4* tab_q = reinterpret_cast<float4*>(hdr + L::TABQ);
+  float4* tab_d = reinterpret_cast<float4*>(hdr + L::TABD);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + L::BARS) + 2 * warp;
+  int* tq = reinterpret_cast<int*>(hdr + L::TQ) + 2 * warp;
+  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + L::NEXT);
+  uint8_t* wsm = smem + warp * L::WARP;          // two fp16 stages
+  uint8_t* cst = wsm + 2 * W::WSTAGE;            // the codes
+  const int sub = lane / W::WROWS;
+  const int rin = lane % W::WROWS;
   fill_tab<D>(tab_q, lam, sgn, false);
   fill_tab<D>(tab_d, lam, sgn, true);
-  if (tid == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
+  if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
+  if (tid == 0) *next = 0;
   __syncthreads();
 
-  const int64_t ntiles = (n + ROWS - 1) / ROWS;
-  const int tstride = gridDim.x;
-  auto issue = [&](int64_t tile, int stage) {
-    if (tile >= ntiles || tid != 0) return;
-    mbar_expect_tx(&bar[stage], T::STAGE);
+  const int64_t ntiles = (n + W::WROWS - 1) / W::WROWS;
+  const unsigned int mine = static_cast<unsigned int>((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  auto claim = [&]() -> int {
+    unsigned int i = 0;
+    if (lane == 0) i = atomicAdd(next, 1u);
+    i = __shfl_sync(kFullMask, i, 0);
+    return i < mine ? static_cast<int>(blockIdx.x + i * gridDim.x) : -1;
+  };
+  auto refill = [&](int stage) {
+    const int t = claim();
+    if (lane == 0) tq[stage] = t;
+    if (t < 0 || lane != 0) return;
+    mbar_expect_tx(&bar[stage], W::WSTAGE);
 #pragma unroll
     for (int q = 0; q < T::Q; ++q)
-      tensor_g2s(smem + stage * T::STAGE + q * T::QB, &in_maps.q[q], 0, static_cast<int>(tile * ROWS), &bar[stage]);
+      tensor_g2s(wsm + stage * W::WSTAGE + q * W::WQB, &in_maps.q[q], 0, t * W::WROWS, &bar[stage]);
   };
-  issue(blockIdx.x, 0);
-  issue(static_cast<int64_t>(blockIdx.x) + tstride, 1);
+  refill(0);
+  refill(1);
   const float2 c2 = make_float2(c, c);
-  const float4* tq = tab_q + sub * (NP / 2);
-  const float4* td = tab_d + sub * (NP / 2);
-  int64_t tile = blockIdx.x;
-  for (uint32_t k = 0; tile < ntiles; ++k, tile += tstride) {
+  const float4* myq = tab_q + sub * (NP / 2);
+  const float4* myd = tab_d + sub * (NP / 2);
+  for (uint32_t k = 0;; ++k) {
     const int stage = k & 1;
+    __syncwarp();
+    const int64_t tile = tq[stage];
+    if (tile < 0) break;
     const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) atomicOr(&g_kvq_fault, 1u);
-      if (tile + tstride < ntiles) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
-      if (tid == 0) bulk_wait0();
+    if (__any_sync(kFullMask, !ok)) {
+      if (lane == 0) atomicOr(&g_kvq_fault, 1u);
+      // only the first iteration has the other stage's copy in flight
+      if (k == 0 && tq[1] >= 0) mbar_wait(&bar[1], 0, kSpinLimit);
+      if (lane == 0) bulk_wait0();
       return;
     }
-    const int64_t row = tile * ROWS + rin;
-    const bool active = row < n;
-    const uint8_t* st = smem + stage * T::STAGE;
+    if (k > 0) {
+      // the other stage holds the previous tile's output: once its stores
+      // have read it, it takes the next tile
+      if (lane == 0) bulk_wait_read0();
+      __syncwarp();
+      refill(stage ^ 1);
+    }
+    const int64_t row = tile * W::WROWS + rin;
+    uint8_t* st = wsm + stage * W::WSTAGE;
     float2 p[NP];
 #pragma unroll
     for (int j = 0; j < NP / 8; ++j) {
+      constexpr int QL = EPT / 64;
       const int ea = 8 * j, eb = HALF + 8 * j;
-      const uint4 a = *reinterpret_cast<const uint4*>(st + tile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8));
-      const uint4 b = *reinterpret_cast<const uint4*>(st + tile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8));
+      const uint4 a = *reinterpret_cast<const uint4*>(st + wtile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8));
+      const uint4 b = *reinterpret_cast<const uint4*>(st + wtile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8));
       const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const float2 fa = half2_bits_to_float2(aw[t]);
         const float2 fb = half2_bits_to_float2(bw[t]);
-        const float4 l = tq[4 * j + t];
+        const float4 l = myq[4 * j + t];
         p[8 * j + 2 * t] = __fmul2_rn(make_float2(fa.x, fb.x), make_float2(l.x, l.y));
         p[8 * j + 2 * t + 1] = __fmul2_rn(make_float2(fa.y, fb.y), make_float2(l.z, l.w));
       }
     }
-    __syncthreads();
-    issue(tile + 2 * static_cast<int64_t>(tstride), stage);
-    fwht_pairs<EPT, LANES>(p, sub);
-#pragma unroll
-    for (int m = 0; m < NP; ++m) p[m] = __fmul2_rn(p[m], c2);
-    float rx[NGH], ry[NGH];
-    uint16_t bx[NGH], by[NGH];
-    if constexpr (G <= HALF) {
-#pragma unroll
-      for (int j = 0; j < NGH; ++j) {
-        float ax = 0.f, ay = 0.f;
-#pragma unroll
-        for (int m = 0; m < GX; m += 2) {
-          ax = amax3(ax, p[j * GX + m].x, p[j * GX + m + 1].x);
-          ay = amax3(ay, p[j * GX + m].y, p[j * GX + m + 1].y);
-        }
-        bx[j] = group_scale(ax, rx[j]);
-        by[j] = group_scale(ay, ry[j]);
-      }
-    } else {
-      float a = 0.f;
-#pragma unroll
-      for (int m = 0; m < NP; ++m) a = amax3(a, p[m].x, p[m].y);
-#pragma unroll
-      for (int bit = 1; bit < G / EPT; bit <<= 1) a = fmaxf(a, __shfl_xor_sync(kFullMask, a, bit));
-      bx[0] = group_scale(a, rx[0]);
-      ry[0] = rx[0];
-      by[0] = bx[0];
-    }
-    // codes (saturated to [-8, 7]), then u = q * S, exact in fp32
     uint32_t out[EPT / 8];
+    uint16_t bx[NGH], by[NGH];
+    quantize_regs<D, G, W::WROWS>(p, sub, c2, out, bx, by);
+    if (with_codes && row < n) store_scales<D, G>(scales, row, sub, bx, by, scale_vec != 0);
+
+    // inverse, from the packed words: the same unpacking, stages and
+    // epilogue as the dequantize kernel
+    uint32_t w[EPT / 8];
 #pragma unroll
-    for (int k8 = 0; k8 < NP / 8; ++k8) {
-      int qa[8], qb[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const int m = 8 * k8 + t;
-        const float2 v = __fmul2_rn(p[m], make_float2(rx[m / GX], ry[m / GX]));
-        qa[t] = min(max(__float2int_rn(v.x), -8), 7);
-        qb[t] = min(max(__float2int_rn(v.y), -8), 7);
-        p[m] = __fmul2_rn(make_float2(__int2float_rn(qa[t]), __int2float_rn(qb[t])),
-                          make_float2(half_bits_to_float(bx[m / GX]), half_bits_to_float(by[m / GX])));
-      }
-      out[k8] = pack8(qa);
-      out[k8 + NP / 8] = pack8(qb);
-    }
-    if (active && packed != nullptr) {
-      uint8_t* dst = packed + row * (D / 2) + sub * (EPT / 2);
-#pragma unroll
-      for (int k4 = 0; k4 < EPT / 32; ++k4) {
-        const uint32_t t4[4] = {out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]};
-        st_v4(dst + 16 * k4, t4);
-      }
-      uint16_t* srow = scales + row * (D / G);
-      if constexpr (G <= HALF) {
-#pragma unroll
-        for (int j = 0; j < NGH; ++j) {
-          srow[sub * (EPT / G) + j] = bx[j];
-          srow[sub * (EPT / G) + NGH + j] = by[j];
-        }
-      } else {
-        if (sub % (G / EPT) == 0) srow[sub / (G / EPT)] = bx[0];
-      }
-    }
-    // inverse: the same butterfly, normalise, s / lambda, fp16
-    fwht_pairs<EPT, LANES>(p, sub);
-    if (tid == 0) bulk_wait_read0();
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < NP / 8; ++j) {
-      uint32_t lo[4], hi[4];
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const float4 l = td[4 * j + t];
-        const float2 a = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t], c2), make_float2(l.x, l.y));
-        const float2 b = __fmul2_rn(__fmul2_rn(p[8 * j + 2 * t + 1], c2), make_float2(l.z, l.w));
-        lo[t] = float2_to_half2_bits(a.x, b.x);
-        hi[t] = float2_to_half2_bits(a.y, b.y);
-      }
-      const int ea = 8 * j, eb = HALF + 8 * j;
-      *reinterpret_cast<uint4*>(stage_out + tile_off<D>(sub * QL + ea / 64, rin, (ea % 64) / 8)) =
-          make_uint4(lo[0], lo[1], lo[2], lo[3]);
-      *reinterpret_cast<uint4*>(stage_out + tile_off<D>(sub * QL + eb / 64, rin, (eb % 64) / 8)) =
-          make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    }
+    for (int i = 0; i < EPT / 8; ++i) w[i] = out[i] ^ 0x88888888u;
+    dequant_front<D, G>(w, bx, by, p);
+    fwht_pairs<EPT, LANES, HG, W::WROWS>(p, sub);
+    // every lane has read its input and the previous stores have read the
+    // code block (waited above): write this tile's output over its input
+    __syncwarp();
+    if (with_codes) stage_codes<D>(cst, out, sub, rin);
+    stage_rows<D>(p, c2, myd, st, sub, rin);
     fence_proxy_async();
-    __syncthreads();
-    if (tid == 0) {
+    __syncwarp();
+    if (lane == 0) {
 #pragma unroll
       for (int q = 0; q < T::Q; ++q)
-        tensor_s2g(&out_maps.q[q], 0, static_cast<int>(tile * ROWS), stage_out + q * T::QB);
+        tensor_s2g(&out_maps.q[q], 0, static_cast<int>(tile * W::WROWS), st + q * W::WQB);
+      if (with_codes) tensor_s2g(&cmap, 0, static_cast<int>(tile * W::WROWS), cst);
       bulk_commit();
     }
   }
-  if (tid == 0) bulk_wait0();
+  if (lane == 0) bulk_wait0();
 }
 
 // A barrier that nothing completes, waited on with a short limit: exercises
@@ -839,21 +878,12 @@ inline int current_device_sms(int& dev) {
   return sms < 1 ? 1 : sms;
 }
 
-template <int KIND, int D, int G, typename Kernel>
-int grid_for(Kernel k, int64_t n, int smem) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-  const int64_t need = (n + Tile<D>::ROWS - 1) / Tile<D>::ROWS;
-  int64_t cap = static_cast<int64_t>(sm_count(dev)) * blocks_per_sm<KIND, D, G, 0>(k, dev, smem, smem, kThreads);
-  if (cap < 1) cap = 1;
-  return static_cast<int>(need < cap ? need : cap);
-}
 
 
 // One 2-D map per 64-channel quarter of the fp16 rows at `base`: 64 channels
-// x n rows, row stride 2D bytes, box 64 x ROWS, 128-byte swizzle.
+// x n rows, row stride 2D bytes, box 64 x box_rows (one warp tile), 128-byte swizzle.
 template <int D>
-int make_row_maps(RowMaps& m, const void* base, int64_t n, int box_rows = Tile<D>::ROWS) {
+int make_row_maps(RowMaps& m, const void* base, int64_t n, int box_rows) {
   const EncodeTiledFn enc = encode_tiled();
   if (enc == nullptr) return KVQ_ERR_LAUNCH;
   for (int q = 0; q < D / 64; ++q) {
@@ -1001,14 +1031,25 @@ template <int D, int G>
 int launch_roundtrip(const uint16_t* x, const float* lam, const int8_t* s, int64_t n,
                      uint16_t* x_hat, uint8_t* packed, uint16_t* scales, cudaStream_t st) {
   auto k = kvq_roundtrip_kernel<D, G>;
-  constexpr int smem = roundtrip_smem_bytes<D>();
+  constexpr int smem = RStream<D>::SMEM;
   RowMaps in_maps, out_maps;
-  int rc = make_row_maps<D>(in_maps, x, n);
-  if (rc == KVQ_OK) rc = make_row_maps<D>(out_maps, x_hat, n);
+  int rc = make_row_maps<D>(in_maps, x, n, WTile<D>::WROWS);
+  if (rc == KVQ_OK) rc = make_row_maps<D>(out_maps, x_hat, n, WTile<D>::WROWS);
   if (rc != KVQ_OK) return rc;
-  const int grid = grid_for<3, D, G>(k, n, smem);
+  CUtensorMap cmap;
+  memset(&cmap, 0, sizeof(cmap));
+  if (packed != nullptr) {
+    rc = make_code_map<D>(cmap, packed, n);
+    if (rc != KVQ_OK) return rc;
+  }
+  constexpr uintptr_t kScaleRow = (D / G) * 2 < 16 ? (D / G) * 2 : 16;
+  const int svec = (reinterpret_cast<uintptr_t>(scales) % kScaleRow) == 0;
+  int dev = 0;
+  const int sms = current_device_sms(dev);
+  const int grid = stream_grid<3, D, G, kRtWarps>(k, dev, sms, n, smem);
   (void)cudaGetLastError();
-  k<<<grid, kThreads, smem, st>>>(in_maps, out_maps, lam, s, n, norm_const(D), packed, scales);
+  k<<<grid, kRtWarps * 32, smem, st>>>(in_maps, out_maps, cmap, lam, s, n, norm_const(D), scales,
+                                       packed != nullptr ? 1 : 0, svec);
   return finish_launch();
 }
 

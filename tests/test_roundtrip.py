@@ -49,3 +49,27 @@ def test_roundtrip_adversarial():
         torch.cuda.synchronize()
         p_ref, s_ref = o.quantize(x16, lam, s, G)
         assert check_dequant(o, p_ref, s_ref, lam, s, G, out.cpu().numpy(), "rt-adv") == 0
+
+
+@pytest.mark.parametrize("D,G", [(128, 32), (256, 64)])
+def test_roundtrip_many_tiles(D, G):
+    """A ragged batch with several warp tiles per warp (the tile-claim loop),
+    codes written: every row against the oracle."""
+    import torch
+    from kv_cache_quantization_02_b200 import kvq
+    o = oracle.get()
+    dev = torch.device("cuda")
+    n = 300_007
+    lam, s = workloads.params(D, seed=5)
+    x16 = workloads.host_rows(workloads.WORKLOADS["qwen3-8b-prefill" if D == 128 else "gemma-3-1b"],
+                              n, seed_offset=D)
+    xt = torch.from_numpy(x16).to(dev)
+    packed = torch.empty((n, D // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((n, D // G), dtype=torch.float16, device=dev)
+    out = kvq.roundtrip(xt, torch.from_numpy(lam).to(dev), torch.from_numpy(s).to(dev), G,
+                        packed=packed, scales=scales)
+    torch.cuda.synchronize()
+    p_ref, s_ref = o.quantize(x16, lam, s, G)
+    assert np.array_equal(packed.cpu().numpy(), p_ref)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint16), s_ref.view(np.uint16))
+    assert check_dequant(o, p_ref, s_ref, lam, s, G, out.cpu().numpy(), "rt-many") == 0
