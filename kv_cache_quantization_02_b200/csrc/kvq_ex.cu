@@ -519,26 +519,47 @@ __device__ __forceinline__ float2 cmul_rn(float2 d, float2 w) {
 }
 
 // Stockham radix-2 FFT of 64 points in registers; INV: conjugate twiddles.
+// One radix-2 stage of the Stockham FFT (sub-transforms of length n = kFN >> ST).
+template <bool INV, int ST>
+__device__ __forceinline__ void stockham_stage(float2 (&x)[kFN], float2 (&y)[kFN], const SrftTw& tw) {
+  constexpr int n = kFN >> ST, m = n / 2, sstr = 1 << ST;
+  // p = 0: w = omega^0 = (cos 0, -+sin 0) = (1, +-0).  Both of cmul_rn's
+  // products with w.x are d itself and both with w.y are signed zeros, all
+  // exact, so each component is one rounding: re = rn(d.x - d.y w.y),
+  // im = rn(d.x w.y + d.y), the same values (zero signs and NaNs included)
+  // as cmul_rn(d, w).
+  const float z0 = INV ? -tw.wn[0].y : tw.wn[0].y;
+#pragma unroll
+  for (int q = 0; q < sstr; ++q) {
+    const float2 a = x[q], b = x[q + sstr * m];
+    y[q] = __fadd2_rn(a, b);
+    const float2 d = fsub2(a, b);
+    y[q + sstr] = make_float2(__fmaf_rn(d.y, -z0, d.x), __fmaf_rn(d.x, z0, d.y));
+  }
+#pragma unroll
+  for (int p = 1; p < m; ++p) {
+    float2 w = tw.wn[p * sstr];
+    if (INV) w.y = -w.y;
+#pragma unroll
+    for (int q = 0; q < sstr; ++q) {
+      const float2 a = x[q + sstr * p], b = x[q + sstr * (p + m)];
+      y[q + sstr * 2 * p] = __fadd2_rn(a, b);
+      y[q + sstr * (2 * p + 1)] = cmul_rn(fsub2(a, b), w);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kFN; ++i) x[i] = y[i];
+}
+
 template <bool INV>
 __device__ __forceinline__ void stockham64(float2 (&x)[kFN], const SrftTw& tw) {
   float2 y[kFN];
-#pragma unroll
-  for (int st = 0; st < 6; ++st) {
-    const int n = kFN >> st, m = n / 2, sstr = 1 << st;
-#pragma unroll
-    for (int p = 0; p < m; ++p) {
-      float2 w = tw.wn[p * sstr];
-      if (INV) w.y = -w.y;
-#pragma unroll
-      for (int q = 0; q < sstr; ++q) {
-        const float2 a = x[q + sstr * p], b = x[q + sstr * (p + m)];
-        y[q + sstr * 2 * p] = __fadd2_rn(a, b);
-        y[q + sstr * (2 * p + 1)] = cmul_rn(fsub2(a, b), w);
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kFN; ++i) x[i] = y[i];
-  }
+  stockham_stage<INV, 0>(x, y, tw);
+  stockham_stage<INV, 1>(x, y, tw);
+  stockham_stage<INV, 2>(x, y, tw);
+  stockham_stage<INV, 3>(x, y, tw);
+  stockham_stage<INV, 4>(x, y, tw);
+  stockham_stage<INV, 5>(x, y, tw);
 }
 
 // Forward extraction: X_k from Z_k and Z_(64-k) (indices mod 64).
