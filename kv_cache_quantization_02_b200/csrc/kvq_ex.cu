@@ -514,8 +514,8 @@ struct SrftTw {
 // im = d.x w.y + d.y w.x, each product and sum rounded once.
 __device__ __forceinline__ float2 cmul_rn(float2 d, float2 w) {
   const float2 p0 = __fmul2_rn(d, make_float2(w.x, w.x));              // (d.x w.x, d.y w.x)
-  const float2 p1 = __fmul2_rn(make_float2(d.y, d.x), make_float2(w.y, w.y));   // (d.y w.y, d.x w.y)
-  return make_float2(__fsub_rn(p0.x, p1.x), __fadd_rn(p1.y, p0.y));
+  const float2 p1 = __fmul2_rn(d, make_float2(w.y, w.y));              // (d.x w.y, d.y w.y)
+  return make_float2(__fsub_rn(p0.x, p1.y), __fadd_rn(p1.x, p0.y));
 }
 
 // Stockham radix-2 FFT of 64 points in registers; INV: conjugate twiddles.
