@@ -36,16 +36,20 @@ __device__ __forceinline__ float amax3(float a, float b, float c) {
   return d;
 }
 
-// fp32 quotient a / 7, correctly rounded: q0 = a * RN(1/7), then one residual
-// correction r = a - 7 q0 (exact by fma), q = q0 + r * RN(1/7) (Markstein's
-// division by a known divisor; equal to IEEE a / 7.0f for every positive
-// finite fp32 a, checked exhaustively).
-__device__ __forceinline__ float div7_rn(float a) {
-  const float zh = 0x1.24924ap-3f;               // RN(1/7)
-  const float q0 = __fmul_rn(a, zh);
-  const float r = __fmaf_rn(-q0, 7.0f, a);
-  return __fmaf_rn(r, zh, q0);
+// fp32 quotient a / Q for the code range Q = 7 (int4) or 127 (int8),
+// correctly rounded: q0 = a * RN(1/Q), then one residual correction
+// r = a - Q q0 (exact by fma), q = q0 + r * RN(1/Q) (Markstein's division by
+// a known divisor).  Equal to IEEE a / Q for every non-negative finite fp32
+// a, checked exhaustively for both divisors.
+template <int Q>
+__device__ __forceinline__ float div_const_rn(float a) {
+  static_assert(Q == 7 || Q == 127, "divisor checked exhaustively");
+  const float z = Q == 7 ? 0x1.24924ap-3f : 0x1.020408p-7f;   // RN(1/Q)
+  const float q0 = __fmul_rn(a, z);
+  const float r = __fmaf_rn(-q0, static_cast<float>(Q), a);
+  return __fmaf_rn(r, z, q0);
 }
+__device__ __forceinline__ float div7_rn(float a) { return div_const_rn<7>(a); }
 // fp32 reciprocal of a positive fp16 value s, correctly rounded: approximate
 // reciprocal plus one Newton-Raphson step.  1/s lies at least 2^-35 (relative)
 // away from every rounding midpoint because s has an 11-bit significand, far
@@ -57,15 +61,17 @@ __device__ __forceinline__ float rcp_f16val(float s) {
   const float e = __fmaf_rn(-s, r0, 1.0f);
   return __fmaf_rn(r0, e, r0);
 }
-// Scale of one group: S = fp16_rne(a / 7) saturated to 65504 (satfinite);
+// Scale of one group: S = fp16_rne(a / Q) saturated to 65504 (satfinite);
 // r = 1/S, or 0 when S = 0 (which makes every code of the group 0).
-__device__ __forceinline__ uint16_t group_scale(float a, float& r) {
+template <int Q>
+__device__ __forceinline__ uint16_t group_scale_q(float a, float& r) {
   uint16_t b;
-  asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(b) : "f"(div7_rn(a)));
+  asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(b) : "f"(div_const_rn<Q>(a)));
   const float sf = half_bits_to_float(b);
   r = (sf == 0.0f) ? 0.0f : rcp_f16val(sf);
   return b;
 }
+__device__ __forceinline__ uint16_t group_scale(float a, float& r) { return group_scale_q<7>(a, r); }
 // Eight codes -> one 32-bit word, code k in bits [4k, 4k+4), each saturated
 // to [-8, 7] by the packing conversion.
 __device__ __forceinline__ uint32_t pack8(const int (&q)[8]) {

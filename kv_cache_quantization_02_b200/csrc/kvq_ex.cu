@@ -70,7 +70,7 @@ struct ExArgs {
 template <int BITS>
 struct Fmt {
   static constexpr int CB = BITS == 4 ? kD / 2 : kD;   // code bytes per row
-  static constexpr float QMAX = BITS == 4 ? 7.0f : 127.0f;
+  static constexpr int QMAX = BITS == 4 ? 7 : 127;
 };
 
 __device__ __forceinline__ int xtile_off(int q, int t, int c) {
@@ -247,11 +247,18 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
         ax = amax3(ax, p[j * G + m].x, p[j * G + m + 1].x);
         ay = amax3(ay, p[j * G + m].y, p[j * G + m + 1].y);
       }
-      asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(bx[j]) : "f"(__fdiv_rn(ax, F::QMAX)));
-      asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(by[j]) : "f"(__fdiv_rn(ay, F::QMAX)));
-      const float sx = half_bits_to_float(bx[j]), sy = half_bits_to_float(by[j]);
-      rx[j] = sx == 0.0f ? 0.0f : __frcp_rn(sx);
-      ry[j] = sy == 0.0f ? 0.0f : __frcp_rn(sy);
+      if constexpr (BITS == 4 && AFTER) {
+        // the IEEE calls give the same values; with the inlined division this
+        // instance spills and measured 2.5% slower
+        asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(bx[j]) : "f"(__fdiv_rn(ax, 7.0f)));
+        asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(by[j]) : "f"(__fdiv_rn(ay, 7.0f)));
+        const float sx = half_bits_to_float(bx[j]), sy = half_bits_to_float(by[j]);
+        rx[j] = sx == 0.0f ? 0.0f : __frcp_rn(sx);
+        ry[j] = sy == 0.0f ? 0.0f : __frcp_rn(sy);
+      } else {
+        bx[j] = group_scale_q<F::QMAX>(ax, rx[j]);
+        by[j] = group_scale_q<F::QMAX>(ay, ry[j]);
+      }
     }
     // codes = rint(y * r), saturated by the packing conversion
     uint32_t out[F::CB / 4];
@@ -783,9 +790,7 @@ kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
       float am = 0.f;
 #pragma unroll
       for (int m = 0; m < GP; ++m) am = amax3(am, z[j * GP + m].x, z[j * GP + m].y);
-      asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(b[j]) : "f"(__fdiv_rn(am, F::QMAX)));
-      const float sf = half_bits_to_float(b[j]);
-      r[j] = sf == 0.0f ? 0.0f : __frcp_rn(sf);
+      b[j] = group_scale_q<F::QMAX>(am, r[j]);
     }
     uint32_t out[F::CB / 4];
     if constexpr (BITS == 4) {
