@@ -149,12 +149,16 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
   __syncthreads();
 
   const int64_t ntiles = (a.n + kWR - 1) / kWR;
-  const unsigned int mine = static_cast<unsigned int>((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  // The block owns a contiguous range of tiles, so a warp's tiles stay in one
+  // lambda table for long stretches (a table spans lambda_rows / 32 tiles).
+  const int64_t per = ntiles / gridDim.x, rem = ntiles % gridDim.x;
+  const int64_t first = blockIdx.x * per + (blockIdx.x < rem ? blockIdx.x : rem);
+  const unsigned int mine = static_cast<unsigned int>(per + (blockIdx.x < rem ? 1 : 0));
   auto claim = [&]() -> int {
     unsigned int i = 0;
     if (lane == 0) i = atomicAdd(next, 1u);
     i = __shfl_sync(kFullMask, i, 0);
-    return i < mine ? static_cast<int>(blockIdx.x + i * gridDim.x) : -1;
+    return i < mine ? static_cast<int>(first + i) : -1;
   };
   auto refill = [&](int stage) {
     const int t = claim();
@@ -379,12 +383,16 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
   __syncthreads();
 
   const int64_t ntiles = (a.n + kWR - 1) / kWR;
-  const unsigned int mine = static_cast<unsigned int>((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  // The block owns a contiguous range of tiles, so a warp's tiles stay in one
+  // lambda table for long stretches (a table spans lambda_rows / 32 tiles).
+  const int64_t per = ntiles / gridDim.x, rem = ntiles % gridDim.x;
+  const int64_t first = blockIdx.x * per + (blockIdx.x < rem ? blockIdx.x : rem);
+  const unsigned int mine = static_cast<unsigned int>(per + (blockIdx.x < rem ? 1 : 0));
   auto claim = [&]() -> int {
     unsigned int i = 0;
     if (lane == 0) i = atomicAdd(next, 1u);
     i = __shfl_sync(kFullMask, i, 0);
-    return i < mine ? static_cast<int>(blockIdx.x + i * gridDim.x) : -1;
+    return i < mine ? static_cast<int>(first + i) : -1;
   };
   auto scale_bytes = [&](int64_t t) -> uint32_t {
     if (!scale_copy) return 0;
@@ -709,12 +717,16 @@ kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
   __syncthreads();
 
   const int64_t ntiles = (a.n + kWR - 1) / kWR;
-  const unsigned int mine = static_cast<unsigned int>((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  // The block owns a contiguous range of tiles, so a warp's tiles stay in one
+  // lambda table for long stretches (a table spans lambda_rows / 32 tiles).
+  const int64_t per = ntiles / gridDim.x, rem = ntiles % gridDim.x;
+  const int64_t first = blockIdx.x * per + (blockIdx.x < rem ? blockIdx.x : rem);
+  const unsigned int mine = static_cast<unsigned int>(per + (blockIdx.x < rem ? 1 : 0));
   auto claim = [&]() -> int {
     unsigned int i = 0;
     if (lane == 0) i = atomicAdd(next, 1u);
     i = __shfl_sync(kFullMask, i, 0);
-    return i < mine ? static_cast<int>(blockIdx.x + i * gridDim.x) : -1;
+    return i < mine ? static_cast<int>(first + i) : -1;
   };
   auto refill = [&](int stage) {
     const int t = claim();
@@ -875,12 +887,16 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const __grid_const
   __syncthreads();
 
   const int64_t ntiles = (a.n + kWR - 1) / kWR;
-  const unsigned int mine = static_cast<unsigned int>((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  // The block owns a contiguous range of tiles, so a warp's tiles stay in one
+  // lambda table for long stretches (a table spans lambda_rows / 32 tiles).
+  const int64_t per = ntiles / gridDim.x, rem = ntiles % gridDim.x;
+  const int64_t first = blockIdx.x * per + (blockIdx.x < rem ? blockIdx.x : rem);
+  const unsigned int mine = static_cast<unsigned int>(per + (blockIdx.x < rem ? 1 : 0));
   auto claim = [&]() -> int {
     unsigned int i = 0;
     if (lane == 0) i = atomicAdd(next, 1u);
     i = __shfl_sync(kFullMask, i, 0);
-    return i < mine ? static_cast<int>(blockIdx.x + i * gridDim.x) : -1;
+    return i < mine ? static_cast<int>(first + i) : -1;
   };
   auto scale_bytes = [&](int64_t t) -> uint32_t {
     if (!scale_copy) return 0;
