@@ -45,7 +45,8 @@ constexpr unsigned kFullMask = 0xffffffffu;
 
 constexpr int kD = 128;                 // channels (one lane per vector)
 constexpr int kNP = kD / 2;             // packed pairs (v[m], v[m+64])
-constexpr int kXW = 4;                  // warps per block
+constexpr int kQW = 12;                 // warps of a WHT quantize block (one per SM, 170 registers)
+constexpr int kDW = 8;                  // warps of a dequantize or SRFT block (one per SM, 255 registers)
 constexpr int kWR = 32;                 // vectors per warp tile
 constexpr int kQB = kWR * 128;          // bytes of one 64-channel quarter of a tile
 constexpr int kXStage = 2 * kQB;        // bytes of one fp16 warp tile
@@ -107,10 +108,11 @@ __device__ __forceinline__ void build_signs(float4* stab, const ExArgs& a, int q
   stab[q] = make_float4(v[0], v[1], v[2], v[3]);
 }
 
-// Header of a block: per-warp tables (kXW x 512 B), the sign table (512 B),
-// then two mbarriers and two tile ids per warp and the claim counter.
-constexpr int kHdrBars = kXW * 512 + 512;
-constexpr int kHdrBytes = kHdrBars + 24 * kXW + 16;
+// Header of a block of nw warps: per-warp tables (nw x 512 B), the sign
+// table (512 B), then two mbarriers and two tile ids per warp and the claim
+// counter.
+__host__ __device__ constexpr int hdr_bars(int nw) { return nw * 512 + 512; }
+__host__ __device__ constexpr int hdr_bytes(int nw) { return hdr_bars(nw) + 24 * nw + 16; }
 
 // Four codes -> one 32-bit word, code k in byte k, each saturated to [-128, 127].
 __device__ __forceinline__ uint32_t pack4_s8(int a0, int a1, int a2, int a3) {
@@ -124,7 +126,7 @@ __device__ __forceinline__ uint32_t pack4_s8(int a0, int a1, int a2, int a3) {
 // Quantize variants: fp16 [n][128] -> codes [n][CB] + fp16 scales [n][128/G].
 // ---------------------------------------------------------------------------
 template <int G, int BITS, bool AFTER>
-__global__ void __launch_bounds__(kXW * 32, 3)
+__global__ void __launch_bounds__(kQW * 32, 1)
 kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
                        uint8_t* __restrict__ codes, const __grid_constant__ CUtensorMap cmap,
                        uint16_t* __restrict__ scales) {
@@ -137,12 +139,12 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* wsm = smem + warp * 2 * kXStage;
-  uint8_t* hdr = smem + kXW * 2 * kXStage;
+  uint8_t* hdr = smem + kQW * 2 * kXStage;
   float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;                       // 512 B per warp
-  float4* stab = reinterpret_cast<float4*>(hdr + kXW * 512);                        // +-1, 512 B
-  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + kHdrBars) + 2 * warp;
-  int* tq = reinterpret_cast<int*>(hdr + kHdrBars + 16 * kXW) + 2 * warp;
-  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + kHdrBars + 24 * kXW);
+  float4* stab = reinterpret_cast<float4*>(hdr + kQW * 512);                        // +-1, 512 B
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + hdr_bars(kQW)) + 2 * warp;
+  int* tq = reinterpret_cast<int*>(hdr + hdr_bars(kQW) + 16 * kQW) + 2 * warp;
+  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + hdr_bars(kQW) + 24 * kQW);
   if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   if (tid == 0) *next = 0;
   if (tid < 32) build_signs(stab, a, tid);
@@ -359,7 +361,7 @@ __device__ __forceinline__ uint4 code_chunk(const uint8_t* tile, int lane, int c
 }
 
 template <int G, int BITS, bool AFTER>
-__global__ void __launch_bounds__(kXW * 32, 2)
+__global__ void __launch_bounds__(kDW * 32, 1)
 kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constant__ CUtensorMap cmap,
                          const uint16_t* __restrict__ scales,
                          const ExArgs a, const __grid_constant__ ExMaps omaps, int scale_copy) {
@@ -371,12 +373,12 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* stage_out = smem + warp * L::WARP;              // swizzled fp16 staging tile
   uint8_t* wsm = stage_out + kXStage;                      // two code tiles, then two scale blocks
-  uint8_t* hdr = smem + kXW * L::WARP;
+  uint8_t* hdr = smem + kDW * L::WARP;
   float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
-  float4* stab = reinterpret_cast<float4*>(hdr + kXW * 512);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + kHdrBars) + 2 * warp;
-  int* tq = reinterpret_cast<int*>(hdr + kHdrBars + 16 * kXW) + 2 * warp;
-  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + kHdrBars + 24 * kXW);
+  float4* stab = reinterpret_cast<float4*>(hdr + kDW * 512);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + hdr_bars(kDW)) + 2 * warp;
+  int* tq = reinterpret_cast<int*>(hdr + hdr_bars(kDW) + 16 * kDW) + 2 * warp;
+  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + hdr_bars(kDW) + 24 * kDW);
   if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   if (tid == 0) *next = 0;
   if (tid < 32) build_signs(stab, a, tid);
@@ -692,7 +694,7 @@ __device__ __forceinline__ void build_signs_nat(float4* stab, const ExArgs& a, i
 }
 
 template <int G, int BITS, bool AFTER>
-__global__ void __launch_bounds__(kXW * 32, 2)
+__global__ void __launch_bounds__(kDW * 32, 1)
 kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
                          const __grid_constant__ SrftTw tw, float c0, float c1,
                          uint8_t* __restrict__ codes,
@@ -705,12 +707,12 @@ kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* wsm = smem + warp * 2 * kXStage;
-  uint8_t* hdr = smem + kXW * 2 * kXStage;
+  uint8_t* hdr = smem + kDW * 2 * kXStage;
   float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
-  float4* stab = reinterpret_cast<float4*>(hdr + kXW * 512);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + kHdrBars) + 2 * warp;
-  int* tq = reinterpret_cast<int*>(hdr + kHdrBars + 16 * kXW) + 2 * warp;
-  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + kHdrBars + 24 * kXW);
+  float4* stab = reinterpret_cast<float4*>(hdr + kDW * 512);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + hdr_bars(kDW)) + 2 * warp;
+  int* tq = reinterpret_cast<int*>(hdr + hdr_bars(kDW) + 16 * kDW) + 2 * warp;
+  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + hdr_bars(kDW) + 24 * kDW);
   if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   if (tid == 0) *next = 0;
   if (tid < 32) build_signs_nat(stab, a, tid);
@@ -861,7 +863,7 @@ kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
 }
 
 template <int G, int BITS, bool AFTER>
-__global__ void __launch_bounds__(kXW * 32, 2)
+__global__ void __launch_bounds__(kDW * 32, 1)
 kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const __grid_constant__ CUtensorMap cmap,
                            const uint16_t* __restrict__ scales,
                            const ExArgs a, const __grid_constant__ SrftTw tw, float c0, float c1,
@@ -875,12 +877,12 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const __grid_const
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* stage_out = smem + warp * L::WARP;              // swizzled fp16 staging tile
   uint8_t* wsm = stage_out + kXStage;                      // two code tiles, then two scale blocks
-  uint8_t* hdr = smem + kXW * L::WARP;
+  uint8_t* hdr = smem + kDW * L::WARP;
   float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
-  float4* stab = reinterpret_cast<float4*>(hdr + kXW * 512);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + kHdrBars) + 2 * warp;
-  int* tq = reinterpret_cast<int*>(hdr + kHdrBars + 16 * kXW) + 2 * warp;
-  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + kHdrBars + 24 * kXW);
+  float4* stab = reinterpret_cast<float4*>(hdr + kDW * 512);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + hdr_bars(kDW)) + 2 * warp;
+  int* tq = reinterpret_cast<int*>(hdr + hdr_bars(kDW) + 16 * kDW) + 2 * warp;
+  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + hdr_bars(kDW) + 24 * kDW);
   if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   if (tid == 0) *next = 0;
   if (tid < 32) build_signs_nat(stab, a, tid);
@@ -1041,13 +1043,13 @@ int ex_sms(int& dev) {
 }
 
 template <typename Kernel>
-int ex_grid(Kernel k, int64_t n, int smem, std::atomic<int>* ready) {
+int ex_grid(Kernel k, int64_t n, int smem, int threads, std::atomic<int>* ready) {
   int dev = 0;
   const int sms = ex_sms(dev);
   int occ = ready[dev].load(std::memory_order_relaxed);
   if (occ == 0) {
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kXW * 32, smem) != cudaSuccess || occ < 1) occ = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, threads, smem) != cudaSuccess || occ < 1) occ = 1;
     ready[dev].store(occ, std::memory_order_relaxed);
   }
   const int64_t tiles = (n + kWR - 1) / kWR;
@@ -1083,9 +1085,9 @@ int launch_qex(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* sca
   const int rc = encode_x_maps(maps, x, a.n);
   if (rc != KVQ_OK) return rc;
   auto k = kvq_quantize_ex_kernel<G, BITS, AFTER>;
-  constexpr int smem = 1024 + kXW * 2 * kXStage + kHdrBytes;
+  constexpr int smem = 1024 + kQW * 2 * kXStage + hdr_bytes(kQW);
   static std::atomic<int> ready[64];
-  const int grid = ex_grid(k, a.n, smem, ready);
+  const int grid = ex_grid(k, a.n, smem, kQW * 32, ready);
   CUtensorMap cmap;
   memset(&cmap, 0, sizeof(cmap));
   if (BITS == 8) {
@@ -1093,7 +1095,7 @@ int launch_qex(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* sca
     if (rc2 != KVQ_OK) return rc2;
   }
   (void)cudaGetLastError();
-  k<<<grid, kXW * 32, smem, st>>>(maps, a, codes, cmap, scales);
+  k<<<grid, kQW * 32, smem, st>>>(maps, a, codes, cmap, scales);
   return finish_ex();
 }
 
@@ -1105,9 +1107,9 @@ int launch_dex(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, ui
   const int rc = encode_x_maps(omaps, out, a.n);
   if (rc != KVQ_OK) return rc;
   auto k = kvq_dequantize_ex_kernel<G, BITS, AFTER>;
-  constexpr int smem = 1024 + kXW * L::WARP + kHdrBytes;
+  constexpr int smem = 1024 + kDW * L::WARP + hdr_bytes(kDW);
   static std::atomic<int> ready[64];
-  const int grid = ex_grid(k, a.n, smem, ready);
+  const int grid = ex_grid(k, a.n, smem, kDW * 32, ready);
   CUtensorMap cmap;
   memset(&cmap, 0, sizeof(cmap));
   if (BITS == 8) {
@@ -1115,7 +1117,7 @@ int launch_dex(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, ui
     if (rc2 != KVQ_OK) return rc2;
   }
   (void)cudaGetLastError();
-  k<<<grid, kXW * 32, smem, st>>>(codes, cmap, scales, a, omaps,
+  k<<<grid, kDW * 32, smem, st>>>(codes, cmap, scales, a, omaps,
                                   (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
   return finish_ex();
 }
@@ -1188,9 +1190,9 @@ int launch_qsrft(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* s
   const int rc = encode_x_maps(maps, x, a.n);
   if (rc != KVQ_OK) return rc;
   auto k = kvq_quantize_srft_kernel<G, BITS, AFTER>;
-  constexpr int smem = 1024 + kXW * 2 * kXStage + kHdrBytes;
+  constexpr int smem = 1024 + kDW * 2 * kXStage + hdr_bytes(kDW);
   static std::atomic<int> ready[64];
-  const int grid = ex_grid(k, a.n, smem, ready);
+  const int grid = ex_grid(k, a.n, smem, kDW * 32, ready);
   CUtensorMap cmap;
   memset(&cmap, 0, sizeof(cmap));
   if (BITS == 8) {
@@ -1198,7 +1200,7 @@ int launch_qsrft(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* s
     if (rc2 != KVQ_OK) return rc2;
   }
   (void)cudaGetLastError();
-  k<<<grid, kXW * 32, smem, st>>>(maps, a, srft_twiddles(), kSrftC0, kSrftC1, codes, cmap, scales);
+  k<<<grid, kDW * 32, smem, st>>>(maps, a, srft_twiddles(), kSrftC0, kSrftC1, codes, cmap, scales);
   return finish_ex();
 }
 
@@ -1210,9 +1212,9 @@ int launch_dsrft(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, 
   const int rc = encode_x_maps(omaps, out, a.n);
   if (rc != KVQ_OK) return rc;
   auto k = kvq_dequantize_srft_kernel<G, BITS, AFTER>;
-  constexpr int smem = 1024 + kXW * L::WARP + kHdrBytes;
+  constexpr int smem = 1024 + kDW * L::WARP + hdr_bytes(kDW);
   static std::atomic<int> ready[64];
-  const int grid = ex_grid(k, a.n, smem, ready);
+  const int grid = ex_grid(k, a.n, smem, kDW * 32, ready);
   CUtensorMap cmap;
   memset(&cmap, 0, sizeof(cmap));
   if (BITS == 8) {
@@ -1220,7 +1222,7 @@ int launch_dsrft(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, 
     if (rc2 != KVQ_OK) return rc2;
   }
   (void)cudaGetLastError();
-  k<<<grid, kXW * 32, smem, st>>>(codes, cmap, scales, a, srft_twiddles(), kSrftC0, kSrftC1, omaps,
+  k<<<grid, kDW * 32, smem, st>>>(codes, cmap, scales, a, srft_twiddles(), kSrftC0, kSrftC1, omaps,
                                   (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
   return finish_ex();
 }
