@@ -253,18 +253,8 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
         ax = amax3(ax, p[j * G + m].x, p[j * G + m + 1].x);
         ay = amax3(ay, p[j * G + m].y, p[j * G + m + 1].y);
       }
-      if constexpr (BITS == 4 && AFTER) {
-        // the IEEE calls give the same values; with the inlined division this
-        // instance spills and measured 2.5% slower
-        asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(bx[j]) : "f"(__fdiv_rn(ax, 7.0f)));
-        asm("cvt.rn.satfinite.f16.f32 %0, %1;" : "=h"(by[j]) : "f"(__fdiv_rn(ay, 7.0f)));
-        const float sx = half_bits_to_float(bx[j]), sy = half_bits_to_float(by[j]);
-        rx[j] = sx == 0.0f ? 0.0f : __frcp_rn(sx);
-        ry[j] = sy == 0.0f ? 0.0f : __frcp_rn(sy);
-      } else {
-        bx[j] = group_scale_q<F::QMAX>(ax, rx[j]);
-        by[j] = group_scale_q<F::QMAX>(ay, ry[j]);
-      }
+      bx[j] = group_scale_q<F::QMAX>(ax, rx[j]);
+      by[j] = group_scale_q<F::QMAX>(ay, ry[j]);
     }
     // codes = rint(y * r), saturated by the packing conversion
     uint32_t out[F::CB / 4];
