@@ -293,7 +293,9 @@ def run_gpu(args):
     d_ms = max_over_ranks(d_ms, world, dev)
 
     extra = {}
-    if not args.no_extra:
+    if args.variants_only:
+        extra = {"codec_variants": run_variants(torch, kvq, dev, stream, x, out, s_t, G, w)}
+    elif not args.no_extra:
         extra = run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, args.attn_seqs)
 
     bpv = bytes_per_vector(D, G)
@@ -752,6 +754,8 @@ def parse(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-extra", action="store_true", help="skip round-trip, append and attention figures")
+    p.add_argument("--variants-only", action="store_true",
+                   help="of the secondary figures, only the codec variants (profiling)")
     p.add_argument("--attn-seqs", type=int, default=64, help="sequences of the attention figure (profiling)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--e2e-chunks", type=int, default=16)
