@@ -128,12 +128,8 @@ __device__ __forceinline__ uint32_t pack4_s8(int a0, int a1, int a2, int a3) {
 template <int G, int BITS, bool AFTER>
 __global__ void __launch_bounds__(kQW * 32, 1)
 kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
-                       uint8_t* __restrict__ codes, const __grid_constant__ CUtensorMap cmap,
-                       uint16_t* __restrict__ scales) {
+                       const __grid_constant__ CUtensorMap cmap, uint16_t* __restrict__ scales) {
   using F = Fmt<BITS>;
-  // int8 codes leave through the tile's input stage and one tensor store; int4
-  // codes (64-byte rows) measured faster with direct stores
-  constexpr bool STG = BITS == 8;
   constexpr int NGH = kNP / G;          // groups per half of the lane's channels
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -182,13 +178,12 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
     const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_ex_fault, 1u);
-      // with staged codes only the first tile has the other stage's copy in flight
-      if (STG ? (k == 0 && tq[1] >= 0) : tq[stage ^ 1] >= 0)
-        mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinX);
-      if (STG && lane == 0) bulk_wait0();
+      // only the first tile has the other stage's copy in flight
+      if (k == 0 && tq[1] >= 0) mbar_wait(&bar[1], 0, kSpinX);
+      if (lane == 0) bulk_wait0();
       return;
     }
-    if (STG && k > 0) {
+    if (k > 0) {
       // the other stage holds the previous tile's staged codes: once their
       // store has read them, it takes the next tile
       if (lane == 0) bulk_wait_read0();
@@ -227,10 +222,6 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
       }
     }
 
-    if constexpr (!STG) {
-      __syncwarp();                     // the tile is in registers: refill its stage
-      refill(stage);
-    }
     fwht_pairs<kD, 1>(p, 0);
 #pragma unroll
     for (int m = 0; m < kNP; ++m) p[m] = __fmul2_rn(p[m], c2);
@@ -287,11 +278,11 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
         out[k4 + kNP / 4] = pack4_s8(qb[0], qb[1], qb[2], qb[3]);
       }
     }
-    if constexpr (STG) {
-      // the codes leave through the stage this tile came from (every lane has
-      // read it), swizzled as code_chunk reads, by one tensor store that
-      // skips rows past n
-      __syncwarp();
+    // the codes leave through the stage this tile came from (every lane has
+    // read it), swizzled as code_chunk reads, by one tensor store that skips
+    // rows past n
+    __syncwarp();
+    {
       uint8_t* cst = wsm + stage * kXStage;
       const int swz = ((lane * F::CB) >> 7) & (F::CB / 16 - 1);
 #pragma unroll
@@ -304,13 +295,6 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
         tensor_s2g(&cmap, 0, static_cast<int>(tile * kWR), cst);
         bulk_commit();
       }
-    } else if (active) {
-      uint8_t* dst = codes + row * F::CB;
-#pragma unroll
-      for (int k4 = 0; k4 < F::CB / 16; ++k4) {
-        const uint32_t t4[4] = {out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]};
-        st_v4(dst + 16 * k4, t4);
-      }
     }
     if (active) {
       uint16_t* srow = scales + row * (kD / G);
@@ -321,7 +305,7 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
       }
     }
   }
-  if (STG && lane == 0) bulk_wait0();
+  if (lane == 0) bulk_wait0();
 }
 
 // ---------------------------------------------------------------------------
@@ -687,10 +671,8 @@ template <int G, int BITS, bool AFTER>
 __global__ void __launch_bounds__(kDW * 32, 1)
 kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
                          const __grid_constant__ SrftTw tw, float c0, float c1,
-                         uint8_t* __restrict__ codes,
                          const __grid_constant__ CUtensorMap cmap, uint16_t* __restrict__ scales) {
   using F = Fmt<BITS>;
-  constexpr bool STG = BITS == 8;   // as in kvq_quantize_ex_kernel
   constexpr int GP = G / 2;             // pairs per group
   constexpr int NG = kD / G;
   extern __shared__ uint8_t smem_raw[];
@@ -739,13 +721,12 @@ kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
     const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_ex_fault, 1u);
-      // with staged codes only the first tile has the other stage's copy in flight
-      if (STG ? (k == 0 && tq[1] >= 0) : tq[stage ^ 1] >= 0)
-        mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinX);
-      if (STG && lane == 0) bulk_wait0();
+      // only the first tile has the other stage's copy in flight
+      if (k == 0 && tq[1] >= 0) mbar_wait(&bar[1], 0, kSpinX);
+      if (lane == 0) bulk_wait0();
       return;
     }
-    if (STG && k > 0) {
+    if (k > 0) {
       // the other stage holds the previous tile's staged codes: once their
       // store has read them, it takes the next tile
       if (lane == 0) bulk_wait_read0();
@@ -774,10 +755,6 @@ kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
       z[4 * c + 3] = __fmul2_rn(half2_bits_to_float2(xw[3]), make_float2(l1.z, l1.w));
     }
 
-    if constexpr (!STG) {
-      __syncwarp();
-      refill(stage);
-    }
     srft_fwd(z, tw, c0, c1);
     if constexpr (AFTER) {
 #pragma unroll
@@ -818,11 +795,11 @@ kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
         out[k4] = pack4_s8(__float2int_rn(v0.x), __float2int_rn(v0.y), __float2int_rn(v1.x), __float2int_rn(v1.y));
       }
     }
-    if constexpr (STG) {
-      // the codes leave through the stage this tile came from (every lane has
-      // read it), swizzled as code_chunk reads, by one tensor store that
-      // skips rows past n
-      __syncwarp();
+    // the codes leave through the stage this tile came from (every lane has
+    // read it), swizzled as code_chunk reads, by one tensor store that skips
+    // rows past n
+    __syncwarp();
+    {
       uint8_t* cst = wsm + stage * kXStage;
       const int swz = ((lane * F::CB) >> 7) & (F::CB / 16 - 1);
 #pragma unroll
@@ -835,13 +812,6 @@ kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
         tensor_s2g(&cmap, 0, static_cast<int>(tile * kWR), cst);
         bulk_commit();
       }
-    } else if (active) {
-      uint8_t* dst = codes + row * F::CB;
-#pragma unroll
-      for (int k4 = 0; k4 < F::CB / 16; ++k4) {
-        const uint32_t t4[4] = {out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]};
-        st_v4(dst + 16 * k4, t4);
-      }
     }
     if (active) {
       uint16_t* srow = scales + row * NG;
@@ -849,7 +819,7 @@ kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
       for (int j = 0; j < NG; ++j) srow[j] = b[j];
     }
   }
-  if (STG && lane == 0) bulk_wait0();
+  if (lane == 0) bulk_wait0();
 }
 
 template <int G, int BITS, bool AFTER>
@@ -1079,13 +1049,10 @@ int launch_qex(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* sca
   static std::atomic<int> ready[64];
   const int grid = ex_grid(k, a.n, smem, kQW * 32, ready);
   CUtensorMap cmap;
-  memset(&cmap, 0, sizeof(cmap));
-  if (BITS == 8) {
-    const int rc2 = encode_code_map(cmap, codes, a.n, Fmt<BITS>::CB);
-    if (rc2 != KVQ_OK) return rc2;
-  }
+  const int rc2 = encode_code_map(cmap, codes, a.n, Fmt<BITS>::CB);
+  if (rc2 != KVQ_OK) return rc2;
   (void)cudaGetLastError();
-  k<<<grid, kQW * 32, smem, st>>>(maps, a, codes, cmap, scales);
+  k<<<grid, kQW * 32, smem, st>>>(maps, a, cmap, scales);
   return finish_ex();
 }
 
@@ -1152,10 +1119,10 @@ int encode_x_maps(ExMaps& maps, const uint16_t* x, int64_t n) {
 
 // The codes [n][cb] (cb = 64 or 128 bytes) as one 2-D map with a box of one
 // warp tile, swizzled over the row's cb bytes (the layout code_chunk reads).
-// The int8 quantisers store their codes and the int8 dequantisers read them
-// through it.  The int4 kernels, whose arithmetic leaves shared memory idle,
-// measured faster with direct stores and plain bulk copies of the linear
-// 64-byte rows.
+// Every variant quantiser stores its codes through it, and the int8
+// dequantisers read them through it (the int4 dequantisers, whose arithmetic
+// leaves shared memory idle, measured faster with plain bulk copies of the
+// linear 64-byte rows).
 int encode_code_map(CUtensorMap& map, const uint8_t* codes, int64_t n, int cb) {
   const EncodeTiledFn enc = encode_tiled();
   if (enc == nullptr) return KVQ_ERR_LAUNCH;
@@ -1184,13 +1151,10 @@ int launch_qsrft(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* s
   static std::atomic<int> ready[64];
   const int grid = ex_grid(k, a.n, smem, kDW * 32, ready);
   CUtensorMap cmap;
-  memset(&cmap, 0, sizeof(cmap));
-  if (BITS == 8) {
-    const int rc2 = encode_code_map(cmap, codes, a.n, Fmt<BITS>::CB);
-    if (rc2 != KVQ_OK) return rc2;
-  }
+  const int rc2 = encode_code_map(cmap, codes, a.n, Fmt<BITS>::CB);
+  if (rc2 != KVQ_OK) return rc2;
   (void)cudaGetLastError();
-  k<<<grid, kDW * 32, smem, st>>>(maps, a, srft_twiddles(), kSrftC0, kSrftC1, codes, cmap, scales);
+  k<<<grid, kDW * 32, smem, st>>>(maps, a, srft_twiddles(), kSrftC0, kSrftC1, cmap, scales);
   return finish_ex();
 }
 
