@@ -13,17 +13,25 @@
 //   * 8-bit codes: S = fp16(max|y| / 127), q in [-128, 127], one byte each;
 //   * one lambda table per range of rows: row r uses table
 //     (r / lambda_rows) % n_lambda (per-(layer, head) smoothing).
+// The rotation is the SRHT above, or (flags bit KVQ_SRFT) the SRFT of the same
+// summary: pack(F diag(s) x), F the unitary DFT, as a 64-point Stockham FFT
+// of the channel pairs plus the Hermitian unpacking.
+//
 // D = 128; G in {16, 32, 64}.  One lane holds a whole vector as 64 packed
-// fp32 pairs (v[m], v[m+64]); each warp streams 32-vector tiles through its
-// own double-buffered ring (fp16 rows by swizzled tensor copies, codes and
-// scales by bulk copies), and the warps of a block claim tiles from a shared
-// counter.  A warp tile lies inside one lambda table (lambda_rows is a
-// multiple of 32 when there are several), so the warp rebuilds its per-channel
-// table in shared memory when a tile's table differs from the last one's.
-// Every step is the oracle's IEEE operation in the oracle's order: the scale is
-// a correctly rounded division by 7 or 127, 1/S and 1/lambda correctly rounded
-// reciprocals, so results are bit-identical.  Bounded waits as in the base
-// kernels (a warp that gives up sets bit 0 of the fault word and returns).
+// fp32 pairs; each warp streams 32-vector tiles through its own
+// double-buffered ring, and the warps of a block (one per SM: 12 warps for the
+// WHT quantisers, 8 for the rest) claim tiles of a contiguous range from a
+// shared counter.  fp16 rows move by swizzled tensor copies; the codes leave
+// the quantisers through the stage their tile came from and one tensor store,
+// and enter the dequantisers by a swizzled tensor copy (int8) or a bulk copy
+// (int4); scales move by bulk copies.  A warp tile lies inside one lambda
+// table (lambda_rows is a multiple of 32 when there are several), so the warp
+// rebuilds its per-channel table in shared memory when a tile's table differs
+// from the last one's.  Every step is the oracle's IEEE operation in the
+// oracle's order: the scale is a correctly rounded division by 7 or 127, 1/S
+// and 1/lambda correctly rounded reciprocals, so results are bit-identical.
+// Bounded waits as in the base kernels (a warp that gives up sets bit 0 of the
+// fault word and returns).
 
 #include <cuda.h>
 #include <cuda_runtime.h>
