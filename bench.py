@@ -295,6 +295,10 @@ def run_gpu(args):
     extra = {}
     if args.variants_only:
         extra = {"codec_variants": run_variants(torch, kvq, dev, stream, x, out, s_t, G, w)}
+    elif args.roundtrip_only:
+        rt_ms = _event_ms(torch, stream,
+                          lambda: kvq.roundtrip(x, lam_t, s_t, G, out=out, stream=stream), 10)
+        extra = {"roundtrip_ms": round(rt_ms, 5)}
     elif not args.no_extra:
         extra = run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, args.attn_seqs)
 
@@ -756,6 +760,8 @@ def parse(argv=None):
     p.add_argument("--no-extra", action="store_true", help="skip round-trip, append and attention figures")
     p.add_argument("--variants-only", action="store_true",
                    help="of the secondary figures, only the codec variants (profiling)")
+    p.add_argument("--roundtrip-only", action="store_true",
+                   help="of the secondary figures, only the fused round trip (profiling)")
     p.add_argument("--attn-seqs", type=int, default=64, help="sequences of the attention figure (profiling)")
     p.add_argument("--e2e-steps", type=int, default=3)
     p.add_argument("--e2e-chunks", type=int, default=16)
