@@ -434,10 +434,10 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
       sx[j] = srow[j];
       sy[j] = srow[NGH + j];
     }
-    // codes of the pair (m, m+64) as exact fp16 integers, then u = q S exactly.
-    // int4: the row is linear (64 bytes); int8: word w of the row is word
-    // w % 4 of swizzled chunk w / 4.
-    float2 p[kNP];
+    // codes of the pair (m, m+64) as exact fp16 integers.  int4: the row is
+    // linear (64 bytes); int8: word w of the row is word w % 4 of swizzled
+    // chunk w / 4.
+    __half2 hq[kNP];
     if constexpr (BITS == 4) {
       const uint2* seg = reinterpret_cast<const uint2*>(st + lane * F::CB);
       const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
@@ -452,11 +452,8 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
           const uint32_t sel = 0x0400u | (t << 8) | t;
           const uint32_t e0 = (__byte_perm(wa, wb, sel) & 0x000F000Fu) | 0x64006400u;
           const uint32_t e1 = (__byte_perm(wa4, wb4, sel) & 0x000F000Fu) | 0x64006400u;
-          const __half2 h0 = __hsub2(*reinterpret_cast<const __half2*>(&e0), bias);
-          const __half2 h1 = __hsub2(*reinterpret_cast<const __half2*>(&e1), bias);
-          const int m0 = 8 * kw + 2 * t, m1 = m0 + 1;
-          p[m0] = make_float2(mul_f16_f32(__low2half(h0), sx[m0 / G]), mul_f16_f32(__high2half(h0), sy[m0 / G]));
-          p[m1] = make_float2(mul_f16_f32(__low2half(h1), sx[m1 / G]), mul_f16_f32(__high2half(h1), sy[m1 / G]));
+          hq[8 * kw + 2 * t] = __hsub2(*reinterpret_cast<const __half2*>(&e0), bias);
+          hq[8 * kw + 2 * t + 1] = __hsub2(*reinterpret_cast<const __half2*>(&e1), bias);
         }
       }
     } else {
@@ -472,12 +469,33 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
         for (int t = 0; t < 4; ++t) {
           const uint32_t sel = 0x0400u | (t << 8) | t;
           const uint32_t e = (__byte_perm(wa, wb, sel) & 0x00FF00FFu) | 0x64006400u;
-          const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&e), bias);
-          const int m = 4 * kw + t;
-          p[m] = make_float2(mul_f16_f32(__low2half(h), sx[m / G]), mul_f16_f32(__high2half(h), sy[m / G]));
+          hq[4 * kw + t] = __hsub2(*reinterpret_cast<const __half2*>(&e), bias);
         }
       }
     }
+    // With lambda before the rotation u = q S, and every butterfly stage inside
+    // a group keeps u an exact multiple of S: the stages h < HF run on the fp16
+    // integers (sums of at most 8 * 64 = 512 for int4 through all in-group
+    // stages, 128 * 16 = 2048 for int8 through four), then u = W S exactly by
+    // one mixed fma (W S has at most 23 significant bits), the same fp32
+    // values as the oracle's stage-by-stage sums.  With lambda after, 1/lambda
+    // comes before the transform and every stage runs in fp32.
+    constexpr int HF = AFTER ? 1 : (BITS == 4 ? (G < kNP ? G : kNP) : 16);
+#pragma unroll
+    for (int h = 1; h < HF; h <<= 1) {
+#pragma unroll
+      for (int m = 0; m < kNP; ++m) {
+        if ((m & h) == 0) {
+          const __half2 a2 = hq[m], b2 = hq[m + h];
+          hq[m] = __hadd2(a2, b2);
+          hq[m + h] = __hsub2(a2, b2);
+        }
+      }
+    }
+    float2 p[kNP];
+#pragma unroll
+    for (int m = 0; m < kNP; ++m)
+      p[m] = make_float2(mul_f16_f32(__low2half(hq[m]), sx[m / G]), mul_f16_f32(__high2half(hq[m]), sy[m / G]));
     __syncwarp();                       // codes and scales consumed: refill the stage
     refill(stage);
     if constexpr (AFTER) {
@@ -488,7 +506,7 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
         p[2 * q + 1] = __fmul2_rn(p[2 * q + 1], make_float2(l.z, l.w));
       }
     }
-    fwht_pairs<kD, 1>(p, 0);
+    fwht_pairs<kD, 1, HF>(p, 0);
     if (lane == 0) bulk_wait_read0();   // the previous tile's stores have read the staging tile
     __syncwarp();
 #pragma unroll
