@@ -38,10 +38,12 @@
  *
  * Memory: every pointer is DEVICE memory owned by the caller.  The library
  * allocates nothing, keeps no state between calls except a per-device cache
- * of launch limits and one per-device fault word (below), and never
- * synchronises.  Calls are asynchronous on `stream` (a cudaStream_t; NULL
- * means the legacy default stream) and launch on the calling thread's
- * current device, which must own the buffers and the stream.
+ * of launch limits, one per-device fault word (below) and the static 8 MiB
+ * scratch array of kvq_attention_decode_static (one per device, shared by
+ * every call of that entry point; see there), and never synchronises.
+ * Calls are asynchronous on `stream` (a cudaStream_t; NULL means the legacy
+ * default stream) and launch on the calling thread's current device, which
+ * must own the buffers and the stream.
  *
  * Errors: a failed precondition returns a negative kvq_status before any
  * launch, and nothing is written.  A launch failure returns
@@ -252,13 +254,20 @@ int64_t kvq_attention_workspace_bytes(int B, int Hq, int Hkv, int T, int D, int 
 /*
  * kvq_attention_decode_static -- kvq_attention_decode without a caller
  * workspace and without any allocation: the key-split scratch is a static
- * 8 MiB device array inside the library (one per device, its address looked
- * up once).  The pages have no counterpart of this entry point; it exists for
- * callers that cannot hand out device memory.  Same arguments, results and
- * checks as kvq_attention_decode; returns KVQ_ERR_COUNT when the shapes need
- * more split scratch than 8 MiB (kvq_attention_workspace_bytes() > 8 MiB).
- * Calls that overlap in time share the scratch and race: serialise them (one
- * stream, or events between streams and host threads).
+ * 8 MiB device array inside the library (one per device, held by every GPU
+ * that loads the library until the process exits).  The pages have no
+ * counterpart of this entry point; it exists for callers that cannot hand out
+ * device memory (a caller inside a stream capture or a callback that may not
+ * allocate, or one whose allocator is owned by a host framework).  Same
+ * arguments, results and checks as kvq_attention_decode; returns
+ * KVQ_ERR_COUNT when the shapes need more split scratch than 8 MiB
+ * (kvq_attention_workspace_bytes() > 8 MiB).  The first call on a device that
+ * needs the scratch looks its device address up (cudaGetSymbolAddress, with
+ * that device current) and caches it: make that first call before any stream
+ * capture, and do not use the entry point across a cudaDeviceReset, which
+ * invalidates the cached address.  Calls that overlap in time share the
+ * scratch and race: serialise them (one stream, or events between streams and
+ * host threads).
  */
 int kvq_attention_decode_static(const uint16_t *q, const uint8_t *k_packed,
                                 const uint16_t *k_scales, const uint8_t *v_packed,
@@ -289,6 +298,18 @@ int kvq_fault_status(int clear);
  * Returns KVQ_OK or KVQ_ERR_LAUNCH.
  */
 int kvq_selftest_wait_timeout(uint32_t limit, void *stream);
+
+/*
+ * kvq_selftest_rcp_f16 -- writes the reciprocal the quantisers use for a group
+ * scale S (r = 1/S, an approximate reciprocal refined by one Newton step) for
+ * every positive finite fp16 value: out[i] = r(S) for the fp16 S whose bit
+ * pattern is i + 1, i = 0 .. 31742.  It exists so that a test can check that r
+ * is the IEEE fp32 quotient 1/S for every scale the codec can store.
+ *   out     [out] float32 [31743], device memory, 4-byte aligned.
+ * Returns KVQ_OK, KVQ_ERR_NULL, KVQ_ERR_ALIGN or KVQ_ERR_LAUNCH; asynchronous
+ * on `stream`.
+ */
+int kvq_selftest_rcp_f16(float *out, void *stream);
 
 /* Human-readable name of a kvq_status value (static storage). */
 const char *kvq_status_string(int status);

@@ -471,6 +471,7 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
     const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_kvq_fault, 1u);
+      mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);   // the stage that gave up, once more
       if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
       if (STG && lane == 0) bulk_wait0();
       return;
@@ -625,6 +626,7 @@ kvq_dequantize_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* 
     const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_kvq_fault, 1u);
+      mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);   // the stage that gave up, once more
       if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
       if (lane == 0) bulk_wait0();
       return;
@@ -744,6 +746,7 @@ kvq_roundtrip_kernel(const __grid_constant__ RowMaps in_maps, const __grid_const
     const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_kvq_fault, 1u);
+      mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);   // the stage that gave up, once more
       // only the first iteration has the other stage's copy in flight
       if (k == 0 && tq[1] >= 0) mbar_wait(&bar[1], 0, kSpinLimit);
       if (lane == 0) bulk_wait0();
@@ -813,6 +816,16 @@ __global__ void kvq_wait_timeout_kernel(uint32_t limit) {
   __syncthreads();
   const bool ok = mbar_wait(&bar, 0, limit);
   if (__syncthreads_or(!ok) && threadIdx.x == 0) atomicOr(&g_kvq_fault, 2u);
+}
+
+// The kernels' reciprocal of a group scale, rcp_f16val, evaluated at every
+// positive finite fp16 value (bit patterns 0x0001 .. 0x7BFF): out[i] is the
+// reciprocal of the fp16 value with bits i + 1, for the host to compare with
+// the IEEE quotient.
+constexpr int kRcpCount = 0x7BFF;
+__global__ void kvq_rcp_table_kernel(float* __restrict__ out) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < kRcpCount) out[i] = rcp_f16val(half_bits_to_float(static_cast<uint16_t>(i + 1)));
 }
 
 // ---------------------------------------------------------------------------
@@ -1158,6 +1171,14 @@ int kvq_fault_status(int clear) {
 int kvq_selftest_wait_timeout(uint32_t limit, void* stream) {
   (void)cudaGetLastError();
   kvq_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit);
+  return finish_launch();
+}
+
+int kvq_selftest_rcp_f16(float* out, void* stream) {
+  if (out == nullptr) return KVQ_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(out) & 3) != 0) return KVQ_ERR_ALIGN;
+  (void)cudaGetLastError();
+  kvq_rcp_table_kernel<<<(kRcpCount + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(out);
   return finish_launch();
 }
 

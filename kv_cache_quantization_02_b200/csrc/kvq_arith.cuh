@@ -53,8 +53,8 @@ __device__ __forceinline__ float div7_rn(float a) { return div_const_rn<7>(a); }
 // fp32 reciprocal of a positive fp16 value s, correctly rounded: approximate
 // reciprocal plus one Newton-Raphson step.  1/s lies at least 2^-35 (relative)
 // away from every rounding midpoint because s has an 11-bit significand, far
-// beyond the step's error; checked against IEEE 1/s for every positive
-// finite fp16 s.
+// beyond the step's error.  kvq_selftest_rcp_f16 evaluates it at every
+// positive finite fp16 s so that a test can compare it with IEEE 1/s.
 __device__ __forceinline__ float rcp_f16val(float s) {
   float r0;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(s));

@@ -417,13 +417,17 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     __syncwarp();                      // the stage is consumed: refill it
     issue(blk + kAStages * kAW, stage);
   }
+  bool lost = false;                   // a copy may still land in this warp's ring
   if (failed) {
     if (lane == 0) atomicOr(&g_attn_fault, 1u);
-    // drain whatever this warp still has in flight before the ring is reused
-    for (int s = 1; s < kAStages; ++s) {
+    // drain whatever this warp still has in flight, the stage that gave up
+    // included, before the ring is reused
+    for (int s = 0; s < kAStages; ++s) {
       const int kk2 = k + s;
-      if (warp + kk2 * kAW < nblk) mbar_wait(&bar[kk2 % kAStages], (kk2 / kAStages) & 1, kSpin);
+      if (warp + kk2 * kAW < nblk && !mbar_wait(&bar[kk2 % kAStages], (kk2 / kAStages) & 1, kSpin))
+        lost = true;
     }
+    lost = __any_sync(kFull, lost);
   }
   l += __shfl_xor_sync(kFull, l, 1);
   l += __shfl_xor_sync(kFull, l, 2);
@@ -432,7 +436,9 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     psum[gi] += __shfl_xor_sync(kFull, psum[gi], 1);
     psum[gi] += __shfl_xor_sync(kFull, psum[gi], 2);
   }
-  __syncthreads();                     // every warp is out of the ring: reuse it for the merge
+  // every warp is out of the ring: reuse it for the merge, unless a copy may
+  // still land there (the fault word is set; the block writes nothing)
+  if (__syncthreads_or(lost)) return;
   if (g < R) {
     float* cw = comb + (warp * kMaxRows + g) * D;
 #pragma unroll
@@ -588,8 +594,12 @@ __attribute__((visibility("hidden"))) unsigned int kvq_attn_fault_word(int clear
 }
 __attribute__((visibility("hidden"))) int kvq_attn_last_cuda_error() { return g_attn_cuda_error; }
 
-// Device address of the static scratch, looked up once per device.
-void* static_scratch(int& rc) {
+// Device address of the static scratch, looked up once per device (on the
+// first kvq_attention_decode_static call that needs it on that device) and
+// kept for the life of the process: a cudaDeviceReset rebuilds the module and
+// leaves the cached address stale, so the entry point is not for use across
+// a device reset.  Internal linkage: the library exports only its C ABI.
+static void* static_scratch(int& rc) {
   static std::atomic<void*> cache[64];
   int dev = 0;
   rc = KVQ_OK;

@@ -186,6 +186,7 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
     const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_ex_fault, 1u);
+      mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);   // the stage that gave up, once more
       // only the first tile has the other stage's copy in flight
       if (k == 0 && tq[1] >= 0) mbar_wait(&bar[1], 0, kSpinX);
       if (lane == 0) bulk_wait0();
@@ -415,6 +416,7 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
     const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_ex_fault, 1u);
+      mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);   // the stage that gave up, once more
       if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinX);
       if (lane == 0) bulk_wait0();
       return;
@@ -747,6 +749,7 @@ kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
     const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_ex_fault, 1u);
+      mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);   // the stage that gave up, once more
       // only the first tile has the other stage's copy in flight
       if (k == 0 && tq[1] >= 0) mbar_wait(&bar[1], 0, kSpinX);
       if (lane == 0) bulk_wait0();
@@ -922,6 +925,7 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const __grid_const
     const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);
     if (__any_sync(kFullMask, !ok)) {
       if (lane == 0) atomicOr(&g_ex_fault, 1u);
+      mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);   // the stage that gave up, once more
       if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinX);
       if (lane == 0) bulk_wait0();
       return;

@@ -64,6 +64,8 @@ _lib.kvq_fault_status.restype = _I
 _lib.kvq_fault_status.argtypes = [_I]
 _lib.kvq_selftest_wait_timeout.restype = _I
 _lib.kvq_selftest_wait_timeout.argtypes = [ctypes.c_uint32, _P]
+_lib.kvq_selftest_rcp_f16.restype = _I
+_lib.kvq_selftest_rcp_f16.argtypes = [_P, _P]
 
 KVQ_OK = 0
 KVQ_ERR_NULL = -1
@@ -170,6 +172,10 @@ def kvq_fault_status(clear: bool = False) -> int:
 
 def kvq_selftest_wait_timeout(limit: int, stream: int = 0) -> int:
     return _lib.kvq_selftest_wait_timeout(limit, stream)
+
+
+def kvq_selftest_rcp_f16(out: int, stream: int = 0) -> int:
+    return _lib.kvq_selftest_rcp_f16(out, stream)
 
 
 # ---- torch-tensor convenience --------------------------------------------
