@@ -83,8 +83,10 @@ class Oracle:
             "kvqo_unpack": (None, [_P, _I64, _P]),
             "kvqo_quantize_ex": (_I, [_P, _P, _P, _I64, _I, _I, _I, _I, _I64, _I, _P, _P]),
             "kvqo_dequantize_ex": (_I, [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _I64, _I, _P]),
-            "kvqo_srft_f32": (None, [_P, _I, _P]),
-            "kvqo_isrft_f32": (None, [_P, _I, _P]),
+            "kvqo_srft_f32": (_I, [_P, _I, _P]),
+            "kvqo_isrft_f32": (_I, [_P, _I, _P]),
+            "kvqo_twiddle": (None, [_I, _I, _P, _P]),
+            "kvqo_fft_f32": (_I, [_P, _P, _I, _I]),
             "kvqo_srft_f64": (None, [_P, _I, _P]),
             "kvqo_isrft_f64": (None, [_P, _I, _P]),
             "kvqo_attention_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -216,19 +218,37 @@ class Oracle:
         return out
 
 
+    def twiddle(self, k: int, M: int) -> tuple[np.float32, np.float32]:
+        """The oracle's fp32 omega_M^k = (cos, -sin)(2 pi k / M)."""
+        wr, wi = ctypes.c_float(), ctypes.c_float()
+        self._lib.kvqo_twiddle(k, M, ctypes.byref(wr), ctypes.byref(wi))
+        return np.float32(wr.value), np.float32(wi.value)
+
+    def fft_f32(self, z, inverse: bool = False) -> np.ndarray:
+        """The oracle's fp32 complex FFT of rows z [n, N] (forward DIF stages,
+        or with inverse=True their transpose: the unnormalised conjugate DFT)."""
+        z = np.atleast_2d(np.asarray(z, dtype=np.complex64))
+        out = np.empty_like(z)
+        for r in range(z.shape[0]):
+            re = np.ascontiguousarray(z[r].real, dtype=np.float32)
+            im = np.ascontiguousarray(z[r].imag, dtype=np.float32)
+            _check(self._lib.kvqo_fft_f32(_ptr(re), _ptr(im), z.shape[1], 1 if inverse else 0))
+            out[r] = re + 1j * im
+        return out
+
     def srft_f32(self, v) -> np.ndarray:
         """fp32 SRFT (packed unitary real DFT) of rows v [n, D]."""
         v = np.ascontiguousarray(np.atleast_2d(v), dtype=np.float32)
         out = np.empty_like(v)
         for r in range(v.shape[0]):
-            self._lib.kvqo_srft_f32(_ptr(v[r]), v.shape[1], _ptr(out[r]))
+            _check(self._lib.kvqo_srft_f32(_ptr(v[r]), v.shape[1], _ptr(out[r])))
         return out
 
     def isrft_f32(self, y) -> np.ndarray:
         y = np.ascontiguousarray(np.atleast_2d(y), dtype=np.float32)
         out = np.empty_like(y)
         for r in range(y.shape[0]):
-            self._lib.kvqo_isrft_f32(_ptr(y[r]), y.shape[1], _ptr(out[r]))
+            _check(self._lib.kvqo_isrft_f32(_ptr(y[r]), y.shape[1], _ptr(out[r])))
         return out
 
     def srft_f64(self, v) -> np.ndarray:

@@ -465,128 +465,268 @@ int kvqo_attention_decode(const uint16_t *q, const uint8_t *k_packed,
 
 /* ------------------------------------------------------------------ */
 /* The SRFT rotation: SRFT(x) = pack(F diag(s) x), F the unitary DFT    */
-/* of length D ([P5] Methodologie 1), computed as in the paper's        */
-/* kernel ([P5] Methodologie 2): a length-N = D/2 complex FFT of        */
-/* z_n = v_2n + i v_2n+1 in log2(N) radix-2 Stockham stages, then the   */
-/* Hermitian unpacking to a real representation.  The packing read     */
+/* of length D ([P5] Methodologie 1), computed as the paper's kernel    */
+/* does ([P5] Methodologie 2): the length-N = D/2 complex FFT of        */
+/* z_n = v_2n + i v_2n+1 in Stockham stages, then the Hermitian         */
+/* unpacking to a real representation.  [P3] picks the SRFT for mixed  */
+/* radix, so N is a power of two (log2 N radix-2 stages) or three times */
+/* one (radix-2 stages, then one radix-3 stage).  The packing read      */
 /* here (orthonormal, so the inverse is the transpose):                 */
 /*   y0 = X_0 / sqrt(D),  y1 = X_N / sqrt(D),                            */
-/*   y_2k = sqrt(2) Re X_k / sqrt(D),  y_2k+1 = sqrt(2) Im X_k / sqrt(D), */
-/*   k = 1 .. N-1, X = DFT(v).                                          */
-/* Twiddles are cos / sin in double, rounded to fp32; every complex     */
-/* product is four fp32 products and two fp32 sums in the order below.  */
+/*   (y_2k, y_2k+1) = sqrt(2) (Re, Im) X_k / sqrt(D),  k = 1 .. N-1,     */
+/* X = DFT(v).  Readings of the arithmetic:                             */
+/*  - twiddles are the fp32 values nearest the exact roots of unity;    */
+/*    a product by 1, -1, i or -i is exact (the operand, negated or     */
+/*    with its parts swapped); any other complex product is four fp32   */
+/*    products and two fp32 sums, re = dr wr - di wi, im = dr wi + di wr;*/
+/*  - the unpacking forms 2 X_k (its factor 1/2 goes into the           */
+/*    normalisation), scaled by fp32(1/sqrt(2D)); X_0 and X_N are       */
+/*    scaled by fp32(1/sqrt(D));                                        */
+/*  - the inverse is the transpose of the forward, step by step in      */
+/*    reverse order: the scaling, the adjoint of the unpacking, then    */
+/*    the adjoint (decimation-in-time) Stockham stages with conjugate   */
+/*    twiddles.                                                         */
 /* ------------------------------------------------------------------ */
 
-/* omega_M^k = (cos(2 pi k / M), -sin(2 pi k / M)) rounded to fp32. */
-static void twiddle(int k, int M, float *wr, float *wi)
+/* omega_M^k = (cos(2 pi k / M), -sin(2 pi k / M)) as the fp32 values
+ * nearest the exact ones.  The angle is reduced by exact symmetries to a
+ * base angle (pi/2) r / M with 0 <= r <= M/2 (at most pi/4), whose cosine
+ * and sine are taken in double and rounded once; quadrant and complement
+ * are exact swaps and negations.  So omega^0 = 1, omega^(M/4) = -i and
+ * omega^(M/2) = -1 exactly, the table keeps every symmetry of the exact
+ * roots, and its zero parts are +0. */
+void kvqo_twiddle(int k, int M, float *wr, float *wi)
 {
-    const double a = 2.0 * 3.14159265358979323846 * (double)k / (double)M;
-    *wr = (float)cos(a);
-    *wi = (float)(-sin(a));
+    long j = ((long)k % M + M) % M;
+    long q = (4 * j) / M;                       /* quadrant */
+    long r = 4 * j - q * M;                     /* angle = q pi/2 + (pi/2) r / M */
+    int comp = 2 * r > M;
+    if (comp) r = M - r;
+    double a = 1.57079632679489661923 * (double)r / (double)M;
+    float c = (float)cos(a), s = (float)sin(a);
+    if (comp) { float t = c; c = s; s = t; }    /* cos, sin of (pi/2) r_0 / M */
+    float cr, sn;                               /* cos, sin of the whole angle */
+    switch (q) {
+    case 0: cr = c; sn = s; break;
+    case 1: cr = -s; sn = c; break;
+    case 2: cr = -c; sn = -s; break;
+    default: cr = s; sn = -c; break;
+    }
+    *wr = cr + 0.0f;                            /* -0 -> +0 */
+    *wi = -sn + 0.0f;
 }
 
-/* Stockham radix-2 FFT of length N (a power of two), unnormalised, in
- * place through a scratch copy.  sign = -1: forward (omega), +1: inverse
- * (conjugate twiddles).  Stage: n = N, N/2, ..., 2 with stride s = N / n:
- *   a = x[q + s p], b = x[q + s (p + n/2)],
- *   y[q + s 2p] = a + b,  y[q + s (2p + 1)] = (a - b) * omega_n^p. */
-static void stockham(float *re, float *im, int N, int sign)
+/* d * w for a table twiddle w (readings above). */
+static void cmul(float dr, float di, float wr, float wi, float *pr, float *pi_)
 {
-    float tr[KVQO_DMAX / 2], ti[KVQO_DMAX / 2];
-    float *xr = re, *xi = im, *yr = tr, *yi = ti;
-    int s = 1;
-    for (int n = N; n > 1; n >>= 1) {
-        int m = n / 2;
-        for (int p = 0; p < m; ++p) {
-            float wr, wi;
-            twiddle(p * s, N, &wr, &wi);      /* omega_n^p = omega_N^(p s) */
-            if (sign > 0) wi = -wi;
-            for (int q = 0; q < s; ++q) {
-                float ar = xr[q + s * p], ai = xi[q + s * p];
-                float br = xr[q + s * (p + m)], bi = xi[q + s * (p + m)];
-                yr[q + s * 2 * p] = ar + br;
-                yi[q + s * 2 * p] = ai + bi;
-                float dr = ar - br, di = ai - bi;
-                float pr = dr * wr, pi_ = di * wi, qr = dr * wi, qi = di * wr;
-                yr[q + s * (2 * p + 1)] = pr - pi_;
-                yi[q + s * (2 * p + 1)] = qr + qi;
+    if (wi == 0.0f && fabsf(wr) == 1.0f) {              /* w = +-1 */
+        *pr = (wr > 0.0f) ? dr : -dr;
+        *pi_ = (wr > 0.0f) ? di : -di;
+    } else if (wr == 0.0f && fabsf(wi) == 1.0f) {       /* w = +-i: (dr + i di)(i wi) */
+        *pr = (wi > 0.0f) ? -di : di;
+        *pi_ = (wi > 0.0f) ? dr : -dr;
+    } else {
+        float a = dr * wr, b = di * wi, c = dr * wi, e = di * wr;
+        *pr = a - b;
+        *pi_ = c + e;
+    }
+}
+
+/* Radices of a length-N transform, first stage first: 2 while the remaining
+ * length is even, then 3 if it is 3.  Returns the number of stages, or -1
+ * for another N. */
+static int fft_radices(int N, int *rad)
+{
+    int n = N, ns = 0;
+    if (N < 1) return -1;
+    while (n % 2 == 0) { rad[ns++] = 2; n /= 2; }
+    if (n == 3) { rad[ns++] = 3; n = 1; }
+    return n == 1 ? ns : -1;
+}
+
+/* One forward (decimation-in-frequency) Stockham stage of radix r on
+ * sub-transforms of length n, stride s = N / n, m = n / r:
+ *   a_j = x[q + s (p + j m)],  j < r,
+ *   y[q + s (r p + t)] = (a_0 + omega_r^t a_1 + ... ) omega_n^(p t),
+ * the sum taken left to right over j.  At r = 2 that is a + b and
+ * (a - b) omega_n^p. */
+static void dif_stage(const float *xr, const float *xi, float *yr, float *yi,
+                      int N, int n, int r)
+{
+    int s = N / n, m = n / r;
+    for (int p = 0; p < m; ++p)
+        for (int q = 0; q < s; ++q)
+            for (int t = 0; t < r; ++t) {
+                float br = xr[q + s * p], bi = xi[q + s * p];
+                for (int j = 1; j < r; ++j) {
+                    float wr, wi, tr, ti;
+                    kvqo_twiddle((N / r) * j * t, N, &wr, &wi);     /* omega_r^(j t) */
+                    cmul(xr[q + s * (p + j * m)], xi[q + s * (p + j * m)], wr, wi, &tr, &ti);
+                    br = br + tr;
+                    bi = bi + ti;
+                }
+                float wr, wi;
+                kvqo_twiddle(s * p * t, N, &wr, &wi);               /* omega_n^(p t) */
+                cmul(br, bi, wr, wi, &yr[q + s * (r * p + t)], &yi[q + s * (r * p + t)]);
+            }
+}
+
+/* The transpose of dif_stage: c_t = y[q + s (r p + t)] conj(omega_n^(p t)),
+ * x[q + s (p + j m)] = c_0 + conj(omega_r^j) c_1 + ..., left to right over
+ * t.  At r = 2 that is x = c_0 + c_1 and c_0 - c_1 with
+ * c_1 = y_odd conj(omega_n^p). */
+static void dit_stage(const float *yr, const float *yi, float *xr, float *xi,
+                      int N, int n, int r)
+{
+    int s = N / n, m = n / r;
+    for (int p = 0; p < m; ++p)
+        for (int q = 0; q < s; ++q) {
+            float cr[3], ci[3];
+            for (int t = 0; t < r; ++t) {
+                float wr, wi;
+                kvqo_twiddle(s * p * t, N, &wr, &wi);
+                cmul(yr[q + s * (r * p + t)], yi[q + s * (r * p + t)], wr, -wi, &cr[t], &ci[t]);
+            }
+            for (int j = 0; j < r; ++j) {
+                float ar = cr[0], ai = ci[0];
+                for (int t = 1; t < r; ++t) {
+                    float wr, wi, tr, ti;
+                    kvqo_twiddle((N / r) * j * t, N, &wr, &wi);
+                    cmul(cr[t], ci[t], wr, -wi, &tr, &ti);
+                    ar = ar + tr;
+                    ai = ai + ti;
+                }
+                xr[q + s * (p + j * m)] = ar;
+                xi[q + s * (p + j * m)] = ai;
             }
         }
+}
+
+/* Length-N complex FFT in place (through a scratch copy), N a power of two
+ * or three times one.  inverse = 0: the forward DIF stages (the unnormalised
+ * DFT X_k = sum_n z_n omega_N^(n k)); inverse = 1: its transpose, the
+ * adjoint stages in reverse order (the unnormalised conjugate DFT).
+ * Returns 0, or -3 for an unsupported N. */
+int kvqo_fft_f32(float *re, float *im, int N, int inverse)
+{
+    int rad[32], len[33];
+    int ns = fft_radices(N, rad);
+    if (ns < 0 || N > KVQO_DMAX / 2) return -3;
+    len[0] = N;
+    for (int i = 0; i < ns; ++i) len[i + 1] = len[i] / rad[i];
+    float tr[KVQO_DMAX / 2], ti[KVQO_DMAX / 2];
+    float *xr = re, *xi = im, *yr = tr, *yi = ti;
+    for (int i = 0; i < ns; ++i) {
+        int st = inverse ? ns - 1 - i : i;
+        if (inverse)
+            dit_stage(xr, xi, yr, yi, N, len[st], rad[st]);
+        else
+            dif_stage(xr, xi, yr, yi, N, len[st], rad[st]);
         float *t;
         t = xr; xr = yr; yr = t;
         t = xi; xi = yi; yi = t;
-        s *= 2;
     }
     if (xr != re) {
         for (int i = 0; i < N; ++i) { re[i] = xr[i]; im[i] = xi[i]; }
     }
+    return 0;
 }
 
-/* One spectrum bin of the real input from the half-length spectrum:
- * X_k = E_k + omega_D^k O_k, E_k = (Z_k + conj Z_(N-k)) / 2,
- * O_k = (Z_k - conj Z_(N-k)) / 2i   (indices mod N). */
-static void real_bin(const float *zr, const float *zi, int N, int k,
-                     float *xr, float *xi)
+/* 2 X_k of the real input from its half-length spectrum Z, k = 1 .. N-1:
+ * A = Z_k, B = conj Z_(N-k), E = A + B, O = (A - B) / i (exact),
+ * 2 X_k = E + omega_D^k O. */
+static void real_bin2(const float *zr, const float *zi, int N, int k,
+                      float *xr, float *xi)
 {
-    int a = k % N, b = (N - k) % N;
-    float Ar = zr[a], Ai = zi[a], Br = zr[b], Bi = -zi[b];
-    float Er = (Ar + Br) * 0.5f, Ei = (Ai + Bi) * 0.5f;
+    float Ar = zr[k], Ai = zi[k], Br = zr[N - k], Bi = -zi[N - k];
+    float Er = Ar + Br, Ei = Ai + Bi;
     float Dr = Ar - Br, Di = Ai - Bi;
-    float Or = Di * 0.5f, Oi = -(Dr * 0.5f);
-    float wr, wi;
-    twiddle(k, 2 * N, &wr, &wi);
-    float Tr = Or * wr - Oi * wi, Ti = Or * wi + Oi * wr;
+    float Or = Di, Oi = -Dr;
+    float wr, wi, Tr, Ti;
+    kvqo_twiddle(k, 2 * N, &wr, &wi);
+    cmul(Or, Oi, wr, wi, &Tr, &Ti);
     *xr = Er + Tr;
     *xi = Ei + Ti;
 }
 
-/* fp32 forward SRFT of one sign-flipped (and scaled) row v[D] -> y[D]. */
-void kvqo_srft_f32(const float *v, int D, float *y)
+/* Is D an SRFT length: even, D/2 a power of two or three times one. */
+static int srft_len_ok(int D)
+{
+    int rad[32];
+    return D >= 2 && D % 2 == 0 && D <= KVQO_DMAX && fft_radices(D / 2, rad) >= 0;
+}
+
+/* Normalisation of packed position i: fp32(1/sqrt(D)) on y0, y1 (X_0, X_N),
+ * fp32(1/sqrt(2D)) on the rest (which hold 2 Re X_k, 2 Im X_k). */
+static float srft_norm(int i, int D)
+{
+    return (i < 2) ? (float)(1.0 / sqrt((double)D)) : (float)(1.0 / sqrt(2.0 * (double)D));
+}
+
+/* Forward SRFT of one sign-flipped row v[D] with per-position factors f:
+ * y0 = (Z0.re + Z0.im) f0, y1 = (Z0.re - Z0.im) f1, (y_2k, y_2k+1) =
+ * 2 X_k . (f_2k, f_2k+1). */
+static void srft_scaled(const float *v, int D, const float *f, float *y)
 {
     int N = D / 2;
     float zr[KVQO_DMAX / 2], zi[KVQO_DMAX / 2];
     for (int n = 0; n < N; ++n) { zr[n] = v[2 * n]; zi[n] = v[2 * n + 1]; }
-    stockham(zr, zi, N, -1);
-    const float c0 = (float)(1.0 / sqrt((double)D));
-    const float c1 = (float)(sqrt(2.0 / (double)D));
-    float xr, xi;
-    real_bin(zr, zi, N, 0, &xr, &xi);
-    y[0] = xr * c0;
-    real_bin(zr, zi, N, N, &xr, &xi);
-    y[1] = xr * c0;
+    kvqo_fft_f32(zr, zi, N, 0);
+    y[0] = (zr[0] + zi[0]) * f[0];
+    y[1] = (zr[0] - zi[0]) * f[1];
     for (int k = 1; k < N; ++k) {
-        real_bin(zr, zi, N, k, &xr, &xi);
-        y[2 * k] = xr * c1;
-        y[2 * k + 1] = xi * c1;
+        float xr, xi;
+        real_bin2(zr, zi, N, k, &xr, &xi);
+        y[2 * k] = xr * f[2 * k];
+        y[2 * k + 1] = xi * f[2 * k + 1];
     }
 }
 
-/* fp32 inverse SRFT (the transpose): y[D] -> v[D] = P^T y. */
-void kvqo_isrft_f32(const float *y, int D, float *v)
+/* Transpose of srft_scaled: U_i = y_i f_i; the adjoint of the unpacking,
+ * z_0 = (U_0 + U_1, U_0 - U_1) and, k = 1 .. N-1, A = U_k, B = conj U_(N-k),
+ * E = A + B, T = (A - B) conj(omega_D^k), Z_k = E + i T; then the
+ * transposed FFT. */
+static void isrft_scaled(const float *y, int D, const float *f, float *v)
 {
     int N = D / 2;
-    const float c0 = (float)(1.0 / sqrt((double)D));
-    const float c1 = (float)(sqrt(2.0 / (double)D));
-    /* U_0 = 2 c0 y0, U_N = 2 c0 y1, U_k = c1 (y_2k + i y_2k+1) */
-    float Ur[KVQO_DMAX / 2 + 1], Ui[KVQO_DMAX / 2 + 1];
-    Ur[0] = (y[0] * c0) * 2.0f; Ui[0] = 0.0f;
-    Ur[N] = (y[1] * c0) * 2.0f; Ui[N] = 0.0f;
-    for (int k = 1; k < N; ++k) { Ur[k] = y[2 * k] * c1; Ui[k] = y[2 * k + 1] * c1; }
     float zr[KVQO_DMAX / 2], zi[KVQO_DMAX / 2];
-    for (int k = 0; k < N; ++k) {
-        float Ar = Ur[k], Ai = Ui[k], Br = Ur[N - k], Bi = -Ui[N - k];
-        float Er = (Ar + Br) * 0.5f, Ei = (Ai + Bi) * 0.5f;
+    float u0 = y[0] * f[0], un = y[1] * f[1];
+    zr[0] = u0 + un;
+    zi[0] = u0 - un;
+    for (int k = 1; k < N; ++k) {
+        float Ar = y[2 * k] * f[2 * k], Ai = y[2 * k + 1] * f[2 * k + 1];
+        float Br = y[2 * (N - k)] * f[2 * (N - k)];
+        float Bi = -(y[2 * (N - k) + 1] * f[2 * (N - k) + 1]);
+        float Er = Ar + Br, Ei = Ai + Bi;
         float Dr = Ar - Br, Di = Ai - Bi;
-        float wr, wi;
-        twiddle(k, D, &wr, &wi);
-        wi = -wi;                                         /* conj(omega_D^k) */
-        float Tr = Dr * wr - Di * wi, Ti = Dr * wi + Di * wr;
-        float Or = Tr * 0.5f, Oi = Ti * 0.5f;
-        zr[k] = Er - Oi;                                  /* E + i O */
-        zi[k] = Ei + Or;
+        float wr, wi, Tr, Ti;
+        kvqo_twiddle(k, D, &wr, &wi);
+        cmul(Dr, Di, wr, -wi, &Tr, &Ti);                 /* conj(omega_D^k) */
+        zr[k] = Er - Ti;                                  /* E + i T */
+        zi[k] = Ei + Tr;
     }
-    stockham(zr, zi, N, +1);
+    kvqo_fft_f32(zr, zi, N, 1);
     for (int n = 0; n < N; ++n) { v[2 * n] = zr[n]; v[2 * n + 1] = zi[n]; }
+}
+
+/* fp32 SRFT of one sign-flipped row v[D] -> y[D] (normalised). */
+int kvqo_srft_f32(const float *v, int D, float *y)
+{
+    float f[KVQO_DMAX];
+    if (!srft_len_ok(D)) return -3;
+    for (int i = 0; i < D; ++i) f[i] = srft_norm(i, D);
+    srft_scaled(v, D, f, y);
+    return 0;
+}
+
+/* fp32 inverse SRFT (the transpose): y[D] -> v[D] = P^T y. */
+int kvqo_isrft_f32(const float *y, int D, float *v)
+{
+    float f[KVQO_DMAX];
+    if (!srft_len_ok(D)) return -3;
+    for (int i = 0; i < D; ++i) f[i] = srft_norm(i, D);
+    isrft_scaled(y, D, f, v);
+    return 0;
 }
 
 /* Definitions in double, for the pins: the packed unitary DFT and its
@@ -635,14 +775,22 @@ void kvqo_isrft_f64(const double *y, int D, double *v)
 /*           complement byte per code;                                  */
 /*   row r uses lambda table (r / lambda_rows) % n_lambda, a table      */
 /*   being D floats (per-(layer, head) smoothing).                      */
-/* The inverse mirrors each order: lambda before -> dequantize_row;     */
-/* lambda after -> w = (q S) * (1/lambda), transform, * c, * s.         */
+/* With lambda after the rotation, the rescale after the transform is   */
+/* the only scaling step ([P5] Methodologie 2 lists no other): channel  */
+/* i is multiplied by fp32(lambda_i c_i), c_i the normalisation of that */
+/* position (1/sqrt(D), or the SRFT's), one product per channel; the    */
+/* inverse multiplies q S by fp32(c_i / lambda_i) before its transform  */
+/* and applies the signs last.  With lambda before it the transform is  */
+/* followed by c_i, and the inverse mirrors that (c_i, transform, signs,*/
+/* 1/lambda).                                                            */
 /* ------------------------------------------------------------------ */
 
-static int check_ex(int D, int G, int bits, int64_t lambda_rows, int n_lambda)
+/* D a power of two in [2, KVQO_DMAX] (an SRFT length with the SRFT),
+ * G a power of two with 2 <= G <= D dividing D.  Returns 0 if valid. */
+static int check_ex(int D, int G, int bits, int64_t lambda_rows, int n_lambda, int srft)
 {
-    int rc = check_shape(D, G);
-    if (rc) return rc;
+    if (srft ? !srft_len_ok(D) : (!is_pow2(D) || D < 2 || D > KVQO_DMAX)) return -3;
+    if (!is_pow2(G) || G < 2 || G > D || D % G != 0) return -4;
     if (bits != 4 && bits != 8) return -4;
     if (lambda_rows < 1 || n_lambda < 1) return -5;
     return 0;
@@ -654,13 +802,19 @@ static const float *table_of(const float *lam, int64_t r, int64_t lambda_rows,
     return lam + ((r / lambda_rows) % n_lambda) * (int64_t)D;
 }
 
+/* Normalisation of position i of a rotated row. */
+static float norm_of(int i, int D, int srft)
+{
+    return srft ? srft_norm(i, D) : kvqo_norm_const(D);
+}
+
 int kvqo_quantize_ex(const uint16_t *x, const float *lam, const int8_t *s,
                      int64_t n, int D, int G, int bits, int flags,
                      int64_t lambda_rows, int n_lambda, uint8_t *codes,
                      uint16_t *scales)
 {
     const int lambda_after = flags & 1, srft = (flags >> 1) & 1;
-    int rc = check_ex(D, G, bits, lambda_rows, n_lambda);
+    int rc = check_ex(D, G, bits, lambda_rows, n_lambda, srft);
     if (rc) return rc;
     if (n < 0) return -5;
     float c = kvqo_norm_const(D);
@@ -675,20 +829,20 @@ int kvqo_quantize_ex(const uint16_t *x, const float *lam, const int8_t *s,
         if (!lambda_after && !srft) {
             rotate_row_f32(xr, lr, s, D, c, y);
         } else {
-            float v[KVQO_DMAX];
+            float v[KVQO_DMAX], f[KVQO_DMAX];
             for (int i = 0; i < D; ++i) {
                 float t = kvqo_f16_to_f32(xr[i]);
                 if (!lambda_after) t = t * lr[i];              /* lambda */
                 v[i] = (s[i] < 0) ? -t : t;                    /* exact  */
+                f[i] = lambda_after ? lr[i] * norm_of(i, D, srft)   /* lambda c_i */
+                                    : norm_of(i, D, srft);
             }
             if (srft) {
-                kvqo_srft_f32(v, D, y);
+                srft_scaled(v, D, f, y);
             } else {
                 kvqo_fwht_f32(v, D);
-                for (int i = 0; i < D; ++i) y[i] = v[i] * c;
+                for (int i = 0; i < D; ++i) y[i] = v[i] * f[i];
             }
-            if (lambda_after)
-                for (int i = 0; i < D; ++i) y[i] = y[i] * lr[i];   /* lambda */
         }
         uint16_t *sc = scales + r * (D / G);
         for (int j = 0; j < D / G; ++j) {
@@ -725,7 +879,7 @@ int kvqo_dequantize_ex(const uint8_t *codes, const uint16_t *scales,
                        int n_lambda, uint16_t *out)
 {
     const int lambda_after = flags & 1, srft = (flags >> 1) & 1;
-    int rc = check_ex(D, G, bits, lambda_rows, n_lambda);
+    int rc = check_ex(D, G, bits, lambda_rows, n_lambda, srft);
     if (rc) return rc;
     if (n < 0) return -5;
     float c = kvqo_norm_const(D);
@@ -743,16 +897,17 @@ int kvqo_dequantize_ex(const uint8_t *codes, const uint16_t *scales,
         if (!lambda_after && !srft) {
             dequantize_row(q, sc, lr, s, D, G, c, w);
         } else {
-            float u[KVQO_DMAX];
+            float u[KVQO_DMAX], f[KVQO_DMAX];
             for (int i = 0; i < D; ++i) {
                 u[i] = (float)q[i] * kvqo_f16_to_f32(sc[i / G]);      /* exact */
-                if (lambda_after) u[i] = u[i] * (1.0f / lr[i]);        /* 1/lambda */
+                f[i] = lambda_after ? norm_of(i, D, srft) / lr[i]     /* c_i / lambda */
+                                    : norm_of(i, D, srft);
             }
             if (srft) {
-                kvqo_isrft_f32(u, D, w);
+                isrft_scaled(u, D, f, w);
             } else {
-                kvqo_fwht_f32(u, D);
-                for (int i = 0; i < D; ++i) w[i] = u[i] * c;
+                for (int i = 0; i < D; ++i) w[i] = u[i] * f[i];
+                kvqo_fwht_f32(w, D);
             }
             for (int i = 0; i < D; ++i) {
                 float z = (s[i] < 0) ? -w[i] : w[i];                   /* exact */
@@ -763,4 +918,3 @@ int kvqo_dequantize_ex(const uint8_t *codes, const uint16_t *scales,
     }
     return 0;
 }
-

@@ -14,7 +14,12 @@ check the oracle against what the pages and the mathematics fix:
   printed compression figure (tests/golden/accounting.json);
 * the SRFT rotation: numpy's rfft (unitary, packed), orthogonality of its
   dense matrix, the fp32 Stockham path within its bound of the float64
-  definition, closed forms, and the codec built on it;
+  definition, closed forms, and the codec built on it, at power-of-two and
+  mixed-radix (three times a power of two) lengths; its twiddle table against
+  the correctly rounded exact roots of unity, computed independently in
+  80-digit decimal arithmetic, and against the exact symmetries of the roots;
+  its complex FFT against numpy's fft, exactly where only the twiddles 1, -1,
+  i, -i occur;
 * format variants (lambda after the rotation, int8 codes, lambda tables):
   the float64 definition with the dense matrix, the int8 code invariants, the
   table indexing, the round-trip bound and the impulse closed form;
@@ -532,7 +537,7 @@ def pin_srft_definition(o):
     """The f64 SRFT equals numpy's rfft packed and scaled; it is orthogonal
     (its dense matrix P has P^T P = I) and the f64 inverse is P^T."""
     rng = np.random.default_rng(41)
-    for D in (4, 8, 32, 128, 256):
+    for D in (4, 8, 12, 24, 32, 96, 128, 192, 256):
         v = rng.standard_normal((5, D))
         assert np.abs(o.srft_f64(v) - _rfft_packed(v)).max() < 1e-12 * math.sqrt(D)
         P = o.srft_f64(np.eye(D)).T                    # column j = P e_j
@@ -546,7 +551,7 @@ def pin_srft_f32(o):
     definition, preserves the norm, and its inverse undoes it."""
     rng = np.random.default_rng(42)
     U = 2.0 ** -24
-    for D in (8, 64, 128, 256):
+    for D in (8, 12, 48, 64, 96, 128, 256):
         v = rng.standard_normal((16, D)).astype(np.float32)
         v[:, 3] *= 30.0
         y32 = o.srft_f32(v).astype(np.float64)
@@ -566,22 +571,23 @@ def pin_srft_closed_forms(o):
     0 elsewhere); an impulse at channel 0 gives y = (1, 1, sqrt2, 0, sqrt2, 0,
     ...) / sqrt(D): codes (5, 5, 7, 0, 7, 0, ...) at int4, (90, 90, 127, 0,
     ...) at int8."""
-    D, G = 32, 8
-    one = np.ones(D, np.float32)
-    s = np.ones(D, np.int8)
-    x = np.full((1, D), 0.5, dtype=np.float16)
-    codes, S = o.quantize_ex(x, one, s, G, srft=True)
-    q = o.unpack(codes)[0]
-    assert q[0] == 7 and np.all(q[1:] == 0)
-    x = np.zeros((1, D), dtype=np.float16)
-    x[0, 0] = 1.0
-    for bits, top, edge in ((4, 7, 5), (8, 127, 90)):
-        codes, S = o.quantize_ex(x, one, s, G, bits=bits, srft=True)
-        q = _codes_ex(o, codes, bits, D)[0]
-        want = np.zeros(D, np.int64)
-        want[0::2] = top
-        want[0] = want[1] = edge
-        assert np.array_equal(q, want), (bits, q)
+    for D, G in ((32, 8), (96, 32)):
+        one = np.ones(D, np.float32)
+        s = np.ones(D, np.int8)
+        x = np.full((1, D), 0.5, dtype=np.float16)
+        codes, S = o.quantize_ex(x, one, s, G, srft=True)
+        q = o.unpack(codes)[0]
+        assert q[0] == 7 and np.all(q[1:] == 0)
+        x = np.zeros((1, D), dtype=np.float16)
+        x[0, 0] = 1.0
+        for bits, top, edge in ((4, 7, 5), (8, 127, 90)):
+            for after in (False, True):
+                codes, S = o.quantize_ex(x, one, s, G, bits=bits, lambda_after=after, srft=True)
+                q = _codes_ex(o, codes, bits, D)[0]
+                want = np.zeros(D, np.int64)
+                want[0::2] = top
+                want[0] = want[1] = edge
+                assert np.array_equal(q, want), (D, bits, after, q)
 
 
 def pin_srft_codec(o):
@@ -589,7 +595,7 @@ def pin_srft_codec(o):
     y = R(lambda . x) or lambda . R(x) with R = P diag(s), and the round trip
     obeys the quantiser bound."""
     rng = np.random.default_rng(43)
-    for D, G in ((16, 16), (128, 32)):
+    for D, G in ((16, 16), (96, 32), (128, 32), (256, 64)):
         for bits in (4, 8):
             for after in (False, True):
                 lam, s = _rand_params(rng, D)
@@ -619,6 +625,116 @@ def pin_srft_codec(o):
                     lhs = np.linalg.norm(d * l64, axis=1)
                 slack = 2.0 ** -10 * np.linalg.norm(x64, axis=1) * (1.0 if after else l64.max())
                 assert np.all(lhs <= bound * 1.001 + slack)
+
+
+# ---- the SRFT's twiddles and complex FFT ----------------------------------
+
+_PI80 = ("3.14159265358979323846264338327950288419716939937510"
+         "58209749445923078164062862089986280348253421170679")
+
+
+def _cos_sin_exact(k: int, M: int):
+    """cos and sin of 2 pi k / M to ~75 digits, by Taylor series in decimal
+    arithmetic (no libm, no float)."""
+    import decimal
+    ctx = decimal.Context(prec=90)
+    pi = decimal.Decimal(_PI80)
+    j = k % M
+    x = ctx.divide(ctx.multiply(2 * pi, decimal.Decimal(j)), decimal.Decimal(M))
+    if x > pi:
+        x = ctx.subtract(x, 2 * pi)                    # |x| <= pi
+    x2 = ctx.multiply(x, x)
+    c, s = decimal.Decimal(1), x
+    tc, ts = decimal.Decimal(1), x
+    eps = decimal.Decimal(10) ** -85
+    n = 1
+    while abs(tc) > eps or abs(ts) > eps:
+        tc = ctx.divide(ctx.multiply(-tc, x2), decimal.Decimal((2 * n - 1) * (2 * n)))
+        ts = ctx.divide(ctx.multiply(-ts, x2), decimal.Decimal((2 * n) * (2 * n + 1)))
+        c, s = ctx.add(c, tc), ctx.add(s, ts)
+        n += 1
+    return c, s
+
+
+def _is_nearest_f32(f: np.float32, exact) -> bool:
+    """f is the fp32 value nearest `exact` (a Decimal), and not a tie."""
+    import decimal
+    f = np.float32(f)
+    d = abs(decimal.Decimal(float(f)) - exact)
+    for nb in (np.nextafter(f, np.float32(np.inf)), np.nextafter(f, np.float32(-np.inf))):
+        if not d < abs(decimal.Decimal(float(nb)) - exact):
+            return False
+    return True
+
+
+def pin_twiddle_exact(o):
+    """The twiddle table is the correctly rounded fp32 value of the exact root
+    of unity, (cos, -sin)(2 pi k / M), checked against an independent 80-digit
+    decimal evaluation; exact zeros are +0."""
+    for M in (1, 2, 3, 4, 6, 8, 12, 16, 24, 32, 48, 64, 96, 128, 192, 256):
+        for k in range(M):
+            wr, wi = o.twiddle(k, M)
+            c, s = _cos_sin_exact(k, M)
+            cos_zero = (4 * k) % M == 0 and ((4 * k) // M) % 2 == 1     # 2 pi k / M = odd * pi/2
+            sin_zero = (2 * k) % M == 0                                 # 2 pi k / M = n pi
+            for got, want, zero in ((wr, c, cos_zero), (wi, -s, sin_zero)):
+                if zero:
+                    assert got == 0.0 and not np.signbit(got), (k, M, got)
+                else:
+                    assert _is_nearest_f32(got, want), (k, M, float(got), str(want)[:20])
+
+
+def pin_twiddle_symmetries(o):
+    """Exact values and symmetries of the roots, bit for bit: omega^0 = 1,
+    omega^(M/4) = -i, omega^(M/2) = -1, omega^(M-k) = conj(omega^k),
+    omega^(k+M/4) = -i omega^k and omega^(M/2-k) = -conj(omega^k)."""
+    def b(v):
+        return np.float32(v).view(np.uint32) if v != 0 else np.uint32(0)
+    for M in (4, 8, 12, 16, 24, 32, 48, 64, 96, 128, 256):
+        assert o.twiddle(0, M) == (1.0, 0.0)
+        assert o.twiddle(M // 4, M) == (0.0, -1.0)
+        assert o.twiddle(M // 2, M) == (-1.0, 0.0)
+        for k in range(M):
+            wr, wi = o.twiddle(k, M)
+            cr, ci = o.twiddle(M - k, M)
+            assert (b(cr), b(ci)) == (b(wr), b(-wi)), (k, M)
+            rr, ri = o.twiddle(k + M // 4, M)
+            assert (b(rr), b(ri)) == (b(wi), b(-wr)), (k, M)
+            hr, hi = o.twiddle(M // 2 - k, M)
+            assert (b(hr), b(hi)) == (b(-wr), b(wi)), (k, M)
+
+
+def pin_fft_definition(o):
+    """The fp32 FFT (forward DIF stages, mixed radix 2 and 3) lies within its
+    rounding bound of numpy's fft; its transpose within the bound of N ifft
+    (the conjugate DFT)."""
+    rng = np.random.default_rng(44)
+    for N in (1, 2, 3, 4, 6, 8, 12, 16, 24, 32, 48, 64, 96, 128):
+        z = (rng.standard_normal((6, N)) + 1j * rng.standard_normal((6, N))).astype(np.complex64)
+        z64 = z.astype(np.complex128)
+        stages = max(1, math.ceil(math.log2(N)) + 1)
+        bound = 8.0 * stages * U32 * np.abs(z64).sum(axis=1, keepdims=True)
+        assert np.all(np.abs(o.fft_f32(z) - np.fft.fft(z64, axis=1)) <= bound), N
+        assert np.all(np.abs(o.fft_f32(z, inverse=True) - N * np.fft.ifft(z64, axis=1)) <= bound), N
+
+
+def pin_fft_exact_trivial_twiddles(o):
+    """Where only the twiddles 1, -1, i and -i occur (N = 2 and 4), products by
+    them are exact: small-integer inputs give numpy's fft exactly, and a unit
+    input at position m gives the row of powers of -i with exact zeros."""
+    rng = np.random.default_rng(45)
+    for N in (2, 4):
+        z = (rng.integers(-9, 10, (20, N)) + 1j * rng.integers(-9, 10, (20, N))).astype(np.complex64)
+        want = np.fft.fft(z.astype(np.complex128), axis=1)
+        assert np.array_equal(o.fft_f32(z).astype(np.complex128), want), N
+        assert np.array_equal(o.fft_f32(z, inverse=True).astype(np.complex128),
+                              N * np.fft.ifft(z.astype(np.complex128), axis=1)), N
+    for m in range(4):
+        e = np.zeros((1, 4), np.complex64)
+        e[0, m] = 1.0
+        got = o.fft_f32(e)[0]
+        want = np.array([(-1j) ** (m * k) for k in range(4)])
+        assert np.array_equal(got.astype(np.complex128), want.round()), (m, got)
 
 
 # ---- decode attention over the int4 cache ------------------------------
@@ -737,4 +853,6 @@ ALL_PINS = [
     pin_ex_matches_base, pin_ex_definition, pin_ex_int8_codes, pin_ex_tables,
     pin_ex_roundtrip_bound, pin_ex_impulse,
     pin_srft_definition, pin_srft_f32, pin_srft_closed_forms, pin_srft_codec,
+    pin_twiddle_exact, pin_twiddle_symmetries, pin_fft_definition,
+    pin_fft_exact_trivial_twiddles,
 ]

@@ -38,22 +38,38 @@ MUTANTS = [
     ("f16_round_trunc", "_Float16 h = (_Float16)f;", "_Float16 h = (_Float16)(f - f * 0x1p-12f);", 0),
     ("ex_int8_qmax", "float qmax = (bits == 4) ? 7.0f : 127.0f;", "float qmax = (bits == 4) ? 7.0f : 126.0f;", 0),
     ("ex_int8_clamp", "float qmin = (bits == 4) ? -8.0f : -128.0f;", "float qmin = (bits == 4) ? -8.0f : -8.0f;", 0),
-    ("ex_after_lambda_dropped", "for (int i = 0; i < D; ++i) y[i] = y[i] * lr[i];   /* lambda */", "(void)lr;", 0),
+    ("ex_after_lambda_dropped", "f[i] = lambda_after ? lr[i] * norm_of(i, D, srft)", "f[i] = lambda_after ? norm_of(i, D, srft)", 0),
     ("ex_variant_sign_dropped", "v[i] = (s[i] < 0) ? -t : t;                    /* exact  */", "v[i] = t;", 0),
     ("ex_table_index", "return lam + ((r / lambda_rows) % n_lambda) * (int64_t)D;", "return lam + (r % n_lambda) * (int64_t)D;", 0),
     ("ex_int8_store", "for (int i = 0; i < D; ++i) cr[i] = (uint8_t)q[i];", "for (int i = 0; i < D; ++i) cr[i] = (uint8_t)(q[i] & 0x7F);", 0),
-    ("ex_deq_lambda_mult", "if (lambda_after) u[i] = u[i] * (1.0f / lr[i]);        /* 1/lambda */", "if (lambda_after) u[i] = u[i] * lr[i];", 0),
+    ("ex_deq_lambda_mult", "f[i] = lambda_after ? norm_of(i, D, srft) / lr[i]", "f[i] = lambda_after ? norm_of(i, D, srft) * lr[i]", 0),
     ("ex_deq_sign_dropped", "float z = (s[i] < 0) ? -w[i] : w[i];                   /* exact */", "float z = w[i];", 0),
     ("ex_deq_before_lambda_mult", "w[i] = lambda_after ? z : z * (1.0f / lr[i]);", "w[i] = lambda_after ? z : z * lr[i];", 0),
     ("ex_deq_int8_unsigned", "for (int i = 0; i < D; ++i) q[i] = (int8_t)cr[i];", "for (int i = 0; i < D; ++i) q[i] = (int8_t)(cr[i] & 0x7F);", 0),
-    ("srft_twiddle_sign", "*wi = (float)(-sin(a));", "*wi = (float)(sin(a));", 0),
-    ("srft_no_sqrt2", "const float c1 = (float)(sqrt(2.0 / (double)D));", "const float c1 = (float)(sqrt(1.0 / (double)D));", 0),
-    ("srft_stage_stride", "twiddle(p * s, N, &wr, &wi);      /* omega_n^p = omega_N^(p s) */", "twiddle(p, N, &wr, &wi);", 0),
-    ("srft_butterfly_sign", "yr[q + s * 2 * p] = ar + br;", "yr[q + s * 2 * p] = ar - br;", 0),
-    ("srft_odd_part_sign", "float Or = Di * 0.5f, Oi = -(Dr * 0.5f);", "float Or = Di * 0.5f, Oi = (Dr * 0.5f);", 0),
-    ("srft_nyquist_slot", "y[1] = xr * c0;", "y[1] = xr * c1;", 0),
-    ("isrft_no_conj", "wi = -wi;                                         /* conj(omega_D^k) */", "wi = wi;", 0),
-    ("isrft_pairing", "zr[k] = Er - Oi;                                  /* E + i O */", "zr[k] = Er + Oi;", 0),
+    ("srft_twiddle_sign", "*wi = -sn + 0.0f;", "*wi = sn + 0.0f;", 0),
+    # the table before exact roots: cos / sin of 2 pi k / M straight in double
+    ("twiddle_unreduced", "    *wr = cr + 0.0f;                            /* -0 -> +0 */\n    *wi = -sn + 0.0f;",
+     "    (void)cr; (void)sn;\n    *wr = (float)cos(6.28318530717958647692 * (double)j / (double)M);\n"
+     "    *wi = (float)(-sin(6.28318530717958647692 * (double)j / (double)M));", 0),
+    ("twiddle_quadrant", "case 1: cr = -s; sn = c; break;", "case 1: cr = s; sn = c; break;", 0),
+    ("twiddle_complement", "if (comp) { float t = c; c = s; s = t; }", "(void)comp;", 0),
+    ("twiddle_signed_zero", "    *wr = cr + 0.0f;                            /* -0 -> +0 */", "    *wr = cr;", 0),
+    ("cmul_trivial_i_sign", "*pr = (wi > 0.0f) ? -di : di;", "*pr = (wi > 0.0f) ? di : -di;", 0),
+    ("srft_no_sqrt2", "(float)(1.0 / sqrt(2.0 * (double)D))", "(float)(1.0 / sqrt((double)D))", 0),
+    ("srft_stage_stride", "kvqo_twiddle(s * p * t, N, &wr, &wi);               /* omega_n^(p t) */",
+     "kvqo_twiddle(p * t, N, &wr, &wi);", 0),
+    ("srft_butterfly_sign", "br = br + tr;", "br = br - tr;", 0),
+    ("radix3_twiddle", "kvqo_twiddle((N / r) * j * t, N, &wr, &wi);     /* omega_r^(j t) */",
+     "kvqo_twiddle((N / r) * j, N, &wr, &wi);", 0),
+    ("dit_stage_conj", "cmul(yr[q + s * (r * p + t)], yi[q + s * (r * p + t)], wr, -wi, &cr[t], &ci[t]);",
+     "cmul(yr[q + s * (r * p + t)], yi[q + s * (r * p + t)], wr, wi, &cr[t], &ci[t]);", 0),
+    ("dit_radix_conj", "cmul(cr[t], ci[t], wr, -wi, &tr, &ti);", "cmul(cr[t], ci[t], wr, wi, &tr, &ti);", 0),
+    ("srft_odd_part_sign", "float Or = Di, Oi = -Dr;", "float Or = Di, Oi = Dr;", 0),
+    ("srft_nyquist_slot", "y[1] = (zr[0] - zi[0]) * f[1];", "y[1] = (zr[0] + zi[0]) * f[1];", 0),
+    ("isrft_no_conj", "cmul(Dr, Di, wr, -wi, &Tr, &Ti);                 /* conj(omega_D^k) */",
+     "cmul(Dr, Di, wr, wi, &Tr, &Ti);", 0),
+    ("isrft_pairing", "zr[k] = Er - Ti;                                  /* E + i T */", "zr[k] = Er + Ti;", 0),
+    ("isrft_dc", "zi[0] = u0 - un;", "zi[0] = u0 + un;", 0),
     ("attn_gqa_index", "int kv = h / R;", "int kv = h % Hkv;", 0),
     ("attn_no_max_shift", "double p = exp(z[t] - m);", "double p = exp(z[t]);", 0),
     ("attn_len_ignored", "for (int t = 0; t < len; ++t) {\n                double p", "for (int t = 0; t < T; ++t) {\n                double p", 0),
