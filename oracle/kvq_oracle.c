@@ -632,11 +632,13 @@ int kvqo_fft_f32(float *re, float *im, int N, int inverse)
     return 0;
 }
 
-/* 2 X_k of the real input from its half-length spectrum Z, k = 1 .. N-1:
- * A = Z_k, B = conj Z_(N-k), E = A + B, O = (A - B) / i (exact),
- * 2 X_k = E + omega_D^k O. */
-static void real_bin2(const float *zr, const float *zi, int N, int k,
-                      float *xr, float *xi)
+/* 2 X_k and 2 X_(N-k) of the real input from its half-length spectrum Z,
+ * for a pair 1 <= k <= N/2 (one bin at k = N/2):  A = Z_k, B = conj Z_(N-k),
+ * E = A + B, O = (A - B) / i (exact), T = omega_D^k O,
+ *   2 X_k = E + T,   2 X_(N-k) = conj(E - T)
+ * (the Hermitian symmetry of a real input's spectrum: both bins of a pair
+ * share E, O and T).  x[0..3] = re, im of 2 X_k, then of 2 X_(N-k). */
+static void real_pair2(const float *zr, const float *zi, int N, int k, float *x)
 {
     float Ar = zr[k], Ai = zi[k], Br = zr[N - k], Bi = -zi[N - k];
     float Er = Ar + Br, Ei = Ai + Bi;
@@ -645,8 +647,11 @@ static void real_bin2(const float *zr, const float *zi, int N, int k,
     float wr, wi, Tr, Ti;
     kvqo_twiddle(k, 2 * N, &wr, &wi);
     cmul(Or, Oi, wr, wi, &Tr, &Ti);
-    *xr = Er + Tr;
-    *xi = Ei + Ti;
+    x[0] = Er + Tr;
+    x[1] = Ei + Ti;
+    float Wr = Er - Tr, Wi = Ei - Ti;
+    x[2] = Wr;
+    x[3] = -Wi;
 }
 
 /* Is D an SRFT length: even, D/2 a power of two or three times one. */
@@ -664,8 +669,8 @@ static float srft_norm(int i, int D)
 }
 
 /* Forward SRFT of one sign-flipped row v[D] with per-position factors f:
- * y0 = (Z0.re + Z0.im) f0, y1 = (Z0.re - Z0.im) f1, (y_2k, y_2k+1) =
- * 2 X_k . (f_2k, f_2k+1). */
+ * y0 = (Z0.re + Z0.im) f0, y1 = (Z0.re - Z0.im) f1 (X_0 and X_N),
+ * (y_2k, y_2k+1) = 2 X_k . (f_2k, f_2k+1), the bins formed in pairs. */
 static void srft_scaled(const float *v, int D, const float *f, float *y)
 {
     int N = D / 2;
@@ -674,18 +679,23 @@ static void srft_scaled(const float *v, int D, const float *f, float *y)
     kvqo_fft_f32(zr, zi, N, 0);
     y[0] = (zr[0] + zi[0]) * f[0];
     y[1] = (zr[0] - zi[0]) * f[1];
-    for (int k = 1; k < N; ++k) {
-        float xr, xi;
-        real_bin2(zr, zi, N, k, &xr, &xi);
-        y[2 * k] = xr * f[2 * k];
-        y[2 * k + 1] = xi * f[2 * k + 1];
+    for (int k = 1; 2 * k <= N; ++k) {
+        float x[4];
+        real_pair2(zr, zi, N, k, x);
+        y[2 * k] = x[0] * f[2 * k];
+        y[2 * k + 1] = x[1] * f[2 * k + 1];
+        if (2 * k < N) {
+            y[2 * (N - k)] = x[2] * f[2 * (N - k)];
+            y[2 * (N - k) + 1] = x[3] * f[2 * (N - k) + 1];
+        }
     }
 }
 
 /* Transpose of srft_scaled: U_i = y_i f_i; the adjoint of the unpacking,
- * z_0 = (U_0 + U_1, U_0 - U_1) and, k = 1 .. N-1, A = U_k, B = conj U_(N-k),
- * E = A + B, T = (A - B) conj(omega_D^k), Z_k = E + i T; then the
- * transposed FFT. */
+ * z_0 = (U_0 + U_1, U_0 - U_1) and, for a pair 1 <= k <= N/2 (one bin at
+ * k = N/2), A = U_k, B = conj U_(N-k), E = A + B, T = (A - B) conj(omega_D^k),
+ *   Z_k = E + i T,   Z_(N-k) = conj(E - i T);
+ * then the transposed FFT. */
 static void isrft_scaled(const float *y, int D, const float *f, float *v)
 {
     int N = D / 2;
@@ -693,7 +703,7 @@ static void isrft_scaled(const float *y, int D, const float *f, float *v)
     float u0 = y[0] * f[0], un = y[1] * f[1];
     zr[0] = u0 + un;
     zi[0] = u0 - un;
-    for (int k = 1; k < N; ++k) {
+    for (int k = 1; 2 * k <= N; ++k) {
         float Ar = y[2 * k] * f[2 * k], Ai = y[2 * k + 1] * f[2 * k + 1];
         float Br = y[2 * (N - k)] * f[2 * (N - k)];
         float Bi = -(y[2 * (N - k) + 1] * f[2 * (N - k) + 1]);
@@ -704,6 +714,11 @@ static void isrft_scaled(const float *y, int D, const float *f, float *v)
         cmul(Dr, Di, wr, -wi, &Tr, &Ti);                 /* conj(omega_D^k) */
         zr[k] = Er - Ti;                                  /* E + i T */
         zi[k] = Ei + Tr;
+        if (2 * k < N) {
+            float Wr = Er + Ti, Wi = Ei - Tr;             /* E - i T */
+            zr[N - k] = Wr;
+            zi[N - k] = -Wi;
+        }
     }
     kvqo_fft_f32(zr, zi, N, 1);
     for (int n = 0; n < N; ++n) { v[2 * n] = zr[n]; v[2 * n + 1] = zi[n]; }

@@ -70,6 +70,11 @@ MUTANTS = [
      "cmul(Dr, Di, wr, wi, &Tr, &Ti);", 0),
     ("isrft_pairing", "zr[k] = Er - Ti;                                  /* E + i T */", "zr[k] = Er + Ti;", 0),
     ("isrft_dc", "zi[0] = u0 - un;", "zi[0] = u0 + un;", 0),
+    ("srft_pair_conj", "x[3] = -Wi;", "x[3] = Wi;", 0),
+    ("srft_pair_sub", "float Wr = Er - Tr, Wi = Ei - Ti;", "float Wr = Er + Tr, Wi = Ei - Ti;", 0),
+    ("isrft_pair_conj", "zi[N - k] = -Wi;", "zi[N - k] = Wi;", 0),
+    ("isrft_pair_sign", "float Wr = Er + Ti, Wi = Ei - Tr;             /* E - i T */",
+     "float Wr = Er - Ti, Wi = Ei - Tr;", 0),
     ("attn_gqa_index", "int kv = h / R;", "int kv = h % Hkv;", 0),
     ("attn_no_max_shift", "double p = exp(z[t] - m);", "double p = exp(z[t]);", 0),
     ("attn_len_ignored", "for (int t = 0; t < len; ++t) {\n                double p", "for (int t = 0; t < T; ++t) {\n                double p", 0),
