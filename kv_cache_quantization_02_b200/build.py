@@ -14,7 +14,8 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SOURCES = [os.path.join(PKG, "csrc", n) for n in ("kvq.cu", "kvq_attn.cu", "kvq_ex.cu")]
+SOURCES = [os.path.join(PKG, "csrc", n) for n in ("kvq.cu", "kvq_attn.cu", "kvq_ex.cu", "kvq_srft_d64.cu",
+                                                        "kvq_srft_d96.cu", "kvq_srft_d128.cu", "kvq_srft_d256.cu")]
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libkvq.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

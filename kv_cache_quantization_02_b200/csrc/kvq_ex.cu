@@ -50,6 +50,7 @@ constexpr unsigned kFullMask = 0xffffffffu;
 
 #include "kvq_async.cuh"
 #include "kvq_arith.cuh"
+#include "kvq_ex.cuh"
 
 constexpr int kD = 128;                 // channels (one lane per vector)
 constexpr int kNP = kD / 2;             // packed pairs (v[m], v[m+64])
@@ -67,15 +68,6 @@ struct ExMaps {
   CUtensorMap q[2];                     // fp16 rows: two 64-channel quarters
 };
 
-struct ExArgs {
-  const float* lam;                     // [n_lambda][128]
-  const int8_t* sgn;                    // [128]
-  int64_t n;
-  int64_t lambda_rows;
-  int n_lambda;
-  float c;                              // fp32 1/sqrt(128)
-};
-
 template <int BITS>
 struct Fmt {
   static constexpr int CB = BITS == 4 ? kD / 2 : kD;   // code bytes per row
@@ -86,23 +78,24 @@ __device__ __forceinline__ int xtile_off(int q, int t, int c) {
   return q * kQB + t * 128 + ((c ^ (t & 7)) << 4);
 }
 
-// Table of the tile starting at row r0 (all 32 rows share it).
-__device__ __forceinline__ int table_id(const ExArgs& a, int64_t r0) {
-  return a.n_lambda == 1 ? 0 : static_cast<int>((r0 / a.lambda_rows) % a.n_lambda);
-}
-
 // The warp's per-channel table in the pair layout of the base kernels:
 // tab[q] = (t[2q], t[2q+64], t[2q+1], t[2q+65]); mode 0: lambda * s,
-// 1: lambda, 2: s * (1/lambda), 3: 1/lambda.  Each lane fills one float4.
+// 1: fp32(lambda c) (lambda after the rotation: lambda and the normalisation
+// are one factor), 2: s * (1/lambda), 3: fp32(c / lambda) (its inverse,
+// applied before the transform).  Each lane fills one float4.
 __device__ __forceinline__ void build_table(float4* tab, const ExArgs& a, int id, int mode, int lane) {
   const float* lr = a.lam + static_cast<int64_t>(id) * kD;
   const int ch[4] = {2 * lane, 2 * lane + kNP, 2 * lane + 1, 2 * lane + 1 + kNP};
   float v[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    float l = lr[ch[k]];
-    if (mode >= 2) l = __frcp_rn(l);
-    v[k] = ((mode == 0 || mode == 2) && a.sgn[ch[k]] < 0) ? -l : l;
+    const float l = lr[ch[k]];
+    float t;
+    if (mode == 0) t = l;
+    else if (mode == 1) t = __fmul_rn(l, a.c);
+    else if (mode == 2) t = __frcp_rn(l);
+    else t = __fdiv_rn(a.c, l);
+    v[k] = ((mode == 0 || mode == 2) && a.sgn[ch[k]] < 0) ? -t : t;
   }
   tab[lane] = make_float4(v[0], v[1], v[2], v[3]);
 }
@@ -121,14 +114,6 @@ __device__ __forceinline__ void build_signs(float4* stab, const ExArgs& a, int q
 // counter.
 __host__ __device__ constexpr int hdr_bars(int nw) { return nw * 512 + 512; }
 __host__ __device__ constexpr int hdr_bytes(int nw) { return hdr_bars(nw) + 24 * nw + 16; }
-
-// Four codes -> one 32-bit word, code k in byte k, each saturated to [-128, 127].
-__device__ __forceinline__ uint32_t pack4_s8(int a0, int a1, int a2, int a3) {
-  uint32_t d;
-  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a3), "r"(a2), "r"(0u));
-  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a1), "r"(a0), "r"(d));
-  return d;
-}
 
 // ---------------------------------------------------------------------------
 // Quantize variants: fp16 [n][128] -> codes [n][CB] + fp16 scales [n][128/G].
@@ -232,15 +217,16 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
     }
 
     fwht_pairs<kD, 1>(p, 0);
-#pragma unroll
-    for (int m = 0; m < kNP; ++m) p[m] = __fmul2_rn(p[m], c2);
     if constexpr (AFTER) {
 #pragma unroll
       for (int q = 0; q < kNP / 2; ++q) {
-        const float4 l = tab[q];                      // lambda
+        const float4 l = tab[q];                      // fp32(lambda c)
         p[2 * q] = __fmul2_rn(p[2 * q], make_float2(l.x, l.y));
         p[2 * q + 1] = __fmul2_rn(p[2 * q + 1], make_float2(l.z, l.w));
       }
+    } else {
+#pragma unroll
+      for (int m = 0; m < kNP; ++m) p[m] = __fmul2_rn(p[m], c2);
     }
     // group abs-max, scale S = fp16(a / QMAX) (saturating), r = 1/S
     float rx[NGH], ry[NGH];
@@ -503,7 +489,7 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
     if constexpr (AFTER) {
 #pragma unroll
       for (int q = 0; q < kNP / 2; ++q) {
-        const float4 l = tab[q];                      // 1/lambda
+        const float4 l = tab[q];                      // fp32(c / lambda)
         p[2 * q] = __fmul2_rn(p[2 * q], make_float2(l.x, l.y));
         p[2 * q + 1] = __fmul2_rn(p[2 * q + 1], make_float2(l.z, l.w));
       }
@@ -517,16 +503,15 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         const int q = 4 * k4 + t;
-        float2 a0 = __fmul2_rn(p[2 * q], c2);
-        float2 a1 = __fmul2_rn(p[2 * q + 1], c2);
+        float2 a0, a1;
         if constexpr (AFTER) {                        // signs only: exact
           const float4 sg = stab[q];
-          a0 = __fmul2_rn(a0, make_float2(sg.x, sg.y));
-          a1 = __fmul2_rn(a1, make_float2(sg.z, sg.w));
+          a0 = __fmul2_rn(p[2 * q], make_float2(sg.x, sg.y));
+          a1 = __fmul2_rn(p[2 * q + 1], make_float2(sg.z, sg.w));
         } else {
           const float4 l = tab[q];                    // s * (1/lambda)
-          a0 = __fmul2_rn(a0, make_float2(l.x, l.y));
-          a1 = __fmul2_rn(a1, make_float2(l.z, l.w));
+          a0 = __fmul2_rn(__fmul2_rn(p[2 * q], c2), make_float2(l.x, l.y));
+          a1 = __fmul2_rn(__fmul2_rn(p[2 * q + 1], c2), make_float2(l.z, l.w));
         }
         lo[t] = float2_to_half2_bits(a0.x, a1.x);    // channels 2q, 2q+1
         hi[t] = float2_to_half2_bits(a0.y, a1.y);    // channels 64+2q, 64+2q+1
@@ -535,477 +520,6 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
       *reinterpret_cast<uint4*>(stage_out + xtile_off(1, lane, k4)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     }
     fence_proxy_async();                // generic-proxy writes -> visible to the tensor stores
-    __syncwarp();
-    if (lane == 0) {
-      tensor_s2g(&omaps.q[0], 0, static_cast<int>(tile * kWR), stage_out);
-      tensor_s2g(&omaps.q[1], 0, static_cast<int>(tile * kWR), stage_out + kQB);
-      bulk_commit();
-    }
-  }
-  if (lane == 0) bulk_wait0();
-}
-
-// ---------------------------------------------------------------------------
-// The SRFT variants.  SRFT(x) = pack(F diag(s) x), F the unitary DFT ("When
-// Quantization Is Free", technical summary, Methodologie 1), computed as the
-// paper's kernel does (Methodologie 2): the length-64 complex FFT of
-// z_n = v_2n + i v_2n+1 in six radix-2 Stockham stages, then the Hermitian
-// unpacking into the orthonormal real packing y0 = X_0, y1 = X_64,
-// (y_2k, y_2k+1) = sqrt(2) (Re, Im) X_k, all / sqrt(128).  The lane holds its
-// vector in the natural pair layout z[n] = (v[2n], v[2n+1]) (two fp16
-// channels of one 32-bit word), every complex product is the oracle's four
-// products and two sums, and the twiddles are the host's double cos / sin
-// rounded to fp32, so the results are bit-identical.
-// ---------------------------------------------------------------------------
-
-constexpr int kFN = kD / 2;             // complex FFT length (64)
-
-struct SrftTw {
-  float2 wn[kFN / 2];                   // omega_64^k, k < 32
-  float2 wd[kFN + 1];                   // omega_128^k, k <= 64
-};
-
-// (a - b) * w with the oracle's operation order: re = d.x w.x - d.y w.y,
-// im = d.x w.y + d.y w.x, each product and sum rounded once.
-__device__ __forceinline__ float2 cmul_rn(float2 d, float2 w) {
-  const float2 p0 = __fmul2_rn(d, make_float2(w.x, w.x));              // (d.x w.x, d.y w.x)
-  const float2 p1 = __fmul2_rn(d, make_float2(w.y, w.y));              // (d.x w.y, d.y w.y)
-  return make_float2(__fsub_rn(p0.x, p1.y), __fadd_rn(p1.x, p0.y));
-}
-
-// Stockham radix-2 FFT of 64 points in registers; INV: conjugate twiddles.
-// One radix-2 stage of the Stockham FFT (sub-transforms of length n = kFN >> ST).
-template <bool INV, int ST>
-__device__ __forceinline__ void stockham_stage(float2 (&x)[kFN], float2 (&y)[kFN], const SrftTw& tw) {
-  constexpr int n = kFN >> ST, m = n / 2, sstr = 1 << ST;
-  // p = 0: w = omega^0 = (cos 0, -+sin 0) = (1, +-0).  Both of cmul_rn's
-  // products with w.x are d itself and both with w.y are signed zeros, all
-  // exact, so each component is one rounding: re = rn(d.x - d.y w.y),
-  // im = rn(d.x w.y + d.y), the same values (zero signs and NaNs included)
-  // as cmul_rn(d, w).
-  const float z0 = INV ? -tw.wn[0].y : tw.wn[0].y;
-#pragma unroll
-  for (int q = 0; q < sstr; ++q) {
-    const float2 a = x[q], b = x[q + sstr * m];
-    y[q] = __fadd2_rn(a, b);
-    const float2 d = fsub2(a, b);
-    y[q + sstr] = make_float2(__fmaf_rn(d.y, -z0, d.x), __fmaf_rn(d.x, z0, d.y));
-  }
-#pragma unroll
-  for (int p = 1; p < m; ++p) {
-    float2 w = tw.wn[p * sstr];
-    if (INV) w.y = -w.y;
-#pragma unroll
-    for (int q = 0; q < sstr; ++q) {
-      const float2 a = x[q + sstr * p], b = x[q + sstr * (p + m)];
-      y[q + sstr * 2 * p] = __fadd2_rn(a, b);
-      y[q + sstr * (2 * p + 1)] = cmul_rn(fsub2(a, b), w);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < kFN; ++i) x[i] = y[i];
-}
-
-template <bool INV>
-__device__ __forceinline__ void stockham64(float2 (&x)[kFN], const SrftTw& tw) {
-  float2 y[kFN];
-  stockham_stage<INV, 0>(x, y, tw);
-  stockham_stage<INV, 1>(x, y, tw);
-  stockham_stage<INV, 2>(x, y, tw);
-  stockham_stage<INV, 3>(x, y, tw);
-  stockham_stage<INV, 4>(x, y, tw);
-  stockham_stage<INV, 5>(x, y, tw);
-}
-
-// Forward extraction: X_k from Z_k and Z_(64-k) (indices mod 64).
-__device__ __forceinline__ float2 real_bin(const float2 (&z)[kFN], int k, const SrftTw& tw) {
-  const float2 A = z[k % kFN];
-  const float2 zb = z[(kFN - k) % kFN];
-  const float2 B = make_float2(zb.x, -zb.y);
-  const float2 E = __fmul2_rn(__fadd2_rn(A, B), make_float2(0.5f, 0.5f));
-  const float2 Dd = fsub2(A, B);
-  const float2 O = __fmul2_rn(make_float2(Dd.y, Dd.x), make_float2(0.5f, -0.5f));   // (A - B) / 2i
-  return __fadd2_rn(E, cmul_rn(O, tw.wd[k]));
-}
-
-// Bins k and 64 - k read the same two spectrum values, so they are computed
-// together and written back in place (each Z is then dead).
-__device__ __forceinline__ void srft_fwd(float2 (&z)[kFN], const SrftTw& tw, float c0, float c1) {
-  stockham64<false>(z, tw);
-  const float2 x0 = real_bin(z, 0, tw), xn = real_bin(z, kFN, tw);
-#pragma unroll
-  for (int k = 1; k < kFN / 2; ++k) {
-    const float2 xk = real_bin(z, k, tw), xm = real_bin(z, kFN - k, tw);
-    z[k] = __fmul2_rn(xk, make_float2(c1, c1));
-    z[kFN - k] = __fmul2_rn(xm, make_float2(c1, c1));
-  }
-  z[kFN / 2] = __fmul2_rn(real_bin(z, kFN / 2, tw), make_float2(c1, c1));
-  z[0] = make_float2(__fmul_rn(x0.x, c0), __fmul_rn(xn.x, c0));
-}
-
-// Inverse (the transpose): packed pairs u[k] = (y_2k, y_2k+1), u[0] = (y0, y1).
-// Z'_k = E + i O from U_k and conj U_(64-k), E = (U_k + conj U_(64-k)) / 2,
-// O = (U_k - conj U_(64-k)) conj(omega_128^k) / 2.
-__device__ __forceinline__ float2 inv_bin(float2 A, float2 Bc, int k, const SrftTw& tw) {
-  const float2 B = make_float2(Bc.x, -Bc.y);
-  const float2 E = __fmul2_rn(__fadd2_rn(A, B), make_float2(0.5f, 0.5f));
-  const float2 w = make_float2(tw.wd[k].x, -tw.wd[k].y);
-  const float2 O = __fmul2_rn(cmul_rn(fsub2(A, B), w), make_float2(0.5f, 0.5f));
-  return make_float2(__fsub_rn(E.x, O.y), __fadd_rn(E.y, O.x));
-}
-
-// Inverse (the transpose): packed pairs z[k] = (y_2k, y_2k+1), z[0] = (y0, y1).
-// U_0 = 2 c0 y0, U_64 = 2 c0 y1, U_k = c1 (y_2k, y_2k+1); bins k and 64 - k
-// are again formed together, in place.
-__device__ __forceinline__ void srft_inv(float2 (&z)[kFN], const SrftTw& tw, float c0, float c1) {
-  const float2 u0 = make_float2(__fmul_rn(__fmul_rn(z[0].x, c0), 2.0f), 0.0f);
-  const float2 un = make_float2(__fmul_rn(__fmul_rn(z[0].y, c0), 2.0f), 0.0f);
-  z[0] = inv_bin(u0, un, 0, tw);
-#pragma unroll
-  for (int k = 1; k < kFN / 2; ++k) {
-    const float2 uk = __fmul2_rn(z[k], make_float2(c1, c1));
-    const float2 um = __fmul2_rn(z[kFN - k], make_float2(c1, c1));
-    z[k] = inv_bin(uk, um, k, tw);
-    z[kFN - k] = inv_bin(um, uk, kFN - k, tw);
-  }
-  {
-    const float2 uh = __fmul2_rn(z[kFN / 2], make_float2(c1, c1));
-    z[kFN / 2] = inv_bin(uh, uh, kFN / 2, tw);
-  }
-  stockham64<true>(z, tw);
-}
-
-// The warp's per-channel table in natural order: tab[q] = (t[4q] .. t[4q+3]).
-__device__ __forceinline__ void build_table_nat(float4* tab, const ExArgs& a, int id, int mode, int lane) {
-  const float* lr = a.lam + static_cast<int64_t>(id) * kD;
-  float v[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int ch = 4 * lane + k;
-    float l = lr[ch];
-    if (mode >= 2) l = __frcp_rn(l);
-    v[k] = ((mode == 0 || mode == 2) && a.sgn[ch] < 0) ? -l : l;
-  }
-  tab[lane] = make_float4(v[0], v[1], v[2], v[3]);
-}
-__device__ __forceinline__ void build_signs_nat(float4* stab, const ExArgs& a, int q) {
-  float v[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) v[k] = a.sgn[4 * q + k] < 0 ? -1.0f : 1.0f;
-  stab[q] = make_float4(v[0], v[1], v[2], v[3]);
-}
-
-template <int G, int BITS, bool AFTER>
-__global__ void __launch_bounds__(kDW * 32, 1)
-kvq_quantize_srft_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
-                         const __grid_constant__ SrftTw tw, float c0, float c1,
-                         const __grid_constant__ CUtensorMap cmap, uint16_t* __restrict__ scales) {
-  using F = Fmt<BITS>;
-  constexpr int GP = G / 2;             // pairs per group
-  constexpr int NG = kD / G;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint8_t* wsm = smem + warp * 2 * kXStage;
-  uint8_t* hdr = smem + kDW * 2 * kXStage;
-  float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
-  float4* stab = reinterpret_cast<float4*>(hdr + kDW * 512);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + hdr_bars(kDW)) + 2 * warp;
-  int* tq = reinterpret_cast<int*>(hdr + hdr_bars(kDW) + 16 * kDW) + 2 * warp;
-  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + hdr_bars(kDW) + 24 * kDW);
-  if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
-  if (tid == 0) *next = 0;
-  if (tid < 32) build_signs_nat(stab, a, tid);
-  __syncthreads();
-
-  const int64_t ntiles = (a.n + kWR - 1) / kWR;
-  // The block owns a contiguous range of tiles, so a warp's tiles stay in one
-  // lambda table for long stretches (a table spans lambda_rows / 32 tiles).
-  const int64_t per = ntiles / gridDim.x, rem = ntiles % gridDim.x;
-  const int64_t first = blockIdx.x * per + (blockIdx.x < rem ? blockIdx.x : rem);
-  const unsigned int mine = static_cast<unsigned int>(per + (blockIdx.x < rem ? 1 : 0));
-  auto claim = [&]() -> int {
-    unsigned int i = 0;
-    if (lane == 0) i = atomicAdd(next, 1u);
-    i = __shfl_sync(kFullMask, i, 0);
-    return i < mine ? static_cast<int>(first + i) : -1;
-  };
-  auto refill = [&](int stage) {
-    const int t = claim();
-    if (lane == 0) tq[stage] = t;
-    if (t < 0 || lane != 0) return;
-    mbar_expect_tx(&bar[stage], kXStage);
-    tensor_g2s(wsm + stage * kXStage, &maps.q[0], 0, t * kWR, &bar[stage]);
-    tensor_g2s(wsm + stage * kXStage + kQB, &maps.q[1], 0, t * kWR, &bar[stage]);
-  };
-  refill(0);
-  refill(1);
-  int cached = -1;
-  for (uint32_t k = 0;; ++k) {
-    const int stage = k & 1;
-    __syncwarp();
-    const int64_t tile = tq[stage];
-    if (tile < 0) break;
-    const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);
-    if (__any_sync(kFullMask, !ok)) {
-      if (lane == 0) atomicOr(&g_ex_fault, 1u);
-      mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);   // the stage that gave up, once more
-      // only the first tile has the other stage's copy in flight
-      if (k == 0 && tq[1] >= 0) mbar_wait(&bar[1], 0, kSpinX);
-      if (lane == 0) bulk_wait0();
-      return;
-    }
-    if (k > 0) {
-      // the other stage holds the previous tile's staged codes: once their
-      // store has read them, it takes the next tile
-      if (lane == 0) bulk_wait_read0();
-      __syncwarp();
-      refill(stage ^ 1);
-    }
-    const int id = table_id(a, tile * kWR);
-    if (id != cached) {
-      build_table_nat(tab, a, id, AFTER ? 1 : 0, lane);
-      cached = id;
-      __syncwarp();
-    }
-    const int64_t row = tile * kWR + lane;
-    const bool active = row < a.n;
-    const uint8_t* st = wsm + stage * kXStage;
-    float2 z[kFN];
-#pragma unroll
-    for (int c = 0; c < kD / 8; ++c) {                 // 16-byte chunk c: channels 8c .. 8c+7
-      const uint4 xv = *reinterpret_cast<const uint4*>(st + xtile_off(c / 8, lane, c % 8));
-      const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-      const float4 l0 = AFTER ? stab[2 * c] : tab[2 * c];          // channels 8c .. 8c+3
-      const float4 l1 = AFTER ? stab[2 * c + 1] : tab[2 * c + 1];  // 8c+4 .. 8c+7
-      z[4 * c] = __fmul2_rn(half2_bits_to_float2(xw[0]), make_float2(l0.x, l0.y));
-      z[4 * c + 1] = __fmul2_rn(half2_bits_to_float2(xw[1]), make_float2(l0.z, l0.w));
-      z[4 * c + 2] = __fmul2_rn(half2_bits_to_float2(xw[2]), make_float2(l1.x, l1.y));
-      z[4 * c + 3] = __fmul2_rn(half2_bits_to_float2(xw[3]), make_float2(l1.z, l1.w));
-    }
-
-    srft_fwd(z, tw, c0, c1);
-    if constexpr (AFTER) {
-#pragma unroll
-      for (int q = 0; q < kFN / 2; ++q) {
-        const float4 l = tab[q];                      // lambda, channels 4q .. 4q+3
-        z[2 * q] = __fmul2_rn(z[2 * q], make_float2(l.x, l.y));
-        z[2 * q + 1] = __fmul2_rn(z[2 * q + 1], make_float2(l.z, l.w));
-      }
-    }
-    float r[NG];
-    uint16_t b[NG];
-#pragma unroll
-    for (int j = 0; j < NG; ++j) {
-      float am = 0.f;
-#pragma unroll
-      for (int m = 0; m < GP; ++m) am = amax3(am, z[j * GP + m].x, z[j * GP + m].y);
-      b[j] = group_scale_q<F::QMAX>(am, r[j]);
-    }
-    uint32_t out[F::CB / 4];
-    if constexpr (BITS == 4) {
-#pragma unroll
-      for (int k8 = 0; k8 < kD / 8; ++k8) {
-        int qv[8];
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int m = 4 * k8 + t;
-          const float2 v = __fmul2_rn(z[m], make_float2(r[m / GP], r[m / GP]));
-          qv[2 * t] = __float2int_rn(v.x);
-          qv[2 * t + 1] = __float2int_rn(v.y);
-        }
-        out[k8] = pack8(qv);
-      }
-    } else {
-#pragma unroll
-      for (int k4 = 0; k4 < kD / 4; ++k4) {
-        const float2 v0 = __fmul2_rn(z[2 * k4], make_float2(r[(2 * k4) / GP], r[(2 * k4) / GP]));
-        const float2 v1 = __fmul2_rn(z[2 * k4 + 1], make_float2(r[(2 * k4 + 1) / GP], r[(2 * k4 + 1) / GP]));
-        out[k4] = pack4_s8(__float2int_rn(v0.x), __float2int_rn(v0.y), __float2int_rn(v1.x), __float2int_rn(v1.y));
-      }
-    }
-    // the codes leave through the stage this tile came from (every lane has
-    // read it), swizzled as code_chunk reads, by one tensor store that skips
-    // rows past n
-    __syncwarp();
-    {
-      uint8_t* cst = wsm + stage * kXStage;
-      const int swz = ((lane * F::CB) >> 7) & (F::CB / 16 - 1);
-#pragma unroll
-      for (int k4 = 0; k4 < F::CB / 16; ++k4)
-        *reinterpret_cast<uint4*>(cst + lane * F::CB + ((k4 ^ swz) << 4)) =
-            make_uint4(out[4 * k4], out[4 * k4 + 1], out[4 * k4 + 2], out[4 * k4 + 3]);
-      fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) {
-        tensor_s2g(&cmap, 0, static_cast<int>(tile * kWR), cst);
-        bulk_commit();
-      }
-    }
-    if (active) {
-      uint16_t* srow = scales + row * NG;
-#pragma unroll
-      for (int j = 0; j < NG; ++j) srow[j] = b[j];
-    }
-  }
-  if (lane == 0) bulk_wait0();
-}
-
-template <int G, int BITS, bool AFTER>
-__global__ void __launch_bounds__(kDW * 32, 1)
-kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const __grid_constant__ CUtensorMap cmap,
-                           const uint16_t* __restrict__ scales,
-                           const ExArgs a, const __grid_constant__ SrftTw tw, float c0, float c1,
-                           const __grid_constant__ ExMaps omaps, int scale_copy) {
-  using F = Fmt<BITS>;
-  using L = DeqLayout<G, BITS>;
-  constexpr int GP = G / 2;
-  constexpr int NG = kD / G;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint8_t* stage_out = smem + warp * L::WARP;              // swizzled fp16 staging tile
-  uint8_t* wsm = stage_out + kXStage;                      // two code tiles, then two scale blocks
-  uint8_t* hdr = smem + kDW * L::WARP;
-  float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
-  float4* stab = reinterpret_cast<float4*>(hdr + kDW * 512);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + hdr_bars(kDW)) + 2 * warp;
-  int* tq = reinterpret_cast<int*>(hdr + hdr_bars(kDW) + 16 * kDW) + 2 * warp;
-  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + hdr_bars(kDW) + 24 * kDW);
-  if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
-  if (tid == 0) *next = 0;
-  if (tid < 32) build_signs_nat(stab, a, tid);
-  __syncthreads();
-
-  const int64_t ntiles = (a.n + kWR - 1) / kWR;
-  // The block owns a contiguous range of tiles, so a warp's tiles stay in one
-  // lambda table for long stretches (a table spans lambda_rows / 32 tiles).
-  const int64_t per = ntiles / gridDim.x, rem = ntiles % gridDim.x;
-  const int64_t first = blockIdx.x * per + (blockIdx.x < rem ? blockIdx.x : rem);
-  const unsigned int mine = static_cast<unsigned int>(per + (blockIdx.x < rem ? 1 : 0));
-  auto claim = [&]() -> int {
-    unsigned int i = 0;
-    if (lane == 0) i = atomicAdd(next, 1u);
-    i = __shfl_sync(kFullMask, i, 0);
-    return i < mine ? static_cast<int>(first + i) : -1;
-  };
-  auto scale_bytes = [&](int64_t t) -> uint32_t {
-    if (!scale_copy) return 0;
-    const int64_t row0 = t * kWR;
-    const int valid = static_cast<int>(a.n - row0 < kWR ? a.n - row0 : kWR);
-    return static_cast<uint32_t>(valid * L::SPR) & ~15u;
-  };
-  auto refill = [&](int stage) {
-    const int t = claim();
-    if (lane == 0) tq[stage] = t;
-    if (t < 0 || lane != 0) return;
-    const int64_t row0 = static_cast<int64_t>(t) * kWR;
-    const uint32_t sb = scale_bytes(t);
-    if constexpr (BITS == 8) {         // swizzled tensor copy: the copy engine fills the whole box
-      mbar_expect_tx(&bar[stage], static_cast<uint32_t>(L::WC) + sb);
-      tensor_g2s(wsm + stage * L::WC, &cmap, 0, static_cast<int>(row0), &bar[stage]);
-    } else {                           // plain bulk copy of the valid rows
-      const uint32_t cbytes = static_cast<uint32_t>(a.n - row0 < kWR ? a.n - row0 : kWR) * F::CB;
-      mbar_expect_tx(&bar[stage], cbytes + sb);
-      bulk_g2s(wsm + stage * L::WC, codes + row0 * F::CB, cbytes, &bar[stage]);
-    }
-    if (sb) bulk_g2s(wsm + L::SC + stage * L::WS, reinterpret_cast<const uint8_t*>(scales) + row0 * L::SPR, sb, &bar[stage]);
-  };
-  refill(0);
-  refill(1);
-  int cached = -1;
-  for (uint32_t k = 0;; ++k) {
-    const int stage = k & 1;
-    __syncwarp();
-    const int64_t tile = tq[stage];
-    if (tile < 0) break;
-    const int64_t row = tile * kWR + lane;
-    const int64_t rrow = row < a.n ? row : a.n - 1;
-    const bool sc_smem = static_cast<uint32_t>((lane + 1) * L::SPR) <= scale_bytes(tile);
-    const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);
-    if (__any_sync(kFullMask, !ok)) {
-      if (lane == 0) atomicOr(&g_ex_fault, 1u);
-      mbar_wait(&bar[stage], (k >> 1) & 1, kSpinX);   // the stage that gave up, once more
-      if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinX);
-      if (lane == 0) bulk_wait0();
-      return;
-    }
-    const int id = table_id(a, tile * kWR);
-    if (id != cached) {
-      build_table_nat(tab, a, id, AFTER ? 3 : 2, lane);
-      cached = id;
-      __syncwarp();
-    }
-    const uint8_t* st = wsm + stage * L::WC;
-    const uint16_t* srow = sc_smem ? reinterpret_cast<const uint16_t*>(wsm + L::SC + stage * L::WS + lane * L::SPR)
-                                   : scales + rrow * NG;
-    uint16_t sv[NG];
-#pragma unroll
-    for (int j = 0; j < NG; ++j) sv[j] = srow[j];
-    float2 z[kFN];
-    if constexpr (BITS == 4) {
-      const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
-#pragma unroll
-      for (int j = 0; j < kD / 8; ++j) {               // word j: channels 8j .. 8j+7
-        const uint32_t w = reinterpret_cast<const uint32_t*>(st + lane * F::CB)[j] ^ 0x88888888u, w4 = w >> 4;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const uint32_t sel = 0x0400u | (t << 8) | t;
-          const uint32_t e = (__byte_perm(w, w4, sel) & 0x000F000Fu) | 0x64006400u;
-          const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&e), bias);
-          const int m = 4 * j + t;                     // pair (2m, 2m+1)
-          z[m] = make_float2(mul_f16_f32(__low2half(h), sv[m / GP]), mul_f16_f32(__high2half(h), sv[m / GP]));
-        }
-      }
-    } else {
-      const __half2 bias = __floats2half2_rn(1152.0f, 1152.0f);
-#pragma unroll
-      for (int j = 0; j < kD / 4; ++j) {               // word j: channels 4j .. 4j+3
-        const uint4 ch = code_chunk<F::CB>(st, lane, j >> 2);
-        const uint32_t cw[4] = {ch.x, ch.y, ch.z, ch.w};
-        const uint32_t w = cw[j & 3] ^ 0x80808080u;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const uint32_t sel = static_cast<uint32_t>(2 * t) | ((2u * t + 1) << 8);   // bytes 2t, 2t+1
-          const uint32_t e = (__byte_perm(w, 0u, sel) & 0x00FF00FFu) | 0x64006400u;
-          const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&e), bias);
-          const int m = 2 * j + t;
-          z[m] = make_float2(mul_f16_f32(__low2half(h), sv[m / GP]), mul_f16_f32(__high2half(h), sv[m / GP]));
-        }
-      }
-    }
-    __syncwarp();
-    refill(stage);
-    if constexpr (AFTER) {
-#pragma unroll
-      for (int q = 0; q < kFN / 2; ++q) {
-        const float4 l = tab[q];                      // 1/lambda
-        z[2 * q] = __fmul2_rn(z[2 * q], make_float2(l.x, l.y));
-        z[2 * q + 1] = __fmul2_rn(z[2 * q + 1], make_float2(l.z, l.w));
-      }
-    }
-    srft_inv(z, tw, c0, c1);
-    if (lane == 0) bulk_wait_read0();
-    __syncwarp();
-#pragma unroll
-    for (int c = 0; c < kD / 8; ++c) {
-      uint32_t hv[4];
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const float4 sg = stab[2 * c + t];
-        float2 v0 = __fmul2_rn(z[4 * c + 2 * t], make_float2(sg.x, sg.y));
-        float2 v1 = __fmul2_rn(z[4 * c + 2 * t + 1], make_float2(sg.z, sg.w));
-        if constexpr (!AFTER) {
-          const float4 l = tab[2 * c + t];            // s * (1/lambda): the sign again, exact
-          v0 = __fmul2_rn(z[4 * c + 2 * t], make_float2(l.x, l.y));
-          v1 = __fmul2_rn(z[4 * c + 2 * t + 1], make_float2(l.z, l.w));
-        }
-        hv[2 * t] = float2_to_half2_bits(v0.x, v0.y);
-        hv[2 * t + 1] = float2_to_half2_bits(v1.x, v1.y);
-      }
-      *reinterpret_cast<uint4*>(stage_out + xtile_off(c / 8, lane, c % 8)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-    }
-    fence_proxy_async();
     __syncwarp();
     if (lane == 0) {
       tensor_s2g(&omaps.q[0], 0, static_cast<int>(tile * kWR), stage_out);
@@ -1056,9 +570,10 @@ int finish_ex() {
   return KVQ_OK;
 }
 
-int check_ex(int D, int G, int bits, int64_t n, int64_t lambda_rows, int n_lambda) {
-  if (D != kD) return KVQ_ERR_DIM;
-  if (G != 16 && G != 32 && G != 64) return KVQ_ERR_GROUP;
+// D: 128 with the Walsh-Hadamard rotation; 64, 96, 128 or 256 with the SRFT.
+int check_ex(int D, int G, int bits, int64_t n, int64_t lambda_rows, int n_lambda, bool srft) {
+  if (srft ? (D != 64 && D != 96 && D != 128 && D != 256) : D != kD) return KVQ_ERR_DIM;
+  if ((G != 16 && G != 32 && G != 64) || D % G != 0) return KVQ_ERR_GROUP;
   if (bits != 4 && bits != 8) return KVQ_ERR_GROUP;
   if (n < 0 || n > (int64_t{1} << 31) - 256 || n_lambda < 1 || lambda_rows < 1 ||
       (n_lambda > 1 && lambda_rows % kWR != 0))
@@ -1109,23 +624,6 @@ int launch_dex(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, ui
   return finish_ex();
 }
 
-// Twiddles of the SRFT: omega_M^k = (cos(2 pi k / M), -sin(2 pi k / M)) in
-// double, rounded to fp32 (built once).
-const SrftTw& srft_twiddles() {
-  static const SrftTw tw = [] {
-    SrftTw t{};
-    auto om = [](int k, int M) {
-      const double a = 2.0 * 3.14159265358979323846 * static_cast<double>(k) / static_cast<double>(M);
-      return make_float2(static_cast<float>(std::cos(a)), static_cast<float>(-std::sin(a)));
-    };
-    for (int k = 0; k < kFN / 2; ++k) t.wn[k] = om(k, kFN);
-    for (int k = 0; k <= kFN; ++k) t.wd[k] = om(k, kD);
-    return t;
-  }();
-  return tw;
-}
-const float kSrftC0 = static_cast<float>(1.0 / std::sqrt(static_cast<double>(kD)));
-const float kSrftC1 = static_cast<float>(std::sqrt(2.0 / static_cast<double>(kD)));
 
 int encode_x_maps(ExMaps& maps, const uint16_t* x, int64_t n) {
   const EncodeTiledFn enc = encode_tiled();
@@ -1171,46 +669,6 @@ int encode_code_map(CUtensorMap& map, const uint8_t* codes, int64_t n, int cb) {
   return KVQ_OK;
 }
 
-template <int G, int BITS, bool AFTER>
-int launch_qsrft(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* scales, cudaStream_t st) {
-  ExMaps maps;
-  const int rc = encode_x_maps(maps, x, a.n);
-  if (rc != KVQ_OK) return rc;
-  auto k = kvq_quantize_srft_kernel<G, BITS, AFTER>;
-  constexpr int smem = 1024 + kDW * 2 * kXStage + hdr_bytes(kDW);
-  static std::atomic<int> ready[64];
-  const int grid = ex_grid(k, a.n, smem, kDW * 32, ready);
-  CUtensorMap cmap;
-  const int rc2 = encode_code_map(cmap, codes, a.n, Fmt<BITS>::CB);
-  if (rc2 != KVQ_OK) return rc2;
-  (void)cudaGetLastError();
-  k<<<grid, kDW * 32, smem, st>>>(maps, a, srft_twiddles(), kSrftC0, kSrftC1, cmap, scales);
-  return finish_ex();
-}
-
-template <int G, int BITS, bool AFTER>
-int launch_dsrft(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, uint16_t* out,
-                 cudaStream_t st) {
-  using L = DeqLayout<G, BITS>;
-  ExMaps omaps;
-  const int rc = encode_x_maps(omaps, out, a.n);
-  if (rc != KVQ_OK) return rc;
-  auto k = kvq_dequantize_srft_kernel<G, BITS, AFTER>;
-  constexpr int smem = 1024 + kDW * L::WARP + hdr_bytes(kDW);
-  static std::atomic<int> ready[64];
-  const int grid = ex_grid(k, a.n, smem, kDW * 32, ready);
-  CUtensorMap cmap;
-  memset(&cmap, 0, sizeof(cmap));
-  if (BITS == 8) {
-    const int rc2 = encode_code_map(cmap, codes, a.n, Fmt<BITS>::CB);
-    if (rc2 != KVQ_OK) return rc2;
-  }
-  (void)cudaGetLastError();
-  k<<<grid, kDW * 32, smem, st>>>(codes, cmap, scales, a, srft_twiddles(), kSrftC0, kSrftC1, omaps,
-                                  (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
-  return finish_ex();
-}
-
 #define KVQ_EX_DISPATCH(FN, ...)                                                        \
   switch (group * 100 + bits * 10 + (lambda_after ? 1 : 0)) {                          \
     case 1640: return FN<16, 4, false>(__VA_ARGS__);                                    \
@@ -1232,8 +690,24 @@ inline bool aligned_to(const void* p, uintptr_t al) { return (reinterpret_cast<u
 
 }  // namespace
 
-// Read (and optionally clear) the variant kernels' fault word; used by
-// kvq_fault_status.
+// The SRFT codec, one translation unit per D (kvq_srft_d<D>.cu), after the
+// checks below.
+#define KVQ_SRFT_DECL(D)                                                                          \
+  int kvq_srft_quantize_##D(const uint16_t* x, const float* lambda, const int8_t* signs, int64_t n, \
+                            int group, int bits, bool after, int64_t lambda_rows, int n_lambda,      \
+                            uint8_t* codes, uint16_t* scales, cudaStream_t st);                      \
+  int kvq_srft_dequantize_##D(const uint8_t* codes, const uint16_t* scales, const float* lambda,     \
+                              const int8_t* signs, int64_t n, int group, int bits, bool after,       \
+                              int64_t lambda_rows, int n_lambda, uint16_t* out, cudaStream_t st);    \
+  unsigned int kvq_srft_fault_word_##D(int clear);                                                   \
+  int kvq_srft_last_cuda_error_##D();
+KVQ_SRFT_DECL(64)
+KVQ_SRFT_DECL(96)
+KVQ_SRFT_DECL(128)
+KVQ_SRFT_DECL(256)
+
+// Read (and optionally clear) the variant kernels' fault words; used by
+// kvq_fault_status.  The SRFT units' words are included.
 __attribute__((visibility("hidden"))) unsigned int kvq_ex_fault_word(int clear) {
   unsigned int v = 0;
   if (cudaMemcpyFromSymbol(&v, g_ex_fault, sizeof(v)) != cudaSuccess) return 0;
@@ -1241,16 +715,23 @@ __attribute__((visibility("hidden"))) unsigned int kvq_ex_fault_word(int clear) 
     const unsigned int zero = 0;
     cudaMemcpyToSymbol(g_ex_fault, &zero, sizeof(zero));
   }
-  return v;
+  return v | kvq_srft_fault_word_64(clear) | kvq_srft_fault_word_96(clear) |
+         kvq_srft_fault_word_128(clear) | kvq_srft_fault_word_256(clear);
 }
-__attribute__((visibility("hidden"))) int kvq_ex_last_cuda_error() { return g_ex_cuda_error; }
+__attribute__((visibility("hidden"))) int kvq_ex_last_cuda_error() {
+  if (g_ex_cuda_error) return g_ex_cuda_error;
+  if (const int e = kvq_srft_last_cuda_error_64()) return e;
+  if (const int e = kvq_srft_last_cuda_error_96()) return e;
+  if (const int e = kvq_srft_last_cuda_error_128()) return e;
+  return kvq_srft_last_cuda_error_256();
+}
 
 extern "C" {
 
 int kvq_quantize_ex(const uint16_t* x, const float* lambda, const int8_t* signs, int64_t n_vec,
                     int D, int group, int bits, int flags, int64_t lambda_rows,
                     int n_lambda, uint8_t* codes, uint16_t* scales, void* stream) {
-  const int rc = check_ex(D, group, bits, n_vec, lambda_rows, n_lambda);
+  const int rc = check_ex(D, group, bits, n_vec, lambda_rows, n_lambda, (flags & 2) != 0);
   if (rc != KVQ_OK) return rc;
   if ((flags & ~3) != 0) return KVQ_ERR_GROUP;
   if (n_vec == 0) return KVQ_OK;
@@ -1262,7 +743,15 @@ int kvq_quantize_ex(const uint16_t* x, const float* lambda, const int8_t* signs,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool lambda_after = (flags & 1) != 0;
   if (flags & 2) {
-    KVQ_EX_DISPATCH(launch_qsrft, x, a, codes, scales, st)
+#define KVQ_SRFT_Q(DD) \
+  return kvq_srft_quantize_##DD(x, lambda, signs, n_vec, group, bits, lambda_after, lambda_rows, n_lambda, codes, scales, st)
+    switch (D) {
+      case 64: KVQ_SRFT_Q(64);
+      case 96: KVQ_SRFT_Q(96);
+      case 128: KVQ_SRFT_Q(128);
+      default: KVQ_SRFT_Q(256);
+    }
+#undef KVQ_SRFT_Q
   }
   KVQ_EX_DISPATCH(launch_qex, x, a, codes, scales, st)
 }
@@ -1271,7 +760,7 @@ int kvq_dequantize_ex(const uint8_t* codes, const uint16_t* scales, const float*
                       const int8_t* signs, int64_t n_vec, int D, int group, int bits,
                       int flags, int64_t lambda_rows, int n_lambda, uint16_t* x_out,
                       void* stream) {
-  const int rc = check_ex(D, group, bits, n_vec, lambda_rows, n_lambda);
+  const int rc = check_ex(D, group, bits, n_vec, lambda_rows, n_lambda, (flags & 2) != 0);
   if (rc != KVQ_OK) return rc;
   if ((flags & ~3) != 0) return KVQ_ERR_GROUP;
   if (n_vec == 0) return KVQ_OK;
@@ -1283,7 +772,15 @@ int kvq_dequantize_ex(const uint8_t* codes, const uint16_t* scales, const float*
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const bool lambda_after = (flags & 1) != 0;
   if (flags & 2) {
-    KVQ_EX_DISPATCH(launch_dsrft, codes, scales, a, x_out, st)
+#define KVQ_SRFT_DQ(DD) \
+  return kvq_srft_dequantize_##DD(codes, scales, lambda, signs, n_vec, group, bits, lambda_after, lambda_rows, n_lambda, x_out, st)
+    switch (D) {
+      case 64: KVQ_SRFT_DQ(64);
+      case 96: KVQ_SRFT_DQ(96);
+      case 128: KVQ_SRFT_DQ(128);
+      default: KVQ_SRFT_DQ(256);
+    }
+#undef KVQ_SRFT_DQ
   }
   KVQ_EX_DISPATCH(launch_dex, codes, scales, a, x_out, st)
 }

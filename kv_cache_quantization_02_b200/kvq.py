@@ -274,9 +274,9 @@ def quantize_ex(x: torch.Tensor, lam: torch.Tensor, signs: torch.Tensor, group: 
                 bits: int = 4, lambda_after: bool = False, lambda_rows: int | None = None,
                 codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
                 stream=None, srft: bool = False):
-    """Format variants.  x fp16 [n, 128]; lam fp32 [n_lambda, 128] (or [128]);
-    row r uses table (r // lambda_rows) % n_lambda.  -> (codes uint8 [n, 64 or
-    128], scales fp16 [n, 128/group])."""
+    """Format variants.  x fp16 [n, D]; lam fp32 [n_lambda, D] (or [D]); row r
+    uses table (r // lambda_rows) % n_lambda.  -> (codes uint8 [n, D/2 or D],
+    scales fp16 [n, D/group]).  D = 128, or 64, 96, 128, 256 with srft=True."""
     if x.dim() != 2:
         raise ValueError("x must be [n_vec, D]")
     n, D = x.shape
@@ -304,7 +304,7 @@ def dequantize_ex(codes: torch.Tensor, scales: torch.Tensor, lam: torch.Tensor,
                   signs: torch.Tensor, group: int, bits: int = 4, lambda_after: bool = False,
                   lambda_rows: int | None = None, out: torch.Tensor | None = None,
                   stream=None, srft: bool = False) -> torch.Tensor:
-    """Inverse of quantize_ex -> fp16 [n, 128]."""
+    """Inverse of quantize_ex -> fp16 [n, D]."""
     if codes.dim() != 2:
         raise ValueError("codes must be [n_vec, bytes]")
     n = codes.shape[0]

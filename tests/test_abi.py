@@ -157,3 +157,13 @@ def test_codec_ex_errors(kvq):
         assert f(n=0) == 0
     assert q(x=0) == -1 and q(codes=0) == -1 and d(codes=0) == -1 and d(out=0) == -1
     assert q(x=A + 8) == -2 and q(lam=A + 2) == -2 and d(codes=A + 8) == -2 and d(out=A + 8) == -2
+    # the SRFT (flags bit 1) takes D = 64, 96, 128 or 256 and a group dividing D
+    sq = lambda **kw: kvq.kvq_quantize_ex(A, A, A, kw.get("n", 64), kw["D"], kw.get("G", 32), 4,
+                                          2 | kw.get("after", 0), 64, 1, A, A)
+    sd = lambda **kw: kvq.kvq_dequantize_ex(A, A, A, A, kw.get("n", 64), kw["D"], kw.get("G", 32), 8,
+                                            2 | kw.get("after", 0), 64, 1, A)
+    for f in (sq, sd):
+        assert f(D=96, G=64) == -4 and f(D=80) == -3 and f(D=512) == -3 and f(D=32) == -3
+        assert f(D=192) == -3 and f(D=256, G=128) == -4
+        for D in (64, 96, 128, 256):
+            assert f(D=D, n=0) == 0 and f(D=D, n=0, after=1) == 0
