@@ -91,6 +91,8 @@ class Oracle:
             "kvqo_isrft_f64": (None, [_P, _I, _P]),
             "kvqo_attention_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            _I, _I, _I, _I, _I, _I, ctypes.c_double, _P]),
+            "kvqo_attention_decode_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                              _I, _I, _I, _I, _I, _I, _I, ctypes.c_double, _P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -300,11 +302,13 @@ class Oracle:
         return out.view(np.float16)
 
     def attention_decode(self, q, k_packed, k_scales, v_packed, v_scales, seq_len,
-                         lam_k, s_k, lam_v, s_v, group: int, sm_scale: float) -> np.ndarray:
+                         lam_k, s_k, lam_v, s_v, group: int, sm_scale: float,
+                         lambda_after: bool = False, srft: bool = False) -> np.ndarray:
         """Decode attention over the int4 cache, float64 [B, Hq, D].
 
         q fp16 [B, Hq, D]; packed u8 [B, Hkv, T, D/2]; scales fp16
-        [B, Hkv, T, D/group]; seq_len int [B]."""
+        [B, Hkv, T, D/group]; seq_len int [B].  lambda_after / srft: the
+        cache's rows are codec-variant rows of that format."""
         q = np.ascontiguousarray(q)
         if q.dtype != np.float16 or q.ndim != 3:
             raise TypeError("q must be float16 [B, Hq, D]")
@@ -320,10 +324,10 @@ class Oracle:
         lk, sk = _params(lam_k, s_k)
         lv, sv = _params(lam_v, s_v)
         out = np.empty((B, Hq, D), dtype=np.float64)
-        _check(self._lib.kvqo_attention_decode(
+        _check(self._lib.kvqo_attention_decode_ex(
             _ptr(q.view(np.uint16)), _ptr(kp), _ptr(ks), _ptr(vp), _ptr(vs), _ptr(sl),
             _ptr(lk), _ptr(sk), _ptr(lv), _ptr(sv), B, Hq, Hkv, T, D, group,
-            float(sm_scale), _ptr(out)))
+            _flags(lambda_after, srft), float(sm_scale), _ptr(out)))
         return out
 
 

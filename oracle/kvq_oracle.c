@@ -391,30 +391,57 @@ int kvqo_quantize_codes_divform(const uint16_t *x, const float *lam,
 /* [B][Hkv][T][D/G]; seq_len [B]; out double [B][Hq][D].                */
 /* ------------------------------------------------------------------ */
 
+void kvqo_isrft_f64(const double *y, int D, double *v);   /* below */
+static int srft_len_ok(int D);
+
 /* One reconstructed row in double: codes times scales, then the exact   */
-/* inverse rotation.                                                     */
+/* inverse of the row's rotation (flags as for the codec variants: bit 0 */
+/* lambda after the rotation, bit 1 the SRFT):                           */
+/*   lambda before: x = (diag(s) R^T y) / lambda,                        */
+/*   lambda after:  x = diag(s) R^T (y / lambda),                        */
+/* R^T = H / sqrt(D) (Walsh-Hadamard) or P^T (the SRFT's packed unitary  */
+/* DFT, transposed).                                                     */
 static void reconstruct_row_f64(const uint8_t *packed, const uint16_t *scales,
                                 const double *lam, const int8_t *s, int D,
-                                int G, double *x)
+                                int G, int flags, double *x)
 {
     int8_t q[KVQO_DMAX];
     double y[KVQO_DMAX];
     kvqo_unpack(packed, D, q);
     for (int i = 0; i < D; ++i)
         y[i] = (double)q[i] * (double)kvqo_f16_to_f32(scales[i / G]);
-    kvqo_unrotate_f64(y, lam, s, D, x);
+    if (flags == 0) {
+        kvqo_unrotate_f64(y, lam, s, D, x);
+        return;
+    }
+    if (flags & 1)
+        for (int i = 0; i < D; ++i) y[i] /= lam[i];
+    if (flags & 2) {
+        kvqo_isrft_f64(y, D, x);
+    } else {
+        double inv = 1.0 / sqrt((double)D);
+        for (int i = 0; i < D; ++i) x[i] = y[i];
+        kvqo_fwht_f64(x, D);
+        for (int i = 0; i < D; ++i) x[i] *= inv;
+    }
+    for (int i = 0; i < D; ++i) {
+        x[i] *= (double)s[i];
+        if (!(flags & 1)) x[i] /= lam[i];
+    }
 }
 
-int kvqo_attention_decode(const uint16_t *q, const uint8_t *k_packed,
-                          const uint16_t *k_scales, const uint8_t *v_packed,
-                          const uint16_t *v_scales, const int32_t *seq_len,
-                          const float *lam_k, const int8_t *s_k,
-                          const float *lam_v, const int8_t *s_v, int B, int Hq,
-                          int Hkv, int T, int D, int G, double sm_scale,
-                          double *out)
+int kvqo_attention_decode_ex(const uint16_t *q, const uint8_t *k_packed,
+                             const uint16_t *k_scales, const uint8_t *v_packed,
+                             const uint16_t *v_scales, const int32_t *seq_len,
+                             const float *lam_k, const int8_t *s_k,
+                             const float *lam_v, const int8_t *s_v, int B,
+                             int Hq, int Hkv, int T, int D, int G, int flags,
+                             double sm_scale, double *out)
 {
-    int rc = check_shape(D, G);
+    int rc = (flags & 2) ? (srft_len_ok(D) ? 0 : -3) : check_shape(D, G);
     if (rc) return rc;
+    if (!is_pow2(G) || G < 2 || G > D || D % G != 0) return -4;
+    if (flags & ~3) return -4;
     if (B < 0 || T < 0 || Hkv < 1 || Hq < Hkv || Hq % Hkv != 0) return -5;
     for (int b = 0; b < B; ++b)
         if (seq_len[b] < 0 || seq_len[b] > T) return -5;
@@ -441,7 +468,7 @@ int kvqo_attention_decode(const uint16_t *q, const uint8_t *k_packed,
             for (int t = 0; t < len; ++t) {
                 reconstruct_row_f64(k_packed + (base + t) * (D / 2),
                                     k_scales + (base + t) * (D / G), lk, s_k,
-                                    D, G, row);
+                                    D, G, flags, row);
                 double dot = 0.0;
                 for (int i = 0; i < D; ++i) dot += qd[i] * row[i];
                 z[t] = sm_scale * dot;
@@ -453,7 +480,7 @@ int kvqo_attention_decode(const uint16_t *q, const uint8_t *k_packed,
                 l += p;
                 reconstruct_row_f64(v_packed + (base + t) * (D / 2),
                                     v_scales + (base + t) * (D / G), lv, s_v,
-                                    D, G, row);
+                                    D, G, flags, row);
                 for (int i = 0; i < D; ++i) o[i] += p * row[i];
             }
             for (int i = 0; i < D; ++i) o[i] /= l;
@@ -461,6 +488,20 @@ int kvqo_attention_decode(const uint16_t *q, const uint8_t *k_packed,
     }
     free(z);
     return 0;
+}
+
+/* The base cache format: Walsh-Hadamard rows, lambda before the rotation. */
+int kvqo_attention_decode(const uint16_t *q, const uint8_t *k_packed,
+                          const uint16_t *k_scales, const uint8_t *v_packed,
+                          const uint16_t *v_scales, const int32_t *seq_len,
+                          const float *lam_k, const int8_t *s_k,
+                          const float *lam_v, const int8_t *s_v, int B, int Hq,
+                          int Hkv, int T, int D, int G, double sm_scale,
+                          double *out)
+{
+    return kvqo_attention_decode_ex(q, k_packed, k_scales, v_packed, v_scales,
+                                    seq_len, lam_k, s_k, lam_v, s_v, B, Hq, Hkv,
+                                    T, D, G, 0, sm_scale, out);
 }
 
 /* ------------------------------------------------------------------ */

@@ -760,6 +760,28 @@ def _rebuild(packed, scales, lam, s, G):
     return (y @ H.T) / math.sqrt(D) * s.astype(np.float64) / lam.astype(np.float64)
 
 
+def _rebuild_fmt(packed, scales, lam, s, G, lambda_after, srft):
+    """Rows of a codec-variant cache in float64: y = codes . S, then
+    (diag(s) R^T y) / lambda (lambda before) or diag(s) R^T (y / lambda)
+    (after), R^T = H / sqrt D (scipy's Hadamard matrix) or P^T, P the packed
+    unitary real DFT built from numpy's rfft of the identity."""
+    import scipy.linalg
+    q = _nibbles(packed)
+    D = q.shape[-1]
+    S = np.repeat(np.asarray(scales, dtype=np.float16).astype(np.float64), G, axis=-1)
+    y = q * S
+    l64, s64 = lam.astype(np.float64), s.astype(np.float64)
+    if lambda_after:
+        y = y / l64
+    if srft:
+        P = _rfft_packed(np.eye(D)).T                   # column j = P e_j
+        x = y @ P                                       # rows of P^T y
+    else:
+        x = (y @ scipy.linalg.hadamard(D).astype(np.float64).T) / math.sqrt(D)
+    x = x * s64
+    return x if lambda_after else x / l64
+
+
 def _attn_case(rng, B, Hq, Hkv, T, D, G, smax=2.0):
     q = rng.standard_normal((B, Hq, D)).astype(np.float16)
     kp = rng.integers(0, 256, (B, Hkv, T, D // 2), dtype=np.uint8)
@@ -828,6 +850,58 @@ def pin_attention_closed_forms(o):
             assert np.abs(hard[b, h] - ref).max() <= 1e-5 * np.abs(ref).max()
 
 
+def pin_attention_formats_vs_sdpa(o):
+    """Over caches of every codec-variant format (lambda before or after the
+    rotation, Walsh-Hadamard or SRFT rows, the mixed-radix D = 96 included),
+    the oracle equals torch's SDPA (float64) on K and V rebuilt independently
+    with scipy's Hadamard matrix or numpy's rfft."""
+    import torch
+    rng = np.random.default_rng(24)
+    cases = ((2, 8, 2, 23, 32, 8), (1, 4, 1, 17, 96, 32), (2, 6, 3, 11, 64, 16))
+    for B, Hq, Hkv, T, D, G in cases:
+        for after in (False, True):
+            for srft in (False, True):
+                if D == 96 and not srft:
+                    continue
+                q, kp, ks, vp, vs, lk, sk, lv, sv = _attn_case(rng, B, Hq, Hkv, T, D, G)
+                lens = rng.integers(1, T + 1, B)
+                got = o.attention_decode(q, kp, ks, vp, vs, lens, lk, sk, lv, sv, G, 0.45,
+                                         lambda_after=after, srft=srft)
+                K = _rebuild_fmt(kp, ks, lk, sk, G, after, srft)
+                V = _rebuild_fmt(vp, vs, lv, sv, G, after, srft)
+                R = Hq // Hkv
+                for b in range(B):
+                    L = int(lens[b])
+                    kt = torch.from_numpy(K[b, :, :L]).repeat_interleave(R, dim=0)[None]
+                    vt = torch.from_numpy(V[b, :, :L]).repeat_interleave(R, dim=0)[None]
+                    qt = torch.from_numpy(q[b].astype(np.float64))[None, :, None, :]
+                    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=0.45)
+                    ref = ref[0, :, 0, :].numpy()
+                    err = np.abs(got[b] - ref).max()
+                    assert err <= 1e-11 * max(1.0, np.abs(ref).max()), (D, after, srft, err)
+
+
+def pin_attention_formats_closed_forms(o):
+    """SRFT and lambda-after caches: one key gives that key's value row (the
+    codec's own fp32 dequantisation of it, within its rounding), a zero score
+    scale gives the mean of the value rows."""
+    rng = np.random.default_rng(25)
+    B, Hq, Hkv, T, D, G = 1, 2, 1, 6, 64, 16
+    for after, srft in ((True, False), (False, True), (True, True)):
+        q, kp, ks, vp, vs, lk, sk, lv, sv = _attn_case(rng, B, Hq, Hkv, T, D, G)
+        rows = o.dequantize_ex(vp[0, 0], vs[0, 0], lv, sv, G, lambda_after=after,
+                               srft=srft).astype(np.float64)
+        one = o.attention_decode(q, kp, ks, vp, vs, [1], lk, sk, lv, sv, G, 0.5,
+                                 lambda_after=after, srft=srft)
+        for h in range(Hq):
+            assert np.abs(one[0, h] - rows[0]).max() <= 2e-3 * np.abs(rows[0]).max()
+        mean = o.attention_decode(q, kp, ks, vp, vs, [T], lk, sk, lv, sv, G, 0.0,
+                                  lambda_after=after, srft=srft)
+        for h in range(Hq):
+            ref = rows.mean(axis=0)
+            assert np.abs(mean[0, h] - ref).max() <= 2e-3 * np.abs(rows).max()
+
+
 def pin_attention_masking(o):
     """Entries past a sequence's length do not matter; length 0 gives 0."""
     rng = np.random.default_rng(23)
@@ -850,6 +924,7 @@ ALL_PINS = [
     pin_special_cases, pin_worked_examples, pin_divform_near_ties,
     pin_pack_layout, pin_accounting,
     pin_attention_vs_sdpa, pin_attention_closed_forms, pin_attention_masking,
+    pin_attention_formats_vs_sdpa, pin_attention_formats_closed_forms,
     pin_ex_matches_base, pin_ex_definition, pin_ex_int8_codes, pin_ex_tables,
     pin_ex_roundtrip_bound, pin_ex_impulse,
     pin_srft_definition, pin_srft_f32, pin_srft_closed_forms, pin_srft_codec,

@@ -79,10 +79,15 @@ MUTANTS = [
     ("attn_no_max_shift", "double p = exp(z[t] - m);", "double p = exp(z[t]);", 0),
     ("attn_len_ignored", "for (int t = 0; t < len; ++t) {\n                double p", "for (int t = 0; t < T; ++t) {\n                double p", 0),
     ("attn_scale_unused", "z[t] = sm_scale * dot;", "z[t] = dot;", 0),
-    ("attn_v_uses_k_lambda", "D, G, row);\n                for (int i = 0; i < D; ++i) o[i] += p * row[i];",
-     "D, G, row);\n                (void)lv; for (int i = 0; i < D; ++i) o[i] += p * row[i] * lv[i] / lk[i];", 0),
+    ("attn_v_uses_k_lambda", "D, G, flags, row);\n                for (int i = 0; i < D; ++i) o[i] += p * row[i];",
+     "D, G, flags, row);\n                (void)lv; for (int i = 0; i < D; ++i) o[i] += p * row[i] * lv[i] / lk[i];", 0),
     ("attn_not_normalised", "for (int i = 0; i < D; ++i) o[i] /= l;", "(void)l;", 0),
     ("attn_scale_index", "(double)kvqo_f16_to_f32(scales[i / G]);", "(double)kvqo_f16_to_f32(scales[0]);", 0),
+    ("attn_fmt_after_divides_late", "    if (flags & 1)\n        for (int i = 0; i < D; ++i) y[i] /= lam[i];",
+     "    if (flags & 1)\n        for (int i = 0; i < D; ++i) y[i] *= 1.0;", 0),
+    ("attn_fmt_srft_as_wht", "    if (flags & 2) {\n        kvqo_isrft_f64(y, D, x);", "    if (0) {\n        kvqo_isrft_f64(y, D, x);", 0),
+    ("attn_fmt_sign_dropped", "        x[i] *= (double)s[i];\n        if (!(flags & 1)) x[i] /= lam[i];",
+     "        if (!(flags & 1)) x[i] /= lam[i];", 0),
 ]
 
 
