@@ -245,6 +245,29 @@ int kvq_attention_decode(const uint16_t *q, const uint8_t *k_packed,
                          int64_t workspace_bytes, void *stream);
 
 /*
+ * kvq_attention_decode_ex -- kvq_attention_decode over a cache written by
+ * kvq_quantize_ex with int4 codes (bits 4): `flags` is the cache's format,
+ * bit 0 (KVQ_LAMBDA_AFTER) lambda after the rotation, bit 1 (KVQ_SRFT) the
+ * SRFT rotation ("When Quantization Is Free", technical summary,
+ * Methodologie 1-2: the paper's own cache is KVQ_SRFT | KVQ_LAMBDA_AFTER).
+ * The rows are rebuilt as (diag(s) R^T (codes . S)) / lambda with lambda
+ * before the rotation, diag(s) R^T ((codes . S) / lambda) with lambda after
+ * it, R^T the inverse Walsh-Hadamard or SRFT rotation; the query is rotated
+ * once to match and the rotated-domain output rotated back once per head.
+ * One lambda table per K and per V (lambda_rows = all rows).  Other flag bits
+ * -> KVQ_ERR_GROUP; other arguments, checks and results as for
+ * kvq_attention_decode, which is this call with flags = 0.
+ */
+int kvq_attention_decode_ex(const uint16_t *q, const uint8_t *k_packed,
+                            const uint16_t *k_scales, const uint8_t *v_packed,
+                            const uint16_t *v_scales, const int32_t *seq_len,
+                            const float *lambda_k, const int8_t *signs_k,
+                            const float *lambda_v, const int8_t *signs_v,
+                            int B, int Hq, int Hkv, int T, int D, int group, int flags,
+                            float sm_scale, uint16_t *out, void *workspace,
+                            int64_t workspace_bytes, void *stream);
+
+/*
  * kvq_attention_workspace_bytes -- bytes of workspace kvq_attention_decode
  * uses for these shapes on the current device (0: it does not split), or -1
  * if the shapes are invalid.  Host-only; launches nothing.

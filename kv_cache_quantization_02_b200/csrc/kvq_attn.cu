@@ -51,12 +51,18 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstring>
+#include <type_traits>
 
 #include "kvq.h"
 
 namespace {
 
+constexpr unsigned kFullMask = 0xffffffffu;
+
 #include "kvq_async.cuh"
+#include "kvq_arith.cuh"
+#include "kvq_fft.cuh"
 
 constexpr int kAW = 4;                       // warps per block
 constexpr int kBK = 64;                      // keys per streamed block
@@ -92,7 +98,14 @@ struct AttnParams {
   int Hkv, T, R, nsplit, chunk;
   float scale_log2;             // sm_scale * log2(e) * 2^24 (the key product comes out scaled by 2^-24)
   float c;                      // fp32 1/sqrt(D)
+  float c1h;                    // fp32 1/sqrt(2D): the SRFT's normalisation of 2 X_k
+  float2 wn[64];                // SRFT twiddles omega_(D/2)^k, k < D/2 (SRFT caches only)
+  float2 wd[65];                // omega_D^k, k <= D/2
 };
+
+// Cache formats (the codec variants' flags): bit 0 lambda after the rotation,
+// bit 1 the SRFT rotation.
+constexpr int kFmtAfter = 1, kFmtSrft = 2;
 
 template <int D, int G>
 struct Attn {
@@ -153,33 +166,71 @@ __device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
   }
 }
 
-// out[d] = fp16((s_V[d] * c * (H y)[d]) / lambda_V[d]) for one head, y = o / l.
-template <int D>
+// One head's output from its merged rotated-domain sum y = o / l, back in
+// the cache's format:
+//   lambda before: out = fp16((s_V . R^T y) / lambda_V),
+//   lambda after:  out = fp16(s_V . R^T (y / lambda_V)),
+// R^T = H / sqrt(D) (a warp-wide butterfly over the lanes' channels) or the
+// SRFT transpose (the codec's adjoint unpacking and transposed FFT, run by one
+// lane on the row gathered in `scr`, D floats of this warp's shared memory).
+template <int D, int FMT>
 __device__ __forceinline__ void finish_head(const AttnParams& P, float (&v)[D / 32], float l,
-                                            uint16_t* out_row, int lane) {
+                                            uint16_t* out_row, int lane, float* scr) {
   constexpr int DPL = D / 32;
   const float inv = l > 0.0f ? 1.0f / l : 0.0f;
 #pragma unroll
   for (int i = 0; i < DPL; ++i) v[i] *= inv;
-  warp_fwht<D>(v, lane);
-  uint16_t h[DPL];
+  if constexpr ((FMT & kFmtSrft) == 0) {
+    if constexpr (FMT & kFmtAfter) {
 #pragma unroll
-  for (int i = 0; i < DPL; ++i) {
-    const int d = DPL * lane + i;
-    const float z = v[i] * P.c;
-    const float zs = P.s_v[d] < 0 ? -z : z;
-    h[i] = __half_as_ushort(__float2half_rn(zs / P.lam_v[d]));
-  }
-  if constexpr (DPL == 4) {
-    *reinterpret_cast<uint2*>(out_row + DPL * lane) =
-        make_uint2(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16));
+      for (int i = 0; i < DPL; ++i) v[i] /= P.lam_v[DPL * lane + i];
+    }
+    warp_fwht<D>(v, lane);
+    uint16_t h[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      const int d = DPL * lane + i;
+      const float z = v[i] * P.c;
+      const float zs = P.s_v[d] < 0 ? -z : z;
+      h[i] = __half_as_ushort(__float2half_rn((FMT & kFmtAfter) ? zs : zs / P.lam_v[d]));
+    }
+    if constexpr (DPL == 4) {
+      *reinterpret_cast<uint2*>(out_row + DPL * lane) =
+          make_uint2(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16));
+    } else {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) out_row[DPL * lane + i] = h[i];
+    }
   } else {
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) out_row[DPL * lane + i] = h[i];
+    for (int i = 0; i < DPL; ++i) scr[DPL * lane + i] = v[i];
+    __syncwarp();
+    if (lane == 0) {
+      float2 z[D / 2];
+#pragma unroll
+      for (int n = 0; n < D / 2; ++n) z[n] = make_float2(scr[2 * n], scr[2 * n + 1]);
+      unpack_inv1<D>(z, P.wd, [&](int n) -> float2 {
+        float2 f = n == 0 ? make_float2(P.c, P.c) : make_float2(P.c1h, P.c1h);
+        if constexpr (FMT & kFmtAfter) f = make_float2(f.x / P.lam_v[2 * n], f.y / P.lam_v[2 * n + 1]);
+        return f;
+      });
+      fft_inv_from<D / 2, D / 2, D / 2>(z, P.wn);
+#pragma unroll
+      for (int n = 0; n < D / 2; ++n) {
+        float a = P.s_v[2 * n] < 0 ? -z[n].x : z[n].x;
+        float b = P.s_v[2 * n + 1] < 0 ? -z[n].y : z[n].y;
+        if constexpr ((FMT & kFmtAfter) == 0) {
+          a = a / P.lam_v[2 * n];
+          b = b / P.lam_v[2 * n + 1];
+        }
+        reinterpret_cast<uint32_t*>(out_row)[n] = float2_to_half2_bits(a, b);
+      }
+    }
+    __syncwarp();
   }
 }
 
-template <int D, int G>
+template <int D, int G, int FMT>
 __global__ void __launch_bounds__(kAW * 32, 2)
 kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   using A = Attn<D, G>;
@@ -213,15 +264,52 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     for (int s = 0; s < kAStages; ++s) mbar_init(&bar[s], 1);
     mbar_fence_init();
   }
-  // q~ = H diag(s_K) (q / lambda_K) / sqrt(D), split into fp16 hi + lo.
+  // The rotated query, split into fp16 hi + lo: q~ = R (s_K . (q / lambda_K))
+  // with lambda before the rotation, q~ = R (s_K . q) / lambda_K with lambda
+  // after it (so that <q, x_t> = <q~, y_t>), R = H / sqrt(D) or the SRFT.
   for (int r = warp; r < kMaxRows; r += kAW) {
+    if constexpr (FMT & kFmtSrft) {
+      if (lane == 0) {
+        float2 z[D / 2];
+        if (r < R) {
+          const uint32_t* qr = reinterpret_cast<const uint32_t*>(
+              P.q + (static_cast<int64_t>(b) * P.Hkv * R + kvh * R + r) * D);
+#pragma unroll
+          for (int n = 0; n < D / 2; ++n) {
+            float2 x = half2_bits_to_float2(qr[n]);
+            if constexpr ((FMT & kFmtAfter) == 0) x = make_float2(x.x / P.lam_k[2 * n], x.y / P.lam_k[2 * n + 1]);
+            z[n] = make_float2(P.s_k[2 * n] < 0 ? -x.x : x.x, P.s_k[2 * n + 1] < 0 ? -x.y : x.y);
+          }
+          fft_fwd_from<D / 2, D / 2, D / 2>(z, P.wn);
+          unpack_fwd1<D>(z, P.wd, [&](int n) -> float2 {
+            float2 f = n == 0 ? make_float2(P.c, P.c) : make_float2(P.c1h, P.c1h);
+            if constexpr (FMT & kFmtAfter) f = make_float2(f.x / P.lam_k[2 * n], f.y / P.lam_k[2 * n + 1]);
+            if (n > D / 4) f.y = -f.y;                 // bins above N/2 come as conj(E - T)
+            return f;
+          });
+        } else {
+#pragma unroll
+          for (int n = 0; n < D / 2; ++n) z[n] = make_float2(0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int n = 0; n < D / 2; ++n) {
+          const __half2 hi = __floats2half2_rn(z[n].x, z[n].y);
+          const float2 hf = __half22float2(hi);
+          const __half2 lo = __floats2half2_rn(z[n].x - hf.x, z[n].y - hf.y);
+          reinterpret_cast<__half2*>(qt + r * D)[n] = hi;
+          reinterpret_cast<__half2*>(qt + (kMaxRows + r) * D)[n] = lo;
+        }
+      }
+      continue;
+    }
     float v[DPL];
     if (r < R) {
       const uint16_t* qr = P.q + (static_cast<int64_t>(b) * P.Hkv * R + kvh * R + r) * D;
 #pragma unroll
       for (int i = 0; i < DPL; ++i) {
         const int d = DPL * lane + i;
-        const float x = __half2float(__ushort_as_half(qr[d])) / P.lam_k[d];
+        float x = __half2float(__ushort_as_half(qr[d]));
+        if constexpr ((FMT & kFmtAfter) == 0) x = x / P.lam_k[d];
         v[i] = P.s_k[d] < 0 ? -x : x;
       }
       warp_fwht<D>(v, lane);
@@ -232,7 +320,8 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
 #pragma unroll
     for (int i = 0; i < DPL; ++i) {
       const int d = DPL * lane + i;
-      const float y = v[i] * P.c;
+      float y = v[i] * P.c;
+      if constexpr (FMT & kFmtAfter) y = y / P.lam_k[d];
       const __half hi = __float2half_rn(y);
       const __half lo = __float2half_rn(y - __half2float(hi));
       qt[r * D + d] = hi;
@@ -471,7 +560,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     }
     if (P.nsplit == 1) {
       uint16_t* orow = P.out + (static_cast<int64_t>(b) * P.Hkv * R + kvh * R + r) * D;
-      finish_head<D>(P, v, lsum, orow, lane);
+      finish_head<D, FMT>(P, v, lsum, orow, lane, comb + r * D);   // row r's first slot: read above
     } else {
       float* pr = P.part + (static_cast<int64_t>(item) * R + r) * (D + 4);
       if (lane == 0) { pr[0] = M; pr[1] = lsum; }
@@ -482,9 +571,10 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
 }
 
 // Merge of the key splits of one (sequence, KV head): one warp per head.
-template <int D>
+template <int D, int FMT>
 __global__ void __launch_bounds__(kMaxRows * 32)
 kvq_attn_combine_kernel(const __grid_constant__ AttnParams P) {
+  __shared__ float scr[kMaxRows][D];
   constexpr int DPL = D / 32;
   const int bh = blockIdx.x, b = bh / P.Hkv, kvh = bh % P.Hkv;
   const int r = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -504,7 +594,7 @@ kvq_attn_combine_kernel(const __grid_constant__ AttnParams P) {
     for (int i = 0; i < DPL; ++i) v[i] += e * pr[4 + DPL * lane + i];
   }
   uint16_t* orow = P.out + (static_cast<int64_t>(b) * P.Hkv * P.R + kvh * P.R + r) * D;
-  finish_head<D>(P, v, lsum, orow, lane);
+  finish_head<D, FMT>(P, v, lsum, orow, lane, scr[r]);
 }
 
 // ---------------------------------------------------------------------------
@@ -555,10 +645,10 @@ int check_attn(int B, int Hq, int Hkv, int T, int D, int G) {
   return KVQ_OK;
 }
 
-template <int D, int G>
-int launch_attn(AttnParams P, int64_t pairs, cudaStream_t st) {
+template <int D, int G, int FMT>
+int launch_attn(const AttnParams& P, int64_t pairs, cudaStream_t st) {
   using A = Attn<D, G>;
-  auto k = kvq_attn_kernel<D, G>;
+  auto k = kvq_attn_kernel<D, G, FMT>;
   static std::atomic<int> ready[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
@@ -570,13 +660,37 @@ int launch_attn(AttnParams P, int64_t pairs, cudaStream_t st) {
   (void)cudaGetLastError();
   k<<<static_cast<unsigned>(items), kAW * 32, A::SMEM, st>>>(P);
   if (P.nsplit > 1)
-    kvq_attn_combine_kernel<D><<<static_cast<unsigned>(pairs), kMaxRows * 32, 0, st>>>(P);
+    kvq_attn_combine_kernel<D, FMT><<<static_cast<unsigned>(pairs), kMaxRows * 32, 0, st>>>(P);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     g_attn_cuda_error = static_cast<int>(e);
     return KVQ_ERR_LAUNCH;
   }
   return KVQ_OK;
+}
+
+template <int D, int G>
+int launch_fmt(const AttnParams& P, int64_t pairs, int flags, cudaStream_t st) {
+  switch (flags) {
+    case 0: return launch_attn<D, G, 0>(P, pairs, st);
+    case 1: return launch_attn<D, G, 1>(P, pairs, st);
+    case 2: return launch_attn<D, G, 2>(P, pairs, st);
+    default: return launch_attn<D, G, 3>(P, pairs, st);
+  }
+}
+
+// The SRFT's twiddles at length D (built once per D).
+template <int D>
+void attn_twiddles(AttnParams& P) {
+  struct Tw { float2 wn[D / 2]; float2 wd[D / 2 + 1]; };
+  static const Tw tw = [] {
+    Tw t{};
+    for (int k = 0; k < D / 2; ++k) t.wn[k] = root_f32(k, D / 2);
+    for (int k = 0; k <= D / 2; ++k) t.wd[k] = root_f32(k, D);
+    return t;
+  }();
+  memcpy(P.wn, tw.wn, sizeof(tw.wn));
+  memcpy(P.wd, tw.wd, sizeof(tw.wd));
 }
 
 }  // namespace
@@ -629,14 +743,15 @@ int64_t kvq_attention_workspace_bytes(int B, int Hq, int Hkv, int T, int D, int 
   return part_bytes(pairs, Hq / Hkv, D, sp.nsplit);
 }
 
-int kvq_attention_decode(const uint16_t* q, const uint8_t* k_packed, const uint16_t* k_scales,
-                         const uint8_t* v_packed, const uint16_t* v_scales, const int32_t* seq_len,
-                         const float* lambda_k, const int8_t* signs_k, const float* lambda_v,
-                         const int8_t* signs_v, int B, int Hq, int Hkv, int T, int D, int group,
-                         float sm_scale, uint16_t* out, void* workspace, int64_t workspace_bytes,
-                         void* stream) {
+int kvq_attention_decode_ex(const uint16_t* q, const uint8_t* k_packed, const uint16_t* k_scales,
+                            const uint8_t* v_packed, const uint16_t* v_scales, const int32_t* seq_len,
+                            const float* lambda_k, const int8_t* signs_k, const float* lambda_v,
+                            const int8_t* signs_v, int B, int Hq, int Hkv, int T, int D, int group,
+                            int flags, float sm_scale, uint16_t* out, void* workspace,
+                            int64_t workspace_bytes, void* stream) {
   const int rc = check_attn(B, Hq, Hkv, T, D, group);
   if (rc != KVQ_OK) return rc;
+  if ((flags & ~3) != 0) return KVQ_ERR_GROUP;
   if (B == 0) return KVQ_OK;
   if (!q || !k_packed || !k_scales || !v_packed || !v_scales || !seq_len || !lambda_k ||
       !signs_k || !lambda_v || !signs_v || !out)
@@ -661,15 +776,33 @@ int kvq_attention_decode(const uint16_t* q, const uint8_t* k_packed, const uint1
   // scores come out of the key product scaled by 2^-24 (subnormal codes)
   P.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634 * 16777216.0);
   P.c = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
+  P.c1h = static_cast<float>(1.0 / std::sqrt(2.0 * static_cast<double>(D)));
+  memset(P.wn, 0, sizeof(P.wn));
+  memset(P.wd, 0, sizeof(P.wd));
+  if (flags & kFmtSrft) {
+    if (D == 64) attn_twiddles<64>(P);
+    else attn_twiddles<128>(P);
+  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (D * 1000 + group) {
-    case 64032: return launch_attn<64, 32>(P, pairs, st);
-    case 64064: return launch_attn<64, 64>(P, pairs, st);
-    case 128032: return launch_attn<128, 32>(P, pairs, st);
-    case 128064: return launch_attn<128, 64>(P, pairs, st);
-    case 128128: return launch_attn<128, 128>(P, pairs, st);
+    case 64032: return launch_fmt<64, 32>(P, pairs, flags, st);
+    case 64064: return launch_fmt<64, 64>(P, pairs, flags, st);
+    case 128032: return launch_fmt<128, 32>(P, pairs, flags, st);
+    case 128064: return launch_fmt<128, 64>(P, pairs, flags, st);
+    case 128128: return launch_fmt<128, 128>(P, pairs, flags, st);
     default: return KVQ_ERR_GROUP;
   }
+}
+
+int kvq_attention_decode(const uint16_t* q, const uint8_t* k_packed, const uint16_t* k_scales,
+                         const uint8_t* v_packed, const uint16_t* v_scales, const int32_t* seq_len,
+                         const float* lambda_k, const int8_t* signs_k, const float* lambda_v,
+                         const int8_t* signs_v, int B, int Hq, int Hkv, int T, int D, int group,
+                         float sm_scale, uint16_t* out, void* workspace, int64_t workspace_bytes,
+                         void* stream) {
+  return kvq_attention_decode_ex(q, k_packed, k_scales, v_packed, v_scales, seq_len, lambda_k,
+                                 signs_k, lambda_v, signs_v, B, Hq, Hkv, T, D, group, 0, sm_scale,
+                                 out, workspace, workspace_bytes, stream);
 }
 
 int kvq_attention_decode_static(const uint16_t* q, const uint8_t* k_packed, const uint16_t* k_scales,

@@ -49,6 +49,9 @@ _lib.kvq_dequantize_ex.argtypes = [_P, _P, _P, _P, _I64, _I, _I, _I, _I, _I64, _
 _lib.kvq_attention_decode.restype = _I
 _lib.kvq_attention_decode.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _I64, _P]
+_lib.kvq_attention_decode_ex.restype = _I
+_lib.kvq_attention_decode_ex.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                         _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P, _I64, _P]
 _lib.kvq_attention_decode_static.restype = _I
 _lib.kvq_attention_decode_static.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                              _I, _I, _I, _I, _I, _I, ctypes.c_float, _P, _P]
@@ -139,6 +142,16 @@ def kvq_attention_decode(q: int, k_packed: int, k_scales: int, v_packed: int, v_
     return _lib.kvq_attention_decode(q, k_packed, k_scales, v_packed, v_scales, seq_len,
                                      lam_k, s_k, lam_v, s_v, B, Hq, Hkv, T, D, group,
                                      sm_scale, out, workspace, workspace_bytes, stream)
+
+
+def kvq_attention_decode_ex(q: int, k_packed: int, k_scales: int, v_packed: int, v_scales: int,
+                            seq_len: int, lam_k: int, s_k: int, lam_v: int, s_v: int,
+                            B: int, Hq: int, Hkv: int, T: int, D: int, group: int, flags: int,
+                            sm_scale: float, out: int, workspace: int = 0,
+                            workspace_bytes: int = 0, stream: int = 0) -> int:
+    return _lib.kvq_attention_decode_ex(q, k_packed, k_scales, v_packed, v_scales, seq_len,
+                                        lam_k, s_k, lam_v, s_v, B, Hq, Hkv, T, D, group, flags,
+                                        sm_scale, out, workspace, workspace_bytes, stream)
 
 
 def kvq_attention_decode_static(q: int, k_packed: int, k_scales: int, v_packed: int,
@@ -331,11 +344,13 @@ def attention_decode(q: torch.Tensor, k_packed: torch.Tensor, k_scales: torch.Te
                      lam_k: torch.Tensor, s_k: torch.Tensor, lam_v: torch.Tensor,
                      s_v: torch.Tensor, group: int, sm_scale: float,
                      out: torch.Tensor | None = None, workspace: torch.Tensor | bool = True,
-                     stream=None) -> torch.Tensor:
+                     stream=None, lambda_after: bool = False, srft: bool = False) -> torch.Tensor:
     """Decode attention over the int4 cache.  q fp16 [B, Hq, D]; packed uint8
     [B, Hkv, T, D/2]; scales fp16 [B, Hkv, T, D/group]; seq_len int32 [B]
     -> fp16 [B, Hq, D].  ``workspace``: a uint8 CUDA tensor, True to allocate
-    the size the library asks for, or False to run without splitting."""
+    the size the library asks for, or False to run without splitting.
+    ``lambda_after`` / ``srft``: the cache's rows are quantize_ex rows of that
+    format (int4)."""
     if q.dim() != 3 or k_packed.dim() != 4:
         raise ValueError("q must be [B, Hq, D] and the caches [B, Hkv, T, D/2]")
     B, Hq, D = q.shape
@@ -364,11 +379,11 @@ def attention_decode(q: torch.Tensor, k_packed: torch.Tensor, k_scales: torch.Te
         if not workspace.is_cuda or workspace.dtype != torch.uint8:
             raise ValueError("workspace must be a uint8 CUDA tensor")
         ws, wsb = workspace.data_ptr(), workspace.numel()
-    rc = kvq_attention_decode(q.data_ptr(), k_packed.data_ptr(), k_scales.data_ptr(),
-                              v_packed.data_ptr(), v_scales.data_ptr(), seq_len.data_ptr(),
-                              lam_k.data_ptr(), s_k.data_ptr(), lam_v.data_ptr(), s_v.data_ptr(),
-                              B, Hq, Hkv, T, D, group, float(sm_scale), out.data_ptr(),
-                              ws, wsb, _stream_handle(stream))
+    rc = kvq_attention_decode_ex(q.data_ptr(), k_packed.data_ptr(), k_scales.data_ptr(),
+                                 v_packed.data_ptr(), v_scales.data_ptr(), seq_len.data_ptr(),
+                                 lam_k.data_ptr(), s_k.data_ptr(), lam_v.data_ptr(), s_v.data_ptr(),
+                                 B, Hq, Hkv, T, D, group, _ex_flags(lambda_after, srft),
+                                 float(sm_scale), out.data_ptr(), ws, wsb, _stream_handle(stream))
     if rc != KVQ_OK:
         raise KvqError(rc)
     return out

@@ -165,3 +165,66 @@ def test_decode_config_sampled():
         ref = _oracle(sub, 1.0 / math.sqrt(D))[0]
         got = out[b, kvh * R:(kvh + 1) * R].cpu().numpy().astype(np.float64)
         _check(got, ref)
+
+
+# ---- caches of the codec variants' formats -----------------------------------
+
+def _case_fmt(B, Hq, Hkv, T, D, G, seed, after, srft, lens=None):
+    """K and V rows that are real kvq_quantize_ex codes (int4) of Gaussian rows
+    with outlier channels, in the given format."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, Hq, D)).astype(np.float16)
+    lk, sk = workloads.params(D, seed)
+    lv, sv = workloads.params(D, seed + 1)
+    o = oracle.get()
+    x = rng.standard_normal((2, B * Hkv * T, D))
+    x[:, :, rng.permutation(D)[:4]] *= 20.0
+    x = x.astype(np.float16)
+    kp, ks = o.quantize_ex(x[0], lk, sk, G, lambda_after=after, srft=srft)
+    vp, vs = o.quantize_ex(x[1], lv, sv, G, lambda_after=after, srft=srft)
+    if lens is None:
+        lens = rng.integers(0, T + 1, B)
+    return dict(q=q, kp=kp.reshape(B, Hkv, T, D // 2), ks=ks.reshape(B, Hkv, T, D // G),
+                vp=vp.reshape(B, Hkv, T, D // 2), vs=vs.reshape(B, Hkv, T, D // G),
+                lens=np.asarray(lens, dtype=np.int32), lk=lk, sk=sk, lv=lv, sv=sv, G=G)
+
+
+FMT_CASES = [
+    # B, Hq, Hkv, T, D, G, lens
+    (3, 8, 2, 256, 128, 32, None),
+    (2, 4, 4, 96, 64, 32, [96, 17]),
+    (4, 32, 8, 80, 128, 64, [0, 1, 80, 33]),
+    (1, 2, 1, 400, 128, 128, [400]),
+]
+
+
+@pytest.mark.parametrize("after,srft", [(True, False), (False, True), (True, True)])
+@pytest.mark.parametrize("case", FMT_CASES)
+def test_attention_formats_match_oracle(case, after, srft):
+    """The paper's cache format (SRFT, lambda after) and the other variants:
+    the query rotated to the cache's domain once, the output rotated back once
+    per head, against the oracle's double-precision definition on the same
+    rows; with and without the key-axis split."""
+    B, Hq, Hkv, T, D, G, lens = case
+    c = _case_fmt(B, Hq, Hkv, T, D, G, seed=B * T + D + int(after) + 2 * int(srft),
+                  after=after, srft=srft, lens=lens)
+    ref = oracle.get().attention_decode(c["q"], c["kp"], c["ks"], c["vp"], c["vs"], c["lens"],
+                                        c["lk"], c["sk"], c["lv"], c["sv"], G, 0.0883,
+                                        lambda_after=after, srft=srft)
+    dev = torch.device("cuda")
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    for ws in (True, False):
+        out = kvq.attention_decode(t(c["q"]), t(c["kp"]), t(c["ks"]), t(c["vp"]), t(c["vs"]),
+                                   t(c["lens"]), t(c["lk"]), t(c["sk"]), t(c["lv"]), t(c["sv"]),
+                                   G, 0.0883, workspace=ws, lambda_after=after, srft=srft)
+        torch.cuda.synchronize()
+        _check(out.cpu().numpy().astype(np.float64), ref)
+
+
+def test_attention_formats_reject_bad_flags():
+    c = _case(1, 2, 1, 16, 128, 32, seed=3)
+    dev = torch.device("cuda")
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    args = [t(c[k]).data_ptr() for k in ("q", "kp", "ks", "vp", "vs", "lens", "lk", "sk", "lv", "sv")]
+    out = torch.empty((1, 2, 128), dtype=torch.float16, device=dev)
+    assert kvq.kvq_attention_decode_ex(*args, 1, 2, 1, 16, 128, 32, 4, 0.1, out.data_ptr()) == kvq.KVQ_ERR_GROUP
