@@ -295,6 +295,8 @@ def run_gpu(args):
     extra = {}
     if args.variants_only:
         extra = {"codec_variants": run_variants(torch, kvq, dev, stream, x, out, s_t, G, w)}
+        if w.D == 128:
+            extra["srft_lengths"] = run_srft_lengths(torch, kvq, dev, stream)
     elif args.roundtrip_only:
         rt_ms = _event_ms(torch, stream,
                           lambda: kvq.roundtrip(x, lam_t, s_t, G, out=out, stream=stream), 10)
@@ -403,8 +405,10 @@ def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, attn_seqs=64):
         "decode_append_us": round(ap_ms * 1e3, 2),
         "decode_append_gvec_s": round(na / (ap_ms / 1e3) / 1e9, 3),
     }
+    res["sustained"] = run_sustained(torch, kvq, dev, stream, x, out, lam_t, s_t, G)
     if D == 128:
         res["codec_variants"] = run_variants(torch, kvq, dev, stream, x, out, s_t, G, w)
+        res["srft_lengths"] = run_srft_lengths(torch, kvq, dev, stream)
         cache = build_decode_cache(torch, kvq, dev, stream, lam_t, s_t, G, attn_seqs)
         res["attention_decode"] = run_attention(torch, kvq, dev, stream, lam_t, s_t, G, cache)
         res["decode_step"] = run_decode_step(torch, kvq, dev, stream, lam_t, s_t, G, cache,
@@ -544,6 +548,86 @@ def run_variants(torch, kvq, dev, stream, x, out, s_t, G, w):
         }
         del codes, scales
     return res
+
+
+def run_srft_lengths(torch, kvq, dev, stream, G=32, in_bytes=1 << 31):
+    """The paper's codec configuration (SRFT rotation, lambda after it, int4
+    codes; \"When Quantization Is Free\", technical summary, Methodologie 1-2)
+    at every length it runs: D = 64, 96 (mixed radix), 128 and 256, on 2 GiB
+    of fp16 rows each (above L2), one lambda table.  Algorithmic bytes per
+    vector: 2D + D/2 + 2D/G."""
+    import numpy as np
+    peak, _ = hbm_peak()
+    res = {"group": G, "fp16_input_bytes": in_bytes}
+    for D in (64, 96, 128, 256):
+        n = in_bytes // (2 * D)
+        gen = torch.Generator(device=dev).manual_seed(D)
+        x = (torch.randn((n, D), generator=gen, device=dev) * 2.0).to(torch.float16)
+        rng = np.random.default_rng(D)
+        lam = torch.from_numpy(rng.uniform(0.5, 2.0, D).astype(np.float32)).to(dev)
+        sg = torch.from_numpy(np.where(rng.random(D) < 0.5, -1, 1).astype(np.int8)).to(dev)
+        codes = torch.empty((n, D // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((n, D // G), dtype=torch.float16, device=dev)
+        out = torch.empty_like(x)
+        q_ms = _event_ms(torch, stream, lambda: kvq.quantize_ex(
+            x, lam, sg, G, lambda_after=True, srft=True, codes=codes, scales=scales,
+            stream=stream), 10)
+        d_ms = _event_ms(torch, stream, lambda: kvq.dequantize_ex(
+            codes, scales, lam, sg, G, lambda_after=True, srft=True, out=out, stream=stream), 10)
+        bpv = bytes_per_vector(D, G)
+        qg, dg = bpv * n / (q_ms / 1e3) / 1e9, bpv * n / (d_ms / 1e3) / 1e9
+        res[f"d{D}"] = {
+            "n_vec": n, "bytes_per_vector": bpv,
+            "quantize_ms": round(q_ms, 4), "quantize_gvec_s": round(n / (q_ms / 1e3) / 1e9, 3),
+            "quantize_gbs": round(qg, 1), "quantize_frac_of_peak": round(qg / peak, 4),
+            "dequantize_ms": round(d_ms, 4), "dequantize_gvec_s": round(n / (d_ms / 1e3) / 1e9, 3),
+            "dequantize_gbs": round(dg, 1), "dequantize_frac_of_peak": round(dg / peak, 4),
+        }
+        del x, codes, scales, out
+        torch.cuda.empty_cache()
+    return res
+
+
+def run_sustained(torch, kvq, dev, stream, x, out, lam_t, s_t, G, seconds=1.5):
+    """Quantize and dequantize of the main batch back to back for about
+    `seconds`, each launch timed by CUDA events: the sustained figure under
+    the board's power cap, with the SM clocks sampled during the loop."""
+    n, D = x.shape
+    packed = torch.empty((n, D // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((n, D // G), dtype=torch.float16, device=dev)
+    kvq.quantize(x, lam_t, s_t, G, packed=packed, scales=scales, stream=stream)
+    kvq.dequantize(packed, scales, lam_t, s_t, G, out=out, stream=stream)
+    torch.cuda.synchronize(dev)
+    # size the loop from one timed pair
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    kvq.quantize(x, lam_t, s_t, G, packed=packed, scales=scales, stream=stream)
+    kvq.dequantize(packed, scales, lam_t, s_t, G, out=out, stream=stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    reps = max(20, int(seconds * 1e3 / max(t0.elapsed_time(t1), 1e-3)))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps + 1)]
+    with ClockSampler(dev.index) as clocks:
+        ev[0].record(stream)
+        for i in range(reps):
+            kvq.quantize(x, lam_t, s_t, G, packed=packed, scales=scales, stream=stream)
+            ev[2 * i + 1].record(stream)
+            kvq.dequantize(packed, scales, lam_t, s_t, G, out=out, stream=stream)
+            ev[2 * i + 2].record(stream)
+        torch.cuda.synchronize(dev)
+    qt = sorted(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(reps))
+    dt = sorted(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(reps))
+    total_s = ev[0].elapsed_time(ev[-1]) / 1e3
+    bpv = bytes_per_vector(D, G)
+    qm, dm = qt[len(qt) // 2], dt[len(dt) // 2]
+    del packed, scales
+    return {
+        "reps": reps, "seconds": round(total_s, 3),
+        "quantize_ms_median": round(qm, 5), "dequantize_ms_median": round(dm, 5),
+        "quantize_gbs": round(bpv * n / (qm / 1e3) / 1e9, 1),
+        "dequantize_gbs": round(bpv * n / (dm / 1e3) / 1e9, 1),
+        "clocks": clocks.summary(),
+    }
 
 
 DECODE_HQ, DECODE_HKV, DECODE_T = 32, 8, 4096
