@@ -44,7 +44,11 @@ constexpr unsigned kFullMask = 0xffffffffu;
 #include "kvq_ex.cuh"
 #include "kvq_fft.cuh"
 
-constexpr int kDW = 8;                  // warps of a block (one block per SM)
+// Warps of a block (one block per SM): 12, whose 168 registers a thread the
+// one-lane kernels fit with a few bytes of spill; 8 for the D = 256
+// dequantiser, whose two-lane unpacking keeps more values live.
+template <int D, bool DEQ>
+__host__ __device__ constexpr int sr_warps() { return (D == 256 && DEQ) ? 8 : 12; }
 constexpr uint32_t kSpinX = 1u << 22;   // bounded mbarrier waits
 
 __device__ unsigned int g_ex_fault = 0;   // bit 0: a bounded wait gave up
@@ -282,12 +286,13 @@ __device__ __forceinline__ void unpack_inv256(float2 (&z)[64], const float2* wd,
 
 // ---- quantize ------------------------------------------------------------
 template <int D, int G, int BITS, bool AFTER>
-__global__ void __launch_bounds__(kDW * 32, 1)
+__global__ void __launch_bounds__(sr_warps<D, false>() * 32, 1)
 kvq_quantize_srft_kernel(const __grid_constant__ SrMaps maps, const ExArgs a,
                          const __grid_constant__ SrTw<D> tw, float c0, float c1h,
                          const __grid_constant__ CUtensorMap cmap, uint16_t* __restrict__ scales) {
   using S = Sr<D>;
   using F = SrFmt<D, BITS>;
+  constexpr int kDW = sr_warps<D, false>();
   constexpr int NG = D / G;             // groups per row
   constexpr int GL = G / 2 / S::LANES;  // pairs of a group a lane holds
   constexpr int NLW = F::CB / 4 / S::LANES;   // code words a lane forms
@@ -560,12 +565,13 @@ __device__ __forceinline__ void sr_decode_word(uint32_t w, float2* z, const uint
 }
 
 template <int D, int G, int BITS, bool AFTER>
-__global__ void __launch_bounds__(kDW * 32, 1)
+__global__ void __launch_bounds__(sr_warps<D, true>() * 32, 1)
 kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
                            const ExArgs a, const __grid_constant__ SrTw<D> tw, float c0, float c1h,
                            const __grid_constant__ SrMaps omaps, int scale_copy) {
   using S = Sr<D>;
   using L = SrDeq<D, G, BITS>;
+  constexpr int kDW = sr_warps<D, true>();
   constexpr int NG = D / G;
   constexpr int GL = G / 2 / S::LANES;  // pairs of a group a lane holds
   constexpr int CB = L::CB;
@@ -830,14 +836,14 @@ int sr_sms(int& dev) {
 
 // Grid: one block per resident slot, at most one per warp tile.
 template <typename Kernel>
-int sr_grid(Kernel k, int64_t tiles, int smem, std::atomic<int>* ready) {
+int sr_grid(Kernel k, int64_t tiles, int smem, int threads, std::atomic<int>* ready) {
   int dev = 0;
   const int sms = sr_sms(dev);
   int occ = ready[dev].load(std::memory_order_relaxed);
   if (occ == 0) {
     cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kDW * 32, smem) != cudaSuccess || occ < 1) occ = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, threads, smem) != cudaSuccess || occ < 1) occ = 1;
     ready[dev].store(occ, std::memory_order_relaxed);
   }
   const int64_t cap = static_cast<int64_t>(sms) * occ;
@@ -862,11 +868,13 @@ int launch_sq(const uint16_t* x, const ExArgs& a, uint8_t* codes, uint16_t* scal
   rc = sr_encode_code_map<D, BITS>(cmap, codes, a.n);
   if (rc != KVQ_OK) return rc;
   auto k = kvq_quantize_srft_kernel<D, G, BITS, AFTER>;
-  constexpr int smem = 1024 + kDW * 2 * S::TILE + sr_hdr_bytes<D>(kDW);
+  constexpr int nw = sr_warps<D, false>();
+  constexpr int smem = 1024 + nw * 2 * S::TILE + sr_hdr_bytes<D>(nw);
+  static_assert(smem <= 227 * 1024, "shared memory");
   static std::atomic<int> ready[64];
-  const int grid = sr_grid(k, (a.n + S::WR - 1) / S::WR, smem, ready);
+  const int grid = sr_grid(k, (a.n + S::WR - 1) / S::WR, smem, nw * 32, ready);
   (void)cudaGetLastError();
-  k<<<grid, kDW * 32, smem, st>>>(maps, a, sr_twiddles<D>(), sr_c0(D), sr_c1h(D), cmap, scales);
+  k<<<grid, nw * 32, smem, st>>>(maps, a, sr_twiddles<D>(), sr_c0(D), sr_c1h(D), cmap, scales);
   return sr_finish();
 }
 
@@ -879,11 +887,13 @@ int launch_sd(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, uin
   const int rc = sr_encode_x_maps<D>(omaps, out, a.n);
   if (rc != KVQ_OK) return rc;
   auto k = kvq_dequantize_srft_kernel<D, G, BITS, AFTER>;
-  constexpr int smem = 1024 + kDW * L::WARP + sr_hdr_bytes<D>(kDW);
+  constexpr int nw = sr_warps<D, true>();
+  constexpr int smem = 1024 + nw * L::WARP + sr_hdr_bytes<D>(nw);
+  static_assert(smem <= 227 * 1024, "shared memory");
   static std::atomic<int> ready[64];
-  const int grid = sr_grid(k, (a.n + S::WR - 1) / S::WR, smem, ready);
+  const int grid = sr_grid(k, (a.n + S::WR - 1) / S::WR, smem, nw * 32, ready);
   (void)cudaGetLastError();
-  k<<<grid, kDW * 32, smem, st>>>(codes, scales, a, sr_twiddles<D>(), sr_c0(D), sr_c1h(D), omaps,
+  k<<<grid, nw * 32, smem, st>>>(codes, scales, a, sr_twiddles<D>(), sr_c0(D), sr_c1h(D), omaps,
                                   (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
   return sr_finish();
 }
