@@ -518,8 +518,9 @@ int kvqo_attention_decode(const uint16_t *q, const uint8_t *k_packed,
 /* X = DFT(v).  Readings of the arithmetic:                             */
 /*  - twiddles are the fp32 values nearest the exact roots of unity;    */
 /*    a product by 1, -1, i or -i is exact (the operand, negated or     */
-/*    with its parts swapped); any other complex product is four fp32   */
-/*    products and two fp32 sums, re = dr wr - di wi, im = dr wi + di wr;*/
+/*    with its parts swapped); in any other complex product each part   */
+/*    is one rounded product and one fused multiply-add:                */
+/*    re = fma(dr, wr, -rn(di wi)), im = fma(di, wr, rn(dr wi));        */
 /*  - the unpacking forms 2 X_k (its factor 1/2 goes into the           */
 /*    normalisation), scaled by fp32(1/sqrt(2D)); X_0 and X_N are       */
 /*    scaled by fp32(1/sqrt(D));                                        */
@@ -567,9 +568,9 @@ static void cmul(float dr, float di, float wr, float wi, float *pr, float *pi_)
         *pr = (wi > 0.0f) ? -di : di;
         *pi_ = (wi > 0.0f) ? dr : -dr;
     } else {
-        float a = dr * wr, b = di * wi, c = dr * wi, e = di * wr;
-        *pr = a - b;
-        *pi_ = c + e;
+        float b = di * wi, c = dr * wi;                 /* rounded products */
+        *pr = fmaf(dr, wr, -b);                         /* dr wr - di wi */
+        *pi_ = fmaf(di, wr, c);                         /* di wr + dr wi */
     }
 }
 

@@ -55,6 +55,8 @@ MUTANTS = [
     ("twiddle_complement", "if (comp) { float t = c; c = s; s = t; }", "(void)comp;", 0),
     ("twiddle_signed_zero", "    *wr = cr + 0.0f;                            /* -0 -> +0 */", "    *wr = cr;", 0),
     ("cmul_trivial_i_sign", "*pr = (wi > 0.0f) ? -di : di;", "*pr = (wi > 0.0f) ? di : -di;", 0),
+    ("cmul_fused_sign", "*pr = fmaf(dr, wr, -b);", "*pr = fmaf(dr, wr, b);", 0),
+    ("cmul_fused_operand", "*pi_ = fmaf(di, wr, c);", "*pi_ = fmaf(di, wi, c);", 0),
     ("srft_no_sqrt2", "(float)(1.0 / sqrt(2.0 * (double)D))", "(float)(1.0 / sqrt((double)D))", 0),
     ("srft_stage_stride", "kvqo_twiddle(s * p * t, N, &wr, &wi);               /* omega_n^(p t) */",
      "kvqo_twiddle(p * t, N, &wr, &wi);", 0),
