@@ -18,7 +18,10 @@ __device__ __forceinline__ void sfor(Fn&& f) {
 }
 
 // d * omega_M^K, or d * conj(omega_M^K) (CONJ), K known at compile time; w is
-// the table of omega_M.
+// the table of omega_M.  A product by 1, -1, i or -i is exact (the operand,
+// negated or with its parts swapped); any other is one rounded product and
+// one fused multiply-add per part: re = fma(d.x, w.x, -rn(d.y w.y)),
+// im = fma(d.y, w.x, rn(d.x w.y)).
 template <int K, int M, bool CONJ>
 __device__ __forceinline__ float2 twmul(float2 d, const float2* w) {
   constexpr int k = K % M;
@@ -28,26 +31,17 @@ __device__ __forceinline__ float2 twmul(float2 d, const float2* w) {
     else if constexpr (e == 1) return make_float2(d.y, -d.x);
     else if constexpr (e == 2) return make_float2(-d.x, -d.y);
     else return make_float2(-d.y, d.x);
-  } else if constexpr ((8 * k) % M == 0) {                // odd multiple of pi/4
-    constexpr int o = (8 * k) / M;
-    constexpr float sr = (o == 1 || o == 7) ? 1.0f : -1.0f;          // sign of Re w
-    constexpr float si0 = (o == 1 || o == 3) ? -1.0f : 1.0f;         // sign of Im w
-    constexpr float si = CONJ ? -si0 : si0;
-    const float c = fabsf(w[k].x);
-    const float2 pq = __fmul2_rn(d, make_float2(c, c));              // |products|
-    return make_float2(__fadd_rn(sr * pq.x, -si * pq.y), __fadd_rn(si * pq.x, sr * pq.y));
   } else {
     const float2 t = w[k];
     const float ty = CONJ ? -t.y : t.y;
-    const float2 p0 = __fmul2_rn(d, make_float2(t.x, t.x));          // (d.x wx, d.y wx)
-    const float2 p1 = __fmul2_rn(d, make_float2(ty, ty));            // (d.x wy, d.y wy)
-    return make_float2(__fsub_rn(p0.x, p1.y), __fadd_rn(p1.x, p0.y));
+    const float b = __fmul_rn(d.y, ty), c = __fmul_rn(d.x, ty);
+    return make_float2(__fmaf_rn(d.x, t.x, -b), __fmaf_rn(d.y, t.x, c));
   }
 }
 
 // omega_M^K (d / i), the forward unpacking's odd part, d / i = (d.y, -d.x):
-// re = d.y wx + d.x wy, im = d.y wy - d.x wx, the same roundings as the four
-// products of (d / i) w.
+// re = fma(d.y, wx, rn(d.x wy)), im = fma(-d.x, wx, rn(d.y wy)), the same
+// roundings as the product of (d / i) and w.
 template <int K, int M>
 __device__ __forceinline__ float2 twmul_odiv(float2 d, const float2* w) {
   constexpr int k = K % M;
@@ -55,21 +49,19 @@ __device__ __forceinline__ float2 twmul_odiv(float2 d, const float2* w) {
     return twmul<K, M, false>(make_float2(d.y, -d.x), w);
   } else {
     const float2 t = w[k];
-    const float2 p0 = __fmul2_rn(d, make_float2(t.x, t.x));
-    const float2 p1 = __fmul2_rn(d, make_float2(t.y, t.y));
-    return make_float2(__fadd_rn(p0.y, p1.x), __fsub_rn(p1.y, p0.x));
+    const float p = __fmul_rn(d.x, t.y), q = __fmul_rn(d.y, t.y);
+    return make_float2(__fmaf_rn(d.y, t.x, p), __fmaf_rn(-d.x, t.x, q));
   }
 }
-// The same with a twiddle known only at run time (general roundings).
+// The same with a twiddle known only at run time (never 1, -1, i or -i).
 __device__ __forceinline__ float2 twmul_odiv_rt(float2 d, float2 t) {
-  const float2 p0 = __fmul2_rn(d, make_float2(t.x, t.x));
-  const float2 p1 = __fmul2_rn(d, make_float2(t.y, t.y));
-  return make_float2(__fadd_rn(p0.y, p1.x), __fsub_rn(p1.y, p0.x));
+  const float p = __fmul_rn(d.x, t.y), q = __fmul_rn(d.y, t.y);
+  return make_float2(__fmaf_rn(d.y, t.x, p), __fmaf_rn(-d.x, t.x, q));
 }
 __device__ __forceinline__ float2 twmul_conj_rt(float2 d, float2 t) {
-  const float2 p0 = __fmul2_rn(d, make_float2(t.x, t.x));
-  const float2 p1 = __fmul2_rn(d, make_float2(-t.y, -t.y));
-  return make_float2(__fsub_rn(p0.x, p1.y), __fadd_rn(p1.x, p0.y));
+  const float ty = -t.y;
+  const float b = __fmul_rn(d.y, ty), c = __fmul_rn(d.x, ty);
+  return make_float2(__fmaf_rn(d.x, t.x, -b), __fmaf_rn(d.y, t.x, c));
 }
 
 // ---- Stockham stages on an L-point register array -------------------------

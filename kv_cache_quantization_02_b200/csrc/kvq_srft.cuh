@@ -65,9 +65,8 @@ __device__ unsigned int g_ex_fault = 0;   // bit 0: a bounded wait gave up
 // operation, the reading the oracle states:
 //   * twiddles are the fp32 values nearest the exact roots of unity (built on
 //     the host); a product by 1, -1, i or -i is exact (the operand, negated or
-//     with its parts swapped); any other complex product is four fp32
-//     products and two fp32 sums (at the odd multiples of pi/4, where
-//     |re w| = |im w|, the four products are two with the same roundings);
+//     with its parts swapped); in any other complex product each part is one
+//     rounded product and one fused multiply-add;
 //   * the unpacking forms bins k and N-k together: E = Z_k + conj Z_(N-k),
 //     O = (Z_k - conj Z_(N-k)) / i, T = omega_D^k O, 2 X_k = E + T,
 //     2 X_(N-k) = conj(E - T); its factor 1/2 sits in the normalisation,
