@@ -297,6 +297,10 @@ def run_gpu(args):
         extra = {"codec_variants": run_variants(torch, kvq, dev, stream, x, out, s_t, G, w)}
         if w.D == 128:
             extra["srft_lengths"] = run_srft_lengths(torch, kvq, dev, stream)
+    elif args.attention_only:
+        cache = build_decode_cache(torch, kvq, dev, stream, lam_t, s_t, G, args.attn_seqs)
+        extra = {"attention_decode": run_attention(torch, kvq, dev, stream, lam_t, s_t, G, cache)}
+        del cache
     elif args.roundtrip_only:
         rt_ms = _event_ms(torch, stream,
                           lambda: kvq.roundtrip(x, lam_t, s_t, G, out=out, stream=stream), 10)
@@ -842,6 +846,8 @@ def parse(argv=None):
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--no-extra", action="store_true", help="skip round-trip, append and attention figures")
+    p.add_argument("--attention-only", action="store_true",
+                   help="of the secondary figures, only the decode attention (profiling)")
     p.add_argument("--variants-only", action="store_true",
                    help="of the secondary figures, only the codec variants (profiling)")
     p.add_argument("--roundtrip-only", action="store_true",
