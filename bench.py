@@ -44,7 +44,7 @@ from kv_cache_quantization_02_b200 import workloads  # noqa: E402
 METRIC = "Gvec/s quantize+pack and dequant at D=128; achieved HBM GB/s vs B200 peak"
 UNIT = "Gvec/s"
 FALLBACK_HBM_GBS = 6650.0
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "kvq_traffic_full_size.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "kvq_traffic_slices.json")
 
 
 def bytes_per_vector(D: int, G: int) -> int:
