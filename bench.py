@@ -215,6 +215,13 @@ class OracleTimer:
         x16 = np.concatenate([pool] * reps)[: self.rows]
         self.parts = [np.ascontiguousarray(p) for p in np.array_split(x16, self.threads)]
 
+    def set_rows(self, n: int, w: workloads.Workload):
+        """Time exactly the n rows of workload w (drawn on the host)."""
+        import numpy as np
+        x16 = workloads.host_rows(w, n, seed_offset=79)
+        self.rows = n
+        self.parts = [np.ascontiguousarray(p) for p in np.array_split(x16, self.threads) if len(p)]
+
     def _one(self, x16):
         packed, scales = self.o.quantize(x16, self.lam, self.s, self.G)
         self.o.dequantize(packed, scales, self.lam, self.s, self.G)
@@ -225,6 +232,28 @@ class OracleTimer:
             t0 = time.perf_counter()
             list(ex.map(self._one, self.parts))
             return time.perf_counter() - t0
+
+
+def oracle_extra_timings(w, G, target_s):
+    """The oracle on one thread (a bounded sample of the same workload, a
+    tenth of the time budget), and the three smaller configurations timed in
+    full on all host threads: tiny (256 vectors), qwen2.5-1.5b (458,752) and
+    gemma-3-1b (212,992, D = 256, G = 32 and 64)."""
+    one = OracleTimer(w, G, max(target_s / 10.0, 0.5), threads=1)
+    dt1 = one.run()
+    res = {"single_thread": {"value": one.rows / dt1 / 1e9, "unit": UNIT,
+                             "sample": f"{one.rows} vectors, {dt1:.2f} s on 1 thread"}}
+    full = {}
+    for name, groups in (("tiny", None), ("qwen2.5-1.5b", None), ("gemma-3-1b", (32, 64))):
+        c = workloads.WORKLOADS[name]
+        for g in groups or (c.groups[0],):
+            ot = OracleTimer(c, g, 0.0)
+            ot.set_rows(c.n_vec, c)
+            dt = ot.run()
+            full[f"{name}_g{g}"] = {"vectors": c.n_vec, "seconds": round(dt, 4),
+                                    "gvec_s": c.n_vec / dt / 1e9, "threads": ot.threads}
+    res["configs_full"] = full
+    return res
 
 
 # ---------------------------------------------------------------------------
@@ -329,7 +358,8 @@ def run_gpu(args):
         cpu = {"value": ot.rows / dt / 1e9, "unit": UNIT, "cores": ot.threads,
                "kind": "oracle",
                "sample": f"{ot.rows} vectors of the {w.name} distribution (host-drawn), "
-                         f"quantize+dequantize, {dt:.1f} s on {ot.threads} threads"}
+                         f"quantize+dequantize, {dt:.1f} s on {ot.threads} threads",
+               **oracle_extra_timings(w, G, args.cpu_seconds)}
 
     if world > 1:
         import torch.distributed as dist
