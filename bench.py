@@ -330,6 +330,8 @@ def run_gpu(args):
         cache = build_decode_cache(torch, kvq, dev, stream, lam_t, s_t, G, args.attn_seqs)
         extra = {"attention_decode": run_attention(torch, kvq, dev, stream, lam_t, s_t, G, cache)}
         del cache
+    elif args.tc_only:
+        extra = {"dequantize_tensor_cores": run_dequant_tc(torch, kvq, dev, stream, x, out, lam_t, s_t)}
     elif args.roundtrip_only:
         rt_ms = _event_ms(torch, stream,
                           lambda: kvq.roundtrip(x, lam_t, s_t, G, out=out, stream=stream), 10)
@@ -442,6 +444,7 @@ def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, attn_seqs=64):
     res["sustained"] = run_sustained(torch, kvq, dev, stream, x, out, lam_t, s_t, G)
     if D == 128:
         res["codec_variants"] = run_variants(torch, kvq, dev, stream, x, out, s_t, G, w)
+        res["dequantize_tensor_cores"] = run_dequant_tc(torch, kvq, dev, stream, x, out, lam_t, s_t)
         res["srft_lengths"] = run_srft_lengths(torch, kvq, dev, stream)
         cache = build_decode_cache(torch, kvq, dev, stream, lam_t, s_t, G, attn_seqs)
         res["attention_decode"] = run_attention(torch, kvq, dev, stream, lam_t, s_t, G, cache)
@@ -581,6 +584,33 @@ def run_variants(torch, kvq, dev, stream, x, out, s_t, G, w):
             "dequantize_frac_of_peak": round(dg / peak, 4),
         }
         del codes, scales
+    return res
+
+
+def run_dequant_tc(torch, kvq, dev, stream, x, out, lam_t, s_t):
+    """The dequantizer with the in-group Hadamard on the tensor cores beside
+    the butterfly dequantizer, on the same batch for G = 16, 32, 64: times,
+    HBM fraction, and whether the two outputs are the same bytes."""
+    n, D = x.shape
+    peak, _ = hbm_peak()
+    res = {}
+    out2 = torch.empty_like(out)
+    for G in (16, 32, 64):
+        pk, sc = kvq.quantize(x, lam_t, s_t, G, stream=stream)
+        b_ms = _event_ms(torch, stream, lambda: kvq.dequantize(
+            pk, sc, lam_t, s_t, G, out=out, stream=stream), 10)
+        t_ms = _event_ms(torch, stream, lambda: kvq.dequantize(
+            pk, sc, lam_t, s_t, G, out=out2, stream=stream, tensor_cores=True), 10)
+        torch.cuda.synchronize()
+        bpv = 2 * D + D // 2 + 2 * (D // G)
+        bg, tg = bpv * n / (b_ms / 1e3) / 1e9, bpv * n / (t_ms / 1e3) / 1e9
+        res[f"G{G}"] = {
+            "butterfly_ms": round(b_ms, 4), "butterfly_frac_of_peak": round(bg / peak, 4),
+            "tensor_core_ms": round(t_ms, 4), "tensor_core_frac_of_peak": round(tg / peak, 4),
+            "same_bytes": bool(torch.equal(out.view(torch.int16), out2.view(torch.int16))),
+        }
+        del pk, sc
+    del out2
     return res
 
 
@@ -880,6 +910,8 @@ def parse(argv=None):
                    help="of the secondary figures, only the decode attention (profiling)")
     p.add_argument("--variants-only", action="store_true",
                    help="of the secondary figures, only the codec variants (profiling)")
+    p.add_argument("--tc-only", action="store_true",
+                   help="of the secondary figures, only the tensor-core dequantizer (profiling)")
     p.add_argument("--roundtrip-only", action="store_true",
                    help="of the secondary figures, only the fused round trip (profiling)")
     p.add_argument("--attn-seqs", type=int, default=64, help="sequences of the attention figure (profiling)")

@@ -134,6 +134,23 @@ int kvq_dequantize(const uint8_t *packed, const uint16_t *scales,
                    uint16_t *x_out, void *stream);
 
 /*
+ * kvq_dequantize_tc -- kvq_dequantize with the Walsh-Hadamard transform's
+ * in-group factor on the tensor cores, bit-identical to kvq_dequantize.
+ * H_D = (H_(D/G) (x) I_G)(I_(D/G) (x) H_G): inside a group u = q S stays an
+ * exact multiple of S, so H_G q is a sum of small integers that a tensor-core
+ * product with fp16 codes and a +-1 matrix (fp32 accumulation) gets exactly;
+ * the stages that cross groups run as fp32 butterflies in the contract's
+ * order.  (The pages' "16x16 matrix-multiply alignment", technical summary,
+ * Methodologie 1, "Redenering"; a variant kept beside the butterfly kernel.)
+ * Same arguments, layouts and results as kvq_dequantize; D must be 128 (else
+ * KVQ_ERR_DIM) and group 16, 32 or 64 (else KVQ_ERR_GROUP).
+ */
+int kvq_dequantize_tc(const uint8_t *packed, const uint16_t *scales,
+                      const float *lambda, const int8_t *signs,
+                      int64_t n_vec, int D, int group,
+                      uint16_t *x_out, void *stream);
+
+/*
  * kvq_roundtrip -- x_hat = kvq_dequantize(kvq_quantize(x)) in one pass over
  * x (the quantise-then-dequantise shape used to simulate the cache's error
  * on the fly), bit-identical to the two calls back to back.

@@ -677,6 +677,223 @@ kvq_dequantize_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* 
 
 
 // ---------------------------------------------------------------------------
+// Dequantize with the in-group Hadamard on the tensor cores (D = 128, G in
+// {16, 32, 64}): the same result as kvq_dequantize_kernel, bit for bit.
+//
+// H_128 = (H_(128/G) (x) I_G)(I_(128/G) (x) H_G): the butterfly stages with
+// half-width h < G act inside a group, and there u = q S stays an exact
+// multiple of S, so W = H_G q is a sum of small integers (|W| <= 8 G) that
+// any order of addition gets exactly; u = W S is exact in fp32.  The tensor
+// cores take that factor: per 16 vectors and 16 channels one m16n8k16 fp16
+// MMA with the codes as A (exact small integers) and a 16 x 8 block of
+// H_G = H_(G/16) (x) H_16 as B (entries +-1), fp32 accumulation (exact).
+// The stages that cross groups (h >= G) then run as fp32 butterflies in the
+// oracle's order.  In the accumulator layout a lane holds, for two vectors,
+// the channels 8 nt + 2t, 8 nt + 2t + 1 of every n-tile nt, so the partners
+// of those stages (channels apart by a multiple of G >= 16) sit in the same
+// lane: no shuffle.  Streaming, tiles, tables and the staged tensor stores
+// are the butterfly dequantizer's.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+               : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+               : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Byte t of the code word w (two nibbles: channel 2b, then 2b + 1) as an
+// fp16 pair of exact integers in [-8, 7], low half first.
+__device__ __forceinline__ uint32_t code_pair_f16(uint32_t w, int t) {
+  const uint32_t wb = w ^ 0x88888888u;
+  const uint32_t e = (__byte_perm(wb, wb >> 4, 0x0400u | (t << 8) | t) & 0x000F000Fu) | 0x64006400u;
+  const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&e), __floats2half2_rn(1032.0f, 1032.0f));
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// (+-1, +-1) fp16 pair: H_16[i][j], H_16[i + 1][j].
+__device__ __forceinline__ uint32_t h16_pair(int i, int j) {
+  const uint32_t lo = (__popc(i & j) & 1) ? 0xBC00u : 0x3C00u;
+  const uint32_t hi = (__popc((i + 1) & j) & 1) ? 0xBC00u : 0x3C00u;
+  return lo | (hi << 16);
+}
+
+template <int G, int NW>
+__global__ void __launch_bounds__(NW * 32, 1)
+kvq_dequantize_tc_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* __restrict__ scales,
+                         const float* __restrict__ lam, const int8_t* __restrict__ sgn,
+                         int64_t n, float c, const __grid_constant__ RowMaps maps, int scale_copy) {
+  constexpr int D = 128;
+  static_assert(G == 16 || G == 32 || G == 64, "in-group Hadamard as 16 x 16 tiles");
+  using W = WTile<D>;
+  using L = Stream<D>;
+  constexpr int WROWS = W::WROWS;                // 32 vectors per warp tile
+  constexpr int WPIN = W::WPIN;
+  constexpr int NG = D / G;                      // groups per row
+  constexpr int SPR = NG * 2;                    // scale bytes per row
+  constexpr int WSC = kScaleBlock;
+  constexpr int KG = G / 16;                     // k-steps per group
+  constexpr int NTG = G / 8;                     // n-tiles per group
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  uint8_t* hdr = smem + NW * L::DWARP;
+  float4* tabw = reinterpret_cast<float4*>(hdr);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + L::BARS) + 2 * warp;
+  int* tq = reinterpret_cast<int*>(hdr + L::TQ) + 2 * warp;
+  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + L::NEXT);
+  uint8_t* stage_out = smem + warp * L::DWARP;
+  uint8_t* stage_in = stage_out + W::WSTAGE;
+  uint8_t* stage_sc = stage_in + 2 * WPIN;
+  fill_tab<D>(tabw, lam, sgn, true);             // s * fp32(1/lambda), pair layout of the butterfly kernels
+  if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
+  if (tid == 0) *next = 0;
+  __syncthreads();
+
+  // B fragments: the two 16 x 8 column blocks of H_16 (and their negatives)
+  const uint32_t hb[2][2] = {{h16_pair(2 * t, g), h16_pair(2 * t + 8, g)},
+                             {h16_pair(2 * t, 8 + g), h16_pair(2 * t + 8, 8 + g)}};
+
+  const int64_t ntiles = (n + WROWS - 1) / WROWS;
+  const unsigned int mine = static_cast<unsigned int>((ntiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+  auto claim = [&]() -> int {
+    unsigned int i = 0;
+    if (lane == 0) i = atomicAdd(next, 1u);
+    i = __shfl_sync(kFullMask, i, 0);
+    return i < mine ? static_cast<int>(blockIdx.x + i * gridDim.x) : -1;
+  };
+  auto scale_bytes = [&](int64_t tile) -> uint32_t {
+    if (!scale_copy) return 0;
+    const int64_t row0 = tile * WROWS;
+    const int valid = static_cast<int>(n - row0 < WROWS ? n - row0 : WROWS);
+    return static_cast<uint32_t>(valid * SPR) & ~15u;
+  };
+  auto issue = [&](int64_t tile, int stage) {
+    if (tile < 0 || lane != 0) return;
+    const int64_t row0 = tile * WROWS;
+    const uint32_t sb = scale_bytes(tile);
+    mbar_expect_tx(&bar[stage], static_cast<uint32_t>(WPIN) + sb);
+    tensor_g2s(stage_in + stage * WPIN, &cmap, 0, static_cast<int>(row0), &bar[stage]);
+    if (sb) bulk_g2s(stage_sc + stage * WSC, reinterpret_cast<const uint8_t*>(scales) + row0 * SPR, sb, &bar[stage]);
+  };
+  auto refill = [&](int stage) {
+    const int tt = claim();
+    if (lane == 0) tq[stage] = tt;
+    issue(tt, stage);
+  };
+  refill(0);
+  refill(1);
+  const float2 c2 = make_float2(c, c);
+  for (uint32_t k = 0;; ++k) {
+    const int stage = k & 1;
+    __syncwarp();
+    const int64_t tile = tq[stage];
+    if (tile < 0) break;
+    const bool ok = mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);
+    if (__any_sync(kFullMask, !ok)) {
+      if (lane == 0) atomicOr(&g_kvq_fault, 1u);
+      mbar_wait(&bar[stage], (k >> 1) & 1, kSpinLimit);   // the stage that gave up, once more
+      if (tq[stage ^ 1] >= 0) mbar_wait(&bar[stage ^ 1], ((k + 1) >> 1) & 1, kSpinLimit);
+      if (lane == 0) bulk_wait0();
+      return;
+    }
+    const uint32_t sbytes = scale_bytes(tile);
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();             // the warp's staging tile is free
+#pragma unroll 1
+    for (int mt = 0; mt < 2; ++mt) {
+      // the lane's rows of this M-tile: 16 mt + g and 16 mt + 8 + g
+      uint32_t a[NG * KG][4];
+      uint16_t sv[2][NG];
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int r = 16 * mt + 8 * hr + g;
+        const int64_t row = tile * WROWS + r;
+        const int64_t rrow = row < n ? row : n - 1;
+        const bool sc_smem = static_cast<uint32_t>((r + 1) * SPR) <= sbytes;
+        const uint16_t* srow = sc_smem ? reinterpret_cast<const uint16_t*>(stage_sc + stage * WSC + r * SPR)
+                                       : scales + rrow * NG;
+#pragma unroll
+        for (int j = 0; j < NG; ++j) sv[hr][j] = srow[j];
+        // the row's codes: 64 bytes swizzled over the row (16-byte chunk ch at ch ^ ((r >> 1) & 3))
+        const uint8_t* crow = stage_in + stage * WPIN + r * (D / 2);
+        const int swz = (r >> 1) & 3;
+#pragma unroll
+        for (int ks = 0; ks < NG * KG; ++ks) {          // 16 channels: bytes 8 ks .. 8 ks + 7
+          const uint2 w = *reinterpret_cast<const uint2*>(crow + (((ks >> 1) ^ swz) << 4) + 8 * (ks & 1));
+          a[ks][hr] = code_pair_f16(w.x, t);             // channels 16 ks + 2t, + 1
+          a[ks][2 + hr] = code_pair_f16(w.y, t);         // channels 16 ks + 8 + 2t, + 1
+        }
+      }
+      float acc[16][4];
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+      // W = H_G q per group: k-step (group gi, ks), n-tile (gi, ntl), block
+      // H_(G/16)[ks][ntl / 2] * H_16[., 8 (ntl & 1) ..]
+#pragma unroll
+      for (int gi = 0; gi < NG; ++gi)
+#pragma unroll
+        for (int ks = 0; ks < KG; ++ks)
+#pragma unroll
+          for (int ntl = 0; ntl < NTG; ++ntl) {
+            const bool neg = __popc(ks & (ntl >> 1)) & 1;
+            const uint32_t b0 = hb[ntl & 1][0] ^ (neg ? 0x80008000u : 0u);
+            const uint32_t b1 = hb[ntl & 1][1] ^ (neg ? 0x80008000u : 0u);
+            mma_f16_16816(acc[gi * NTG + ntl], a[gi * KG + ks], b0, b1);
+          }
+      // u = W S (exact), then the stages that cross groups, in fp32
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        const float s0 = half_bits_to_float(sv[0][nt / NTG]), s1 = half_bits_to_float(sv[1][nt / NTG]);
+        acc[nt][0] = __fmul_rn(acc[nt][0], s0);
+        acc[nt][1] = __fmul_rn(acc[nt][1], s0);
+        acc[nt][2] = __fmul_rn(acc[nt][2], s1);
+        acc[nt][3] = __fmul_rn(acc[nt][3], s1);
+      }
+#pragma unroll
+      for (int h = G; h < D; h <<= 1) {
+#pragma unroll
+        for (int nt = 0; nt < 16; ++nt) {
+          if (((8 * nt) & h) == 0) {
+            const int mt2 = nt + h / 8;
+            const float2 a0 = make_float2(acc[nt][0], acc[nt][1]), b0 = make_float2(acc[mt2][0], acc[mt2][1]);
+            const float2 a1 = make_float2(acc[nt][2], acc[nt][3]), b1 = make_float2(acc[mt2][2], acc[mt2][3]);
+            const float2 s0 = __fadd2_rn(a0, b0), d0 = fsub2(a0, b0);
+            const float2 s1 = __fadd2_rn(a1, b1), d1 = fsub2(a1, b1);
+            acc[nt][0] = s0.x; acc[nt][1] = s0.y; acc[nt][2] = s1.x; acc[nt][3] = s1.y;
+            acc[mt2][0] = d0.x; acc[mt2][1] = d0.y; acc[mt2][2] = d1.x; acc[mt2][3] = d1.y;
+          }
+        }
+      }
+      // x c, x s (1/lambda), fp16: channels 8 nt + 2t, + 1 of rows 16 mt + g (+ 8)
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        const int ch = 8 * nt + 2 * t;
+        const float4 tv = tabw[(ch & 63) >> 1];       // (c[2q], c[2q+64], c[2q+1], c[2q+65])
+        const float2 f = ch < 64 ? make_float2(tv.x, tv.z) : make_float2(tv.y, tv.w);
+        const float2 v0 = __fmul2_rn(__fmul2_rn(make_float2(acc[nt][0], acc[nt][1]), c2), f);
+        const float2 v1 = __fmul2_rn(__fmul2_rn(make_float2(acc[nt][2], acc[nt][3]), c2), f);
+        const int q = nt >> 3, cc = nt & 7;
+        const int r0 = 16 * mt + g, r1 = r0 + 8;
+        *reinterpret_cast<uint32_t*>(stage_out + wtile_off<D>(q, r0, cc) + 4 * t) = float2_to_half2_bits(v0.x, v0.y);
+        *reinterpret_cast<uint32_t*>(stage_out + wtile_off<D>(q, r1, cc) + 4 * t) = float2_to_half2_bits(v1.x, v1.y);
+      }
+    }
+    __syncwarp();             // codes and scales consumed: the input stage can be refilled
+    refill(stage);
+    fence_proxy_async();
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+      for (int q = 0; q < 2; ++q)
+        tensor_s2g(&maps.q[q], 0, static_cast<int>(tile * WROWS), stage_out + q * W::WQB);
+      bulk_commit();
+    }
+  }
+  if (lane == 0) bulk_wait0();
+}
+
+// ---------------------------------------------------------------------------
 // Round trip: fp16 [n][D] -> x_hat = dequantize(quantize(x)) fp16 [n][D], and
 // optionally the codes and scales, in one pass (the quantise-then-dequantise
 // shape used to simulate the cache's error).  Each warp streams its tiles as
@@ -1040,6 +1257,29 @@ int launch_dequantize(const uint8_t* packed, const uint16_t* scales, const float
   return launch_dequantize_nw<D, G, kSmallWarps>(maps, dev, sms, packed, scales, lam, s, n, st);
 }
 
+// The tensor-core dequantizer: one block of kWarps warps per SM (or fewer
+// blocks than SMs for small batches: never more blocks than warp tiles).
+template <int G>
+int launch_dequantize_tc(const uint8_t* packed, const uint16_t* scales, const float* lam,
+                         const int8_t* s, int64_t n, uint16_t* out, cudaStream_t st) {
+  constexpr int D = 128;
+  RowMaps maps;
+  int rc = make_row_maps<D>(maps, out, n, WTile<D>::WROWS);
+  if (rc != KVQ_OK) return rc;
+  CUtensorMap cmap;
+  rc = make_code_map<D>(cmap, const_cast<uint8_t*>(packed), n);
+  if (rc != KVQ_OK) return rc;
+  int dev = 0;
+  const int sms = current_device_sms(dev);
+  auto k = kvq_dequantize_tc_kernel<G, kWarps>;
+  constexpr int smem = Stream<D>::smem(Stream<D>::DWARP, kWarps);
+  const int grid = stream_grid<3, D, G, kWarps>(k, dev, sms, n, smem);
+  (void)cudaGetLastError();
+  k<<<grid, kWarps * 32, smem, st>>>(cmap, scales, lam, s, n, norm_const(D), maps,
+                                     (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
+  return finish_launch();
+}
+
 template <int D, int G>
 int launch_roundtrip(const uint16_t* x, const float* lam, const int8_t* s, int64_t n,
                      uint16_t* x_hat, uint8_t* packed, uint16_t* scales, cudaStream_t st) {
@@ -1172,6 +1412,25 @@ int kvq_selftest_wait_timeout(uint32_t limit, void* stream) {
   (void)cudaGetLastError();
   kvq_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit);
   return finish_launch();
+}
+
+int kvq_dequantize_tc(const uint8_t* packed, const uint16_t* scales, const float* lambda,
+                      const int8_t* signs, int64_t n_vec, int D, int group, uint16_t* x_out,
+                      void* stream) {
+  const int rc = check_shape(D, group, n_vec);
+  if (rc != KVQ_OK) return rc;
+  if (D != 128) return KVQ_ERR_DIM;
+  if (group != 16 && group != 32 && group != 64) return KVQ_ERR_GROUP;
+  if (n_vec == 0) return KVQ_OK;
+  if (!packed || !scales || !lambda || !signs || !x_out) return KVQ_ERR_NULL;
+  if (!aligned(x_out, 16) || !aligned(packed, 16) || !aligned(scales, 2) || !aligned(lambda, 4))
+    return KVQ_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (group) {
+    case 16: return launch_dequantize_tc<16>(packed, scales, lambda, signs, n_vec, x_out, st);
+    case 32: return launch_dequantize_tc<32>(packed, scales, lambda, signs, n_vec, x_out, st);
+    default: return launch_dequantize_tc<64>(packed, scales, lambda, signs, n_vec, x_out, st);
+  }
 }
 
 int kvq_selftest_rcp_f16(float* out, void* stream) {

@@ -42,6 +42,8 @@ _lib.kvq_roundtrip.restype = _I
 _lib.kvq_roundtrip.argtypes = [_P, _P, _P, _I64, _I, _I, _P, _P, _P, _P]
 _lib.kvq_dequantize.restype = _I
 _lib.kvq_dequantize.argtypes = [_P, _P, _P, _P, _I64, _I, _I, _P, _P]
+_lib.kvq_dequantize_tc.restype = _I
+_lib.kvq_dequantize_tc.argtypes = [_P, _P, _P, _P, _I64, _I, _I, _P, _P]
 _lib.kvq_quantize_ex.restype = _I
 _lib.kvq_quantize_ex.argtypes = [_P, _P, _P, _I64, _I, _I, _I, _I, _I64, _I, _P, _P, _P]
 _lib.kvq_dequantize_ex.restype = _I
@@ -114,6 +116,11 @@ def kvq_dequantize(packed: int, scales: int, lam: int, signs: int, n_vec: int,
 
 KVQ_LAMBDA_AFTER = 1
 KVQ_SRFT = 2
+
+
+def kvq_dequantize_tc(packed: int, scales: int, lam: int, signs: int, n_vec: int,
+                      D: int, group: int, x_out: int, stream: int = 0) -> int:
+    return _lib.kvq_dequantize_tc(packed, scales, lam, signs, n_vec, D, group, x_out, stream)
 
 
 def kvq_quantize_ex(x: int, lam: int, signs: int, n_vec: int, D: int, group: int, bits: int,
@@ -391,8 +398,10 @@ def attention_decode(q: torch.Tensor, k_packed: torch.Tensor, k_scales: torch.Te
 
 def dequantize(packed: torch.Tensor, scales: torch.Tensor, lam: torch.Tensor,
                signs: torch.Tensor, group: int, out: torch.Tensor | None = None,
-               stream=None) -> torch.Tensor:
-    """(packed uint8 [n, D/2], scales fp16 [n, D/group]) -> fp16 [n, D]."""
+               stream=None, tensor_cores: bool = False) -> torch.Tensor:
+    """(packed uint8 [n, D/2], scales fp16 [n, D/group]) -> fp16 [n, D].
+    ``tensor_cores``: run kvq_dequantize_tc (the in-group Hadamard on the
+    tensor cores; D = 128, group 16/32/64), bit-identical."""
     if packed.dim() != 2:
         raise ValueError("packed must be [n_vec, D/2]")
     n, D = packed.shape[0], packed.shape[1] * 2
@@ -403,9 +412,10 @@ def dequantize(packed: torch.Tensor, scales: torch.Tensor, lam: torch.Tensor,
     if out is None:
         out = torch.empty((n, D), dtype=torch.float16, device=packed.device)
     _need(out, torch.float16, (n, D), "out")
-    rc = kvq_dequantize(packed.data_ptr(), scales.data_ptr(), lam.data_ptr(),
-                        signs.data_ptr(), n, D, group, out.data_ptr(),
-                        _stream_handle(stream))
+    fn = kvq_dequantize_tc if tensor_cores else kvq_dequantize
+    rc = fn(packed.data_ptr(), scales.data_ptr(), lam.data_ptr(),
+            signs.data_ptr(), n, D, group, out.data_ptr(),
+            _stream_handle(stream))
     if rc != KVQ_OK:
         raise KvqError(rc)
     return out

@@ -140,6 +140,15 @@ def test_attention_errors(kvq):
     assert kvq.kvq_attention_workspace_bytes(4096, 32, 8, 4096, 128, 32) == 0
 
 
+def test_dequantize_tc_errors(kvq):
+    d = lambda **kw: kvq.kvq_dequantize_tc(kw.get("p", A), A, A, A, kw.get("n", 64), kw.get("D", 128),
+                                           kw.get("G", 32), kw.get("out", A))
+    assert d(D=64) == -3 and d(D=256) == -3 and d(D=96) == -3
+    assert d(G=128) == -4 and d(G=8) == -4
+    assert d(n=-1) == -5 and d(n=0) == 0
+    assert d(p=0) == -1 and d(out=0) == -1 and d(out=A + 8) == -2
+
+
 def test_codec_ex_errors(kvq):
     q = lambda **kw: kvq.kvq_quantize_ex(kw.get("x", A), kw.get("lam", A), A, kw.get("n", 64),
                                          kw.get("D", 128), kw.get("G", 32), kw.get("bits", 4),
