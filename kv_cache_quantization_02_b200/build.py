@@ -14,8 +14,15 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SOURCES = [os.path.join(PKG, "csrc", n) for n in ("kvq.cu", "kvq_attn.cu", "kvq_ex.cu", "kvq_srft_d64.cu",
+SOURCES = [os.path.join(PKG, "csrc", n) for n in ("kvq.cu", "kvq_attn.cu", "kvq_attn_d64.cu", "kvq_attn_d128.cu",
+                                                        "kvq_attn_d256.cu", "kvq_ex.cu", "kvq_srft_d64.cu",
                                                         "kvq_srft_d96.cu", "kvq_srft_d128.cu", "kvq_srft_d256.cu")]
+# Per-unit flags.  The codec units keep --fmad=false: their results are
+# defined bit for bit, and a contracted multiply-add rounds once where the
+# codec's definition rounds twice.  The decode attention is checked against
+# the oracle to a derived tolerance, not bit for bit, so its multiply-add
+# pairs may contract (one rounding instead of two only shrinks the error).
+UNIT_FLAGS = {n: ["--fmad=true"] for n in ("kvq_attn_d64.cu", "kvq_attn_d128.cu", "kvq_attn_d256.cu")}
 INCLUDE = os.path.join(ROOT, "include")
 LIBRARY = os.path.join(PKG, "libkvq.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -42,7 +49,9 @@ def build(verbose: bool = False, extra: list[str] | None = None) -> str:
         objs = [os.path.join(td, os.path.basename(src) + ".o") for src in SOURCES]
 
         def one(src, obj):
-            cmd = [NVCC, *compile_flags, *(extra or []), "-I", INCLUDE, "-c", src, "-o", obj]
+            unit = UNIT_FLAGS.get(os.path.basename(src), [])
+            flags = [f for f in compile_flags if not (unit and f.startswith("--fmad="))] + unit
+            cmd = [NVCC, *flags, *(extra or []), "-I", INCLUDE, "-c", src, "-o", obj]
             if verbose:
                 cmd.insert(1, "-Xptxas=-v")
             return subprocess.run(cmd, capture_output=True, text=True)

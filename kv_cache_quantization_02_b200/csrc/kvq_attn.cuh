@@ -1,0 +1,815 @@
+// kvq_attn.cuh -- fused decode attention over the int4 rotated-domain KV
+// cache for B200 (sm_100a): the kernels behind kvq_attention_decode[_ex]
+// (include/kvq.h) at one head dimension, D = KVQ_ATTN_D; kvq_attn_d<D>.cu
+// instantiate it and kvq_attn.cu holds the C ABI.
+//
+// Method: "The Kernel That Finally Did Something -- And Didn't Quite Agree
+// With Itself" (VeloxQuant-MLX blog), "Fused group-affine (KIVI-style)
+// attention": the quantised keys and values are reconstructed in registers
+// inside a FlashAttention-style online softmax, so no dequantised K or V ever
+// reaches memory, and the key axis is split flash-decoding style when there
+// are few sequences.  The cache rows here are int4 codes of the rotated vector
+// y = R diag(s) (lambda . x) (or R diag(s) x / lambda with lambda after the
+// rotation; R = H / sqrt(D) or the SRFT) with fp16 group scales ("When
+// Quantization Is Free", technical summary, Methodologie 1-3), so the rotation
+// moves to the query, once per head, instead of running once per key:
+//     <q, x_t> = <q~, y_t>,   q~ = R diag(s_K) (q / lambda_K),
+// and the values are summed in the rotated domain and rotated back once:
+//     o = (diag(s_V) R^T (sum_t p_t y_t)) / lambda_V.
+//
+// Work decomposition.  A block of four warps owns one (sequence, KV head,
+// key split); each warp streams 32-key blocks (codes and scales of K and V,
+// four bulk copies into a private ring of 3 stages, 2 at D = 256) and keeps
+// its own online-softmax state; the block merges the four states at the end.
+// Both products run on the tensor cores as m16n8k16 fp16 MMAs with fp32
+// accumulation, with the N dimension = 4 query heads x 2 parts (q~ and p S_V
+// each as an fp16 value plus its fp16 remainder, ~2^-22 together):
+//   * scores: M = 16 keys, K = 16 channels.  A lane reads one 32-bit code
+//     word per key and 32 channels; its four nibble pairs are the A fragments
+//     of two k-steps (low nibbles as n 2^-24, high nibbles as 16 n 2^-24,
+//     their query entries divided by 16), and every k-step stays inside one
+//     scale group (G = 16: a k-step spans two groups and runs once per group
+//     with the other group's entries zero).  The group's scale multiplies
+//     the per-group partial sums key by key after the MMA.  In the
+//     accumulator layout lane (g, t) holds keys g and g + 8 of head t, both
+//     parts: every lane's epilogue is useful work.
+//   * values: M = 16 channels, K = 16 keys: the probabilities pass through a
+//     per-warp shared-memory row so that lane (g, t) gets keys 2t, 2t+1,
+//     2t+8, 2t+9 of head g/2; p S_V per scale group is the B fragment, and
+//     byte permutes pair a channel's codes of four keys.  The output columns
+//     of lane (g, t) are head t again, so the softmax rescale needs no
+//     exchange.
+// A biased code n = q + 8 in [0, 15] is the fp16 subnormal n 2^-24, exact,
+// made by one mask-and-xor.  The key side starts its accumulators at
+// -8 2^-24 times the query's group sums; the value side keeps the running sum
+// of p S_V per group and subtracts 8 times it once at the end.
+//
+// Every mbarrier wait is bounded; a warp that gives up sets the fault word
+// and the block writes nothing.  A sequence length outside [0, T] is clamped
+// and flagged.  Compiled with --fmad=true: the result is checked against the
+// oracle to a derived tolerance, and a contracted multiply-add only removes a
+// rounding.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "kvq.h"
+#include "kvq_attn_common.cuh"
+
+#ifndef KVQ_ATTN_D
+#error "define KVQ_ATTN_D (64, 128 or 256) before including kvq_attn.cuh"
+#endif
+
+namespace {
+
+using namespace kvqa;
+constexpr unsigned kFullMask = 0xffffffffu;
+
+#include "kvq_async.cuh"
+#include "kvq_arith.cuh"
+#include "kvq_fft.cuh"
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr uint32_t kSpin = 1u << 22;         // bounded mbarrier waits
+
+__device__ unsigned int g_attn_fault = 0;    // bit 0: a wait gave up; bit 3: bad sequence length
+thread_local int g_attn_cuda_error = 0;
+
+template <int D, int G>
+struct Attn {
+  static constexpr int NG = D / G;                  // scale groups of a row
+  static constexpr int NBK = D / 32;                // 32-channel blocks (score k-step pairs)
+  static constexpr int KS = D / 16;                 // k-steps of the score product
+  static constexpr int NCT = D / 16;                // 16-channel tiles of the value product
+  static constexpr int W32 = D / 8;                 // 32-bit words of one code row
+  static constexpr int ST = D >= 256 ? 2 : 3;       // ring depth per warp
+  static constexpr int CB = kBK * D / 2;            // code bytes of one block
+  static constexpr int SB = kBK * NG * 2;           // scale bytes of one block
+  static constexpr int STAGE = 2 * CB + 2 * SB;     // K codes, V codes, K scales, V scales
+  static constexpr int RING = kAW * ST * STAGE;
+  static constexpr int COMB = kAW * kMaxRows * D * 4;
+  static constexpr int AREA = RING > COMB ? RING : COMB;   // the merge reuses the ring
+  static constexpr int QF = kMaxRows * D * 4;       // rotated query rows, fp32
+  static constexpr int SC = 2 * kBK * NG * 4;       // per warp: the block's K and V scales, fp32
+  static constexpr int PS = kBK + 8;                // row stride of the probability rows
+  static constexpr int PB = kMaxRows * PS * 4;      // per warp: probabilities [head][key]
+  static constexpr int SMEM = AREA + QF + kAW * (SC + PB) + kAW * ST * 8 + kAW * kMaxRows * 8;
+  static constexpr int DPL = D / 32;                // channels per lane in the row transforms
+  static_assert(STAGE % 16 == 0 && (SC + PB) % 16 == 0, "16-byte aligned areas");
+};
+
+// Biased code pairs as fp16 subnormals.  A word of codes xor 0x88888888
+// holds n = q + 8 in [0, 15] in every nibble (the two's-complement nibble q
+// xor 8); of such a word x, lo_pair takes the nibbles at bits 0-3 and 16-19
+// (the low nibbles of bytes 0 and 2) and hi_pair those at bits 4-7 and 20-23
+// (the high nibbles): the half holding n (low) or 16 n (high) is the
+// subnormal n 2^-24 or 16 n 2^-24, exact, in one mask.
+constexpr uint32_t kBias8 = 0x88888888u;
+__device__ __forceinline__ uint32_t lo_pair(uint32_t x) { return x & 0x000F000Fu; }
+__device__ __forceinline__ uint32_t hi_pair(uint32_t x) { return x & 0x00F000F0u; }
+
+// d = a b + c on the tensor cores (m16n8k16, fp16 operands, fp32 accumulate).
+__device__ __forceinline__ void mma_acc(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_init(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
+                                         float c0, float c1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%10,%11};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
+}
+
+// v as fp16 (part 0) or the fp16 remainder v - fp16(v) (part 1): the two parts
+// sum to v within 2^-22 |v|.
+__device__ __forceinline__ uint16_t f16_part(float v, int part) {
+  const __half h = __float2half_rn(v);
+  return __half_as_ushort(part ? __float2half_rn(v - __half2float(h)) : h);
+}
+
+// N consecutive floats of shared memory into registers, in 16-byte loads
+// where N allows (the rows are 16-byte aligned when N is a multiple of 4).
+template <int N>
+__device__ __forceinline__ void load_row(float (&r)[N], const float* p) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      const float4 v = *reinterpret_cast<const float4*>(p + i);
+      r[i] = v.x; r[i + 1] = v.y; r[i + 2] = v.z; r[i + 3] = v.w;
+    }
+  } else if constexpr (N == 2) {
+    const float2 v = *reinterpret_cast<const float2*>(p);
+    r[0] = v.x; r[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; ++i) r[i] = p[i];
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
+  constexpr int DPL = D / 32;
+#pragma unroll
+  for (int h = 1; h < DPL; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i], b = v[i + h];
+        v[i] = a + b;
+        v[i + h] = a - b;
+      }
+    }
+  }
+#pragma unroll
+  for (int h = DPL; h < D; h <<= 1) {
+    const int lb = h / DPL;
+    const bool upper = (lane & lb) != 0;
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      const float o = __shfl_xor_sync(kFull, v[i], lb);
+      v[i] = upper ? o - v[i] : v[i] + o;
+    }
+  }
+}
+
+// One head's output from its merged rotated-domain sum y = o / l, back in
+// the cache's format:
+//   lambda before: out = fp16((s_V . R^T y) / lambda_V),
+//   lambda after:  out = fp16(s_V . R^T (y / lambda_V)),
+// R^T = H / sqrt(D) (a warp-wide butterfly over the lanes' channels) or the
+// SRFT transpose (the codec's adjoint unpacking and transposed FFT, run by one
+// lane on the row gathered in `scr`, D floats of this warp's shared memory).
+template <int D>
+__device__ __forceinline__ void finish_head(const AttnParams& P, float (&v)[D / 32], float l,
+                                            uint16_t* out_row, int lane, float* scr) {
+  constexpr int DPL = D / 32;
+  const bool after = (P.fmt & kFmtAfter) != 0;
+  const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) v[i] *= inv;
+  if ((P.fmt & kFmtSrft) == 0) {
+    if (after) {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) v[i] /= P.lam_v[DPL * lane + i];
+    }
+    warp_fwht<D>(v, lane);
+    uint16_t h[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      const int d = DPL * lane + i;
+      const float z = v[i] * P.c;
+      const float zs = P.s_v[d] < 0 ? -z : z;
+      h[i] = __half_as_ushort(__float2half_rn(after ? zs : zs / P.lam_v[d]));
+    }
+    if constexpr (DPL == 4) {
+      *reinterpret_cast<uint2*>(out_row + DPL * lane) =
+          make_uint2(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16));
+    } else {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) out_row[DPL * lane + i] = h[i];
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) scr[DPL * lane + i] = v[i];
+    __syncwarp();
+    if (lane == 0) {
+      float2 z[D / 2];
+#pragma unroll
+      for (int n = 0; n < D / 2; ++n) z[n] = make_float2(scr[2 * n], scr[2 * n + 1]);
+      unpack_inv1<D>(z, P.wd, [&](int n) -> float2 {
+        float2 f = n == 0 ? make_float2(P.c, P.c) : make_float2(P.c1h, P.c1h);
+        if (after) f = make_float2(f.x / P.lam_v[2 * n], f.y / P.lam_v[2 * n + 1]);
+        return f;
+      });
+      fft_inv_from<D / 2, D / 2, D / 2>(z, P.wn);
+#pragma unroll
+      for (int n = 0; n < D / 2; ++n) {
+        float a = P.s_v[2 * n] < 0 ? -z[n].x : z[n].x;
+        float b = P.s_v[2 * n + 1] < 0 ? -z[n].y : z[n].y;
+        if (!after) {
+          a = a / P.lam_v[2 * n];
+          b = b / P.lam_v[2 * n + 1];
+        }
+        reinterpret_cast<uint32_t*>(out_row)[n] = float2_to_half2_bits(a, b);
+      }
+    }
+    __syncwarp();
+  }
+}
+
+// One block of four warps per (sequence, KV head, key split); head tiles of
+// four query heads (NH = 1 for up to four heads per KV head, 2 for up to 8).
+template <int D, int G, int NH>
+__global__ void __launch_bounds__(kAW * 32, (D >= 256 || NH > 1 || G == 16) ? 2 : 3)
+kvq_attn_kernel(const __grid_constant__ AttnParams P) {
+  using A = Attn<D, G>;
+  constexpr int NG = A::NG, NBK = A::NBK, KS = A::KS, NCT = A::NCT, W32 = A::W32, DPL = A::DPL;
+  constexpr int ST = A::ST, PS = A::PS;
+  constexpr int CPG = (G >= 32) ? G / 32 : 1;     // score k-step pairs per group (G = 16: two groups per pair)
+  extern __shared__ __align__(128) uint8_t sm[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint8_t* ring = sm;                                                  // [warp][stage][STAGE]
+  float* qf = reinterpret_cast<float*>(sm + A::AREA);                  // [8][D]
+  float* scw = qf + kMaxRows * D + warp * ((A::SC + A::PB) / 4);       // this warp's area:
+  float* sk = scw;                                                     //   K scales [kBK][NG], fp32
+  float* sv = scw + kBK * NG;                                          //   V scales [kBK][NG], fp32
+  float* pw = scw + A::SC / 4;                                         //   probabilities [8][PS]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + A::AREA + A::QF + kAW * (A::SC + A::PB));
+  float* ml = reinterpret_cast<float*>(bars + kAW * ST);               // [warp][8][2]: m, l
+  float* comb = reinterpret_cast<float*>(sm);                          // [warp][8][D], after the key loop
+
+  const int g = lane >> 2, t = lane & 3;
+  const int item = blockIdx.x;
+  const int split = item % P.nsplit;
+  const int bh = item / P.nsplit;                                      // b * Hkv + kv head
+  const int b = bh / P.Hkv, kvh = bh % P.Hkv;
+  const int R = P.R;
+  int L = P.seq_len[b];
+  if (L < 0 || L > P.T) {
+    if (tid == 0) atomicOr(&g_attn_fault, 8u);
+    L = L < 0 ? 0 : P.T;
+  }
+  const int k0 = split * P.chunk;
+  const int k1 = min(L, k0 + P.chunk);
+  const int nkeys = k1 > k0 ? k1 - k0 : 0;
+  const int nblk = (nkeys + kBK - 1) / kBK;
+
+  uint64_t* bar = bars + ST * warp;
+  if (lane == 0) {
+    for (int s = 0; s < ST; ++s) mbar_init(&bar[s], 1);
+    mbar_fence_init();
+  }
+  const int64_t row_base = static_cast<int64_t>(bh) * P.T;
+  auto issue = [&](int blk, int stage) {
+    if (blk >= nblk || lane != 0) return;
+    const int kb = k0 + blk * kBK;
+    const int nk = min(kBK, k1 - kb);
+    const int nk16 = (nk + 15) & ~15;                            // stays inside T (T % 16 == 0)
+    const int64_t row0 = row_base + kb;
+    uint8_t* st = ring + (warp * ST + stage) * A::STAGE;
+    const uint32_t cb = static_cast<uint32_t>(nk16 * (D / 2));
+    const uint32_t sb = static_cast<uint32_t>(nk16 * NG * 2);
+    mbar_expect_tx(&bar[stage], 2 * cb + 2 * sb);
+    bulk_g2s(st, P.kp + row0 * (D / 2), cb, &bar[stage]);
+    bulk_g2s(st + A::CB, P.vp + row0 * (D / 2), cb, &bar[stage]);
+    bulk_g2s(st + 2 * A::CB, P.ks + row0 * NG, sb, &bar[stage]);
+    bulk_g2s(st + 2 * A::CB + A::SB, P.vs + row0 * NG, sb, &bar[stage]);
+  };
+  __syncwarp();
+  for (int s = 0; s < ST; ++s) issue(warp + s * kAW, s);
+
+  // The rotated query, fp32: q~ = R (s_K . (q / lambda_K)) with lambda before
+  // the rotation, q~ = R (s_K . q) / lambda_K with lambda after it (so that
+  // <q, x_t> = <q~, y_t>), R = H / sqrt(D) or the SRFT; rows R..7 are zero.
+  const bool after = (P.fmt & kFmtAfter) != 0;
+  for (int r = warp; r < kMaxRows; r += kAW) {
+    float* qr_out = qf + r * D;
+    if (P.fmt & kFmtSrft) {
+      if (lane == 0) {
+        float2 z[D / 2];
+        if (r < R) {
+          const uint32_t* qr = reinterpret_cast<const uint32_t*>(
+              P.q + (static_cast<int64_t>(b) * P.Hkv * R + kvh * R + r) * D);
+#pragma unroll
+          for (int n = 0; n < D / 2; ++n) {
+            float2 x = half2_bits_to_float2(qr[n]);
+            if (!after) x = make_float2(x.x / P.lam_k[2 * n], x.y / P.lam_k[2 * n + 1]);
+            z[n] = make_float2(P.s_k[2 * n] < 0 ? -x.x : x.x, P.s_k[2 * n + 1] < 0 ? -x.y : x.y);
+          }
+          fft_fwd_from<D / 2, D / 2, D / 2>(z, P.wn);
+          unpack_fwd1<D>(z, P.wd, [&](int n) -> float2 {
+            float2 f = n == 0 ? make_float2(P.c, P.c) : make_float2(P.c1h, P.c1h);
+            if (after) f = make_float2(f.x / P.lam_k[2 * n], f.y / P.lam_k[2 * n + 1]);
+            if (n > D / 4) f.y = -f.y;                 // bins above N/2 come as conj(E - T)
+            return f;
+          });
+        } else {
+#pragma unroll
+          for (int n = 0; n < D / 2; ++n) z[n] = make_float2(0.0f, 0.0f);
+        }
+#pragma unroll
+        for (int n = 0; n < D / 2; ++n) reinterpret_cast<float2*>(qr_out)[n] = z[n];
+      }
+      continue;
+    }
+    float v[DPL];
+    if (r < R) {
+      const uint16_t* qr = P.q + (static_cast<int64_t>(b) * P.Hkv * R + kvh * R + r) * D;
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) {
+        const int d = DPL * lane + i;
+        float x = __half2float(__ushort_as_half(qr[d]));
+        if (!after) x = x / P.lam_k[d];
+        v[i] = P.s_k[d] < 0 ? -x : x;
+      }
+      warp_fwht<D>(v, lane);
+    } else {
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) v[i] = 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      const int d = DPL * lane + i;
+      float y = v[i] * P.c;
+      if (after) y = y / P.lam_k[d];
+      qr_out[d] = y;
+    }
+  }
+  __syncthreads();
+
+  // Score B fragments.  k-step j = 2 bb + s of 32-channel block bb: lane
+  // (g, t) reads code word w = 4 bb + t of its two keys, and the k-indices
+  // (2t, 2t+1) are channels 8w + 2s, 8w + 2s + 4 (low nibbles), (2t+8, 2t+9)
+  // are 8w + 2s + 1, 8w + 2s + 5 (high nibbles, which arrive as 16 n: their
+  // query entries are divided by 16).  Column g is head 4 ht + g/2, part g & 1
+  // (the fp16 value, or its fp16 remainder).  With G = 16 a k-step spans two
+  // groups (lanes t < 2 and t >= 2), and runs once per group with the other
+  // group's k-indices zero in B.
+  constexpr int BQ = (G == 16) ? 2 : 1;
+  uint32_t bq[NH][KS][BQ][2];
+#pragma unroll
+  for (int ht = 0; ht < NH; ++ht)
+#pragma unroll
+    for (int j = 0; j < KS; ++j) {
+      const float* qr = qf + (4 * ht + (g >> 1)) * D;
+      const int c0 = 8 * (4 * (j >> 1) + t) + 2 * (j & 1);
+      const int part = g & 1;
+      const uint32_t b0 = f16_part(qr[c0], part) | (uint32_t(f16_part(qr[c0 + 4], part)) << 16);
+      const uint32_t b1 = f16_part(qr[c0 + 1] * 0.0625f, part) |
+                          (uint32_t(f16_part(qr[c0 + 5] * 0.0625f, part)) << 16);
+      if constexpr (G == 16) {
+        const bool upper = t >= 2;
+        bq[ht][j][0][0] = upper ? 0u : b0;
+        bq[ht][j][0][1] = upper ? 0u : b1;
+        bq[ht][j][1][0] = upper ? b0 : 0u;
+        bq[ht][j][1][1] = upper ? b1 : 0u;
+      } else {
+        bq[ht][j][0][0] = b0;
+        bq[ht][j][0][1] = b1;
+      }
+    }
+  // Score accumulators start at the bias of the biased codes: -8 2^-24 times
+  // the group's sum of the B entries (times 16 for the high-nibble entries),
+  // per column of this lane: head 4 ht + t, both parts.  The eight lanes of a
+  // column split the group's channels and add up by shuffles.
+  float bias[NH][NG][2];
+#pragma unroll
+  for (int ht = 0; ht < NH; ++ht) {
+    const float* qr = qf + (4 * ht + t) * D;
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+      float s0 = 0.0f, s1 = 0.0f;
+      for (int c = gi * G + g; c < (gi + 1) * G; c += 8) {
+        const bool odd = c & 1;
+        const float v = odd ? qr[c] * 0.0625f : qr[c];
+        const float w = odd ? 16.0f : 1.0f;
+        s0 += w * __half2float(__ushort_as_half(f16_part(v, 0)));
+        s1 += w * __half2float(__ushort_as_half(f16_part(v, 1)));
+      }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        s0 += __shfl_xor_sync(kFull, s0, o);
+        s1 += __shfl_xor_sync(kFull, s1, o);
+      }
+      bias[ht][gi][0] = -8.0f * 0x1p-24f * s0;
+      bias[ht][gi][1] = -8.0f * 0x1p-24f * s1;
+    }
+  }
+  const float part_f = static_cast<float>(g & 1);
+
+  float O[NH][NCT][4];
+#pragma unroll
+  for (int ht = 0; ht < NH; ++ht)
+#pragma unroll
+    for (int n = 0; n < NCT; ++n) O[ht][n][0] = O[ht][n][1] = O[ht][n][2] = O[ht][n][3] = 0.0f;
+  float m[NH], l[NH];
+#pragma unroll
+  for (int ht = 0; ht < NH; ++ht) { m[ht] = -INFINITY; l[ht] = 0.0f; }
+  // sum of p S_V per group over this lane's keys, head 4 ht + g/2: the value
+  // product runs on biased codes, and 8 times this is its bias
+  float pc[NH][NG];
+#pragma unroll
+  for (int ht = 0; ht < NH; ++ht)
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) pc[ht][gi] = 0.0f;
+  bool failed = false;
+  int k = 0;
+  for (int blk = warp; blk < nblk; blk += kAW, ++k) {
+    const int stage = k % ST;
+    const bool ok = mbar_wait(&bar[stage], (k / ST) & 1, kSpin);
+    if (__any_sync(kFull, !ok)) {
+      failed = true;
+      break;
+    }
+    const uint8_t* st = ring + (warp * ST + stage) * A::STAGE;
+    const uint32_t* kc = reinterpret_cast<const uint32_t*>(st);
+    const uint32_t* vc = reinterpret_cast<const uint32_t*>(st + A::CB);
+    const uint16_t* ksh = reinterpret_cast<const uint16_t*>(st + 2 * A::CB);
+    const uint16_t* vsh = reinterpret_cast<const uint16_t*>(st + 2 * A::CB + A::SB);
+    const int nk = min(kBK, k1 - (k0 + blk * kBK));
+
+    // The block's scales as fp32; keys at or past nk (stale or unwritten
+    // rows) get 0, so that their zero weights stay exactly 0.
+#pragma unroll
+    for (int i0 = 0; i0 < kBK * NG; i0 += 128) {
+      const int i = i0 + 4 * lane;
+      if (i < kBK * NG) {
+        const uint2 kw = *reinterpret_cast<const uint2*>(ksh + i);
+        const uint2 vw = *reinterpret_cast<const uint2*>(vsh + i);
+        const float2 k01 = half2_bits_to_float2(kw.x), k23 = half2_bits_to_float2(kw.y);
+        const float2 v01 = half2_bits_to_float2(vw.x), v23 = half2_bits_to_float2(vw.y);
+        const float kv[4] = {k01.x, k01.y, k23.x, k23.y}, vv[4] = {v01.x, v01.y, v23.x, v23.y};
+        float ko[4], vo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const bool live = (i + e) / NG < nk;
+          ko[e] = live ? kv[e] : 0.0f;
+          vo[e] = live ? vv[e] : 0.0f;
+        }
+        *reinterpret_cast<float4*>(sk + i) = make_float4(ko[0], ko[1], ko[2], ko[3]);
+        *reinterpret_cast<float4*>(sv + i) = make_float4(vo[0], vo[1], vo[2], vo[3]);
+      }
+    }
+    __syncwarp();
+
+    // Scores, log2 units: zs[ht][mt][r] for key 16 mt + g + 8 r of head 4 ht + t.
+    float zs[NH][2][2];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      float acc[NH][NG][4];
+#pragma unroll
+      for (int bb = 0; bb < NBK; ++bb) {
+        const uint32_t w0 = kc[(16 * mt + g) * W32 + 4 * bb + t] ^ kBias8;
+        const uint32_t w1 = kc[(16 * mt + 8 + g) * W32 + 4 * bb + t] ^ kBias8;
+        const uint32_t a0[4] = {lo_pair(w0), lo_pair(w1), hi_pair(w0), hi_pair(w1)};
+        const uint32_t a1[4] = {lo_pair(w0 >> 8), lo_pair(w1 >> 8), hi_pair(w0 >> 8), hi_pair(w1 >> 8)};
+#pragma unroll
+        for (int ht = 0; ht < NH; ++ht) {
+          if constexpr (G == 16) {
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int gi = 2 * bb + h2;
+              mma_init(acc[ht][gi], a0, bq[ht][2 * bb][h2][0], bq[ht][2 * bb][h2][1],
+                       bias[ht][gi][0], bias[ht][gi][1]);
+              mma_acc(acc[ht][gi], a1, bq[ht][2 * bb + 1][h2][0], bq[ht][2 * bb + 1][h2][1]);
+            }
+          } else {
+            const int gi = bb / CPG;
+            if (bb % CPG == 0)
+              mma_init(acc[ht][gi], a0, bq[ht][2 * bb][0][0], bq[ht][2 * bb][0][1],
+                       bias[ht][gi][0], bias[ht][gi][1]);
+            else
+              mma_acc(acc[ht][gi], a0, bq[ht][2 * bb][0][0], bq[ht][2 * bb][0][1]);
+            mma_acc(acc[ht][gi], a1, bq[ht][2 * bb + 1][0][0], bq[ht][2 * bb + 1][0][1]);
+          }
+        }
+      }
+      // z = sum over groups of S_K times the group's partial product (both parts)
+      float s0[NG], s1[NG];
+      load_row<NG>(s0, sk + (16 * mt + g) * NG);
+      load_row<NG>(s1, sk + (16 * mt + 8 + g) * NG);
+#pragma unroll
+      for (int ht = 0; ht < NH; ++ht) {
+        float z0 = 0.0f, z1 = 0.0f;
+#pragma unroll
+        for (int gi = 0; gi < NG; ++gi) {
+          z0 = __fmaf_rn(s0[gi], acc[ht][gi][0] + acc[ht][gi][1], z0);
+          z1 = __fmaf_rn(s1[gi], acc[ht][gi][2] + acc[ht][gi][3], z1);
+        }
+        const bool head = 4 * ht + t < R;
+        zs[ht][mt][0] = (head && 16 * mt + g < nk) ? z0 * P.scale_log2 : -INFINITY;
+        zs[ht][mt][1] = (head && 16 * mt + 8 + g < nk) ? z1 * P.scale_log2 : -INFINITY;
+      }
+    }
+
+    // Online softmax per head, over the block's 32 keys: the eight lanes of a
+    // head (same t) hold four keys each.
+#pragma unroll
+    for (int ht = 0; ht < NH; ++ht) {
+      float mx = fmaxf(fmaxf(zs[ht][0][0], zs[ht][0][1]), fmaxf(zs[ht][1][0], zs[ht][1][1]));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+      const float mnew = fmaxf(m[ht], mx);
+      const float alpha = (mnew == -INFINITY) ? 1.0f : exp2f(m[ht] - mnew);
+      m[ht] = mnew;
+      if (__any_sync(kFull, alpha != 1.0f)) {   // skipped once the running maxima settle
+        l[ht] *= alpha;
+#pragma unroll
+        for (int n = 0; n < NCT; ++n) {       // this lane's output columns are head 4 ht + t
+          O[ht][n][0] *= alpha; O[ht][n][1] *= alpha; O[ht][n][2] *= alpha; O[ht][n][3] *= alpha;
+        }
+        const float alpha_b = __shfl_sync(kFull, alpha, g >> 1);   // head 4 ht + g/2
+#pragma unroll
+        for (int gi = 0; gi < NG; ++gi) pc[ht][gi] *= alpha_b;
+      }
+      // key 16 mt + 8 r + g goes to slot 16 mt + 8 r + 2 (g & 3) + (g >> 2):
+      // the value product's lane t reads keys t, t + 4 (and t + 8, t + 12) of
+      // each 16 as one 8-byte pair
+      float* prow = pw + (4 * ht + t) * PS + 2 * (g & 3) + (g >> 2);
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const float z = zs[ht][mt][r];
+          const float p = (z == -INFINITY) ? 0.0f : exp2f(z - mnew);
+          l[ht] += p;
+          prow[16 * mt + 8 * r] = p;
+        }
+    }
+    __syncwarp();
+
+    // Values, per 16-key step: O[ht][ct] (rows = 16 channels of tile ct,
+    // columns = head 4 ht + c/2, part c & 1) += V codes x (p S_V); the codes
+    // of a channel pair of four keys come together with byte permutes.  The
+    // k-indices (2t, 2t+1, 2t+8, 2t+9) are keys t, t + 4, t + 8, t + 12 of
+    // the step, so that the four lanes t of a load read rows of both
+    // parities (two-way, not four-way, bank conflicts on 64-byte rows).
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+      const int ka = 16 * ks + t;                    // keys ka, ka + 4, ka + 8, ka + 12
+      float2 pa[NH], pb[NH];
+#pragma unroll
+      for (int ht = 0; ht < NH; ++ht) {
+        const float* prow = pw + (4 * ht + (g >> 1)) * PS + 16 * ks + 2 * t;
+        pa[ht] = *reinterpret_cast<const float2*>(prow);
+        pb[ht] = *reinterpret_cast<const float2*>(prow + 8);
+      }
+      constexpr int GC = NG < 4 ? NG : 4;             // groups per scale load
+      float sq[4][GC];
+#pragma unroll
+      for (int gi = 0; gi < NG; ++gi) {
+        // B fragments of this group: p S_V for the four keys, as part g & 1
+        if (gi % GC == 0) {
+          load_row<GC>(sq[0], sv + ka * NG + gi);
+          load_row<GC>(sq[1], sv + (ka + 4) * NG + gi);
+          load_row<GC>(sq[2], sv + (ka + 8) * NG + gi);
+          load_row<GC>(sq[3], sv + (ka + 12) * NG + gi);
+        }
+        const float s0 = sq[0][gi % GC], s1 = sq[1][gi % GC], s2 = sq[2][gi % GC], s3 = sq[3][gi % GC];
+        uint32_t bv[NH][2];
+#pragma unroll
+        for (int ht = 0; ht < NH; ++ht) {
+          const float x0 = pa[ht].x * s0, x1 = pa[ht].y * s1, x2 = pb[ht].x * s2, x3 = pb[ht].y * s3;
+          pc[ht][gi] += (x0 + x1) + (x2 + x3);
+          const float2 h01 = half2_bits_to_float2(float2_to_half2_bits(x0, x1));
+          const float2 h23 = half2_bits_to_float2(float2_to_half2_bits(x2, x3));
+          bv[ht][0] = float2_to_half2_bits(__fmaf_rn(-part_f, h01.x, x0), __fmaf_rn(-part_f, h01.y, x1));
+          bv[ht][1] = float2_to_half2_bits(__fmaf_rn(-part_f, h23.x, x2), __fmaf_rn(-part_f, h23.y, x3));
+        }
+        if constexpr (G == 16) {
+          // tile gi: channels 16 gi + 2 g (low nibble, row g) and + 1 (row g + 8):
+          // byte g & 3 of word 2 gi + g / 4
+          const int wv = 2 * gi + (g >> 2), by = g & 3;
+          const uint32_t w0 = vc[ka * W32 + wv], w1 = vc[(ka + 4) * W32 + wv];
+          const uint32_t w2 = vc[(ka + 8) * W32 + wv], w3 = vc[(ka + 12) * W32 + wv];
+          const uint32_t sel = static_cast<uint32_t>(by | ((4 + by) << 4));
+          const uint32_t x = __byte_perm(__byte_perm(w0, w1, sel), __byte_perm(w2, w3, sel), 0x5140u) ^ kBias8;
+          const uint32_t av[4] = {lo_pair(x), hi_pair(x), lo_pair(x >> 8), hi_pair(x >> 8)};
+#pragma unroll
+          for (int ht = 0; ht < NH; ++ht) mma_acc(O[ht][gi], av, bv[ht][0], bv[ht][1]);
+        } else {
+          // tile pair j (32 channels, in group gi): tile 2j takes byte 2 (g & 1)
+          // of word 4j + g/2 (channels 32j + 4g, + 1), tile 2j + 1 the next byte
+#pragma unroll
+          for (int j = gi * (G / 32); j < (gi + 1) * (G / 32); ++j) {
+            const int wv = 4 * j + (g >> 1), ba = 2 * (g & 1);
+            const uint32_t w0 = vc[ka * W32 + wv], w1 = vc[(ka + 4) * W32 + wv];
+            const uint32_t w2 = vc[(ka + 8) * W32 + wv], w3 = vc[(ka + 12) * W32 + wv];
+            const uint32_t sel = static_cast<uint32_t>(ba | ((4 + ba) << 4) | ((ba + 1) << 8) | ((5 + ba) << 12));
+            const uint32_t pp = __byte_perm(w0, w1, sel), qq = __byte_perm(w2, w3, sel);
+            const uint32_t xa = __byte_perm(pp, qq, 0x5140u) ^ kBias8, xb = __byte_perm(pp, qq, 0x7362u) ^ kBias8;
+            const uint32_t aa[4] = {lo_pair(xa), hi_pair(xa), lo_pair(xa >> 8), hi_pair(xa >> 8)};
+            const uint32_t ab[4] = {lo_pair(xb), hi_pair(xb), lo_pair(xb >> 8), hi_pair(xb >> 8)};
+#pragma unroll
+            for (int ht = 0; ht < NH; ++ht) {
+              mma_acc(O[ht][2 * j], aa, bv[ht][0], bv[ht][1]);
+              mma_acc(O[ht][2 * j + 1], ab, bv[ht][0], bv[ht][1]);
+            }
+          }
+        }
+      }
+    }
+    __syncwarp();                      // the stage and the probability rows are consumed
+    issue(blk + ST * kAW, stage);
+  }
+  bool lost = false;                   // a copy may still land in this warp's ring
+  if (failed) {
+    if (lane == 0) atomicOr(&g_attn_fault, 1u);
+    // drain whatever this warp still has in flight, the stage that gave up
+    // included, before the ring is reused
+    for (int s = 0; s < ST; ++s) {
+      const int kk2 = k + s;
+      if (warp + kk2 * kAW < nblk && !mbar_wait(&bar[kk2 % ST], (kk2 / ST) & 1, kSpin))
+        lost = true;
+    }
+    lost = __any_sync(kFull, lost);
+  }
+#pragma unroll
+  for (int ht = 0; ht < NH; ++ht) {
+    l[ht] += __shfl_xor_sync(kFull, l[ht], 4);
+    l[ht] += __shfl_xor_sync(kFull, l[ht], 8);
+    l[ht] += __shfl_xor_sync(kFull, l[ht], 16);
+  }
+  // the bias sums of head 4 ht + t (lanes 8t .. 8t + 3 hold them after the
+  // reduction over t)
+  float bsum[NH][NG];
+#pragma unroll
+  for (int ht = 0; ht < NH; ++ht)
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+      float v = pc[ht][gi];
+      v += __shfl_xor_sync(kFull, v, 1);
+      v += __shfl_xor_sync(kFull, v, 2);
+      bsum[ht][gi] = 8.0f * __shfl_sync(kFull, v, 8 * t);
+    }
+  // every warp is out of the ring: reuse it for the merge, unless a copy may
+  // still land there (the fault word is set; the block writes nothing)
+  if (__syncthreads_or(lost)) return;
+  // this warp's rotated-domain sums: y = 2^24 (both parts), high-nibble rows
+  // / 16, less the bias of the biased codes
+#pragma unroll
+  for (int ht = 0; ht < NH; ++ht) {
+    const int h = 4 * ht + t;
+    if (h < R) {
+      float* cw = comb + (warp * kMaxRows + h) * D;
+#pragma unroll
+      for (int ct = 0; ct < NCT; ++ct) {
+        const int byte = (G == 16) ? 8 * ct + g : 16 * (ct >> 1) + 2 * g + (ct & 1);
+        const float bz = bsum[ht][(G == 16) ? ct : (32 * (ct >> 1)) / G];
+        cw[2 * byte] = __fmaf_rn(O[ht][ct][0] + O[ht][ct][1], 0x1p24f, -bz);
+        cw[2 * byte + 1] = __fmaf_rn(O[ht][ct][2] + O[ht][ct][3], 0x1p20f, -bz);
+      }
+      if (g == 0) {
+        ml[(warp * kMaxRows + h) * 2] = m[ht];
+        ml[(warp * kMaxRows + h) * 2 + 1] = l[ht];
+      }
+    }
+  }
+  __syncthreads();
+  for (int r = warp; r < R; r += kAW) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w2 = 0; w2 < kAW; ++w2) M = fmaxf(M, ml[(w2 * kMaxRows + r) * 2]);
+    float lsum = 0.0f, v[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) v[i] = 0.0f;
+#pragma unroll
+    for (int w2 = 0; w2 < kAW; ++w2) {
+      const float mw = ml[(w2 * kMaxRows + r) * 2];
+      const float e = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
+      lsum += e * ml[(w2 * kMaxRows + r) * 2 + 1];
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) v[i] += e * comb[(w2 * kMaxRows + r) * D + DPL * lane + i];
+    }
+    if (P.nsplit == 1) {
+      uint16_t* orow = P.out + (static_cast<int64_t>(b) * P.Hkv * R + kvh * R + r) * D;
+      finish_head<D>(P, v, lsum, orow, lane, comb + r * D);   // row r's first slot: read above
+    } else {
+      float* pr = P.part + (static_cast<int64_t>(item) * R + r) * (D + 4);
+      if (lane == 0) { pr[0] = M; pr[1] = lsum; }
+#pragma unroll
+      for (int i = 0; i < DPL; ++i) pr[4 + DPL * lane + i] = v[i];
+    }
+  }
+}
+
+// Merge of the key splits of one (sequence, KV head): one warp per head.
+template <int D>
+__global__ void __launch_bounds__(kMaxRows * 32)
+kvq_attn_combine_kernel(const __grid_constant__ AttnParams P) {
+  __shared__ float scr[kMaxRows][D];
+  constexpr int DPL = D / 32;
+  const int bh = blockIdx.x, b = bh / P.Hkv, kvh = bh % P.Hkv;
+  const int r = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (r >= P.R) return;
+  const int64_t stride = static_cast<int64_t>(P.R) * (D + 4);
+  const float* base = P.part + (static_cast<int64_t>(bh) * P.nsplit * P.R + r) * (D + 4);
+  float M = -INFINITY;
+  for (int s = 0; s < P.nsplit; ++s) M = fmaxf(M, base[s * stride]);
+  float lsum = 0.0f, v[DPL];
+#pragma unroll
+  for (int i = 0; i < DPL; ++i) v[i] = 0.0f;
+  for (int s = 0; s < P.nsplit; ++s) {
+    const float* pr = base + s * stride;
+    const float e = (pr[0] == -INFINITY) ? 0.0f : exp2f(pr[0] - M);
+    lsum += e * pr[1];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) v[i] += e * pr[4 + DPL * lane + i];
+  }
+  uint16_t* orow = P.out + (static_cast<int64_t>(b) * P.Hkv * P.R + kvh * P.R + r) * D;
+  finish_head<D>(P, v, lsum, orow, lane, scr[r]);
+}
+
+
+// ---------------------------------------------------------------------------
+// Launch plumbing.
+// ---------------------------------------------------------------------------
+
+template <int D, int G, int NH>
+int launch_attn(const AttnParams& P, int64_t pairs, cudaStream_t st) {
+  using A = Attn<D, G>;
+  auto k = kvq_attn_kernel<D, G, NH>;
+  static std::atomic<int> ready[64];             // the shared-memory opt-in, once per device
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (dev < 0 || dev >= 64 || ready[dev].load(std::memory_order_relaxed) == 0) {
+    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, A::SMEM);
+    if (dev >= 0 && dev < 64) ready[dev].store(1, std::memory_order_relaxed);
+  }
+  const int64_t items = pairs * P.nsplit;
+  (void)cudaGetLastError();
+  k<<<static_cast<unsigned>(items), kAW * 32, A::SMEM, st>>>(P);
+  if (P.nsplit > 1)
+    kvq_attn_combine_kernel<D><<<static_cast<unsigned>(pairs), kMaxRows * 32, 0, st>>>(P);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    g_attn_cuda_error = static_cast<int>(e);
+    return KVQ_ERR_LAUNCH;
+  }
+  return KVQ_OK;
+}
+
+template <int D, int G>
+int launch_nh(const AttnParams& P, int64_t pairs, cudaStream_t st) {
+  return P.R <= 4 ? launch_attn<D, G, 1>(P, pairs, st) : launch_attn<D, G, 2>(P, pairs, st);
+}
+
+}  // namespace
+
+#define KVQA_CAT2(a, b) a##b
+#define KVQA_CAT(a, b) KVQA_CAT2(a, b)
+
+__attribute__((visibility("hidden"))) int KVQA_CAT(kvq_attn_launch_, KVQ_ATTN_D)(
+    const kvqa::AttnParams& P, int64_t pairs, int group, cudaStream_t st) {
+  constexpr int D = KVQ_ATTN_D;
+  switch (group) {
+    case 16: return launch_nh<D, 16>(P, pairs, st);
+    case 32: return launch_nh<D, 32>(P, pairs, st);
+    case 64: return launch_nh<D, 64>(P, pairs, st);
+    default:
+      if constexpr (D >= 128) return launch_nh<D, 128>(P, pairs, st);
+      return KVQ_ERR_GROUP;
+  }
+}
+
+// Read (and optionally clear) this unit's fault word.
+__attribute__((visibility("hidden"))) unsigned int KVQA_CAT(kvq_attn_fault_word_, KVQ_ATTN_D)(int clear) {
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_attn_fault, sizeof(v)) != cudaSuccess) return 0;
+  if (clear && v) {
+    const unsigned int zero = 0;
+    cudaMemcpyToSymbol(g_attn_fault, &zero, sizeof(zero));
+  }
+  return v;
+}
+__attribute__((visibility("hidden"))) int KVQA_CAT(kvq_attn_last_cuda_error_, KVQ_ATTN_D)() {
+  return g_attn_cuda_error;
+}

@@ -127,8 +127,8 @@ def test_attention_errors(kvq):
     def call(q=A_, B=1, Hq=32, Hkv=8, T=4096, D=128, G=32, out=A_, lens=A_):
         return kvq.kvq_attention_decode(q, A_, A_, A_, A_, lens, A_, A_, A_, A_,
                                         B, Hq, Hkv, T, D, G, 0.1, out)
-    assert call(D=256) == -3 and call(D=96) == -3
-    assert call(G=16) == -4 and call(D=64, G=128) == -4
+    assert call(D=512) == -3 and call(D=96) == -3 and call(D=32) == -3
+    assert call(G=8) == -4 and call(G=256) == -4 and call(D=64, G=128) == -4
     assert call(Hq=40, Hkv=4) == -5          # 10 query heads per KV head
     assert call(Hq=30) == -5                 # not a multiple of Hkv
     assert call(T=4000 + 8) == -5            # T % 16 != 0
@@ -136,7 +136,8 @@ def test_attention_errors(kvq):
     assert call(q=0) == -1 and call(out=0) == -1 and call(lens=0) == -1
     assert call(q=A_ + 8) == -2 and call(out=A_ + 8) == -2 and call(lens=A_ + 2) == -2
     assert call(B=0, q=0, out=0, lens=0) == 0
-    assert kvq.kvq_attention_workspace_bytes(1, 32, 8, 4096, 256, 32) == -1
+    assert kvq.kvq_attention_workspace_bytes(1, 32, 8, 4096, 96, 32) == -1
+    assert kvq.kvq_attention_workspace_bytes(1, 32, 8, 4096, 256, 16) > 0
     assert kvq.kvq_attention_workspace_bytes(4096, 32, 8, 4096, 128, 32) == 0
 
 

@@ -6,10 +6,10 @@ products: the rotated query is split into fp16 hi + lo parts (relative error
 ~2^-22), codes are exact, the scores and the weighted value sums accumulate in
 fp32, p * S_V is split hi + lo again, and the result is rounded once to fp16
 (half an fp16 ulp, 2^-11 relative).  The value product runs on biased codes
-n = q + 8 in [0, 15] and removes the bias 8 sum p S_V once at the end, so the
-fp32 rounding of the accumulated biased sum is not relative to the result:
-each of the ~L/8 tensor-core accumulations of a value entry (hi and lo parts,
-16 keys each) rounds an accumulator of at most 15 sum_t p_t S_V,t 2^-24,
+n = q + 8 in [0, 15] and removes the bias 8 sum p S_V by a second product per
+16 keys, so the fp32 rounding of the accumulated sums is not relative to the
+result: each of the ~L/8 tensor-core accumulations of a value entry (codes
+and bias, 16 keys each) rounds an accumulator of at most 15 sum_t p_t S_V,t 2^-24,
 which after the division by l = sum_t p_t is at most 2 u 15 (L/8 + 8) max S_V
 in the rotated domain (u = 2^-24, eight more for the online rescalings), and
 the inverse rotation (orthonormal) and 1/lambda_V carry that into each output
@@ -110,6 +110,12 @@ CASES = [
     (2, 32, 8, 208, 128, 32, [65, 208]),
     (1, 2, 2, 1024, 128, 32, [1000]),          # few pairs: the key axis splits
     (1, 8, 1, 4096, 64, 32, [4095]),
+    (2, 8, 2, 96, 128, 16, [96, 50]),           # groups of 16 (the paper's)
+    (1, 4, 4, 64, 64, 16, [64]),
+    (2, 8, 2, 64, 256, 32, [64, 23]),           # D = 256 (Gemma-3-1B)
+    (1, 4, 1, 128, 256, 16, [128]),
+    (2, 16, 2, 48, 256, 64, [48, 31]),
+    (1, 8, 1, 64, 256, 128, [60]),
 ]
 
 
@@ -219,6 +225,9 @@ FMT_CASES = [
     (2, 4, 4, 96, 64, 32, [96, 17]),
     (4, 32, 8, 80, 128, 64, [0, 1, 80, 33]),
     (1, 2, 1, 400, 128, 128, [400]),
+    (2, 4, 2, 64, 128, 16, [64, 21]),           # the paper's groups of 16
+    (2, 8, 2, 96, 256, 32, [96, 40]),           # D = 256
+    (1, 8, 1, 64, 256, 16, [64]),
 ]
 
 
