@@ -127,6 +127,14 @@ __device__ __forceinline__ void mma_init(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
 }
 
+// 2^x by the SFU's approximation (relative error about 2^-22, results below
+// 2^-126 flushed to 0, 2^-inf = +0); the softmax weights need no more.
+__device__ __forceinline__ float exp2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // v as fp16 (part 0) or the fp16 remainder v - fp16(v) (part 1): the two parts
 // sum to v within 2^-22 |v|.
 __device__ __forceinline__ uint16_t f16_part(float v, int part) {
@@ -439,6 +447,10 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   for (int ht = 0; ht < NH; ++ht)
 #pragma unroll
     for (int gi = 0; gi < NG; ++gi) pc[ht][gi] = 0.0f;
+  bool head_ok[NH];                    // this lane's score head is a real head
+#pragma unroll
+  for (int ht = 0; ht < NH; ++ht) head_ok[ht] = 4 * ht + t < R;
+  const float scale = P.scale_log2;
   bool failed = false;
   int k = 0;
   for (int blk = warp; blk < nblk; blk += kAW, ++k) {
@@ -455,8 +467,10 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     const uint16_t* vsh = reinterpret_cast<const uint16_t*>(st + 2 * A::CB + A::SB);
     const int nk = min(kBK, k1 - (k0 + blk * kBK));
 
-    // The block's scales as fp32; keys at or past nk (stale or unwritten
-    // rows) get 0, so that their zero weights stay exactly 0.
+    const bool tail = nk < kBK;          // the split's last block may hold fewer keys
+
+    // The block's scales as fp32; in a tail block, keys at or past nk (stale
+    // or unwritten rows) get 0, so that their zero weights stay exactly 0.
 #pragma unroll
     for (int i0 = 0; i0 < kBK * NG; i0 += 128) {
       const int i = i0 + 4 * lane;
@@ -465,13 +479,14 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         const uint2 vw = *reinterpret_cast<const uint2*>(vsh + i);
         const float2 k01 = half2_bits_to_float2(kw.x), k23 = half2_bits_to_float2(kw.y);
         const float2 v01 = half2_bits_to_float2(vw.x), v23 = half2_bits_to_float2(vw.y);
-        const float kv[4] = {k01.x, k01.y, k23.x, k23.y}, vv[4] = {v01.x, v01.y, v23.x, v23.y};
-        float ko[4], vo[4];
+        float ko[4] = {k01.x, k01.y, k23.x, k23.y}, vo[4] = {v01.x, v01.y, v23.x, v23.y};
+        if (tail) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const bool live = (i + e) / NG < nk;
-          ko[e] = live ? kv[e] : 0.0f;
-          vo[e] = live ? vv[e] : 0.0f;
+          for (int e = 0; e < 4; ++e) {
+            const bool live = (i + e) / NG < nk;
+            ko[e] = live ? ko[e] : 0.0f;
+            vo[e] = live ? vo[e] : 0.0f;
+          }
         }
         *reinterpret_cast<float4*>(sk + i) = make_float4(ko[0], ko[1], ko[2], ko[3]);
         *reinterpret_cast<float4*>(sv + i) = make_float4(vo[0], vo[1], vo[2], vo[3]);
@@ -523,9 +538,12 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
           z0 = __fmaf_rn(s0[gi], acc[ht][gi][0] + acc[ht][gi][1], z0);
           z1 = __fmaf_rn(s1[gi], acc[ht][gi][2] + acc[ht][gi][3], z1);
         }
-        const bool head = 4 * ht + t < R;
-        zs[ht][mt][0] = (head && 16 * mt + g < nk) ? z0 * P.scale_log2 : -INFINITY;
-        zs[ht][mt][1] = (head && 16 * mt + 8 + g < nk) ? z1 * P.scale_log2 : -INFINITY;
+        zs[ht][mt][0] = z0 * scale;
+        zs[ht][mt][1] = z1 * scale;
+        if (tail || !head_ok[ht]) {          // keys past nk and padded heads weigh 0
+          if (!head_ok[ht] || 16 * mt + g >= nk) zs[ht][mt][0] = -INFINITY;
+          if (!head_ok[ht] || 16 * mt + 8 + g >= nk) zs[ht][mt][1] = -INFINITY;
+        }
       }
     }
 
@@ -538,7 +556,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
       const float mnew = fmaxf(m[ht], mx);
-      const float alpha = (mnew == -INFINITY) ? 1.0f : exp2f(m[ht] - mnew);
+      const float alpha = (mnew == -INFINITY) ? 1.0f : exp2_fast(m[ht] - mnew);
       m[ht] = mnew;
       if (__any_sync(kFull, alpha != 1.0f)) {   // skipped once the running maxima settle
         l[ht] *= alpha;
@@ -558,8 +576,9 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          const float z = zs[ht][mt][r];
-          const float p = (z == -INFINITY) ? 0.0f : exp2f(z - mnew);
+          // a real head has a finite maximum from its first block on, so a
+          // masked key gives 2^-inf = 0; a padded head's weights are never read
+          const float p = exp2_fast(zs[ht][mt][r] - mnew);
           l[ht] += p;
           prow[16 * mt + 8 * r] = p;
         }
