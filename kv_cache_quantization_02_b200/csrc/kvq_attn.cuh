@@ -114,17 +114,17 @@ constexpr uint32_t kBias8 = 0x88888888u;
 __device__ __forceinline__ uint32_t lo_pair(uint32_t x) { return x & 0x000F000Fu; }
 __device__ __forceinline__ uint32_t hi_pair(uint32_t x) { return x & 0x00F000F0u; }
 
-// d = a b + c on the tensor cores (m16n8k16, fp16 operands, fp32 accumulate).
+// d = a b + d on the tensor cores (m16n8k16, fp16 operands, fp32 accumulate),
+// and d = a b.
 __device__ __forceinline__ void mma_acc(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ void mma_init(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1,
-                                         float c0, float c1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%10,%11};"
+__device__ __forceinline__ void mma_init(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c0), "f"(c1));
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
 // 2^x by the SFU's approximation (relative error about 2^-22, results below
@@ -403,11 +403,11 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         bq[ht][j][0][1] = b1;
       }
     }
-  // Score accumulators start at the bias of the biased codes: -8 2^-24 times
+  // The bias of the biased codes in a group's partial score: -8 2^-24 times
   // the group's sum of the B entries (times 16 for the high-nibble entries),
-  // per column of this lane: head 4 ht + t, both parts.  The eight lanes of a
-  // column split the group's channels and add up by shuffles.
-  float bias[NH][NG][2];
+  // both parts, of this lane's score head 4 ht + t.  The eight lanes of a
+  // head split the group's channels and add up by shuffles.
+  float bias[NH][NG];
 #pragma unroll
   for (int ht = 0; ht < NH; ++ht) {
     const float* qr = qf + (4 * ht + t) * D;
@@ -426,8 +426,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         s0 += __shfl_xor_sync(kFull, s0, o);
         s1 += __shfl_xor_sync(kFull, s1, o);
       }
-      bias[ht][gi][0] = -8.0f * 0x1p-24f * s0;
-      bias[ht][gi][1] = -8.0f * 0x1p-24f * s1;
+      bias[ht][gi] = -8.0f * 0x1p-24f * (s0 + s1);
     }
   }
   const float part_f = static_cast<float>(g & 1);
@@ -511,15 +510,13 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int gi = 2 * bb + h2;
-              mma_init(acc[ht][gi], a0, bq[ht][2 * bb][h2][0], bq[ht][2 * bb][h2][1],
-                       bias[ht][gi][0], bias[ht][gi][1]);
+              mma_init(acc[ht][gi], a0, bq[ht][2 * bb][h2][0], bq[ht][2 * bb][h2][1]);
               mma_acc(acc[ht][gi], a1, bq[ht][2 * bb + 1][h2][0], bq[ht][2 * bb + 1][h2][1]);
             }
           } else {
             const int gi = bb / CPG;
             if (bb % CPG == 0)
-              mma_init(acc[ht][gi], a0, bq[ht][2 * bb][0][0], bq[ht][2 * bb][0][1],
-                       bias[ht][gi][0], bias[ht][gi][1]);
+              mma_init(acc[ht][gi], a0, bq[ht][2 * bb][0][0], bq[ht][2 * bb][0][1]);
             else
               mma_acc(acc[ht][gi], a0, bq[ht][2 * bb][0][0], bq[ht][2 * bb][0][1]);
             mma_acc(acc[ht][gi], a1, bq[ht][2 * bb + 1][0][0], bq[ht][2 * bb + 1][0][1]);
@@ -535,8 +532,8 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         float z0 = 0.0f, z1 = 0.0f;
 #pragma unroll
         for (int gi = 0; gi < NG; ++gi) {
-          z0 = __fmaf_rn(s0[gi], acc[ht][gi][0] + acc[ht][gi][1], z0);
-          z1 = __fmaf_rn(s1[gi], acc[ht][gi][2] + acc[ht][gi][3], z1);
+          z0 = __fmaf_rn(s0[gi], (acc[ht][gi][0] + acc[ht][gi][1]) + bias[ht][gi], z0);
+          z1 = __fmaf_rn(s1[gi], (acc[ht][gi][2] + acc[ht][gi][3]) + bias[ht][gi], z1);
         }
         zs[ht][mt][0] = z0 * scale;
         zs[ht][mt][1] = z1 * scale;
