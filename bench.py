@@ -330,6 +330,9 @@ def run_gpu(args):
         cache = build_decode_cache(torch, kvq, dev, stream, lam_t, s_t, G, args.attn_seqs)
         extra = {"attention_decode": run_attention(torch, kvq, dev, stream, lam_t, s_t, G, cache)}
         del cache
+        torch.cuda.empty_cache()
+        extra["attention_decode_paper_format"] = run_attention_paper_format(torch, kvq, dev, stream,
+                                                                            args.attn_seqs)
     elif args.tc_only:
         extra = {"dequantize_tensor_cores": run_dequant_tc(torch, kvq, dev, stream, x, out, lam_t, s_t)}
     elif args.roundtrip_only:
@@ -452,6 +455,7 @@ def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, attn_seqs=64):
                                              steps=1000 if attn_seqs == 64 else 20)
         del cache
         torch.cuda.empty_cache()
+        res["attention_decode_paper_format"] = run_attention_paper_format(torch, kvq, dev, stream, attn_seqs)
         res["configs"] = run_configs(torch, kvq, dev, stream)
         res["d256"] = run_d256(torch, kvq, dev, stream)
     return res
@@ -754,6 +758,52 @@ def run_attention(torch, kvq, dev, stream, lam_t, s_t, G, cache):
         "frac_of_peak": round(gbs / peak, 4),
         "peak_kind": kind,
         "traffic": traffic_per_launch("kvq_attention", rows),
+    }
+
+
+def run_attention_paper_format(torch, kvq, dev, stream, seqs=64):
+    """The same decode step over a cache in the paper's own format (SRFT
+    rotation, lambda after it, groups of 16: technical summary, Methodologie
+    1-3), written by kvq_quantize_ex from the same N(0,1) rows.  Algorithmic
+    bytes: every K and V code and scale once (2 x (64 + 16) per row pair),
+    plus q and the output."""
+    import numpy as np
+    c = workloads.WORKLOADS["decode-cache"]
+    B, Hkv, T, D, G = seqs * 36, DECODE_HKV, DECODE_T, 128, 16
+    Hq = DECODE_HQ
+    rows = 2 * B * Hkv * T
+    pk = torch.empty((2, B, Hkv, T, D // 2), dtype=torch.uint8, device=dev)
+    sc = torch.empty((2, B, Hkv, T, D // G), dtype=torch.float16, device=dev)
+    pk2, sc2 = pk.view(rows, D // 2), sc.view(rows, D // G)
+    lam, sgn = workloads.params(D, c.seed + 7)
+    lam_t, s_t = torch.from_numpy(lam).to(dev), torch.from_numpy(sgn).to(dev)
+    chunk = 1 << 23
+    buf = torch.empty((chunk, D), dtype=torch.float16, device=dev)
+    for i, a in enumerate(range(0, rows, chunk)):
+        b = min(rows, a + chunk)
+        xr = workloads.device_rows(c, b - a, dev, seed_offset=i, out=buf[: b - a])
+        kvq.quantize_ex(xr, lam_t, s_t, G, lambda_after=True, srft=True,
+                        codes=pk2[a:b], scales=sc2[a:b], stream=stream)
+    del buf
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(c.seed)
+    q = torch.randn((B, Hq, D), device=dev, generator=gen).half()
+    lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    scale = 1.0 / math.sqrt(D)
+    ms = _event_ms(torch, stream, lambda: kvq.attention_decode(
+        q, pk[0], sc[0], pk[1], sc[1], lens, lam_t, s_t, lam_t, s_t, G, scale, out=out,
+        stream=stream, lambda_after=True, srft=True), 10)
+    byts = rows * (D // 2 + 2 * (D // G)) + 2 * q.numel() * 2
+    peak, kind = hbm_peak()
+    gbs = byts / (ms / 1e3) / 1e9
+    del q, out, pk, sc
+    torch.cuda.empty_cache()
+    return {
+        "shape": f"B={B} ({seqs} sequences x 36 layers), Hq={Hq}, Hkv={Hkv}, T={T}, D={D}, G={G}, "
+                 "SRFT, lambda after",
+        "ms": round(ms, 4), "algorithmic_bytes": byts, "gbs": round(gbs, 1),
+        "frac_of_peak": round(gbs / peak, 4), "peak_kind": kind,
     }
 
 

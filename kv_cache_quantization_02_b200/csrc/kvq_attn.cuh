@@ -127,6 +127,20 @@ __device__ __forceinline__ void mma_init(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
+// Four 8x8 matrices of 16-bit elements from shared memory (ldmatrix): lane
+// i gives the address of row i % 8 of matrix i / 8 (16 bytes, 16-byte
+// aligned).  Lane (g, t) = (i / 4, i % 4) receives, of matrix j, elements
+// (g, 2t) and (g, 2t + 1) (plain: the 32-bit word t of row g), or with .trans
+// elements (2t, g) and (2t + 1, g) (the 16-bit column g of rows 2t, 2t + 1).
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* row) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_addr(row)));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* row) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_addr(row)));
+}
+
 // 2^x by the SFU's approximation (relative error about 2^-22, results below
 // 2^-126 flushed to 0, 2^-inf = +0); the softmax weights need no more.
 __device__ __forceinline__ float exp2_fast(float x) {
@@ -498,10 +512,16 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
       float acc[NH][NG][4];
+      uint32_t kw[4];
 #pragma unroll
       for (int bb = 0; bb < NBK; ++bb) {
-        const uint32_t w0 = kc[(16 * mt + g) * W32 + 4 * bb + t] ^ kBias8;
-        const uint32_t w1 = kc[(16 * mt + 8 + g) * W32 + 4 * bb + t] ^ kBias8;
+        // words 4 bb + t of keys g and g + 8, two blocks bb per load: matrix
+        // j = (keys 8 (j & 1) .. + 7 of the M-tile, 16-byte chunk bb + j / 2)
+        if (bb % 2 == 0)
+          ldsm_x4(kw, reinterpret_cast<const uint8_t*>(kc) + (16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1)) * (D / 2) +
+                          16 * (bb + (lane >> 4)));
+        const uint32_t w0 = kw[2 * (bb & 1)] ^ kBias8;
+        const uint32_t w1 = kw[2 * (bb & 1) + 1] ^ kBias8;
         const uint32_t a0[4] = {lo_pair(w0), lo_pair(w1), hi_pair(w0), hi_pair(w1)};
         const uint32_t a1[4] = {lo_pair(w0 >> 8), lo_pair(w1 >> 8), hi_pair(w0 >> 8), hi_pair(w1 >> 8)};
 #pragma unroll
@@ -565,10 +585,10 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
 #pragma unroll
         for (int gi = 0; gi < NG; ++gi) pc[ht][gi] *= alpha_b;
       }
-      // key 16 mt + 8 r + g goes to slot 16 mt + 8 r + 2 (g & 3) + (g >> 2):
-      // the value product's lane t reads keys t, t + 4 (and t + 8, t + 12) of
-      // each 16 as one 8-byte pair
-      float* prow = pw + (4 * ht + t) * PS + 2 * (g & 3) + (g >> 2);
+      // key 16 mt + 8 r + g goes to slot 16 mt + 8 r + g (G >= 32), or to
+      // 16 mt + 8 r + 2 (g & 3) + (g >> 2) (G = 16, whose value product's
+      // lane t reads keys t, t + 4 and t + 8, t + 12 of each 16 as 8-byte pairs)
+      float* prow = pw + (4 * ht + t) * PS + ((G == 16) ? 2 * (g & 3) + (g >> 2) : g);
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
@@ -583,14 +603,18 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     __syncwarp();
 
     // Values, per 16-key step: O[ht][ct] (rows = 16 channels of tile ct,
-    // columns = head 4 ht + c/2, part c & 1) += V codes x (p S_V); the codes
-    // of a channel pair of four keys come together with byte permutes.  The
-    // k-indices (2t, 2t+1, 2t+8, 2t+9) are keys t, t + 4, t + 8, t + 12 of
-    // the step, so that the four lanes t of a load read rows of both
-    // parities (two-way, not four-way, bank conflicts on 64-byte rows).
+    // columns = head 4 ht + c/2, part c & 1) += V codes x (p S_V).  G >= 32:
+    // the k-indices (2t, 2t+1, 2t+8, 2t+9) are keys 2t, 2t+1, 2t+8, 2t+9 of
+    // the step, and a transposing ldmatrix gives lane (g, t) bytes 2g, 2g+1
+    // of a 16-byte chunk of keys 2t and 2t+1 in one word (the same channel of
+    // both keys at bits 0-3 and 16-19).  G = 16: they are keys t, t + 4,
+    // t + 8, t + 12, gathered with byte permutes from word reads (the four
+    // lanes t of a read then hit rows of both parities: two-way, not
+    // four-way, bank conflicts on 64-byte rows).
+    constexpr int KSTEP = (G == 16) ? 4 : 1;         // key stride inside a k-index pair
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
-      const int ka = 16 * ks + t;                    // keys ka, ka + 4, ka + 8, ka + 12
+      const int ka = 16 * ks + ((G == 16) ? t : 2 * t);   // keys ka, ka + KSTEP (+ 8)
       float2 pa[NH], pb[NH];
 #pragma unroll
       for (int ht = 0; ht < NH; ++ht) {
@@ -600,14 +624,15 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
       }
       constexpr int GC = NG < 4 ? NG : 4;             // groups per scale load
       float sq[4][GC];
+      uint32_t vw[4];                                 // two chunks of V codes, transposed
 #pragma unroll
       for (int gi = 0; gi < NG; ++gi) {
         // B fragments of this group: p S_V for the four keys, as part g & 1
         if (gi % GC == 0) {
           load_row<GC>(sq[0], sv + ka * NG + gi);
-          load_row<GC>(sq[1], sv + (ka + 4) * NG + gi);
+          load_row<GC>(sq[1], sv + (ka + KSTEP) * NG + gi);
           load_row<GC>(sq[2], sv + (ka + 8) * NG + gi);
-          load_row<GC>(sq[3], sv + (ka + 12) * NG + gi);
+          load_row<GC>(sq[3], sv + (ka + 8 + KSTEP) * NG + gi);
         }
         const float s0 = sq[0][gi % GC], s1 = sq[1][gi % GC], s2 = sq[2][gi % GC], s3 = sq[3][gi % GC];
         uint32_t bv[NH][2];
@@ -632,18 +657,20 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
 #pragma unroll
           for (int ht = 0; ht < NH; ++ht) mma_acc(O[ht][gi], av, bv[ht][0], bv[ht][1]);
         } else {
-          // tile pair j (32 channels, in group gi): tile 2j takes byte 2 (g & 1)
-          // of word 4j + g/2 (channels 32j + 4g, + 1), tile 2j + 1 the next byte
+          // tile pair j (16-byte chunk j: 32 channels, in group gi): tile 2j
+          // holds channels 32j + 4g (row g, low nibble of byte 2g) and + 1 (row
+          // g + 8), tile 2j + 1 channels + 2 and + 3 (byte 2g + 1)
 #pragma unroll
           for (int j = gi * (G / 32); j < (gi + 1) * (G / 32); ++j) {
-            const int wv = 4 * j + (g >> 1), ba = 2 * (g & 1);
-            const uint32_t w0 = vc[ka * W32 + wv], w1 = vc[(ka + 4) * W32 + wv];
-            const uint32_t w2 = vc[(ka + 8) * W32 + wv], w3 = vc[(ka + 12) * W32 + wv];
-            const uint32_t sel = static_cast<uint32_t>(ba | ((4 + ba) << 4) | ((ba + 1) << 8) | ((5 + ba) << 12));
-            const uint32_t pp = __byte_perm(w0, w1, sel), qq = __byte_perm(w2, w3, sel);
-            const uint32_t xa = __byte_perm(pp, qq, 0x5140u) ^ kBias8, xb = __byte_perm(pp, qq, 0x7362u) ^ kBias8;
-            const uint32_t aa[4] = {lo_pair(xa), hi_pair(xa), lo_pair(xa >> 8), hi_pair(xa >> 8)};
-            const uint32_t ab[4] = {lo_pair(xb), hi_pair(xb), lo_pair(xb >> 8), hi_pair(xb >> 8)};
+            // matrix m = (keys 8 (m & 1) .. + 7 of the step, chunk (j & ~1) + m / 2)
+            if (j % 2 == 0)
+              ldsm_x4_t(vw, reinterpret_cast<const uint8_t*>(vc) +
+                                (16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1)) * (D / 2) +
+                                16 * ((j & ~1) + (lane >> 4)));
+            const uint32_t x0 = vw[2 * (j & 1)] ^ kBias8;       // keys 2t, 2t + 1
+            const uint32_t x1 = vw[2 * (j & 1) + 1] ^ kBias8;   // keys 2t + 8, 2t + 9
+            const uint32_t aa[4] = {lo_pair(x0), hi_pair(x0), lo_pair(x1), hi_pair(x1)};
+            const uint32_t ab[4] = {lo_pair(x0 >> 8), hi_pair(x0 >> 8), lo_pair(x1 >> 8), hi_pair(x1 >> 8)};
 #pragma unroll
             for (int ht = 0; ht < NH; ++ht) {
               mma_acc(O[ht][2 * j], aa, bv[ht][0], bv[ht][1]);
