@@ -2,12 +2,11 @@
 // int4 rotated-domain KV cache (include/kvq.h: kvq_attention_decode,
 // kvq_attention_decode_ex, kvq_attention_decode_static,
 // kvq_attention_workspace_bytes): argument checks, the key-axis split, the
-// SRFT twiddle tables, the static scratch, and the dispatch to the unit of
-// the head dimension (kvq_attn.cuh, compiled once per D in kvq_attn_d<D>.cu).
+// static scratch, and the dispatch to the unit of the head dimension
+// (kvq_attn.cuh, compiled once per D in kvq_attn_d<D>.cu).
 
 #include <cuda.h>
 #include <cuda_runtime.h>
-#include <cuda_fp16.h>
 
 #include <atomic>
 #include <cmath>
@@ -20,10 +19,6 @@
 namespace {
 
 using namespace kvqa;
-constexpr unsigned kFullMask = 0xffffffffu;
-
-#include "kvq_arith.cuh"
-#include "kvq_fft.cuh"                               // root_f32: the SRFT's twiddle table
 
 // Scratch of kvq_attention_decode_static: the partial (max, sum, rotated
 // output) rows of the key splits, 8 MiB per device.  Nothing in it has to
@@ -76,19 +71,6 @@ int check_attn(int B, int Hq, int Hkv, int T, int D, int G) {
     return KVQ_ERR_COUNT;
   if (static_cast<int64_t>(B) * Hkv * T >= (int64_t{1} << 40)) return KVQ_ERR_COUNT;
   return KVQ_OK;
-}
-
-template <int D>
-void attn_twiddles(AttnParams& P) {
-  struct Tw { float2 wn[D / 2]; float2 wd[D / 2 + 1]; };
-  static const Tw tw = [] {
-    Tw t{};
-    for (int k = 0; k < D / 2; ++k) t.wn[k] = root_f32(k, D / 2);
-    for (int k = 0; k <= D / 2; ++k) t.wd[k] = root_f32(k, D);
-    return t;
-  }();
-  memcpy(P.wn, tw.wn, sizeof(tw.wn));
-  memcpy(P.wd, tw.wd, sizeof(tw.wd));
 }
 
 }  // namespace
@@ -176,11 +158,6 @@ int kvq_attention_decode_ex(const uint16_t* q, const uint8_t* k_packed, const ui
   P.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634 * 16777216.0);
   P.c = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   P.c1h = static_cast<float>(1.0 / std::sqrt(2.0 * static_cast<double>(D)));
-  if (flags & kFmtSrft) {
-    if (D == 64) attn_twiddles<64>(P);
-    else if (D == 128) attn_twiddles<128>(P);
-    else attn_twiddles<256>(P);
-  }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (D) {
     case 64: return kvq_attn_launch_64(P, pairs, group, st);

@@ -58,6 +58,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <vector>
 
 #include "kvq.h"
 #include "kvq_attn_common.cuh"
@@ -73,12 +74,50 @@ constexpr unsigned kFullMask = 0xffffffffu;
 
 #include "kvq_async.cuh"
 #include "kvq_arith.cuh"
-#include "kvq_fft.cuh"
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr uint32_t kSpin = 1u << 22;         // bounded mbarrier waits
 
 __device__ unsigned int g_attn_fault = 0;    // bit 0: a wait gave up; bit 3: bad sequence length
+
+// The SRFT at this head dimension as a real D x D matrix, fp32, written once
+// per device by the first launch that needs it: g_srft[j][i] = M[j][i] with
+// y = M x (y_0 = X_0 / sqrt(D), y_1 = X_(D/2) / sqrt(D), (y_2k, y_2k+1) =
+// sqrt(2) (Re, Im) X_k / sqrt(D), X the length-D DFT of x), and g_srft_t its
+// transpose.  The query's and the output's rotations are one warp-wide
+// product each per head (every lane DPL outputs, coalesced rows); no FFT
+// sits on one lane, where its working set spilled to local memory.
+__device__ float g_srft[KVQ_ATTN_D * KVQ_ATTN_D];
+__device__ float g_srft_t[KVQ_ATTN_D * KVQ_ATTN_D];
+
+// out[DPL lane + k] = sum_i mat[i][DPL lane + k] x[i], x in shared memory.
+template <int D>
+__device__ __forceinline__ void warp_matvec(float (&out)[D / 32], const float* __restrict__ mat,
+                                            const float* x, int lane) {
+  constexpr int DPL = D / 32;
+  constexpr int UNR = 64 / DPL;                  // rows in flight: the loads come from L2
+#pragma unroll
+  for (int k = 0; k < DPL; ++k) out[k] = 0.0f;
+#pragma unroll UNR
+  for (int i = 0; i < D; ++i) {
+    const float xi = x[i];
+    const float* row = mat + i * D + DPL * lane;
+    if constexpr (DPL % 4 == 0) {
+#pragma unroll
+      for (int k = 0; k < DPL; k += 4) {
+        const float4 m4 = __ldg(reinterpret_cast<const float4*>(row + k));
+        out[k] = __fmaf_rn(m4.x, xi, out[k]);
+        out[k + 1] = __fmaf_rn(m4.y, xi, out[k + 1]);
+        out[k + 2] = __fmaf_rn(m4.z, xi, out[k + 2]);
+        out[k + 3] = __fmaf_rn(m4.w, xi, out[k + 3]);
+      }
+    } else {
+      const float2 m2 = __ldg(reinterpret_cast<const float2*>(row));
+      out[0] = __fmaf_rn(m2.x, xi, out[0]);
+      out[1] = __fmaf_rn(m2.y, xi, out[1]);
+    }
+  }
+}
 thread_local int g_attn_cuda_error = 0;
 
 template <int D, int G>
@@ -206,8 +245,8 @@ __device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
 //   lambda before: out = fp16((s_V . R^T y) / lambda_V),
 //   lambda after:  out = fp16(s_V . R^T (y / lambda_V)),
 // R^T = H / sqrt(D) (a warp-wide butterfly over the lanes' channels) or the
-// SRFT transpose (the codec's adjoint unpacking and transposed FFT, run by one
-// lane on the row gathered in `scr`, D floats of this warp's shared memory).
+// SRFT's transpose (a warp-wide product with the SRFT matrix, the row
+// gathered in `scr`, D floats of this warp's shared memory).
 template <int D>
 __device__ __forceinline__ void finish_head(const AttnParams& P, float (&v)[D / 32], float l,
                                             uint16_t* out_row, int lane, float* scr) {
@@ -238,30 +277,25 @@ __device__ __forceinline__ void finish_head(const AttnParams& P, float (&v)[D / 
       for (int i = 0; i < DPL; ++i) out_row[DPL * lane + i] = h[i];
     }
   } else {
+    // y (the merged rotated-domain sum) through shared memory, then
+    // out_i = s_V,i sum_j M[j][i] y_j (lambda after: y / lambda_V first, per j)
 #pragma unroll
-    for (int i = 0; i < DPL; ++i) scr[DPL * lane + i] = v[i];
-    __syncwarp();
-    if (lane == 0) {
-      float2 z[D / 2];
-#pragma unroll
-      for (int n = 0; n < D / 2; ++n) z[n] = make_float2(scr[2 * n], scr[2 * n + 1]);
-      unpack_inv1<D>(z, P.wd, [&](int n) -> float2 {
-        float2 f = n == 0 ? make_float2(P.c, P.c) : make_float2(P.c1h, P.c1h);
-        if (after) f = make_float2(f.x / P.lam_v[2 * n], f.y / P.lam_v[2 * n + 1]);
-        return f;
-      });
-      fft_inv_from<D / 2, D / 2, D / 2>(z, P.wn);
-#pragma unroll
-      for (int n = 0; n < D / 2; ++n) {
-        float a = P.s_v[2 * n] < 0 ? -z[n].x : z[n].x;
-        float b = P.s_v[2 * n + 1] < 0 ? -z[n].y : z[n].y;
-        if (!after) {
-          a = a / P.lam_v[2 * n];
-          b = b / P.lam_v[2 * n + 1];
-        }
-        reinterpret_cast<uint32_t*>(out_row)[n] = float2_to_half2_bits(a, b);
-      }
+    for (int i = 0; i < DPL; ++i) {
+      const int d = DPL * lane + i;
+      scr[d] = after ? v[i] / P.lam_v[d] : v[i];
     }
+    __syncwarp();
+    float o[DPL];
+    warp_matvec<D>(o, g_srft, scr, lane);
+    uint16_t h[DPL];
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) {
+      const int d = DPL * lane + i;
+      const float zs = P.s_v[d] < 0 ? -o[i] : o[i];
+      h[i] = __half_as_ushort(__float2half_rn(after ? zs : zs / P.lam_v[d]));
+    }
+#pragma unroll
+    for (int i = 0; i < DPL; ++i) out_row[DPL * lane + i] = h[i];
     __syncwarp();
   }
 }
@@ -334,30 +368,29 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   for (int r = warp; r < kMaxRows; r += kAW) {
     float* qr_out = qf + r * D;
     if (P.fmt & kFmtSrft) {
-      if (lane == 0) {
-        float2 z[D / 2];
-        if (r < R) {
-          const uint32_t* qr = reinterpret_cast<const uint32_t*>(
-              P.q + (static_cast<int64_t>(b) * P.Hkv * R + kvh * R + r) * D);
+      // q' = s_K . q (lambda before: . / lambda_K) in this row's qf slot, then
+      // q~_j = sum_i M[j][i] q'_i (lambda after: / lambda_K,j)
+      if (r < R) {
+        const uint16_t* qr = P.q + (static_cast<int64_t>(b) * P.Hkv * R + kvh * R + r) * D;
 #pragma unroll
-          for (int n = 0; n < D / 2; ++n) {
-            float2 x = half2_bits_to_float2(qr[n]);
-            if (!after) x = make_float2(x.x / P.lam_k[2 * n], x.y / P.lam_k[2 * n + 1]);
-            z[n] = make_float2(P.s_k[2 * n] < 0 ? -x.x : x.x, P.s_k[2 * n + 1] < 0 ? -x.y : x.y);
-          }
-          fft_fwd_from<D / 2, D / 2, D / 2>(z, P.wn);
-          unpack_fwd1<D>(z, P.wd, [&](int n) -> float2 {
-            float2 f = n == 0 ? make_float2(P.c, P.c) : make_float2(P.c1h, P.c1h);
-            if (after) f = make_float2(f.x / P.lam_k[2 * n], f.y / P.lam_k[2 * n + 1]);
-            if (n > D / 4) f.y = -f.y;                 // bins above N/2 come as conj(E - T)
-            return f;
-          });
-        } else {
-#pragma unroll
-          for (int n = 0; n < D / 2; ++n) z[n] = make_float2(0.0f, 0.0f);
+        for (int i = 0; i < DPL; ++i) {
+          const int d = DPL * lane + i;
+          float x = __half2float(__ushort_as_half(qr[d]));
+          if (!after) x = x / P.lam_k[d];
+          qr_out[d] = P.s_k[d] < 0 ? -x : x;
         }
+        __syncwarp();
+        float y[DPL];
+        warp_matvec<D>(y, g_srft_t, qr_out, lane);
+        __syncwarp();
 #pragma unroll
-        for (int n = 0; n < D / 2; ++n) reinterpret_cast<float2*>(qr_out)[n] = z[n];
+        for (int i = 0; i < DPL; ++i) {
+          const int d = DPL * lane + i;
+          qr_out[d] = after ? y[i] / P.lam_k[d] : y[i];
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < DPL; ++i) qr_out[DPL * lane + i] = 0.0f;
       }
       continue;
     }
@@ -796,6 +829,40 @@ kvq_attn_combine_kernel(const __grid_constant__ AttnParams P) {
 // Launch plumbing.
 // ---------------------------------------------------------------------------
 
+// The SRFT matrix and its transpose into this unit's device memory, once per
+// device (synchronous copies: the first SRFT call on a device must not be
+// inside a stream capture).  Entries from the definition, in long double,
+// each rounded once to fp32.
+int upload_srft_matrix() {
+  constexpr int D = KVQ_ATTN_D, N = D / 2;
+  static std::atomic<int> done[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire)) return KVQ_OK;
+  std::vector<float> m(D * D), mt(D * D);
+  const long double pi = 3.141592653589793238462643383279502884L;
+  const long double c = 1.0L / sqrtl(static_cast<long double>(D));
+  for (int i = 0; i < D; ++i) {
+    m[0 * D + i] = static_cast<float>(c);
+    m[1 * D + i] = static_cast<float>((i % 2 ? -1.0L : 1.0L) * c);
+    for (int k = 1; k < N; ++k) {
+      const long double ang = 2.0L * pi * static_cast<long double>((static_cast<long>(i) * k) % D) / D;
+      m[(2 * k) * D + i] = static_cast<float>(sqrtl(2.0L) * c * cosl(ang));
+      m[(2 * k + 1) * D + i] = static_cast<float>(-sqrtl(2.0L) * c * sinl(ang));
+    }
+  }
+  for (int j = 0; j < D; ++j)
+    for (int i = 0; i < D; ++i) mt[i * D + j] = m[j * D + i];
+  cudaError_t e = cudaMemcpyToSymbol(g_srft, m.data(), m.size() * sizeof(float));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_srft_t, mt.data(), mt.size() * sizeof(float));
+  if (e != cudaSuccess) {
+    g_attn_cuda_error = static_cast<int>(e);
+    return KVQ_ERR_LAUNCH;
+  }
+  if (dev >= 0 && dev < 64) done[dev].store(1, std::memory_order_release);
+  return KVQ_OK;
+}
+
 template <int D, int G, int NH>
 int launch_attn(const AttnParams& P, int64_t pairs, cudaStream_t st) {
   using A = Attn<D, G>;
@@ -833,6 +900,10 @@ int launch_nh(const AttnParams& P, int64_t pairs, cudaStream_t st) {
 __attribute__((visibility("hidden"))) int KVQA_CAT(kvq_attn_launch_, KVQ_ATTN_D)(
     const kvqa::AttnParams& P, int64_t pairs, int group, cudaStream_t st) {
   constexpr int D = KVQ_ATTN_D;
+  if (P.fmt & kFmtSrft) {
+    const int rc = upload_srft_matrix();
+    if (rc != KVQ_OK) return rc;
+  }
   switch (group) {
     case 16: return launch_nh<D, 16>(P, pairs, st);
     case 32: return launch_nh<D, 32>(P, pairs, st);

@@ -37,8 +37,6 @@ struct AttnParams {
   float scale_log2;             // sm_scale * log2(e) * 2^24 (the key product comes out scaled by 2^-24)
   float c;                      // fp32 1/sqrt(D)
   float c1h;                    // fp32 1/sqrt(2D): the SRFT's normalisation of 2 X_k
-  float2 wn[128];               // SRFT twiddles omega_(D/2)^k, k < D/2 (SRFT caches only)
-  float2 wd[129];               // omega_D^k, k <= D/2
 };
 
 }  // namespace kvqa
