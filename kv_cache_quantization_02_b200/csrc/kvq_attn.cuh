@@ -127,7 +127,7 @@ struct Attn {
   static constexpr int KS = D / 16;                 // k-steps of the score product
   static constexpr int NCT = D / 16;                // 16-channel tiles of the value product
   static constexpr int W32 = D / 8;                 // 32-bit words of one code row
-  static constexpr int ST = D >= 256 ? 2 : 3;       // ring depth per warp
+  static constexpr int ST = (D >= 256 || G == 16) ? 2 : 3;   // ring depth per warp
   static constexpr int CB = kBK * D / 2;            // code bytes of one block
   static constexpr int SB = kBK * NG * 2;           // scale bytes of one block
   static constexpr int STAGE = 2 * CB + 2 * SB;     // K codes, V codes, K scales, V scales
@@ -303,7 +303,7 @@ __device__ __forceinline__ void finish_head(const AttnParams& P, float (&v)[D / 
 // One block of four warps per (sequence, KV head, key split); head tiles of
 // four query heads (NH = 1 for up to four heads per KV head, 2 for up to 8).
 template <int D, int G, int NH>
-__global__ void __launch_bounds__(kAW * 32, (D >= 256 || NH > 1 || G == 16) ? 2 : 3)
+__global__ void __launch_bounds__(kAW * 32, (D >= 256 || NH > 1) ? 2 : 3)
 kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   using A = Attn<D, G>;
   constexpr int NG = A::NG, NBK = A::NBK, KS = A::KS, NCT = A::NCT, W32 = A::W32, DPL = A::DPL;
@@ -541,10 +541,20 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     __syncwarp();
 
     // Scores, log2 units: zs[ht][mt][r] for key 16 mt + g + 8 r of head 4 ht + t.
+    // A group's partial products fold into the score (times the key's group
+    // scale) as soon as its last k-step is done, so one group's accumulators
+    // (two at G = 16) are live at a time.
     float zs[NH][2][2];
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
-      float acc[NH][NG][4];
+      constexpr int GPB = (G == 16) ? 2 : 1;          // groups finished per 32-channel block
+      float acc[NH][GPB][4];
+      float s0[NG], s1[NG];
+      load_row<NG>(s0, sk + (16 * mt + g) * NG);
+      load_row<NG>(s1, sk + (16 * mt + 8 + g) * NG);
+      float z0[NH], z1[NH];
+#pragma unroll
+      for (int ht = 0; ht < NH; ++ht) z0[ht] = z1[ht] = 0.0f;
       uint32_t kw[4];
 #pragma unroll
       for (int bb = 0; bb < NBK; ++bb) {
@@ -562,34 +572,31 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
           if constexpr (G == 16) {
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
-              const int gi = 2 * bb + h2;
-              mma_init(acc[ht][gi], a0, bq[ht][2 * bb][h2][0], bq[ht][2 * bb][h2][1]);
-              mma_acc(acc[ht][gi], a1, bq[ht][2 * bb + 1][h2][0], bq[ht][2 * bb + 1][h2][1]);
+              mma_init(acc[ht][h2], a0, bq[ht][2 * bb][h2][0], bq[ht][2 * bb][h2][1]);
+              mma_acc(acc[ht][h2], a1, bq[ht][2 * bb + 1][h2][0], bq[ht][2 * bb + 1][h2][1]);
             }
           } else {
-            const int gi = bb / CPG;
             if (bb % CPG == 0)
-              mma_init(acc[ht][gi], a0, bq[ht][2 * bb][0][0], bq[ht][2 * bb][0][1]);
+              mma_init(acc[ht][0], a0, bq[ht][2 * bb][0][0], bq[ht][2 * bb][0][1]);
             else
-              mma_acc(acc[ht][gi], a0, bq[ht][2 * bb][0][0], bq[ht][2 * bb][0][1]);
-            mma_acc(acc[ht][gi], a1, bq[ht][2 * bb + 1][0][0], bq[ht][2 * bb + 1][0][1]);
+              mma_acc(acc[ht][0], a0, bq[ht][2 * bb][0][0], bq[ht][2 * bb][0][1]);
+            mma_acc(acc[ht][0], a1, bq[ht][2 * bb + 1][0][0], bq[ht][2 * bb + 1][0][1]);
+          }
+          // z += S_K (both parts + the codes' bias) for each group done here
+          if (G == 16 || bb % CPG == CPG - 1) {
+#pragma unroll
+            for (int h2 = 0; h2 < GPB; ++h2) {
+              const int gi = (G == 16) ? 2 * bb + h2 : bb / CPG;
+              z0[ht] = __fmaf_rn(s0[gi], (acc[ht][h2][0] + acc[ht][h2][1]) + bias[ht][gi], z0[ht]);
+              z1[ht] = __fmaf_rn(s1[gi], (acc[ht][h2][2] + acc[ht][h2][3]) + bias[ht][gi], z1[ht]);
+            }
           }
         }
       }
-      // z = sum over groups of S_K times the group's partial product (both parts)
-      float s0[NG], s1[NG];
-      load_row<NG>(s0, sk + (16 * mt + g) * NG);
-      load_row<NG>(s1, sk + (16 * mt + 8 + g) * NG);
 #pragma unroll
       for (int ht = 0; ht < NH; ++ht) {
-        float z0 = 0.0f, z1 = 0.0f;
-#pragma unroll
-        for (int gi = 0; gi < NG; ++gi) {
-          z0 = __fmaf_rn(s0[gi], (acc[ht][gi][0] + acc[ht][gi][1]) + bias[ht][gi], z0);
-          z1 = __fmaf_rn(s1[gi], (acc[ht][gi][2] + acc[ht][gi][3]) + bias[ht][gi], z1);
-        }
-        zs[ht][mt][0] = z0 * scale;
-        zs[ht][mt][1] = z1 * scale;
+        zs[ht][mt][0] = z0[ht] * scale;
+        zs[ht][mt][1] = z1[ht] * scale;
         if (tail || !head_ok[ht]) {          // keys past nk and padded heads weigh 0
           if (!head_ok[ht] || 16 * mt + g >= nk) zs[ht][mt][0] = -INFINITY;
           if (!head_ok[ht] || 16 * mt + 8 + g >= nk) zs[ht][mt][1] = -INFINITY;
