@@ -333,6 +333,8 @@ def run_gpu(args):
         torch.cuda.empty_cache()
         extra["attention_decode_paper_format"] = run_attention_paper_format(torch, kvq, dev, stream,
                                                                             args.attn_seqs)
+    elif args.configs_only:
+        extra = {"configs": run_configs(torch, kvq, dev, stream)}
     elif args.tc_only:
         extra = {"dequantize_tensor_cores": run_dequant_tc(torch, kvq, dev, stream, x, out, lam_t, s_t)}
     elif args.roundtrip_only:
@@ -461,15 +463,20 @@ def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, attn_seqs=64):
     return res
 
 
-def _flushed_ms(torch, stream, fn, reps, flush):
+def _flushed_ms(torch, stream, fn, reps, flush, clean=None):
     """Per-rep CUDA-event times of fn, the L2 flushed before each rep by a
-    write of `flush` (twice the L2's 126 MB).  (median, min, max) in ms."""
+    write of `flush` (twice the L2's 126 MB); with `clean` (another buffer
+    larger than L2), a read of it follows the write, so the L2 holds clean
+    lines and the timed kernel does not pay for writing back the flush's
+    dirty ones.  (median, min, max) in ms."""
     fn()
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(reps)]
     for a, b in ev:
         flush.zero_()
+        if clean is not None:
+            clean.max()
         a.record(stream)
         fn()
         b.record(stream)
@@ -484,10 +491,15 @@ CONFIG_CASES = (("tiny", 32), ("qwen2.5-1.5b", 32), ("gemma-3-1b", 32), ("gemma-
 def run_configs(torch, kvq, dev, stream, reps=20):
     """The smaller configurations (each batch fits in L2): quantize and
     dequantize timed one rep at a time with the L2 flushed before each rep;
-    median, min and max in microseconds."""
+    median, min and max in microseconds.  A second pair of figures reads a
+    second 256 MB buffer after the flush's write: the write leaves up to the
+    L2's 126 MB of dirty lines, whose write-back the timed kernel otherwise
+    pays (comparable to these batches' own bytes)."""
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    clean = torch.zeros(256 << 20, dtype=torch.uint8, device=dev)
     peak, _ = hbm_peak()
-    res = {"protocol": f"{reps} reps, L2 flushed (256 MB write) before each; median/min/max"}
+    res = {"protocol": f"{reps} reps, L2 flushed (256 MB write) before each; median/min/max; "
+                       "*_clean: the write followed by a 256 MB read"}
     for name, G in CONFIG_CASES:
         w = workloads.WORKLOADS[name]
         D, n = w.D, w.n_vec
@@ -501,6 +513,10 @@ def run_configs(torch, kvq, dev, stream, reps=20):
             x, lt, st, G, packed=pk, scales=sc, stream=stream), reps, flush)
         d = _flushed_ms(torch, stream, lambda: kvq.dequantize(
             pk, sc, lt, st, G, out=out, stream=stream), reps, flush)
+        qc = _flushed_ms(torch, stream, lambda: kvq.quantize(
+            x, lt, st, G, packed=pk, scales=sc, stream=stream), reps, flush, clean)
+        dc = _flushed_ms(torch, stream, lambda: kvq.dequantize(
+            pk, sc, lt, st, G, out=out, stream=stream), reps, flush, clean)
         bpv = bytes_per_vector(D, G)
         res[f"{name}_g{G}"] = {
             "n_vec": n, "D": D, "G": G, "bytes_per_vector": bpv,
@@ -510,9 +526,13 @@ def run_configs(torch, kvq, dev, stream, reps=20):
             "dequantize_gvec_s": round(n / (d[0] / 1e3) / 1e9, 3),
             "quantize_gbs": round(bpv * n / (q[0] / 1e3) / 1e9, 1),
             "dequantize_gbs": round(bpv * n / (d[0] / 1e3) / 1e9, 1),
+            "quantize_us_clean": [round(v * 1e3, 2) for v in qc],
+            "dequantize_us_clean": [round(v * 1e3, 2) for v in dc],
+            "quantize_gbs_clean": round(bpv * n / (qc[0] / 1e3) / 1e9, 1),
+            "dequantize_gbs_clean": round(bpv * n / (dc[0] / 1e3) / 1e9, 1),
         }
         del x, pk, sc, out
-    del flush
+    del flush, clean
     torch.cuda.empty_cache()
     return res
 
@@ -960,6 +980,8 @@ def parse(argv=None):
                    help="of the secondary figures, only the decode attention (profiling)")
     p.add_argument("--variants-only", action="store_true",
                    help="of the secondary figures, only the codec variants (profiling)")
+    p.add_argument("--configs-only", action="store_true",
+                   help="of the secondary figures, only the smaller configurations (profiling)")
     p.add_argument("--tc-only", action="store_true",
                    help="of the secondary figures, only the tensor-core dequantizer (profiling)")
     p.add_argument("--roundtrip-only", action="store_true",
