@@ -180,6 +180,20 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* row) {
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(smem_addr(row)));
 }
 
+// The two parts of a pair: (x0, x1) as fp16 (part 0), or their fp16
+// remainders x - fp16(x) (part 1; negp = -1 as fp16 bits, else -0).  The
+// remainder comes from one mixed-precision multiply-add per value with the
+// packed fp16 value as operand (exact: x and fp16(x) agree to 11 bits), so
+// no conversion back to fp32 is needed.
+__device__ __forceinline__ uint32_t part_pair(float x0, float x1, uint16_t negp) {
+  const uint32_t h = float2_to_half2_bits(x0, x1);
+  float d0, d1;
+  asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "fma.rn.f32.f16 %0, a, %3, %4;\n\tfma.rn.f32.f16 %1, b, %3, %5;\n\t}"
+      : "=f"(d0), "=f"(d1) : "r"(h), "h"(negp), "f"(x0), "f"(x1));
+  return float2_to_half2_bits(d0, d1);
+}
+
 // 2^x by the SFU's approximation (relative error about 2^-22, results below
 // 2^-126 flushed to 0, 2^-inf = +0); the softmax weights need no more.
 __device__ __forceinline__ float exp2_fast(float x) {
@@ -476,7 +490,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
       bias[ht][gi] = -8.0f * 0x1p-24f * (s0 + s1);
     }
   }
-  const float part_f = static_cast<float>(g & 1);
+  const uint16_t neg_part = (g & 1) ? 0xBC00u : 0x8000u;   // -1 or -0 as fp16
 
   float O[NH][NCT][4];
 #pragma unroll
@@ -680,10 +694,8 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         for (int ht = 0; ht < NH; ++ht) {
           const float x0 = pa[ht].x * s0, x1 = pa[ht].y * s1, x2 = pb[ht].x * s2, x3 = pb[ht].y * s3;
           pc[ht][gi] += (x0 + x1) + (x2 + x3);
-          const float2 h01 = half2_bits_to_float2(float2_to_half2_bits(x0, x1));
-          const float2 h23 = half2_bits_to_float2(float2_to_half2_bits(x2, x3));
-          bv[ht][0] = float2_to_half2_bits(__fmaf_rn(-part_f, h01.x, x0), __fmaf_rn(-part_f, h01.y, x1));
-          bv[ht][1] = float2_to_half2_bits(__fmaf_rn(-part_f, h23.x, x2), __fmaf_rn(-part_f, h23.y, x3));
+          bv[ht][0] = part_pair(x0, x1, neg_part);
+          bv[ht][1] = part_pair(x2, x3, neg_part);
         }
         if constexpr (G == 16) {
           // tile gi: channels 16 gi + 2 g (low nibble, row g) and + 1 (row g + 8):
