@@ -197,6 +197,45 @@ def test_decode_config_sampled():
         _check(got[None], ref[None], sub)
 
 
+def test_decode_config_sampled_paper_format():
+    """The paper's own cache format (SRFT, lambda after, groups of 16) at the
+    bench's decode shape on a slice of sequences: the cache written on the
+    GPU by kvq_quantize_ex from device-drawn rows, sampled (sequence, KV head)
+    pairs checked against the oracle on the same codes."""
+    B, Hq, Hkv, T, D, G = 12, 32, 8, 4096, 128, 16
+    dev = torch.device("cuda")
+    c = workloads.WORKLOADS["decode-cache"]
+    rows = 2 * B * Hkv * T
+    lam, sgn = workloads.params(D, 21)
+    lt, st = torch.from_numpy(lam).to(dev), torch.from_numpy(sgn).to(dev)
+    x = workloads.device_rows(c, rows, dev, seed_offset=3)
+    codes, scales = kvq.quantize_ex(x, lt, st, G, lambda_after=True, srft=True)
+    del x
+    pk = codes.view(2, B, Hkv, T, D // 2)
+    sc = scales.view(2, B, Hkv, T, D // G)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(6)
+    q = torch.randn((B, Hq, D), device=dev, generator=gen).half()
+    lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+    lens[::3] = 2000
+    scale = 1.0 / math.sqrt(D)
+    out = kvq.attention_decode(q, pk[0], sc[0], pk[1], sc[1], lens, lt, st, lt, st, G, scale,
+                               lambda_after=True, srft=True)
+    torch.cuda.synchronize()
+    R = Hq // Hkv
+    for b, kvh in ((0, 0), (5, 7), (11, 3)):
+        L = int(lens[b])
+        sub = dict(q=q[b:b + 1, kvh * R:(kvh + 1) * R].cpu().numpy(),
+                   kp=pk[0, b:b + 1, kvh:kvh + 1].cpu().numpy(), ks=sc[0, b:b + 1, kvh:kvh + 1].cpu().numpy(),
+                   vp=pk[1, b:b + 1, kvh:kvh + 1].cpu().numpy(), vs=sc[1, b:b + 1, kvh:kvh + 1].cpu().numpy(),
+                   lens=np.array([L], dtype=np.int32), lk=lam, sk=sgn, lv=lam, sv=sgn, G=G)
+        ref = oracle.get().attention_decode(sub["q"], sub["kp"], sub["ks"], sub["vp"], sub["vs"],
+                                            sub["lens"], lam, sgn, lam, sgn, G, scale,
+                                            lambda_after=True, srft=True)[0]
+        got = out[b, kvh * R:(kvh + 1) * R].cpu().numpy().astype(np.float64)
+        _check(got[None], ref[None], sub)
+
+
 # ---- caches of the codec variants' formats -----------------------------------
 
 def _case_fmt(B, Hq, Hkv, T, D, G, seed, after, srft, lens=None):
