@@ -357,23 +357,35 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     mbar_fence_init();
   }
   const int64_t row_base = static_cast<int64_t>(bh) * P.T;
-  auto issue = [&](int blk, int stage) {
-    if (blk >= nblk || lane != 0) return;
-    const int kb = k0 + blk * kBK;
-    const int nk = min(kBK, k1 - kb);
-    const int nk16 = (nk + 15) & ~15;                            // stays inside T (T % 16 == 0)
-    const int64_t row0 = row_base + kb;
-    uint8_t* st = ring + (warp * ST + stage) * A::STAGE;
-    const uint32_t cb = static_cast<uint32_t>(nk16 * (D / 2));
-    const uint32_t sb = static_cast<uint32_t>(nk16 * NG * 2);
-    mbar_expect_tx(&bar[stage], 2 * cb + 2 * sb);
-    bulk_g2s(st, P.kp + row0 * (D / 2), cb, &bar[stage]);
-    bulk_g2s(st + A::CB, P.vp + row0 * (D / 2), cb, &bar[stage]);
-    bulk_g2s(st + 2 * A::CB, P.ks + row0 * NG, sb, &bar[stage]);
-    bulk_g2s(st + 2 * A::CB + A::SB, P.vs + row0 * NG, sb, &bar[stage]);
+  // The warp's blocks are warp, warp + kAW, ...; each issue copies the next
+  // one into the given stage, the sources advancing by kAW blocks of rows.
+  int next_blk = warp, next_kb = k0 + warp * kBK;
+  const uint8_t* kp_next = P.kp + (row_base + next_kb) * (D / 2);
+  const uint8_t* vp_next = P.vp + (row_base + next_kb) * (D / 2);
+  const uint16_t* ks_next = P.ks + (row_base + next_kb) * NG;
+  const uint16_t* vs_next = P.vs + (row_base + next_kb) * NG;
+  auto issue = [&](int stage) {
+    if (next_blk < nblk && lane == 0) {
+      const int nk = min(kBK, k1 - next_kb);
+      const int nk16 = (nk + 15) & ~15;                          // stays inside T (T % 16 == 0)
+      uint8_t* st = ring + (warp * ST + stage) * A::STAGE;
+      const uint32_t cb = static_cast<uint32_t>(nk16 * (D / 2));
+      const uint32_t sb = static_cast<uint32_t>(nk16 * NG * 2);
+      mbar_expect_tx(&bar[stage], 2 * cb + 2 * sb);
+      bulk_g2s(st, kp_next, cb, &bar[stage]);
+      bulk_g2s(st + A::CB, vp_next, cb, &bar[stage]);
+      bulk_g2s(st + 2 * A::CB, ks_next, sb, &bar[stage]);
+      bulk_g2s(st + 2 * A::CB + A::SB, vs_next, sb, &bar[stage]);
+    }
+    next_blk += kAW;
+    next_kb += kAW * kBK;
+    kp_next += kAW * kBK * (D / 2);
+    vp_next += kAW * kBK * (D / 2);
+    ks_next += kAW * kBK * NG;
+    vs_next += kAW * kBK * NG;
   };
   __syncwarp();
-  for (int s = 0; s < ST; ++s) issue(warp + s * kAW, s);
+  for (int s = 0; s < ST; ++s) issue(s);
 
   // The rotated query, fp32: q~ = R (s_K . (q / lambda_K)) with lambda before
   // the rotation, q~ = R (s_K . q) / lambda_K with lambda after it (so that
@@ -513,9 +525,10 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   const float scale = P.scale_log2;
   bool failed = false;
   int k = 0;
+  int stage = 0;
+  uint32_t phase = 0;                  // parity of the stage's current fill
   for (int blk = warp; blk < nblk; blk += kAW, ++k) {
-    const int stage = k % ST;
-    const bool ok = mbar_wait(&bar[stage], (k / ST) & 1, kSpin);
+    const bool ok = mbar_wait(&bar[stage], phase, kSpin);
     if (__any_sync(kFull, !ok)) {
       failed = true;
       break;
@@ -733,7 +746,8 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
       }
     }
     __syncwarp();                      // the stage and the probability rows are consumed
-    issue(blk + ST * kAW, stage);
+    issue(stage);
+    if (++stage == ST) { stage = 0; phase ^= 1u; }
   }
   bool lost = false;                   // a copy may still land in this warp's ring
   if (failed) {
