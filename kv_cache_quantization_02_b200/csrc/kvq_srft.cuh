@@ -144,7 +144,14 @@ __device__ __forceinline__ int sr_code_off(int t, int k) {
 template <int D>
 __host__ __device__ constexpr int sr_hdr_bars(int nw) { return nw * 4 * D + (2 * D + 15) / 16 * 16; }
 template <int D>
-__host__ __device__ constexpr int sr_hdr_bytes(int nw) { return sr_hdr_bars<D>(nw) + 24 * nw + 16; }
+__host__ __device__ constexpr int sr_hdr_bytes(int nw) {
+  return sr_hdr_bars<D>(nw) + 24 * nw + 16 + (D / 2 + 1) * 8;   // ... then the omega_D table
+}
+// Offset of the block's copy of omega_D^k, k <= D/2, in the header: the
+// two-lane unpacking (D = 256) picks its twiddles by the lane's parity, at
+// run time, which shared memory serves in one load.
+template <int D>
+__host__ __device__ constexpr int sr_hdr_wd(int nw) { return sr_hdr_bars<D>(nw) + 24 * nw + 16; }
 
 // The warp's per-channel table for one lambda table, D floats in channel
 // order.  mode 0: lambda s (forward, lambda before); 1: fp32(lambda c_i), with
@@ -306,9 +313,11 @@ kvq_quantize_srft_kernel(const __grid_constant__ SrMaps maps, const ExArgs a,
   uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + sr_hdr_bars<D>(kDW)) + 2 * warp;
   int* tq = reinterpret_cast<int*>(hdr + sr_hdr_bars<D>(kDW) + 16 * kDW) + 2 * warp;
   unsigned int* next = reinterpret_cast<unsigned int*>(hdr + sr_hdr_bars<D>(kDW) + 24 * kDW);
+  float2* wds = reinterpret_cast<float2*>(hdr + sr_hdr_wd<D>(kDW));
   if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   if (tid == 0) *next = 0;
   sr_build_masks<D>(const_cast<uint32_t*>(mk), a, tid, blockDim.x);
+  for (int i = tid; i <= D / 2; i += blockDim.x) wds[i] = tw.wd[i];
   __syncthreads();
 
   const int64_t ntiles = (a.n + S::WR - 1) / S::WR;
@@ -429,7 +438,7 @@ kvq_quantize_srft_kernel(const __grid_constant__ SrMaps maps, const ExArgs a,
         });
       });
       fft_fwd_from<64, 64, 128>(z, tw.wn);
-      unpack_fwd256(z, tw.wd, AFTER ? tab : nullptr, c0, c1h, sub);
+      unpack_fwd256(z, wds, AFTER ? tab : nullptr, c0, c1h, sub);
     }
     // group abs-max (across the two lanes at D = 256), S = fp16(a / QMAX), r = 1/S
     float r[NG];
@@ -585,9 +594,11 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
   uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + sr_hdr_bars<D>(kDW)) + 2 * warp;
   int* tq = reinterpret_cast<int*>(hdr + sr_hdr_bars<D>(kDW) + 16 * kDW) + 2 * warp;
   unsigned int* next = reinterpret_cast<unsigned int*>(hdr + sr_hdr_bars<D>(kDW) + 24 * kDW);
+  float2* wds = reinterpret_cast<float2*>(hdr + sr_hdr_wd<D>(kDW));
   if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   if (tid == 0) *next = 0;
   sr_build_masks<D>(const_cast<uint32_t*>(mk), a, tid, blockDim.x);
+  for (int i = tid; i <= D / 2; i += blockDim.x) wds[i] = tw.wd[i];
   __syncthreads();
 
   const int64_t ntiles = (a.n + S::WR - 1) / S::WR;
@@ -699,7 +710,7 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
         *reinterpret_cast<uint4*>(stage_out + sr_off<D>(rin, c)) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
       }
     } else {
-      unpack_inv256(z, tw.wd, AFTER ? tab : nullptr, c0, c1h, sub);
+      unpack_inv256(z, wds, AFTER ? tab : nullptr, c0, c1h, sub);
       fft_inv_from<64, 64, 128>(z, tw.wn);
       // the transpose of the first stage: c_p = Y_2p+1 conj(omega_128^p) (lane
       // 1's bins), z_p = Y_2p + c_p, z_(p+64) = Y_2p - c_p; lane 0 forms
