@@ -576,9 +576,11 @@ template <int D, int G, int BITS, bool AFTER>
 __global__ void __launch_bounds__(sr_warps<D, true>() * 32, 1)
 kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __restrict__ scales,
                            const ExArgs a, const __grid_constant__ SrTw<D> tw, float c0, float c1h,
-                           const __grid_constant__ SrMaps omaps, int scale_copy) {
+                           const __grid_constant__ SrMaps omaps, int scale_copy,
+                           const __grid_constant__ CUtensorMap cmap) {
   using S = Sr<D>;
   using L = SrDeq<D, G, BITS>;
+  using F = SrFmt<D, BITS>;
   constexpr int kDW = sr_warps<D, true>();
   constexpr int NG = D / G;
   constexpr int GL = G / 2 / S::LANES;  // pairs of a group a lane holds
@@ -623,9 +625,17 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
     if (t < 0 || lane != 0) return;
     const int64_t row0 = static_cast<int64_t>(t) * S::WR;
     const uint32_t sb = scale_bytes(t);
-    const uint32_t cbytes = static_cast<uint32_t>(a.n - row0 < S::WR ? a.n - row0 : S::WR) * CB;
-    mbar_expect_tx(&bar[stage], cbytes + sb);
-    bulk_g2s(stage_out + S::TILE + stage * L::WCA, codes + row0 * CB, cbytes, &bar[stage]);
+    if constexpr (F::SWZ != 0) {
+      // 64- or 128-byte code rows: one tensor copy of the whole tile, swizzled
+      // over the row so that the lanes' 16-byte reads of consecutive rows
+      // fall in distinct banks (rows past n read as zeros)
+      mbar_expect_tx(&bar[stage], static_cast<uint32_t>(S::WR * CB) + sb);
+      tensor_g2s(stage_out + S::TILE + stage * L::WCA, &cmap, 0, static_cast<int>(row0), &bar[stage]);
+    } else {
+      const uint32_t cbytes = static_cast<uint32_t>(a.n - row0 < S::WR ? a.n - row0 : S::WR) * CB;
+      mbar_expect_tx(&bar[stage], cbytes + sb);
+      bulk_g2s(stage_out + S::TILE + stage * L::WCA, codes + row0 * CB, cbytes, &bar[stage]);
+    }
     if (sb) bulk_g2s(stage_out + L::SC + stage * L::WS, reinterpret_cast<const uint8_t*>(scales) + row0 * L::SPR, sb, &bar[stage]);
   };
   refill(0);
@@ -654,7 +664,7 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
       cached = id;
       __syncwarp();
     }
-    const uint8_t* cst = stage_out + S::TILE + stage * L::WCA + rin * CB;   // this row's codes
+    const uint8_t* cst = stage_out + S::TILE + stage * L::WCA;   // the tile's codes (row rin)
     const uint16_t* srow = sc_smem ? reinterpret_cast<const uint16_t*>(stage_out + L::SC + stage * L::WS + rin * L::SPR)
                                    : scales + rrow * NG;
     uint16_t sv[NG];
@@ -665,7 +675,7 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
       constexpr int PW = BITS == 4 ? 4 : 2;            // pairs per code word
 #pragma unroll
       for (int c = 0; c < CB / 16; ++c) {
-        const uint4 cv = *reinterpret_cast<const uint4*>(cst + 16 * c);
+        const uint4 cv = *reinterpret_cast<const uint4*>(cst + sr_code_off<CB, F::SWZ>(rin, c));
         const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
         for (int t = 0; t < 4; ++t) sr_decode_word<BITS>(cw[t], &z[(4 * c + t) * PW], sv, (4 * c + t) * PW, GL);
@@ -676,7 +686,7 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
       const uint32_t sel = BITS == 4 ? (sub ? 0x7531u : 0x6420u) : (sub ? 0x7632u : 0x5410u);
 #pragma unroll
       for (int c = 0; c < CB / 16; ++c) {
-        const uint4 cv = *reinterpret_cast<const uint4*>(cst + 16 * c);
+        const uint4 cv = *reinterpret_cast<const uint4*>(cst + sr_code_off<CB, F::SWZ>(rin, c));
         const uint32_t w0 = __byte_perm(cv.x, cv.y, sel), w1 = __byte_perm(cv.z, cv.w, sel);
         sr_decode_word<BITS>(w0, &z[(2 * c) * PW], sv, (2 * c) * PW, GL);
         sr_decode_word<BITS>(w1, &z[(2 * c + 1) * PW], sv, (2 * c + 1) * PW, GL);
@@ -894,8 +904,14 @@ int launch_sd(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, uin
   using S = Sr<D>;
   using L = SrDeq<D, G, BITS>;
   SrMaps omaps;
-  const int rc = sr_encode_x_maps<D>(omaps, out, a.n);
+  int rc = sr_encode_x_maps<D>(omaps, out, a.n);
   if (rc != KVQ_OK) return rc;
+  CUtensorMap cmap;
+  memset(&cmap, 0, sizeof(cmap));
+  if (SrFmt<D, BITS>::SWZ != 0) {
+    rc = sr_encode_code_map<D, BITS>(cmap, codes, a.n);
+    if (rc != KVQ_OK) return rc;
+  }
   auto k = kvq_dequantize_srft_kernel<D, G, BITS, AFTER>;
   constexpr int nw = sr_warps<D, true>();
   constexpr int smem = 1024 + nw * L::WARP + sr_hdr_bytes<D>(nw);
@@ -904,7 +920,7 @@ int launch_sd(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, uin
   const int grid = sr_grid(k, (a.n + S::WR - 1) / S::WR, smem, nw * 32, ready);
   (void)cudaGetLastError();
   k<<<grid, nw * 32, smem, st>>>(codes, scales, a, sr_twiddles<D>(), sr_c0(D), sr_c1h(D), omaps,
-                                  (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
+                                  (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0, cmap);
   return sr_finish();
 }
 
