@@ -418,6 +418,8 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
   constexpr bool STG = !INDEXED;                // codes leave through a staged tensor store
   constexpr int QW = STG ? Stream<D>::QWARP_S : Stream<D>::QWARP;
   extern __shared__ uint8_t smem_raw[];
+  // a generic pointer here: this kernel measured 5% faster with it than with
+  // the shared-space one of align_smem_1k (the other codec kernels the reverse)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -561,7 +563,7 @@ kvq_dequantize_kernel(const __grid_constant__ CUtensorMap cmap, const uint16_t* 
   constexpr int NGH = Grp<D, G>::NGH;
   constexpr int HG = Grp<D, G>::HG;               // butterfly stages h < HG stay inside a group
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   using L = Stream<D>;

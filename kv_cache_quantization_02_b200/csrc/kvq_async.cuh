@@ -29,6 +29,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
   return false;
 }
+// The first 1 KiB-aligned byte of a dynamic shared-memory array, as an
+// offset from the array itself, so that the pointer stays in the shared
+// address space (shared loads and stores, not generic ones); the caller
+// allocates 1 KiB of slack.
+__device__ __forceinline__ uint8_t* align_smem_1k(uint8_t* base) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(base));
+  return base + ((1024u - (a & 1023u)) & 1023u);
+}
+
 // global -> shared bulk copy completing on an mbarrier (no multicast)
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"

@@ -303,7 +303,7 @@ kvq_quantize_srft_kernel(const __grid_constant__ SrMaps maps, const ExArgs a,
   constexpr int GL = G / 2 / S::LANES;  // pairs of a group a lane holds
   constexpr int NLW = F::CB / 4 / S::LANES;   // code words a lane forms
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sub = S::LANES == 1 ? 0 : lane / S::WR, rin = S::LANES == 1 ? lane : lane % S::WR;
   uint8_t* wsm = smem + warp * 2 * S::TILE;
@@ -586,7 +586,7 @@ kvq_dequantize_srft_kernel(const uint8_t* __restrict__ codes, const uint16_t* __
   constexpr int GL = G / 2 / S::LANES;  // pairs of a group a lane holds
   constexpr int CB = L::CB;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int sub = S::LANES == 1 ? 0 : lane / S::WR, rin = S::LANES == 1 ? lane : lane % S::WR;
   uint8_t* stage_out = smem + warp * L::WARP;
