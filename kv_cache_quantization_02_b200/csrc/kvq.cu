@@ -419,7 +419,8 @@ kvq_quantize_kernel(const __grid_constant__ RowMaps maps, const float* __restric
   constexpr int QW = STG ? Stream<D>::QWARP_S : Stream<D>::QWARP;
   extern __shared__ uint8_t smem_raw[];
   // a generic pointer here: this kernel measured 5% faster with it than with
-  // the shared-space one of align_smem_1k (the other codec kernels the reverse)
+  // the shared-space one of align_smem_1k (the dequantizer, the variant
+  // quantizer and the SRFT kernels measured the reverse)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -916,7 +917,7 @@ kvq_roundtrip_kernel(const __grid_constant__ RowMaps in_maps, const __grid_const
   constexpr int EPT = T::EPT, LANES = T::LANES, NP = T::NP, HALF = T::HALF;
   constexpr int NGH = Grp<D, G>::NGH, HG = Grp<D, G>::HG;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   uint8_t* hdr = smem + kRtWarps * L::WARP;

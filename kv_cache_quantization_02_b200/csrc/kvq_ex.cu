@@ -125,7 +125,7 @@ kvq_quantize_ex_kernel(const __grid_constant__ ExMaps maps, const ExArgs a,
   using F = Fmt<BITS>;
   constexpr int NGH = kNP / G;          // groups per half of the lane's channels
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1k(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* wsm = smem + warp * 2 * kXStage;
   uint8_t* hdr = smem + kQW * 2 * kXStage;
