@@ -331,7 +331,7 @@ __device__ __forceinline__ uint4 code_chunk(const uint8_t* tile, int lane, int c
 
 template <int G, int BITS, bool AFTER>
 __global__ void __launch_bounds__(kDW * 32, 1)
-kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constant__ CUtensorMap cmap,
+kvq_dequantize_ex_kernel(const __grid_constant__ CUtensorMap cmap,
                          const uint16_t* __restrict__ scales,
                          const ExArgs a, const __grid_constant__ ExMaps omaps, int scale_copy) {
   using F = Fmt<BITS>;
@@ -377,14 +377,10 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
     if (t < 0 || lane != 0) return;
     const int64_t row0 = static_cast<int64_t>(t) * kWR;
     const uint32_t sb = scale_bytes(t);
-    if constexpr (BITS == 8) {         // swizzled tensor copy: the copy engine fills the whole box
-      mbar_expect_tx(&bar[stage], static_cast<uint32_t>(L::WC) + sb);
-      tensor_g2s(wsm + stage * L::WC, &cmap, 0, static_cast<int>(row0), &bar[stage]);
-    } else {                           // plain bulk copy of the valid rows
-      const uint32_t cbytes = static_cast<uint32_t>(a.n - row0 < kWR ? a.n - row0 : kWR) * F::CB;
-      mbar_expect_tx(&bar[stage], cbytes + sb);
-      bulk_g2s(wsm + stage * L::WC, codes + row0 * F::CB, cbytes, &bar[stage]);
-    }
+    // swizzled tensor copy of the code rows: the copy engine fills the whole
+    // box (zeros past the last row)
+    mbar_expect_tx(&bar[stage], static_cast<uint32_t>(L::WC) + sb);
+    tensor_g2s(wsm + stage * L::WC, &cmap, 0, static_cast<int>(row0), &bar[stage]);
     if (sb) bulk_g2s(wsm + L::SC + stage * L::WS, reinterpret_cast<const uint8_t*>(scales) + row0 * L::SPR, sb, &bar[stage]);
   };
   refill(0);
@@ -422,18 +418,19 @@ kvq_dequantize_ex_kernel(const uint8_t* __restrict__ codes, const __grid_constan
       sx[j] = srow[j];
       sy[j] = srow[NGH + j];
     }
-    // codes of the pair (m, m+64) as exact fp16 integers.  int4: the row is
-    // linear (64 bytes); int8: word w of the row is word w % 4 of swizzled
-    // chunk w / 4.
+    // codes of the pair (m, m+64) as exact fp16 integers.  Word w of a row is
+    // word w % 4 of its swizzled 16-byte chunk w / 4.
     __half2 hq[kNP];
     if constexpr (BITS == 4) {
-      const uint2* seg = reinterpret_cast<const uint2*>(st + lane * F::CB);
+      const uint4 c0 = code_chunk<F::CB>(st, lane, 0), c1 = code_chunk<F::CB>(st, lane, 1);
+      const uint4 c2 = code_chunk<F::CB>(st, lane, 2), c3 = code_chunk<F::CB>(st, lane, 3);
+      const uint32_t ra[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+      const uint32_t rb[8] = {c2.x, c2.y, c2.z, c2.w, c3.x, c3.y, c3.z, c3.w};
       const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
 #pragma unroll
       for (int kw = 0; kw < kNP / 8; ++kw) {
-        const uint2 da = seg[kw / 2], db = seg[(kw + kNP / 8) / 2];
-        const uint32_t wa = ((kw & 1) ? da.y : da.x) ^ 0x88888888u;
-        const uint32_t wb = ((kw & 1) ? db.y : db.x) ^ 0x88888888u;
+        const uint32_t wa = ra[kw] ^ 0x88888888u;
+        const uint32_t wb = rb[kw] ^ 0x88888888u;
         const uint32_t wa4 = wa >> 4, wb4 = wb >> 4;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -613,13 +610,10 @@ int launch_dex(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, ui
   static std::atomic<int> ready[64];
   const int grid = ex_grid(k, a.n, smem, kDW * 32, ready);
   CUtensorMap cmap;
-  memset(&cmap, 0, sizeof(cmap));
-  if (BITS == 8) {
-    const int rc2 = encode_code_map(cmap, codes, a.n, Fmt<BITS>::CB);
-    if (rc2 != KVQ_OK) return rc2;
-  }
+  const int rc2 = encode_code_map(cmap, codes, a.n, Fmt<BITS>::CB);
+  if (rc2 != KVQ_OK) return rc2;
   (void)cudaGetLastError();
-  k<<<grid, kDW * 32, smem, st>>>(codes, cmap, scales, a, omaps,
+  k<<<grid, kDW * 32, smem, st>>>(cmap, scales, a, omaps,
                                   (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
   return finish_ex();
 }
