@@ -55,7 +55,6 @@ constexpr unsigned kFullMask = 0xffffffffu;
 constexpr int kD = 128;                 // channels (one lane per vector)
 constexpr int kNP = kD / 2;             // packed pairs (v[m], v[m+64])
 constexpr int kQW = 12;                 // warps of a WHT quantize block (one per SM, 170 registers)
-constexpr int kDW = 8;                  // warps of a dequantize or SRFT block (one per SM, 255 registers)
 constexpr int kWR = 32;                 // vectors per warp tile
 constexpr int kQB = kWR * 128;          // bytes of one 64-channel quarter of a tile
 constexpr int kXStage = 2 * kQB;        // bytes of one fp16 warp tile
@@ -319,6 +318,12 @@ struct DeqLayout {
   static constexpr int WARP = (kXStage + 2 * WC + 2 * WS + 1023) / 1024 * 1024;
 };
 
+// Warps of a dequantize block (one block per SM): 12 with lambda after the
+// rotation (every stage in fp32 from the codes, at most 168 registers), 8
+// with lambda before (the fp16 in-group stages hold the codes' halves beside
+// the fp32 row: up to 255 registers).
+__host__ __device__ constexpr int deq_warps(bool after) { return after ? 12 : 8; }
+
 // 16-byte chunk c of lane `lane`'s row of a code tile written by a tensor copy
 // swizzled over the row's CB bytes (64 or 128): chunk c of row t sits at
 // chunk c ^ ((t * CB / 128) mod CB/16), so the eight rows a quarter-warp
@@ -330,24 +335,25 @@ __device__ __forceinline__ uint4 code_chunk(const uint8_t* tile, int lane, int c
 }
 
 template <int G, int BITS, bool AFTER>
-__global__ void __launch_bounds__(kDW * 32, 1)
+__global__ void __launch_bounds__(deq_warps(AFTER) * 32, 1)
 kvq_dequantize_ex_kernel(const __grid_constant__ CUtensorMap cmap,
                          const uint16_t* __restrict__ scales,
                          const ExArgs a, const __grid_constant__ ExMaps omaps, int scale_copy) {
   using F = Fmt<BITS>;
   using L = DeqLayout<G, BITS>;
+  constexpr int NW = deq_warps(AFTER);
   constexpr int NGH = kNP / G;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* stage_out = smem + warp * L::WARP;              // swizzled fp16 staging tile
   uint8_t* wsm = stage_out + kXStage;                      // two code tiles, then two scale blocks
-  uint8_t* hdr = smem + kDW * L::WARP;
+  uint8_t* hdr = smem + NW * L::WARP;
   float4* tab = reinterpret_cast<float4*>(hdr) + warp * 32;
-  float4* stab = reinterpret_cast<float4*>(hdr + kDW * 512);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + hdr_bars(kDW)) + 2 * warp;
-  int* tq = reinterpret_cast<int*>(hdr + hdr_bars(kDW) + 16 * kDW) + 2 * warp;
-  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + hdr_bars(kDW) + 24 * kDW);
+  float4* stab = reinterpret_cast<float4*>(hdr + NW * 512);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(hdr + hdr_bars(NW)) + 2 * warp;
+  int* tq = reinterpret_cast<int*>(hdr + hdr_bars(NW) + 16 * NW) + 2 * warp;
+  unsigned int* next = reinterpret_cast<unsigned int*>(hdr + hdr_bars(NW) + 24 * NW);
   if (lane == 0) { mbar_init(&bar[0], 1); mbar_init(&bar[1], 1); mbar_fence_init(); }
   if (tid == 0) *next = 0;
   if (tid < 32) build_signs(stab, a, tid);
@@ -419,18 +425,30 @@ kvq_dequantize_ex_kernel(const __grid_constant__ CUtensorMap cmap,
       sy[j] = srow[NGH + j];
     }
     // codes of the pair (m, m+64) as exact fp16 integers.  Word w of a row is
-    // word w % 4 of its swizzled 16-byte chunk w / 4.
+    // word w % 4 of its swizzled 16-byte chunk w / 4.  With lambda after the
+    // rotation each pair goes straight on to u = q S (exact) and u fp32(c /
+    // lambda), so that only the fp32 row stays live.
     __half2 hq[kNP];
+    float2 p[kNP];
+    auto to_row = [&](int m) {
+      p[m] = make_float2(mul_f16_f32(__low2half(hq[m]), sx[m / G]), mul_f16_f32(__high2half(hq[m]), sy[m / G]));
+      if constexpr (AFTER) {
+        const float4 l = tab[m / 2];                  // fp32(c / lambda) of the pairs 2q, 2q + 1
+        p[m] = __fmul2_rn(p[m], (m & 1) ? make_float2(l.z, l.w) : make_float2(l.x, l.y));
+      }
+    };
     if constexpr (BITS == 4) {
-      const uint4 c0 = code_chunk<F::CB>(st, lane, 0), c1 = code_chunk<F::CB>(st, lane, 1);
-      const uint4 c2 = code_chunk<F::CB>(st, lane, 2), c3 = code_chunk<F::CB>(st, lane, 3);
-      const uint32_t ra[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-      const uint32_t rb[8] = {c2.x, c2.y, c2.z, c2.w, c3.x, c3.y, c3.z, c3.w};
       const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
+      uint32_t ra[4], rb[4];
 #pragma unroll
       for (int kw = 0; kw < kNP / 8; ++kw) {
-        const uint32_t wa = ra[kw] ^ 0x88888888u;
-        const uint32_t wb = rb[kw] ^ 0x88888888u;
+        if (kw % 4 == 0) {              // channels 8 kw .. 8 kw + 31 and 64 + the same
+          const uint4 ca = code_chunk<F::CB>(st, lane, kw / 4), cb = code_chunk<F::CB>(st, lane, 2 + kw / 4);
+          ra[0] = ca.x; ra[1] = ca.y; ra[2] = ca.z; ra[3] = ca.w;
+          rb[0] = cb.x; rb[1] = cb.y; rb[2] = cb.z; rb[3] = cb.w;
+        }
+        const uint32_t wa = ra[kw % 4] ^ 0x88888888u;
+        const uint32_t wb = rb[kw % 4] ^ 0x88888888u;
         const uint32_t wa4 = wa >> 4, wb4 = wb >> 4;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -439,6 +457,10 @@ kvq_dequantize_ex_kernel(const __grid_constant__ CUtensorMap cmap,
           const uint32_t e1 = (__byte_perm(wa4, wb4, sel) & 0x000F000Fu) | 0x64006400u;
           hq[8 * kw + 2 * t] = __hsub2(*reinterpret_cast<const __half2*>(&e0), bias);
           hq[8 * kw + 2 * t + 1] = __hsub2(*reinterpret_cast<const __half2*>(&e1), bias);
+          if constexpr (AFTER) {
+            to_row(8 * kw + 2 * t);
+            to_row(8 * kw + 2 * t + 1);
+          }
         }
       }
     } else {
@@ -455,6 +477,7 @@ kvq_dequantize_ex_kernel(const __grid_constant__ CUtensorMap cmap,
           const uint32_t sel = 0x0400u | (t << 8) | t;
           const uint32_t e = (__byte_perm(wa, wb, sel) & 0x00FF00FFu) | 0x64006400u;
           hq[4 * kw + t] = __hsub2(*reinterpret_cast<const __half2*>(&e), bias);
+          if constexpr (AFTER) to_row(4 * kw + t);
         }
       }
     }
@@ -477,20 +500,12 @@ kvq_dequantize_ex_kernel(const __grid_constant__ CUtensorMap cmap,
         }
       }
     }
-    float2 p[kNP];
+    if constexpr (!AFTER) {
 #pragma unroll
-    for (int m = 0; m < kNP; ++m)
-      p[m] = make_float2(mul_f16_f32(__low2half(hq[m]), sx[m / G]), mul_f16_f32(__high2half(hq[m]), sy[m / G]));
+      for (int m = 0; m < kNP; ++m) to_row(m);
+    }
     __syncwarp();                       // codes and scales consumed: refill the stage
     refill(stage);
-    if constexpr (AFTER) {
-#pragma unroll
-      for (int q = 0; q < kNP / 2; ++q) {
-        const float4 l = tab[q];                      // fp32(c / lambda)
-        p[2 * q] = __fmul2_rn(p[2 * q], make_float2(l.x, l.y));
-        p[2 * q + 1] = __fmul2_rn(p[2 * q + 1], make_float2(l.z, l.w));
-      }
-    }
     fwht_pairs<kD, 1, HF>(p, 0);
     if (lane == 0) bulk_wait_read0();   // the previous tile's stores have read the staging tile
     __syncwarp();
@@ -606,14 +621,15 @@ int launch_dex(const uint8_t* codes, const uint16_t* scales, const ExArgs& a, ui
   const int rc = encode_x_maps(omaps, out, a.n);
   if (rc != KVQ_OK) return rc;
   auto k = kvq_dequantize_ex_kernel<G, BITS, AFTER>;
-  constexpr int smem = 1024 + kDW * L::WARP + hdr_bytes(kDW);
+  constexpr int NW = deq_warps(AFTER);
+  constexpr int smem = 1024 + NW * L::WARP + hdr_bytes(NW);
   static std::atomic<int> ready[64];
-  const int grid = ex_grid(k, a.n, smem, kDW * 32, ready);
+  const int grid = ex_grid(k, a.n, smem, NW * 32, ready);
   CUtensorMap cmap;
   const int rc2 = encode_code_map(cmap, codes, a.n, Fmt<BITS>::CB);
   if (rc2 != KVQ_OK) return rc2;
   (void)cudaGetLastError();
-  k<<<grid, kDW * 32, smem, st>>>(cmap, scales, a, omaps,
+  k<<<grid, NW * 32, smem, st>>>(cmap, scales, a, omaps,
                                   (reinterpret_cast<uintptr_t>(scales) & 15) == 0 ? 1 : 0);
   return finish_ex();
 }
