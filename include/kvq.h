@@ -274,10 +274,10 @@ int kvq_attention_decode(const uint16_t *q, const uint8_t *k_packed,
  * once to match and the rotated-domain output rotated back once per head.
  * One lambda table per K and per V (lambda_rows = all rows).  Other flag bits
  * -> KVQ_ERR_GROUP; other arguments, checks and results as for
- * kvq_attention_decode, which is this call with flags = 0.  The first call
- * with KVQ_SRFT at a head dimension on a device copies that dimension's
- * twiddle table into the library's constant memory (synchronously): make it
- * outside any stream capture.
+ * kvq_attention_decode, which is this call with flags = 0.  The SRFT
+ * rotations run inside the kernels (a warp-wide real FFT per row, roots
+ * computed on the device): no call copies tables from the host, so every
+ * call may sit inside a stream capture.
  */
 int kvq_attention_decode_ex(const uint16_t *q, const uint8_t *k_packed,
                             const uint16_t *k_scales, const uint8_t *v_packed,

@@ -58,7 +58,6 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
-#include <vector>
 
 #include "kvq.h"
 #include "kvq_attn_common.cuh"
@@ -80,43 +79,159 @@ constexpr uint32_t kSpin = 1u << 22;         // bounded mbarrier waits
 
 __device__ unsigned int g_attn_fault = 0;    // bit 0: a wait gave up; bit 3: bad sequence length
 
-// The SRFT at this head dimension as a real D x D matrix, fp32, written once
-// per device by the first launch that needs it: g_srft[j][i] = M[j][i] with
-// y = M x (y_0 = X_0 / sqrt(D), y_1 = X_(D/2) / sqrt(D), (y_2k, y_2k+1) =
-// sqrt(2) (Re, Im) X_k / sqrt(D), X the length-D DFT of x), and g_srft_t its
-// transpose.  The query's and the output's rotations are one warp-wide
-// product each per head (every lane DPL outputs, coalesced rows); no FFT
-// sits on one lane, where its working set spilled to local memory.
-__device__ float g_srft[KVQ_ATTN_D * KVQ_ATTN_D];
-__device__ float g_srft_t[KVQ_ATTN_D * KVQ_ATTN_D];
+// ---- the SRFT of one row across a warp ---------------------------------------
+// y = M x: y_0 = X_0 / sqrt(D), y_1 = X_(D/2) / sqrt(D), (y_2k, y_2k+1) =
+// sqrt(2) (Re, Im) X_k / sqrt(D), X the length-D DFT of x with the root
+// omega_D = exp(-2 pi i / D) ("When Quantization Is Free", technical summary,
+// Methodologie 1).  M is orthogonal.  The real DFT runs as a complex one of
+// length N = D/2 on z_n = x_2n + i x_2n+1, lane L holding z_(ZPL L + j) (j <
+// ZPL = N / 32), in four steps (n = j + ZPL L, k = k1 + 32 k2): 32-point
+// butterflies across the lanes for each j (decimation in frequency, so lane
+// L ends with k1 = bitrev5(L)), a twiddle omega_N^(j k1), ZPL-point DFTs in
+// the lane over j; then the Hermitian unpacking, 2 X_k = (Z_k + conj Z_(N-k))
+// - i omega_D^k (Z_k - conj Z_(N-k)).  The adjoint runs the same steps
+// backwards with conjugate roots.  tw holds omega_D^e, e in [0, D/2].
 
-// out[DPL lane + k] = sum_i mat[i][DPL lane + k] x[i], x in shared memory.
+// omega_D^e, e in [0, D), from the half table: omega_D^(e + D/2) = -omega_D^e.
 template <int D>
-__device__ __forceinline__ void warp_matvec(float (&out)[D / 32], const float* __restrict__ mat,
-                                            const float* x, int lane) {
-  constexpr int DPL = D / 32;
-  constexpr int UNR = 64 / DPL;                  // rows in flight: the loads come from L2
+__device__ __forceinline__ float2 tw_pow(const float2* tw, int e) {
+  if (e <= D / 2) return tw[e];
+  const float2 w = tw[e - D / 2];
+  return make_float2(-w.x, -w.y);
+}
+__device__ __forceinline__ float2 cmul(float2 a, float2 b) {
+  return make_float2(a.x * b.x - a.y * b.y, a.x * b.y + a.y * b.x);
+}
+__device__ __forceinline__ float2 cmul_conj(float2 a, float2 b) {     // a conj(b)
+  return make_float2(a.x * b.x + a.y * b.y, a.y * b.x - a.x * b.y);
+}
+__device__ __forceinline__ float2 shfl_xor2(float2 v, int m) {
+  return make_float2(__shfl_xor_sync(kFull, v.x, m), __shfl_xor_sync(kFull, v.y, m));
+}
+
+// This warp's table of omega_D^e, e in [0, D/2] (shared memory).
+template <int D>
+__device__ __forceinline__ void build_roots(float2* tw, int lane) {
+  for (int e = lane; e <= D / 2; e += 32) {
+    float sn, cs;
+    sincospif(2.0f * static_cast<float>(e) / static_cast<float>(D), &sn, &cs);
+    tw[e] = make_float2(cs, -sn);
+  }
+  __syncwarp();
+}
+
+// In the lane: Z_k2 = sum_j omega_ZPL^(+-j k2) z_j (INV: the + sign).
+template <int ZPL, bool INV>
+__device__ __forceinline__ void lane_dft(float2 (&z)[ZPL]) {
+  if constexpr (ZPL == 2) {
+    const float2 a = z[0], b = z[1];
+    z[0] = make_float2(a.x + b.x, a.y + b.y);
+    z[1] = make_float2(a.x - b.x, a.y - b.y);
+  } else if constexpr (ZPL == 4) {
+    const float2 a = make_float2(z[0].x + z[2].x, z[0].y + z[2].y), b = make_float2(z[0].x - z[2].x, z[0].y - z[2].y);
+    const float2 c = make_float2(z[1].x + z[3].x, z[1].y + z[3].y), d = make_float2(z[1].x - z[3].x, z[1].y - z[3].y);
+    const float2 id = INV ? make_float2(-d.y, d.x) : make_float2(d.y, -d.x);     // (+-i) d
+    z[0] = make_float2(a.x + c.x, a.y + c.y);
+    z[2] = make_float2(a.x - c.x, a.y - c.y);
+    z[1] = make_float2(b.x + id.x, b.y + id.y);
+    z[3] = make_float2(b.x - id.x, b.y - id.y);
+  }
+}
+
+// y = M x for one row in shared memory, written over x; y_i / div[i] when
+// div is not null.
+template <int D>
+__device__ __forceinline__ void warp_srft_fwd(float* row, const float2* tw, const float* div, float c,
+                                              float c1h, int lane) {
+  constexpr int N = D / 2, ZPL = N / 32;
+  float2 z[ZPL];
 #pragma unroll
-  for (int k = 0; k < DPL; ++k) out[k] = 0.0f;
-#pragma unroll UNR
-  for (int i = 0; i < D; ++i) {
-    const float xi = x[i];
-    const float* row = mat + i * D + DPL * lane;
-    if constexpr (DPL % 4 == 0) {
+  for (int j = 0; j < ZPL; ++j) z[j] = *reinterpret_cast<const float2*>(row + 2 * (ZPL * lane + j));
+  __syncwarp();
 #pragma unroll
-      for (int k = 0; k < DPL; k += 4) {
-        const float4 m4 = __ldg(reinterpret_cast<const float4*>(row + k));
-        out[k] = __fmaf_rn(m4.x, xi, out[k]);
-        out[k + 1] = __fmaf_rn(m4.y, xi, out[k + 1]);
-        out[k + 2] = __fmaf_rn(m4.z, xi, out[k + 2]);
-        out[k + 3] = __fmaf_rn(m4.w, xi, out[k + 3]);
-      }
-    } else {
-      const float2 m2 = __ldg(reinterpret_cast<const float2*>(row));
-      out[0] = __fmaf_rn(m2.x, xi, out[0]);
-      out[1] = __fmaf_rn(m2.y, xi, out[1]);
+  for (int h = 16; h >= 1; h >>= 1) {
+    const bool hi = (lane & h) != 0;
+    const float2 w = hi ? tw[(lane & (h - 1)) * (D / (2 * h))] : make_float2(1.0f, 0.0f);
+#pragma unroll
+    for (int j = 0; j < ZPL; ++j) {
+      const float2 u = shfl_xor2(z[j], h);
+      const float2 v = hi ? make_float2(u.x - z[j].x, u.y - z[j].y) : make_float2(z[j].x + u.x, z[j].y + u.y);
+      z[j] = cmul(v, w);
     }
   }
+  const int k1 = static_cast<int>(__brev(static_cast<unsigned>(lane)) >> 27);
+#pragma unroll
+  for (int j = 1; j < ZPL; ++j) z[j] = cmul(z[j], tw_pow<D>(tw, 2 * j * k1));
+  lane_dft<ZPL, false>(z);
+  // z[k2] = Z_(k1 + 32 k2); Z_(N-k) is register ZPL-1-k2 of lane bitrev5(32 - k1)
+  // (k1 > 0), or register (ZPL - k2) mod ZPL of this lane (k1 = 0)
+  const int src = static_cast<int>(__brev(static_cast<unsigned>((32 - k1) & 31)) >> 27);
+  float2 zp[ZPL];
+#pragma unroll
+  for (int k2 = 0; k2 < ZPL; ++k2) {
+    const float2 v = make_float2(__shfl_sync(kFull, z[ZPL - 1 - k2].x, src), __shfl_sync(kFull, z[ZPL - 1 - k2].y, src));
+    zp[k2] = k1 == 0 ? z[(ZPL - k2) % ZPL] : v;
+  }
+#pragma unroll
+  for (int k2 = 0; k2 < ZPL; ++k2) {
+    const int k = k1 + 32 * k2;
+    float y0, y1;
+    if (k == 0) {                                  // X_0 and X_N, both real
+      y0 = c * (z[0].x + z[0].y);
+      y1 = c * (z[0].x - z[0].y);
+    } else {
+      const float2 e = make_float2(z[k2].x + zp[k2].x, z[k2].y - zp[k2].y);    // Z_k + conj Z_(N-k)
+      const float2 f = make_float2(z[k2].x - zp[k2].x, z[k2].y + zp[k2].y);    // Z_k - conj Z_(N-k)
+      const float2 tt = cmul(f, tw[k]);
+      y0 = c1h * (e.x + tt.y);                     // (e - i tt) / sqrt(2 D)
+      y1 = c1h * (e.y - tt.x);
+    }
+    if (div != nullptr) { y0 /= div[2 * k]; y1 /= div[2 * k + 1]; }
+    *reinterpret_cast<float2*>(row + 2 * k) = make_float2(y0, y1);
+  }
+}
+
+// o = M^T y for one row: y read from shared memory, lane L gets o_(DPL L + i)
+// in o[i].  With X_0 = y_0, X_N = y_1, X_k = (y_2k + i y_2k+1) / sqrt 2, o_2m +
+// i o_2m+1 = z_m / sqrt(D), z the inverse length-N DFT of Z_k = (X_k + conj
+// X_(N-k)) + i omega_D^-k (X_k - conj X_(N-k)).
+template <int D>
+__device__ __forceinline__ void warp_srft_adj(float (&o)[D / 32], const float* row, const float2* tw, float c,
+                                              float c1h, int lane) {
+  constexpr int N = D / 2, ZPL = N / 32;
+  const int k1 = static_cast<int>(__brev(static_cast<unsigned>(lane)) >> 27);
+  float2 z[ZPL];
+#pragma unroll
+  for (int k2 = 0; k2 < ZPL; ++k2) {
+    const int k = k1 + 32 * k2;
+    if (k == 0) {
+      const float y0 = row[0], y1 = row[1];
+      z[k2] = make_float2(c * (y0 + y1), c * (y0 - y1));
+    } else {
+      const float2 yk = *reinterpret_cast<const float2*>(row + 2 * k);
+      const float2 yp = *reinterpret_cast<const float2*>(row + 2 * (N - k));
+      const float2 e = make_float2(yk.x + yp.x, yk.y - yp.y);
+      const float2 f = make_float2(yk.x - yp.x, yk.y + yp.y);
+      const float2 tt = cmul_conj(f, tw[k]);
+      z[k2] = make_float2(c1h * (e.x - tt.y), c1h * (e.y + tt.x));     // (e + i tt) / sqrt(2 D)
+    }
+  }
+  lane_dft<ZPL, true>(z);
+#pragma unroll
+  for (int j = 1; j < ZPL; ++j) z[j] = cmul_conj(z[j], tw_pow<D>(tw, 2 * j * k1));
+#pragma unroll
+  for (int h = 1; h <= 16; h <<= 1) {
+    const bool hi = (lane & h) != 0;
+    const float2 w = hi ? tw[(lane & (h - 1)) * (D / (2 * h))] : make_float2(1.0f, 0.0f);
+#pragma unroll
+    for (int j = 0; j < ZPL; ++j) {
+      const float2 tt = cmul_conj(z[j], w);
+      const float2 u = shfl_xor2(tt, h);
+      z[j] = hi ? make_float2(u.x - tt.x, u.y - tt.y) : make_float2(z[j].x + u.x, z[j].y + u.y);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < ZPL; ++j) { o[2 * j] = z[j].x; o[2 * j + 1] = z[j].y; }
 }
 thread_local int g_attn_cuda_error = 0;
 
@@ -259,11 +374,11 @@ __device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
 //   lambda before: out = fp16((s_V . R^T y) / lambda_V),
 //   lambda after:  out = fp16(s_V . R^T (y / lambda_V)),
 // R^T = H / sqrt(D) (a warp-wide butterfly over the lanes' channels) or the
-// SRFT's transpose (a warp-wide product with the SRFT matrix, the row
-// gathered in `scr`, D floats of this warp's shared memory).
+// SRFT's transpose (the warp-wide adjoint above, the row gathered in `scr`,
+// D floats of this warp's shared memory; tw this warp's table of roots).
 template <int D>
 __device__ __forceinline__ void finish_head(const AttnParams& P, float (&v)[D / 32], float l,
-                                            uint16_t* out_row, int lane, float* scr) {
+                                            uint16_t* out_row, int lane, float* scr, const float2* tw) {
   constexpr int DPL = D / 32;
   const bool after = (P.fmt & kFmtAfter) != 0;
   const float inv = l > 0.0f ? 1.0f / l : 0.0f;
@@ -300,7 +415,7 @@ __device__ __forceinline__ void finish_head(const AttnParams& P, float (&v)[D / 
     }
     __syncwarp();
     float o[DPL];
-    warp_matvec<D>(o, g_srft, scr, lane);
+    warp_srft_adj<D>(o, scr, tw, P.c, P.c1h, lane);
     uint16_t h[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) {
@@ -391,6 +506,8 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   // the rotation, q~ = R (s_K . q) / lambda_K with lambda after it (so that
   // <q, x_t> = <q~, y_t>), R = H / sqrt(D) or the SRFT; rows R..7 are zero.
   const bool after = (P.fmt & kFmtAfter) != 0;
+  float2* tw = reinterpret_cast<float2*>(scw);          // the SRFT's roots, in this warp's scale area until the key loop
+  if (P.fmt & kFmtSrft) build_roots<D>(tw, lane);
   for (int r = warp; r < kMaxRows; r += kAW) {
     float* qr_out = qf + r * D;
     if (P.fmt & kFmtSrft) {
@@ -406,14 +523,8 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
           qr_out[d] = P.s_k[d] < 0 ? -x : x;
         }
         __syncwarp();
-        float y[DPL];
-        warp_matvec<D>(y, g_srft_t, qr_out, lane);
+        warp_srft_fwd<D>(qr_out, tw, after ? P.lam_k : nullptr, P.c, P.c1h, lane);
         __syncwarp();
-#pragma unroll
-        for (int i = 0; i < DPL; ++i) {
-          const int d = DPL * lane + i;
-          qr_out[d] = after ? y[i] / P.lam_k[d] : y[i];
-        }
       } else {
 #pragma unroll
         for (int i = 0; i < DPL; ++i) qr_out[DPL * lane + i] = 0.0f;
@@ -803,6 +914,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     }
   }
   __syncthreads();
+  if ((P.fmt & kFmtSrft) && P.nsplit == 1) build_roots<D>(tw, lane);   // the scale area is free again
   for (int r = warp; r < R; r += kAW) {
     float M = -INFINITY;
 #pragma unroll
@@ -820,7 +932,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     }
     if (P.nsplit == 1) {
       uint16_t* orow = P.out + (static_cast<int64_t>(b) * P.Hkv * R + kvh * R + r) * D;
-      finish_head<D>(P, v, lsum, orow, lane, comb + r * D);   // row r's first slot: read above
+      finish_head<D>(P, v, lsum, orow, lane, comb + r * D, tw);   // row r's first slot: read above
     } else {
       float* pr = P.part + (static_cast<int64_t>(item) * R + r) * (D + 4);
       if (lane == 0) { pr[0] = M; pr[1] = lsum; }
@@ -835,10 +947,12 @@ template <int D>
 __global__ void __launch_bounds__(kMaxRows * 32)
 kvq_attn_combine_kernel(const __grid_constant__ AttnParams P) {
   __shared__ float scr[kMaxRows][D];
+  __shared__ float2 tws[kMaxRows][D / 2 + 1];
   constexpr int DPL = D / 32;
   const int bh = blockIdx.x, b = bh / P.Hkv, kvh = bh % P.Hkv;
   const int r = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (r >= P.R) return;
+  if (P.fmt & kFmtSrft) build_roots<D>(tws[r], lane);
   const int64_t stride = static_cast<int64_t>(P.R) * (D + 4);
   const float* base = P.part + (static_cast<int64_t>(bh) * P.nsplit * P.R + r) * (D + 4);
   float M = -INFINITY;
@@ -854,47 +968,13 @@ kvq_attn_combine_kernel(const __grid_constant__ AttnParams P) {
     for (int i = 0; i < DPL; ++i) v[i] += e * pr[4 + DPL * lane + i];
   }
   uint16_t* orow = P.out + (static_cast<int64_t>(b) * P.Hkv * P.R + kvh * P.R + r) * D;
-  finish_head<D>(P, v, lsum, orow, lane, scr[r]);
+  finish_head<D>(P, v, lsum, orow, lane, scr[r], tws[r]);
 }
 
 
 // ---------------------------------------------------------------------------
 // Launch plumbing.
 // ---------------------------------------------------------------------------
-
-// The SRFT matrix and its transpose into this unit's device memory, once per
-// device (synchronous copies: the first SRFT call on a device must not be
-// inside a stream capture).  Entries from the definition, in long double,
-// each rounded once to fp32.
-int upload_srft_matrix() {
-  constexpr int D = KVQ_ATTN_D, N = D / 2;
-  static std::atomic<int> done[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-  if (dev >= 0 && dev < 64 && done[dev].load(std::memory_order_acquire)) return KVQ_OK;
-  std::vector<float> m(D * D), mt(D * D);
-  const long double pi = 3.141592653589793238462643383279502884L;
-  const long double c = 1.0L / sqrtl(static_cast<long double>(D));
-  for (int i = 0; i < D; ++i) {
-    m[0 * D + i] = static_cast<float>(c);
-    m[1 * D + i] = static_cast<float>((i % 2 ? -1.0L : 1.0L) * c);
-    for (int k = 1; k < N; ++k) {
-      const long double ang = 2.0L * pi * static_cast<long double>((static_cast<long>(i) * k) % D) / D;
-      m[(2 * k) * D + i] = static_cast<float>(sqrtl(2.0L) * c * cosl(ang));
-      m[(2 * k + 1) * D + i] = static_cast<float>(-sqrtl(2.0L) * c * sinl(ang));
-    }
-  }
-  for (int j = 0; j < D; ++j)
-    for (int i = 0; i < D; ++i) mt[i * D + j] = m[j * D + i];
-  cudaError_t e = cudaMemcpyToSymbol(g_srft, m.data(), m.size() * sizeof(float));
-  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_srft_t, mt.data(), mt.size() * sizeof(float));
-  if (e != cudaSuccess) {
-    g_attn_cuda_error = static_cast<int>(e);
-    return KVQ_ERR_LAUNCH;
-  }
-  if (dev >= 0 && dev < 64) done[dev].store(1, std::memory_order_release);
-  return KVQ_OK;
-}
 
 template <int D, int G, int NH>
 int launch_attn(const AttnParams& P, int64_t pairs, cudaStream_t st) {
@@ -933,10 +1013,6 @@ int launch_nh(const AttnParams& P, int64_t pairs, cudaStream_t st) {
 __attribute__((visibility("hidden"))) int KVQA_CAT(kvq_attn_launch_, KVQ_ATTN_D)(
     const kvqa::AttnParams& P, int64_t pairs, int group, cudaStream_t st) {
   constexpr int D = KVQ_ATTN_D;
-  if (P.fmt & kFmtSrft) {
-    const int rc = upload_srft_matrix();
-    if (rc != KVQ_OK) return rc;
-  }
   switch (group) {
     case 16: return launch_nh<D, 16>(P, pairs, st);
     case 32: return launch_nh<D, 32>(P, pairs, st);
