@@ -44,11 +44,10 @@ constexpr unsigned kFullMask = 0xffffffffu;
 #include "kvq_ex.cuh"
 #include "kvq_fft.cuh"
 
-// Warps of a block (one block per SM): 12, whose 168 registers a thread the
-// one-lane kernels fit with a few bytes of spill; 8 for the D = 256
-// dequantiser, whose two-lane unpacking keeps more values live.
+// Warps of a block (one block per SM): 12 for every kernel, whose 168
+// registers a thread they fit with at most a few bytes of spill.
 template <int D, bool DEQ>
-__host__ __device__ constexpr int sr_warps() { return (D == 256 && DEQ) ? 8 : 12; }
+__host__ __device__ constexpr int sr_warps() { return 12; }
 constexpr uint32_t kSpinX = 1u << 22;   // bounded mbarrier waits
 
 __device__ unsigned int g_ex_fault = 0;   // bit 0: a bounded wait gave up

@@ -300,3 +300,30 @@ def test_attention_formats_reject_bad_flags():
     args = [t(c[k]).data_ptr() for k in ("q", "kp", "ks", "vp", "vs", "lens", "lk", "sk", "lv", "sv")]
     out = torch.empty((1, 2, 128), dtype=torch.float16, device=dev)
     assert kvq.kvq_attention_decode_ex(*args, 1, 2, 1, 16, 128, 32, 4, 0.1, out.data_ptr()) == kvq.KVQ_ERR_GROUP
+
+
+def test_paper_format_inside_cuda_graph():
+    """The SRFT rotations run inside the kernels (no host-side table), so the
+    paper-format call can be captured in a CUDA graph: its replay gives the
+    eager call's bytes, with and without the key-axis split."""
+    B, Hq, Hkv, T, D, G = 2, 8, 2, 512, 128, 16
+    c = _case_fmt(B, Hq, Hkv, T, D, G, seed=77, after=True, srft=True, lens=[512, 301])
+    dev = torch.device("cuda")
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    args = [t(c[k]) for k in ("q", "kp", "ks", "vp", "vs", "lens", "lk", "sk", "lv", "sv")]
+    need = kvq.kvq_attention_workspace_bytes(B, Hq, Hkv, T, D, G)
+    for ws in (torch.empty(max(need, 16), dtype=torch.uint8, device=dev), False):
+        eager = kvq.attention_decode(*args, G, 0.0883, workspace=ws, lambda_after=True, srft=True)
+        out = torch.empty_like(eager)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(s), torch.cuda.graph(graph, stream=s):
+            kvq.attention_decode(*args, G, 0.0883, out=out, workspace=ws, lambda_after=True,
+                                 srft=True, stream=s)
+        torch.cuda.current_stream().wait_stream(s)
+        out.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+        del graph
