@@ -44,10 +44,11 @@ constexpr unsigned kFullMask = 0xffffffffu;
 #include "kvq_ex.cuh"
 #include "kvq_fft.cuh"
 
-// Warps of a block (one block per SM): 12 for every kernel, whose 168
-// registers a thread they fit with at most a few bytes of spill.
+// Warps of a block (one block per SM): 12, whose 168 registers a thread the
+// kernels fit with at most a few bytes of spill; 16 at D = 64, whose kernels
+// need fewer than 128.
 template <int D, bool DEQ>
-__host__ __device__ constexpr int sr_warps() { return 12; }
+__host__ __device__ constexpr int sr_warps() { return D == 64 ? 16 : 12; }
 constexpr uint32_t kSpinX = 1u << 22;   // bounded mbarrier waits
 
 __device__ unsigned int g_ex_fault = 0;   // bit 0: a bounded wait gave up
