@@ -40,9 +40,12 @@
 //     of lane (g, t) are head t again, so the softmax rescale needs no
 //     exchange.
 // A biased code n = q + 8 in [0, 15] is the fp16 subnormal n 2^-24, exact,
-// made by one mask-and-xor.  The key side starts its accumulators at
-// -8 2^-24 times the query's group sums; the value side keeps the running sum
-// of p S_V per group and subtracts 8 times it once at the end.
+// made by one mask-and-xor.  The key side adds -8 2^-24 times the query's
+// group sums to each group's partial score before its scale multiplies it;
+// the value side keeps the running sum of p S_V per group and subtracts 8
+// times it once at the end.  The rotations of the query and of the output
+// are one warp's work per head: the fast Walsh-Hadamard transform across the
+// lanes, or the SRFT as a warp-wide real FFT.
 //
 // Every mbarrier wait is bounded; a warp that gives up sets the fault word
 // and the block writes nothing.  A sequence length outside [0, T] is clamped

@@ -20,11 +20,11 @@
 // D = 128; G in {16, 32, 64}.  One lane holds a whole vector as 64 packed
 // fp32 pairs; each warp streams 32-vector tiles through its own
 // double-buffered ring, and the warps of a block (one per SM: 12 warps for the
-// WHT quantisers, 8 for the rest) claim tiles of a contiguous range from a
-// shared counter.  fp16 rows move by swizzled tensor copies; the codes leave
-// the quantisers through the stage their tile came from and one tensor store,
-// and enter the dequantisers by a swizzled tensor copy (int8) or a bulk copy
-// (int4); scales move by bulk copies.  A warp tile lies inside one lambda
+// quantisers and the lambda-after dequantisers, 8 for the lambda-before ones)
+// claim tiles of a contiguous range from a shared counter.  fp16 rows move by
+// swizzled tensor copies; the codes leave the quantisers through the stage
+// their tile came from and one tensor store, and enter the dequantisers by a
+// swizzled tensor copy; scales move by bulk copies.  A warp tile lies inside one lambda
 // table (lambda_rows is a multiple of 32 when there are several), so the warp
 // rebuilds its per-channel table in shared memory when a tile's table differs
 // from the last one's.  Every step is the oracle's IEEE operation in the
