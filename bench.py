@@ -446,7 +446,6 @@ def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, attn_seqs=64):
         "decode_append_us": round(ap_ms * 1e3, 2),
         "decode_append_gvec_s": round(na / (ap_ms / 1e3) / 1e9, 3),
     }
-    res["sustained"] = run_sustained(torch, kvq, dev, stream, x, out, lam_t, s_t, G)
     if D == 128:
         res["codec_variants"] = run_variants(torch, kvq, dev, stream, x, out, s_t, G, w)
         res["dequantize_tensor_cores"] = run_dequant_tc(torch, kvq, dev, stream, x, out, lam_t, s_t)
@@ -460,6 +459,8 @@ def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, attn_seqs=64):
         res["attention_decode_paper_format"] = run_attention_paper_format(torch, kvq, dev, stream, attn_seqs)
         res["configs"] = run_configs(torch, kvq, dev, stream)
         res["d256"] = run_d256(torch, kvq, dev, stream)
+    # last, so that its seconds under the power cap do not slow the figures above
+    res["sustained"] = run_sustained(torch, kvq, dev, stream, x, out, lam_t, s_t, G)
     return res
 
 
@@ -591,12 +592,13 @@ def run_variants(torch, kvq, dev, stream, x, out, s_t, G, w):
         cb = D // 2 if bits == 4 else D
         codes = torch.empty((n, cb), dtype=torch.uint8, device=dev)
         scales = torch.empty((n, D // G), dtype=torch.float16, device=dev)
-        q_ms = _event_ms(torch, stream, lambda: kvq.quantize_ex(
-            x, tables, s_t, G, bits=bits, lambda_after=after, lambda_rows=rows,
-            codes=codes, scales=scales, stream=stream, srft=srft), 10)
-        d_ms = _event_ms(torch, stream, lambda: kvq.dequantize_ex(
-            codes, scales, tables, s_t, G, bits=bits, lambda_after=after, lambda_rows=rows,
-            out=out, stream=stream, srft=srft), 10)
+        with ClockSampler(dev.index) as clk:
+            q_ms = _event_ms(torch, stream, lambda: kvq.quantize_ex(
+                x, tables, s_t, G, bits=bits, lambda_after=after, lambda_rows=rows,
+                codes=codes, scales=scales, stream=stream, srft=srft), 10)
+            d_ms = _event_ms(torch, stream, lambda: kvq.dequantize_ex(
+                codes, scales, tables, s_t, G, bits=bits, lambda_after=after, lambda_rows=rows,
+                out=out, stream=stream, srft=srft), 10)
         bpv = 2 * D + cb + 2 * (D // G)
         qg, dg = bpv * n / (q_ms / 1e3) / 1e9, bpv * n / (d_ms / 1e3) / 1e9
         name = f"int{bits}_lambda_{'after' if after else 'before'}" + ("_srft" if srft else "")
@@ -606,6 +608,7 @@ def run_variants(torch, kvq, dev, stream, x, out, s_t, G, w):
             "quantize_frac_of_peak": round(qg / peak, 4),
             "dequantize_ms": round(d_ms, 4), "dequantize_gbs": round(dg, 1),
             "dequantize_frac_of_peak": round(dg / peak, 4),
+            "sm_mhz": clk.summary()["sm_mhz"],
         }
         del codes, scales
     return res
@@ -657,11 +660,12 @@ def run_srft_lengths(torch, kvq, dev, stream, G=32, in_bytes=1 << 31):
         codes = torch.empty((n, D // 2), dtype=torch.uint8, device=dev)
         scales = torch.empty((n, D // G), dtype=torch.float16, device=dev)
         out = torch.empty_like(x)
-        q_ms = _event_ms(torch, stream, lambda: kvq.quantize_ex(
-            x, lam, sg, G, lambda_after=True, srft=True, codes=codes, scales=scales,
-            stream=stream), 10)
-        d_ms = _event_ms(torch, stream, lambda: kvq.dequantize_ex(
-            codes, scales, lam, sg, G, lambda_after=True, srft=True, out=out, stream=stream), 10)
+        with ClockSampler(dev.index) as clk:
+            q_ms = _event_ms(torch, stream, lambda: kvq.quantize_ex(
+                x, lam, sg, G, lambda_after=True, srft=True, codes=codes, scales=scales,
+                stream=stream), 10)
+            d_ms = _event_ms(torch, stream, lambda: kvq.dequantize_ex(
+                codes, scales, lam, sg, G, lambda_after=True, srft=True, out=out, stream=stream), 10)
         bpv = bytes_per_vector(D, G)
         qg, dg = bpv * n / (q_ms / 1e3) / 1e9, bpv * n / (d_ms / 1e3) / 1e9
         res[f"d{D}"] = {
@@ -670,6 +674,7 @@ def run_srft_lengths(torch, kvq, dev, stream, G=32, in_bytes=1 << 31):
             "quantize_gbs": round(qg, 1), "quantize_frac_of_peak": round(qg / peak, 4),
             "dequantize_ms": round(d_ms, 4), "dequantize_gvec_s": round(n / (d_ms / 1e3) / 1e9, 3),
             "dequantize_gbs": round(dg, 1), "dequantize_frac_of_peak": round(dg / peak, 4),
+            "sm_mhz": clk.summary()["sm_mhz"],
         }
         del x, codes, scales, out
         torch.cuda.empty_cache()
