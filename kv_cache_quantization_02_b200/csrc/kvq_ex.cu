@@ -19,9 +19,8 @@
 //
 // D = 128; G in {16, 32, 64}.  One lane holds a whole vector as 64 packed
 // fp32 pairs; each warp streams 32-vector tiles through its own
-// double-buffered ring, and the warps of a block (one per SM: 12 warps for the
-// quantisers and the lambda-after dequantisers, 8 for the lambda-before ones)
-// claim tiles of a contiguous range from a shared counter.  fp16 rows move by
+// double-buffered ring, and the 12 warps of a block (one block per SM) claim
+// tiles of a contiguous range from a shared counter.  fp16 rows move by
 // swizzled tensor copies; the codes leave the quantisers through the stage
 // their tile came from and one tensor store, and enter the dequantisers by a
 // swizzled tensor copy; scales move by bulk copies.  A warp tile lies inside one lambda
@@ -318,11 +317,10 @@ struct DeqLayout {
   static constexpr int WARP = (kXStage + 2 * WC + 2 * WS + 1023) / 1024 * 1024;
 };
 
-// Warps of a dequantize block (one block per SM): 12 with lambda after the
-// rotation (every stage in fp32 from the codes, at most 168 registers), 8
-// with lambda before (the fp16 in-group stages hold the codes' halves beside
-// the fp32 row: up to 255 registers).
-__host__ __device__ constexpr int deq_warps(bool after) { return after ? 12 : 8; }
+// Warps of a dequantize block (one block per SM): 12, at most 168 registers a
+// thread (the codes are unpacked, staged and converted a block of pairs at a
+// time, so that only that block's fp16 halves sit beside the fp32 row).
+__host__ __device__ constexpr int deq_warps(bool) { return 12; }
 
 // 16-byte chunk c of lane `lane`'s row of a code tile written by a tensor copy
 // swizzled over the row's CB bytes (64 or 128): chunk c of row t sits at
@@ -424,10 +422,21 @@ kvq_dequantize_ex_kernel(const __grid_constant__ CUtensorMap cmap,
       sx[j] = srow[j];
       sy[j] = srow[NGH + j];
     }
-    // codes of the pair (m, m+64) as exact fp16 integers.  Word w of a row is
-    // word w % 4 of its swizzled 16-byte chunk w / 4.  With lambda after the
-    // rotation each pair goes straight on to u = q S (exact) and u fp32(c /
-    // lambda), so that only the fp32 row stays live.
+    // With lambda before the rotation u = q S, and every butterfly stage inside
+    // a group keeps u an exact multiple of S: the stages h < HF run on the fp16
+    // integers (sums of at most 8 * 64 = 512 for int4 through all in-group
+    // stages, 128 * 16 = 2048 for int8 through four), then u = W S exactly by
+    // one mixed fma (W S has at most 23 significant bits), the same fp32
+    // values as the oracle's stage-by-stage sums.  With lambda after, 1/lambda
+    // comes before the transform and every stage runs in fp32: u = q S
+    // (exact), then u fp32(c / lambda).
+    constexpr int HF = AFTER ? 1 : (BITS == 4 ? (G < kNP ? G : kNP) : 16);
+    constexpr int PW = BITS == 4 ? 8 : 4;               // pairs a code word (of each half) holds
+    constexpr int HB = HF > PW ? HF : PW;               // pairs unpacked, staged and converted at a time
+    // The codes of the pair (m, m+64) as exact fp16 integers, one block of HB
+    // pairs at a time (the in-group stages stay inside a block), so that only
+    // a block's halves sit beside the fp32 row.  Word w of a row is word w % 4
+    // of its swizzled 16-byte chunk w / 4.
     __half2 hq[kNP];
     float2 p[kNP];
     auto to_row = [&](int m) {
@@ -437,11 +446,10 @@ kvq_dequantize_ex_kernel(const __grid_constant__ CUtensorMap cmap,
         p[m] = __fmul2_rn(p[m], (m & 1) ? make_float2(l.z, l.w) : make_float2(l.x, l.y));
       }
     };
-    if constexpr (BITS == 4) {
-      const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
-      uint32_t ra[4], rb[4];
-#pragma unroll
-      for (int kw = 0; kw < kNP / 8; ++kw) {
+    uint32_t ra[4], rb[4];
+    auto unpack_word = [&](int kw) {                    // the pairs PW kw .. PW kw + PW - 1
+      if constexpr (BITS == 4) {
+        const __half2 bias = __floats2half2_rn(1032.0f, 1032.0f);
         if (kw % 4 == 0) {              // channels 8 kw .. 8 kw + 31 and 64 + the same
           const uint4 ca = code_chunk<F::CB>(st, lane, kw / 4), cb = code_chunk<F::CB>(st, lane, 2 + kw / 4);
           ra[0] = ca.x; ra[1] = ca.y; ra[2] = ca.z; ra[3] = ca.w;
@@ -457,52 +465,39 @@ kvq_dequantize_ex_kernel(const __grid_constant__ CUtensorMap cmap,
           const uint32_t e1 = (__byte_perm(wa4, wb4, sel) & 0x000F000Fu) | 0x64006400u;
           hq[8 * kw + 2 * t] = __hsub2(*reinterpret_cast<const __half2*>(&e0), bias);
           hq[8 * kw + 2 * t + 1] = __hsub2(*reinterpret_cast<const __half2*>(&e1), bias);
-          if constexpr (AFTER) {
-            to_row(8 * kw + 2 * t);
-            to_row(8 * kw + 2 * t + 1);
-          }
         }
-      }
-    } else {
-      const __half2 bias = __floats2half2_rn(1152.0f, 1152.0f);
-#pragma unroll
-      for (int kw = 0; kw < kNP / 4; ++kw) {
+      } else {
+        const __half2 bias = __floats2half2_rn(1152.0f, 1152.0f);
         const uint4 ca = code_chunk<F::CB>(st, lane, kw >> 2);
         const uint4 cb = code_chunk<F::CB>(st, lane, (kw + kNP / 4) >> 2);
-        const uint32_t ra[4] = {ca.x, ca.y, ca.z, ca.w}, rb[4] = {cb.x, cb.y, cb.z, cb.w};
-        const uint32_t wa = ra[kw & 3] ^ 0x80808080u;
-        const uint32_t wb = rb[kw & 3] ^ 0x80808080u;
+        const uint32_t xa[4] = {ca.x, ca.y, ca.z, ca.w}, xb[4] = {cb.x, cb.y, cb.z, cb.w};
+        const uint32_t wa = xa[kw & 3] ^ 0x80808080u;
+        const uint32_t wb = xb[kw & 3] ^ 0x80808080u;
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const uint32_t sel = 0x0400u | (t << 8) | t;
           const uint32_t e = (__byte_perm(wa, wb, sel) & 0x00FF00FFu) | 0x64006400u;
           hq[4 * kw + t] = __hsub2(*reinterpret_cast<const __half2*>(&e), bias);
-          if constexpr (AFTER) to_row(4 * kw + t);
         }
       }
-    }
-    // With lambda before the rotation u = q S, and every butterfly stage inside
-    // a group keeps u an exact multiple of S: the stages h < HF run on the fp16
-    // integers (sums of at most 8 * 64 = 512 for int4 through all in-group
-    // stages, 128 * 16 = 2048 for int8 through four), then u = W S exactly by
-    // one mixed fma (W S has at most 23 significant bits), the same fp32
-    // values as the oracle's stage-by-stage sums.  With lambda after, 1/lambda
-    // comes before the transform and every stage runs in fp32.
-    constexpr int HF = AFTER ? 1 : (BITS == 4 ? (G < kNP ? G : kNP) : 16);
+    };
 #pragma unroll
-    for (int h = 1; h < HF; h <<= 1) {
+    for (int b0 = 0; b0 < kNP; b0 += HB) {
 #pragma unroll
-      for (int m = 0; m < kNP; ++m) {
-        if ((m & h) == 0) {
-          const __half2 a2 = hq[m], b2 = hq[m + h];
-          hq[m] = __hadd2(a2, b2);
-          hq[m + h] = __hsub2(a2, b2);
+      for (int kw = b0 / PW; kw < (b0 + HB) / PW; ++kw) unpack_word(kw);
+#pragma unroll
+      for (int h = 1; h < HF; h <<= 1) {
+#pragma unroll
+        for (int m = b0; m < b0 + HB; ++m) {
+          if ((m & h) == 0) {
+            const __half2 a2 = hq[m], b2 = hq[m + h];
+            hq[m] = __hadd2(a2, b2);
+            hq[m + h] = __hsub2(a2, b2);
+          }
         }
       }
-    }
-    if constexpr (!AFTER) {
 #pragma unroll
-      for (int m = 0; m < kNP; ++m) to_row(m);
+      for (int m = b0; m < b0 + HB; ++m) to_row(m);
     }
     __syncwarp();                       // codes and scales consumed: refill the stage
     refill(stage);
