@@ -333,6 +333,7 @@ def run_gpu(args):
         torch.cuda.empty_cache()
         extra["attention_decode_paper_format"] = run_attention_paper_format(torch, kvq, dev, stream,
                                                                             args.attn_seqs)
+        extra["attention_decode_gemma"] = run_attention_gemma(torch, kvq, dev, stream, args.attn_seqs)
     elif args.configs_only:
         extra = {"configs": run_configs(torch, kvq, dev, stream)}
     elif args.tc_only:
@@ -457,6 +458,7 @@ def run_extras(torch, kvq, dev, stream, x, out, lam_t, s_t, G, w, attn_seqs=64):
         del cache
         torch.cuda.empty_cache()
         res["attention_decode_paper_format"] = run_attention_paper_format(torch, kvq, dev, stream, attn_seqs)
+        res["attention_decode_gemma"] = run_attention_gemma(torch, kvq, dev, stream, attn_seqs)
         res["configs"] = run_configs(torch, kvq, dev, stream)
         res["d256"] = run_d256(torch, kvq, dev, stream)
     # last, so that its seconds under the power cap do not slow the figures above
@@ -830,6 +832,53 @@ def run_attention_paper_format(torch, kvq, dev, stream, seqs=64):
         "ms": round(ms, 4), "algorithmic_bytes": byts, "gbs": round(gbs, 1),
         "frac_of_peak": round(gbs / peak, 4), "peak_kind": kind,
     }
+
+
+def run_attention_gemma(torch, kvq, dev, stream, seqs=64):
+    """Decode attention at Gemma-3-1B's shape: D = 256, 4 query heads on one KV
+    head, 26 layers (folded into the batch with `seqs` sequences), 4096
+    positions, over real quantize output of the gemma-3-1b rows, in the base
+    format at G = 32 and in the paper's format (SRFT, lambda after, G = 16).
+    Algorithmic bytes: every K and V code and scale once, plus q and the
+    output."""
+    w = workloads.WORKLOADS["gemma-3-1b"]
+    D, Hq, Hkv, T = 256, 4, 1, 4096
+    B = seqs * 26
+    rows = 2 * B * Hkv * T
+    lam, sgn = workloads.params(D, w.seed + 11)
+    lam_t, s_t = torch.from_numpy(lam).to(dev), torch.from_numpy(sgn).to(dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(w.seed)
+    q = torch.randn((B, Hq, D), device=dev, generator=gen).half()
+    lens = torch.full((B,), T, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    peak, kind = hbm_peak()
+    res = {"shape": f"B={B} ({seqs} sequences x 26 layers), Hq={Hq}, Hkv={Hkv}, T={T}, D={D}"}
+    chunk = 1 << 22
+    buf = torch.empty((chunk, D), dtype=torch.float16, device=dev)
+    for name, G, fmt in (("g32", 32, False), ("paper_format_g16", 16, True)):
+        pk = torch.empty((2, B, Hkv, T, D // 2), dtype=torch.uint8, device=dev)
+        sc = torch.empty((2, B, Hkv, T, D // G), dtype=torch.float16, device=dev)
+        pk2, sc2 = pk.view(rows, D // 2), sc.view(rows, D // G)
+        for i, a in enumerate(range(0, rows, chunk)):
+            b = min(rows, a + chunk)
+            xr = workloads.device_rows(w, b - a, dev, seed_offset=i, out=buf[: b - a])
+            if fmt:
+                kvq.quantize_ex(xr, lam_t, s_t, G, lambda_after=True, srft=True,
+                                codes=pk2[a:b], scales=sc2[a:b], stream=stream)
+            else:
+                kvq.quantize(xr, lam_t, s_t, G, packed=pk2[a:b], scales=sc2[a:b], stream=stream)
+        ms = _event_ms(torch, stream, lambda: kvq.attention_decode(
+            q, pk[0], sc[0], pk[1], sc[1], lens, lam_t, s_t, lam_t, s_t, G, 1.0 / math.sqrt(D),
+            out=out, stream=stream, lambda_after=fmt, srft=fmt), 10)
+        byts = rows * (D // 2 + 2 * (D // G)) + 2 * q.numel() * 2
+        gbs = byts / (ms / 1e3) / 1e9
+        res[name] = {"G": G, "ms": round(ms, 4), "algorithmic_bytes": byts, "gbs": round(gbs, 1),
+                     "frac_of_peak": round(gbs / peak, 4), "peak_kind": kind}
+        del pk, sc
+    del buf, q, out
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_decode_step(torch, kvq, dev, stream, lam_t, s_t, G, cache, steps=1000):
