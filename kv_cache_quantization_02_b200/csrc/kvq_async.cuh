@@ -29,6 +29,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
   return false;
 }
+// One arrival on the barrier (release at CTA scope: this thread's earlier
+// shared-memory writes are visible to a thread that then sees the phase
+// complete).
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_addr(bar)) : "memory");
+}
 // The first 1 KiB-aligned byte of a dynamic shared-memory array, as an
 // offset from the array itself, so that the pointer stays in the shared
 // address space (shared loads and stores, not generic ones); the caller

@@ -240,23 +240,32 @@ thread_local int g_attn_cuda_error = 0;
 
 template <int D, int G>
 struct Attn {
+  // D = 256 runs in warp pairs: the two warps of a pair take the same key
+  // blocks, each the channels of one half, and add their partial scores
+  // through shared memory; the pair streams one ring of key blocks.
+  static constexpr bool PAIR = D == 256;
+  static constexpr int NRG = PAIR ? kAW / 2 : kAW;  // key-block streams (rings) per block
+  static constexpr int DH = PAIR ? D / 2 : D;       // channels of one warp
   static constexpr int NG = D / G;                  // scale groups of a row
-  static constexpr int NBK = D / 32;                // 32-channel blocks (score k-step pairs)
-  static constexpr int KS = D / 16;                 // k-steps of the score product
-  static constexpr int NCT = D / 16;                // 16-channel tiles of the value product
+  static constexpr int NGH = DH / G;                // scale groups of one warp
+  static constexpr int NBK = DH / 32;               // 32-channel blocks (score k-step pairs) of one warp
+  static constexpr int KS = DH / 16;                // k-steps of one warp's score product
+  static constexpr int NCT = DH / 16;               // 16-channel tiles of one warp's value product
   static constexpr int W32 = D / 8;                 // 32-bit words of one code row
-  static constexpr int ST = (D >= 256 || G == 16) ? 2 : 3;   // ring depth per warp
+  static constexpr int ST = (D >= 256 || G == 16) ? 2 : 3;   // ring depth
   static constexpr int CB = kBK * D / 2;            // code bytes of one block
   static constexpr int SB = kBK * NG * 2;           // scale bytes of one block
   static constexpr int STAGE = 2 * CB + 2 * SB;     // K codes, V codes, K scales, V scales
-  static constexpr int RING = kAW * ST * STAGE;
-  static constexpr int COMB = kAW * kMaxRows * D * 4;
+  static constexpr int RING = NRG * ST * STAGE;
+  static constexpr int COMB = NRG * kMaxRows * D * 4;
   static constexpr int AREA = RING > COMB ? RING : COMB;   // the merge reuses the ring
   static constexpr int QF = kMaxRows * D * 4;       // rotated query rows, fp32
-  static constexpr int SC = 2 * kBK * NG * 4;       // per warp: the block's K and V scales, fp32
+  static constexpr int SC = 2 * kBK * NGH * 4;      // per warp: the block's K and V scales, fp32
   static constexpr int PS = kBK + 8;                // row stride of the probability rows
   static constexpr int PB = kMaxRows * PS * 4;      // per warp: probabilities [head][key]
-  static constexpr int SMEM = AREA + QF + kAW * (SC + PB) + kAW * ST * 8 + kAW * kMaxRows * 8;
+  static constexpr int XZ = PAIR ? NRG * 2 * 2 * 2 * 4 * 32 * 4 : 0;   // partial scores [ring][parity][half][2 head tiles][4][lane]
+  static constexpr int NBAR = PAIR ? NRG * (2 * ST + 1) : kAW * ST;     // full (and empty, exchange) barriers
+  static constexpr int SMEM = AREA + QF + kAW * (SC + PB) + XZ + NBAR * 8 + kAW * kMaxRows * 8;
   static constexpr int DPL = D / 32;                // channels per lane in the row transforms
   static_assert(STAGE % 16 == 0 && (SC + PB) % 16 == 0, "16-byte aligned areas");
 };
@@ -343,6 +352,38 @@ __device__ __forceinline__ void load_row(float (&r)[N], const float* p) {
   } else {
 #pragma unroll
     for (int i = 0; i < N; ++i) r[i] = p[i];
+  }
+}
+
+// N fp16 scales from shared memory as fp32, in the widest loads their
+// alignment allows (the N halves start at a multiple of 2N bytes).
+template <int N>
+__device__ __forceinline__ void load_scales(float (&r)[N], const uint16_t* p) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      const uint2 u = *reinterpret_cast<const uint2*>(p + i);
+      const float2 a = half2_bits_to_float2(u.x), b = half2_bits_to_float2(u.y);
+      r[i] = a.x; r[i + 1] = a.y; r[i + 2] = b.x; r[i + 3] = b.y;
+    }
+  } else if constexpr (N == 2) {
+    const float2 a = half2_bits_to_float2(*reinterpret_cast<const uint32_t*>(p));
+    r[0] = a.x; r[1] = a.y;
+  } else {
+    r[0] = __half2float(__ushort_as_half(p[0]));
+  }
+}
+
+// N floats into shared memory (16-byte aligned when N is a multiple of 4).
+template <int N>
+__device__ __forceinline__ void store_row(float* p, const float (&r)[N]) {
+  if constexpr (N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) *reinterpret_cast<float4*>(p + i) = make_float4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+  } else if constexpr (N == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(r[0], r[1]);
+  } else {
+    p[0] = r[0];
   }
 }
 
@@ -435,23 +476,30 @@ __device__ __forceinline__ void finish_head(const AttnParams& P, float (&v)[D / 
 // One block of four warps per (sequence, KV head, key split); head tiles of
 // four query heads (NH = 1 for up to four heads per KV head, 2 for up to 8).
 template <int D, int G, int NH>
-__global__ void __launch_bounds__(kAW * 32, (D >= 256 || NH > 1) ? 2 : 3)
+__global__ void __launch_bounds__(kAW * 32, (NH > 1) ? 2 : 3)
 kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   using A = Attn<D, G>;
-  constexpr int NG = A::NG, NBK = A::NBK, KS = A::KS, NCT = A::NCT, W32 = A::W32, DPL = A::DPL;
+  constexpr bool PAIR = A::PAIR;
+  constexpr int NRG = A::NRG, DH = A::DH;
+  constexpr int NG = A::NG, NGH = A::NGH, NBK = A::NBK, KS = A::KS, NCT = A::NCT, W32 = A::W32, DPL = A::DPL;
   constexpr int ST = A::ST, PS = A::PS;
   constexpr int CPG = (G >= 32) ? G / 32 : 1;     // score k-step pairs per group (G = 16: two groups per pair)
   extern __shared__ __align__(128) uint8_t sm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint8_t* ring = sm;                                                  // [warp][stage][STAGE]
+  const int rg = PAIR ? warp >> 1 : warp;          // this warp's ring (key-block stream)
+  const int half = PAIR ? warp & 1 : 0;            // the channel half of a pair's warp
+  const bool issuer = half == 0;                   // the warp that issues the ring's copies
+  const int cofs = half * DH, gofs = cofs / G;     // this warp's first channel and group
+  uint8_t* ring = sm;                                                  // [ring][stage][STAGE]
   float* qf = reinterpret_cast<float*>(sm + A::AREA);                  // [8][D]
   float* scw = qf + kMaxRows * D + warp * ((A::SC + A::PB) / 4);       // this warp's area:
-  float* sk = scw;                                                     //   K scales [kBK][NG], fp32
-  float* sv = scw + kBK * NG;                                          //   V scales [kBK][NG], fp32
+  float* sk = scw;                                                     //   K scales [kBK][NGH], fp32
+  float* sv = scw + kBK * NGH;                                         //   V scales [kBK][NGH], fp32
   float* pw = scw + A::SC / 4;                                         //   probabilities [8][PS]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + A::AREA + A::QF + kAW * (A::SC + A::PB));
-  float* ml = reinterpret_cast<float*>(bars + kAW * ST);               // [warp][8][2]: m, l
-  float* comb = reinterpret_cast<float*>(sm);                          // [warp][8][D], after the key loop
+  float* xz = reinterpret_cast<float*>(sm + A::AREA + A::QF + kAW * (A::SC + A::PB));   // pairs' partial scores
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + A::AREA + A::QF + kAW * (A::SC + A::PB) + A::XZ);
+  float* ml = reinterpret_cast<float*>(bars + A::NBAR);               // [ring][8][2]: m, l
+  float* comb = reinterpret_cast<float*>(sm);                          // [ring][8][D], after the key loop
 
   const int g = lane >> 2, t = lane & 3;
   const int item = blockIdx.x;
@@ -469,24 +517,30 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   const int nkeys = k1 > k0 ? k1 - k0 : 0;
   const int nblk = (nkeys + kBK - 1) / kBK;
 
-  uint64_t* bar = bars + ST * warp;
-  if (lane == 0) {
+  uint64_t* bar = bars + ST * rg;                  // the ring's stages are full
+  uint64_t* empty = bars + NRG * ST + ST * rg;     // pairs: both warps are done with a stage
+  uint64_t* xch = bars + 2 * NRG * ST + rg;        // pairs: both warps wrote their partial scores
+  if (lane == 0 && issuer) {
     for (int s = 0; s < ST; ++s) mbar_init(&bar[s], 1);
+    if constexpr (PAIR) {
+      for (int s = 0; s < ST; ++s) mbar_init(&empty[s], 2);
+      mbar_init(xch, 64);
+    }
     mbar_fence_init();
   }
   const int64_t row_base = static_cast<int64_t>(bh) * P.T;
-  // The warp's blocks are warp, warp + kAW, ...; each issue copies the next
-  // one into the given stage, the sources advancing by kAW blocks of rows.
-  int next_blk = warp, next_kb = k0 + warp * kBK;
+  // The ring's blocks are rg, rg + NRG, ...; each issue copies the next one
+  // into the given stage, the sources advancing by NRG blocks of rows.
+  int next_blk = rg, next_kb = k0 + rg * kBK;
   const uint8_t* kp_next = P.kp + (row_base + next_kb) * (D / 2);
   const uint8_t* vp_next = P.vp + (row_base + next_kb) * (D / 2);
   const uint16_t* ks_next = P.ks + (row_base + next_kb) * NG;
   const uint16_t* vs_next = P.vs + (row_base + next_kb) * NG;
   auto issue = [&](int stage) {
-    if (next_blk < nblk && lane == 0) {
+    if (next_blk < nblk && lane == 0 && issuer) {
       const int nk = min(kBK, k1 - next_kb);
       const int nk16 = (nk + 15) & ~15;                          // stays inside T (T % 16 == 0)
-      uint8_t* st = ring + (warp * ST + stage) * A::STAGE;
+      uint8_t* st = ring + (rg * ST + stage) * A::STAGE;
       const uint32_t cb = static_cast<uint32_t>(nk16 * (D / 2));
       const uint32_t sb = static_cast<uint32_t>(nk16 * NG * 2);
       mbar_expect_tx(&bar[stage], 2 * cb + 2 * sb);
@@ -495,12 +549,12 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
       bulk_g2s(st + 2 * A::CB, ks_next, sb, &bar[stage]);
       bulk_g2s(st + 2 * A::CB + A::SB, vs_next, sb, &bar[stage]);
     }
-    next_blk += kAW;
-    next_kb += kAW * kBK;
-    kp_next += kAW * kBK * (D / 2);
-    vp_next += kAW * kBK * (D / 2);
-    ks_next += kAW * kBK * NG;
-    vs_next += kAW * kBK * NG;
+    next_blk += NRG;
+    next_kb += NRG * kBK;
+    kp_next += NRG * kBK * (D / 2);
+    vp_next += NRG * kBK * (D / 2);
+    ks_next += NRG * kBK * NG;
+    vs_next += NRG * kBK * NG;
   };
   __syncwarp();
   for (int s = 0; s < ST; ++s) issue(s);
@@ -574,7 +628,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
 #pragma unroll
     for (int j = 0; j < KS; ++j) {
       const float* qr = qf + (4 * ht + (g >> 1)) * D;
-      const int c0 = 8 * (4 * (j >> 1) + t) + 2 * (j & 1);
+      const int c0 = cofs + 8 * (4 * (j >> 1) + t) + 2 * (j & 1);
       const int part = g & 1;
       const uint32_t b0 = f16_part(qr[c0], part) | (uint32_t(f16_part(qr[c0 + 4], part)) << 16);
       const uint32_t b1 = f16_part(qr[c0 + 1] * 0.0625f, part) |
@@ -594,14 +648,14 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   // the group's sum of the B entries (times 16 for the high-nibble entries),
   // both parts, of this lane's score head 4 ht + t.  The eight lanes of a
   // head split the group's channels and add up by shuffles.
-  float bias[NH][NG];
+  float bias[NH][NGH];
 #pragma unroll
   for (int ht = 0; ht < NH; ++ht) {
     const float* qr = qf + (4 * ht + t) * D;
 #pragma unroll
-    for (int gi = 0; gi < NG; ++gi) {
+    for (int gi = 0; gi < NGH; ++gi) {
       float s0 = 0.0f, s1 = 0.0f;
-      for (int c = gi * G + g; c < (gi + 1) * G; c += 8) {
+      for (int c = (gofs + gi) * G + g; c < (gofs + gi + 1) * G; c += 8) {
         const bool odd = c & 1;
         const float v = odd ? qr[c] * 0.0625f : qr[c];
         const float w = odd ? 16.0f : 1.0f;
@@ -628,11 +682,11 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   for (int ht = 0; ht < NH; ++ht) { m[ht] = -INFINITY; l[ht] = 0.0f; }
   // sum of p S_V per group over this lane's keys, head 4 ht + g/2: the value
   // product runs on biased codes, and 8 times this is its bias
-  float pc[NH][NG];
+  float pc[NH][NGH];
 #pragma unroll
   for (int ht = 0; ht < NH; ++ht)
 #pragma unroll
-    for (int gi = 0; gi < NG; ++gi) pc[ht][gi] = 0.0f;
+    for (int gi = 0; gi < NGH; ++gi) pc[ht][gi] = 0.0f;
   bool head_ok[NH];                    // this lane's score head is a real head
 #pragma unroll
   for (int ht = 0; ht < NH; ++ht) head_ok[ht] = 4 * ht + t < R;
@@ -641,13 +695,13 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   int k = 0;
   int stage = 0;
   uint32_t phase = 0;                  // parity of the stage's current fill
-  for (int blk = warp; blk < nblk; blk += kAW, ++k) {
+  for (int blk = rg; blk < nblk; blk += NRG, ++k) {
     const bool ok = mbar_wait(&bar[stage], phase, kSpin);
     if (__any_sync(kFull, !ok)) {
       failed = true;
       break;
     }
-    const uint8_t* st = ring + (warp * ST + stage) * A::STAGE;
+    const uint8_t* st = ring + (rg * ST + stage) * A::STAGE;
     const uint32_t* kc = reinterpret_cast<const uint32_t*>(st);
     const uint32_t* vc = reinterpret_cast<const uint32_t*>(st + A::CB);
     const uint16_t* ksh = reinterpret_cast<const uint16_t*>(st + 2 * A::CB);
@@ -658,6 +712,20 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
 
     // The block's scales as fp32; in a tail block, keys at or past nk (stale
     // or unwritten rows) get 0, so that their zero weights stay exactly 0.
+    if constexpr (PAIR) {
+      // lane = key: the scales of this warp's groups
+      const bool live = !tail || lane < nk;
+      float kf[NGH], vf[NGH];
+      load_scales<NGH>(kf, ksh + lane * NG + gofs);
+      load_scales<NGH>(vf, vsh + lane * NG + gofs);
+#pragma unroll
+      for (int e = 0; e < NGH; ++e) {
+        kf[e] = live ? kf[e] : 0.0f;
+        vf[e] = live ? vf[e] : 0.0f;
+      }
+      store_row<NGH>(sk + lane * NGH, kf);
+      store_row<NGH>(sv + lane * NGH, vf);
+    } else {
 #pragma unroll
     for (int i0 = 0; i0 < kBK * NG; i0 += 128) {
       const int i = i0 + 4 * lane;
@@ -679,6 +747,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         *reinterpret_cast<float4*>(sv + i) = make_float4(vo[0], vo[1], vo[2], vo[3]);
       }
     }
+    }
     __syncwarp();
 
     // Scores, log2 units: zs[ht][mt][r] for key 16 mt + g + 8 r of head 4 ht + t.
@@ -690,9 +759,9 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     for (int mt = 0; mt < 2; ++mt) {
       constexpr int GPB = (G == 16) ? 2 : 1;          // groups finished per 32-channel block
       float acc[NH][GPB][4];
-      float s0[NG], s1[NG];
-      load_row<NG>(s0, sk + (16 * mt + g) * NG);
-      load_row<NG>(s1, sk + (16 * mt + 8 + g) * NG);
+      float s0[NGH], s1[NGH];
+      load_row<NGH>(s0, sk + (16 * mt + g) * NGH);
+      load_row<NGH>(s1, sk + (16 * mt + 8 + g) * NGH);
       float z0[NH], z1[NH];
 #pragma unroll
       for (int ht = 0; ht < NH; ++ht) z0[ht] = z1[ht] = 0.0f;
@@ -703,7 +772,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         // j = (keys 8 (j & 1) .. + 7 of the M-tile, 16-byte chunk bb + j / 2)
         if (bb % 2 == 0)
           ldsm_x4(kw, reinterpret_cast<const uint8_t*>(kc) + (16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1)) * (D / 2) +
-                          16 * (bb + (lane >> 4)));
+                          16 * (half * NBK + bb + (lane >> 4)));
         const uint32_t w0 = kw[2 * (bb & 1)] ^ kBias8;
         const uint32_t w1 = kw[2 * (bb & 1) + 1] ^ kBias8;
         const uint32_t a0[4] = {lo_pair(w0), lo_pair(w1), hi_pair(w0), hi_pair(w1)};
@@ -736,14 +805,46 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
       }
 #pragma unroll
       for (int ht = 0; ht < NH; ++ht) {
-        zs[ht][mt][0] = z0[ht] * scale;
-        zs[ht][mt][1] = z1[ht] * scale;
+        zs[ht][mt][0] = z0[ht];
+        zs[ht][mt][1] = z1[ht];
+      }
+    }
+    if constexpr (PAIR) {
+      // the two halves' partial scores through shared memory (one buffer per
+      // block parity, so that a warp one block ahead writes the other one),
+      // added in the same order by both warps
+      float* xo = xz + ((rg * 2 + (k & 1)) * 2 + half) * 256;
+      const float* xi = xz + ((rg * 2 + (k & 1)) * 2 + (half ^ 1)) * 256;
+#pragma unroll
+      for (int ht = 0; ht < NH; ++ht)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xo[(ht * 4 + i) * 32 + lane] = zs[ht][i >> 1][i & 1];
+      mbar_arrive(xch);
+      const bool okx = mbar_wait(xch, k & 1, kSpin);
+      if (__any_sync(kFull, !okx)) {
+        failed = true;
+        break;
+      }
+#pragma unroll
+      for (int ht = 0; ht < NH; ++ht)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float o = xi[(ht * 4 + i) * 32 + lane];
+          float& z = zs[ht][i >> 1][i & 1];
+          z = half ? o + z : z + o;
+        }
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int ht = 0; ht < NH; ++ht) {
+        zs[ht][mt][0] *= scale;
+        zs[ht][mt][1] *= scale;
         if (tail || !head_ok[ht]) {          // keys past nk and padded heads weigh 0
           if (!head_ok[ht] || 16 * mt + g >= nk) zs[ht][mt][0] = -INFINITY;
           if (!head_ok[ht] || 16 * mt + 8 + g >= nk) zs[ht][mt][1] = -INFINITY;
         }
       }
-    }
 
     // Online softmax per head, over the block's 32 keys: the eight lanes of a
     // head (same t) hold four keys each.
@@ -764,7 +865,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         }
         const float alpha_b = __shfl_sync(kFull, alpha, g >> 1);   // head 4 ht + g/2
 #pragma unroll
-        for (int gi = 0; gi < NG; ++gi) pc[ht][gi] *= alpha_b;
+        for (int gi = 0; gi < NGH; ++gi) pc[ht][gi] *= alpha_b;
       }
       // key 16 mt + 8 r + g goes to slot 16 mt + 8 r + g (G >= 32), or to
       // 16 mt + 8 r + 2 (g & 3) + (g >> 2) (G = 16, whose value product's
@@ -803,17 +904,17 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         pa[ht] = *reinterpret_cast<const float2*>(prow);
         pb[ht] = *reinterpret_cast<const float2*>(prow + 8);
       }
-      constexpr int GC = NG < 4 ? NG : 4;             // groups per scale load
+      constexpr int GC = NGH < 4 ? NGH : 4;           // groups per scale load
       float sq[4][GC];
       uint32_t vw[4];                                 // two chunks of V codes, transposed
 #pragma unroll
-      for (int gi = 0; gi < NG; ++gi) {
+      for (int gi = 0; gi < NGH; ++gi) {
         // B fragments of this group: p S_V for the four keys, as part g & 1
         if (gi % GC == 0) {
-          load_row<GC>(sq[0], sv + ka * NG + gi);
-          load_row<GC>(sq[1], sv + (ka + KSTEP) * NG + gi);
-          load_row<GC>(sq[2], sv + (ka + 8) * NG + gi);
-          load_row<GC>(sq[3], sv + (ka + 8 + KSTEP) * NG + gi);
+          load_row<GC>(sq[0], sv + ka * NGH + gi);
+          load_row<GC>(sq[1], sv + (ka + KSTEP) * NGH + gi);
+          load_row<GC>(sq[2], sv + (ka + 8) * NGH + gi);
+          load_row<GC>(sq[3], sv + (ka + 8 + KSTEP) * NGH + gi);
         }
         const float s0 = sq[0][gi % GC], s1 = sq[1][gi % GC], s2 = sq[2][gi % GC], s3 = sq[3][gi % GC];
         uint32_t bv[NH][2];
@@ -827,7 +928,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         if constexpr (G == 16) {
           // tile gi: channels 16 gi + 2 g (low nibble, row g) and + 1 (row g + 8):
           // byte g & 3 of word 2 gi + g / 4
-          const int wv = 2 * gi + (g >> 2), by = g & 3;
+          const int wv = half * (DH / 8) + 2 * gi + (g >> 2), by = g & 3;
           const uint32_t w0 = vc[ka * W32 + wv], w1 = vc[(ka + 4) * W32 + wv];
           const uint32_t w2 = vc[(ka + 8) * W32 + wv], w3 = vc[(ka + 12) * W32 + wv];
           const uint32_t sel = static_cast<uint32_t>(by | ((4 + by) << 4));
@@ -845,7 +946,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
             if (j % 2 == 0)
               ldsm_x4_t(vw, reinterpret_cast<const uint8_t*>(vc) +
                                 (16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1)) * (D / 2) +
-                                16 * ((j & ~1) + (lane >> 4)));
+                                16 * (half * (DH / 32) + (j & ~1) + (lane >> 4)));
             const uint32_t x0 = vw[2 * (j & 1)] ^ kBias8;       // keys 2t, 2t + 1
             const uint32_t x1 = vw[2 * (j & 1) + 1] ^ kBias8;   // keys 2t + 8, 2t + 9
             const uint32_t aa[4] = {lo_pair(x0), hi_pair(x0), lo_pair(x1), hi_pair(x1)};
@@ -860,6 +961,17 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
       }
     }
     __syncwarp();                      // the stage and the probability rows are consumed
+    if constexpr (PAIR) {
+      // the issuing warp refills the stage once its partner is done with it too
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      if (issuer) {
+        const bool oke = mbar_wait(&empty[stage], phase, kSpin);
+        if (__any_sync(kFull, !oke)) {
+          failed = true;
+          break;
+        }
+      }
+    }
     issue(stage);
     if (++stage == ST) { stage = 0; phase ^= 1u; }
   }
@@ -870,7 +982,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
     // included, before the ring is reused
     for (int s = 0; s < ST; ++s) {
       const int kk2 = k + s;
-      if (warp + kk2 * kAW < nblk && !mbar_wait(&bar[kk2 % ST], (kk2 / ST) & 1, kSpin))
+      if (issuer && rg + kk2 * NRG < nblk && !mbar_wait(&bar[kk2 % ST], (kk2 / ST) & 1, kSpin))
         lost = true;
     }
     lost = __any_sync(kFull, lost);
@@ -883,11 +995,11 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   }
   // the bias sums of head 4 ht + t (lanes 8t .. 8t + 3 hold them after the
   // reduction over t)
-  float bsum[NH][NG];
+  float bsum[NH][NGH];
 #pragma unroll
   for (int ht = 0; ht < NH; ++ht)
 #pragma unroll
-    for (int gi = 0; gi < NG; ++gi) {
+    for (int gi = 0; gi < NGH; ++gi) {
       float v = pc[ht][gi];
       v += __shfl_xor_sync(kFull, v, 1);
       v += __shfl_xor_sync(kFull, v, 2);
@@ -902,7 +1014,7 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   for (int ht = 0; ht < NH; ++ht) {
     const int h = 4 * ht + t;
     if (h < R) {
-      float* cw = comb + (warp * kMaxRows + h) * D;
+      float* cw = comb + (rg * kMaxRows + h) * D + cofs;
 #pragma unroll
       for (int ct = 0; ct < NCT; ++ct) {
         const int byte = (G == 16) ? 8 * ct + g : 16 * (ct >> 1) + 2 * g + (ct & 1);
@@ -910,9 +1022,9 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         cw[2 * byte] = __fmaf_rn(O[ht][ct][0] + O[ht][ct][1], 0x1p24f, -bz);
         cw[2 * byte + 1] = __fmaf_rn(O[ht][ct][2] + O[ht][ct][3], 0x1p20f, -bz);
       }
-      if (g == 0) {
-        ml[(warp * kMaxRows + h) * 2] = m[ht];
-        ml[(warp * kMaxRows + h) * 2 + 1] = l[ht];
+      if (g == 0 && issuer) {
+        ml[(rg * kMaxRows + h) * 2] = m[ht];
+        ml[(rg * kMaxRows + h) * 2 + 1] = l[ht];
       }
     }
   }
@@ -921,12 +1033,12 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
   for (int r = warp; r < R; r += kAW) {
     float M = -INFINITY;
 #pragma unroll
-    for (int w2 = 0; w2 < kAW; ++w2) M = fmaxf(M, ml[(w2 * kMaxRows + r) * 2]);
+    for (int w2 = 0; w2 < NRG; ++w2) M = fmaxf(M, ml[(w2 * kMaxRows + r) * 2]);
     float lsum = 0.0f, v[DPL];
 #pragma unroll
     for (int i = 0; i < DPL; ++i) v[i] = 0.0f;
 #pragma unroll
-    for (int w2 = 0; w2 < kAW; ++w2) {
+    for (int w2 = 0; w2 < NRG; ++w2) {
       const float mw = ml[(w2 * kMaxRows + r) * 2];
       const float e = (mw == -INFINITY) ? 0.0f : exp2f(mw - M);
       lsum += e * ml[(w2 * kMaxRows + r) * 2 + 1];
