@@ -255,7 +255,10 @@ struct Attn {
   static constexpr int ST = (D >= 256 || G == 16) ? 2 : 3;   // ring depth
   static constexpr int CB = kBK * D / 2;            // code bytes of one block
   static constexpr int SB = kBK * NG * 2;           // scale bytes of one block
-  static constexpr int STAGE = 2 * CB + 2 * SB;     // K codes, V codes, K scales, V scales
+  // K codes, V codes, K scales, V scales; in pairs (128-byte code rows, which
+  // arrive by 128-byte-swizzled tensor copies) a multiple of 1 KiB, the
+  // swizzle's period
+  static constexpr int STAGE = PAIR ? (2 * CB + 2 * SB + 1023) / 1024 * 1024 : 2 * CB + 2 * SB;
   static constexpr int RING = NRG * ST * STAGE;
   static constexpr int COMB = NRG * kMaxRows * D * 4;
   static constexpr int AREA = RING > COMB ? RING : COMB;   // the merge reuses the ring
@@ -265,7 +268,7 @@ struct Attn {
   static constexpr int PB = kMaxRows * PS * 4;      // per warp: probabilities [head][key]
   static constexpr int XZ = PAIR ? NRG * 2 * 2 * 2 * 4 * 32 * 4 : 0;   // partial scores [ring][parity][half][2 head tiles][4][lane]
   static constexpr int NBAR = PAIR ? NRG * (2 * ST + 1) : kAW * ST;     // full (and empty, exchange) barriers
-  static constexpr int SMEM = AREA + QF + kAW * (SC + PB) + XZ + NBAR * 8 + kAW * kMaxRows * 8;
+  static constexpr int SMEM = AREA + QF + kAW * (SC + PB) + XZ + NBAR * 8 + kAW * kMaxRows * 8 + (PAIR ? 1024 : 0);
   static constexpr int DPL = D / 32;                // channels per lane in the row transforms
   static_assert(STAGE % 16 == 0 && (SC + PB) % 16 == 0, "16-byte aligned areas");
 };
@@ -477,14 +480,16 @@ __device__ __forceinline__ void finish_head(const AttnParams& P, float (&v)[D / 
 // four query heads (NH = 1 for up to four heads per KV head, 2 for up to 8).
 template <int D, int G, int NH>
 __global__ void __launch_bounds__(kAW * 32, (NH > 1) ? 2 : 3)
-kvq_attn_kernel(const __grid_constant__ AttnParams P) {
+kvq_attn_kernel(const __grid_constant__ AttnParams P, const __grid_constant__ CUtensorMap kmap,
+                const __grid_constant__ CUtensorMap vmap) {
   using A = Attn<D, G>;
   constexpr bool PAIR = A::PAIR;
   constexpr int NRG = A::NRG, DH = A::DH;
-  constexpr int NG = A::NG, NGH = A::NGH, NBK = A::NBK, KS = A::KS, NCT = A::NCT, W32 = A::W32, DPL = A::DPL;
+  constexpr int NG = A::NG, NGH = A::NGH, NBK = A::NBK, KS = A::KS, NCT = A::NCT, DPL = A::DPL;
   constexpr int ST = A::ST, PS = A::PS;
   constexpr int CPG = (G >= 32) ? G / 32 : 1;     // score k-step pairs per group (G = 16: two groups per pair)
-  extern __shared__ __align__(128) uint8_t sm[];
+  extern __shared__ __align__(128) uint8_t sm_raw[];
+  uint8_t* sm = PAIR ? align_smem_1k(sm_raw) : sm_raw;   // pairs: 1 KiB-aligned stages
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rg = PAIR ? warp >> 1 : warp;          // this warp's ring (key-block stream)
   const int half = PAIR ? warp & 1 : 0;            // the channel half of a pair's warp
@@ -543,9 +548,16 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
       uint8_t* st = ring + (rg * ST + stage) * A::STAGE;
       const uint32_t cb = static_cast<uint32_t>(nk16 * (D / 2));
       const uint32_t sb = static_cast<uint32_t>(nk16 * NG * 2);
-      mbar_expect_tx(&bar[stage], 2 * cb + 2 * sb);
-      bulk_g2s(st, kp_next, cb, &bar[stage]);
-      bulk_g2s(st + A::CB, vp_next, cb, &bar[stage]);
+      if constexpr (PAIR) {        // whole 32-row boxes (rows past the split are masked)
+        mbar_expect_tx(&bar[stage], 2 * A::CB + 2 * sb);
+        const int y = static_cast<int>(row_base + next_kb);
+        tensor_g2s(st, &kmap, 0, y, &bar[stage]);
+        tensor_g2s(st + A::CB, &vmap, 0, y, &bar[stage]);
+      } else {
+        mbar_expect_tx(&bar[stage], 2 * cb + 2 * sb);
+        bulk_g2s(st, kp_next, cb, &bar[stage]);
+        bulk_g2s(st + A::CB, vp_next, cb, &bar[stage]);
+      }
       bulk_g2s(st + 2 * A::CB, ks_next, sb, &bar[stage]);
       bulk_g2s(st + 2 * A::CB + A::SB, vs_next, sb, &bar[stage]);
     }
@@ -691,6 +703,9 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
 #pragma unroll
   for (int ht = 0; ht < NH; ++ht) head_ok[ht] = 4 * ht + t < R;
   const float scale = P.scale_log2;
+  // byte offset of 16-byte chunk c of code row r in a stage's code tile (pairs:
+  // the tensor copy's 128-byte swizzle puts it at chunk c ^ (r mod 8))
+  auto code_at = [](int r, int c) -> int { return r * (D / 2) + ((PAIR ? (c ^ (r & 7)) : c) << 4); };
   bool failed = false;
   int k = 0;
   int stage = 0;
@@ -771,8 +786,8 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
         // words 4 bb + t of keys g and g + 8, two blocks bb per load: matrix
         // j = (keys 8 (j & 1) .. + 7 of the M-tile, 16-byte chunk bb + j / 2)
         if (bb % 2 == 0)
-          ldsm_x4(kw, reinterpret_cast<const uint8_t*>(kc) + (16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1)) * (D / 2) +
-                          16 * (half * NBK + bb + (lane >> 4)));
+          ldsm_x4(kw, reinterpret_cast<const uint8_t*>(kc) +
+                          code_at(16 * mt + (lane & 7) + 8 * ((lane >> 3) & 1), half * NBK + bb + (lane >> 4)));
         const uint32_t w0 = kw[2 * (bb & 1)] ^ kBias8;
         const uint32_t w1 = kw[2 * (bb & 1) + 1] ^ kBias8;
         const uint32_t a0[4] = {lo_pair(w0), lo_pair(w1), hi_pair(w0), hi_pair(w1)};
@@ -929,8 +944,8 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
           // tile gi: channels 16 gi + 2 g (low nibble, row g) and + 1 (row g + 8):
           // byte g & 3 of word 2 gi + g / 4
           const int wv = half * (DH / 8) + 2 * gi + (g >> 2), by = g & 3;
-          const uint32_t w0 = vc[ka * W32 + wv], w1 = vc[(ka + 4) * W32 + wv];
-          const uint32_t w2 = vc[(ka + 8) * W32 + wv], w3 = vc[(ka + 12) * W32 + wv];
+          auto word = [&](int r) { return vc[code_at(r, wv >> 2) / 4 + (wv & 3)]; };
+          const uint32_t w0 = word(ka), w1 = word(ka + 4), w2 = word(ka + 8), w3 = word(ka + 12);
           const uint32_t sel = static_cast<uint32_t>(by | ((4 + by) << 4));
           const uint32_t x = __byte_perm(__byte_perm(w0, w1, sel), __byte_perm(w2, w3, sel), 0x5140u) ^ kBias8;
           const uint32_t av[4] = {lo_pair(x), hi_pair(x), lo_pair(x >> 8), hi_pair(x >> 8)};
@@ -945,8 +960,8 @@ kvq_attn_kernel(const __grid_constant__ AttnParams P) {
             // matrix m = (keys 8 (m & 1) .. + 7 of the step, chunk (j & ~1) + m / 2)
             if (j % 2 == 0)
               ldsm_x4_t(vw, reinterpret_cast<const uint8_t*>(vc) +
-                                (16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1)) * (D / 2) +
-                                16 * (half * (DH / 32) + (j & ~1) + (lane >> 4)));
+                                code_at(16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1),
+                                        half * (DH / 32) + (j & ~1) + (lane >> 4)));
             const uint32_t x0 = vw[2 * (j & 1)] ^ kBias8;       // keys 2t, 2t + 1
             const uint32_t x1 = vw[2 * (j & 1) + 1] ^ kBias8;   // keys 2t + 8, 2t + 9
             const uint32_t aa[4] = {lo_pair(x0), hi_pair(x0), lo_pair(x1), hi_pair(x1)};
@@ -1091,10 +1106,39 @@ kvq_attn_combine_kernel(const __grid_constant__ AttnParams P) {
 // Launch plumbing.
 // ---------------------------------------------------------------------------
 
+// A tensor map over the code rows [rows][D/2 bytes] in 32-row boxes with the
+// 128-byte swizzle (D = 256, whose rows are 128 bytes).
+int encode_code_rows(CUtensorMap& map, const uint8_t* codes, int64_t rows) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (enc == nullptr) return KVQ_ERR_LAUNCH;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(KVQ_ATTN_D / 2), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(KVQ_ATTN_D / 2)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(KVQ_ATTN_D / 2), static_cast<cuuint32_t>(kBK)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    g_attn_cuda_error = static_cast<int>(r);
+    return KVQ_ERR_LAUNCH;
+  }
+  return KVQ_OK;
+}
+
 template <int D, int G, int NH>
 int launch_attn(const AttnParams& P, int64_t pairs, cudaStream_t st) {
   using A = Attn<D, G>;
   auto k = kvq_attn_kernel<D, G, NH>;
+  CUtensorMap kmap, vmap;                        // pairs only: the code tiles' tensor copies
+  memset(&kmap, 0, sizeof(kmap));
+  memset(&vmap, 0, sizeof(vmap));
+  if constexpr (A::PAIR) {
+    const int64_t rows = pairs * P.T;
+    if (rows >= (int64_t{1} << 31)) return KVQ_ERR_COUNT;   // tensor-copy row coordinates are int32
+    int rc = encode_code_rows(kmap, P.kp, rows);
+    if (rc == KVQ_OK) rc = encode_code_rows(vmap, P.vp, rows);
+    if (rc != KVQ_OK) return rc;
+  }
   static std::atomic<int> ready[64];             // the shared-memory opt-in, once per device
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
@@ -1104,7 +1148,7 @@ int launch_attn(const AttnParams& P, int64_t pairs, cudaStream_t st) {
   }
   const int64_t items = pairs * P.nsplit;
   (void)cudaGetLastError();
-  k<<<static_cast<unsigned>(items), kAW * 32, A::SMEM, st>>>(P);
+  k<<<static_cast<unsigned>(items), kAW * 32, A::SMEM, st>>>(P, kmap, vmap);
   if (P.nsplit > 1)
     kvq_attn_combine_kernel<D><<<static_cast<unsigned>(pairs), kMaxRows * 32, 0, st>>>(P);
   const cudaError_t e = cudaGetLastError();
