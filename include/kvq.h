@@ -236,8 +236,10 @@ int kvq_dequantize_ex(const uint8_t *codes, const uint16_t *scales,
  *                   int8 [D] with values +-1).
  *   B, Hq, Hkv, T  sequences, query heads, KV heads, cache positions:
  *                   B >= 0, Hkv >= 1, Hq a multiple of Hkv with Hq / Hkv <= 8,
- *                   T >= 0 a multiple of 16, B * Hkv * T < 2^40 cache rows
- *                   (else KVQ_ERR_COUNT).
+ *                   T >= 0 a multiple of 16, B * Hkv * T < 2^40 cache rows,
+ *                   < 2^31 at D = 256 (whose code tiles arrive by tensor
+ *                   copies with 32-bit row coordinates; 2^31 rows of K codes
+ *                   alone are 256 GiB) (else KVQ_ERR_COUNT).
  *   D, group  D in {64, 128, 256} (else KVQ_ERR_DIM); group in
  *                   {16, 32, 64, 128}, group <= D (else KVQ_ERR_GROUP).
  *   sm_scale  softmax scale, finite (usually 1/sqrt(D)).
