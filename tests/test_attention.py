@@ -116,6 +116,9 @@ CASES = [
     (1, 4, 1, 128, 256, 16, [128]),
     (2, 16, 2, 48, 256, 64, [48, 31]),
     (1, 8, 1, 64, 256, 128, [60]),
+    (1, 8, 1, 256, 256, 16, [256]),             # D = 256, 8 heads per KV head: two head tiles per warp pair
+    (2, 16, 2, 512, 256, 32, [512, 300]),       # many blocks per pair, a ragged last block
+    (1, 4, 1, 4096, 256, 32, [4000]),           # one pair: the key axis splits
 ]
 
 
