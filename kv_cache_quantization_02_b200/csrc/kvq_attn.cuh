@@ -19,8 +19,12 @@
 //
 // Work decomposition.  A block of four warps owns one (sequence, KV head,
 // key split); each warp streams 32-key blocks (codes and scales of K and V,
-// four bulk copies into a private ring of 3 stages, 2 at D = 256) and keeps
+// four bulk copies into a private ring of 3 stages, 2 at G = 16) and keeps
 // its own online-softmax state; the block merges the four states at the end.
+// At D = 256 the warps work in pairs: both warps of a pair take the same
+// blocks (one ring of 2 stages, the 128-byte code rows by swizzled tensor
+// copies), each the channels of one half, and they add their partial scores
+// through shared memory before the softmax.
 // Both products run on the tensor cores as m16n8k16 fp16 MMAs with fp32
 // accumulation, with the N dimension = 4 query heads x 2 parts (q~ and p S_V
 // each as an fp16 value plus its fp16 remainder, ~2^-22 together):
